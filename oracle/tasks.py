@@ -1,0 +1,78 @@
+"""Expected task set of one decode step — test infrastructure only.
+
+"Event Tensor: A Unified Abstraction for Compiling Dynamic Megakernel",
+section "Core method": an event is the completion of a set of SM-granular
+tasks, and its dimensions may be symbolic (the batch size); "Lecture 112:
+Production Megakernels for Real-World Inference", section "Symbolic
+Representation of Work": extents are expressions of the runtime sizes (the
+context length).  The set of tasks one step must run is therefore a function
+of the step's batch size and per-sequence context lengths plus the tile
+sizes, which are passed in here as plain numbers.
+
+Task families of one dense layer, in the order a layer runs them:
+
+* ``qkv``    — one per ``tile_qkv`` output rows of the stacked Q/K/V weights;
+* ``attn``   — one per (sequence b, kv head g, key chunk c),
+  ``c < ceil((ctx_b + 1) / chunk)``;
+* ``merge``  — one per (b, g): combine that head group's chunk partials;
+* ``oproj``  — one per ``tile_o`` rows of the output projection;
+* ``gateup`` — one per ``tile_gu`` rows of the gate (and the same rows of up);
+* ``down``   — one per (``tile_down`` rows, K segment of ``kseg`` columns);
+* ``dred``   — one per ``tile_down`` rows: sum the K-segment partials.
+
+After the last layer: ``lm`` (``tile_lm`` vocabulary rows each), ``lmgrp``
+(one per ``lm_group`` lm tiles) and ``lmfin`` (one).
+
+Linear index of an ``attn`` task: ``Hkv * sum_{b'<b} nch_{b'} + g * nch_b + c``.
+``down`` tasks are numbered K-segment-major: ``kc * (H / tile_down) + n``.
+"""
+from __future__ import annotations
+
+
+def _ceil(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+def dense_family_extents(shape, B: int, ctx, tiles: dict) -> dict:
+    """Number of tasks of each family in one layer (and after the last)."""
+    H, D = shape.hidden, shape.head_dim
+    Hq, Hkv = shape.n_q_heads, shape.n_kv_heads
+    nch = [_ceil(int(ctx[b]) + 1, tiles["chunk"]) for b in range(B)]
+    n_lm = _ceil(shape.vocab, tiles["tile_lm"])
+    return {
+        "qkv": (Hq + 2 * Hkv) * D // tiles["tile_qkv"],
+        "attn": Hkv * sum(nch),
+        "merge": Hkv * B,
+        "oproj": H // tiles["tile_o"],
+        "gateup": shape.ffn // tiles["tile_gu"],
+        "down": (H // tiles["tile_down"]) * (shape.ffn // tiles["kseg"]),
+        "dred": H // tiles["tile_down"],
+        "lm": n_lm,
+        "lmgrp": _ceil(n_lm, tiles["lm_group"]),
+        "lmfin": 1,
+    }
+
+
+def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
+    """The set of ``(family, layer, index)`` one decode step runs exactly once.
+
+    Per-layer families carry their layer; ``lm``, ``lmgrp`` and ``lmfin``
+    carry layer ``-1``.  ``attn`` indices are enumerated from the (b, g, c)
+    triples, so the set also pins the linear numbering stated above.
+    """
+    ext = dense_family_extents(shape, B, ctx, tiles)
+    Hkv = shape.n_kv_heads
+    out = set()
+    for l in range(shape.n_layers):
+        for fam in ("qkv", "merge", "oproj", "gateup", "down", "dred"):
+            out.update((fam, l, i) for i in range(ext[fam]))
+        base = 0
+        for b in range(B):
+            nch = _ceil(int(ctx[b]) + 1, tiles["chunk"])
+            for g in range(Hkv):
+                for c in range(nch):
+                    out.add(("attn", l, Hkv * base + g * nch + c))
+            base += nch
+    for fam in ("lm", "lmgrp", "lmfin"):
+        out.update((fam, -1, i) for i in range(ext[fam]))
+    return out
