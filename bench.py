@@ -1,0 +1,308 @@
+"""Decode-step benchmark of the B200 megakernel (one JSON line on rank 0).
+
+Workload: the Llama-1B-shaped dense decoder (16 layers, hidden 2048, 32/8
+heads x 64, FFN 8192, vocab 128256, tied embeddings), bf16 N(0, 0.02)
+random weights, batch 1, KV cache bf16 N(0, 1) at context 1024; each timed
+step is one greedy decode step, the steps cycling through the 32-step decode
+window (positions 1024..1055) with the argmax token fed back on the device.
+The weights (2.47 GB) stream from HBM every step, far above the 126 MB L2,
+so no L2 flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--sched static|dynamic]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+N > 1 (under torchrun) runs N independent replicas, one per GPU (the decode
+step has no data-path exchange); the value is all ranks' tokens over the
+slowest rank's device time.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("decode step µs & tokens/s (1B dense, B=1..64; MoE); achieved HBM GB/s vs 8 TB/s")
+CTX0 = 1024
+WINDOW = 32
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def setup_model(dev, seed=0):
+    import torch
+    import workloads as wl
+    s = wl.LLAMA_1B
+    w_cpu = wl.dense_weights(s, seed=seed)
+    max_ctx = CTX0 + WINDOW + 32
+    K_cpu, V_cpu = wl.kv_cache(s, 1, max_ctx, [CTX0], seed=seed)
+    w = {k: v.to(dev, non_blocking=False) for k, v in w_cpu.items()}
+    K, V = K_cpu.to(dev), V_cpu.to(dev)
+    torch.cuda.synchronize()
+    return s, w_cpu, w, K_cpu, V_cpu, K, V, max_ctx
+
+
+def cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, n_steps):
+    """The oracle as it stands: tokens/s over n_steps decode steps after one
+    untimed warm-up step (which also widens the weights to fp64 once)."""
+    import torch
+    import oracle
+    import workloads as wl
+    o = oracle.DenseOracle(s, w_cpu)
+    K, V = K_cpu.clone(), V_cpu.clone()
+    tok = int(wl.token_ids(1, s.vocab)[0])
+    r = o.step(K, V, [tok], [0], [CTX0])
+    tok = int(r["next_tokens"][0])
+    t0 = time.perf_counter()
+    for i in range(n_steps):
+        r = o.step(K, V, [tok], [0], [CTX0 + 1 + i])
+        tok = int(r["next_tokens"][0])
+    dt = time.perf_counter() - t0
+    return n_steps / dt, torch.get_num_threads(), dt
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    import torch
+    import workloads as wl
+    s = wl.LLAMA_1B
+    w_cpu = wl.dense_weights(s)
+    K_cpu, V_cpu = wl.kv_cache(s, 1, CTX0 + WINDOW + 32, [CTX0])
+    n = max(1, min(args.steps, 4))
+    rate, cores, dt = cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, n)
+    sample = (f"{n} full decode steps of the 1B model (B=1, positions {CTX0 + 1}..{CTX0 + n}) after one "
+              f"untimed warm-up step; fp64 CPU oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": n, "warmup": 1, "ms_per_step": 1000.0 * dt / n, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args),
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args):
+    return {"workload": "llama-1b-shaped dense decode (16L, hidden 2048, 32q/8kv x 64, ffn 8192, vocab 128256, "
+                        "tied), greedy 32-step window from context 1024",
+            "batch": 1, "ctx": f"{CTX0}..{CTX0 + WINDOW - 1}", "sched": args.sched,
+            "l2": "2.5 GB weights streamed per step > 126 MB L2; no flush",
+            "parallelism": "replicas" if args.gpus > 1 else "single-gpu"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--sched", default="static", choices=["static", "dynamic"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import event_tensor_task_b200 as mk
+
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device(dev))
+
+    s, w_cpu, w, K_cpu, V_cpu, K, V, max_ctx = setup_model(dev)
+    sched = mk.MK_SCHED_STATIC if args.sched == "static" else mk.MK_SCHED_DYNAMIC
+    dec = mk.DenseDecoder(s, w, K, V, max_batch=1, max_ctx=max_ctx, n_slots=1, sched=sched)
+    stream = torch.cuda.current_stream()
+
+    import workloads as wl
+    tok0 = int(wl.token_ids(1, s.vocab)[0])
+    ctx_tab = torch.arange(CTX0, CTX0 + WINDOW, dtype=torch.int32, device=dev)
+    slot = torch.zeros(1, dtype=torch.int32, device=dev)
+    toks = torch.full((2,), tok0, dtype=torch.int32, device=dev)  # ping-pong greedy tokens
+
+    def run(n, start=0):
+        for i in range(start, start + n):
+            a, b = toks[i % 2: i % 2 + 1], toks[(i + 1) % 2: (i + 1) % 2 + 1]
+            dec.step(a, slot, ctx_tab[i % WINDOW: i % WINDOW + 1], b)
+
+    run(args.warmup)
+    torch.cuda.synchronize()
+    code, st = dec.status()
+    if code != 0:
+        raise SystemExit(f"device status {code} after warm-up (family {st.family} index {st.index})")
+
+    # ---- device-timed region: K steps, inputs resident in HBM
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device() if world == 1 else local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        run(args.steps, args.warmup)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    code, st = dec.status()
+    if code != 0:
+        raise SystemExit(f"device status {code} in the timed region")
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    tokens = world * 1 * args.steps
+    value = tokens / (ms / 1000.0)
+
+    # algorithmic bytes per launch (mean over the context window)
+    step_bytes = statistics.mean(mk.mk_plan_step_bytes(dec.plan, 1, [CTX0 + (i % WINDOW)])
+                                 for i in range(WINDOW))
+    peak, peak_kind = peaks()
+    achieved = step_bytes / (ms_step / 1000.0) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    h_in = torch.empty(3, dtype=torch.int32, pin_memory=True)
+    h_out = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    d_in = torch.empty(3, dtype=torch.int32, device=dev)
+    d_out = torch.empty(1, dtype=torch.int32, device=dev)
+    tok = tok0
+    n_e2e = min(args.steps, 1000)
+
+    def e2e_steps(n, start):
+        nonlocal tok
+        for i in range(start, start + n):
+            h_in[0], h_in[1], h_in[2] = tok, 0, CTX0 + (i % WINDOW)
+            d_in.copy_(h_in, non_blocking=True)
+            dec.step(d_in[0:1], d_in[1:2], d_in[2:3], d_out)
+            h_out.copy_(d_out, non_blocking=True)
+            stream.synchronize()
+            tok = int(h_out[0])
+
+    e2e_steps(args.warmup, 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_steps(n_e2e, args.warmup)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_value = world * n_e2e / (e_ms / 1000.0)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, dt = cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, 2)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": "2 full decode steps of the 1B model (B=1, ctx 1025, 1026) after one untimed "
+                         "warm-up step; fp64 CPU oracle"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "us_per_step": 1000.0 * ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) KV cache)", "config": workload_config(args),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "frac_of_8tbs": achieved / 8000.0, "bytes_per_launch": step_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 12, "d2h_bytes_per_step": 4},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

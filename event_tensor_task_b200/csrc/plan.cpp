@@ -1,0 +1,799 @@
+// plan.cpp — host task-graph compiler, validator and plan simulator.
+//
+// The graph of one dense decode step, per layer l (events in brackets):
+//   QKV tiles        wait EV_IN[l]        notify EV_QKV[l][g]
+//   ATTN chunks      wait EV_QKV[l][g]    notify EV_CHUNK[l][b][g] -> MERGE(b,g)
+//   MERGE (follow-up)                     notify EV_ATTN[l]
+//   OPROJ tiles      wait EV_ATTN[l]      notify EV_O[l]
+//   GATEUP tiles     wait EV_O[l]         notify EV_GU[l][kc]
+//   DOWN tiles       wait EV_GU[l][kc]    notify EV_DSUM[l][n] -> DRED(n)
+//   DRED (follow-up)                      notify EV_IN[l+1]
+// then LM tiles (wait EV_IN[L], notify EV_LMG[grp] -> LMGRP), LMGRP
+// (notify EV_LM -> LMFIN) and LMFIN.  Fine-grained events let a consumer
+// start on the subset of producer output it reads ("Event Tensor: A Unified
+// Abstraction for Compiling Dynamic Megakernel", section "Problem": coarse
+// kernel-boundary synchronisation; "Lecture 112: Production Megakernels for
+// Real-World Inference", section "Dependency Tracking (Barriers)": partition
+// tensor dimensions by dependency to maximise the number of barriers).
+#include "plan.hpp"
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <random>
+#include <set>
+#include <unordered_map>
+
+namespace mk {
+
+static const char* kOpNames[OP_COUNT] = {"end", "qkv", "attn", "merge", "oproj", "gateup",
+                                         "down", "dred", "lm", "lmgrp", "lmfin"};
+static const int kLayerOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_DRED};
+static const int kLmOps[] = {OP_LM, OP_LMGRP, OP_LMFIN};
+static constexpr int kFamPerLayer = 7;
+
+// ---------------------------------------------------------------- expressions
+namespace {
+struct Emit {
+  std::vector<int32_t>& c;
+  int start;
+  explicit Emit(std::vector<int32_t>& code) : c(code), start((int)code.size()) {}
+  Emit& push(int v) { c.push_back(X_PUSH); c.push_back(v); return *this; }
+  Emit& op(int o) { c.push_back(o); return *this; }
+  Emit& coord(int d) { c.push_back(X_COORD); c.push_back(d); return *this; }
+  int ret() { c.push_back(X_RET); return start; }
+};
+int emit_const(std::vector<int32_t>& code, int v) { return Emit(code).push(v).ret(); }
+}  // namespace
+
+int Plan::fam_index(int op, int layer) const {
+  if (op >= OP_LM) return dp.n_layers * kFamPerLayer + (op - OP_LM);
+  for (int k = 0; k < kFamPerLayer; ++k)
+    if (kLayerOps[k] == op) return layer * kFamPerLayer + k;
+  return -1;
+}
+
+int Plan::counter(int ev, int c0, int c1, int c2) const {
+  const EventTensorDesc& e = dp.ev[ev];
+  int lin = c0;
+  if (e.ndim > 1) lin = lin * e.dims[1] + c1;
+  if (e.ndim > 2) lin = lin * e.dims[2] + c2;
+  return e.base + lin;
+}
+
+int Plan::event_count(int ev, int c0, int c1, int c2, const Binding& bd) const {
+  ExprEnv env{bd.B, bd.ctx.data(), {c0, c1, c2}};
+  return expr_eval(code.data(), dp.ev[ev].count_expr, env);
+}
+
+int Plan::family_extent(int f, const Binding& bd) const {
+  ExprEnv env{bd.B, bd.ctx.data(), {0, 0, 0}};
+  return expr_eval(code.data(), fams[f].extent_expr, env);
+}
+
+// ---------------------------------------------------------------- task model
+void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
+  const DevPlan& P = dp;
+  t = TaskRec();
+  t.fam = f;
+  t.idx = idx;
+  int op = fams[f].op, l = fams[f].layer;
+  int B = bd.B, H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads;
+  int qpg = Hq / Hkv, F = P.ffn;
+  long long QD = (long long)Hq * D;
+  auto kv_row = [&](int layer, int slot, int g, int pos) -> long long {
+    return ((((long long)layer * P.n_slots + slot) * Hkv + g) * P.max_ctx + pos) * D;
+  };
+  // sequence b uses slot b in the host model (slots are distinct by contract)
+  switch (op) {
+    case OP_QKV: {
+      QkvTile q = decode_qkv(P, idx);
+      t.wait_ev = counter(EV_IN, l);
+      t.notify_ev = counter(EV_QKV, l, q.group);
+      int half = P.tile_qkv / 2;
+      for (int b = 0; b < B; ++b) {
+        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        for (int part = 0; part < 2; ++part) {
+          int j = q.j0 + part * (D / 2);
+          if (q.kind == 0) {
+            long long base = b * QD + (long long)q.head * D + j;
+            t.writes.push_back({BUF_Q, base, base + half});
+          } else {
+            long long base = kv_row(l, b, q.group, bd.ctx[b]) + j;
+            t.writes.push_back({q.kind == 1 ? BUF_KC : BUF_VC, base, base + half});
+          }
+        }
+      }
+    } break;
+    case OP_ATTN: {
+      std::vector<int> nch(B), pre(B + 1, 0);
+      for (int b = 0; b < B; ++b) { nch[b] = ceil_div(bd.ctx[b] + 1, P.chunk); pre[b + 1] = pre[b] + nch[b]; }
+      AttnTask a = decode_attn(idx, B, Hkv, nch.data(), pre.data());
+      t.wait_ev = counter(EV_QKV, l, a.g);
+      t.notify_ev = counter(EV_CHUNK, l, a.b, a.g);
+      t.follow_fam = fam_index(OP_MERGE, l);
+      t.follow_idx = a.b * Hkv + a.g;
+      long long qb = a.b * QD + (long long)a.g * qpg * D;
+      t.reads.push_back({BUF_Q, qb, qb + (long long)qpg * D});
+      int p0 = a.c * P.chunk, p1 = std::min(p0 + P.chunk, bd.ctx[a.b] + 1);
+      long long kb = kv_row(l, a.b, a.g, p0);
+      t.reads.push_back({BUF_KC, kb, kb + (long long)(p1 - p0) * D});
+      t.reads.push_back({BUF_VC, kb, kb + (long long)(p1 - p0) * D});
+      long long pb = ((long long)a.b * Hkv + a.g) * P.max_chunks + a.c;
+      t.writes.push_back({BUF_APART, pb, pb + 1});
+    } break;
+    case OP_MERGE: {
+      int b = idx / Hkv, g = idx % Hkv;
+      int nch = ceil_div(bd.ctx[b] + 1, P.chunk);
+      long long pb = ((long long)b * Hkv + g) * P.max_chunks;
+      t.reads.push_back({BUF_APART, pb, pb + nch});
+      long long ob = b * QD + (long long)g * qpg * D;
+      t.writes.push_back({BUF_ATTN, ob, ob + (long long)qpg * D});
+      t.notify_ev = counter(EV_ATTN, l);
+    } break;
+    case OP_OPROJ: {
+      t.wait_ev = counter(EV_ATTN, l);
+      t.notify_ev = counter(EV_O, l);
+      for (int b = 0; b < B; ++b) {
+        t.reads.push_back({BUF_ATTN, b * QD, (b + 1) * QD});
+        long long xb = (long long)b * H + (long long)idx * P.tile_o;
+        t.reads.push_back({BUF_X, xb, xb + P.tile_o});
+        t.writes.push_back({BUF_X, xb, xb + P.tile_o});
+      }
+    } break;
+    case OP_GATEUP: {
+      t.wait_ev = counter(EV_O, l);
+      t.notify_ev = counter(EV_GU, l, idx * P.tile_gu / P.kseg);
+      for (int b = 0; b < B; ++b) {
+        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        long long hb = (long long)b * F + (long long)idx * P.tile_gu;
+        t.writes.push_back({BUF_H, hb, hb + P.tile_gu});
+      }
+    } break;
+    case OP_DOWN: {
+      int kc = idx / P.n_dtiles, n = idx % P.n_dtiles;
+      t.wait_ev = counter(EV_GU, l, kc);
+      t.notify_ev = counter(EV_DSUM, l, n);
+      t.follow_fam = fam_index(OP_DRED, l);
+      t.follow_idx = n;
+      for (int b = 0; b < B; ++b) {
+        long long hb = (long long)b * F + (long long)kc * P.kseg;
+        t.reads.push_back({BUF_H, hb, hb + P.kseg});
+        long long pb = ((long long)kc * P.max_batch + b) * H + (long long)n * P.tile_down;
+        t.writes.push_back({BUF_DPART, pb, pb + P.tile_down});
+      }
+    } break;
+    case OP_DRED: {
+      t.notify_ev = counter(EV_IN, l + 1);
+      for (int b = 0; b < B; ++b) {
+        for (int kc = 0; kc < P.n_kc; ++kc) {
+          long long pb = ((long long)kc * P.max_batch + b) * H + (long long)idx * P.tile_down;
+          t.reads.push_back({BUF_DPART, pb, pb + P.tile_down});
+        }
+        long long xb = (long long)b * H + (long long)idx * P.tile_down;
+        t.reads.push_back({BUF_X, xb, xb + P.tile_down});
+        t.writes.push_back({BUF_X, xb, xb + P.tile_down});
+      }
+    } break;
+    case OP_LM: {
+      t.wait_ev = counter(EV_IN, P.n_layers);
+      int grp = idx / P.lm_group;
+      t.notify_ev = counter(EV_LMG, grp);
+      t.follow_fam = fam_index(OP_LMGRP, -1);
+      t.follow_idx = grp;
+      int r0 = idx * P.tile_lm, r1 = std::min(P.vocab, r0 + P.tile_lm);
+      for (int b = 0; b < B; ++b) {
+        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        t.writes.push_back({BUF_LOGITS, (long long)b * P.vocab + r0, (long long)b * P.vocab + r1});
+        long long pb = (long long)b * P.n_lm_tiles + idx;
+        t.writes.push_back({BUF_LMPART, pb, pb + 1});
+      }
+    } break;
+    case OP_LMGRP: {
+      t.notify_ev = counter(EV_LM, 0);
+      t.follow_fam = fam_index(OP_LMFIN, -1);
+      t.follow_idx = 0;
+      int t0 = idx * P.lm_group, t1 = std::min(P.n_lm_tiles, t0 + P.lm_group);
+      for (int b = 0; b < B; ++b) {
+        t.reads.push_back({BUF_LMPART, (long long)b * P.n_lm_tiles + t0, (long long)b * P.n_lm_tiles + t1});
+        long long gb = (long long)b * P.n_lmgrp + idx;
+        t.writes.push_back({BUF_LMG, gb, gb + 1});
+      }
+    } break;
+    case OP_LMFIN: {
+      for (int b = 0; b < B; ++b) {
+        t.reads.push_back({BUF_LMG, (long long)b * P.n_lmgrp, (long long)(b + 1) * P.n_lmgrp});
+        t.writes.push_back({BUF_NEXT, b, b + 1});
+      }
+    } break;
+    default: break;
+  }
+}
+
+void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
+  // find the tensor and coordinates of counter ci
+  int ev = -1;
+  for (int e = 0; e < EV_COUNT; ++e) {
+    int n = dp.ev[e].dims[0] * (dp.ev[e].ndim > 1 ? dp.ev[e].dims[1] : 1) *
+            (dp.ev[e].ndim > 2 ? dp.ev[e].dims[2] : 1);
+    if (ci >= dp.ev[e].base && ci < dp.ev[e].base + n) { ev = e; break; }
+  }
+  if (ev < 0) return;
+  int lin = ci - dp.ev[ev].base;
+  int c[3] = {0, 0, 0};
+  for (int d = dp.ev[ev].ndim - 1; d >= 0; --d) { c[d] = lin % dp.ev[ev].dims[d]; lin /= dp.ev[ev].dims[d]; }
+  auto add = [&](int f, int lo, int n) { if (n > 0) { out.push_back(f); out.push_back(lo); out.push_back(n); } };
+  switch (ev) {
+    case EV_IN:
+      if (c[0] < dp.n_layers) add(fam_index(OP_QKV, c[0]), 0, dp.n_qkv_tiles);
+      else add(fam_index(OP_LM, -1), 0, dp.n_lm_tiles);
+      break;
+    case EV_QKV: {
+      int pre = 0;
+      for (int b = 0; b < bd.B; ++b) {
+        int nch = ceil_div(bd.ctx[b] + 1, dp.chunk);
+        add(fam_index(OP_ATTN, c[0]), dp.n_kv_heads * pre + c[1] * nch, nch);
+        pre += nch;
+      }
+    } break;
+    case EV_ATTN: add(fam_index(OP_OPROJ, c[0]), 0, dp.n_otiles); break;
+    case EV_O: add(fam_index(OP_GATEUP, c[0]), 0, dp.n_gutiles); break;
+    case EV_GU: add(fam_index(OP_DOWN, c[0]), c[1] * dp.n_dtiles, dp.n_dtiles); break;
+    default: break;  // EV_CHUNK, EV_DSUM, EV_LMG, EV_LM trigger follow-ups
+  }
+}
+
+// ---------------------------------------------------------------- build
+static bool pow2_divides(int a, int b) { return a > 0 && b % a == 0; }
+
+mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, int smem_bytes,
+                     Plan& p, std::string& err) {
+  if (!m || !o) { err = "null model or options"; return MK_ERR_INVALID_ARG; }
+  if (m->kind != MK_MODEL_DENSE) { err = "only MK_MODEL_DENSE plans are implemented"; return MK_ERR_UNSUPPORTED; }
+  const int H = m->hidden, D = m->head_dim, Hq = m->n_q_heads, Hkv = m->n_kv_heads, F = m->ffn;
+  if (m->n_layers < 1 || m->vocab < 1 || Hkv < 1 || Hq < 1) { err = "non-positive dimension"; return MK_ERR_INVALID_ARG; }
+  if (D != 64) { err = "head_dim must be 64"; return MK_ERR_UNSUPPORTED; }
+  if (Hq % Hkv) { err = "n_q_heads must be a multiple of n_kv_heads"; return MK_ERR_INVALID_ARG; }
+  if (Hq * D != H) { err = "n_q_heads * head_dim must equal hidden"; return MK_ERR_UNSUPPORTED; }
+  if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
+  if (F % 256) { err = "ffn must be a multiple of 256"; return MK_ERR_UNSUPPORTED; }
+  if (m->max_batch < 1 || m->max_batch > 4) { err = "max_batch must be in [1, 4] for this build"; return MK_ERR_UNSUPPORTED; }
+  if (m->max_ctx < 2 || m->n_slots < m->max_batch) { err = "max_ctx >= 2 and n_slots >= max_batch required"; return MK_ERR_INVALID_ARG; }
+  if (o->sched != MK_SCHED_STATIC && o->sched != MK_SCHED_DYNAMIC) { err = "unknown schedule"; return MK_ERR_INVALID_ARG; }
+  if (n_sm < 1 || n_sm > 1024) { err = "n_sm out of range"; return MK_ERR_INVALID_ARG; }
+
+  p.m = *m;
+  p.o = *o;
+  p.layer_w.assign(m->layers ? m->layers : nullptr, m->layers ? m->layers + m->n_layers : nullptr);
+  if (!m->layers) p.layer_w.assign(m->n_layers, mk_layer_weights{});
+  p.m.layers = nullptr;
+  DevPlan& P = p.dp;
+  P = DevPlan();
+  P.sched = o->sched;
+  P.n_sm = n_sm;
+  P.n_layers = m->n_layers; P.hidden = H; P.n_q_heads = Hq; P.n_kv_heads = Hkv; P.head_dim = D;
+  P.ffn = F; P.vocab = m->vocab; P.max_batch = m->max_batch; P.max_ctx = m->max_ctx;
+  P.n_slots = m->n_slots; P.eps = m->eps;
+  P.debug_flags = o->debug_flags;
+  P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
+
+  // tiles: about 32 KB of weights per task, whole rotate-half pairs per QKV tile
+  int kseg = o->kseg ? o->kseg : std::min(F, 2048);
+  while (kseg > 256 && F % kseg) kseg -= 256;
+  P.kseg = kseg;
+  P.tile_qkv = o->tile_qkv ? o->tile_qkv : std::min(64, 16384 / H);
+  P.tile_o = o->tile_o ? o->tile_o : 16384 / H;
+  P.tile_gu = o->tile_gu ? o->tile_gu : 8192 / H;
+  P.tile_down = o->tile_down ? o->tile_down : 16384 / kseg;
+  P.tile_lm = o->tile_lm ? o->tile_lm : 32768 / H;
+  P.lm_group = o->lm_group ? o->lm_group : 64;
+  P.chunk = o->attn_chunk ? o->attn_chunk : 64;
+  P.slot_bytes = 16384;
+  const int rows_per_slot_h = P.slot_bytes / (2 * H);
+  const int rows_per_slot_k = P.slot_bytes / (2 * kseg);
+  if (!(P.kseg % 256 == 0 && F % P.kseg == 0 && P.kseg >= 1024 && P.kseg <= 2048))
+    { err = "kseg must be a multiple of 256 in [1024, 2048] dividing ffn"; return MK_ERR_INVALID_ARG; }
+  if (Hq / Hkv > 4) { err = "at most 4 query heads per kv head"; return MK_ERR_UNSUPPORTED; }
+  if (!(pow2_divides(P.tile_qkv, D) && P.tile_qkv % 2 == 0 && (P.tile_qkv / 2) % rows_per_slot_h == 0 &&
+        P.tile_qkv / 2 <= 32))
+    { err = "tile_qkv must be even, divide head_dim and fill whole ring slots per half"; return MK_ERR_INVALID_ARG; }
+  if (!(pow2_divides(P.tile_o, H) && P.tile_o % rows_per_slot_h == 0))
+    { err = "tile_o must divide hidden and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
+  if (!(pow2_divides(P.tile_gu, P.kseg) && P.tile_gu % rows_per_slot_h == 0))
+    { err = "tile_gu must divide kseg and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
+  if (!(pow2_divides(P.tile_down, H) && P.tile_down % rows_per_slot_k == 0))
+    { err = "tile_down must divide hidden and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
+  if (!(P.tile_lm > 0 && P.tile_lm % rows_per_slot_h == 0)) { err = "tile_lm must fill whole ring slots"; return MK_ERR_INVALID_ARG; }
+  if (P.chunk != 64) { err = "attn_chunk must be 64"; return MK_ERR_UNSUPPORTED; }
+  if (P.lm_group < 1) { err = "lm_group must be positive"; return MK_ERR_INVALID_ARG; }
+  // a task spans at most 4 ring slots (16 accumulated rows per compute thread)
+  if (P.tile_qkv / rows_per_slot_h > 4 || P.tile_o / rows_per_slot_h > 4 || 2 * P.tile_gu / rows_per_slot_h > 4 ||
+      P.tile_down / rows_per_slot_k > 4 || ceil_div(P.tile_lm, rows_per_slot_h) > 4)
+    { err = "a tile spans more than 4 ring slots"; return MK_ERR_UNSUPPORTED; }
+  P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
+  P.n_otiles = H / P.tile_o;
+  P.n_gutiles = F / P.tile_gu;
+  P.n_dtiles = H / P.tile_down;
+  P.n_kc = F / P.kseg;
+  P.n_lm_tiles = ceil_div(P.vocab, P.tile_lm);
+  P.n_lmgrp = ceil_div(P.n_lm_tiles, P.lm_group);
+  P.max_chunks = ceil_div(P.max_ctx, P.chunk);
+
+  // shared memory: ring of 16 KB slots plus a fixed control area
+  const int reserve = 14 * 1024;  // fixed shared-memory area of the kernel
+  P.smem_bytes = smem_bytes;
+  P.ring_slots = std::min(16, (smem_bytes - reserve) / P.slot_bytes);
+  if (P.ring_slots < 3) { err = "not enough shared memory for a 3-slot ring"; return MK_ERR_UNSUPPORTED; }
+
+  // ---- expressions and families
+  p.code.clear();
+  p.fams.clear();
+  p.fam_names.clear();
+  int debug_base = 0;
+  auto add_family = [&](int op, int layer, int extent_expr, int max_extent, int followup) {
+    FamilyDesc f{};
+    f.op = op; f.layer = layer; f.extent_expr = extent_expr; f.max_extent = max_extent;
+    f.debug_base = debug_base; f.followup = followup;
+    debug_base += max_extent;
+    p.fams.push_back(f);
+    p.fam_names.push_back(std::string(kOpNames[op]) + (layer >= 0 ? "." + std::to_string(layer) : ""));
+  };
+  // ATTN extent: Hkv * sum_b ceil((ctx_b + 1) / chunk)
+  int e_attn;
+  {
+    Emit e(p.code);
+    e.push(Hkv);
+    p.code.push_back(X_SUM_B);
+    size_t len_at = p.code.size();
+    p.code.push_back(0);
+    size_t body = p.code.size();
+    p.code.push_back(X_VAR); p.code.push_back(X_CTX_AT);
+    p.code.push_back(X_PUSH); p.code.push_back(1); p.code.push_back(X_ADD);
+    p.code.push_back(X_PUSH); p.code.push_back(P.chunk); p.code.push_back(X_CEILDIV);
+    p.code.push_back(X_RET);
+    p.code[len_at] = (int)(p.code.size() - body);
+    p.code.push_back(X_MUL);
+    p.code.push_back(X_RET);
+    e_attn = e.start;
+  }
+  int e_merge = Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret();
+  for (int l = 0; l < P.n_layers; ++l) {
+    add_family(OP_QKV, l, emit_const(p.code, P.n_qkv_tiles), P.n_qkv_tiles, 0);
+    add_family(OP_ATTN, l, e_attn, Hkv * P.max_batch * P.max_chunks, 0);
+    add_family(OP_MERGE, l, e_merge, Hkv * P.max_batch, 1);
+    add_family(OP_OPROJ, l, emit_const(p.code, P.n_otiles), P.n_otiles, 0);
+    add_family(OP_GATEUP, l, emit_const(p.code, P.n_gutiles), P.n_gutiles, 0);
+    add_family(OP_DOWN, l, emit_const(p.code, P.n_dtiles * P.n_kc), P.n_dtiles * P.n_kc, 0);
+    add_family(OP_DRED, l, emit_const(p.code, P.n_dtiles), P.n_dtiles, 1);
+  }
+  add_family(OP_LM, -1, emit_const(p.code, P.n_lm_tiles), P.n_lm_tiles, 0);
+  add_family(OP_LMGRP, -1, emit_const(p.code, P.n_lmgrp), P.n_lmgrp, 1);
+  add_family(OP_LMFIN, -1, emit_const(p.code, 1), 1, 1);
+  P.n_families = (int)p.fams.size();
+  if (P.n_families > kMaxFamilies) { err = "too many task families"; return MK_ERR_UNSUPPORTED; }
+  P.debug_slots = debug_base;
+  P.fam_stride = kFamPerLayer;
+  for (int op = 0; op < OP_COUNT; ++op) P.fam_first_layer[op] = -1;
+  for (int k = 0; k < kFamPerLayer; ++k) P.fam_first_layer[kLayerOps[k]] = k;
+  for (int k = 0; k < 3; ++k) P.fam_first_layer[kLmOps[k]] = P.n_layers * kFamPerLayer + k;
+
+  // ---- event tensors (shapes at the symbols' maxima, wait counts symbolic)
+  int base = 0;
+  auto add_event = [&](int id, int ndim, int d0, int d1, int d2, int count_expr) {
+    EventTensorDesc& e = P.ev[id];
+    e.base = base; e.ndim = ndim; e.dims[0] = d0; e.dims[1] = d1; e.dims[2] = d2;
+    e.count_expr = count_expr;
+    base += d0 * (ndim > 1 ? d1 : 1) * (ndim > 2 ? d2 : 1);
+  };
+  const int L = P.n_layers;
+  const int qkv_per_group = (Hq / Hkv + 2) * (D / P.tile_qkv);
+  add_event(EV_IN, 1, L + 1, 1, 1, Emit(p.code).push(0).coord(0).op(X_LT).push(P.n_dtiles).op(X_MUL).ret());
+  add_event(EV_QKV, 2, L, Hkv, 1, emit_const(p.code, qkv_per_group));
+  add_event(EV_CHUNK, 3, L, P.max_batch, Hkv,
+            Emit(p.code).coord(1).op(X_B).op(X_LT).coord(1).op(X_CTX_AT).push(1).op(X_ADD)
+                .push(P.chunk).op(X_CEILDIV).op(X_MUL).ret());
+  add_event(EV_ATTN, 1, L, 1, 1, Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret());
+  add_event(EV_O, 1, L, 1, 1, emit_const(p.code, P.n_otiles));
+  add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu));
+  add_event(EV_DSUM, 2, L, P.n_dtiles, 1, emit_const(p.code, P.n_kc));
+  add_event(EV_LMG, 1, P.n_lmgrp, 1, 1,
+            Emit(p.code).push(P.lm_group).push(P.n_lm_tiles).coord(0).push(P.lm_group).op(X_MUL)
+                .op(X_SUB).op(X_MIN).ret());
+  add_event(EV_LM, 1, 1, 1, 1, emit_const(p.code, P.n_lmgrp));
+  P.n_counters = base;
+
+  // ---- static schedule: per-SM queues of range instructions in topological
+  // (family) order; family f's task i runs on SM (i + rot_f) mod n_sm, with
+  // rot_f continuing the round robin where the previous family stopped.
+  std::vector<int> regular;
+  for (int f = 0; f < P.n_families; ++f)
+    if (!p.fams[f].followup) regular.push_back(f);
+  P.n_instr_per_sm = (int)regular.size() + 1;
+  p.instr.assign((size_t)n_sm * P.n_instr_per_sm, Instr{});
+  Binding typical{1, {std::min(1024, P.max_ctx - 1)}};
+  long long rot = 0;
+  for (size_t k = 0; k < regular.size(); ++k) {
+    int f = regular[k];
+    for (int s = 0; s < n_sm; ++s) {
+      Instr& in = p.instr[(size_t)s * P.n_instr_per_sm + k];
+      in.family = f;
+      in.start = (int)(((s - rot) % n_sm + n_sm) % n_sm);
+      in.stride = n_sm;
+    }
+    rot += p.family_extent(f, typical);
+  }
+  for (int s = 0; s < n_sm; ++s) {
+    Instr& in = p.instr[(size_t)s * P.n_instr_per_sm + regular.size()];
+    in.family = -1; in.start = 0; in.stride = 0;
+  }
+
+  // ---- dynamic queue capacity: pushes per step at the symbols' maxima
+  P.queue_ranges = L * (2 + Hkv * P.max_batch + P.n_kc) + 8;
+
+  // ---- layer pointers and the rotary table
+  p.layers.resize(L);
+  for (int l = 0; l < L; ++l) {
+    const mk_layer_weights& w = p.layer_w[l];
+    p.layers[l] = LayerPtrs{w.attn_norm, w.wq, w.wk, w.wv, w.wo, w.ffn_norm, w.w_gate, w.w_up, w.w_down};
+  }
+  P.embed = m->embed;
+  P.lm_head = m->lm_head ? m->lm_head : m->embed;
+  P.final_norm = m->final_norm;
+  P.k_cache = m->k_cache;
+  P.v_cache = m->v_cache;
+  p.rope.resize((size_t)P.max_ctx * (D / 2) * 2);
+  for (int pos = 0; pos < P.max_ctx; ++pos)
+    for (int i = 0; i < D / 2; ++i) {
+      double ang = (double)pos * std::pow((double)m->rope_theta, -2.0 * i / D);
+      p.rope[((size_t)pos * (D / 2) + i) * 2 + 0] = (float)std::cos(ang);
+      p.rope[((size_t)pos * (D / 2) + i) * 2 + 1] = (float)std::sin(ang);
+    }
+  std::vector<unsigned char> image;
+  lower_plan(p, image);
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------- lowering
+void lower_plan(Plan& p, std::vector<unsigned char>& image) {
+  DevPlan& P = p.dp;
+  const int qpg = P.n_q_heads / P.n_kv_heads;
+  long long off = 0;
+  auto take = [&](long long bytes) { long long at = off; off += (bytes + 255) / 256 * 256; return at; };
+  P.off_control = take(sizeof(Control));
+  P.off_counters = take(4LL * P.n_counters);
+  P.off_families = take((long long)sizeof(FamilyDesc) * P.n_families);
+  P.off_expr = take(4LL * (long long)p.code.size());
+  P.off_instr = take((long long)sizeof(Instr) * (long long)p.instr.size());
+  P.off_layers = take((long long)sizeof(LayerPtrs) * P.n_layers);
+  P.off_rope = take(4LL * (long long)p.rope.size());
+  P.off_queue = take((long long)sizeof(QRange) * P.queue_ranges);
+  P.off_x = take(4LL * P.max_batch * P.hidden);
+  P.off_q = take(4LL * P.max_batch * P.n_q_heads * P.head_dim);
+  P.off_apart = take(4LL * P.max_batch * P.n_kv_heads * P.max_chunks * qpg * (P.head_dim + 2));
+  P.off_attn = take(4LL * P.max_batch * P.n_q_heads * P.head_dim);
+  P.off_h = take(4LL * P.max_batch * P.ffn);
+  P.off_dpart = take(4LL * P.n_kc * P.max_batch * P.hidden);
+  P.off_lmpart = take(8LL * P.max_batch * P.n_lm_tiles);
+  P.off_lmgpart = take(8LL * P.max_batch * P.n_lmgrp);
+  P.ws_bytes = off;
+  // image = [off_families, off_queue): the read-only plan arrays
+  image.assign((size_t)(P.off_queue - P.off_families), 0);
+  auto put = [&](long long at, const void* src, size_t n) {
+    if (n) std::memcpy(image.data() + (at - P.off_families), src, n);
+  };
+  put(P.off_families, p.fams.data(), sizeof(FamilyDesc) * p.fams.size());
+  put(P.off_expr, p.code.data(), 4 * p.code.size());
+  put(P.off_instr, p.instr.data(), sizeof(Instr) * p.instr.size());
+  put(P.off_layers, p.layers.data(), sizeof(LayerPtrs) * p.layers.size());
+  put(P.off_rope, p.rope.data(), 4 * p.rope.size());
+}
+
+// ---------------------------------------------------------------- bytes
+double step_bytes(const Plan& p, const Binding& bd, bool with_logits) {
+  const DevPlan& P = p.dp;
+  double H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads, F = P.ffn;
+  double per_layer = ((Hq + 2 * Hkv) * D * H + H * Hq * D + 3 * F * H + 2 * H) * 2.0;
+  double w = P.n_layers * per_layer + (double)P.vocab * H * 2.0 + H * 2.0;
+  double kv_row = Hkv * D * 2.0 * 2.0 * P.n_layers;  // K and V, all layers
+  double ctx_sum = 0;
+  for (int b = 0; b < bd.B; ++b) ctx_sum += bd.ctx[b];
+  double bytes = w + bd.B * H * 2.0 + kv_row * ctx_sum + kv_row * bd.B + bd.B * 4.0 * 2;
+  if (with_logits) bytes += 4.0 * P.vocab * bd.B;
+  return bytes;
+}
+
+// ---------------------------------------------------------------- validation
+static bool check_binding(const Plan& p, const Binding& bd, std::string& err) {
+  if (bd.B < 1 || bd.B > p.dp.max_batch) { err = "batch out of range"; return false; }
+  if ((int)bd.ctx.size() < bd.B) { err = "ctx_lens shorter than batch"; return false; }
+  for (int b = 0; b < bd.B; ++b)
+    if (bd.ctx[b] < 0 || bd.ctx[b] >= p.dp.max_ctx) { err = "ctx_lens[b] out of [0, max_ctx)"; return false; }
+  return true;
+}
+
+mk_status validate_plan(const Plan& p, const Binding& bd, std::string& err) {
+  if (!check_binding(p, bd, err)) return MK_ERR_INVALID_ARG;
+  const DevPlan& P = p.dp;
+  std::vector<int> notifiers(P.n_counters, 0);
+  std::vector<int> last_notifier_fam(P.n_counters, -1);
+  std::vector<int> wait_fams;  // (counter, fam) pairs
+  std::vector<std::pair<int, int>> waits;
+  TaskRec t;
+  std::vector<int> followups_seen(P.n_families, 0);
+  for (int f = 0; f < P.n_families; ++f) {
+    int n = p.family_extent(f, bd);
+    if (n < 0 || n > p.fams[f].max_extent) {
+      err = "family " + p.fam_names[f] + " extent exceeds its reserved maximum";
+      return MK_ERR_PLAN;
+    }
+    for (int i = 0; i < n; ++i) {
+      p.task(f, i, bd, t);
+      if (t.notify_ev >= 0) {
+        notifiers[t.notify_ev]++;
+        last_notifier_fam[t.notify_ev] = std::max(last_notifier_fam[t.notify_ev], f);
+      }
+      if (t.wait_ev >= 0) waits.push_back({t.wait_ev, f});
+      if (t.follow_fam >= 0 && t.follow_fam <= f) {
+        err = "follow-up family precedes its trigger";
+        return MK_ERR_PLAN;
+      }
+    }
+  }
+  // every armed count equals its number of notifiers
+  for (int e = 0; e < EV_COUNT; ++e) {
+    const EventTensorDesc& d = P.ev[e];
+    int d1 = d.ndim > 1 ? d.dims[1] : 1, d2 = d.ndim > 2 ? d.dims[2] : 1;
+    for (int a = 0; a < d.dims[0]; ++a)
+      for (int b = 0; b < d1; ++b)
+        for (int c = 0; c < d2; ++c) {
+          int ci = p.counter(e, a, b, c);
+          int cnt = p.event_count(e, a, b, c, bd);
+          if (cnt != notifiers[ci]) {
+            err = "event " + std::to_string(e) + " element (" + std::to_string(a) + "," + std::to_string(b) +
+                  "," + std::to_string(c) + ") waits for " + std::to_string(cnt) + " but has " +
+                  std::to_string(notifiers[ci]) + " notifiers";
+            return MK_ERR_PLAN;
+          }
+        }
+  }
+  // waits only on events notified by earlier families (acyclic, topological)
+  for (auto& w : waits)
+    if (last_notifier_fam[w.first] >= w.second) {
+      err = "family " + p.fam_names[w.second] + " waits on an event notified by a later family";
+      return MK_ERR_PLAN;
+    }
+  // static queues are sorted in family order (deadlock freedom)
+  for (int s = 0; s < P.n_sm; ++s) {
+    int prev = -1;
+    for (int k = 0; k < P.n_instr_per_sm; ++k) {
+      const Instr& in = p.instr[(size_t)s * P.n_instr_per_sm + k];
+      if (in.family < 0) break;
+      if (in.family <= prev) { err = "static queue out of topological order"; return MK_ERR_PLAN; }
+      prev = in.family;
+    }
+  }
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------- simulator
+namespace {
+
+struct VC {
+  std::vector<unsigned> c;
+  void join(const VC& o) { for (size_t i = 0; i < c.size(); ++i) c[i] = std::max(c[i], o.c[i]); }
+};
+
+struct Shadow {
+  int w_worker = -1;
+  unsigned w_clock = 0;
+  std::vector<unsigned> reads;  // per worker
+};
+
+struct Sim {
+  const Plan& p;
+  const Binding& bd;
+  int nw;
+  std::vector<VC> wvc;
+  std::vector<VC> evc;
+  std::vector<int> counters;
+  std::vector<std::unordered_map<long long, Shadow>> shadow;
+  int races = 0;
+  std::string first;
+  Sim(const Plan& pl, const Binding& b, int n) : p(pl), bd(b), nw(n), shadow(BUF_COUNT) {}
+
+  void access(int w, const Region& r, bool write) {
+    // shadow units: 4 elements for row data, 1 for per-task records
+    const long long G = (r.buf == BUF_APART || r.buf == BUF_LMPART || r.buf == BUF_LMG || r.buf == BUF_NEXT) ? 1 : 4;
+    for (long long u = r.lo / G; u <= (r.hi - 1) / G; ++u) {
+      Shadow& s = shadow[r.buf][u];
+      if (s.reads.empty()) s.reads.assign(nw, 0);
+      const VC& me = wvc[w];
+      bool ok = s.w_worker < 0 || s.w_worker == w || me.c[s.w_worker] >= s.w_clock;
+      if (write)
+        for (int r2 = 0; r2 < nw && ok; ++r2)
+          if (r2 != w && s.reads[r2] > me.c[r2]) ok = false;
+      if (!ok) {
+        if (!races) first = "unordered access to buffer " + std::to_string(r.buf) + " unit " + std::to_string(u);
+        races++;
+      }
+      if (write) { s.w_worker = w; s.w_clock = me.c[w]; std::fill(s.reads.begin(), s.reads.end(), 0); }
+      else s.reads[w] = std::max(s.reads[w], me.c[w]);
+    }
+  }
+};
+
+struct Work {
+  int fam, idx;
+  std::vector<unsigned> vc;  // dynamic: clock snapshot carried by a pushed task
+};
+
+}  // namespace
+
+static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt19937& rng, int fault,
+                     int fault_family, std::vector<int>& exec_count, mk_sim_report* rep) {
+  const DevPlan& P = p.dp;
+  int nw = std::max(1, std::min(P.n_sm, 64));
+  Sim sim(p, bd, nw);
+  sim.wvc.assign(nw, VC{std::vector<unsigned>(nw, 0)});
+  sim.evc.assign(P.n_counters, VC{std::vector<unsigned>(nw, 0)});
+  sim.counters.assign(P.n_counters, 0);
+  bool fault_done = false;
+  for (int e = 0; e < EV_COUNT; ++e) {
+    const EventTensorDesc& d = P.ev[e];
+    int d1 = d.ndim > 1 ? d.dims[1] : 1, d2 = d.ndim > 2 ? d.dims[2] : 1;
+    for (int a = 0; a < d.dims[0]; ++a)
+      for (int b = 0; b < d1; ++b)
+        for (int c = 0; c < d2; ++c) sim.counters[p.counter(e, a, b, c)] = p.event_count(e, a, b, c, bd);
+  }
+  if (fault == MK_SIM_FAULT_COUNT_PLUS_ONE && fault_family >= 0 && fault_family < P.n_families) {
+    TaskRec t0;
+    if (p.family_extent(fault_family, bd) > 0) {
+      p.task(fault_family, 0, bd, t0);
+      if (t0.notify_ev >= 0) sim.counters[t0.notify_ev] += 1;
+    }
+  }
+  std::vector<int> ext(P.n_families);
+  for (int f = 0; f < P.n_families; ++f) ext[f] = p.family_extent(f, bd);
+
+  // per-worker task sources
+  std::vector<std::vector<Work>> local(nw);   // static: own queue; both: follow-ups
+  std::vector<size_t> pos(nw, 0);
+  std::vector<std::vector<Work>> follow(nw);
+  std::vector<Work> shared;                   // dynamic queue (FIFO)
+  size_t shared_head = 0;
+  if (!dynamic) {
+    // simulated SM w plays the SMs congruent to w mod nw, in queue order
+    for (int s = 0; s < P.n_sm; ++s) {
+      int w = s % nw;
+      for (int k = 0; k < P.n_instr_per_sm; ++k) {
+        const Instr& in = p.instr[(size_t)s * P.n_instr_per_sm + k];
+        if (in.family < 0) break;
+        for (int i = in.start; i < ext[in.family]; i += in.stride) local[w].push_back({in.family, i, {}});
+      }
+    }
+    for (int w = 0; w < nw; ++w)
+      std::stable_sort(local[w].begin(), local[w].end(),
+                       [](const Work& a, const Work& b) { return a.fam < b.fam; });
+  } else {
+    std::vector<int> succ;
+    for (int ci = 0; ci < P.n_counters; ++ci)
+      if (sim.counters[ci] == 0) {
+        succ.clear();
+        p.successors(ci, bd, succ);
+        for (size_t k = 0; k < succ.size(); k += 3)
+          for (int i = 0; i < succ[k + 2]; ++i) shared.push_back({succ[k], succ[k + 1] + i, std::vector<unsigned>(nw, 0)});
+      }
+  }
+  TaskRec t;
+  int executed = 0;
+  auto exec = [&](int w, const Work& wk) {
+    VC& me = sim.wvc[w];
+    me.c[w]++;
+    p.task(wk.fam, wk.idx, bd, t);
+    if (!wk.vc.empty()) { VC v{wk.vc}; me.join(v); }
+    bool skip_wait = fault == MK_SIM_FAULT_NO_WAIT && wk.fam == fault_family;
+    if (t.wait_ev >= 0 && !skip_wait) me.join(sim.evc[t.wait_ev]);
+    for (auto& r : t.reads) sim.access(w, r, false);
+    for (auto& r : t.writes) sim.access(w, r, true);
+    exec_count[p.fams[wk.fam].debug_base + wk.idx]++;
+    executed++;
+    if (t.notify_ev >= 0) {
+      if (fault == MK_SIM_FAULT_DROP_NOTIFY && wk.fam == fault_family && !fault_done) { fault_done = true; return; }
+      sim.evc[t.notify_ev].join(me);
+      int old = sim.counters[t.notify_ev]--;
+      if (old == 1) {
+        me.join(sim.evc[t.notify_ev]);  // the last notifier acquires every release
+        if (t.follow_fam >= 0) follow[w].push_back({t.follow_fam, t.follow_idx, {}});
+        if (dynamic) {
+          std::vector<int> succ;
+          p.successors(t.notify_ev, bd, succ);
+          for (size_t k = 0; k < succ.size(); k += 3)
+            for (int i = 0; i < succ[k + 2]; ++i) shared.push_back({succ[k], succ[k + 1] + i, me.c});
+        }
+      }
+    }
+  };
+  auto ready = [&](int w) -> int {  // 1 follow-up, 2 regular, 0 blocked
+    if (!follow[w].empty()) return 1;
+    if (!dynamic) {
+      if (pos[w] >= local[w].size()) return 0;
+      TaskRec tr;
+      p.task(local[w][pos[w]].fam, local[w][pos[w]].idx, bd, tr);
+      bool skip_wait = fault == MK_SIM_FAULT_NO_WAIT && local[w][pos[w]].fam == fault_family;
+      if (tr.wait_ev >= 0 && sim.counters[tr.wait_ev] != 0 && !skip_wait) return 0;
+      return 2;
+    }
+    return shared_head < shared.size() ? 2 : 0;
+  };
+  std::vector<int> cand;
+  for (;;) {
+    cand.clear();
+    for (int w = 0; w < nw; ++w)
+      if (ready(w)) cand.push_back(w);
+    if (cand.empty()) break;
+    int w = cand[rng() % cand.size()];
+    int kind = ready(w);
+    if (kind == 1) {
+      // follow-ups run in LIFO order on the notifier, like the device
+      Work wk = follow[w].back();
+      follow[w].pop_back();
+      exec(w, wk);
+    } else if (!dynamic) {
+      exec(w, local[w][pos[w]++]);
+    } else {
+      Work wk = shared[shared_head++];
+      exec(w, wk);
+    }
+  }
+  bool left = false;
+  for (int w = 0; w < nw; ++w)
+    if ((!dynamic && pos[w] < local[w].size()) || !follow[w].empty()) left = true;
+  if (dynamic && shared_head < shared.size()) left = true;
+  // a plan that stops before the final task has deadlocked
+  int fin = p.fam_index(OP_LMFIN, -1);
+  if (exec_count[p.fams[fin].debug_base] == 0) left = true;
+  if (left) rep->deadlocks++;
+  for (int ci = 0; ci < P.n_counters; ++ci)
+    if (sim.counters[ci] != 0) { rep->nonzero_counters++; break; }
+  rep->races += sim.races;
+  if (sim.races && !rep->first_error[0])
+    std::snprintf(rep->first_error, sizeof(rep->first_error), "%s", sim.first.c_str());
+  if (left && !rep->first_error[0])
+    std::snprintf(rep->first_error, sizeof(rep->first_error), "order stopped with tasks left (deadlock)");
+  rep->tasks_per_order = executed;
+  return executed;
+}
+
+mk_status simulate_plan(const Plan& p, const Binding& bd, int n_orders, unsigned seed, int fault,
+                        int fault_family, mk_sim_report* rep) {
+  std::string err;
+  std::memset(rep, 0, sizeof(*rep));
+  if (!check_binding(p, bd, err)) {
+    std::snprintf(rep->first_error, sizeof(rep->first_error), "%s", err.c_str());
+    return MK_ERR_INVALID_ARG;
+  }
+  std::mt19937 rng(seed);
+  std::vector<int> want(p.dp.debug_slots, 0);
+  for (int f = 0; f < p.dp.n_families; ++f)
+    for (int i = 0; i < p.family_extent(f, bd); ++i) want[p.fams[f].debug_base + i] = 1;
+  std::vector<int> first_set;
+  for (int k = 0; k < n_orders; ++k) {
+    bool dynamic = (k % 2) == 1;
+    std::vector<int> exec_count(p.dp.debug_slots, 0);
+    run_order(p, bd, dynamic, rng, fault, fault_family, exec_count, rep);
+    rep->orders_run++;
+    if (exec_count != want) {
+      rep->exactly_once_violations++;
+      if (!rep->first_error[0]) std::snprintf(rep->first_error, sizeof(rep->first_error), "task set differs from the plan's");
+    }
+    std::vector<int> set(exec_count.size());
+    for (size_t i = 0; i < set.size(); ++i) set[i] = exec_count[i] > 0;
+    if (k == 0) first_set = set;
+    else if (set != first_set) rep->static_dynamic_mismatch = 1;
+  }
+  bool bad = rep->races || rep->deadlocks || rep->exactly_once_violations || rep->nonzero_counters ||
+             rep->static_dynamic_mismatch;
+  return bad ? MK_ERR_PLAN : MK_OK;
+}
+
+}  // namespace mk

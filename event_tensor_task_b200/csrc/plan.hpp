@@ -1,0 +1,86 @@
+// plan.hpp — host task-graph compiler for the decode megakernel.
+//
+// Builds, from a model description, the task families (tiles of every op,
+// with symbolic extents), the Event Tensors (shapes and symbolic wait
+// counts), the static per-SM instruction queues and the dynamic successor
+// rules, and lowers them into the flat arrays the device interpreter reads
+// ("Event Tensor: A Unified Abstraction for Compiling Dynamic Megakernel",
+// section "Core method": event tensors as first-class compiler objects,
+// static and dynamic scheduling transformations, lowering of events to plain
+// integer counters).
+#pragma once
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "plan_format.h"
+
+namespace mk {
+
+// Host-side record of one task for one binding of the symbols.
+enum Buf : int {
+  BUF_X = 0, BUF_Q, BUF_KC, BUF_VC, BUF_APART, BUF_ATTN, BUF_H, BUF_DPART,
+  BUF_LMPART, BUF_LMG, BUF_LOGITS, BUF_NEXT, BUF_COUNT
+};
+
+struct Region {
+  int buf;
+  long long lo, hi;  // element range [lo, hi)
+};
+
+struct TaskRec {
+  int fam = -1;
+  int idx = -1;
+  int wait_ev = -1;       // counter index waited on (-1: none)
+  int notify_ev = -1;     // counter index decremented at completion (-1: none)
+  int follow_fam = -1;    // follow-up family run by the notifier that reaches zero
+  int follow_idx = -1;
+  std::vector<Region> reads, writes;
+};
+
+struct Binding {
+  int B;
+  std::vector<int> ctx;
+};
+
+struct Plan {
+  mk_model_desc m{};
+  std::vector<mk_layer_weights> layer_w;
+  mk_plan_opts o{};
+  DevPlan dp{};
+  std::vector<FamilyDesc> fams;
+  std::vector<std::string> fam_names;
+  std::vector<int32_t> code;
+  std::vector<Instr> instr;         // [n_sm][n_instr_per_sm]
+  std::vector<LayerPtrs> layers;
+  std::vector<float> rope;          // [max_ctx][head_dim/2][2] cos, sin
+  int device = -1;
+  void* ws = nullptr;
+  size_t ws_bound = 0;
+  unsigned epoch = 0;
+  long long launches = 0;
+
+  // host model of the task graph
+  int fam_index(int op, int layer) const;
+  int counter(int ev, int c0, int c1 = 0, int c2 = 0) const;
+  int event_count(int ev, int c0, int c1, int c2, const Binding& bd) const;
+  int family_extent(int f, const Binding& bd) const;
+  void task(int f, int idx, const Binding& bd, TaskRec& t) const;
+  // dynamic successors of a counter that reached zero: (family, lo, count) ranges
+  void successors(int counter_index, const Binding& bd, std::vector<int>& out3) const;
+  int total_counters() const { return dp.n_counters; }
+};
+
+// Build; returns MK_OK or an error with `err` set.
+mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, int smem_bytes,
+                     Plan& p, std::string& err);
+mk_status validate_plan(const Plan& p, const Binding& bd, std::string& err);
+mk_status simulate_plan(const Plan& p, const Binding& bd, int n_orders, unsigned seed, int fault,
+                        int fault_family, mk_sim_report* rep);
+double step_bytes(const Plan& p, const Binding& bd, bool with_logits);
+
+// Lowered plan image (families, expressions, instructions, layer pointers,
+// rope table) with the offsets recorded in p.dp.
+void lower_plan(Plan& p, std::vector<unsigned char>& image);
+
+}  // namespace mk

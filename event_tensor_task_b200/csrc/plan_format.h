@@ -1,0 +1,250 @@
+// plan_format.h — the lowered plan as the megakernel reads it, plus the
+// symbolic-expression bytecode and the task-index decoding that the host
+// compiler and the device interpreter share.
+//
+// Symbolic extents follow "Event Tensor: A Unified Abstraction for Compiling
+// Dynamic Megakernel", section "Core method" (shape dynamism: event-tensor
+// dimensions may be symbolic, e.g. the batch size B, and one runtime is
+// instantiated from the actual values) and "Lecture 112: Production
+// Megakernels for Real-World Inference", section "Symbolic Representation of
+// Work" (extents and barriers are expressions in the runtime sizes, so the
+// work queue is never rebuilt).  Every extent and every wait count is a small
+// postfix program over the symbols B (batch), ctx[b] (per-sequence context)
+// and the coordinates of the event element being armed.
+#pragma once
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define MK_HD __host__ __device__ __forceinline__
+#else
+#define MK_HD inline
+#endif
+
+namespace mk {
+
+// ---------------------------------------------------------------- ops
+enum Op : int32_t {
+  OP_END = 0,
+  OP_QKV = 1,     // RMSNorm -> Q/K/V rows -> RoPE -> KV append
+  OP_ATTN = 2,    // one key chunk of one (sequence, kv head) -> softmax partials
+  OP_MERGE = 3,   // follow-up: merge a head group's chunk partials
+  OP_OPROJ = 4,   // output projection rows + residual
+  OP_GATEUP = 5,  // RMSNorm -> gate and up rows -> SwiGLU
+  OP_DOWN = 6,    // down projection rows over one K segment -> partial
+  OP_DRED = 7,    // follow-up: sum the K-segment partials into the residual
+  OP_LM = 8,      // final RMSNorm -> vocabulary rows -> logits + tile argmax
+  OP_LMGRP = 9,   // follow-up: argmax over a group of LM tiles
+  OP_LMFIN = 10,  // follow-up: argmax over the groups -> next token
+  OP_COUNT = 11
+};
+
+// ---------------------------------------------------------------- expressions
+// Postfix bytecode; every program ends with X_RET.  X_SUM_B len sums the
+// next `len` words (a program without X_SUM_B, ended by X_RET) over
+// b = 0..B-1 with X_VAR pushing b.
+enum XOp : int32_t {
+  X_RET = 0,
+  X_PUSH = 1,     // operand follows
+  X_B = 2,        // batch size
+  X_COORD = 3,    // operand d: coordinate d of the element being evaluated
+  X_CTX_AT = 4,   // pop i; push ctx[i] (0 when i >= B)
+  X_VAR = 5,      // loop variable of the enclosing X_SUM_B
+  X_ADD = 6, X_SUB = 7, X_MUL = 8,
+  X_CEILDIV = 9,  // pop d, a; push ceil(a / d)
+  X_MIN = 10, X_MAX = 11,
+  X_LT = 12,      // pop b, a; push a < b
+  X_SUM_B = 13,   // operand len; body of len words follows
+};
+
+struct ExprEnv {
+  int B;
+  const int* ctx;   // [B]
+  int coord[3];
+};
+
+MK_HD int expr_flat(const int32_t* code, int pc, const ExprEnv& env, int var) {
+  int st[12];
+  int sp = 0;
+  for (;;) {
+    int op = code[pc++];
+    switch (op) {
+      case X_RET: return sp > 0 ? st[sp - 1] : 0;
+      case X_PUSH: st[sp++] = code[pc++]; break;
+      case X_B: st[sp++] = env.B; break;
+      case X_COORD: st[sp++] = env.coord[code[pc++]]; break;
+      case X_CTX_AT: { int i = st[sp - 1]; st[sp - 1] = (i >= 0 && i < env.B) ? env.ctx[i] : 0; } break;
+      case X_VAR: st[sp++] = var; break;
+      case X_ADD: sp--; st[sp - 1] = st[sp - 1] + st[sp]; break;
+      case X_SUB: sp--; st[sp - 1] = st[sp - 1] - st[sp]; break;
+      case X_MUL: sp--; st[sp - 1] = st[sp - 1] * st[sp]; break;
+      case X_CEILDIV: sp--; st[sp - 1] = (st[sp - 1] + st[sp] - 1) / st[sp]; break;
+      case X_MIN: sp--; st[sp - 1] = st[sp - 1] < st[sp] ? st[sp - 1] : st[sp]; break;
+      case X_MAX: sp--; st[sp - 1] = st[sp - 1] > st[sp] ? st[sp - 1] : st[sp]; break;
+      case X_LT: sp--; st[sp - 1] = st[sp - 1] < st[sp] ? 1 : 0; break;
+      default: return -1;
+    }
+  }
+}
+
+MK_HD int expr_eval(const int32_t* code, int pc, const ExprEnv& env) {
+  int st[12];
+  int sp = 0;
+  for (;;) {
+    int op = code[pc++];
+    switch (op) {
+      case X_RET: return sp > 0 ? st[sp - 1] : 0;
+      case X_PUSH: st[sp++] = code[pc++]; break;
+      case X_B: st[sp++] = env.B; break;
+      case X_COORD: st[sp++] = env.coord[code[pc++]]; break;
+      case X_CTX_AT: { int i = st[sp - 1]; st[sp - 1] = (i >= 0 && i < env.B) ? env.ctx[i] : 0; } break;
+      case X_ADD: sp--; st[sp - 1] = st[sp - 1] + st[sp]; break;
+      case X_SUB: sp--; st[sp - 1] = st[sp - 1] - st[sp]; break;
+      case X_MUL: sp--; st[sp - 1] = st[sp - 1] * st[sp]; break;
+      case X_CEILDIV: sp--; st[sp - 1] = (st[sp - 1] + st[sp] - 1) / st[sp]; break;
+      case X_MIN: sp--; st[sp - 1] = st[sp - 1] < st[sp] ? st[sp - 1] : st[sp]; break;
+      case X_MAX: sp--; st[sp - 1] = st[sp - 1] > st[sp] ? st[sp - 1] : st[sp]; break;
+      case X_LT: sp--; st[sp - 1] = st[sp - 1] < st[sp] ? 1 : 0; break;
+      case X_SUM_B: {
+        int len = code[pc++];
+        int s = 0;
+        for (int b = 0; b < env.B; ++b) s += expr_flat(code, pc, env, b);
+        st[sp++] = s;
+        pc += len;
+      } break;
+      default: return -1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- lowered plan
+// Event-tensor slots of the dense decoder (index into DevPlan::ev).
+enum EvId : int32_t {
+  EV_IN = 0,     // [L+1]        layer input ready (element l+1 notified by layer l's reductions)
+  EV_QKV = 1,    // [L][Hkv]     Q/K/V rows of one kv-head group written
+  EV_CHUNK = 2,  // [L][maxB][Hkv] key-chunk partials of one (b, g) written
+  EV_ATTN = 3,   // [L]          all head groups merged
+  EV_O = 4,      // [L]          output projection done
+  EV_GU = 5,     // [L][n_kc]    SwiGLU outputs of one K segment written
+  EV_DSUM = 6,   // [L][n_dtiles] K-segment partials of one row tile written
+  EV_LMG = 7,    // [n_lmgrp]    LM tiles of one group done
+  EV_LM = 8,     // [1]          all LM groups reduced
+  EV_COUNT = 9
+};
+
+struct EventTensorDesc {
+  int32_t base;        // first counter of this tensor in the counter array
+  int32_t ndim;
+  int32_t dims[3];     // maximum extents
+  int32_t count_expr;  // wait count of an element, a program over its coordinates
+};
+
+struct FamilyDesc {
+  int32_t op;
+  int32_t layer;       // -1 for the LM families
+  int32_t extent_expr; // number of tasks, a program over B and ctx
+  int32_t max_extent;
+  int32_t debug_base;
+  int32_t followup;    // 1: executed by the last notifier of its trigger event
+  int32_t pad[2];
+};
+
+// One static-schedule instruction: run tasks start, start+stride, ... of a
+// family while the index is below the family's evaluated extent.
+struct Instr {
+  int32_t family;
+  int32_t start;
+  int32_t stride;
+  int32_t pad;
+};
+
+struct LayerPtrs {
+  const void* attn_norm; const void* wq; const void* wk; const void* wv; const void* wo;
+  const void* ffn_norm; const void* w_gate; const void* w_up; const void* w_down;
+};
+
+constexpr int kMaxFamilies = 256;
+constexpr int kMaxBatch = 128;
+
+// Fixed header of the plan; passed to the kernel by value.  Offsets are in
+// bytes from the workspace base.
+struct DevPlan {
+  int32_t sched, n_sm, n_families, n_instr_per_sm;
+  int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+  int32_t max_batch, max_ctx, n_slots;
+  float eps;
+  int32_t tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, lm_group, chunk;
+  int32_t n_qkv_tiles, n_otiles, n_gutiles, n_dtiles, n_kc, n_lm_tiles, n_lmgrp, max_chunks;
+  int32_t ring_slots, slot_bytes, smem_bytes;
+  int32_t n_counters, debug_slots, queue_ranges;
+  uint32_t debug_flags;
+  int32_t pad0;
+  int64_t spin_timeout_ns;
+  EventTensorDesc ev[EV_COUNT];
+  int32_t fam_first_layer[OP_COUNT];  // family index of (op, layer 0), or of the op for LM families
+  int32_t fam_stride;                 // families per layer
+  int32_t pad1;
+  // workspace offsets
+  int64_t off_control, off_counters, off_families, off_expr, off_instr, off_layers, off_rope;
+  int64_t off_queue, off_x, off_q, off_apart, off_attn, off_h, off_dpart, off_lmpart, off_lmgpart;
+  int64_t ws_bytes;
+  // global weights (device)
+  const void* embed; const void* lm_head; const void* final_norm;
+  void* k_cache; void* v_cache;
+};
+
+// Control block at off_control (first 256 bytes of the workspace).
+struct Control {
+  int32_t status_code, status_family, status_index, status_event, status_sm;
+  int32_t abort;
+  uint32_t grid_bar;        // monotonic grid-barrier arrivals
+  uint32_t pad0;
+  unsigned long long q_tail;  // dynamic queue: (ranges << 40) | tasks reserved
+  unsigned long long q_head;  // dynamic queue: tasks popped
+  int32_t pad[52];
+};
+
+// Dynamic queue entry: a contiguous range of tasks of one family.
+struct QRange {
+  int32_t family;
+  int32_t lo;          // first task index
+  int32_t count;
+  uint32_t seq;        // (epoch << 20 | range index) + 1 once published
+  unsigned long long start;  // ticket of the first task of the range
+};
+
+// ---------------------------------------------------------------- task decoding
+// QKV tile i covers rows j0..j0+R/2-1 and j0+D/2.. of head hh (q heads, then
+// k heads, then v heads); R = tile_qkv, rotate-half pairs stay in one tile.
+struct QkvTile { int hh; int kind; int head; int group; int j0; };
+MK_HD QkvTile decode_qkv(const DevPlan& P, int i) {
+  QkvTile t;
+  int per_head = P.head_dim / P.tile_qkv;
+  t.hh = i / per_head;
+  t.j0 = (i % per_head) * (P.tile_qkv / 2);
+  int qpg = P.n_q_heads / P.n_kv_heads;
+  if (t.hh < P.n_q_heads) { t.kind = 0; t.head = t.hh; t.group = t.hh / qpg; }
+  else if (t.hh < P.n_q_heads + P.n_kv_heads) { t.kind = 1; t.head = t.hh - P.n_q_heads; t.group = t.head; }
+  else { t.kind = 2; t.head = t.hh - P.n_q_heads - P.n_kv_heads; t.group = t.head; }
+  return t;
+}
+
+// ATTN task i -> (b, g, c) given per-sequence chunk counts nch[] and their
+// exclusive prefix pre[] (index = Hkv * pre[b] + g * nch[b] + c).
+struct AttnTask { int b, g, c; };
+MK_HD AttnTask decode_attn(int i, int B, int Hkv, const int* nch, const int* pre) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {  // largest b with Hkv * pre[b] <= i
+    int mid = (lo + hi + 1) >> 1;
+    if (Hkv * pre[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  AttnTask t;
+  t.b = lo;
+  int r = i - Hkv * pre[lo];
+  t.g = r / nch[lo];
+  t.c = r % nch[lo];
+  return t;
+}
+
+MK_HD int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace mk

@@ -1,0 +1,220 @@
+/*
+ * mk.h — C ABI of the B200 decode megakernel (libmk.so).
+ *
+ * One persistent kernel runs a whole transformer decode step as a task graph
+ * synchronised by Event Tensors ("Event Tensor: A Unified Abstraction for
+ * Compiling Dynamic Megakernel", section "Core method": an event tensor is a
+ * multi-dimensional array of events, each the completion of a set of
+ * SM-granular tasks with a wait count; notify() is an atomic decrement and
+ * wait() spins until zero; event dimensions may be symbolic in the batch
+ * size; tasks are scheduled statically to per-SM queues or dynamically
+ * through a shared queue).  The on-device interpreter is a loop over a switch
+ * that takes tasks from a queue in device memory ("Lecture 112: Production
+ * Megakernels for Real-World Inference", section "Execution Model").
+ *
+ * Conventions for every call below:
+ *  - No C++ exception crosses this boundary.  Every call returns an
+ *    mk_status; on failure mk_last_error() returns a message for the calling
+ *    thread (valid until that thread's next mk_* call).
+ *  - "device" pointers are CUDA device addresses on the plan's device;
+ *    "host" pointers are ordinary host memory.  All weights, caches, inputs,
+ *    outputs and the workspace are owned by the caller and must outlive the
+ *    plan.  A plan owns host memory only.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Shapes are symbolic: one plan and one compiled kernel serve every batch
+ *    size B <= max_batch and every context length < max_ctx, with no
+ *    recompilation and no graph re-capture.
+ */
+#ifndef MK_H_
+#define MK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int mk_status;
+#define MK_OK 0
+#define MK_ERR_INVALID_ARG -1   /* a pointer, size or option is out of range */
+#define MK_ERR_UNSUPPORTED -2   /* valid request that this build does not implement */
+#define MK_ERR_WORKSPACE -3     /* workspace missing, too small or misaligned */
+#define MK_ERR_CUDA -4          /* a CUDA runtime call failed (message has the CUDA error) */
+#define MK_ERR_DEVICE_TIMEOUT -5 /* a device spin-wait ran past its limit (see mk_get_status) */
+#define MK_ERR_DEVICE_BOUNDS -6 /* the device rejected an index (bad token, slot or context) */
+#define MK_ERR_PLAN -7          /* plan validation or simulation found an error */
+
+#define MK_SCHED_STATIC 0   /* per-SM task queues fixed at plan build, counter waits */
+#define MK_SCHED_DYNAMIC 1  /* shared device queue; a task is pushed when its event fires */
+
+#define MK_MODEL_DENSE 0     /* dense decoder: attention + SwiGLU FFN per layer */
+
+#define MK_DEBUG_TASK_COUNTS 1u  /* each executed task increments its slot in mk_step_args.task_counts */
+
+/* Per-layer weights of a dense decoder; bf16, row-major [out][in], device. */
+typedef struct mk_layer_weights {
+  const void* attn_norm;  /* [hidden] RMSNorm gain before attention */
+  const void* wq;         /* [n_q_heads*head_dim][hidden] */
+  const void* wk;         /* [n_kv_heads*head_dim][hidden] */
+  const void* wv;         /* [n_kv_heads*head_dim][hidden] */
+  const void* wo;         /* [hidden][n_q_heads*head_dim] */
+  const void* ffn_norm;   /* [hidden] RMSNorm gain before the FFN */
+  const void* w_gate;     /* [ffn][hidden] */
+  const void* w_up;       /* [ffn][hidden] */
+  const void* w_down;     /* [hidden][ffn] */
+} mk_layer_weights;
+
+/* Model description.  Dimensions must satisfy: head_dim == 64,
+ * n_q_heads % n_kv_heads == 0, hidden and ffn multiples of 256 with
+ * hidden <= 2048, n_q_heads*head_dim == hidden. */
+typedef struct mk_model_desc {
+  int kind;               /* MK_MODEL_DENSE */
+  int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+  float eps;              /* RMSNorm epsilon */
+  float rope_theta;       /* rotary base; pair i of a head turns by pos*theta^(-2i/head_dim) */
+  int max_batch;          /* largest B a step may use */
+  int max_ctx;            /* cache capacity in positions (ctx_lens[b] < max_ctx) */
+  int n_slots;            /* sequences the KV cache holds */
+  const void* embed;      /* [vocab][hidden] bf16, device */
+  const void* lm_head;    /* [vocab][hidden] bf16, device; NULL = tied to embed */
+  const void* final_norm; /* [hidden] bf16, device */
+  const mk_layer_weights* layers; /* host array [n_layers] of device pointers */
+  void* k_cache;          /* bf16 [n_layers][n_slots][n_kv_heads][max_ctx][head_dim], device, post-RoPE keys */
+  void* v_cache;          /* bf16, same layout as k_cache */
+} mk_model_desc;
+
+/* Plan options; zero-initialise and set what you need (0 = default). */
+typedef struct mk_plan_opts {
+  int sched;              /* MK_SCHED_STATIC or MK_SCHED_DYNAMIC */
+  int n_sm;               /* CTAs of the persistent kernel; 0 = SMs of the current device */
+  int host_only;          /* 1: build without touching a GPU (validation/simulation only) */
+  int smem_bytes;         /* dynamic shared memory per CTA; 0 = device opt-in maximum */
+  int tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, lm_group, attn_chunk;
+  long long spin_timeout_ns; /* device spin-wait limit; 0 = 2 s */
+  unsigned debug_flags;   /* MK_DEBUG_* bits */
+} mk_plan_opts;
+
+typedef struct mk_plan mk_plan;
+
+/* Arguments of one decode step.  All arrays are device memory. */
+typedef struct mk_step_args {
+  int batch;              /* B, 1 <= B <= max_batch */
+  const int* token_ids;   /* int32 [B]: input token of each sequence */
+  const int* slot_ids;    /* int32 [B]: KV-cache slot of each sequence (distinct) */
+  const int* ctx_lens;    /* int32 [B]: cached tokens; the new token sits at this position */
+  float* logits;          /* fp32 [B][vocab] or NULL */
+  int* next_tokens;       /* int32 [B]: greedy argmax (ties -> lowest id) */
+  unsigned* task_counts;  /* uint32 [mk_plan_task_slots()] or NULL; zeroed by the caller */
+} mk_step_args;
+
+typedef struct mk_device_status {
+  int code;               /* MK_OK or MK_ERR_DEVICE_* */
+  int family;             /* family index of the task that failed, or -1 */
+  int index;              /* task index within its family, or -1 */
+  int event;              /* event counter index involved, or -1 */
+  int sm;                 /* CTA that recorded the error */
+} mk_device_status;
+
+typedef struct mk_family_info {
+  int op;                 /* MK_OP_* */
+  int layer;              /* layer, or -1 for the LM-head families */
+  int debug_base;         /* first slot of this family in task_counts */
+  int max_extent;         /* slots reserved (largest extent over all bindings) */
+  int followup;           /* 1: run by the task whose notify took an event to zero */
+  char name[16];
+} mk_family_info;
+
+#define MK_OP_QKV 1
+#define MK_OP_ATTN 2
+#define MK_OP_MERGE 3
+#define MK_OP_OPROJ 4
+#define MK_OP_GATEUP 5
+#define MK_OP_DOWN 6
+#define MK_OP_DRED 7
+#define MK_OP_LM 8
+#define MK_OP_LMGRP 9
+#define MK_OP_LMFIN 10
+
+typedef struct mk_sim_report {
+  int orders_run;         /* random interleavings executed */
+  int tasks_per_order;    /* tasks executed in the last order */
+  int races;              /* conflicting accesses not ordered by events */
+  int deadlocks;          /* orders that stopped with work left */
+  int exactly_once_violations;
+  int nonzero_counters;   /* event counters not at zero after an order */
+  int static_dynamic_mismatch; /* 1 if the two schedules executed different task sets */
+  char first_error[160];
+} mk_sim_report;
+
+/* Fault injected into the plan simulator (host only). */
+#define MK_SIM_FAULT_NONE 0
+#define MK_SIM_FAULT_DROP_NOTIFY 1   /* one task of `fault_family` skips its notify */
+#define MK_SIM_FAULT_COUNT_PLUS_ONE 2 /* the wait count of one event of `fault_family` is one too high */
+#define MK_SIM_FAULT_NO_WAIT 3       /* tasks of `fault_family` do not wait on their event */
+
+/* Last error message of the calling thread ("" if none). */
+const char* mk_last_error(void);
+
+/* Build a plan: validates `m`, tiles every op into task families with
+ * symbolic extents, derives the Event Tensors (shapes and wait-count
+ * expressions), builds the static per-SM queues and the dynamic successor
+ * rules, lowers them to flat integer arrays and validates the result.
+ * Host-only and synchronous; touches no GPU when opts->host_only is 1.
+ * On success *out owns the plan (free with mk_plan_destroy). */
+mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_plan** out);
+
+/* Device workspace the plan needs (bytes, 256-byte aligned start required). */
+size_t mk_plan_workspace_bytes(const mk_plan* p);
+
+/* Bind caller-allocated device workspace and upload the lowered plan into it
+ * (asynchronous on `stream`).  Must be called before mk_decode_step. */
+mk_status mk_plan_bind_workspace(mk_plan* p, void* dev_ptr, size_t bytes, void* stream);
+
+/* One decode step: a single launch of the persistent megakernel on `stream`.
+ * Asynchronous; returns launch and argument errors only.  Device-side errors
+ * are read with mk_get_status after the stream has synchronised. */
+mk_status mk_decode_step(mk_plan* p, const mk_step_args* a, void* stream);
+
+/* Read the device status word (synchronous copy).  Returns the recorded
+ * device code (MK_OK if none).  After a device error, call mk_plan_reset. */
+mk_status mk_get_status(mk_plan* p, mk_device_status* st);
+
+/* Clear the device control block (status, barrier and queue counters). */
+mk_status mk_plan_reset(mk_plan* p, void* stream);
+
+/* Task-count slots of the debug counter array (mk_step_args.task_counts). */
+int mk_plan_task_slots(const mk_plan* p);
+int mk_plan_num_families(const mk_plan* p);
+mk_status mk_plan_family_info(const mk_plan* p, int family, mk_family_info* out);
+
+/* Tile sizes the plan chose, in this order: tile_qkv, tile_o, tile_gu,
+ * tile_down, kseg, tile_lm, lm_group, attn_chunk, n_sm, ring_slots. */
+mk_status mk_plan_tiles(const mk_plan* p, int* out10);
+
+/* Host validation for one binding of the symbols (B, ctx_lens host array):
+ * every event's wait count equals its number of notifiers, every wait
+ * targets an event notified only by tasks earlier in the topological order,
+ * and the static queues are deadlock-free.  MK_OK or MK_ERR_PLAN. */
+mk_status mk_plan_validate(const mk_plan* p, int batch, const int* ctx_lens_host);
+
+/* Plan simulator (race detector): executes the lowered plan on the host in
+ * `n_orders` seeded random interleavings of n_sm simulated SMs, with task
+ * bodies that only record the memory regions they read and write.  Checks
+ * that every conflicting access pair is ordered by events (vector clocks),
+ * that every task runs exactly once, that every counter ends at zero, and
+ * that the static and dynamic schedules run the same task set. */
+mk_status mk_plan_simulate(const mk_plan* p, int batch, const int* ctx_lens_host,
+                           int n_orders, unsigned seed, int fault, int fault_family,
+                           mk_sim_report* report);
+
+/* Total bytes of weights, KV reads/writes and outputs one step moves for a
+ * binding (the algorithmic HBM traffic of the step). */
+double mk_plan_step_bytes(const mk_plan* p, int batch, const int* ctx_lens_host, int with_logits);
+
+void mk_plan_destroy(mk_plan* p);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H_ */

@@ -1,0 +1,115 @@
+"""Host-only tests of the C ABI and the task-graph compiler (no GPU needed).
+
+The plan simulator is the race detector: it runs the lowered plan in seeded
+random interleavings with vector clocks over the regions each task reads and
+writes, and checks exactly-once execution, counters at zero, and that static
+and dynamic scheduling run the same task set.
+"""
+import os
+import re
+
+import pytest
+
+import event_tensor_task_b200 as mk
+import workloads as wl
+from oracle import tasks as ot
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_library_exports_every_declared_symbol():
+    hdr = open(os.path.join(ROOT, "include", "mk.h")).read()
+    declared = set(re.findall(r"\b(mk_[a-z_]+)\s*\(", hdr))
+    assert declared, "no declarations found"
+    lib = mk.lib()
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(mk._abi.PROTOTYPES), declared ^ set(mk._abi.PROTOTYPES)
+
+
+def _host(shape, max_batch=4, max_ctx=320, sched=mk.MK_SCHED_STATIC, n_sm=16, **tiles):
+    return mk.DenseDecoder(shape, max_batch=max_batch, max_ctx=max_ctx, n_slots=max_batch, sched=sched,
+                           n_sm=n_sm, host_only=True, **tiles)
+
+
+def test_plan_build_and_tiles():
+    d = _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148)
+    t = d.tiles()
+    assert t["tile_qkv"] == 8 and t["tile_o"] == 8 and t["tile_gu"] == 4 and t["tile_down"] == 8
+    assert t["kseg"] == 2048 and t["tile_lm"] == 16 and t["chunk"] == 64 and t["n_sm"] == 148
+    fams = d.families()
+    assert len(fams) == 16 * 7 + 3
+    assert [f.name.decode() for f in fams[:7]] == ["qkv.0", "attn.0", "merge.0", "oproj.0", "gateup.0",
+                                                   "down.0", "dred.0"]
+    assert sum(f.followup for f in fams) == 16 * 2 + 2
+
+
+def test_plan_rejects_bad_shapes():
+    bad = wl.DenseShape(n_layers=1, hidden=320, n_q_heads=5, n_kv_heads=1, head_dim=64, ffn=1024, vocab=64)
+    with pytest.raises(mk.MkError) as e:
+        _host(bad)
+    assert e.value.status in (mk._abi.MK_ERR_UNSUPPORTED, mk._abi.MK_ERR_INVALID_ARG)
+    with pytest.raises(mk.MkError):
+        _host(wl.TINY, tile_qkv=6)
+    with pytest.raises(mk.MkError):
+        _host(wl.TINY, max_batch=9)
+
+
+def test_step_bytes_matches_hand_count():
+    d = _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148)
+    s = wl.LLAMA_1B
+    H, F, D = s.hidden, s.ffn, s.head_dim
+    per_layer = ((s.n_q_heads + 2 * s.n_kv_heads) * D * H + H * H + 3 * F * H + 2 * H) * 2
+    weights = s.n_layers * per_layer + s.vocab * H * 2 + H * 2
+    kv = 1024 * 16 * 8 * 64 * 2 * 2
+    want = weights + H * 2 + kv + 16 * 8 * 64 * 2 * 2 + 8
+    assert mk.mk_plan_step_bytes(d.plan, 1, [1024]) == pytest.approx(want, rel=1e-12)
+    assert abs(want / 1e9 - 2.505) < 0.01  # 2.505 GB per step at B=1, ctx 1024
+
+
+@pytest.mark.parametrize("B,ctx", [(1, [64]), (2, [0, 130]), (4, [5, 63, 64, 255])])
+def test_validate_bindings(B, ctx):
+    d = _host(wl.TINY)
+    mk.mk_plan_validate(d.plan, B, ctx)
+
+
+@pytest.mark.parametrize("sched", [mk.MK_SCHED_STATIC, mk.MK_SCHED_DYNAMIC])
+@pytest.mark.parametrize("B,ctx", [(1, [64]), (3, [0, 70, 190])])
+def test_simulator_clean(sched, B, ctx):
+    d = _host(wl.TINY, sched=sched, n_sm=8)
+    code, rep = mk.mk_plan_simulate(d.plan, B, ctx, n_orders=60, seed=7)
+    assert code == 0, rep.first_error
+    assert rep.races == 0 and rep.deadlocks == 0 and rep.exactly_once_violations == 0
+    assert rep.nonzero_counters == 0 and rep.static_dynamic_mismatch == 0
+    tiles = dict(tile_qkv=64, chunk=64, tile_o=64, tile_gu=32, tile_down=16, kseg=1024, tile_lm=128,
+                 lm_group=64)
+    assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, tiles))
+
+
+def test_simulator_many_orders():
+    d = _host(wl.TINY, n_sm=5)
+    code, rep = mk.mk_plan_simulate(d.plan, 2, [3, 128], n_orders=1000, seed=11)
+    assert code == 0 and rep.orders_run == 1000, rep.first_error
+
+
+def _family(d, name):
+    return [f.name.decode() for f in d.families()].index(name)
+
+
+def test_fault_dropped_notify_is_detected():
+    d = _host(wl.TINY, n_sm=4)
+    code, rep = mk.mk_plan_simulate(d.plan, 1, [64], 4, 1, mk.MK_SIM_FAULT_DROP_NOTIFY, _family(d, "gateup.1"))
+    assert code != 0 and rep.deadlocks == rep.orders_run
+
+
+def test_fault_wrong_wait_count_is_detected():
+    d = _host(wl.TINY, n_sm=4)
+    code, rep = mk.mk_plan_simulate(d.plan, 1, [64], 4, 1, mk.MK_SIM_FAULT_COUNT_PLUS_ONE, _family(d, "qkv.0"))
+    assert code != 0 and rep.deadlocks == rep.orders_run and rep.nonzero_counters == rep.orders_run
+
+
+@pytest.mark.parametrize("fam", ["oproj.0", "down.1", "attn.0", "lm"])
+def test_fault_missing_wait_is_a_race(fam):
+    d = _host(wl.TINY, n_sm=8)
+    code, rep = mk.mk_plan_simulate(d.plan, 2, [10, 100], 20, 3, mk.MK_SIM_FAULT_NO_WAIT, _family(d, fam))
+    assert code != 0 and rep.races > 0, rep.first_error
