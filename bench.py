@@ -61,7 +61,10 @@ class ClockSampler:
                  "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
-            time.sleep(0.3)
+            # start timing only once the sampler is producing samples
+            t0 = time.time()
+            while len(self.lines) < 2 and time.time() - t0 < 10:
+                time.sleep(0.05)
         except Exception:
             self.proc = None
         return self

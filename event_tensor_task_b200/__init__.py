@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes as C
 
 from . import _abi
-from ._abi import (MK_OK, MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS,
+from ._abi import (MK_OK, MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS, MK_DEBUG_TRACE,
                    MK_SIM_FAULT_NONE, MK_SIM_FAULT_DROP_NOTIFY, MK_SIM_FAULT_COUNT_PLUS_ONE,
                    MK_SIM_FAULT_NO_WAIT, OP_NAMES, mk_model_desc, mk_plan_opts, mk_step_args,
                    mk_layer_weights, mk_device_status, mk_family_info, mk_sim_report)
@@ -91,10 +91,9 @@ def mk_plan_family_info(plan: int, f: int) -> mk_family_info:
 
 
 def mk_plan_tiles(plan: int) -> dict:
-    out = (C.c_int * 10)()
+    out = (C.c_int * 9)()
     _check(lib().mk_plan_tiles(plan, out))
-    keys = ("tile_qkv", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm", "lm_group", "chunk",
-            "n_sm", "ring_slots")
+    keys = ("tile_qkv", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm", "chunk", "n_sm", "ring_slots")
     return dict(zip(keys, list(out)))
 
 
@@ -136,7 +135,7 @@ class DenseDecoder:
 
     def __init__(self, shape, weights=None, k_cache=None, v_cache=None, max_batch=1, max_ctx=None,
                  n_slots=None, sched=MK_SCHED_STATIC, n_sm=0, host_only=False, debug=False,
-                 spin_timeout_ns=0, **tiles):
+                 spin_timeout_ns=0, trace=False, **tiles):
         import torch
         self.shape = shape
         w = weights or {}
@@ -165,7 +164,7 @@ class DenseDecoder:
         o = mk_plan_opts()
         o.sched, o.n_sm, o.host_only = sched, n_sm, int(host_only)
         o.spin_timeout_ns = spin_timeout_ns
-        o.debug_flags = MK_DEBUG_TASK_COUNTS if debug else 0
+        o.debug_flags = (MK_DEBUG_TASK_COUNTS if debug else 0) | (MK_DEBUG_TRACE if trace else 0)
         for k, v in tiles.items():
             setattr(o, k, int(v))
         self.desc, self.opts = d, o
@@ -183,10 +182,13 @@ class DenseDecoder:
     def tiles(self):
         return mk_plan_tiles(self.plan)
 
-    def step(self, token_ids, slot_ids, ctx_lens, next_tokens, logits=None, task_counts=None, stream=None):
+    def step(self, token_ids, slot_ids, ctx_lens, next_tokens, logits=None, task_counts=None, stream=None,
+             trace=None):
         """One decode step on ``stream`` (default: torch's current stream)."""
         import torch
         a = mk_step_args()
+        if trace is not None:
+            a.trace, a.trace_cap = _ptr(trace), int(trace.shape[1])
         a.batch = int(token_ids.numel())
         a.token_ids, a.slot_ids, a.ctx_lens = _ptr(token_ids), _ptr(slot_ids), _ptr(ctx_lens)
         a.logits, a.next_tokens, a.task_counts = _ptr(logits), _ptr(next_tokens), _ptr(task_counts)

@@ -21,14 +21,15 @@ MK_SCHED_STATIC = 0
 MK_SCHED_DYNAMIC = 1
 MK_MODEL_DENSE = 0
 MK_DEBUG_TASK_COUNTS = 1
+MK_DEBUG_TRACE = 2
 
 MK_SIM_FAULT_NONE = 0
 MK_SIM_FAULT_DROP_NOTIFY = 1
 MK_SIM_FAULT_COUNT_PLUS_ONE = 2
 MK_SIM_FAULT_NO_WAIT = 3
 
-OP_NAMES = {1: "qkv", 2: "attn", 3: "merge", 4: "oproj", 5: "gateup", 6: "down", 7: "dred",
-            8: "lm", 9: "lmgrp", 10: "lmfin"}
+OP_NAMES = {1: "qkv", 2: "attn", 3: "merge", 4: "oproj", 5: "gateup", 6: "down",
+            8: "lm", 10: "lmfin"}
 
 
 class mk_layer_weights(C.Structure):
@@ -50,7 +51,7 @@ class mk_plan_opts(C.Structure):
     _fields_ = [
         ("sched", C.c_int), ("n_sm", C.c_int), ("host_only", C.c_int), ("smem_bytes", C.c_int),
         ("tile_qkv", C.c_int), ("tile_o", C.c_int), ("tile_gu", C.c_int), ("tile_down", C.c_int),
-        ("kseg", C.c_int), ("tile_lm", C.c_int), ("lm_group", C.c_int), ("attn_chunk", C.c_int),
+        ("kseg", C.c_int), ("tile_lm", C.c_int), ("attn_chunk", C.c_int),
         ("spin_timeout_ns", C.c_longlong), ("debug_flags", C.c_uint),
     ]
 
@@ -59,6 +60,7 @@ class mk_step_args(C.Structure):
     _fields_ = [
         ("batch", C.c_int), ("token_ids", C.c_void_p), ("slot_ids", C.c_void_p), ("ctx_lens", C.c_void_p),
         ("logits", C.c_void_p), ("next_tokens", C.c_void_p), ("task_counts", C.c_void_p),
+        ("trace", C.c_void_p), ("trace_cap", C.c_int),
     ]
 
 

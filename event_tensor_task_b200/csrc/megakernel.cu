@@ -7,24 +7,33 @@
 // switch — over tasks taken from a queue in device memory (static: this SM's
 // instruction list; dynamic: a shared queue that tasks are pushed onto when
 // their event fires).  Tasks synchronise only through Event Tensor counters:
-// notify() is an acquire-release atomic decrement, wait() spins until zero.
+// notify() is an atomic decrement with release semantics, wait() spins with
+// acquire loads until the counter is zero.
 //
-// Warp roles inside a CTA (320 threads):
-//   warp 0  producer   walks the task stream ahead of execution and streams
-//                      each task's weights (and cached KV rows) into a ring of
-//                      16 KB shared-memory slots with bulk async copies; it
-//                      never waits on events, so weight traffic runs ahead of
-//                      synchronisation (weights do not depend on activations).
-//   warp 1  controller waits on each task's event, hands the task to the
-//                      compute warps, and notifies its events afterwards; the
-//                      notifier whose decrement reaches zero runs the event's
-//                      follow-up task (merge / reduction) and, in dynamic mode,
-//                      pushes the event's consumer tasks.
-//   warps 2-9 compute  RMSNorm-fused GEMV tiles, split-KV attention, merges.
+// Warp roles inside a CTA (352 threads):
+//   warp 0     producer   walks the task stream ahead of execution and streams
+//                         each task's weights (and cached KV rows) into a ring
+//                         of 16 KB shared-memory slots with bulk async copies;
+//                         it never waits on events, so weight traffic runs
+//                         ahead of synchronisation.
+//   warp 1     controller takes tasks in order, waits on their events and
+//                         releases them to the compute warps through a
+//                         two-deep buffer (the next task is staged while the
+//                         current one runs).
+//   warp 2     notifier   publishes finished tasks: one gpu-scope release
+//                         fence per batch, then the counter decrements; the
+//                         decrement that takes a counter to zero queues the
+//                         event's follow-up task and, in dynamic mode, pushes
+//                         the consumer tasks.
+//   warps 3-10 compute    each warp works through whole weight rows of a task
+//                         (dot products reduced inside the warp, no block
+//                         barriers), or one attention head of a key chunk.
 // Every spin is bounded by the plan's timeout; on expiry the kernel records an
 // error in the control block, raises an abort flag that every spin polls,
 // drains its in-flight copies and exits.
 #include <cuda_runtime.h>
+
+#include <cstddef>
 
 #include "../../include/mk.h"
 #include "device.cuh"
@@ -34,14 +43,14 @@ namespace mk {
 
 constexpr int kComputeWarps = 8;
 constexpr int kComputeThreads = kComputeWarps * 32;
-constexpr int kThreads = kComputeThreads + 64;
-constexpr int kCtlThreads = kComputeThreads + 32;
+constexpr int kComputeBase = 96;  // producer, controller and notifier warps come first
+constexpr int kThreads = kComputeThreads + kComputeBase;
 constexpr int kFifo = 16;
 constexpr int kMaxSlots = 16;
-constexpr int kMaxFollow = 8;
-constexpr int kMaxB = 4;        // batch rows a GEMV task keeps in registers
-constexpr int kAccRows = 16;    // rows a compute thread accumulates per task
-constexpr int BAR_GO = 1, BAR_DONE = 2, BAR_COMP = 3;
+constexpr int kDoneQ = 32;    // controller -> notifier
+constexpr int kFollowQ = 16;  // notifier -> controller
+constexpr int kMaxB = 4;      // batch rows per step on this path
+constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
 constexpr int kDynLookahead = 2;
 
 struct StepParams {
@@ -52,32 +61,45 @@ struct StepParams {
   float* logits;
   int* next_tokens;
   unsigned* task_counts;
+  uint32_t* trace;
+  int trace_cap;
   unsigned epoch;
 };
 
 struct TaskDesc {
   int32_t fam, op, layer, idx;
-  int32_t ring_seq, nslots, pad0, pad1;
+  int32_t ring_seq, nslots;
+  int32_t rec;       // trace record of the task (0: none)
+  uint32_t t_issue;  // trace: when the producer queued the task (low 32 bits of ns)
 };
 
 struct Smem {
   uint64_t full[kMaxSlots], empty[kMaxSlots];
+  uint64_t go_bar[2];    // controller -> compute: task k is in cur[k & 1] (count 1)
+  uint64_t done_bar[2];  // compute -> controller: task k finished (one arrive per warp)
   uint64_t fifo_full[kFifo], fifo_empty[kFifo];
   TaskDesc fifo[kFifo];
-  TaskDesc cur;
-  TaskDesc follow[kMaxFollow];
+  TaskDesc cur[2];
+  TaskDesc doneq[kDoneQ];
+  TaskDesc followq[kFollowQ];
   int ctx[kMaxBatch], slot[kMaxBatch], tok[kMaxBatch], nch[kMaxBatch], pre[kMaxBatch + 1];
   int fam_ext[kMaxFamilies];
-  float red[kComputeWarps][kAccRows * kMaxB];
-  float fin[128 * kMaxB];
-  float qs[256];
-  float sc[4][64];
-  float hm[4], hl[4];
-  float newk[64], newv[64];
+  signed char fam_op[kMaxFamilies], fam_layer[kMaxFamilies];
+  // activation staging: one batch row, loaded once per CTA for all warps
+  alignas(16) float xs[2048];  // read and written as float4
+  float red8[kComputeWarps];
+  float yw[kComputeWarps][8];  // a warp's row results of the current task
+  uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
+  // attention scratch, one row per head warp
+  float qs[4][64], ps[4][64], newk[4][64], newv[4][64];
   volatile int released;  // regular tasks the controller has handed to compute
+  volatile int dq_head, dq_tail, fq_head, fq_tail, notifier_stop;
   int bad;
 };
-static_assert(sizeof(Smem) <= 14 * 1024, "fixed shared-memory area exceeds its reserve");
+static_assert(sizeof(Smem) <= 19 * 1024, "fixed shared-memory area exceeds its reserve");
+static_assert(offsetof(Smem, xs) % 16 == 0, "vector accesses to the staging buffer need 16-byte alignment");
+static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, fifo_full) % 8 == 0, "mbarriers need 8-byte alignment");
+constexpr int BAR_COMP = 3;  // named barrier of the 8 compute warps
 
 // ---------------------------------------------------------------- errors
 __device__ void record_error(Control* ctl, int code, int fam, int idx, int ev) {
@@ -108,6 +130,20 @@ __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, Control* ctl, long lon
   }
 }
 
+// ---------------------------------------------------------------- trace
+// MK_DEBUG_TRACE: per CTA, records of 16 uint32 (low 32 bits of the global
+// timer in ns); record 0 is the CTA's header.
+enum TraceField : int {
+  TR_FAM = 0, TR_IDX = 1, TR_POP = 2, TR_READY = 3, TR_GO = 4, TR_DONE = 5, TR_NOTIFIED = 6,
+  TR_CSTART = 7, TR_CEND = 8, TR_ISSUE = 9, TR_DATA = 10,
+  // header fields
+  TRH_RECORDS = 0, TRH_BATCHES = 1, TRH_NOTIFIED = 2, TRH_FENCE_NS = 3
+};
+__device__ __forceinline__ uint32_t* trace_rec(const StepParams& S, int rec) {
+  return (S.trace && rec >= 0 && rec < S.trace_cap) ? S.trace + ((size_t)blockIdx.x * S.trace_cap + rec) * 16
+                                                    : nullptr;
+}
+
 // ---------------------------------------------------------------- plan helpers
 __device__ __forceinline__ int ev_ctr(const DevPlan& P, int ev, int c0, int c1 = 0, int c2 = 0) {
   const EventTensorDesc& e = P.ev[ev];
@@ -119,9 +155,7 @@ __device__ __forceinline__ int ev_ctr(const DevPlan& P, int ev, int c0, int c1 =
 __device__ __forceinline__ int fam_of(const DevPlan& P, int op, int layer) {
   return op >= OP_LM ? P.fam_first_layer[op] : P.fam_first_layer[op] + layer * P.fam_stride;
 }
-__device__ __forceinline__ bool is_followup(int op) {
-  return op == OP_MERGE || op == OP_DRED || op == OP_LMGRP || op == OP_LMFIN;
-}
+__device__ __forceinline__ bool is_followup(int op) { return op == OP_MERGE || op == OP_LMFIN; }
 
 // Counter a regular task waits on (-1: none).
 __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t, int B) {
@@ -140,124 +174,165 @@ __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t,
 }
 
 // ---------------------------------------------------------------- producer
-struct Copy {
-  const unsigned char* src;
-  uint32_t dst_off;
-  uint32_t bytes;
+// Copy geometry of the tasks of one family, set up once per family so that a
+// slot costs the producer a handful of instructions (no divisions).
+struct ProdFam {
+  int fam, op, layer;
+  const unsigned char* w[3];  // q/k/v (QKV) or the parts' base matrices
+  uint32_t row_bytes;         // bytes of one row copy
+  uint32_t row_stride;        // bytes between consecutive rows in memory
+  int rps;                    // rows per ring slot
+  int slots_per_part;
+  int parts;
+  size_t task_stride;         // bytes between consecutive tasks' first rows
 };
 
-// Fills `cp` with the copies of slot j of a task; returns their count.
-__device__ int slot_copies(const DevPlan& P, const Smem& sm, const LayerPtrs* layers, int op, int layer, int idx,
-                           int j, int B, Copy* cp) {
-  const int H = P.hidden, D = P.head_dim;
-  const int rps = P.slot_bytes / (2 * H);
+__device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, int fam, int op, int layer, ProdFam& f) {
+  const uint32_t H2 = (uint32_t)P.hidden * 2;
+  f.fam = fam; f.op = op; f.layer = layer;
+  f.row_bytes = H2; f.row_stride = H2; f.rps = P.slot_bytes / (int)H2; f.parts = 1;
+  f.w[0] = f.w[1] = f.w[2] = nullptr;
+  f.task_stride = 0;
+  f.slots_per_part = 1;
   switch (op) {
     case OP_QKV: {
-      QkvTile q = decode_qkv(P, idx);
       const LayerPtrs& lp = layers[layer];
-      const unsigned char* w =
-          (const unsigned char*)(q.kind == 0 ? lp.wq : (q.kind == 1 ? lp.wk : lp.wv)) + (size_t)q.head * D * H * 2;
-      int half_slots = (P.tile_qkv / 2) / rps;
-      int part = j / half_slots, js = j % half_slots;
-      int row = q.j0 + part * (D / 2) + js * rps;
-      cp[0] = {w + (size_t)row * H * 2, 0, (uint32_t)(rps * H * 2)};
-      return 1;
-    }
-    case OP_OPROJ: {
-      const unsigned char* w = (const unsigned char*)layers[layer].wo;
-      int row = idx * P.tile_o + j * rps;
-      cp[0] = {w + (size_t)row * H * 2, 0, (uint32_t)(rps * H * 2)};
-      return 1;
-    }
-    case OP_GATEUP: {
-      int half_slots = P.tile_gu / rps;
-      int part = j / half_slots, js = j % half_slots;
-      const unsigned char* w = (const unsigned char*)(part == 0 ? layers[layer].w_gate : layers[layer].w_up);
-      int row = idx * P.tile_gu + js * rps;
-      cp[0] = {w + (size_t)row * H * 2, 0, (uint32_t)(rps * H * 2)};
-      return 1;
-    }
-    case OP_DOWN: {
-      int kc = idx / P.n_dtiles, n = idx % P.n_dtiles;
-      int rpsk = P.slot_bytes / (2 * P.kseg);
-      const unsigned char* w = (const unsigned char*)layers[layer].w_down;
-      for (int r = 0; r < rpsk; ++r) {
-        int row = n * P.tile_down + j * rpsk + r;
-        cp[r] = {w + ((size_t)row * P.ffn + (size_t)kc * P.kseg) * 2, (uint32_t)(r * P.kseg * 2),
-                 (uint32_t)(P.kseg * 2)};
-      }
-      return rpsk;
-    }
-    case OP_LM: {
-      int r0 = idx * P.tile_lm + j * rps;
-      int rows = min(rps, P.vocab - r0);
-      if (rows <= 0) return 0;
-      cp[0] = {(const unsigned char*)P.lm_head + (size_t)r0 * H * 2, 0, (uint32_t)(rows * H * 2)};
-      return 1;
-    }
-    case OP_ATTN: {
-      AttnTask a = decode_attn(idx, B, P.n_kv_heads, sm.nch, sm.pre);
-      int p = sm.ctx[a.b];
-      int n_old = min(P.chunk, p - a.c * P.chunk);
-      if (n_old <= 0) return 0;
-      size_t row0 = (((size_t)layer * P.n_slots + sm.slot[a.b]) * P.n_kv_heads + a.g) * P.max_ctx + (size_t)a.c * P.chunk;
-      cp[0] = {(const unsigned char*)P.k_cache + row0 * D * 2, 0, (uint32_t)(n_old * D * 2)};
-      cp[1] = {(const unsigned char*)P.v_cache + row0 * D * 2, (uint32_t)(P.chunk * D * 2), (uint32_t)(n_old * D * 2)};
-      return 2;
-    }
-    default: return 0;
+      f.w[0] = (const unsigned char*)lp.wq; f.w[1] = (const unsigned char*)lp.wk; f.w[2] = (const unsigned char*)lp.wv;
+      f.parts = 2; f.slots_per_part = (P.tile_qkv / 2) / f.rps;
+    } break;
+    case OP_OPROJ:
+      f.w[0] = (const unsigned char*)layers[layer].wo;
+      f.slots_per_part = P.tile_o / f.rps; f.task_stride = (size_t)P.tile_o * H2;
+      break;
+    case OP_GATEUP:
+      f.w[0] = (const unsigned char*)layers[layer].w_gate; f.w[1] = (const unsigned char*)layers[layer].w_up;
+      f.parts = 2; f.slots_per_part = P.tile_gu / f.rps; f.task_stride = (size_t)P.tile_gu * H2;
+      break;
+    case OP_DOWN:
+      f.w[0] = (const unsigned char*)layers[layer].w_down;
+      f.row_bytes = (uint32_t)P.kseg * 2; f.row_stride = (uint32_t)P.ffn * 2;
+      f.rps = P.slot_bytes / (int)f.row_bytes; f.slots_per_part = P.tile_down / f.rps;
+      break;
+    case OP_LM:
+      f.w[0] = (const unsigned char*)P.lm_head;
+      f.slots_per_part = ceil_div(P.tile_lm, f.rps); f.task_stride = (size_t)P.tile_lm * H2;
+      break;
+    default: break;  // ATTN: per task
   }
 }
 
-__device__ int task_slots(const DevPlan& P, int op, int idx) {
-  const int rps = P.slot_bytes / (2 * P.hidden);
-  switch (op) {
-    case OP_QKV: return P.tile_qkv / rps;
-    case OP_OPROJ: return P.tile_o / rps;
-    case OP_GATEUP: return 2 * P.tile_gu / rps;
-    case OP_DOWN: return P.tile_down / (P.slot_bytes / (2 * P.kseg));
-    case OP_LM: return ceil_div(min(P.tile_lm, P.vocab - idx * P.tile_lm), rps);
-    case OP_ATTN: return 1;
-    default: return 0;
-  }
+__device__ __forceinline__ int task_slots(const DevPlan& P, const ProdFam& f, int idx) {
+  if (f.op == OP_ATTN) return 1;
+  if (f.op == OP_LM) return ceil_div(min(P.tile_lm, P.vocab - idx * P.tile_lm), f.rps);
+  return f.parts * f.slots_per_part;
 }
 
 __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                          unsigned char* ws, Control* ctl) {
-  const FamilyDesc* fams = reinterpret_cast<const FamilyDesc*>(ws + P.off_families);
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const long long tmo = P.spin_timeout_ns;
   uint32_t ring_seq = 0, fifo_seq = 0;
+  int slot = 0;          // ring_seq % ring_slots
+  uint32_t phase = 0;    // (ring_seq / ring_slots) & 1
   int emitted = 0;
   int qr = 0;  // dynamic queue: range cursor of this CTA
   QRange* Q = reinterpret_cast<QRange*>(ws + P.off_queue);
   bool ok = true;
+  ProdFam f;
+  f.fam = -2;
+
+  // acquire the next ring slot: wait until the compute warps released it
+  auto next_slot = [&](int fam, int idx, unsigned char*& dst, uint64_t*& bar) -> bool {
+    if (!wait_mbar(&sm.empty[slot], phase ^ 1, ctl, tmo, fam, idx)) return false;
+    if (S.trace) sm.slot_t[slot] = (uint32_t)global_ns();
+    dst = ring + (size_t)slot * P.slot_bytes;
+    bar = &sm.full[slot];
+    ring_seq++;
+    if (++slot == P.ring_slots) { slot = 0; phase ^= 1; }
+    return true;
+  };
+  // rows [0, nrows) of a part starting at src into consecutive slots
+  auto stream_part = [&](int fam, int idx, const unsigned char* src, int nrows) -> bool {
+    while (nrows > 0) {
+      unsigned char* dst;
+      uint64_t* bar;
+      if (!next_slot(fam, idx, dst, bar)) return false;
+      int rows = min(nrows, f.rps);
+      mbar_arrive_expect_tx(bar, (uint32_t)rows * f.row_bytes);
+      if (f.row_stride == f.row_bytes) {
+        bulk_g2s(dst, src, (uint32_t)rows * f.row_bytes, bar);
+      } else {
+        for (int r = 0; r < rows; ++r) bulk_g2s(dst + r * f.row_bytes, src + (size_t)r * f.row_stride, f.row_bytes, bar);
+      }
+      src += (size_t)rows * f.row_stride;
+      nrows -= rows;
+    }
+    return true;
+  };
 
   auto emit = [&](int fam, int idx) -> bool {
+    int op = OP_END, layer = -1;
+    if (fam >= 0) {
+      op = sm.fam_op[fam];
+      layer = sm.fam_layer[fam];
+      if (fam != f.fam) prod_setup(P, layers, fam, op, layer, f);
+    }
     TaskDesc d;
-    d.fam = fam;
-    d.idx = idx;
-    d.op = fam >= 0 ? fams[fam].op : OP_END;
-    d.layer = fam >= 0 ? fams[fam].layer : -1;
-    d.nslots = fam >= 0 ? task_slots(P, d.op, idx) : 0;
+    d.fam = fam; d.idx = idx; d.op = op; d.layer = layer;
+    d.nslots = fam >= 0 ? task_slots(P, f, idx) : 0;
     d.ring_seq = (int)ring_seq;
-    d.pad0 = d.pad1 = 0;
+    d.rec = 0;
     int k = fifo_seq % kFifo;
     if (!wait_mbar(&sm.fifo_empty[k], ((fifo_seq / kFifo) & 1) ^ 1, ctl, tmo, fam, idx)) return false;
+    d.t_issue = S.trace ? (uint32_t)global_ns() : 0u;
     sm.fifo[k] = d;
     mbar_arrive(&sm.fifo_full[k]);
     fifo_seq++;
-    Copy cp[8];
-    for (int j = 0; j < d.nslots; ++j) {
-      int s = ring_seq % P.ring_slots;
-      if (!wait_mbar(&sm.empty[s], ((ring_seq / P.ring_slots) & 1) ^ 1, ctl, tmo, fam, idx)) return false;
-      int n = slot_copies(P, sm, layers, d.op, d.layer, idx, j, S.B, cp);
-      uint32_t bytes = 0;
-      for (int c = 0; c < n; ++c) bytes += cp[c].bytes;
-      mbar_arrive_expect_tx(&sm.full[s], bytes);
-      unsigned char* dst = ring + (size_t)s * P.slot_bytes;
-      for (int c = 0; c < n; ++c) bulk_g2s(dst + cp[c].dst_off, cp[c].src, cp[c].bytes, &sm.full[s]);
-      ring_seq++;
+    if (fam < 0) return true;
+    switch (op) {
+      case OP_QKV: {
+        QkvTile q = decode_qkv(P, idx);
+        const unsigned char* base = f.w[q.kind] + ((size_t)q.head * P.head_dim + q.j0) * f.row_stride;
+        const int half = P.tile_qkv / 2;
+        if (!stream_part(fam, idx, base, half)) return false;
+        if (!stream_part(fam, idx, base + (size_t)(P.head_dim / 2) * f.row_stride, half)) return false;
+      } break;
+      case OP_OPROJ:
+        if (!stream_part(fam, idx, f.w[0] + (size_t)idx * f.task_stride, P.tile_o)) return false;
+        break;
+      case OP_GATEUP:
+        if (!stream_part(fam, idx, f.w[0] + (size_t)idx * f.task_stride, P.tile_gu)) return false;
+        if (!stream_part(fam, idx, f.w[1] + (size_t)idx * f.task_stride, P.tile_gu)) return false;
+        break;
+      case OP_DOWN: {
+        int kc = idx / P.n_dtiles, n = idx - kc * P.n_dtiles;
+        const unsigned char* base = f.w[0] + (size_t)n * P.tile_down * f.row_stride + (size_t)kc * f.row_bytes;
+        if (!stream_part(fam, idx, base, P.tile_down)) return false;
+      } break;
+      case OP_LM:
+        if (!stream_part(fam, idx, f.w[0] + (size_t)idx * f.task_stride, min(P.tile_lm, P.vocab - idx * P.tile_lm)))
+          return false;
+        break;
+      case OP_ATTN: {
+        // the chunk's cached (already rotated) keys and values, minus the row
+        // this step appends; K rows at the slot start, V rows half a slot in
+        AttnTask a = decode_attn(idx, S.B, P.n_kv_heads, sm.nch, sm.pre);
+        int p = sm.ctx[a.b];
+        int n_old = max(0, min(P.chunk, p - a.c * P.chunk));
+        unsigned char* dst;
+        uint64_t* bar;
+        if (!next_slot(fam, idx, dst, bar)) return false;
+        uint32_t bytes = (uint32_t)n_old * P.head_dim * 2;
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        if (n_old > 0) {
+          size_t row0 = (((size_t)layer * P.n_slots + sm.slot[a.b]) * P.n_kv_heads + a.g) * P.max_ctx +
+                        (size_t)a.c * P.chunk;
+          bulk_g2s(dst, (const unsigned char*)P.k_cache + row0 * P.head_dim * 2, bytes, bar);
+          bulk_g2s(dst + (size_t)P.chunk * P.head_dim * 2, (const unsigned char*)P.v_cache + row0 * P.head_dim * 2,
+                   bytes, bar);
+        }
+      } break;
+      default: break;
     }
     emitted++;
     return true;
@@ -268,8 +343,9 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     for (int k = 0; k < P.n_instr_per_sm && ok; ++k) {
       Instr in = ins[k];
       if (in.family < 0) break;
-      int ext = sm.fam_ext[in.family];
-      for (int i = in.start; i < ext && ok; i += in.stride) ok = emit(in.family, i);
+      int lo, hi;
+      instr_range(in, sm.fam_ext[in.family], lo, hi);
+      for (int i = lo; i < hi && ok; ++i) ok = emit(in.family, i);
     }
   } else {
     for (;;) {
@@ -322,11 +398,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
   }
 }
 
-// ---------------------------------------------------------------- controller
-struct CtlState {
-  int nf;
-};
-
+// ---------------------------------------------------------------- notifier
 __device__ void push_range(const DevPlan& P, const StepParams& S, Control* ctl, unsigned char* ws, int fam,
                            int lo, int count) {
   if (count <= 0) return;
@@ -341,427 +413,779 @@ __device__ void push_range(const DevPlan& P, const StepParams& S, Control* ctl, 
   st_release_u32(&Q[r].seq, S.epoch);
 }
 
-// notify() of a finished task: decrement its counter; the notifier whose
-// decrement reaches zero queues the follow-up and (dynamic) pushes consumers.
-// Runs on lane 0 of the controller warp; returns the number of follow-ups.
-__device__ int notify_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, Control* ctl,
-                           int* counters, const TaskDesc& t, int nf) {
-  const int B = S.B, Hkv = P.n_kv_heads;
+// What notify() of a finished task does: the counter it decrements, whether
+// the decrement's result is needed (a follow-up or a dynamic push hangs on
+// it), and the follow-up it triggers when the counter reaches zero.
+struct NotifyInfo {
+  int ctr, ffam, fop, flayer, fidx, need_old;
+};
+
+__device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const Smem& sm, const TaskDesc& t) {
+  const int Hkv = P.n_kv_heads;
   const bool dyn = P.sched == MK_SCHED_DYNAMIC;
-  int ctr = -1, ffam = -1, fidx = 0;
-  int ag = 0, akc = 0;
+  NotifyInfo n;
+  n.ctr = -1; n.ffam = -1; n.fop = 0; n.flayer = -1; n.fidx = 0; n.need_old = 0;
   switch (t.op) {
-    case OP_QKV: ag = decode_qkv(P, t.idx).group; ctr = ev_ctr(P, EV_QKV, t.layer, ag); break;
+    case OP_QKV: n.ctr = ev_ctr(P, EV_QKV, t.layer, decode_qkv(P, t.idx).group); break;
     case OP_ATTN: {
-      AttnTask a = decode_attn(t.idx, B, Hkv, sm.nch, sm.pre);
-      ctr = ev_ctr(P, EV_CHUNK, t.layer, a.b, a.g);
-      ffam = fam_of(P, OP_MERGE, t.layer);
-      fidx = a.b * Hkv + a.g;
+      AttnTask a = decode_attn(t.idx, S.B, Hkv, sm.nch, sm.pre);
+      n.ctr = ev_ctr(P, EV_CHUNK, t.layer, a.b, a.g);
+      n.ffam = fam_of(P, OP_MERGE, t.layer); n.fop = OP_MERGE; n.flayer = t.layer; n.fidx = a.b * Hkv + a.g;
     } break;
-    case OP_MERGE: ctr = ev_ctr(P, EV_ATTN, t.layer); break;
-    case OP_OPROJ: ctr = ev_ctr(P, EV_O, t.layer); break;
-    case OP_GATEUP: akc = t.idx * P.tile_gu / P.kseg; ctr = ev_ctr(P, EV_GU, t.layer, akc); break;
-    case OP_DOWN: {
-      int n = t.idx % P.n_dtiles;
-      ctr = ev_ctr(P, EV_DSUM, t.layer, n);
-      ffam = fam_of(P, OP_DRED, t.layer);
-      fidx = n;
-    } break;
-    case OP_DRED: ctr = ev_ctr(P, EV_IN, t.layer + 1); break;
-    case OP_LM: {
-      int grp = t.idx / P.lm_group;
-      ctr = ev_ctr(P, EV_LMG, grp);
-      ffam = fam_of(P, OP_LMGRP, -1);
-      fidx = grp;
-    } break;
-    case OP_LMGRP: ctr = ev_ctr(P, EV_LM, 0); ffam = fam_of(P, OP_LMFIN, -1); fidx = 0; break;
-    case OP_LMFIN:
-      if (dyn) push_range(P, S, ctl, ws, -1, 0, P.n_sm);  // one END per CTA
-      return nf;
-    default: return nf;
+    case OP_MERGE: n.ctr = ev_ctr(P, EV_ATTN, t.layer); break;
+    case OP_OPROJ: n.ctr = ev_ctr(P, EV_O, t.layer); break;
+    case OP_GATEUP: n.ctr = ev_ctr(P, EV_GU, t.layer, t.idx * P.tile_gu / P.kseg); break;
+    case OP_DOWN: n.ctr = ev_ctr(P, EV_IN, t.layer + 1); break;
+    case OP_LM:
+      n.ctr = ev_ctr(P, EV_LM, 0);
+      n.ffam = fam_of(P, OP_LMFIN, -1); n.fop = OP_LMFIN; n.fidx = 0;
+      break;
+    default: break;
   }
-  __threadfence();
-  int old = atom_add_acq_rel(&counters[ctr], -1);
-  if (old <= 0) { record_error(ctl, MK_ERR_DEVICE_BOUNDS, t.fam, t.idx, ctr); return nf; }
-  if (old != 1) return nf;
-  // the event fired
-  if (ffam >= 0 && nf < kMaxFollow) {
-    TaskDesc f;
-    f.fam = ffam; f.op = (t.op == OP_ATTN) ? OP_MERGE : (t.op == OP_DOWN) ? OP_DRED : (t.op == OP_LM) ? OP_LMGRP : OP_LMFIN;
-    f.layer = (f.op == OP_LMGRP || f.op == OP_LMFIN) ? -1 : t.layer;
-    f.idx = fidx; f.ring_seq = 0; f.nslots = 0; f.pad0 = f.pad1 = 0;
-    sm.follow[nf++] = f;
-  }
-  if (dyn) {
-    switch (t.op) {
-      case OP_QKV:
-        for (int b = 0; b < B; ++b)
-          push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b] + ag * sm.nch[b], sm.nch[b]);
-        break;
-      case OP_MERGE: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
-      case OP_OPROJ: push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles); break;
-      case OP_GATEUP: push_range(P, S, ctl, ws, fam_of(P, OP_DOWN, t.layer), akc * P.n_dtiles, P.n_dtiles); break;
-      case OP_DRED:
-        if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
-        else push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
-        break;
-      default: break;
-    }
-  }
-  return nf;
+  n.need_old = (n.ctr >= 0 && (n.ffam >= 0 || dyn)) ? 1 : 0;
+  return n;
 }
 
+// Dynamic mode: the notifier whose decrement took a counter to zero pushes
+// the tasks that wait on it.
+__device__ void push_successors(const DevPlan& P, const StepParams& S, const Smem& sm, Control* ctl,
+                                unsigned char* ws, const TaskDesc& t) {
+  const int Hkv = P.n_kv_heads;
+  switch (t.op) {
+    case OP_QKV: {
+      int g = decode_qkv(P, t.idx).group;
+      for (int b = 0; b < S.B; ++b)
+        push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b] + g * sm.nch[b], sm.nch[b]);
+    } break;
+    case OP_MERGE: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
+    case OP_OPROJ: push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles); break;
+    case OP_GATEUP: {
+      int kc = t.idx * P.tile_gu / P.kseg;
+      push_range(P, S, ctl, ws, fam_of(P, OP_DOWN, t.layer), kc * P.n_dtiles, P.n_dtiles);
+    } break;
+    case OP_DOWN:
+      if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
+      else push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
+      break;
+    default: break;
+  }
+}
+
+// Notifier warp: drains up to kFollowQ entries of the done queue at a time,
+// orders all their outputs with ONE gpu-scope release fence, then decrements
+// the counters (one lane per task; result-free decrements of the same counter
+// are combined into one add).
+__device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, Control* ctl,
+                         int* counters) {
+  const int lane = threadIdx.x & 31;
+  const bool trace = S.trace != nullptr;
+  int tail = 0;
+  unsigned long long n_batches = 0, fence_ns = 0;
+  for (;;) {
+    int head = sm.dq_head;
+    if (head == tail) {
+      if (sm.notifier_stop || aborted(ctl)) break;
+      __nanosleep(20);
+      continue;
+    }
+    __threadfence_block();
+    const int n = min(head - tail, kFollowQ);  // at most kFollowQ follow-ups per batch
+    TaskDesc t;
+    NotifyInfo ni;
+    ni.ctr = -1; ni.need_old = 0; ni.ffam = -1;
+    if (lane < n) {
+      t = sm.doneq[(tail + lane) % kDoneQ];
+      ni = notify_info(P, S, sm, t);
+    }
+    __syncwarp();
+    unsigned long long tf0 = trace ? global_ns() : 0;
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    if (trace) { fence_ns += global_ns() - tf0; n_batches++; }
+    int old = 0;
+    if (lane < n && ni.ctr >= 0 && ni.need_old) {
+      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], -1;" : "=r"(old) : "l"(counters + ni.ctr) : "memory");
+    }
+    int key = (lane < n && ni.ctr >= 0 && !ni.need_old) ? ni.ctr : -1 - lane;
+    unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(peers) - 1) {
+      int cnt = __popc(peers);
+      asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(counters + key), "r"(-cnt) : "memory");
+    }
+    if (lane < n && ni.need_old && old <= 0) record_error(ctl, MK_ERR_DEVICE_BOUNDS, t.fam, t.idx, ni.ctr);
+    const bool fired = lane < n && ni.need_old && old == 1;
+    if (fired && P.sched == MK_SCHED_DYNAMIC) push_successors(P, S, sm, ctl, ws, t);
+    if (lane < n && t.op == OP_LMFIN && P.sched == MK_SCHED_DYNAMIC)
+      push_range(P, S, ctl, ws, -1, 0, P.n_sm);  // one END per CTA
+    unsigned fb = __ballot_sync(0xffffffffu, fired && ni.ffam >= 0);
+    if (fb) {
+      int fh = sm.fq_head;
+      int rank = __popc(fb & ((1u << lane) - 1));
+      int room_ok = 1;
+      if (lane == 0) {
+        unsigned long long t0 = global_ns();
+        while (fh + __popc(fb) - sm.fq_tail > kFollowQ) {
+          if (aborted(ctl) || (long long)(global_ns() - t0) > P.spin_timeout_ns) { room_ok = 0; break; }
+        }
+        if (!room_ok) record_error(ctl, MK_ERR_DEVICE_TIMEOUT, -1, -1, -1);
+      }
+      room_ok = __shfl_sync(0xffffffffu, room_ok, 0);
+      if (room_ok && fired && ni.ffam >= 0) {
+        TaskDesc f;
+        f.fam = ni.ffam; f.op = ni.fop; f.layer = ni.flayer; f.idx = ni.fidx;
+        f.ring_seq = 0; f.nslots = 0; f.rec = 0; f.t_issue = 0;
+        sm.followq[(fh + rank) % kFollowQ] = f;
+      }
+      __syncwarp();
+      __threadfence_block();
+      if (lane == 0 && room_ok) sm.fq_head = fh + __popc(fb);
+    }
+    if (trace && lane < n && t.rec > 0) {
+      uint32_t* r = trace_rec(S, t.rec);
+      if (r) r[TR_NOTIFIED] = (uint32_t)global_ns();
+    }
+    __syncwarp();
+    __threadfence_block();
+    tail += n;
+    if (lane == 0) sm.dq_tail = tail;
+  }
+  if (trace && lane == 0) {
+    uint32_t* h = trace_rec(S, 0);
+    h[TRH_BATCHES] = (uint32_t)n_batches;
+    h[TRH_NOTIFIED] = (uint32_t)tail;
+    h[TRH_FENCE_NS] = (uint32_t)fence_ns;
+  }
+}
+
+// ---------------------------------------------------------------- controller
+// Releases tasks to the compute warps in order, at most two at a time: task k
+// goes to cur[k & 1] and completes phase k >> 1 of go_bar[k & 1]; the warps
+// report it done on done_bar[k & 1].  Per-buffer barriers keep every barrier
+// at most one phase ahead of any warp.
 __device__ void controller(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, Control* ctl,
                            int* counters) {
   const int lane = threadIdx.x & 31;
   const long long tmo = P.spin_timeout_ns;
   const FamilyDesc* fams = reinterpret_cast<const FamilyDesc*>(ws + P.off_families);
-  uint32_t fifo_seq = 0;
-  TaskDesc p, held, t;
-  bool have_p = false, have_held = false;
-  int nf = 0;
+  uint32_t fifo_seq = 0, nrel = 0, ndone = 0;
+  TaskDesc held, t;
+  TaskDesc inflight[2];
+  inflight[0].fam = inflight[1].fam = -1;
+  inflight[0].idx = inflight[1].idx = -1;
+  inflight[0].rec = inflight[1].rec = 0;
+  bool have_held = false;
   int known = -1;
   int released = 0;
+  int dq_head = 0, fq_tail = 0;
   bool dead = false;
-
-  auto finish_p = [&]() {
-    bar_sync(BAR_DONE, kCtlThreads);
-    int r = 0;
-    if (lane == 0) r = notify_task(P, S, sm, ws, ctl, counters, p, nf);
-    nf = __shfl_sync(0xffffffffu, r, 0);
+  const bool trace = S.trace != nullptr;
+  int nrec = 0;
+  uint32_t t_pop = 0, t_ready = 0;
+  auto stamp = [&](int rec, int field, uint32_t v) {
+    if (trace && lane == 0 && rec > 0) {
+      uint32_t* r = trace_rec(S, rec);
+      if (r) r[field] = v;
+    }
+  };
+  // hand a finished task to the notifier (lane 0; the caller broadcasts)
+  auto enqueue = [&](const TaskDesc& e) -> bool {
+    unsigned long long t0 = global_ns();
+    while (dq_head - sm.dq_tail >= kDoneQ) {
+      if (aborted(ctl) || (long long)(global_ns() - t0) > tmo) return false;
+    }
+    sm.doneq[dq_head % kDoneQ] = e;
+    __threadfence_block();
+    sm.dq_head = dq_head + 1;
+    return true;
+  };
+  // completion of the oldest in-flight task: block (wait) or test only
+  auto complete_oldest = [&](bool block) -> int {  // 1 completed, 0 not yet, -1 dead
+    int st = 0;
+    if (lane == 0) {
+      uint64_t* bar = &sm.done_bar[ndone & 1];
+      const uint32_t par = (ndone >> 1) & 1;
+      bool ok = block ? wait_mbar(bar, par, ctl, tmo, inflight[ndone & 1].fam, inflight[ndone & 1].idx)
+                      : mbar_test(bar, par);
+      if (ok) {
+        const TaskDesc& e = inflight[ndone & 1];
+        if (trace && e.rec > 0) { uint32_t* r = trace_rec(S, e.rec); if (r) r[TR_DONE] = (uint32_t)global_ns(); }
+        st = enqueue(e) ? 1 : -1;
+      } else {
+        st = block ? -1 : 0;
+      }
+    }
+    st = __shfl_sync(0xffffffffu, st, 0);
+    if (st == 1) { ndone++; dq_head++; }
+    return st;
+  };
+  // spin helper: notify finished tasks as they complete; report follow-ups
+  auto idle_poll = [&]() -> int {  // 2 follow-up pending, -1 dead, 0 otherwise
+    if (nrel != ndone && complete_oldest(false) < 0) return -1;
+    return sm.fq_head != fq_tail ? 2 : 0;
+  };
+  auto release = [&](TaskDesc& r) {
+    r.rec = (trace && r.op != OP_END) ? ++nrec : 0;
+    inflight[nrel & 1] = r;
+    if (lane == 0) {
+      sm.cur[nrel & 1] = r;
+      if (r.op != OP_END && S.task_counts && (P.debug_flags & MK_DEBUG_TASK_COUNTS))
+        atomicAdd(&S.task_counts[fams[r.fam].debug_base + r.idx], 1u);
+      if (r.op != OP_END && !is_followup(r.op)) sm.released = ++released;
+      mbar_arrive(&sm.go_bar[nrel & 1]);
+    }
     __syncwarp();
-    have_p = false;
+    nrel++;
+    if (r.rec > 0) {
+      stamp(r.rec, TR_FAM, (uint32_t)r.fam);
+      stamp(r.rec, TR_IDX, (uint32_t)r.idx);
+      stamp(r.rec, TR_POP, t_pop);
+      stamp(r.rec, TR_READY, t_ready);
+      stamp(r.rec, TR_GO, (uint32_t)global_ns());
+    }
   };
 
   for (;;) {
-    if (nf > 0) {
-      t = sm.follow[nf - 1];
-      nf--;
+    if (aborted(ctl)) { dead = true; break; }
+    if (sm.fq_head != fq_tail) {
+      __threadfence_block();
+      t = sm.followq[fq_tail % kFollowQ];
+      __syncwarp();
+      fq_tail++;
+      if (lane == 0) sm.fq_tail = fq_tail;
     } else if (have_held) {
       t = held;
       have_held = false;
     } else {
       int k = fifo_seq % kFifo;
-      if (have_p) {
-        // never block on the FIFO while holding an un-notified task: its
-        // notify may be what the producer's next task (or pop) waits for
+      const uint32_t par = (fifo_seq / kFifo) & 1;
+      int st = 0;  // 1 ready, 2 follow-up, 3 dead
+      unsigned long long t0 = global_ns();
+      for (int it = 0;; ++it) {
         int ready = 0;
-        if (lane == 0) ready = mbar_test(&sm.fifo_full[k], (fifo_seq / kFifo) & 1);
+        if (lane == 0) ready = mbar_test(&sm.fifo_full[k], par);
         ready = __shfl_sync(0xffffffffu, ready, 0);
-        if (!ready) {
-          finish_p();
-          if (nf > 0) continue;
+        if (ready) { st = 1; break; }
+        int ip = idle_poll();
+        if (ip < 0) { st = 3; break; }
+        if (ip == 2) { st = 2; break; }
+        if ((it & 15) == 15) {
+          int bad = 0;
+          if (lane == 0) {
+            if (aborted(ctl)) bad = 1;
+            else if ((long long)(global_ns() - t0) > tmo) { record_error(ctl, MK_ERR_DEVICE_TIMEOUT, -1, -1, -1); bad = 1; }
+          }
+          if (__shfl_sync(0xffffffffu, bad, 0)) { st = 3; break; }
         }
       }
-      int okw = 1;
-      if (lane == 0) okw = wait_mbar(&sm.fifo_full[k], (fifo_seq / kFifo) & 1, ctl, tmo, -1, -1);
-      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (st == 3) { dead = true; break; }
+      if (st == 2) continue;
       __syncwarp();
-      if (!okw) { dead = true; break; }
       t = sm.fifo[k];
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.fifo_empty[k]);
       fifo_seq++;
     }
+    if (trace) t_pop = (uint32_t)global_ns();
     if (t.op == OP_END) {
-      if (have_p) {
-        finish_p();
-        if (nf > 0) { held = t; have_held = true; continue; }
+      // quiesce: every task finished and notified, no follow-up left
+      while (nrel != ndone) {
+        if (complete_oldest(true) < 0) { dead = true; break; }
       }
-    } else if (!is_followup(t.op)) {
+      if (dead) break;
+      int st = 0;  // 1 quiet, 2 follow-up, 3 dead
+      if (lane == 0) {
+        unsigned long long t0 = global_ns();
+        for (;;) {
+          if (sm.fq_head != fq_tail) { st = 2; break; }
+          if (sm.dq_tail == dq_head) {
+            __threadfence_block();
+            st = sm.fq_head != fq_tail ? 2 : 1;
+            break;
+          }
+          if (aborted(ctl)) { st = 3; break; }
+          if ((long long)(global_ns() - t0) > tmo) { record_error(ctl, MK_ERR_DEVICE_TIMEOUT, -1, -1, -1); st = 3; break; }
+        }
+      }
+      st = __shfl_sync(0xffffffffu, st, 0);
+      if (st == 3) { dead = true; break; }
+      if (st == 2) { held = t; have_held = true; continue; }
+      release(t);
+      break;
+    }
+    if (!is_followup(t.op)) {
       int w = wait_counter(P, sm, t, S.B);
       if (w >= 0 && w != known) {
-        int zero = 0;
-        if (lane == 0) zero = ld_acquire(&counters[w]) == 0;
-        zero = __shfl_sync(0xffffffffu, zero, 0);
-        if (!zero && have_p) {
-          // never spin while holding an un-notified task
-          finish_p();
-          if (nf > 0) { held = t; have_held = true; continue; }
-        }
-        if (!zero) {
-          int okw = 1;
-          if (lane == 0) {
-            unsigned long long t0 = global_ns();
-            for (int it = 0;; ++it) {
-              if (ld_acquire(&counters[w]) == 0) break;
-              if ((it & 15) == 15) {
-                if (aborted(ctl)) { okw = 0; break; }
-                if ((long long)(global_ns() - t0) > tmo) {
-                  record_error(ctl, MK_ERR_DEVICE_TIMEOUT, t.fam, t.idx, w);
-                  okw = 0;
-                  break;
-                }
-              }
+        int st = 0;  // 1 fired, 2 follow-up, 3 dead
+        unsigned long long t0 = global_ns();
+        for (int it = 0;; ++it) {
+          int zero = 0;
+          if (lane == 0) zero = ld_acquire(&counters[w]) == 0;
+          if (__shfl_sync(0xffffffffu, zero, 0)) { st = 1; break; }
+          // never sit on finished tasks while waiting: their notify may be
+          // what this event needs
+          int ip = idle_poll();
+          if (ip < 0) { st = 3; break; }
+          if (ip == 2) { st = 2; break; }
+          if ((it & 15) == 15) {
+            int bad = 0;
+            if (lane == 0) {
+              if (aborted(ctl)) bad = 1;
+              else if ((long long)(global_ns() - t0) > tmo) { record_error(ctl, MK_ERR_DEVICE_TIMEOUT, t.fam, t.idx, w); bad = 1; }
             }
+            if (__shfl_sync(0xffffffffu, bad, 0)) { st = 3; break; }
           }
-          okw = __shfl_sync(0xffffffffu, okw, 0);
-          if (!okw) { dead = true; break; }
         }
+        if (st == 3) { dead = true; break; }
+        if (st == 2) { held = t; have_held = true; continue; }
         known = w;
       }
     }
-    if (have_p) bar_sync(BAR_DONE, kCtlThreads);
-    if (lane == 0) {
-      sm.cur = t;
-      if (t.op != OP_END && S.task_counts && (P.debug_flags & MK_DEBUG_TASK_COUNTS))
-        atomicAdd(&S.task_counts[fams[t.fam].debug_base + t.idx], 1u);
-      if (t.op != OP_END && !is_followup(t.op)) sm.released = ++released;
-    }
-    __syncwarp();
-    bar_sync(BAR_GO, kCtlThreads);
-    if (have_p) {
-      int r = 0;
-      if (lane == 0) r = notify_task(P, S, sm, ws, ctl, counters, p, nf);
-      nf = __shfl_sync(0xffffffffu, r, 0);
-      __syncwarp();
-    }
-    if (t.op == OP_END) break;
-    p = t;
-    have_p = true;
+    if (trace) t_ready = (uint32_t)global_ns();
+    // at most two tasks in flight
+    if (nrel - ndone == 2 && complete_oldest(true) < 0) { dead = true; break; }
+    release(t);
   }
+  if (trace && lane == 0) trace_rec(S, 0)[TRH_RECORDS] = (uint32_t)nrec;
   if (dead) {
-    // shut the compute warps down: finish the task they hold, then send END
-    if (have_p) bar_sync(BAR_DONE, kCtlThreads);
+    // shut the compute warps down: let them finish what they hold, then END
+    while (nrel != ndone) {
+      int st = 0;
+      if (lane == 0) st = wait_mbar(&sm.done_bar[ndone & 1], (ndone >> 1) & 1, ctl, tmo, -1, -1) ? 1 : 0;
+      st = __shfl_sync(0xffffffffu, st, 0);
+      ndone++;
+      if (!st) break;
+    }
+    TaskDesc e;
+    e.fam = -1; e.op = OP_END; e.layer = -1; e.idx = 0; e.ring_seq = 0; e.nslots = 0; e.rec = 0; e.t_issue = 0;
     if (lane == 0) {
-      TaskDesc e;
-      e.fam = -1; e.op = OP_END; e.layer = -1; e.idx = 0; e.ring_seq = 0; e.nslots = 0; e.pad0 = e.pad1 = 0;
-      sm.cur = e;
+      sm.cur[nrel & 1] = e;
       sm.released = 1 << 30;
+      mbar_arrive(&sm.go_bar[nrel & 1]);
     }
     __syncwarp();
-    bar_sync(BAR_GO, kCtlThreads);
   }
+  if (lane == 0) sm.notifier_stop = 1;
 }
 
 // ---------------------------------------------------------------- compute
-struct Act {
-  int tag;
-  float v[kMaxB][8];
+struct GemvSpec {
+  int kind;           // 0: RMSNorm(x) * gamma, 1: attention output, 2: SwiGLU segment
+  const void* gamma;  // RMSNorm gain (kind 0)
+  int kc;             // K segment (kind 2)
+  int K;              // columns
+  bool parts;         // kind 0: add the previous layer's down-projection partials to x
+  int tag;            // identifies the activation; unchanged tag = reuse the registers
+  int rows;           // valid rows of the task
 };
 
-// Loads the activation columns this thread owns (8 per row, block cb) for the
-// B rows; kind 0: RMSNorm(x) * gamma, 1: attention output, 2: SwiGLU segment.
-__device__ void load_act(const DevPlan& P, Smem& sm, unsigned char* ws, int B, int kind, const void* gamma,
-                         int kc, int K, Act& a) {
-  const int ct = threadIdx.x - 64, cw = ct >> 5, lane = ct & 31;
-  const int kb = K / 8, cb = ct % kb;
-  const float* src;
-  size_t rstride;
-  if (kind == 0) { src = reinterpret_cast<const float*>(ws + P.off_x); rstride = P.hidden; }
-  else if (kind == 1) { src = reinterpret_cast<const float*>(ws + P.off_attn); rstride = (size_t)P.n_q_heads * P.head_dim; }
-  else { src = reinterpret_cast<const float*>(ws + P.off_h) + (size_t)kc * P.kseg; rstride = P.ffn; }
-#pragma unroll
-  for (int b = 0; b < kMaxB; ++b) {
-    if (b < B) {
-      const float4* p4 = reinterpret_cast<const float4*>(src + b * rstride + cb * 8);
-      float4 u = __ldcg(p4), w = __ldcg(p4 + 1);
-      a.v[b][0] = u.x; a.v[b][1] = u.y; a.v[b][2] = u.z; a.v[b][3] = u.w;
-      a.v[b][4] = w.x; a.v[b][5] = w.y; a.v[b][6] = w.z; a.v[b][7] = w.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) a.v[b][j] = 0.f;
-    }
+__device__ __forceinline__ bool gemv_spec(const DevPlan& P, const LayerPtrs* layers, const TaskDesc& d, GemvSpec& g) {
+  g.gamma = nullptr; g.kc = 0; g.parts = false; g.K = P.hidden;
+  switch (d.op) {
+    case OP_QKV:
+      g.kind = 0; g.gamma = layers[d.layer].attn_norm; g.parts = d.layer > 0; g.tag = d.layer * 64; g.rows = P.tile_qkv;
+      return true;
+    case OP_OPROJ:
+      g.kind = 1; g.tag = d.layer * 64 + 1; g.rows = P.tile_o;
+      return true;
+    case OP_GATEUP:
+      g.kind = 0; g.gamma = layers[d.layer].ffn_norm; g.tag = d.layer * 64 + 2; g.rows = 2 * P.tile_gu;
+      return true;
+    case OP_DOWN:
+      g.kind = 2; g.kc = d.idx / P.n_dtiles; g.K = P.kseg; g.tag = d.layer * 64 + 8 + g.kc; g.rows = P.tile_down;
+      return true;
+    case OP_LM:
+      g.kind = 0; g.gamma = P.final_norm; g.parts = true; g.tag = 60 * 64;
+      g.rows = min(P.tile_lm, P.vocab - d.idx * P.tile_lm);
+      return true;
+    default:
+      return false;
   }
-  if (kind != 0) return;
-  // RMSNorm: sum of squares over the K columns of each row
-  const int wpg = kb / 32;  // warps per row group
-#pragma unroll
-  for (int b = 0; b < kMaxB; ++b) {
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) ss = fmaf(a.v[b][j], a.v[b][j], ss);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) sm.red[cw][b] = ss;
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  const int g0 = (cw / wpg) * wpg;
-  uint4 gw = __ldg(reinterpret_cast<const uint4*>(gamma) + cb);
-  float gf[8];
-  bf16x8_to_f32(gw, gf);
-#pragma unroll
-  for (int b = 0; b < kMaxB; ++b) {
-    float ss = 0.f;
-    for (int w = 0; w < wpg; ++w) ss += sm.red[g0 + w][b];
-    float inv = 1.0f / sqrtf(ss / (float)K + P.eps);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) a.v[b][j] = a.v[b][j] * inv * gf[j];
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
 }
 
-// GEMV over a task's ring slots: rows of K bf16 weights, 4 rows per thread per
-// slot; leaves sm.fin[row * kMaxB + b] = sum_k W[row][k] * act[b][k].
-__device__ bool gemv_rows(const DevPlan& P, Smem& sm, unsigned char* ring, Control* ctl, const TaskDesc& d, int K,
-                          int valid_rows, int B, const Act& a) {
-  const int ct = threadIdx.x - 64, cw = ct >> 5, lane = ct & 31;
-  const int kb = K / 8, G = kComputeThreads / kb, cb = ct % kb, rg = ct / kb;
-  const int rps = 4 * G;  // rows per 16 KB slot
-  float acc[kAccRows][kMaxB];
+
+__device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
-  for (int k = 0; k < kAccRows; ++k)
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Activation row b of a GEMV family into shared memory (sm.xs, fp32): the 8
+// compute warps load it once for the CTA (adding the previous layer's down
+// partials to x when asked), reduce its sum of squares and apply the RMSNorm
+// in place.  Called by all compute warps for the same task (the tag sequence
+// is the same for all warps).
+__device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int b) {
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
+  const int K = g.K;
+  const float* src;
+  size_t rstride;
+  if (g.kind == 0) { src = reinterpret_cast<const float*>(ws + P.off_x); rstride = P.hidden; }
+  else if (g.kind == 1) { src = reinterpret_cast<const float*>(ws + P.off_attn); rstride = (size_t)P.n_q_heads * P.head_dim; }
+  else { src = reinterpret_cast<const float*>(ws + P.off_h) + (size_t)g.kc * P.kseg; rstride = P.ffn; }
+  const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
+  bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the previous activation
+  float ss = 0.f;
+  for (int c = ct * 8; c < K; c += kComputeThreads * 8) {
+    const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
+    float4 u = __ldcg(p4), v = __ldcg(p4 + 1);
+    if (g.parts) {
+      float4 du[4], dv[4];
+      const int nq = min(P.n_kc, 4);
 #pragma unroll
-    for (int b = 0; b < kMaxB; ++b) acc[k][b] = 0.f;
-  bool ok = true;
+      for (int q = 0; q < 4; ++q)
+        if (q < nq) {
+          const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
+          du[q] = __ldcg(d4);
+          dv[q] = __ldcg(d4 + 1);
+        }
 #pragma unroll
-  for (int s = 0; s < kAccRows / 4; ++s) {
-    if (s < d.nslots) {
-      uint32_t seq = (uint32_t)d.ring_seq + s;
-      int slot = seq % P.ring_slots;
-      if (!wait_mbar(&sm.full[slot], (seq / P.ring_slots) & 1, ctl, P.spin_timeout_ns, d.fam, d.idx)) ok = false;
-      const unsigned char* base = ring + (size_t)slot * P.slot_bytes;
+      for (int q = 0; q < 4; ++q)
+        if (q < nq) {
+          u.x += du[q].x; u.y += du[q].y; u.z += du[q].z; u.w += du[q].w;
+          v.x += dv[q].x; v.y += dv[q].y; v.z += dv[q].z; v.w += dv[q].w;
+        }
+      for (int q = 4; q < P.n_kc; ++q) {
+        const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
+        float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
+        u.x += a4.x; u.y += a4.y; u.z += a4.z; u.w += a4.w;
+        v.x += b4.x; v.y += b4.y; v.z += b4.z; v.w += b4.w;
+      }
+    }
+    *reinterpret_cast<float4*>(&sm.xs[c]) = u;
+    *reinterpret_cast<float4*>(&sm.xs[c + 4]) = v;
+    ss += u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w + v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  if (g.kind == 0) {
+    ss = warp_sum(ss);
+    if (lane == 0) sm.red8[w] = ss;
+    bar_sync(BAR_COMP, kComputeThreads);
+    float tot = 0.f;
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        int rl = rg + rr * G;
-        if (s * rps + rl < valid_rows) {
-          uint4 w = *reinterpret_cast<const uint4*>(base + (size_t)rl * K * 2 + cb * 16);
-          float wf[8];
-          bf16x8_to_f32(w, wf);
+    for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[q];
+    const float inv = 1.0f / sqrtf(tot / (float)K + P.eps);
+    const uint4* gam = reinterpret_cast<const uint4*>(g.gamma);
+    for (int c = ct * 8; c < K; c += kComputeThreads * 8) {
+      float gf[8];
+      bf16x8_to_f32(__ldg(gam + c / 8), gf);
+      float4* x4 = reinterpret_cast<float4*>(&sm.xs[c]);
+      float4 u = x4[0], v = x4[1];
+      u.x *= inv * gf[0]; u.y *= inv * gf[1]; u.z *= inv * gf[2]; u.w *= inv * gf[3];
+      v.x *= inv * gf[4]; v.y *= inv * gf[5]; v.z *= inv * gf[6]; v.w *= inv * gf[7];
+      x4[0] = u;
+      x4[1] = v;
+    }
+  }
+  bar_sync(BAR_COMP, kComputeThreads);  // the activation is complete
+}
+
+// A lane holds columns 256*i + 8*lane + j (i < K/256, j < 8) of the staged
+// activation row in registers, so the dot products read only weights from
+// shared memory.
+typedef float ActRegs[kMaxBlk][8];
+
+__device__ __forceinline__ void act_to_regs(const float* xs, int nblk, ActRegs& av) {
+  const int lane = threadIdx.x & 31;
+  const float4* a4 = reinterpret_cast<const float4*>(xs) + 2 * lane;
 #pragma unroll
-          for (int b = 0; b < kMaxB; ++b) {
-            float t = acc[s * 4 + rr][b];
+  for (int i = 0; i < kMaxBlk; ++i) {
+    if (i < nblk) {
+      const float4 u = a4[i * 64], v = a4[i * 64 + 1];
+      av[i][0] = u.x; av[i][1] = u.y; av[i][2] = u.z; av[i][3] = u.w;
+      av[i][4] = v.x; av[i][5] = v.y; av[i][6] = v.z; av[i][7] = v.w;
+    } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) t = fmaf(wf[j], a.v[b][j], t);
-            acc[s * 4 + rr][b] = t;
+      for (int j = 0; j < 8; ++j) av[i][j] = 0.f;
+    }
+  }
+}
+
+// Dot product of one weight row (bf16, in a ring slot) with the activation
+// registers, reduced over the warp.
+__device__ __forceinline__ float warp_dot(const unsigned char* rowp, int nblk, const ActRegs& av) {
+  const int lane = threadIdx.x & 31;
+  const uint4* r4 = reinterpret_cast<const uint4*>(rowp) + lane;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < kMaxBlk; ++i) {
+    if (i < nblk) {
+      float wf[8];
+      bf16x8_to_f32(r4[i * 32], wf);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j & 3] = fmaf(wf[j], av[i][j], acc[j & 3]);
+    }
+  }
+  return warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
+}
+
+// Ring position of the task's slots.
+struct TaskSlots {
+  int n;
+  int idx[4];
+  uint32_t par[4];
+};
+__device__ __forceinline__ void task_slots_of(const DevPlan& P, const TaskDesc& d, TaskSlots& ts) {
+  ts.n = d.nslots;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t q = (uint32_t)d.ring_seq + j;
+    ts.idx[j] = (int)(q % (uint32_t)P.ring_slots);
+    ts.par[j] = (q / (uint32_t)P.ring_slots) & 1;
+  }
+}
+
+// One warp's share of a GEMV task for batch row b: whole rows (or
+// rotate-half / gate-up row pairs, first rows of part 0 then of part 1), each
+// reduced inside the warp and written by lane 0.  The warp releases a ring
+// slot as soon as it has no more rows in it.
+__device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
+                                               unsigned char* ws, Control* ctl, const TaskDesc& d,
+                                               const GemvSpec& g, const TaskSlots& ts, const ActRegs& av, int b,
+                                               uint32_t* trec, bool release) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int K = g.K, nblk = K >> 8;
+  const int rps = P.slot_bytes / (2 * K);
+  const int lg = __ffs(rps) - 1;
+  const int H = P.hidden;
+  unsigned ready = 0;  // slots waited on
+  // this warp's rows, in increasing order (so in non-decreasing slot order):
+  // row ops take rows w, w+8, ...; pair ops take pairs p = w, w+8, ... and
+  // visit rows p of part 0, then rows half + p of part 1
+  const bool pairs = d.op == OP_QKV || d.op == OP_GATEUP;
+  const int half = d.op == OP_QKV ? P.tile_qkv / 2 : P.tile_gu;
+  const int nrow_task = pairs ? half : (d.op == OP_OPROJ ? P.tile_o : (d.op == OP_DOWN ? P.tile_down : g.rows));
+  const int npair = pairs ? max(0, (half - w + kComputeWarps - 1) / kComputeWarps) : 0;
+  const int nr = pairs ? 2 * npair : max(0, (nrow_task - w + kComputeWarps - 1) / kComputeWarps);
+  auto row_of = [&](int k) -> int {
+    return pairs ? (k < npair ? w + kComputeWarps * k : half + w + kComputeWarps * (k - npair))
+                 : w + kComputeWarps * k;
+  };
+  if (release && lane == 0) {
+    unsigned mine = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < nr) mine |= 1u << (row_of(k) >> lg);
+    for (int j = 0; j < ts.n; ++j)
+      if (!(mine & (1u << j))) mbar_arrive(&sm.empty[ts.idx[j]]);
+  }
+  float* y = sm.yw[w];
+#pragma unroll 1
+  for (int k = 0; k < 8; ++k) {
+    if (k < nr) {
+      const int r = row_of(k), js = r >> lg;
+      if (!(ready & (1u << js))) {
+        wait_mbar(&sm.full[ts.idx[js]], ts.par[js], ctl, P.spin_timeout_ns, d.fam, d.idx);
+        ready |= 1u << js;
+        if (js == 0 && trec && lane == 0) {
+          trec[TR_DATA] = (uint32_t)global_ns();
+          trec[TR_ISSUE] = sm.slot_t[ts.idx[0]];
+        }
+      }
+      const float yk = warp_dot(ring + (size_t)ts.idx[js] * P.slot_bytes + (size_t)(r & (rps - 1)) * K * 2, nblk, av);
+      if (lane == 0) y[k] = yk;
+      // release the slot once this warp has no further row in it
+      if (release && (k + 1 >= nr || (row_of(k + 1) >> lg) != js)) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[ts.idx[js]]);
+      }
+    }
+  }
+  if (lane != 0) return;
+  switch (d.op) {
+    case OP_QKV: {
+      // RoPE on q and k (rotate-half pairs j, j + D/2), then q -> buffer, k/v -> cache
+      QkvTile q = decode_qkv(P, d.idx);
+      const int pos = sm.ctx[b];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (k >= npair) break;
+        const int j = q.j0 + row_of(k);
+        const float x0 = y[k], x1 = y[npair + k];
+        if (q.kind == 2) {
+          size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
+          __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * P.head_dim;
+          vc[j] = __float2bfloat16_rn(x0);
+          vc[j + 32] = __float2bfloat16_rn(x1);
+        } else {
+          const float* rope = reinterpret_cast<const float*>(ws + P.off_rope) + ((size_t)pos * 32 + j) * 2;
+          const float c = __ldg(rope), sn = __ldg(rope + 1);
+          const float r0 = x0 * c - x1 * sn, r1 = x1 * c + x0 * sn;
+          if (q.kind == 0) {
+            float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * P.head_dim +
+                        q.head * P.head_dim;
+            qb[j] = r0;
+            qb[j + 32] = r1;
+          } else {
+            size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
+            __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * P.head_dim;
+            kc[j] = __float2bfloat16_rn(r0);
+            kc[j + 32] = __float2bfloat16_rn(r1);
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[slot]);
-    }
-  }
-  // reduce each (row, b) over the K/8 threads of the row group
+    } break;
+    case OP_GATEUP: {
+      float* h = reinterpret_cast<float*>(ws + P.off_h) + (size_t)b * P.ffn + (size_t)d.idx * P.tile_gu;
 #pragma unroll
-  for (int k = 0; k < kAccRows; ++k) {
-    if (k < 4 * d.nslots) {
-#pragma unroll
-      for (int b = 0; b < kMaxB; ++b) {
-        if (b < B) {
-          float v = acc[k][b];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == 0) sm.red[cw][k * kMaxB + b] = v;
-        }
+      for (int k = 0; k < 4; ++k) {
+        if (k >= npair) break;
+        const float gt = y[k], up = y[npair + k];
+        h[row_of(k)] = gt / (1.0f + expf(-gt)) * up;
       }
-    }
+    } break;
+    case OP_OPROJ: {
+      // residual: x = (x + previous layer's down partials) + o W_o^T
+      float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
+      const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k >= nr) break;
+        const size_t col = (size_t)d.idx * P.tile_o + row_of(k);
+        float xv = __ldcg(x + col);
+        if (d.layer > 0)
+          for (int q = 0; q < P.n_kc; ++q) xv += __ldcg(dp + ((size_t)q * P.max_batch + b) * H + col);
+        x[col] = xv + y[k];
+      }
+    } break;
+    case OP_DOWN: {
+      const int n = d.idx - g.kc * P.n_dtiles;
+      float* part = reinterpret_cast<float*>(ws + P.off_dpart) + ((size_t)g.kc * P.max_batch + b) * H +
+                    (size_t)n * P.tile_down;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (k < nr) part[row_of(k)] = y[k];
+    } break;
+    case OP_LM: {
+      // logits and this warp's best (logit, id) key, folded into the running
+      // maximum with an atomic max (order independent)
+      const int r0 = d.idx * P.tile_lm;
+      unsigned long long best = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k >= nr) break;
+        if (S.logits) S.logits[(size_t)b * P.vocab + r0 + row_of(k)] = y[k];
+        unsigned long long key = argmax_key(y[k], r0 + row_of(k));
+        best = key > best ? key : best;
+      }
+      if (best) atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, best);
+    } break;
+    default: break;
   }
-  bar_sync(BAR_COMP, kComputeThreads);
-  const int wpg = kb / 32;
-  const int rows = d.nslots * rps;
-  for (int e = ct; e < rows * kMaxB; e += kComputeThreads) {
-    int row = e / kMaxB, b = e % kMaxB;
-    if (b >= B) continue;
-    int s = row / rps, rl = row % rps;
-    int g = rl % G, rr = rl / G;
-    int k = s * 4 + rr;
-    float v = 0.f;
-    for (int w = 0; w < wpg; ++w) v += sm.red[g * wpg + w][k * kMaxB + b];
-    sm.fin[row * kMaxB + b] = v;
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  return ok;
 }
 
-__device__ void task_attn(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
-                          Control* ctl, const TaskDesc& d) {
-  const int ct = threadIdx.x - 64, cw = ct >> 5, lane = ct & 31;
+__device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
+                                       unsigned char* ws, Control* ctl, const TaskDesc& d) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, D = P.head_dim, CH = P.chunk;
-  AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
-  const int p = sm.ctx[a.b];
-  const int n_old = max(0, min(CH, p - a.c * CH));
-  const bool has_new = (p - a.c * CH) < CH;
-  const int n_keys = n_old + (has_new ? 1 : 0);
-  const float* q = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D + (size_t)a.g * qpg * D;
-  if (ct < qpg * D) sm.qs[ct] = __ldcg(q + ct) * 0.125f;  // 1/sqrt(64)
-  if (has_new && ct < 2 * D) {
-    size_t row = (((size_t)d.layer * P.n_slots + sm.slot[a.b]) * Hkv + a.g) * P.max_ctx + p;
-    const unsigned short* src =
-        reinterpret_cast<const unsigned short*>(ct < D ? P.k_cache : P.v_cache) + row * D + (ct % D);
-    float v = bf16_bits_to_f32(__ldcg(src));
-    if (ct < D) sm.newk[ct] = v; else sm.newv[ct - D] = v;
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  uint32_t seq = (uint32_t)d.ring_seq;
-  int slot = seq % P.ring_slots;
-  wait_mbar(&sm.full[slot], (seq / P.ring_slots) & 1, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
-  const unsigned char* vbase = kbase + (size_t)CH * D * 2;
-  // scores: thread -> (key kk, head h)
-  {
-    int kk = ct >> 2, h = ct & 3;
-    if (h < qpg) {
+  const uint32_t seq = (uint32_t)d.ring_seq;
+  const int slot = (int)(seq % (uint32_t)P.ring_slots);
+  if (w < qpg) {
+    // warp w: query head g*qpg + w over this chunk's keys
+    AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
+    const int p = sm.ctx[a.b];
+    const int n_old = max(0, min(CH, p - a.c * CH));
+    const bool has_new = (p - a.c * CH) < CH;
+    const int n_keys = n_old + (has_new ? 1 : 0);
+    float* qs = sm.qs[w];
+    float* ps = sm.ps[w];
+    const float* q = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D +
+                     (size_t)(a.g * qpg + w) * D;
+    qs[lane] = __ldcg(q + lane) * 0.125f;  // 1/sqrt(64)
+    qs[lane + 32] = __ldcg(q + lane + 32) * 0.125f;
+    if (has_new) {
+      size_t row = (((size_t)d.layer * P.n_slots + sm.slot[a.b]) * Hkv + a.g) * P.max_ctx + p;
+      const unsigned short* kn = reinterpret_cast<const unsigned short*>(P.k_cache) + row * D;
+      const unsigned short* vn = reinterpret_cast<const unsigned short*>(P.v_cache) + row * D;
+      sm.newk[w][lane] = bf16_bits_to_f32(__ldcg(kn + lane));
+      sm.newk[w][lane + 32] = bf16_bits_to_f32(__ldcg(kn + lane + 32));
+      sm.newv[w][lane] = bf16_bits_to_f32(__ldcg(vn + lane));
+      sm.newv[w][lane + 32] = bf16_bits_to_f32(__ldcg(vn + lane + 32));
+    }
+    __syncwarp();
+    wait_mbar(&sm.full[slot], (seq / (uint32_t)P.ring_slots) & 1, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
+    const unsigned char* vbase = kbase + (size_t)CH * D * 2;
+    // scores of keys lane and lane + 32
+    float sc[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int kk = lane + 32 * h2;
       float s = -INFINITY;
       if (kk < n_old) {
         s = 0.f;
         const uint4* kr = reinterpret_cast<const uint4*>(kbase + (size_t)kk * D * 2);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          int ci = (i + kk) & 7;  // rotate the start so the warp's rows hit distinct banks
+          const int ci = (i + kk) & 7;  // rotate the start so the lanes' rows hit distinct banks
           float kf[8];
           bf16x8_to_f32(kr[ci], kf);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) s = fmaf(kf[j], sm.qs[h * D + ci * 8 + j], s);
+          for (int j = 0; j < 8; ++j) s = fmaf(kf[j], qs[ci * 8 + j], s);
         }
       } else if (kk < n_keys) {
         s = 0.f;
-        for (int j = 0; j < D; ++j) s = fmaf(sm.newk[j], sm.qs[h * D + j], s);
+        for (int j = 0; j < D; ++j) s = fmaf(sm.newk[w][j], qs[j], s);
       }
-      sm.sc[h][kk] = s;
+      sc[h2] = s;
     }
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  if (cw < qpg) {
-    float v0 = sm.sc[cw][lane], v1 = sm.sc[cw][lane + 32];
-    float m = fmaxf(v0, v1);
+    float m = fmaxf(sc[0], sc[1]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float e0 = lane < n_keys ? expf(v0 - m) : 0.f;
-    float e1 = lane + 32 < n_keys ? expf(v1 - m) : 0.f;
-    float l = e0 + e1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    sm.sc[cw][lane] = e0;
-    sm.sc[cw][lane + 32] = e1;
-    if (lane == 0) { sm.hm[cw] = m; sm.hl[cw] = l; }
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  {
-    int h = ct >> 6, dd = ct & 63;
-    if (h < qpg) {
-      float o = 0.f;
-      for (int kk = 0; kk < n_old; ++kk) {
-        unsigned short vb = *reinterpret_cast<const unsigned short*>(vbase + (size_t)kk * D * 2 + dd * 2);
-        o = fmaf(sm.sc[h][kk], bf16_bits_to_f32(vb), o);
-      }
-      if (has_new) o = fmaf(sm.sc[h][n_old], sm.newv[dd], o);
-      float* part = reinterpret_cast<float*>(ws + P.off_apart) +
-                    (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2));
-      part[h * (D + 2) + dd] = o;
-      if (dd == 0) { part[h * (D + 2) + D] = sm.hm[h]; part[h * (D + 2) + D + 1] = sm.hl[h]; }
+    const float e0 = lane < n_keys ? expf(sc[0] - m) : 0.f;
+    const float e1 = lane + 32 < n_keys ? expf(sc[1] - m) : 0.f;
+    const float l = warp_sum(e0 + e1);
+    ps[lane] = e0;
+    ps[lane + 32] = e1;
+    __syncwarp();
+    float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int kk = 0; kk < n_old; ++kk) {
+      const unsigned short* vr = reinterpret_cast<const unsigned short*>(vbase + (size_t)kk * D * 2);
+      const float pk = ps[kk];
+      o0[kk & 3] = fmaf(pk, bf16_bits_to_f32(vr[lane]), o0[kk & 3]);
+      o1[kk & 3] = fmaf(pk, bf16_bits_to_f32(vr[lane + 32]), o1[kk & 3]);
     }
+    float r0 = (o0[0] + o0[1]) + (o0[2] + o0[3]), r1 = (o1[0] + o1[1]) + (o1[2] + o1[3]);
+    if (has_new) {
+      r0 = fmaf(ps[n_old], sm.newv[w][lane], r0);
+      r1 = fmaf(ps[n_old], sm.newv[w][lane + 32], r1);
+    }
+    float* part = reinterpret_cast<float*>(ws + P.off_apart) +
+                  (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2)) + w * (D + 2);
+    part[lane] = r0;
+    part[lane + 32] = r1;
+    if (lane == 0) { part[D] = m; part[D + 1] = l; }
   }
   __syncwarp();
   if (lane == 0) mbar_arrive(&sm.empty[slot]);
 }
 
-__device__ void task_merge(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, const TaskDesc& d) {
-  const int ct = threadIdx.x - 64;
+// Merge of a head group's chunk partials, softmax-weighted in chunk order:
+// the chunk maxima and weights are computed lane-parallel (lane c holds chunk
+// c, c + 32, ...), then each lane sums its output dimension over the chunks.
+__device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws,
+                                        const TaskDesc& d) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, D = P.head_dim;
+  const int h = w >> 1, dd = (w & 1) * 32 + lane;
+  if (h >= qpg) return;
   const int b = d.idx / Hkv, g = d.idx % Hkv;
   const int nch = sm.nch[b];
-  int h = ct >> 6, dd = ct & 63;
-  if (h >= qpg) return;
-  const float* part = reinterpret_cast<const float*>(ws + P.off_apart) +
-                      ((size_t)b * Hkv + g) * P.max_chunks * (size_t)(qpg * (D + 2)) + h * (D + 2);
   const size_t cs = (size_t)qpg * (D + 2);
+  const float* part = reinterpret_cast<const float*>(ws + P.off_apart) + ((size_t)b * Hkv + g) * P.max_chunks * cs +
+                      h * (D + 2);
   float M = -INFINITY;
-  for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(part + c * cs + D));
+  for (int c = lane; c < nch; c += 32) M = fmaxf(M, __ldcg(part + c * cs + D));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float L = 0.f, O = 0.f;
-  for (int c = 0; c < nch; ++c) {
-    float w = expf(__ldcg(part + c * cs + D) - M);
-    L = fmaf(__ldcg(part + c * cs + D + 1), w, L);
-    O = fmaf(__ldcg(part + c * cs + dd), w, O);
+  for (int c0 = 0; c0 < nch; c0 += 32) {
+    const int c = c0 + lane;
+    const float e = c < nch ? expf(__ldcg(part + c * cs + D) - M) : 0.f;
+    L += warp_sum(c < nch ? __ldcg(part + c * cs + D + 1) * e : 0.f);
+    const int n = min(32, nch - c0);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int q = 0; q < n; ++q) acc[q & 3] = fmaf(__ldcg(part + (c0 + q) * cs + dd), __shfl_sync(0xffffffffu, e, q), acc[q & 3]);
+    O += (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
   float* out = reinterpret_cast<float*>(ws + P.off_attn) + (size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D;
   out[dd] = O / L;
@@ -769,160 +1193,46 @@ __device__ void task_merge(const DevPlan& P, const StepParams& S, Smem& sm, unsi
 
 __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
                         Control* ctl) {
-  const int ct = threadIdx.x - 64, cw = ct >> 5, lane = ct & 31;
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
-  const int B = S.B, H = P.hidden;
-  float* x = reinterpret_cast<float*>(ws + P.off_x);
-  Act a;
-  a.tag = -1;
-  for (;;) {
-    bar_sync(BAR_GO, kCtlThreads);
-    const TaskDesc d = sm.cur;
+  const int B = S.B;
+  int a_tag = -1;
+  ActRegs av;
+  for (uint32_t k = 0;; ++k) {
+    // task k: released into cur[k & 1] as phase k >> 1 of go_bar[k & 1]
+    if (!wait_mbar(&sm.go_bar[k & 1], (k >> 1) & 1, ctl, P.spin_timeout_ns, -1, -1)) break;
+    const TaskDesc d = sm.cur[k & 1];
     if (d.op == OP_END) break;
-    switch (d.op) {
-      case OP_QKV: {
-        int tag = d.layer * 64 + 0;
-        if (a.tag != tag) { load_act(P, sm, ws, B, 0, layers[d.layer].attn_norm, 0, H, a); a.tag = tag; }
-        gemv_rows(P, sm, ring, ctl, d, H, P.tile_qkv, B, a);
-        QkvTile q = decode_qkv(P, d.idx);
-        int half = P.tile_qkv / 2;
-        for (int e = ct; e < half * kMaxB; e += kComputeThreads) {
-          int jj = e / kMaxB, b = e % kMaxB;
-          if (b >= B) continue;
-          int j = q.j0 + jj;
-          float x0 = sm.fin[jj * kMaxB + b], x1 = sm.fin[(half + jj) * kMaxB + b];
-          int pos = sm.ctx[b];
-          if (q.kind == 2) {
-            size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
-            __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * P.head_dim;
-            vc[j] = __float2bfloat16_rn(x0);
-            vc[j + 32] = __float2bfloat16_rn(x1);
-          } else {
-            const float* rope = reinterpret_cast<const float*>(ws + P.off_rope) + ((size_t)pos * 32 + j) * 2;
-            float c = __ldg(rope), s = __ldg(rope + 1);
-            float y0 = x0 * c - x1 * s, y1 = x1 * c + x0 * s;
-            if (q.kind == 0) {
-              float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * P.head_dim + q.head * P.head_dim;
-              qb[j] = y0;
-              qb[j + 32] = y1;
-            } else {
-              size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
-              __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * P.head_dim;
-              kc[j] = __float2bfloat16_rn(y0);
-              kc[j + 32] = __float2bfloat16_rn(y1);
-            }
-          }
+    uint32_t* trec = (d.rec > 0 && w == 0) ? trace_rec(S, d.rec) : nullptr;
+    if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
+    GemvSpec g;
+    if (gemv_spec(P, layers, d, g)) {
+      TaskSlots ts;
+      task_slots_of(P, d, ts);
+      // one pass per batch row (the activation is restaged each pass when
+      // B > 1); the ring slots are released after the last pass
+      for (int b = 0; b < B; ++b) {
+        if (B > 1 || g.tag != a_tag) {
+          stage_act(P, ws, sm, g, b);
+          act_to_regs(sm.xs, g.K >> 8, av);
+          a_tag = B > 1 ? -1 : g.tag;
         }
-      } break;
-      case OP_ATTN: task_attn(P, S, sm, ring, ws, ctl, d); break;
-      case OP_MERGE: task_merge(P, S, sm, ws, d); break;
-      case OP_OPROJ: {
-        int tag = d.layer * 64 + 1;
-        if (a.tag != tag) { load_act(P, sm, ws, B, 1, nullptr, 0, H, a); a.tag = tag; }
-        gemv_rows(P, sm, ring, ctl, d, H, P.tile_o, B, a);
-        for (int e = ct; e < P.tile_o * kMaxB; e += kComputeThreads) {
-          int r = e / kMaxB, b = e % kMaxB;
-          if (b >= B) continue;
-          float* xp = x + (size_t)b * H + d.idx * P.tile_o + r;
-          *xp = __ldcg(xp) + sm.fin[r * kMaxB + b];
-        }
-      } break;
-      case OP_GATEUP: {
-        int tag = d.layer * 64 + 2;
-        if (a.tag != tag) { load_act(P, sm, ws, B, 0, layers[d.layer].ffn_norm, 0, H, a); a.tag = tag; }
-        gemv_rows(P, sm, ring, ctl, d, H, 2 * P.tile_gu, B, a);
-        float* h = reinterpret_cast<float*>(ws + P.off_h);
-        for (int e = ct; e < P.tile_gu * kMaxB; e += kComputeThreads) {
-          int r = e / kMaxB, b = e % kMaxB;
-          if (b >= B) continue;
-          float g = sm.fin[r * kMaxB + b], u = sm.fin[(P.tile_gu + r) * kMaxB + b];
-          h[(size_t)b * P.ffn + d.idx * P.tile_gu + r] = g / (1.0f + expf(-g)) * u;
-        }
-      } break;
-      case OP_DOWN: {
-        int kc = d.idx / P.n_dtiles, n = d.idx % P.n_dtiles;
-        int tag = d.layer * 64 + 8 + kc;
-        if (a.tag != tag) { load_act(P, sm, ws, B, 2, nullptr, kc, P.kseg, a); a.tag = tag; }
-        gemv_rows(P, sm, ring, ctl, d, P.kseg, P.tile_down, B, a);
-        float* part = reinterpret_cast<float*>(ws + P.off_dpart);
-        for (int e = ct; e < P.tile_down * kMaxB; e += kComputeThreads) {
-          int r = e / kMaxB, b = e % kMaxB;
-          if (b >= B) continue;
-          part[((size_t)kc * P.max_batch + b) * H + n * P.tile_down + r] = sm.fin[r * kMaxB + b];
-        }
-      } break;
-      case OP_DRED: {
-        const float* part = reinterpret_cast<const float*>(ws + P.off_dpart);
-        for (int e = ct; e < P.tile_down * kMaxB; e += kComputeThreads) {
-          int r = e / kMaxB, b = e % kMaxB;
-          if (b >= B) continue;
-          size_t col = (size_t)d.idx * P.tile_down + r;
-          float y = 0.f;
-          for (int kc = 0; kc < P.n_kc; ++kc) y += __ldcg(part + ((size_t)kc * P.max_batch + b) * H + col);
-          float* xp = x + (size_t)b * H + col;
-          *xp = __ldcg(xp) + y;
-        }
-      } break;
-      case OP_LM: {
-        int tag = 60 * 64;
-        if (a.tag != tag) { load_act(P, sm, ws, B, 0, P.final_norm, 0, H, a); a.tag = tag; }
-        int r0 = d.idx * P.tile_lm;
-        int vr = min(P.tile_lm, P.vocab - r0);
-        gemv_rows(P, sm, ring, ctl, d, H, vr, B, a);
-        if (S.logits)
-          for (int e = ct; e < vr * kMaxB; e += kComputeThreads) {
-            int r = e / kMaxB, b = e % kMaxB;
-            if (b < B) S.logits[(size_t)b * P.vocab + r0 + r] = sm.fin[r * kMaxB + b];
-          }
-        if (cw < B) {
-          unsigned long long best = 0;
-          for (int r = lane; r < vr; r += 32) {
-            unsigned long long k = argmax_key(sm.fin[r * kMaxB + cw], r0 + r);
-            best = k > best ? k : best;
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            unsigned long long v = __shfl_xor_sync(0xffffffffu, best, o);
-            best = v > best ? v : best;
-          }
-          if (lane == 0)
-            reinterpret_cast<unsigned long long*>(ws + P.off_lmpart)[(size_t)cw * P.n_lm_tiles + d.idx] = best;
-        }
-      } break;
-      case OP_LMGRP:
-      case OP_LMFIN: {
-        if (cw < B) {
-          const unsigned long long* src;
-          int n;
-          if (d.op == OP_LMGRP) {
-            int t0 = d.idx * P.lm_group;
-            n = min(P.lm_group, P.n_lm_tiles - t0);
-            src = reinterpret_cast<const unsigned long long*>(ws + P.off_lmpart) + (size_t)cw * P.n_lm_tiles + t0;
-          } else {
-            n = P.n_lmgrp;
-            src = reinterpret_cast<const unsigned long long*>(ws + P.off_lmgpart) + (size_t)cw * P.n_lmgrp;
-          }
-          unsigned long long best = 0;
-          for (int i = lane; i < n; i += 32) {
-            unsigned long long k = __ldcg(src + i);
-            best = k > best ? k : best;
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            unsigned long long v = __shfl_xor_sync(0xffffffffu, best, o);
-            best = v > best ? v : best;
-          }
-          if (lane == 0) {
-            if (d.op == OP_LMGRP)
-              reinterpret_cast<unsigned long long*>(ws + P.off_lmgpart)[(size_t)cw * P.n_lmgrp + d.idx] = best;
-            else
-              S.next_tokens[cw] = argmax_key_index(best);
-          }
-        }
-      } break;
-      default: break;
+        warp_gemv_task(P, S, sm, ring, ws, ctl, d, g, ts, av, b, trec, b == B - 1);
+      }
+    } else if (d.op == OP_ATTN) {
+      task_attn(P, S, sm, ring, ws, ctl, d);
+    } else if (d.op == OP_MERGE) {
+      task_merge(P, S, sm, ws, d);
+    } else if (d.op == OP_LMFIN) {
+      if (w < B && lane == 0) {
+        unsigned long long k = __ldcg(reinterpret_cast<const unsigned long long*>(ws + P.off_lmbest) + w);
+        S.next_tokens[w] = argmax_key_index(k);
+      }
     }
-    bar_arrive(BAR_DONE, kCtlThreads);
+    if (trec && lane == 0) trec[TR_CEND] = (uint32_t)global_ns();
+    // every lane of the warp has finished its writes before lane 0 arrives
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.done_bar[k & 1]);
   }
 }
 
@@ -939,7 +1249,11 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   const int B = S.B;
 
   // ---- prologue: resolve the symbols, arm the Event Tensors, gather embeddings
-  if (tid == 0) { sm.bad = (B < 1 || B > P.max_batch || B > kMaxB) ? 1 : 0; sm.released = 0; }
+  if (tid == 0) {
+    sm.bad = (B < 1 || B > P.max_batch || B > kMaxB) ? 1 : 0;
+    sm.released = 0;
+    sm.dq_head = sm.dq_tail = sm.fq_head = sm.fq_tail = sm.notifier_stop = 0;
+  }
   __syncthreads();
   if (!sm.bad && tid < B) {
     int c = S.ctx[tid], s = S.slots[tid], t = S.tokens[tid];
@@ -967,6 +1281,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   for (int f = tid; f < P.n_families; f += blockDim.x) {
     ExprEnv env{B, sm.ctx, {0, 0, 0}};
     sm.fam_ext[f] = expr_eval(code, fams[f].extent_expr, env);
+    sm.fam_op[f] = (signed char)fams[f].op;
+    sm.fam_layer[f] = (signed char)fams[f].layer;
   }
   const int gtid = blockIdx.x * blockDim.x + tid, gthreads = gridDim.x * blockDim.x;
   for (int i = gtid; i < P.n_counters; i += gthreads) {
@@ -990,6 +1306,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
       dst[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
   }
+  if (blockIdx.x == 0 && tid < P.max_batch)
+    reinterpret_cast<unsigned long long*>(ws + P.off_lmbest)[tid] = 0ull;  // running argmax keys
   if (blockIdx.x == 0 && tid == 0 && P.sched == MK_SCHED_DYNAMIC) {
     ctl->q_head = 0;
     ctl->q_tail = 0;
@@ -997,6 +1315,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   }
   if (tid == 0) {
     for (int s = 0; s < P.ring_slots; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], kComputeWarps); }
+    for (int j = 0; j < 2; ++j) { mbar_init(&sm.go_bar[j], 1); mbar_init(&sm.done_bar[j], kComputeWarps); }
     for (int k = 0; k < kFifo; ++k) { mbar_init(&sm.fifo_full[k], 1); mbar_init(&sm.fifo_empty[k], 1); }
     fence_proxy_async_smem();
   }
@@ -1022,6 +1341,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     if ((tid & 31) == 0) producer(P, S, sm, ring, ws, ctl);
   } else if (warp == 1) {
     controller(P, S, sm, ws, ctl, counters);
+  } else if (warp == 2) {
+    notifier(P, S, sm, ws, ctl, counters);
   } else {
     compute(P, S, sm, ring, ws, ctl);
   }
@@ -1078,6 +1399,9 @@ mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& 
   sp.logits = a->logits;
   sp.next_tokens = a->next_tokens;
   sp.task_counts = a->task_counts;
+  sp.trace = (p.dp.debug_flags & MK_DEBUG_TRACE) ? (uint32_t*)a->trace : nullptr;
+  sp.trace_cap = a->trace_cap;
+  if (sp.trace && sp.trace_cap < 2) sp.trace = nullptr;
   sp.epoch = p.epoch + 1;
   unsigned char* ws = (unsigned char*)p.ws;
   DevPlan dp = p.dp;

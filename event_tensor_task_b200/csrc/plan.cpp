@@ -6,10 +6,15 @@
 //   MERGE (follow-up)                     notify EV_ATTN[l]
 //   OPROJ tiles      wait EV_ATTN[l]      notify EV_O[l]
 //   GATEUP tiles     wait EV_O[l]         notify EV_GU[l][kc]
-//   DOWN tiles       wait EV_GU[l][kc]    notify EV_DSUM[l][n] -> DRED(n)
-//   DRED (follow-up)                      notify EV_IN[l+1]
-// then LM tiles (wait EV_IN[L], notify EV_LMG[grp] -> LMGRP), LMGRP
-// (notify EV_LM -> LMFIN) and LMFIN.  Fine-grained events let a consumer
+//   DOWN tiles       wait EV_GU[l][kc]    notify EV_IN[l+1]
+// The residual after layer l's FFN is never materialised: it is the residual
+// after the attention block (X, updated in place by OPROJ) plus the sum of
+// layer l's K-segment partials of the down projection, and every reader of
+// the layer input (QKV and OPROJ of layer l+1, the LM head) adds the partials
+// itself.  This removes a reduction hop from every layer.
+// then LM tiles (wait EV_IN[L], notify EV_LM -> LMFIN) and LMFIN.  The LM
+// tiles fold their best (logit, id) key into a running maximum with an
+// atomic max; the order of those updates does not change the result.  Fine-grained events let a consumer
 // start on the subset of producer output it reads ("Event Tensor: A Unified
 // Abstraction for Compiling Dynamic Megakernel", section "Problem": coarse
 // kernel-boundary synchronisation; "Lecture 112: Production Megakernels for
@@ -27,10 +32,10 @@
 namespace mk {
 
 static const char* kOpNames[OP_COUNT] = {"end", "qkv", "attn", "merge", "oproj", "gateup",
-                                         "down", "dred", "lm", "lmgrp", "lmfin"};
-static const int kLayerOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_GATEUP, OP_DOWN, OP_DRED};
-static const int kLmOps[] = {OP_LM, OP_LMGRP, OP_LMFIN};
-static constexpr int kFamPerLayer = 7;
+                                         "down", "-", "lm", "-", "lmfin"};
+static const int kLayerOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_GATEUP, OP_DOWN};
+static const int kLmOps[] = {OP_LM, OP_LMFIN};
+static constexpr int kFamPerLayer = 6;
 
 // ---------------------------------------------------------------- expressions
 namespace {
@@ -47,7 +52,8 @@ int emit_const(std::vector<int32_t>& code, int v) { return Emit(code).push(v).re
 }  // namespace
 
 int Plan::fam_index(int op, int layer) const {
-  if (op >= OP_LM) return dp.n_layers * kFamPerLayer + (op - OP_LM);
+  if (op == OP_LM) return dp.n_layers * kFamPerLayer;
+  if (op == OP_LMFIN) return dp.n_layers * kFamPerLayer + 1;
   for (int k = 0; k < kFamPerLayer; ++k)
     if (kLayerOps[k] == op) return layer * kFamPerLayer + k;
   return -1;
@@ -93,6 +99,11 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       int half = P.tile_qkv / 2;
       for (int b = 0; b < B; ++b) {
         t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        if (l > 0)
+          for (int kc = 0; kc < P.n_kc; ++kc) {
+            long long pb = ((long long)kc * P.max_batch + b) * H;
+            t.reads.push_back({BUF_DPART, pb, pb + H});
+          }
         for (int part = 0; part < 2; ++part) {
           int j = q.j0 + part * (D / 2);
           if (q.kind == 0) {
@@ -138,6 +149,11 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
         t.reads.push_back({BUF_ATTN, b * QD, (b + 1) * QD});
         long long xb = (long long)b * H + (long long)idx * P.tile_o;
         t.reads.push_back({BUF_X, xb, xb + P.tile_o});
+        if (l > 0)
+          for (int kc = 0; kc < P.n_kc; ++kc) {
+            long long pb = ((long long)kc * P.max_batch + b) * H + (long long)idx * P.tile_o;
+            t.reads.push_back({BUF_DPART, pb, pb + P.tile_o});
+          }
         t.writes.push_back({BUF_X, xb, xb + P.tile_o});
       }
     } break;
@@ -153,9 +169,7 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
     case OP_DOWN: {
       int kc = idx / P.n_dtiles, n = idx % P.n_dtiles;
       t.wait_ev = counter(EV_GU, l, kc);
-      t.notify_ev = counter(EV_DSUM, l, n);
-      t.follow_fam = fam_index(OP_DRED, l);
-      t.follow_idx = n;
+      t.notify_ev = counter(EV_IN, l + 1);
       for (int b = 0; b < B; ++b) {
         long long hb = (long long)b * F + (long long)kc * P.kseg;
         t.reads.push_back({BUF_H, hb, hb + P.kseg});
@@ -163,48 +177,23 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
         t.writes.push_back({BUF_DPART, pb, pb + P.tile_down});
       }
     } break;
-    case OP_DRED: {
-      t.notify_ev = counter(EV_IN, l + 1);
-      for (int b = 0; b < B; ++b) {
-        for (int kc = 0; kc < P.n_kc; ++kc) {
-          long long pb = ((long long)kc * P.max_batch + b) * H + (long long)idx * P.tile_down;
-          t.reads.push_back({BUF_DPART, pb, pb + P.tile_down});
-        }
-        long long xb = (long long)b * H + (long long)idx * P.tile_down;
-        t.reads.push_back({BUF_X, xb, xb + P.tile_down});
-        t.writes.push_back({BUF_X, xb, xb + P.tile_down});
-      }
-    } break;
     case OP_LM: {
       t.wait_ev = counter(EV_IN, P.n_layers);
-      int grp = idx / P.lm_group;
-      t.notify_ev = counter(EV_LMG, grp);
-      t.follow_fam = fam_index(OP_LMGRP, -1);
-      t.follow_idx = grp;
-      int r0 = idx * P.tile_lm, r1 = std::min(P.vocab, r0 + P.tile_lm);
-      for (int b = 0; b < B; ++b) {
-        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
-        t.writes.push_back({BUF_LOGITS, (long long)b * P.vocab + r0, (long long)b * P.vocab + r1});
-        long long pb = (long long)b * P.n_lm_tiles + idx;
-        t.writes.push_back({BUF_LMPART, pb, pb + 1});
-      }
-    } break;
-    case OP_LMGRP: {
       t.notify_ev = counter(EV_LM, 0);
       t.follow_fam = fam_index(OP_LMFIN, -1);
       t.follow_idx = 0;
-      int t0 = idx * P.lm_group, t1 = std::min(P.n_lm_tiles, t0 + P.lm_group);
+      int r0 = idx * P.tile_lm, r1 = std::min(P.vocab, r0 + P.tile_lm);
       for (int b = 0; b < B; ++b) {
-        t.reads.push_back({BUF_LMPART, (long long)b * P.n_lm_tiles + t0, (long long)b * P.n_lm_tiles + t1});
-        long long gb = (long long)b * P.n_lmgrp + idx;
-        t.writes.push_back({BUF_LMG, gb, gb + 1});
+        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        for (int kc = 0; kc < P.n_kc; ++kc) {
+          long long pb = ((long long)kc * P.max_batch + b) * H;
+          t.reads.push_back({BUF_DPART, pb, pb + H});
+        }
+        t.writes.push_back({BUF_LOGITS, (long long)b * P.vocab + r0, (long long)b * P.vocab + r1});
       }
     } break;
     case OP_LMFIN: {
-      for (int b = 0; b < B; ++b) {
-        t.reads.push_back({BUF_LMG, (long long)b * P.n_lmgrp, (long long)(b + 1) * P.n_lmgrp});
-        t.writes.push_back({BUF_NEXT, b, b + 1});
-      }
+      for (int b = 0; b < B; ++b) t.writes.push_back({BUF_NEXT, b, b + 1});
     } break;
     default: break;
   }
@@ -239,7 +228,7 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
     case EV_ATTN: add(fam_index(OP_OPROJ, c[0]), 0, dp.n_otiles); break;
     case EV_O: add(fam_index(OP_GATEUP, c[0]), 0, dp.n_gutiles); break;
     case EV_GU: add(fam_index(OP_DOWN, c[0]), c[1] * dp.n_dtiles, dp.n_dtiles); break;
-    default: break;  // EV_CHUNK, EV_DSUM, EV_LMG, EV_LM trigger follow-ups
+    default: break;  // EV_CHUNK and EV_LM trigger follow-ups
   }
 }
 
@@ -281,12 +270,15 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   int kseg = o->kseg ? o->kseg : std::min(F, 2048);
   while (kseg > 256 && F % kseg) kseg -= 256;
   P.kseg = kseg;
-  P.tile_qkv = o->tile_qkv ? o->tile_qkv : std::min(64, 16384 / H);
-  P.tile_o = o->tile_o ? o->tile_o : 16384 / H;
-  P.tile_gu = o->tile_gu ? o->tile_gu : 8192 / H;
-  P.tile_down = o->tile_down ? o->tile_down : 16384 / kseg;
-  P.tile_lm = o->tile_lm ? o->tile_lm : 32768 / H;
-  P.lm_group = o->lm_group ? o->lm_group : 64;
+  // rows per 16 KB ring slot of a hidden-wide (and a kseg-wide) row
+  const int rps_h = 8192 / H, rps_k = 8192 / kseg;
+  // tiles split evenly over the 8 compute warps: QKV and gate/up tiles hand
+  // each warp whole row pairs, the others whole rows
+  P.tile_qkv = o->tile_qkv ? o->tile_qkv : std::max(16, 2 * rps_h);
+  P.tile_o = o->tile_o ? o->tile_o : std::max(8, rps_h);
+  P.tile_gu = o->tile_gu ? o->tile_gu : std::max(8, rps_h);
+  P.tile_down = o->tile_down ? o->tile_down : std::max(8, rps_k);
+  P.tile_lm = o->tile_lm ? o->tile_lm : std::max(16, rps_h);
   P.chunk = o->attn_chunk ? o->attn_chunk : 64;
   P.slot_bytes = 16384;
   const int rows_per_slot_h = P.slot_bytes / (2 * H);
@@ -294,33 +286,34 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (!(P.kseg % 256 == 0 && F % P.kseg == 0 && P.kseg >= 1024 && P.kseg <= 2048))
     { err = "kseg must be a multiple of 256 in [1024, 2048] dividing ffn"; return MK_ERR_INVALID_ARG; }
   if (Hq / Hkv > 4) { err = "at most 4 query heads per kv head"; return MK_ERR_UNSUPPORTED; }
-  if (!(pow2_divides(P.tile_qkv, D) && P.tile_qkv % 2 == 0 && (P.tile_qkv / 2) % rows_per_slot_h == 0 &&
-        P.tile_qkv / 2 <= 32))
-    { err = "tile_qkv must be even, divide head_dim and fill whole ring slots per half"; return MK_ERR_INVALID_ARG; }
-  if (!(pow2_divides(P.tile_o, H) && P.tile_o % rows_per_slot_h == 0))
+  if (!(pow2_divides(P.tile_qkv, D) && P.tile_qkv % 16 == 0 && (P.tile_qkv / 2) % rows_per_slot_h == 0))
+    { err = "tile_qkv must be a multiple of 16 dividing head_dim, whole ring slots per half"; return MK_ERR_INVALID_ARG; }
+  if (!(pow2_divides(P.tile_o, H) && P.tile_o % rows_per_slot_h == 0 && P.tile_o % 8 == 0))
     { err = "tile_o must divide hidden and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
-  if (!(pow2_divides(P.tile_gu, P.kseg) && P.tile_gu % rows_per_slot_h == 0))
+  if (!(pow2_divides(P.tile_gu, P.kseg) && P.tile_gu % rows_per_slot_h == 0 && P.tile_gu % 8 == 0))
     { err = "tile_gu must divide kseg and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
-  if (!(pow2_divides(P.tile_down, H) && P.tile_down % rows_per_slot_k == 0))
+  if (!(pow2_divides(P.tile_down, H) && P.tile_down % rows_per_slot_k == 0 && P.tile_down % 8 == 0))
     { err = "tile_down must divide hidden and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
-  if (!(P.tile_lm > 0 && P.tile_lm % rows_per_slot_h == 0)) { err = "tile_lm must fill whole ring slots"; return MK_ERR_INVALID_ARG; }
+  if (!(P.tile_lm > 0 && P.tile_lm % rows_per_slot_h == 0 && P.tile_lm % 8 == 0))
+    { err = "tile_lm must be a multiple of 8 filling whole ring slots"; return MK_ERR_INVALID_ARG; }
   if (P.chunk != 64) { err = "attn_chunk must be 64"; return MK_ERR_UNSUPPORTED; }
-  if (P.lm_group < 1) { err = "lm_group must be positive"; return MK_ERR_INVALID_ARG; }
   // a task spans at most 4 ring slots (16 accumulated rows per compute thread)
   if (P.tile_qkv / rows_per_slot_h > 4 || P.tile_o / rows_per_slot_h > 4 || 2 * P.tile_gu / rows_per_slot_h > 4 ||
       P.tile_down / rows_per_slot_k > 4 || ceil_div(P.tile_lm, rows_per_slot_h) > 4)
     { err = "a tile spans more than 4 ring slots"; return MK_ERR_UNSUPPORTED; }
+  // a warp handles at most 8 rows (4 row pairs) of a task
+  if (P.tile_qkv / 2 > 32 || P.tile_o > 64 || P.tile_gu > 32 || P.tile_down > 64 || P.tile_lm > 64)
+    { err = "a tile gives a warp more than 8 rows"; return MK_ERR_UNSUPPORTED; }
   P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
   P.n_otiles = H / P.tile_o;
   P.n_gutiles = F / P.tile_gu;
   P.n_dtiles = H / P.tile_down;
   P.n_kc = F / P.kseg;
   P.n_lm_tiles = ceil_div(P.vocab, P.tile_lm);
-  P.n_lmgrp = ceil_div(P.n_lm_tiles, P.lm_group);
   P.max_chunks = ceil_div(P.max_ctx, P.chunk);
 
   // shared memory: ring of 16 KB slots plus a fixed control area
-  const int reserve = 14 * 1024;  // fixed shared-memory area of the kernel
+  const int reserve = 19 * 1024;  // fixed shared-memory area of the kernel
   P.smem_bytes = smem_bytes;
   P.ring_slots = std::min(16, (smem_bytes - reserve) / P.slot_bytes);
   if (P.ring_slots < 3) { err = "not enough shared memory for a 3-slot ring"; return MK_ERR_UNSUPPORTED; }
@@ -364,18 +357,16 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     add_family(OP_OPROJ, l, emit_const(p.code, P.n_otiles), P.n_otiles, 0);
     add_family(OP_GATEUP, l, emit_const(p.code, P.n_gutiles), P.n_gutiles, 0);
     add_family(OP_DOWN, l, emit_const(p.code, P.n_dtiles * P.n_kc), P.n_dtiles * P.n_kc, 0);
-    add_family(OP_DRED, l, emit_const(p.code, P.n_dtiles), P.n_dtiles, 1);
   }
   add_family(OP_LM, -1, emit_const(p.code, P.n_lm_tiles), P.n_lm_tiles, 0);
-  add_family(OP_LMGRP, -1, emit_const(p.code, P.n_lmgrp), P.n_lmgrp, 1);
   add_family(OP_LMFIN, -1, emit_const(p.code, 1), 1, 1);
   P.n_families = (int)p.fams.size();
-  if (P.n_families > kMaxFamilies) { err = "too many task families"; return MK_ERR_UNSUPPORTED; }
+  if (P.n_families > kMaxFamilies || P.n_layers > 127) { err = "too many task families or layers"; return MK_ERR_UNSUPPORTED; }
   P.debug_slots = debug_base;
   P.fam_stride = kFamPerLayer;
   for (int op = 0; op < OP_COUNT; ++op) P.fam_first_layer[op] = -1;
   for (int k = 0; k < kFamPerLayer; ++k) P.fam_first_layer[kLayerOps[k]] = k;
-  for (int k = 0; k < 3; ++k) P.fam_first_layer[kLmOps[k]] = P.n_layers * kFamPerLayer + k;
+  for (int k = 0; k < 2; ++k) P.fam_first_layer[kLmOps[k]] = P.n_layers * kFamPerLayer + k;
 
   // ---- event tensors (shapes at the symbols' maxima, wait counts symbolic)
   int base = 0;
@@ -387,7 +378,8 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   };
   const int L = P.n_layers;
   const int qkv_per_group = (Hq / Hkv + 2) * (D / P.tile_qkv);
-  add_event(EV_IN, 1, L + 1, 1, 1, Emit(p.code).push(0).coord(0).op(X_LT).push(P.n_dtiles).op(X_MUL).ret());
+  add_event(EV_IN, 1, L + 1, 1, 1,
+            Emit(p.code).push(0).coord(0).op(X_LT).push(P.n_dtiles * P.n_kc).op(X_MUL).ret());
   add_event(EV_QKV, 2, L, Hkv, 1, emit_const(p.code, qkv_per_group));
   add_event(EV_CHUNK, 3, L, P.max_batch, Hkv,
             Emit(p.code).coord(1).op(X_B).op(X_LT).coord(1).op(X_CTX_AT).push(1).op(X_ADD)
@@ -395,16 +387,12 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   add_event(EV_ATTN, 1, L, 1, 1, Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret());
   add_event(EV_O, 1, L, 1, 1, emit_const(p.code, P.n_otiles));
   add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu));
-  add_event(EV_DSUM, 2, L, P.n_dtiles, 1, emit_const(p.code, P.n_kc));
-  add_event(EV_LMG, 1, P.n_lmgrp, 1, 1,
-            Emit(p.code).push(P.lm_group).push(P.n_lm_tiles).coord(0).push(P.lm_group).op(X_MUL)
-                .op(X_SUB).op(X_MIN).ret());
-  add_event(EV_LM, 1, 1, 1, 1, emit_const(p.code, P.n_lmgrp));
+  add_event(EV_LM, 1, 1, 1, 1, emit_const(p.code, P.n_lm_tiles));
   P.n_counters = base;
 
-  // ---- static schedule: per-SM queues of range instructions in topological
-  // (family) order; family f's task i runs on SM (i + rot_f) mod n_sm, with
-  // rot_f continuing the round robin where the previous family stopped.
+  // ---- static schedule: per-SM queues of block instructions in topological
+  // (family) order; SM s takes block v = (s - rot_f) mod n_sm of family f, the
+  // rotation rot_f spreading the blocks that get one task more.
   std::vector<int> regular;
   for (int f = 0; f < P.n_families; ++f)
     if (!p.fams[f].followup) regular.push_back(f);
@@ -417,18 +405,20 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     for (int s = 0; s < n_sm; ++s) {
       Instr& in = p.instr[(size_t)s * P.n_instr_per_sm + k];
       in.family = f;
-      in.start = (int)(((s - rot) % n_sm + n_sm) % n_sm);
-      in.stride = n_sm;
+      in.v = (int)(((s - rot) % n_sm + n_sm) % n_sm);
+      in.n = n_sm;
     }
     rot += p.family_extent(f, typical);
   }
   for (int s = 0; s < n_sm; ++s) {
     Instr& in = p.instr[(size_t)s * P.n_instr_per_sm + regular.size()];
-    in.family = -1; in.start = 0; in.stride = 0;
+    in.family = -1; in.v = 0; in.n = 1;
   }
 
   // ---- dynamic queue capacity: pushes per step at the symbols' maxima
-  P.queue_ranges = L * (2 + Hkv * P.max_batch + P.n_kc) + 8;
+  // per layer: QKV (1), ATTN (one per sequence and kv head), OPROJ (1),
+  // GATEUP (1), DOWN (one per K segment); then LM (1) and END (1)
+  P.queue_ranges = L * (3 + Hkv * P.max_batch + P.n_kc) + 2;
 
   // ---- layer pointers and the rotary table
   p.layers.resize(L);
@@ -473,8 +463,7 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_attn = take(4LL * P.max_batch * P.n_q_heads * P.head_dim);
   P.off_h = take(4LL * P.max_batch * P.ffn);
   P.off_dpart = take(4LL * P.n_kc * P.max_batch * P.hidden);
-  P.off_lmpart = take(8LL * P.max_batch * P.n_lm_tiles);
-  P.off_lmgpart = take(8LL * P.max_batch * P.n_lmgrp);
+  P.off_lmbest = take(8LL * P.max_batch);
   P.ws_bytes = off;
   // image = [off_families, off_queue): the read-only plan arrays
   image.assign((size_t)(P.off_queue - P.off_families), 0);
@@ -603,7 +592,7 @@ struct Sim {
 
   void access(int w, const Region& r, bool write) {
     // shadow units: 4 elements for row data, 1 for per-task records
-    const long long G = (r.buf == BUF_APART || r.buf == BUF_LMPART || r.buf == BUF_LMG || r.buf == BUF_NEXT) ? 1 : 4;
+    const long long G = (r.buf == BUF_APART || r.buf == BUF_NEXT) ? 1 : 4;
     for (long long u = r.lo / G; u <= (r.hi - 1) / G; ++u) {
       Shadow& s = shadow[r.buf][u];
       if (s.reads.empty()) s.reads.assign(nw, 0);
@@ -661,6 +650,7 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
   std::vector<std::vector<Work>> follow(nw);
   std::vector<Work> shared;                   // dynamic queue (FIFO)
   size_t shared_head = 0;
+  int ranges_pushed = 0;                      // queue entries the device would write
   if (!dynamic) {
     // simulated SM w plays the SMs congruent to w mod nw, in queue order
     for (int s = 0; s < P.n_sm; ++s) {
@@ -668,7 +658,9 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
       for (int k = 0; k < P.n_instr_per_sm; ++k) {
         const Instr& in = p.instr[(size_t)s * P.n_instr_per_sm + k];
         if (in.family < 0) break;
-        for (int i = in.start; i < ext[in.family]; i += in.stride) local[w].push_back({in.family, i, {}});
+        int lo, hi;
+        instr_range(in, ext[in.family], lo, hi);
+        for (int i = lo; i < hi; ++i) local[w].push_back({in.family, i, {}});
       }
     }
     for (int w = 0; w < nw; ++w)
@@ -680,6 +672,7 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
       if (sim.counters[ci] == 0) {
         succ.clear();
         p.successors(ci, bd, succ);
+        ranges_pushed += (int)succ.size() / 3;
         for (size_t k = 0; k < succ.size(); k += 3)
           for (int i = 0; i < succ[k + 2]; ++i) shared.push_back({succ[k], succ[k + 1] + i, std::vector<unsigned>(nw, 0)});
       }
@@ -707,6 +700,7 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
         if (dynamic) {
           std::vector<int> succ;
           p.successors(t.notify_ev, bd, succ);
+          ranges_pushed += (int)succ.size() / 3;
           for (size_t k = 0; k < succ.size(); k += 3)
             for (int i = 0; i < succ[k + 2]; ++i) shared.push_back({succ[k], succ[k + 1] + i, me.c});
         }
@@ -743,6 +737,15 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
     } else {
       Work wk = shared[shared_head++];
       exec(w, wk);
+    }
+  }
+  if (dynamic) {
+    ranges_pushed += 1;  // the END range pushed after the last task
+    if (ranges_pushed > P.queue_ranges) {
+      rep->deadlocks++;
+      if (!rep->first_error[0])
+        std::snprintf(rep->first_error, sizeof(rep->first_error), "dynamic queue needs %d ranges, plan reserves %d",
+                      ranges_pushed, P.queue_ranges);
     }
   }
   bool left = false;

@@ -20,7 +20,7 @@ namespace mk {
 // Host-side record of one task for one binding of the symbols.
 enum Buf : int {
   BUF_X = 0, BUF_Q, BUF_KC, BUF_VC, BUF_APART, BUF_ATTN, BUF_H, BUF_DPART,
-  BUF_LMPART, BUF_LMG, BUF_LOGITS, BUF_NEXT, BUF_COUNT
+  BUF_LOGITS, BUF_NEXT, BUF_COUNT
 };
 
 struct Region {

@@ -31,10 +31,10 @@ enum Op : int32_t {
   OP_OPROJ = 4,   // output projection rows + residual
   OP_GATEUP = 5,  // RMSNorm -> gate and up rows -> SwiGLU
   OP_DOWN = 6,    // down projection rows over one K segment -> partial
-  OP_DRED = 7,    // follow-up: sum the K-segment partials into the residual
-  OP_LM = 8,      // final RMSNorm -> vocabulary rows -> logits + tile argmax
-  OP_LMGRP = 9,   // follow-up: argmax over a group of LM tiles
-  OP_LMFIN = 10,  // follow-up: argmax over the groups -> next token
+                  // (7 is unused)
+  OP_LM = 8,      // final RMSNorm -> vocabulary rows -> logits + running argmax
+                  // (9 is unused)
+  OP_LMFIN = 10,  // follow-up: the running argmax -> next token
   OP_COUNT = 11
 };
 
@@ -119,16 +119,14 @@ MK_HD int expr_eval(const int32_t* code, int pc, const ExprEnv& env) {
 // ---------------------------------------------------------------- lowered plan
 // Event-tensor slots of the dense decoder (index into DevPlan::ev).
 enum EvId : int32_t {
-  EV_IN = 0,     // [L+1]        layer input ready (element l+1 notified by layer l's reductions)
+  EV_IN = 0,     // [L+1]        layer input ready (element l+1 notified by layer l's down tiles)
   EV_QKV = 1,    // [L][Hkv]     Q/K/V rows of one kv-head group written
   EV_CHUNK = 2,  // [L][maxB][Hkv] key-chunk partials of one (b, g) written
   EV_ATTN = 3,   // [L]          all head groups merged
   EV_O = 4,      // [L]          output projection done
   EV_GU = 5,     // [L][n_kc]    SwiGLU outputs of one K segment written
-  EV_DSUM = 6,   // [L][n_dtiles] K-segment partials of one row tile written
-  EV_LMG = 7,    // [n_lmgrp]    LM tiles of one group done
-  EV_LM = 8,     // [1]          all LM groups reduced
-  EV_COUNT = 9
+  EV_LM = 6,     // [1]          all LM tiles done
+  EV_COUNT = 7
 };
 
 struct EventTensorDesc {
@@ -148,14 +146,21 @@ struct FamilyDesc {
   int32_t pad[2];
 };
 
-// One static-schedule instruction: run tasks start, start+stride, ... of a
-// family while the index is below the family's evaluated extent.
+// One static-schedule instruction: this SM runs the contiguous block
+// [v*ext/n, (v+1)*ext/n) of a family's tasks, ext being the family's
+// evaluated extent (a contiguous block keeps a CTA's activation registers
+// valid across its tasks).
 struct Instr {
   int32_t family;
-  int32_t start;
-  int32_t stride;
+  int32_t v;  // this SM's virtual index for the family
+  int32_t n;  // number of virtual SMs
   int32_t pad;
 };
+
+MK_HD void instr_range(const Instr& in, int ext, int& lo, int& hi) {
+  lo = (int)(((long long)in.v * ext) / in.n);
+  hi = (int)(((long long)(in.v + 1) * ext) / in.n);
+}
 
 struct LayerPtrs {
   const void* attn_norm; const void* wq; const void* wk; const void* wv; const void* wo;
@@ -172,8 +177,8 @@ struct DevPlan {
   int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
   int32_t max_batch, max_ctx, n_slots;
   float eps;
-  int32_t tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, lm_group, chunk;
-  int32_t n_qkv_tiles, n_otiles, n_gutiles, n_dtiles, n_kc, n_lm_tiles, n_lmgrp, max_chunks;
+  int32_t tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, chunk;
+  int32_t n_qkv_tiles, n_otiles, n_gutiles, n_dtiles, n_kc, n_lm_tiles, max_chunks;
   int32_t ring_slots, slot_bytes, smem_bytes;
   int32_t n_counters, debug_slots, queue_ranges;
   uint32_t debug_flags;
@@ -185,7 +190,7 @@ struct DevPlan {
   int32_t pad1;
   // workspace offsets
   int64_t off_control, off_counters, off_families, off_expr, off_instr, off_layers, off_rope;
-  int64_t off_queue, off_x, off_q, off_apart, off_attn, off_h, off_dpart, off_lmpart, off_lmgpart;
+  int64_t off_queue, off_x, off_q, off_apart, off_attn, off_h, off_dpart, off_lmbest;
   int64_t ws_bytes;
   // global weights (device)
   const void* embed; const void* lm_head; const void* final_norm;

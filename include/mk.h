@@ -51,6 +51,7 @@ typedef int mk_status;
 #define MK_MODEL_DENSE 0     /* dense decoder: attention + SwiGLU FFN per layer */
 
 #define MK_DEBUG_TASK_COUNTS 1u  /* each executed task increments its slot in mk_step_args.task_counts */
+#define MK_DEBUG_TRACE 2u        /* the controller records per-task timestamps in mk_step_args.trace */
 
 /* Per-layer weights of a dense decoder; bf16, row-major [out][in], device. */
 typedef struct mk_layer_weights {
@@ -90,7 +91,7 @@ typedef struct mk_plan_opts {
   int n_sm;               /* CTAs of the persistent kernel; 0 = SMs of the current device */
   int host_only;          /* 1: build without touching a GPU (validation/simulation only) */
   int smem_bytes;         /* dynamic shared memory per CTA; 0 = device opt-in maximum */
-  int tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, lm_group, attn_chunk;
+  int tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, attn_chunk;
   long long spin_timeout_ns; /* device spin-wait limit; 0 = 2 s */
   unsigned debug_flags;   /* MK_DEBUG_* bits */
 } mk_plan_opts;
@@ -106,6 +107,12 @@ typedef struct mk_step_args {
   float* logits;          /* fp32 [B][vocab] or NULL */
   int* next_tokens;       /* int32 [B]: greedy argmax (ties -> lowest id) */
   unsigned* task_counts;  /* uint32 [mk_plan_task_slots()] or NULL; zeroed by the caller */
+  unsigned* trace;        /* uint32 [n_sm][trace_cap][16] or NULL (MK_DEBUG_TRACE): per CTA, record 0
+                             is a header {records, notifier batches, notified tasks, fence ns} and
+                             records 1.. are tasks {family, index, t_pop, t_ready, t_go, t_done,
+                             t_notified, t_compute_start, t_compute_end, t_issue, t_data, 0...};
+                             times are the low 32 bits of %globaltimer in ns */
+  int trace_cap;          /* records per CTA in `trace` */
 } mk_step_args;
 
 typedef struct mk_device_status {
@@ -131,9 +138,7 @@ typedef struct mk_family_info {
 #define MK_OP_OPROJ 4
 #define MK_OP_GATEUP 5
 #define MK_OP_DOWN 6
-#define MK_OP_DRED 7
 #define MK_OP_LM 8
-#define MK_OP_LMGRP 9
 #define MK_OP_LMFIN 10
 
 typedef struct mk_sim_report {
@@ -189,8 +194,8 @@ int mk_plan_num_families(const mk_plan* p);
 mk_status mk_plan_family_info(const mk_plan* p, int family, mk_family_info* out);
 
 /* Tile sizes the plan chose, in this order: tile_qkv, tile_o, tile_gu,
- * tile_down, kseg, tile_lm, lm_group, attn_chunk, n_sm, ring_slots. */
-mk_status mk_plan_tiles(const mk_plan* p, int* out10);
+ * tile_down, kseg, tile_lm, attn_chunk, n_sm, ring_slots. */
+mk_status mk_plan_tiles(const mk_plan* p, int* out9);
 
 /* Host validation for one binding of the symbols (B, ctx_lens host array):
  * every event's wait count equals its number of notifiers, every wait

@@ -17,11 +17,10 @@ Task families of one dense layer, in the order a layer runs them:
 * ``merge``  — one per (b, g): combine that head group's chunk partials;
 * ``oproj``  — one per ``tile_o`` rows of the output projection;
 * ``gateup`` — one per ``tile_gu`` rows of the gate (and the same rows of up);
-* ``down``   — one per (``tile_down`` rows, K segment of ``kseg`` columns);
-* ``dred``   — one per ``tile_down`` rows: sum the K-segment partials.
+* ``down``   — one per (``tile_down`` rows, K segment of ``kseg`` columns).
 
-After the last layer: ``lm`` (``tile_lm`` vocabulary rows each), ``lmgrp``
-(one per ``lm_group`` lm tiles) and ``lmfin`` (one).
+After the last layer: ``lm`` (``tile_lm`` vocabulary rows each) and
+``lmfin`` (one: the greedy token from the LM tiles' running maximum).
 
 Linear index of an ``attn`` task: ``Hkv * sum_{b'<b} nch_{b'} + g * nch_b + c``.
 ``down`` tasks are numbered K-segment-major: ``kc * (H / tile_down) + n``.
@@ -46,9 +45,7 @@ def dense_family_extents(shape, B: int, ctx, tiles: dict) -> dict:
         "oproj": H // tiles["tile_o"],
         "gateup": shape.ffn // tiles["tile_gu"],
         "down": (H // tiles["tile_down"]) * (shape.ffn // tiles["kseg"]),
-        "dred": H // tiles["tile_down"],
         "lm": n_lm,
-        "lmgrp": _ceil(n_lm, tiles["lm_group"]),
         "lmfin": 1,
     }
 
@@ -56,7 +53,7 @@ def dense_family_extents(shape, B: int, ctx, tiles: dict) -> dict:
 def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
     """The set of ``(family, layer, index)`` one decode step runs exactly once.
 
-    Per-layer families carry their layer; ``lm``, ``lmgrp`` and ``lmfin``
+    Per-layer families carry their layer; ``lm`` and ``lmfin``
     carry layer ``-1``.  ``attn`` indices are enumerated from the (b, g, c)
     triples, so the set also pins the linear numbering stated above.
     """
@@ -64,7 +61,7 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
     Hkv = shape.n_kv_heads
     out = set()
     for l in range(shape.n_layers):
-        for fam in ("qkv", "merge", "oproj", "gateup", "down", "dred"):
+        for fam in ("qkv", "merge", "oproj", "gateup", "down"):
             out.update((fam, l, i) for i in range(ext[fam]))
         base = 0
         for b in range(B):
@@ -73,6 +70,6 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
                 for c in range(nch):
                     out.add(("attn", l, Hkv * base + g * nch + c))
             base += nch
-    for fam in ("lm", "lmgrp", "lmfin"):
+    for fam in ("lm", "lmfin"):
         out.update((fam, -1, i) for i in range(ext[fam]))
     return out

@@ -38,7 +38,7 @@ class DenseCase:
     def tiles_for_oracle(self):
         t = self.dec.tiles()
         return dict(tile_qkv=t["tile_qkv"], chunk=t["chunk"], tile_o=t["tile_o"], tile_gu=t["tile_gu"],
-                    tile_down=t["tile_down"], kseg=t["kseg"], tile_lm=t["tile_lm"], lm_group=t["lm_group"])
+                    tile_down=t["tile_down"], kseg=t["kseg"], tile_lm=t["tile_lm"])
 
     def gpu_step(self, tokens, slots, ctx, with_logits=True, counts=True):
         dev = "cuda:0"

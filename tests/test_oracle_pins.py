@@ -395,7 +395,7 @@ def test_moe_skewed_bias_concentrates_routing():
 
 # ---------------------------------------------------------------- task set
 TILES_TINY = dict(tile_qkv=8, chunk=64, tile_o=8, tile_gu=4, tile_down=8, kseg=1024,
-                  tile_lm=16, lm_group=64)
+                  tile_lm=16)
 
 
 def test_task_counts_golden():

@@ -35,13 +35,13 @@ def _host(shape, max_batch=4, max_ctx=320, sched=mk.MK_SCHED_STATIC, n_sm=16, **
 def test_plan_build_and_tiles():
     d = _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148)
     t = d.tiles()
-    assert t["tile_qkv"] == 8 and t["tile_o"] == 8 and t["tile_gu"] == 4 and t["tile_down"] == 8
+    assert t["tile_qkv"] == 16 and t["tile_o"] == 8 and t["tile_gu"] == 8 and t["tile_down"] == 8
     assert t["kseg"] == 2048 and t["tile_lm"] == 16 and t["chunk"] == 64 and t["n_sm"] == 148
     fams = d.families()
-    assert len(fams) == 16 * 7 + 3
-    assert [f.name.decode() for f in fams[:7]] == ["qkv.0", "attn.0", "merge.0", "oproj.0", "gateup.0",
-                                                   "down.0", "dred.0"]
-    assert sum(f.followup for f in fams) == 16 * 2 + 2
+    assert len(fams) == 16 * 6 + 2
+    assert [f.name.decode() for f in fams[:6]] == ["qkv.0", "attn.0", "merge.0", "oproj.0", "gateup.0",
+                                                   "down.0"]
+    assert sum(f.followup for f in fams) == 16 + 1
 
 
 def test_plan_rejects_bad_shapes():
@@ -50,7 +50,7 @@ def test_plan_rejects_bad_shapes():
         _host(bad)
     assert e.value.status in (mk._abi.MK_ERR_UNSUPPORTED, mk._abi.MK_ERR_INVALID_ARG)
     with pytest.raises(mk.MkError):
-        _host(wl.TINY, tile_qkv=6)
+        _host(wl.TINY, tile_qkv=24)
     with pytest.raises(mk.MkError):
         _host(wl.TINY, max_batch=9)
 
@@ -81,8 +81,9 @@ def test_simulator_clean(sched, B, ctx):
     assert code == 0, rep.first_error
     assert rep.races == 0 and rep.deadlocks == 0 and rep.exactly_once_violations == 0
     assert rep.nonzero_counters == 0 and rep.static_dynamic_mismatch == 0
-    tiles = dict(tile_qkv=64, chunk=64, tile_o=64, tile_gu=32, tile_down=16, kseg=1024, tile_lm=128,
-                 lm_group=64)
+    t = d.tiles()
+    tiles = {k: t[k] for k in ("tile_qkv", "chunk", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm")}
+    assert tiles == dict(tile_qkv=64, chunk=64, tile_o=32, tile_gu=32, tile_down=8, kseg=1024, tile_lm=32)
     assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, tiles))
 
 
@@ -113,3 +114,14 @@ def test_fault_missing_wait_is_a_race(fam):
     d = _host(wl.TINY, n_sm=8)
     code, rep = mk.mk_plan_simulate(d.plan, 2, [10, 100], 20, 3, mk.MK_SIM_FAULT_NO_WAIT, _family(d, fam))
     assert code != 0 and rep.races > 0, rep.first_error
+
+
+def test_dynamic_queue_capacity_deep_model():
+    # 16 layers: the per-layer queue pushes add up; the simulator checks the
+    # plan's reserved range count against the pushes of a full step
+    deep = wl.DenseShape(n_layers=16, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=1024,
+                         vocab=1024)
+    d = _host(deep, max_batch=2, sched=mk.MK_SCHED_DYNAMIC, n_sm=8)
+    for B, ctx in [(1, [64]), (2, [300, 5])]:
+        code, rep = mk.mk_plan_simulate(d.plan, B, ctx, n_orders=4, seed=5)
+        assert code == 0, rep.first_error
