@@ -102,7 +102,7 @@ static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, fifo_full) % 8 == 
 constexpr int BAR_COMP = 3;  // named barrier of the 8 compute warps
 
 // ---------------------------------------------------------------- errors
-__device__ void record_error(Control* ctl, int code, int fam, int idx, int ev) {
+__device__ __noinline__ void record_error(Control* ctl, int code, int fam, int idx, int ev) {
   if (atomicCAS(&ctl->status_code, 0, code) == 0) {
     ctl->status_family = fam;
     ctl->status_index = idx;
@@ -114,8 +114,10 @@ __device__ void record_error(Control* ctl, int code, int fam, int idx, int ev) {
 
 __device__ __forceinline__ bool aborted(Control* ctl) { return *(volatile int*)&ctl->abort != 0; }
 
-// Bounded wait on an mbarrier phase; false if the kernel is aborting.
-__device__ bool wait_mbar(uint64_t* bar, uint32_t parity, Control* ctl, long long timeout_ns, int fam, int idx) {
+// Bounded wait on an mbarrier phase; false if the kernel is aborting.  Inline
+// (no call on the hot path: a call would save the caller's live registers).
+__device__ __forceinline__ bool wait_mbar(uint64_t* bar, uint32_t parity, Control* ctl, long long timeout_ns, int fam,
+                                          int idx) {
   if (mbar_try(bar, parity)) return true;
   unsigned long long t0 = global_ns();
   for (int it = 0;; ++it) {
@@ -769,7 +771,8 @@ __device__ void controller(const DevPlan& P, const StepParams& S, Smem& sm, unsi
 // ---------------------------------------------------------------- compute
 struct GemvSpec {
   int kind;           // 0: RMSNorm(x) * gamma, 1: attention output, 2: SwiGLU segment
-  const void* gamma;  // RMSNorm gain (kind 0)
+  int gamma_sel;      // kind 0: 0 attention-norm gain of `layer`, 1 FFN-norm gain, 2 final-norm gain
+  int layer;
   int kc;             // K segment (kind 2)
   int K;              // columns
   bool parts;         // kind 0: add the previous layer's down-projection partials to x
@@ -777,23 +780,23 @@ struct GemvSpec {
   int rows;           // valid rows of the task
 };
 
-__device__ __forceinline__ bool gemv_spec(const DevPlan& P, const LayerPtrs* layers, const TaskDesc& d, GemvSpec& g) {
-  g.gamma = nullptr; g.kc = 0; g.parts = false; g.K = P.hidden;
+__device__ __forceinline__ bool gemv_spec(const DevPlan& P, const TaskDesc& d, GemvSpec& g) {
+  g.gamma_sel = 0; g.layer = d.layer; g.kc = 0; g.parts = false; g.K = P.hidden;
   switch (d.op) {
     case OP_QKV:
-      g.kind = 0; g.gamma = layers[d.layer].attn_norm; g.parts = d.layer > 0; g.tag = d.layer * 64; g.rows = P.tile_qkv;
+      g.kind = 0; g.gamma_sel = 0; g.parts = d.layer > 0; g.tag = d.layer * 64; g.rows = P.tile_qkv;
       return true;
     case OP_OPROJ:
       g.kind = 1; g.tag = d.layer * 64 + 1; g.rows = P.tile_o;
       return true;
     case OP_GATEUP:
-      g.kind = 0; g.gamma = layers[d.layer].ffn_norm; g.tag = d.layer * 64 + 2; g.rows = 2 * P.tile_gu;
+      g.kind = 0; g.gamma_sel = 1; g.tag = d.layer * 64 + 2; g.rows = 2 * P.tile_gu;
       return true;
     case OP_DOWN:
       g.kind = 2; g.kc = d.idx / P.n_dtiles; g.K = P.kseg; g.tag = d.layer * 64 + 8 + g.kc; g.rows = P.tile_down;
       return true;
     case OP_LM:
-      g.kind = 0; g.gamma = P.final_norm; g.parts = true; g.tag = 60 * 64;
+      g.kind = 0; g.gamma_sel = 2; g.parts = true; g.tag = 60 * 64;
       g.rows = min(P.tile_lm, P.vocab - d.idx * P.tile_lm);
       return true;
     default:
@@ -814,6 +817,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // in place.  Called by all compute warps for the same task (the tag sequence
 // is the same for all warps).
 __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int b) {
+  const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int K = g.K;
   const float* src;
@@ -862,7 +866,9 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
 #pragma unroll
     for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[q];
     const float inv = 1.0f / sqrtf(tot / (float)K + P.eps);
-    const uint4* gam = reinterpret_cast<const uint4*>(g.gamma);
+    const void* gp = g.gamma_sel == 2 ? P.final_norm
+                                      : (g.gamma_sel == 1 ? layers[g.layer].ffn_norm : layers[g.layer].attn_norm);
+    const uint4* gam = reinterpret_cast<const uint4*>(gp);
     for (int c = ct * 8; c < K; c += kComputeThreads * 8) {
       float gf[8];
       bf16x8_to_f32(__ldg(gam + c / 8), gf);
@@ -988,6 +994,23 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
       }
     }
   }
+  if (d.op == OP_OPROJ) {
+    // residual: x = (x + previous layer's down partials) + o W_o^T; lane 0
+    // reads x, lanes 1..n_kc the partials, in one round trip
+    float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
+    const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
+    const int nq = d.layer > 0 ? P.n_kc : 0;
+#pragma unroll 1
+    for (int k = 0; k < nr; ++k) {
+      const size_t col = (size_t)d.idx * P.tile_o + row_of(k);
+      float v = 0.f;
+      if (lane == 0) v = __ldcg(x + col);
+      else if (lane <= nq) v = __ldcg(dp + ((size_t)(lane - 1) * P.max_batch + b) * H + col);
+      v = warp_sum(v);
+      if (lane == 0) x[col] = v + y[k];
+    }
+    return;
+  }
   if (lane != 0) return;
   switch (d.op) {
     case OP_QKV: {
@@ -1029,20 +1052,6 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
         if (k >= npair) break;
         const float gt = y[k], up = y[npair + k];
         h[row_of(k)] = gt / (1.0f + expf(-gt)) * up;
-      }
-    } break;
-    case OP_OPROJ: {
-      // residual: x = (x + previous layer's down partials) + o W_o^T
-      float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
-      const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (k >= nr) break;
-        const size_t col = (size_t)d.idx * P.tile_o + row_of(k);
-        float xv = __ldcg(x + col);
-        if (d.layer > 0)
-          for (int q = 0; q < P.n_kc; ++q) xv += __ldcg(dp + ((size_t)q * P.max_batch + b) * H + col);
-        x[col] = xv + y[k];
       }
     } break;
     case OP_DOWN: {
@@ -1194,7 +1203,6 @@ __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S
 __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
                         Control* ctl) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int B = S.B;
   int a_tag = -1;
   ActRegs av;
@@ -1206,7 +1214,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     uint32_t* trec = (d.rec > 0 && w == 0) ? trace_rec(S, d.rec) : nullptr;
     if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
     GemvSpec g;
-    if (gemv_spec(P, layers, d, g)) {
+    if (gemv_spec(P, d, g)) {
       TaskSlots ts;
       task_slots_of(P, d, ts);
       // one pass per batch row (the activation is restaged each pass when
