@@ -1391,6 +1391,10 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
   if (e == cudaSuccess)
     e = cudaMemcpyAsync((unsigned char*)ws + p.dp.off_families, image.data(), image.size(), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync((unsigned char*)ws + p.dp.off_control, 0, sizeof(Control), s);
+  // a queue entry counts as published when its tag equals the launch epoch, and
+  // epochs restart at 1 here: clear whatever the memory held before
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync((unsigned char*)ws + p.dp.off_queue, 0, sizeof(QRange) * (size_t)p.dp.queue_ranges, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) { err = std::string("bind failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   p.dp.smem_bytes = (int)smem;
@@ -1436,6 +1440,10 @@ mk_status dev_status(Plan& p, mk_device_status* st, std::string& err) {
 
 mk_status dev_reset(Plan& p, void* stream, std::string& err) {
   cudaError_t e = cudaMemsetAsync((unsigned char*)p.ws + p.dp.off_control, 0, sizeof(Control), (cudaStream_t)stream);
+  // epochs restart at 1: entries tagged by the old epochs must not read as published
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync((unsigned char*)p.ws + p.dp.off_queue, 0, sizeof(QRange) * (size_t)p.dp.queue_ranges,
+                        (cudaStream_t)stream);
   if (e != cudaSuccess) { err = std::string("reset failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   p.epoch = 0;
   return MK_OK;

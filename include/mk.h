@@ -185,7 +185,8 @@ mk_status mk_decode_step(mk_plan* p, const mk_step_args* a, void* stream);
  * device code (MK_OK if none).  After a device error, call mk_plan_reset. */
 mk_status mk_get_status(mk_plan* p, mk_device_status* st);
 
-/* Clear the device control block (status, barrier and queue counters). */
+/* Clear the device control block (status, barrier and queue counters) and the
+ * dynamic queue's entries. */
 mk_status mk_plan_reset(mk_plan* p, void* stream);
 
 /* Task-count slots of the debug counter array (mk_step_args.task_counts). */

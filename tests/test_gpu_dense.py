@@ -71,6 +71,21 @@ def test_tiny_static_equals_dynamic_bitwise(tiny):
     dyn.check_task_set(b["task_counts"], 3, ctx)
 
 
+def test_tiny_dynamic_steps_after_reset(tiny):
+    # a reset restarts the launch epochs; queue entries tagged by the epochs
+    # before it must not be taken for entries of the steps after it
+    dyn = DenseCase(wl.TINY, max_batch=4, max_ctx=320, n_slots=4, ctx_fill=[64, 0, 70, 190],
+                    sched=mk.MK_SCHED_DYNAMIC)
+    tokens, slots, ctx = [3, 900, 511], [1, 2, 3], [0, 70, 190]
+    ref, _, _ = _oracle_step(dyn, tokens, slots, ctx)
+    for rnd in range(2):
+        for i in range(4):
+            got = dyn.gpu_step(tokens, slots, ctx)
+            assert rel_err(got["logits"], ref["logits"]) <= TOL
+            dyn.check_task_set(got["task_counts"], 3, ctx)
+        dyn.dec.reset()
+
+
 def test_tiny_greedy_walk(tiny):
     # greedy decode; both sides continue from the oracle's token
     tok, pos = 42, 64
