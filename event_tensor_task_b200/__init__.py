@@ -11,7 +11,8 @@ from __future__ import annotations
 import ctypes as C
 
 from . import _abi
-from ._abi import (MK_OK, MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS, MK_DEBUG_TRACE,
+from ._abi import (MK_OK, MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_STATIC_SCRATCH_BYTES,
+                   MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS, MK_DEBUG_TRACE,
                    MK_SIM_FAULT_NONE, MK_SIM_FAULT_DROP_NOTIFY, MK_SIM_FAULT_COUNT_PLUS_ONE,
                    MK_SIM_FAULT_NO_WAIT, OP_NAMES, mk_model_desc, mk_plan_opts, mk_step_args,
                    mk_layer_weights, mk_device_status, mk_family_info, mk_sim_report)
@@ -64,6 +65,10 @@ def mk_plan_bind_workspace(plan: int, dev_ptr: int, nbytes: int, stream: int = 0
 
 def mk_decode_step(plan: int, args: mk_step_args, stream: int = 0):
     _check(lib().mk_decode_step(plan, C.byref(args), stream))
+
+
+def mk_decode_step_static(plan: int, args: mk_step_args, stream: int = 0):
+    _check(lib().mk_decode_step_static(plan, C.byref(args), stream))
 
 
 def mk_get_status(plan: int):
@@ -131,11 +136,13 @@ class DenseDecoder:
     w_gate,w_up,w_down}`` (and ``lm_head`` when untied) to bf16 tensors on the
     device.  ``k_cache``/``v_cache`` are bf16 ``[L][slots][Hkv][max_ctx][64]``.
     With ``host_only`` no GPU is touched (plan validation and simulation only).
+    With ``workspace=False`` the plan gets no workspace and steps only through
+    ``step(..., static_scratch=True)`` (mk_decode_step_static).
     """
 
     def __init__(self, shape, weights=None, k_cache=None, v_cache=None, max_batch=1, max_ctx=None,
                  n_slots=None, sched=MK_SCHED_STATIC, n_sm=0, host_only=False, debug=False,
-                 spin_timeout_ns=0, trace=False, **tiles):
+                 spin_timeout_ns=0, trace=False, workspace=True, **tiles):
         import torch
         self.shape = shape
         w = weights or {}
@@ -170,7 +177,7 @@ class DenseDecoder:
         self.desc, self.opts = d, o
         self.plan = mk_plan_build(d, o)
         self.ws = None
-        if not host_only:
+        if not host_only and workspace:
             nbytes = mk_plan_workspace_bytes(self.plan)
             self.ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=k_cache.device)
             base = (_ptr(self.ws) + 255) // 256 * 256
@@ -183,8 +190,9 @@ class DenseDecoder:
         return mk_plan_tiles(self.plan)
 
     def step(self, token_ids, slot_ids, ctx_lens, next_tokens, logits=None, task_counts=None, stream=None,
-             trace=None):
-        """One decode step on ``stream`` (default: torch's current stream)."""
+             trace=None, static_scratch=False):
+        """One decode step on ``stream`` (default: torch's current stream);
+        through mk_decode_step_static when ``static_scratch``."""
         import torch
         a = mk_step_args()
         if trace is not None:
@@ -193,7 +201,7 @@ class DenseDecoder:
         a.token_ids, a.slot_ids, a.ctx_lens = _ptr(token_ids), _ptr(slot_ids), _ptr(ctx_lens)
         a.logits, a.next_tokens, a.task_counts = _ptr(logits), _ptr(next_tokens), _ptr(task_counts)
         s = stream if stream is not None else torch.cuda.current_stream()
-        mk_decode_step(self.plan, a, s.cuda_stream)
+        (mk_decode_step_static if static_scratch else mk_decode_step)(self.plan, a, s.cuda_stream)
 
     def status(self):
         return mk_get_status(self.plan)

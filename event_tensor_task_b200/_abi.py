@@ -22,6 +22,7 @@ MK_SCHED_DYNAMIC = 1
 MK_MODEL_DENSE = 0
 MK_DEBUG_TASK_COUNTS = 1
 MK_DEBUG_TRACE = 2
+MK_STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 MK_SIM_FAULT_NONE = 0
 MK_SIM_FAULT_DROP_NOTIFY = 1
@@ -86,6 +87,7 @@ PROTOTYPES = {
     "mk_plan_workspace_bytes": (C.c_size_t, [C.c_void_p]),
     "mk_plan_bind_workspace": (C.c_int, [C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "mk_decode_step": (C.c_int, [C.c_void_p, C.POINTER(mk_step_args), C.c_void_p]),
+    "mk_decode_step_static": (C.c_int, [C.c_void_p, C.POINTER(mk_step_args), C.c_void_p]),
     "mk_get_status": (C.c_int, [C.c_void_p, C.POINTER(mk_device_status)]),
     "mk_plan_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
     "mk_plan_task_slots": (C.c_int, [C.c_void_p]),

@@ -1,6 +1,7 @@
 // api.cpp — the extern "C" boundary of libmk.so (declared in include/mk.h).
 // No exception crosses it; every failure returns an mk_status and leaves a
 // message for mk_last_error().
+#include <atomic>
 #include <cstring>
 #include <new>
 #include <string>
@@ -63,7 +64,9 @@ mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_pla
       delete hp;
       return fail(s, err);
     }
+    static std::atomic<unsigned long long> next_uid{1};
     hp->p.device = device;
+    hp->p.uid = next_uid++;
     *out = hp;
     return MK_OK;
   } catch (const std::bad_alloc&) {
@@ -106,6 +109,26 @@ mk_status mk_decode_step(mk_plan* hp, const mk_step_args* a, void* stream) {
   std::string err;
   mk_status s = mk::dev_launch(hp->p, a, stream, err);
   return s == MK_OK ? MK_OK : fail(s, err);
+}
+
+mk_status mk_decode_step_static(mk_plan* hp, const mk_step_args* a, void* stream) {
+  g_err.clear();
+  if (!hp || !a) return fail(MK_ERR_INVALID_ARG, "null argument");
+  if (hp->p.device < 0) return fail(MK_ERR_UNSUPPORTED, "plan was built host_only");
+  if (a->batch < 1 || a->batch > hp->p.dp.max_batch) return fail(MK_ERR_INVALID_ARG, "batch out of [1, max_batch]");
+  if (!a->token_ids || !a->slot_ids || !a->ctx_lens || !a->next_tokens)
+    return fail(MK_ERR_INVALID_ARG, "token_ids, slot_ids, ctx_lens and next_tokens are required");
+  if ((unsigned long long)hp->p.dp.ws_bytes > (unsigned long long)MK_STATIC_SCRATCH_BYTES)
+    return fail(MK_ERR_WORKSPACE, "plan needs " + std::to_string(hp->p.dp.ws_bytes) +
+                                      " bytes of scratch; the static scratch holds " +
+                                      std::to_string((unsigned long long)MK_STATIC_SCRATCH_BYTES));
+  try {
+    std::string err;
+    mk_status s = mk::dev_launch_static(hp->p, a, stream, err);
+    return s == MK_OK ? MK_OK : fail(s, err);
+  } catch (...) {
+    return fail(MK_ERR_CUDA, "unexpected error in the static-scratch decode step");
+  }
 }
 
 mk_status mk_get_status(mk_plan* hp, mk_device_status* st) {

@@ -34,6 +34,7 @@
 #include <cuda_runtime.h>
 
 #include <cstddef>
+#include <mutex>
 
 #include "../../include/mk.h"
 #include "device.cuh"
@@ -1423,6 +1424,100 @@ mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& 
   if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   p.epoch++;
   p.launches++;
+  return MK_OK;
+}
+
+// ---------------------------------------------------------------- static scratch
+// Scratch of mk_decode_step_static: a module-scope device array, so that the
+// step needs no device allocation at all.  Each CUDA context (one per device)
+// holds its own copy of it.  The array is shared by every plan and call on the
+// device and keeps the last call's contents; g_static records whose plan
+// arrays it holds, so they are uploaded again only when the plan changes.
+static __device__ __align__(256) unsigned char g_static_scratch[MK_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxStaticDevices = 64;
+struct StaticScratchState {
+  unsigned char* addr = nullptr;  // device address of g_static_scratch in this device's context
+  unsigned long long owner = 0;   // uid of the plan whose arrays it holds (0: none)
+};
+std::mutex g_static_mu;
+StaticScratchState g_static[kMaxStaticDevices];
+}  // namespace
+
+mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::string& err) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) { err = std::string("cudaGetDevice failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
+  if (dev != p.device) { err = "the current device is not the one the plan was built on"; return MK_ERR_INVALID_ARG; }
+  if (dev < 0 || dev >= kMaxStaticDevices) { err = "device ordinal beyond the static-scratch table"; return MK_ERR_UNSUPPORTED; }
+  const DevPlan& P0 = p.dp;
+  if ((unsigned long long)P0.ws_bytes > (unsigned long long)MK_STATIC_SCRATCH_BYTES) {
+    err = "plan scratch exceeds MK_STATIC_SCRATCH_BYTES";
+    return MK_ERR_WORKSPACE;
+  }
+  // the plan arrays below are exactly what the workspace image holds
+  const long long rope_end = P0.off_rope + (4LL * (long long)p.rope.size() + 255) / 256 * 256;
+  if (rope_end != P0.off_queue) { err = "plan arrays do not match the workspace layout"; return MK_ERR_PLAN; }
+
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  StaticScratchState& st = g_static[dev];
+  if (!st.addr) {
+    // first call on this device: resolve the array's address with the device current
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess) {
+      err = std::string("cudaGetSymbolAddress of the static scratch failed: ") + cudaGetErrorString(e);
+      return MK_ERR_CUDA;
+    }
+    st.addr = static_cast<unsigned char*>(ptr);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned char* ws = st.addr;
+  const size_t smem = (size_t)P0.ring_slots * P0.slot_bytes + sizeof(Smem);
+  if (st.owner != p.uid) {
+    st.owner = 0;
+    e = cudaFuncSetAttribute(megakernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) {
+      int nb = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, megakernel, kThreads, smem);
+      if (e == cudaSuccess && nb < 1) { err = "megakernel does not fit on an SM"; return MK_ERR_UNSUPPORTED; }
+    }
+    // the read-only plan arrays, copied from the plan's own host vectors
+    auto put = [&](long long off, const void* src, size_t n) {
+      if (e == cudaSuccess && n) e = cudaMemcpyAsync(ws + off, src, n, cudaMemcpyHostToDevice, s);
+    };
+    put(P0.off_families, p.fams.data(), sizeof(FamilyDesc) * p.fams.size());
+    put(P0.off_expr, p.code.data(), 4 * p.code.size());
+    put(P0.off_instr, p.instr.data(), sizeof(Instr) * p.instr.size());
+    put(P0.off_layers, p.layers.data(), sizeof(LayerPtrs) * p.layers.size());
+    put(P0.off_rope, p.rope.data(), 4 * p.rope.size());
+    if (e != cudaSuccess) { err = std::string("plan upload failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
+    st.owner = p.uid;
+  }
+  // every call starts at epoch 1 from a cleared control block and queue; the
+  // counters, activations and argmax keys are set by the kernel's prologue
+  e = cudaMemsetAsync(ws + P0.off_control, 0, sizeof(Control), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws + P0.off_queue, 0, sizeof(QRange) * (size_t)P0.queue_ranges, s);
+  if (e != cudaSuccess) { err = std::string("scratch clear failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
+
+  StepParams sp;
+  sp.B = a->batch;
+  sp.tokens = a->token_ids;
+  sp.slots = a->slot_ids;
+  sp.ctx = a->ctx_lens;
+  sp.logits = a->logits;
+  sp.next_tokens = a->next_tokens;
+  sp.task_counts = a->task_counts;
+  sp.trace = (P0.debug_flags & MK_DEBUG_TRACE) ? (uint32_t*)a->trace : nullptr;
+  sp.trace_cap = a->trace_cap;
+  if (sp.trace && sp.trace_cap < 2) sp.trace = nullptr;
+  sp.epoch = 1;
+  DevPlan dp = P0;
+  dp.smem_bytes = (int)smem;
+  void* args[] = {(void*)&dp, (void*)&sp, (void*)&ws};
+  e = cudaLaunchCooperativeKernel((const void*)megakernel, dim3(dp.n_sm), dim3(kThreads), args, smem, s);
+  if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   return MK_OK;
 }
 

@@ -55,6 +55,7 @@ struct Plan {
   std::vector<LayerPtrs> layers;
   std::vector<float> rope;          // [max_ctx][head_dim/2][2] cos, sin
   int device = -1;
+  unsigned long long uid = 0;       // unique per plan built in this process
   void* ws = nullptr;
   size_t ws_bound = 0;
   unsigned epoch = 0;

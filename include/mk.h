@@ -181,6 +181,38 @@ mk_status mk_plan_bind_workspace(mk_plan* p, void* dev_ptr, size_t bytes, void* 
  * are read with mk_get_status after the stream has synchronised. */
 mk_status mk_decode_step(mk_plan* p, const mk_step_args* a, void* stream);
 
+/* Largest plan scratch (mk_plan_workspace_bytes) that mk_decode_step_static
+ * serves: 8 MiB, enough for the 16-layer, 2048-wide model at max_batch 4 and
+ * max_ctx 8192 (6.7 MiB).  The array is part of libmk.so's device image, so
+ * every process that loads the library holds it on each device it uses. */
+#define MK_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/* mk_decode_step with no workspace and no device allocation.  The Event
+ * Tensor pages have no counterpart of this call: it exists for callers that
+ * cannot allocate device memory or hand out a workspace, for instance a
+ * serving engine that gives all free HBM to its KV-cache pool at start-up and
+ * forbids allocation afterwards, or a plain C host program with no device
+ * allocator.  The scratch is a module-scope `__device__` array of
+ * MK_STATIC_SCRATCH_BYTES (256-byte aligned), one per device.
+ *  - The plan must have been built on the current device (not host_only); a
+ *    plan needing more scratch than MK_STATIC_SCRATCH_BYTES is rejected with
+ *    MK_ERR_WORKSPACE.  mk_plan_bind_workspace is not needed.
+ *  - The first call on a device resolves the array's address with
+ *    cudaGetSymbolAddress (which may load the module), and the first call
+ *    with a plan uploads that plan's arrays with cudaMemcpyAsync from host
+ *    memory: make both before any stream capture.  No graph capture of this
+ *    call is supported.
+ *  - The array is shared by every plan and every call on the device and keeps
+ *    the last call's contents; each call clears the control block and task
+ *    queue (cudaMemsetAsync) and starts at launch epoch 1.  Calls that overlap
+ *    on the device (other streams, other host threads' streams) race on it.
+ *  - Device-side errors are not reported: the control block holding them is
+ *    cleared by the next call.  A step stopped by one before its last task
+ *    leaves next_tokens unwritten; run the step through mk_decode_step with a
+ *    workspace to read the code with mk_get_status.
+ * Arguments and launch errors as for mk_decode_step. */
+mk_status mk_decode_step_static(mk_plan* p, const mk_step_args* a, void* stream);
+
 /* Read the device status word (synchronous copy).  Returns the recorded
  * device code (MK_OK if none).  After a device error, call mk_plan_reset. */
 mk_status mk_get_status(mk_plan* p, mk_device_status* st);
