@@ -74,6 +74,10 @@ struct TaskDesc {
   uint32_t t_issue;  // trace: when the producer queued the task (low 32 bits of ns)
 };
 
+// batch rows the per-CTA sequence tables hold (the kernel runs B <= kMaxB)
+constexpr int kSmemBatch = 64;
+static_assert(kMaxB <= kSmemBatch, "sequence tables too small");
+
 struct Smem {
   uint64_t full[kMaxSlots], empty[kMaxSlots];
   uint64_t go_bar[2];    // controller -> compute: task k is in cur[k & 1] (count 1)
@@ -83,13 +87,14 @@ struct Smem {
   TaskDesc cur[2];
   TaskDesc doneq[kDoneQ];
   TaskDesc followq[kFollowQ];
-  int ctx[kMaxBatch], slot[kMaxBatch], tok[kMaxBatch], nch[kMaxBatch], pre[kMaxBatch + 1];
+  int ctx[kSmemBatch], slot[kSmemBatch], tok[kSmemBatch], nch[kSmemBatch], pre[kSmemBatch + 1];
   int fam_ext[kMaxFamilies];
   signed char fam_op[kMaxFamilies], fam_layer[kMaxFamilies];
   // activation staging: one batch row, loaded once per CTA for all warps
   alignas(16) float xs[2048];  // read and written as float4
   float red8[kComputeWarps];
   float yw[kComputeWarps][8];  // a warp's row results of the current task
+  unsigned long long lm_seen[kComputeWarps][kMaxB];  // per compute warp: best argmax key it has published
   uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
   // attention scratch, one row per head warp
   float qs[4][64], ps[4][64], newk[4][64], newv[4][64];
@@ -504,18 +509,26 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     unsigned long long tf0 = trace ? global_ns() : 0;
     asm volatile("fence.acq_rel.gpu;" ::: "memory");
     if (trace) { fence_ns += global_ns() - tf0; n_batches++; }
-    int old = 0;
-    if (lane < n && ni.ctr >= 0 && ni.need_old) {
-      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], -1;" : "=r"(old) : "l"(counters + ni.ctr) : "memory");
+    // one atomic per distinct counter of the batch: the lowest lane of each
+    // group subtracts the group's size; when the old value is needed, the
+    // counter reached zero iff it equalled that size (the follow-up and the
+    // successors depend on the counter only, so the leader's task stands for
+    // the group)
+    const int key = (lane < n && ni.ctr >= 0) ? ni.ctr : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    const bool leader = key >= 0 && lane == __ffs(peers) - 1;
+    const int cnt = __popc(peers);
+    bool fired = false;
+    if (leader) {
+      if (ni.need_old) {
+        int old;
+        asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(counters + key), "r"(-cnt) : "memory");
+        if (old < cnt) record_error(ctl, MK_ERR_DEVICE_BOUNDS, t.fam, t.idx, key);
+        fired = old == cnt;
+      } else {
+        asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(counters + key), "r"(-cnt) : "memory");
+      }
     }
-    int key = (lane < n && ni.ctr >= 0 && !ni.need_old) ? ni.ctr : -1 - lane;
-    unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (key >= 0 && lane == __ffs(peers) - 1) {
-      int cnt = __popc(peers);
-      asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(counters + key), "r"(-cnt) : "memory");
-    }
-    if (lane < n && ni.need_old && old <= 0) record_error(ctl, MK_ERR_DEVICE_BOUNDS, t.fam, t.idx, ni.ctr);
-    const bool fired = lane < n && ni.need_old && old == 1;
     if (fired && P.sched == MK_SCHED_DYNAMIC) push_successors(P, S, sm, ctl, ws, t);
     if (lane < n && t.op == OP_LMFIN && P.sched == MK_SCHED_DYNAMIC)
       push_range(P, S, ctl, ws, -1, 0, P.n_sm);  // one END per CTA
@@ -924,19 +937,22 @@ __device__ __forceinline__ float warp_dot(const unsigned char* rowp, int nblk, c
 }
 
 // Ring position of the task's slots.
+// The ring slots of a task: consecutive from the slot of its first copy,
+// wrapping (with a parity flip) at the end of the ring.  Kept as a base slot
+// and parity rather than per-slot arrays, so that nothing indexed by a run-time
+// slot number has to live in local memory.
 struct TaskSlots {
-  int n;
-  int idx[4];
-  uint32_t par[4];
+  int n, s0, R;
+  uint32_t p0;
+  __device__ __forceinline__ int idx(int j) const { return s0 + j < R ? s0 + j : s0 + j - R; }
+  __device__ __forceinline__ uint32_t par(int j) const { return s0 + j < R ? p0 : p0 ^ 1u; }
 };
 __device__ __forceinline__ void task_slots_of(const DevPlan& P, const TaskDesc& d, TaskSlots& ts) {
+  const uint32_t q = (uint32_t)d.ring_seq;
   ts.n = d.nslots;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint32_t q = (uint32_t)d.ring_seq + j;
-    ts.idx[j] = (int)(q % (uint32_t)P.ring_slots);
-    ts.par[j] = (q / (uint32_t)P.ring_slots) & 1;
-  }
+  ts.R = P.ring_slots;
+  ts.s0 = (int)(q % (uint32_t)P.ring_slots);
+  ts.p0 = (q / (uint32_t)P.ring_slots) & 1;
 }
 
 // One warp's share of a GEMV task for batch row b: whole rows (or
@@ -971,7 +987,7 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
     for (int k = 0; k < 8; ++k)
       if (k < nr) mine |= 1u << (row_of(k) >> lg);
     for (int j = 0; j < ts.n; ++j)
-      if (!(mine & (1u << j))) mbar_arrive(&sm.empty[ts.idx[j]]);
+      if (!(mine & (1u << j))) mbar_arrive(&sm.empty[ts.idx(j)]);
   }
   float* y = sm.yw[w];
 #pragma unroll 1
@@ -979,19 +995,19 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
     if (k < nr) {
       const int r = row_of(k), js = r >> lg;
       if (!(ready & (1u << js))) {
-        wait_mbar(&sm.full[ts.idx[js]], ts.par[js], ctl, P.spin_timeout_ns, d.fam, d.idx);
+        wait_mbar(&sm.full[ts.idx(js)], ts.par(js), ctl, P.spin_timeout_ns, d.fam, d.idx);
         ready |= 1u << js;
         if (js == 0 && trec && lane == 0) {
           trec[TR_DATA] = (uint32_t)global_ns();
-          trec[TR_ISSUE] = sm.slot_t[ts.idx[0]];
+          trec[TR_ISSUE] = sm.slot_t[ts.idx(0)];
         }
       }
-      const float yk = warp_dot(ring + (size_t)ts.idx[js] * P.slot_bytes + (size_t)(r & (rps - 1)) * K * 2, nblk, av);
+      const float yk = warp_dot(ring + (size_t)ts.idx(js) * P.slot_bytes + (size_t)(r & (rps - 1)) * K * 2, nblk, av);
       if (lane == 0) y[k] = yk;
       // release the slot once this warp has no further row in it
       if (release && (k + 1 >= nr || (row_of(k + 1) >> lg) != js)) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[ts.idx[js]]);
+        if (lane == 0) mbar_arrive(&sm.empty[ts.idx(js)]);
       }
     }
   }
@@ -1075,7 +1091,11 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
         unsigned long long key = argmax_key(y[k], r0 + row_of(k));
         best = key > best ? key : best;
       }
-      if (best) atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, best);
+      // only a key above this warp's best so far can raise the maximum
+      if (best > sm.lm_seen[w][b]) {
+        sm.lm_seen[w][b] = best;
+        atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, best);
+      }
     } break;
     default: break;
   }
@@ -1246,6 +1266,29 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
 }
 
 // ---------------------------------------------------------------- kernel
+// Prologue: every family's extent for this step's symbols (into shared
+// memory), and every Event Tensor counter armed with its wait count (this
+// thread's share of the grid-wide range).
+__device__ __forceinline__ void arm_events(const DevPlan& P, Smem& sm, const FamilyDesc* fams, const int32_t* code,
+                                        int* counters, int B) {
+  const int tid = threadIdx.x;
+  for (int f = tid; f < P.n_families; f += blockDim.x) {
+    ExprEnv env{B, sm.ctx, {0, 0, 0}};
+    sm.fam_ext[f] = expr_eval(code, fams[f].extent_expr, env);
+    sm.fam_op[f] = (signed char)fams[f].op;
+    sm.fam_layer[f] = (signed char)fams[f].layer;
+  }
+  const int gtid = blockIdx.x * blockDim.x + tid, gthreads = gridDim.x * blockDim.x;
+  for (int i = gtid; i < P.n_counters; i += gthreads) {
+    int e = 0;
+    while (e + 1 < EV_COUNT && i >= P.ev[e + 1].base) ++e;
+    int lin = i - P.ev[e].base;
+    ExprEnv env{B, sm.ctx, {0, 0, 0}};
+    for (int dd = P.ev[e].ndim - 1; dd >= 0; --dd) { env.coord[dd] = lin % P.ev[e].dims[dd]; lin /= P.ev[e].dims[dd]; }
+    counters[i] = expr_eval(code, P.ev[e].count_expr, env);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const StepParams S, unsigned char* ws) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring = smem_raw;
@@ -1263,6 +1306,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     sm.released = 0;
     sm.dq_head = sm.dq_tail = sm.fq_head = sm.fq_tail = sm.notifier_stop = 0;
   }
+  if (tid < kComputeWarps * kMaxB) sm.lm_seen[tid / kMaxB][tid % kMaxB] = 0ull;
   __syncthreads();
   if (!sm.bad && tid < B) {
     int c = S.ctx[tid], s = S.slots[tid], t = S.tokens[tid];
@@ -1287,21 +1331,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     sm.pre[B] = run;
   }
   __syncthreads();
-  for (int f = tid; f < P.n_families; f += blockDim.x) {
-    ExprEnv env{B, sm.ctx, {0, 0, 0}};
-    sm.fam_ext[f] = expr_eval(code, fams[f].extent_expr, env);
-    sm.fam_op[f] = (signed char)fams[f].op;
-    sm.fam_layer[f] = (signed char)fams[f].layer;
-  }
+  arm_events(P, sm, fams, code, counters, B);
   const int gtid = blockIdx.x * blockDim.x + tid, gthreads = gridDim.x * blockDim.x;
-  for (int i = gtid; i < P.n_counters; i += gthreads) {
-    int e = 0;
-    while (e + 1 < EV_COUNT && i >= P.ev[e + 1].base) ++e;
-    int lin = i - P.ev[e].base;
-    ExprEnv env{B, sm.ctx, {0, 0, 0}};
-    for (int dd = P.ev[e].ndim - 1; dd >= 0; --dd) { env.coord[dd] = lin % P.ev[e].dims[dd]; lin /= P.ev[e].dims[dd]; }
-    counters[i] = expr_eval(code, P.ev[e].count_expr, env);
-  }
   {
     float* x = reinterpret_cast<float*>(ws + P.off_x);
     const int cpr = P.hidden / 8;
