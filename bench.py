@@ -33,6 +33,37 @@ CTX0 = 1024
 WINDOW = 32
 
 
+def kernel_source_sha():
+    """sha256 over the kernel sources, as recorded in the ncu summaries."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "event_tensor_task_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
+                   glob.glob(os.path.join(csrc, "*.h")))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(summary="megakernel_llama1b_b1_ncu.md"):
+    """DRAM bytes per launch (read + write) from the committed ncu summary,
+    or None when the kernel sources changed since that capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", summary)) as f:
+            text = f.read()
+    except OSError:
+        return None
+    import re
+    sha = re.search(r"Kernel source sha256[^`]*`([0-9a-f]{64})`", text)
+    tr = re.search(r"traffic: (\d+) bytes", text)
+    if not sha or not tr or sha.group(1) != kernel_source_sha():
+        return None
+    return int(tr.group(1))
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -297,7 +328,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) KV cache)", "config": workload_config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "frac": achieved / peak, "traffic": ncu_traffic(), "peak_kind": peak_kind,
                      "frac_of_8tbs": achieved / 8000.0, "bytes_per_launch": step_bytes},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 12, "d2h_bytes_per_step": 4},
