@@ -69,9 +69,23 @@ struct StepParams {
 
 struct TaskDesc {
   int32_t fam, op, layer, idx;
-  int32_t ring_seq, nslots;
+  int32_t slot_ph;   // ring slot of the task's first copy | parity of its phase << 16
+  int32_t nslots;
   int32_t rec;       // trace record of the task (0: none)
   uint32_t t_issue;  // trace: when the producer queued the task (low 32 bits of ns)
+};
+
+// Ring geometry of a GEMV op's tasks, fixed for the plan: the producer copies
+// part 0's rows (and, for the rotate-half and gate/up pair ops, part 1's rows
+// from a fresh slot) into consecutive ring slots, rps rows per slot.  Compute
+// warp w owns rows [w * rpw, (w + 1) * rpw) of each part.
+struct OpGeo {
+  int nblk;       // 256-column blocks per row (K / 256)
+  int row_bytes;  // 2 K
+  int rps_lg;     // log2(rows per slot)
+  int rpw;        // rows per warp per part
+  int spp;        // slots per part
+  int pairs;      // 1: two parts (rotate-half or gate/up pairs)
 };
 
 // batch rows the per-CTA sequence tables hold (the kernel runs B <= kMaxB)
@@ -93,7 +107,7 @@ struct Smem {
   // activation staging: one batch row, loaded once per CTA for all warps
   alignas(16) float xs[2048];  // read and written as float4
   float red8[kComputeWarps];
-  float yw[kComputeWarps][8];  // a warp's row results of the current task
+  OpGeo geo[OP_COUNT];  // GEMV geometry per op, set in the prologue
   unsigned long long lm_seen[kComputeWarps][kMaxB];  // per compute warp: best argmax key it has published
   uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
   // attention scratch, one row per head warp
@@ -288,7 +302,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     TaskDesc d;
     d.fam = fam; d.idx = idx; d.op = op; d.layer = layer;
     d.nslots = fam >= 0 ? task_slots(P, f, idx) : 0;
-    d.ring_seq = (int)ring_seq;
+    d.slot_ph = slot | (int)(phase << 16);
     d.rec = 0;
     int k = fifo_seq % kFifo;
     if (!wait_mbar(&sm.fifo_empty[k], ((fifo_seq / kFifo) & 1) ^ 1, ctl, tmo, fam, idx)) return false;
@@ -548,7 +562,7 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       if (room_ok && fired && ni.ffam >= 0) {
         TaskDesc f;
         f.fam = ni.ffam; f.op = ni.fop; f.layer = ni.flayer; f.idx = ni.fidx;
-        f.ring_seq = 0; f.nslots = 0; f.rec = 0; f.t_issue = 0;
+        f.slot_ph = 0; f.nslots = 0; f.rec = 0; f.t_issue = 0;
         sm.followq[(fh + rank) % kFollowQ] = f;
       }
       __syncwarp();
@@ -771,7 +785,7 @@ __device__ void controller(const DevPlan& P, const StepParams& S, Smem& sm, unsi
       if (!st) break;
     }
     TaskDesc e;
-    e.fam = -1; e.op = OP_END; e.layer = -1; e.idx = 0; e.ring_seq = 0; e.nslots = 0; e.rec = 0; e.t_issue = 0;
+    e.fam = -1; e.op = OP_END; e.layer = -1; e.idx = 0; e.slot_ph = 0; e.nslots = 0; e.rec = 0; e.t_issue = 0;
     if (lane == 0) {
       sm.cur[nrel & 1] = e;
       sm.released = 1 << 30;
@@ -920,181 +934,180 @@ __device__ __forceinline__ void act_to_regs(const float* xs, int nblk, ActRegs& 
 
 // Dot product of one weight row (bf16, in a ring slot) with the activation
 // registers, reduced over the warp.
-__device__ __forceinline__ float warp_dot(const unsigned char* rowp, int nblk, const ActRegs& av) {
+
+// Ring position of the task's slots.
+// Dot products of two rows held in shared memory (bf16, 16-byte chunks per
+// lane, 256 columns per block) with the activation in registers, interleaved
+// for instruction-level parallelism; summed across the warp (every lane gets
+// both sums).
+__device__ __forceinline__ void warp_dot2(const unsigned char* ra, const unsigned char* rb, int nblk,
+                                          const ActRegs& av, float& sa, float& sb) {
   const int lane = threadIdx.x & 31;
-  const uint4* r4 = reinterpret_cast<const uint4*>(rowp) + lane;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint4* a4 = reinterpret_cast<const uint4*>(ra) + lane;
+  const uint4* b4 = reinterpret_cast<const uint4*>(rb) + lane;
+  float acc_a[2] = {0.f, 0.f}, acc_b[2] = {0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < kMaxBlk; ++i) {
     if (i < nblk) {
-      float wf[8];
-      bf16x8_to_f32(r4[i * 32], wf);
+      float wa[8], wb[8];
+      bf16x8_to_f32(a4[i * 32], wa);
+      bf16x8_to_f32(b4[i * 32], wb);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j & 3] = fmaf(wf[j], av[i][j], acc[j & 3]);
+      for (int j = 0; j < 8; ++j) {
+        acc_a[j & 1] = fmaf(wa[j], av[i][j], acc_a[j & 1]);
+        acc_b[j & 1] = fmaf(wb[j], av[i][j], acc_b[j & 1]);
+      }
     }
   }
-  return warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
+  float va = acc_a[0] + acc_a[1], vb = acc_b[0] + acc_b[1];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    va += __shfl_xor_sync(0xffffffffu, va, o);
+    vb += __shfl_xor_sync(0xffffffffu, vb, o);
+  }
+  sa = va;
+  sb = vb;
 }
 
-// Ring position of the task's slots.
-// The ring slots of a task: consecutive from the slot of its first copy,
-// wrapping (with a parity flip) at the end of the ring.  Kept as a base slot
-// and parity rather than per-slot arrays, so that nothing indexed by a run-time
-// slot number has to live in local memory.
-struct TaskSlots {
-  int n, s0, R;
-  uint32_t p0;
-  __device__ __forceinline__ int idx(int j) const { return s0 + j < R ? s0 + j : s0 + j - R; }
-  __device__ __forceinline__ uint32_t par(int j) const { return s0 + j < R ? p0 : p0 ^ 1u; }
-};
-__device__ __forceinline__ void task_slots_of(const DevPlan& P, const TaskDesc& d, TaskSlots& ts) {
-  const uint32_t q = (uint32_t)d.ring_seq;
-  ts.n = d.nslots;
-  ts.R = P.ring_slots;
-  ts.s0 = (int)(q % (uint32_t)P.ring_slots);
-  ts.p0 = (q / (uint32_t)P.ring_slots) & 1;
-}
-
-// One warp's share of a GEMV task for batch row b: whole rows (or
-// rotate-half / gate-up row pairs, first rows of part 0 then of part 1), each
-// reduced inside the warp and written by lane 0.  The warp releases a ring
-// slot as soon as it has no more rows in it.
+// One warp's share of a GEMV task for batch row b.  The warp owns a
+// contiguous block of rows (row ops) or of row pairs (rotate-half q/k pairs,
+// gate/up pairs), so it waits on one ring slot (two for pair ops) and
+// releases every other slot of the task at once.  Its row sums end up in all
+// lanes; lane i then runs the epilogue of its row (or pair) i.
 __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                                unsigned char* ws, Control* ctl, const TaskDesc& d,
-                                               const GemvSpec& g, const TaskSlots& ts, const ActRegs& av, int b,
-                                               uint32_t* trec, bool release) {
+                                               const GemvSpec& g, const ActRegs& av, int b, uint32_t* trec,
+                                               bool release) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int K = g.K, nblk = K >> 8;
-  const int rps = P.slot_bytes / (2 * K);
-  const int lg = __ffs(rps) - 1;
-  const int H = P.hidden;
-  unsigned ready = 0;  // slots waited on
-  // this warp's rows, in increasing order (so in non-decreasing slot order):
-  // row ops take rows w, w+8, ...; pair ops take pairs p = w, w+8, ... and
-  // visit rows p of part 0, then rows half + p of part 1
-  const bool pairs = d.op == OP_QKV || d.op == OP_GATEUP;
-  const int half = d.op == OP_QKV ? P.tile_qkv / 2 : P.tile_gu;
-  const int nrow_task = pairs ? half : (d.op == OP_OPROJ ? P.tile_o : (d.op == OP_DOWN ? P.tile_down : g.rows));
-  const int npair = pairs ? max(0, (half - w + kComputeWarps - 1) / kComputeWarps) : 0;
-  const int nr = pairs ? 2 * npair : max(0, (nrow_task - w + kComputeWarps - 1) / kComputeWarps);
-  auto row_of = [&](int k) -> int {
-    return pairs ? (k < npair ? w + kComputeWarps * k : half + w + kComputeWarps * (k - npair))
-                 : w + kComputeWarps * k;
-  };
-  if (release && lane == 0) {
-    unsigned mine = 0;
+  const OpGeo geo = sm.geo[d.op];
+  const int R = P.ring_slots;
+  const int s0 = d.slot_ph & 0xffff;
+  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
+  const int r0 = w * geo.rpw;                                   // first row of this warp in part 0
+  const int n = max(0, min(geo.rpw, g.rows - r0));              // rows (pairs) of this warp
+  const int ja = r0 >> geo.rps_lg;                              // task slot of part 0's rows
+  const int jb = geo.pairs ? geo.spp + ja : -1;                 // task slot of part 1's rows
+  // the task's slots this warp reads none of: released right away, one lane each
+  if (release && lane < d.nslots && lane != ja && lane != jb) {
+    const int j = s0 + lane;
+    mbar_arrive(&sm.empty[j < R ? j : j - R]);
+  }
+  if (n == 0) return;
+  const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R;
+  const uint32_t pa = s0 + ja < R ? p0 : p0 ^ 1u;
+  wait_mbar(&sm.full[sa], pa, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  int sb = sa;
+  if (geo.pairs) {
+    sb = s0 + jb < R ? s0 + jb : s0 + jb - R;
+    wait_mbar(&sm.full[sb], s0 + jb < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  }
+  if (trec && lane == 0) {
+    trec[TR_DATA] = (uint32_t)global_ns();
+    trec[TR_ISSUE] = sm.slot_t[sa];
+  }
+  const int roff = (r0 & ((1 << geo.rps_lg) - 1)) * geo.row_bytes;
+  const unsigned char* base_a = ring + (size_t)sa * P.slot_bytes + roff;
+  const unsigned char* base_b = ring + (size_t)sb * P.slot_bytes + roff;
+  // y[2t], y[2t+1]: pair ops: part-0 and part-1 row of pair t; row ops: rows 2t, 2t+1
+  float y[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (k < nr) mine |= 1u << (row_of(k) >> lg);
-    for (int j = 0; j < ts.n; ++j)
-      if (!(mine & (1u << j))) mbar_arrive(&sm.empty[ts.idx(j)]);
-  }
-  float* y = sm.yw[w];
-#pragma unroll 1
-  for (int k = 0; k < 8; ++k) {
-    if (k < nr) {
-      const int r = row_of(k), js = r >> lg;
-      if (!(ready & (1u << js))) {
-        wait_mbar(&sm.full[ts.idx(js)], ts.par(js), ctl, P.spin_timeout_ns, d.fam, d.idx);
-        ready |= 1u << js;
-        if (js == 0 && trec && lane == 0) {
-          trec[TR_DATA] = (uint32_t)global_ns();
-          trec[TR_ISSUE] = sm.slot_t[ts.idx(0)];
-        }
-      }
-      const float yk = warp_dot(ring + (size_t)ts.idx(js) * P.slot_bytes + (size_t)(r & (rps - 1)) * K * 2, nblk, av);
-      if (lane == 0) y[k] = yk;
-      // release the slot once this warp has no further row in it
-      if (release && (k + 1 >= nr || (row_of(k + 1) >> lg) != js)) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[ts.idx(js)]);
-      }
+  for (int t = 0; t < 4; ++t) {
+    y[2 * t] = y[2 * t + 1] = 0.f;
+    if (geo.pairs) {
+      if (t < n) warp_dot2(base_a + t * geo.row_bytes, base_b + t * geo.row_bytes, geo.nblk, av, y[2 * t], y[2 * t + 1]);
+    } else if (2 * t < n) {
+      const int t1 = 2 * t + 1 < n ? 2 * t + 1 : 2 * t;  // an odd last row is paired with itself
+      warp_dot2(base_a + 2 * t * geo.row_bytes, base_a + t1 * geo.row_bytes, geo.nblk, av, y[2 * t], y[2 * t + 1]);
     }
   }
-  if (d.op == OP_OPROJ) {
-    // residual: x = (x + previous layer's down partials) + o W_o^T; lane 0
-    // reads x, lanes 1..n_kc the partials, in one round trip
-    float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
-    const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
-    const int nq = d.layer > 0 ? P.n_kc : 0;
-#pragma unroll 1
-    for (int k = 0; k < nr; ++k) {
-      const size_t col = (size_t)d.idx * P.tile_o + row_of(k);
-      float v = 0.f;
-      if (lane == 0) v = __ldcg(x + col);
-      else if (lane <= nq) v = __ldcg(dp + ((size_t)(lane - 1) * P.max_batch + b) * H + col);
-      v = warp_sum(v);
-      if (lane == 0) x[col] = v + y[k];
+  if (release) {
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&sm.empty[sa]);
+      if (geo.pairs) mbar_arrive(&sm.empty[sb]);
     }
-    return;
   }
-  if (lane != 0) return;
+  // lane i takes row i (row ops) or pair i (pair ops)
+  float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    if (geo.pairs) {
+      if (t < 4 && lane == t) { v0 = y[2 * t]; v1 = y[2 * t + 1]; }
+    } else if (lane == t) {
+      v0 = y[t];
+    }
+  }
+  const int H = P.hidden;
+  const bool mine = lane < n;
   switch (d.op) {
     case OP_QKV: {
       // RoPE on q and k (rotate-half pairs j, j + D/2), then q -> buffer, k/v -> cache
+      if (!mine) break;
       QkvTile q = decode_qkv(P, d.idx);
       const int pos = sm.ctx[b];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (k >= npair) break;
-        const int j = q.j0 + row_of(k);
-        const float x0 = y[k], x1 = y[npair + k];
-        if (q.kind == 2) {
-          size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
-          __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * P.head_dim;
-          vc[j] = __float2bfloat16_rn(x0);
-          vc[j + 32] = __float2bfloat16_rn(x1);
+      const int j = q.j0 + r0 + lane;
+      if (q.kind == 2) {
+        size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
+        __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * P.head_dim;
+        vc[j] = __float2bfloat16_rn(v0);
+        vc[j + 32] = __float2bfloat16_rn(v1);
+      } else {
+        const float* rope = reinterpret_cast<const float*>(ws + P.off_rope) + ((size_t)pos * 32 + j) * 2;
+        const float c = __ldg(rope), sn = __ldg(rope + 1);
+        const float x0 = v0 * c - v1 * sn, x1 = v1 * c + v0 * sn;
+        if (q.kind == 0) {
+          float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * P.head_dim +
+                      q.head * P.head_dim;
+          qb[j] = x0;
+          qb[j + 32] = x1;
         } else {
-          const float* rope = reinterpret_cast<const float*>(ws + P.off_rope) + ((size_t)pos * 32 + j) * 2;
-          const float c = __ldg(rope), sn = __ldg(rope + 1);
-          const float r0 = x0 * c - x1 * sn, r1 = x1 * c + x0 * sn;
-          if (q.kind == 0) {
-            float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * P.head_dim +
-                        q.head * P.head_dim;
-            qb[j] = r0;
-            qb[j + 32] = r1;
-          } else {
-            size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
-            __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * P.head_dim;
-            kc[j] = __float2bfloat16_rn(r0);
-            kc[j + 32] = __float2bfloat16_rn(r1);
-          }
+          size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
+          __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * P.head_dim;
+          kc[j] = __float2bfloat16_rn(x0);
+          kc[j + 32] = __float2bfloat16_rn(x1);
         }
       }
     } break;
+    case OP_OPROJ: {
+      // residual: x = (x + previous layer's down partials) + o W_o^T
+      if (!mine) break;
+      const size_t col = (size_t)d.idx * P.tile_o + r0 + lane;
+      float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
+      const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H + col;
+      float acc = __ldcg(x + col);
+      if (d.layer > 0)
+        for (int kc = 0; kc < P.n_kc; ++kc) acc += __ldcg(dp + (size_t)kc * P.max_batch * H);
+      x[col] = acc + v0;
+    } break;
     case OP_GATEUP: {
-      float* h = reinterpret_cast<float*>(ws + P.off_h) + (size_t)b * P.ffn + (size_t)d.idx * P.tile_gu;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (k >= npair) break;
-        const float gt = y[k], up = y[npair + k];
-        h[row_of(k)] = gt / (1.0f + expf(-gt)) * up;
-      }
+      if (!mine) break;
+      float* h = reinterpret_cast<float*>(ws + P.off_h) + (size_t)b * P.ffn + (size_t)d.idx * P.tile_gu + r0;
+      h[lane] = v0 / (1.0f + expf(-v0)) * v1;
     } break;
     case OP_DOWN: {
-      const int n = d.idx - g.kc * P.n_dtiles;
+      if (!mine) break;
+      const int nt = d.idx - g.kc * P.n_dtiles;
       float* part = reinterpret_cast<float*>(ws + P.off_dpart) + ((size_t)g.kc * P.max_batch + b) * H +
-                    (size_t)n * P.tile_down;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (k < nr) part[row_of(k)] = y[k];
+                    (size_t)nt * P.tile_down + r0;
+      part[lane] = v0;
     } break;
     case OP_LM: {
-      // logits and this warp's best (logit, id) key, folded into the running
-      // maximum with an atomic max (order independent)
-      const int r0 = d.idx * P.tile_lm;
-      unsigned long long best = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (k >= nr) break;
-        if (S.logits) S.logits[(size_t)b * P.vocab + r0 + row_of(k)] = y[k];
-        unsigned long long key = argmax_key(y[k], r0 + row_of(k));
-        best = key > best ? key : best;
+      // logits, then the warp's best (logit, id) key; published with an atomic
+      // max only when it beats what this warp published before (order independent)
+      const int r = d.idx * P.tile_lm + r0 + lane;
+      unsigned long long key = 0ull;
+      if (mine) {
+        if (S.logits) S.logits[(size_t)b * P.vocab + r] = v0;
+        key = argmax_key(v0, r);
       }
-      // only a key above this warp's best so far can raise the maximum
-      if (best > sm.lm_seen[w][b]) {
-        sm.lm_seen[w][b] = best;
-        atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, best);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+        key = other > key ? other : key;
+      }
+      if (lane == 0 && key > sm.lm_seen[w][b]) {
+        sm.lm_seen[w][b] = key;
+        atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, key);
       }
     } break;
     default: break;
@@ -1105,8 +1118,8 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
                                        unsigned char* ws, Control* ctl, const TaskDesc& d) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, D = P.head_dim, CH = P.chunk;
-  const uint32_t seq = (uint32_t)d.ring_seq;
-  const int slot = (int)(seq % (uint32_t)P.ring_slots);
+  const int slot = d.slot_ph & 0xffff;
+  const uint32_t par = (uint32_t)d.slot_ph >> 16;
   if (w < qpg) {
     // warp w: query head g*qpg + w over this chunk's keys
     AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
@@ -1130,7 +1143,7 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
       sm.newv[w][lane + 32] = bf16_bits_to_f32(__ldcg(vn + lane + 32));
     }
     __syncwarp();
-    wait_mbar(&sm.full[slot], (seq / (uint32_t)P.ring_slots) & 1, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
     const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
     const unsigned char* vbase = kbase + (size_t)CH * D * 2;
     // scores of keys lane and lane + 32
@@ -1236,8 +1249,6 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
     GemvSpec g;
     if (gemv_spec(P, d, g)) {
-      TaskSlots ts;
-      task_slots_of(P, d, ts);
       // one pass per batch row (the activation is restaged each pass when
       // B > 1); the ring slots are released after the last pass
       for (int b = 0; b < B; ++b) {
@@ -1246,7 +1257,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
           act_to_regs(sm.xs, g.K >> 8, av);
           a_tag = B > 1 ? -1 : g.tag;
         }
-        warp_gemv_task(P, S, sm, ring, ws, ctl, d, g, ts, av, b, trec, b == B - 1);
+        warp_gemv_task(P, S, sm, ring, ws, ctl, d, g, av, b, trec, b == B - 1);
       }
     } else if (d.op == OP_ATTN) {
       task_attn(P, S, sm, ring, ws, ctl, d);
@@ -1322,6 +1333,22 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     return;
   }
   if (tid == 0) {
+    // GEMV geometry of each op (see OpGeo)
+    auto set_geo = [&](int op, int K, int rows_part, int pairs) {
+      OpGeo& gg = sm.geo[op];
+      const int rps = P.slot_bytes / (2 * K);
+      gg.nblk = K >> 8;
+      gg.row_bytes = 2 * K;
+      gg.rps_lg = __ffs(rps) - 1;
+      gg.rpw = rows_part / kComputeWarps;
+      gg.spp = ceil_div(rows_part, rps);
+      gg.pairs = pairs;
+    };
+    set_geo(OP_QKV, P.hidden, P.tile_qkv / 2, 1);
+    set_geo(OP_OPROJ, P.hidden, P.tile_o, 0);
+    set_geo(OP_GATEUP, P.hidden, P.tile_gu, 1);
+    set_geo(OP_DOWN, P.kseg, P.tile_down, 0);
+    set_geo(OP_LM, P.hidden, P.tile_lm, 0);
     int run = 0;
     for (int b = 0; b < B; ++b) {
       sm.pre[b] = run;

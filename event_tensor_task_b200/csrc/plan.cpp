@@ -266,19 +266,22 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.debug_flags = o->debug_flags;
   P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
 
-  // tiles: about 32 KB of weights per task, whole rotate-half pairs per QKV tile
+  // K segment of the down projection (split-K), at most 2048 columns
   int kseg = o->kseg ? o->kseg : std::min(F, 2048);
   while (kseg > 256 && F % kseg) kseg -= 256;
   P.kseg = kseg;
   // rows per 16 KB ring slot of a hidden-wide (and a kseg-wide) row
   const int rps_h = 8192 / H, rps_k = 8192 / kseg;
-  // tiles split evenly over the 8 compute warps: QKV and gate/up tiles hand
-  // each warp whole row pairs, the others whole rows
-  P.tile_qkv = o->tile_qkv ? o->tile_qkv : std::max(16, 2 * rps_h);
-  P.tile_o = o->tile_o ? o->tile_o : std::max(8, rps_h);
-  P.tile_gu = o->tile_gu ? o->tile_gu : std::max(8, rps_h);
-  P.tile_down = o->tile_down ? o->tile_down : std::max(8, rps_k);
-  P.tile_lm = o->tile_lm ? o->tile_lm : std::max(16, rps_h);
+  // tiles split evenly over the 8 compute warps (QKV and gate/up tiles hand
+  // each warp whole row pairs, the others whole rows).  Defaults: the largest
+  // legal tiles up to 8 ring slots per task (gate/up: 4 + 4; down: 8; O: 4
+  // slots, as O sits on the critical path), which amortise the fixed
+  // per-task cost best on the 1B shape
+  P.tile_qkv = o->tile_qkv ? o->tile_qkv : std::max(16, std::min(D, 8 * rps_h));
+  P.tile_o = o->tile_o ? o->tile_o : std::max(8, std::min(64, 4 * rps_h));
+  P.tile_gu = o->tile_gu ? o->tile_gu : std::max(8, std::min(32, 4 * rps_h));
+  P.tile_down = o->tile_down ? o->tile_down : std::max(8, std::min(64, 8 * rps_k));
+  P.tile_lm = o->tile_lm ? o->tile_lm : std::max(16, std::min(64, 8 * rps_h));
   P.chunk = o->attn_chunk ? o->attn_chunk : 64;
   P.slot_bytes = 16384;
   const int rows_per_slot_h = P.slot_bytes / (2 * H);
@@ -297,13 +300,17 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (!(P.tile_lm > 0 && P.tile_lm % rows_per_slot_h == 0 && P.tile_lm % 8 == 0))
     { err = "tile_lm must be a multiple of 8 filling whole ring slots"; return MK_ERR_INVALID_ARG; }
   if (P.chunk != 64) { err = "attn_chunk must be 64"; return MK_ERR_UNSUPPORTED; }
-  // a task spans at most 4 ring slots (16 accumulated rows per compute thread)
-  if (P.tile_qkv / rows_per_slot_h > 4 || P.tile_o / rows_per_slot_h > 4 || 2 * P.tile_gu / rows_per_slot_h > 4 ||
-      P.tile_down / rows_per_slot_k > 4 || ceil_div(P.tile_lm, rows_per_slot_h) > 4)
-    { err = "a tile spans more than 4 ring slots"; return MK_ERR_UNSUPPORTED; }
-  // a warp handles at most 8 rows (4 row pairs) of a task
+  // a task spans at most 8 ring slots
+  if (P.tile_qkv / rows_per_slot_h > 8 || P.tile_o / rows_per_slot_h > 8 || 2 * P.tile_gu / rows_per_slot_h > 8 ||
+      P.tile_down / rows_per_slot_k > 8 || ceil_div(P.tile_lm, rows_per_slot_h) > 8)
+    { err = "a tile spans more than 8 ring slots"; return MK_ERR_UNSUPPORTED; }
+  // each compute warp owns a contiguous block of rows (row pairs) of a task,
+  // inside one ring slot: at most 8 rows or 4 pairs, and no more than a slot holds
   if (P.tile_qkv / 2 > 32 || P.tile_o > 64 || P.tile_gu > 32 || P.tile_down > 64 || P.tile_lm > 64)
     { err = "a tile gives a warp more than 8 rows"; return MK_ERR_UNSUPPORTED; }
+  if (P.tile_qkv / 16 > rows_per_slot_h || P.tile_o / 8 > rows_per_slot_h || P.tile_gu / 8 > rows_per_slot_h ||
+      P.tile_down / 8 > rows_per_slot_k || P.tile_lm / 8 > rows_per_slot_h)
+    { err = "a tile gives a warp more rows than one ring slot holds"; return MK_ERR_UNSUPPORTED; }
   P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
   P.n_otiles = H / P.tile_o;
   P.n_gutiles = F / P.tile_gu;
