@@ -847,44 +847,55 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int b) {
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
-  const int K = g.K;
+  const int K = g.K;  // at most 8 * kComputeThreads: each thread stages one 8-column chunk
+  const int c = ct * 8;
+  const bool has = c < K;
   const float* src;
   size_t rstride;
   if (g.kind == 0) { src = reinterpret_cast<const float*>(ws + P.off_x); rstride = P.hidden; }
   else if (g.kind == 1) { src = reinterpret_cast<const float*>(ws + P.off_attn); rstride = (size_t)P.n_q_heads * P.head_dim; }
   else { src = reinterpret_cast<const float*>(ws + P.off_h) + (size_t)g.kc * P.kseg; rstride = P.ffn; }
   const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
+  // every load of the chunk (activation, split-K partials, norm gain) is
+  // issued before the first use, so staging costs one round trip to L2
+  float4 u = make_float4(0.f, 0.f, 0.f, 0.f), v = u;
+  float4 du[4], dv[4];
+  uint4 graw = make_uint4(0u, 0u, 0u, 0u);
+  const int nq = g.parts ? min(P.n_kc, 4) : 0;
+  if (has) {
+    const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
+    u = __ldcg(p4);
+    v = __ldcg(p4 + 1);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < nq) {
+        const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
+        du[q] = __ldcg(d4);
+        dv[q] = __ldcg(d4 + 1);
+      }
+    if (g.kind == 0) {
+      const void* gp = g.gamma_sel == 2 ? P.final_norm
+                                        : (g.gamma_sel == 1 ? layers[g.layer].ffn_norm : layers[g.layer].attn_norm);
+      graw = __ldg(reinterpret_cast<const uint4*>(gp) + c / 8);
+    }
+  }
   bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the previous activation
   float ss = 0.f;
-  for (int c = ct * 8; c < K; c += kComputeThreads * 8) {
-    const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
-    float4 u = __ldcg(p4), v = __ldcg(p4 + 1);
-    if (g.parts) {
-      float4 du[4], dv[4];
-      const int nq = min(P.n_kc, 4);
+  if (has) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (q < nq) {
-          const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
-          du[q] = __ldcg(d4);
-          dv[q] = __ldcg(d4 + 1);
-        }
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (q < nq) {
-          u.x += du[q].x; u.y += du[q].y; u.z += du[q].z; u.w += du[q].w;
-          v.x += dv[q].x; v.y += dv[q].y; v.z += dv[q].z; v.w += dv[q].w;
-        }
+    for (int q = 0; q < 4; ++q)
+      if (q < nq) {
+        u.x += du[q].x; u.y += du[q].y; u.z += du[q].z; u.w += du[q].w;
+        v.x += dv[q].x; v.y += dv[q].y; v.z += dv[q].z; v.w += dv[q].w;
+      }
+    if (g.parts)
       for (int q = 4; q < P.n_kc; ++q) {
         const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
         float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
         u.x += a4.x; u.y += a4.y; u.z += a4.z; u.w += a4.w;
         v.x += b4.x; v.y += b4.y; v.z += b4.z; v.w += b4.w;
       }
-    }
-    *reinterpret_cast<float4*>(&sm.xs[c]) = u;
-    *reinterpret_cast<float4*>(&sm.xs[c + 4]) = v;
-    ss += u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w + v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    ss = u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w + v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
   if (g.kind == 0) {
     ss = warp_sum(ss);
@@ -894,19 +905,14 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
 #pragma unroll
     for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[q];
     const float inv = 1.0f / sqrtf(tot / (float)K + P.eps);
-    const void* gp = g.gamma_sel == 2 ? P.final_norm
-                                      : (g.gamma_sel == 1 ? layers[g.layer].ffn_norm : layers[g.layer].attn_norm);
-    const uint4* gam = reinterpret_cast<const uint4*>(gp);
-    for (int c = ct * 8; c < K; c += kComputeThreads * 8) {
-      float gf[8];
-      bf16x8_to_f32(__ldg(gam + c / 8), gf);
-      float4* x4 = reinterpret_cast<float4*>(&sm.xs[c]);
-      float4 u = x4[0], v = x4[1];
-      u.x *= inv * gf[0]; u.y *= inv * gf[1]; u.z *= inv * gf[2]; u.w *= inv * gf[3];
-      v.x *= inv * gf[4]; v.y *= inv * gf[5]; v.z *= inv * gf[6]; v.w *= inv * gf[7];
-      x4[0] = u;
-      x4[1] = v;
-    }
+    float gf[8];
+    bf16x8_to_f32(graw, gf);
+    u.x *= inv * gf[0]; u.y *= inv * gf[1]; u.z *= inv * gf[2]; u.w *= inv * gf[3];
+    v.x *= inv * gf[4]; v.y *= inv * gf[5]; v.z *= inv * gf[6]; v.w *= inv * gf[7];
+  }
+  if (has) {
+    *reinterpret_cast<float4*>(&sm.xs[c]) = u;
+    *reinterpret_cast<float4*>(&sm.xs[c + 4]) = v;
   }
   bar_sync(BAR_COMP, kComputeThreads);  // the activation is complete
 }
