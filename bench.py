@@ -146,6 +146,124 @@ def setup_model(dev, seed=0):
     return s, w_cpu, w, K_cpu, V_cpu, K, V, max_ctx
 
 
+class TorchPerOpDecoder:
+    """Same-box comparison point: the same decode step as ordinary per-op
+    PyTorch on the same bf16 weights (cuBLAS bf16 GEMVs with the q/k/v and
+    gate/up weights concatenated, fp32 RMSNorm/RoPE/softmax, a masked GQA
+    attention over the padded cache), run eagerly or replayed as one CUDA
+    graph.  The position and the greedy token advance on the device, so one
+    captured graph serves every step of the decode window."""
+
+    def __init__(self, s, w, K, V, max_ctx, ctx0, window, tok0, dev):
+        import torch
+        self.s, self.max_ctx, self.ctx0, self.window = s, max_ctx, ctx0, window
+        L, D = s.n_layers, s.head_dim
+        self.K, self.V = K.clone(), V.clone()
+        self.embed = w["embed"]
+        self.final_norm = w["final_norm"].float()
+        self.layers = []
+        for l in range(L):
+            p = f"layers.{l}."
+            self.layers.append({
+                "attn_norm": w[p + "attn_norm"].float(), "ffn_norm": w[p + "ffn_norm"].float(),
+                "wqkv": torch.cat([w[p + "wq"], w[p + "wk"], w[p + "wv"]], 0), "wo": w[p + "wo"],
+                "wgu": torch.cat([w[p + "w_gate"], w[p + "w_up"]], 0), "wd": w[p + "w_down"]})
+        i = torch.arange(D // 2, dtype=torch.float64)
+        ang = torch.arange(max_ctx, dtype=torch.float64)[:, None] * s.rope_theta ** (-2.0 * i / D)
+        self.cos, self.sin = ang.cos().float().to(dev), ang.sin().float().to(dev)
+        self.keypos = torch.arange(max_ctx, device=dev)
+        self.tok = torch.full((1,), tok0, dtype=torch.long, device=dev)
+        self.counter = torch.zeros((), dtype=torch.long, device=dev)
+        self.graph = None
+
+    def _rms(self, x, g):
+        import torch
+        return x * torch.rsqrt(x.pow(2).mean(-1, keepdim=True) + self.s.eps) * g
+
+    def _rope(self, t, c, sn):
+        import torch
+        h = t.shape[-1] // 2
+        a, b = t[..., :h], t[..., h:]
+        return torch.cat([a * c - b * sn, b * c + a * sn], -1)
+
+    def step(self):
+        """One greedy decode step (all on the device, graph-capturable)."""
+        import torch
+        s = self.s
+        Hq, Hkv, D = s.n_q_heads, s.n_kv_heads, s.head_dim
+        pos = (self.ctx0 + torch.remainder(self.counter, self.window)).view(1)
+        c, sn = self.cos.index_select(0, pos), self.sin.index_select(0, pos)  # [1, D/2]
+        mask = self.keypos > pos  # keys after the new token's position
+        x = self.embed.index_select(0, self.tok).float()  # [1, H]
+        for l, lw in enumerate(self.layers):
+            h = self._rms(x, lw["attn_norm"]).to(torch.bfloat16)
+            qkv = (h @ lw["wqkv"].T).float()
+            q = self._rope(qkv[:, :Hq * D].view(Hq, D), c, sn)
+            k = self._rope(qkv[:, Hq * D:(Hq + Hkv) * D].view(Hkv, D), c, sn)
+            v = qkv[:, (Hq + Hkv) * D:].view(Hkv, D)
+            self.K[l, 0].index_copy_(1, pos, k.to(torch.bfloat16).view(Hkv, 1, D))
+            self.V[l, 0].index_copy_(1, pos, v.to(torch.bfloat16).view(Hkv, 1, D))
+            qg = q.view(Hkv, Hq // Hkv, D)
+            sc = torch.matmul(qg, self.K[l, 0].float().transpose(1, 2)) * (1.0 / math.sqrt(D))
+            sc = sc.masked_fill(mask, float("-inf"))
+            o = torch.matmul(torch.softmax(sc, -1), self.V[l, 0].float()).reshape(1, Hq * D)
+            x = x + (o.to(torch.bfloat16) @ lw["wo"].T).float()
+            h = self._rms(x, lw["ffn_norm"]).to(torch.bfloat16)
+            gu = (h @ lw["wgu"].T).float()
+            g, u = gu[:, :s.ffn], gu[:, s.ffn:]
+            act = (g * torch.sigmoid(g) * u).to(torch.bfloat16)
+            x = x + (act @ lw["wd"].T).float()
+        logits = self._rms(x, self.final_norm).to(torch.bfloat16) @ self.embed.T
+        self.tok.copy_(torch.argmax(logits.float(), -1))
+        self.counter.add_(1)
+
+    def capture(self):
+        """Capture one step as a CUDA graph; returns the capture time in ms."""
+        import torch
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                self.step()  # warm-up on a side stream, as graph capture requires
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        torch.cuda.synchronize()
+        return 1000.0 * (time.perf_counter() - t0)
+
+    def timed(self, n, graph):
+        """Mean device ms per step over n steps (CUDA events)."""
+        import torch
+        run = self.graph.replay if graph else self.step
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+
+def torch_baselines(s, w, K, V, max_ctx, tok0, dev, n_steps):
+    """Per-op PyTorch eager and CUDA-graph decode steps on the same model."""
+    base = TorchPerOpDecoder(s, w, K, V, max_ctx, CTX0, WINDOW, tok0, dev)
+    eager_ms = base.timed(max(10, n_steps // 10), graph=False)
+    capture_ms = base.capture()
+    graph_ms = base.timed(n_steps, graph=True)
+    return {"torch_eager": {"us_per_step": 1000.0 * eager_ms, "tokens_per_s": 1000.0 / eager_ms},
+            "torch_cuda_graph": {"us_per_step": 1000.0 * graph_ms, "tokens_per_s": 1000.0 / graph_ms,
+                                 "capture_ms": capture_ms},
+            "what": "same model, weights and cache on the same GPU: per-op PyTorch (cuBLAS bf16 GEMV, "
+                    "fused q/k/v and gate/up weights, masked GQA attention over the padded cache), "
+                    "eager and as one captured CUDA graph; device-timed with CUDA events"}
+
+
 def cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, n_steps):
     """The oracle as it stands: tokens/s over n_steps decode steps after one
     untimed warm-up step (which also widens the weights to fp64 once)."""
@@ -204,6 +322,7 @@ def main():
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--sched", default="static", choices=["static", "dynamic"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-torch-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -310,6 +429,15 @@ def main():
         e_ms = float(t.item())
     e2e_value = world * n_e2e / (e_ms / 1000.0)
 
+    baselines = None
+    if world == 1 and not args.no_torch_baseline:
+        baselines = torch_baselines(s, w, K, V, max_ctx, tok0, dev, min(args.steps, 500))
+        t0 = time.perf_counter()
+        tmp = mk.DenseDecoder(s, w, K, V, max_batch=1, max_ctx=max_ctx, n_slots=1, sched=sched)
+        torch.cuda.synchronize()
+        baselines["megakernel_plan_build_and_bind_ms"] = 1000.0 * (time.perf_counter() - t0)
+        tmp.close()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, dt = cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, 2)
@@ -331,6 +459,7 @@ def main():
                      "frac": achieved / peak, "traffic": ncu_traffic(), "peak_kind": peak_kind,
                      "frac_of_8tbs": achieved / 8000.0, "bytes_per_launch": step_bytes},
         "cpu_baseline": cpu,
+        "torch_baselines": baselines,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 12, "d2h_bytes_per_step": 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
