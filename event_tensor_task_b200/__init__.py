@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes as C
 
 from . import _abi
-from ._abi import (MK_OK, MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_STATIC_SCRATCH_BYTES,
+from ._abi import (MK_MODEL_MOE_LAYER, mk_moe_weights, mk_moe_args, MK_OK, MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_STATIC_SCRATCH_BYTES,
                    MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS, MK_DEBUG_TRACE,
                    MK_SIM_FAULT_NONE, MK_SIM_FAULT_DROP_NOTIFY, MK_SIM_FAULT_COUNT_PLUS_ONE,
                    MK_SIM_FAULT_NO_WAIT, OP_NAMES, mk_model_desc, mk_plan_opts, mk_step_args,
@@ -69,6 +69,10 @@ def mk_decode_step(plan: int, args: mk_step_args, stream: int = 0):
 
 def mk_decode_step_static(plan: int, args: mk_step_args, stream: int = 0):
     _check(lib().mk_decode_step_static(plan, C.byref(args), stream))
+
+
+def mk_moe_layer(plan: int, args: mk_moe_args, stream: int = 0):
+    _check(lib().mk_moe_layer(plan, C.byref(args), stream))
 
 
 def mk_get_status(plan: int):
@@ -209,6 +213,70 @@ class DenseDecoder:
     def reset(self):
         import torch
         mk_plan_reset(self.plan, torch.cuda.current_stream().cuda_stream)
+
+    def close(self):
+        if self.plan:
+            mk_plan_destroy(self.plan)
+            self.plan = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class MoELayer:
+    """A plan for one mixture-of-experts FFN layer plus the tensors it points at.
+
+    ``weights`` maps ``router`` ([E][H]), ``w_gate``/``w_up`` ([E][F][H]) and
+    ``w_down`` ([E][H][F]) to bf16 device tensors; ``bias`` is an fp32 [E]
+    device tensor added to the router logits, or None.  The plan runs on the
+    dynamic schedule (its task counts follow the routing).
+    """
+
+    def __init__(self, shape, weights, bias=None, max_tokens=512, n_sm=0, debug=False, spin_timeout_ns=0,
+                 host_only=False):
+        import torch
+        self.shape = shape
+        self._keep = [weights, bias]
+        d = mk_model_desc()
+        d.kind = MK_MODEL_MOE_LAYER
+        d.hidden, d.n_experts, d.top_k, d.expert_ffn = shape.hidden, shape.n_experts, shape.top_k, shape.expert_ffn
+        d.max_tokens = max_tokens
+        w = weights or {}
+        d.moe = mk_moe_weights(_ptr(w.get("router")), _ptr(bias), _ptr(w.get("w_gate")), _ptr(w.get("w_up")),
+                               _ptr(w.get("w_down")))
+        o = mk_plan_opts()
+        o.sched, o.n_sm, o.host_only = MK_SCHED_DYNAMIC, n_sm, int(host_only)
+        o.spin_timeout_ns = spin_timeout_ns
+        o.debug_flags = MK_DEBUG_TASK_COUNTS if debug else 0
+        self.desc, self.opts = d, o
+        self.plan = mk_plan_build(d, o)
+        self.ws = None
+        if not host_only:
+            nbytes = mk_plan_workspace_bytes(self.plan)
+            self.ws = torch.empty(nbytes + 256, dtype=torch.uint8, device="cuda")
+            base = (_ptr(self.ws) + 255) // 256 * 256
+            mk_plan_bind_workspace(self.plan, base, nbytes, torch.cuda.current_stream().cuda_stream)
+
+    def families(self):
+        return [mk_plan_family_info(self.plan, f) for f in range(mk_plan_num_families(self.plan))]
+
+    def __call__(self, x, out, topk_idx=None, topk_w=None, hist=None, indptr=None, logits=None,
+                 task_counts=None, stream=None):
+        """out = MoE(x) for x, out bf16 [T][H] on the device (one launch)."""
+        import torch
+        a = mk_moe_args()
+        a.n_tokens = int(x.shape[0])
+        a.x, a.out = _ptr(x), _ptr(out)
+        a.topk_idx, a.topk_w, a.hist, a.indptr = _ptr(topk_idx), _ptr(topk_w), _ptr(hist), _ptr(indptr)
+        a.logits, a.task_counts = _ptr(logits), _ptr(task_counts)
+        s = stream if stream is not None else torch.cuda.current_stream()
+        mk_moe_layer(self.plan, a, s.cuda_stream)
+
+    def status(self):
+        return mk_get_status(self.plan)
 
     def close(self):
         if self.plan:

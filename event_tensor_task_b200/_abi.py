@@ -29,13 +29,21 @@ MK_SIM_FAULT_DROP_NOTIFY = 1
 MK_SIM_FAULT_COUNT_PLUS_ONE = 2
 MK_SIM_FAULT_NO_WAIT = 3
 
+MK_MODEL_MOE_LAYER = 1
+
 OP_NAMES = {1: "qkv", 2: "attn", 3: "merge", 4: "oproj", 5: "gateup", 6: "down",
-            8: "lm", 10: "lmfin"}
+            8: "lm", 10: "lmfin", 11: "route", 12: "mindptr", 13: "egu", 14: "edown", 15: "combine",
+            16: "mfin"}
 
 
 class mk_layer_weights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in
                 ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down")]
+
+
+class mk_moe_weights(C.Structure):
+    _fields_ = [("w_router", C.c_void_p), ("router_bias", C.c_void_p), ("w_gate", C.c_void_p),
+                ("w_up", C.c_void_p), ("w_down", C.c_void_p)]
 
 
 class mk_model_desc(C.Structure):
@@ -45,6 +53,16 @@ class mk_model_desc(C.Structure):
         ("eps", C.c_float), ("rope_theta", C.c_float), ("max_batch", C.c_int), ("max_ctx", C.c_int),
         ("n_slots", C.c_int), ("embed", C.c_void_p), ("lm_head", C.c_void_p), ("final_norm", C.c_void_p),
         ("layers", C.POINTER(mk_layer_weights)), ("k_cache", C.c_void_p), ("v_cache", C.c_void_p),
+        ("n_experts", C.c_int), ("top_k", C.c_int), ("expert_ffn", C.c_int), ("max_tokens", C.c_int),
+        ("moe", mk_moe_weights),
+    ]
+
+
+class mk_moe_args(C.Structure):
+    _fields_ = [
+        ("n_tokens", C.c_int), ("x", C.c_void_p), ("out", C.c_void_p), ("topk_idx", C.c_void_p),
+        ("topk_w", C.c_void_p), ("hist", C.c_void_p), ("indptr", C.c_void_p), ("logits", C.c_void_p),
+        ("task_counts", C.c_void_p),
     ]
 
 
@@ -88,6 +106,7 @@ PROTOTYPES = {
     "mk_plan_bind_workspace": (C.c_int, [C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "mk_decode_step": (C.c_int, [C.c_void_p, C.POINTER(mk_step_args), C.c_void_p]),
     "mk_decode_step_static": (C.c_int, [C.c_void_p, C.POINTER(mk_step_args), C.c_void_p]),
+    "mk_moe_layer": (C.c_int, [C.c_void_p, C.POINTER(mk_moe_args), C.c_void_p]),
     "mk_get_status": (C.c_int, [C.c_void_p, C.POINTER(mk_device_status)]),
     "mk_plan_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
     "mk_plan_task_slots": (C.c_int, [C.c_void_p]),

@@ -54,7 +54,7 @@ mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_pla
     }
     mk_plan* hp = new mk_plan();
     mk_status s = mk::build_plan(m, opts, n_sm, smem, hp->p, err);
-    if (s == MK_OK) {
+    if (s == MK_OK && hp->p.dp.kind == MK_MODEL_DENSE) {
       // the plan must validate on a small binding of the symbols before use
       std::vector<int> ctx(hp->p.dp.max_batch, std::min(hp->p.dp.max_ctx - 1, 3 * hp->p.dp.chunk - 1));
       mk::Binding bd{hp->p.dp.max_batch, ctx};
@@ -102,6 +102,7 @@ mk_status mk_plan_bind_workspace(mk_plan* hp, void* dev_ptr, size_t bytes, void*
 mk_status mk_decode_step(mk_plan* hp, const mk_step_args* a, void* stream) {
   g_err.clear();
   if (!hp || !a) return fail(MK_ERR_INVALID_ARG, "null argument");
+  if (hp->p.dp.kind != MK_MODEL_DENSE) return fail(MK_ERR_INVALID_ARG, "plan is not a dense decoder");
   if (!hp->p.ws) return fail(MK_ERR_WORKSPACE, "no workspace bound");
   if (a->batch < 1 || a->batch > hp->p.dp.max_batch) return fail(MK_ERR_INVALID_ARG, "batch out of [1, max_batch]");
   if (!a->token_ids || !a->slot_ids || !a->ctx_lens || !a->next_tokens)
@@ -114,6 +115,7 @@ mk_status mk_decode_step(mk_plan* hp, const mk_step_args* a, void* stream) {
 mk_status mk_decode_step_static(mk_plan* hp, const mk_step_args* a, void* stream) {
   g_err.clear();
   if (!hp || !a) return fail(MK_ERR_INVALID_ARG, "null argument");
+  if (hp->p.dp.kind != MK_MODEL_DENSE) return fail(MK_ERR_INVALID_ARG, "plan is not a dense decoder");
   if (hp->p.device < 0) return fail(MK_ERR_UNSUPPORTED, "plan was built host_only");
   if (a->batch < 1 || a->batch > hp->p.dp.max_batch) return fail(MK_ERR_INVALID_ARG, "batch out of [1, max_batch]");
   if (!a->token_ids || !a->slot_ids || !a->ctx_lens || !a->next_tokens)
@@ -129,6 +131,19 @@ mk_status mk_decode_step_static(mk_plan* hp, const mk_step_args* a, void* stream
   } catch (...) {
     return fail(MK_ERR_CUDA, "unexpected error in the static-scratch decode step");
   }
+}
+
+mk_status mk_moe_layer(mk_plan* hp, const mk_moe_args* a, void* stream) {
+  g_err.clear();
+  if (!hp || !a) return fail(MK_ERR_INVALID_ARG, "null argument");
+  if (hp->p.dp.kind != MK_MODEL_MOE_LAYER) return fail(MK_ERR_INVALID_ARG, "plan is not an MoE layer");
+  if (!hp->p.ws) return fail(MK_ERR_WORKSPACE, "no workspace bound");
+  if (a->n_tokens < 1 || a->n_tokens > hp->p.dp.max_tokens)
+    return fail(MK_ERR_INVALID_ARG, "n_tokens out of [1, max_tokens]");
+  if (!a->x || !a->out) return fail(MK_ERR_INVALID_ARG, "x and out are required");
+  std::string err;
+  mk_status s = mk::dev_launch_moe(hp->p, a, stream, err);
+  return s == MK_OK ? MK_OK : fail(s, err);
 }
 
 mk_status mk_get_status(mk_plan* hp, mk_device_status* st) {

@@ -14,4 +14,5 @@ mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& 
 mk_status dev_status(Plan& p, mk_device_status* st, std::string& err);
 mk_status dev_reset(Plan& p, void* stream, std::string& err);
 mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::string& err);
+mk_status dev_launch_moe(Plan& p, const mk_moe_args* a, void* stream, std::string& err);
 }  // namespace mk

@@ -55,7 +55,15 @@ constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
 constexpr int kDynLookahead = 2;
 
 struct StepParams {
-  int B;
+  int B;                 // batch size; the token count T for an MoE layer
+  // MoE layer
+  const __nv_bfloat16* moe_x;
+  __nv_bfloat16* moe_out;
+  int* dbg_idx;
+  float* dbg_w;
+  int* dbg_hist;
+  int* dbg_indptr;
+  float* dbg_logits;
   const int* tokens;
   const int* slots;
   const int* ctx;
@@ -177,7 +185,9 @@ __device__ __forceinline__ int ev_ctr(const DevPlan& P, int ev, int c0, int c1 =
 __device__ __forceinline__ int fam_of(const DevPlan& P, int op, int layer) {
   return op >= OP_LM ? P.fam_first_layer[op] : P.fam_first_layer[op] + layer * P.fam_stride;
 }
-__device__ __forceinline__ bool is_followup(int op) { return op == OP_MERGE || op == OP_LMFIN; }
+__device__ __forceinline__ bool is_followup(int op) {
+  return op == OP_MERGE || op == OP_LMFIN || op == OP_MINDPTR || op == OP_MFIN;
+}
 
 // Counter a regular task waits on (-1: none).
 __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t, int B) {
@@ -191,7 +201,9 @@ __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t,
     case OP_GATEUP: return ev_ctr(P, EV_O, t.layer);
     case OP_DOWN: return ev_ctr(P, EV_GU, t.layer, t.idx / P.n_dtiles);
     case OP_LM: return ev_ctr(P, EV_IN, P.n_layers);
-    default: return -1;
+    case OP_EDOWN: return ev_ctr(P, EV_MH, t.idx / P.nt_d);
+    case OP_COMBINE: return ev_ctr(P, EV_MY, 0);
+    default: return -1;  // ROUTE; EGU is pushed only once its tile table exists
   }
 }
 
@@ -203,6 +215,7 @@ struct ProdFam {
   const unsigned char* w[3];  // q/k/v (QKV) or the parts' base matrices
   uint32_t row_bytes;         // bytes of one row copy
   uint32_t row_stride;        // bytes between consecutive rows in memory
+  uint32_t row_pitch;         // bytes between consecutive rows in a ring slot
   int rps;                    // rows per ring slot
   int slots_per_part;
   int parts;
@@ -212,7 +225,7 @@ struct ProdFam {
 __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, int fam, int op, int layer, ProdFam& f) {
   const uint32_t H2 = (uint32_t)P.hidden * 2;
   f.fam = fam; f.op = op; f.layer = layer;
-  f.row_bytes = H2; f.row_stride = H2; f.rps = P.slot_bytes / (int)H2; f.parts = 1;
+  f.row_bytes = H2; f.row_stride = H2; f.row_pitch = H2; f.rps = P.slot_bytes / (int)H2; f.parts = 1;
   f.w[0] = f.w[1] = f.w[2] = nullptr;
   f.task_stride = 0;
   f.slots_per_part = 1;
@@ -232,8 +245,17 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, int fam, i
       break;
     case OP_DOWN:
       f.w[0] = (const unsigned char*)layers[layer].w_down;
-      f.row_bytes = (uint32_t)P.kseg * 2; f.row_stride = (uint32_t)P.ffn * 2;
+      f.row_bytes = (uint32_t)P.kseg * 2; f.row_stride = (uint32_t)P.ffn * 2; f.row_pitch = f.row_bytes;
       f.rps = P.slot_bytes / (int)f.row_bytes; f.slots_per_part = P.tile_down / f.rps;
+      break;
+    case OP_EGU:  // an expert's gate rows, then its up rows (the expert is per task)
+      f.w[0] = (const unsigned char*)P.w_egate; f.w[1] = (const unsigned char*)P.w_eup;
+      f.parts = 2; f.slots_per_part = ceil_div(P.moe_tn, f.rps);
+      break;
+    case OP_EDOWN:  // an expert's down rows (expert_ffn long), placed at a 4 KB pitch
+      f.w[0] = (const unsigned char*)P.w_edown;
+      f.row_bytes = (uint32_t)P.eff * 2; f.row_stride = f.row_bytes; f.row_pitch = 4096;
+      f.rps = P.slot_bytes / 4096; f.slots_per_part = ceil_div(P.moe_td, f.rps);
       break;
     case OP_LM:
       f.w[0] = (const unsigned char*)P.lm_head;
@@ -245,6 +267,7 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, int fam, i
 
 __device__ __forceinline__ int task_slots(const DevPlan& P, const ProdFam& f, int idx) {
   if (f.op == OP_ATTN) return 1;
+  if (f.op == OP_ROUTE || f.op == OP_COMBINE || f.op == OP_MINDPTR || f.op == OP_MFIN) return 0;
   if (f.op == OP_LM) return ceil_div(min(P.tile_lm, P.vocab - idx * P.tile_lm), f.rps);
   return f.parts * f.slots_per_part;
 }
@@ -281,10 +304,10 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       if (!next_slot(fam, idx, dst, bar)) return false;
       int rows = min(nrows, f.rps);
       mbar_arrive_expect_tx(bar, (uint32_t)rows * f.row_bytes);
-      if (f.row_stride == f.row_bytes) {
+      if (f.row_stride == f.row_bytes && f.row_pitch == f.row_bytes) {
         bulk_g2s(dst, src, (uint32_t)rows * f.row_bytes, bar);
       } else {
-        for (int r = 0; r < rows; ++r) bulk_g2s(dst + r * f.row_bytes, src + (size_t)r * f.row_stride, f.row_bytes, bar);
+        for (int r = 0; r < rows; ++r) bulk_g2s(dst + r * f.row_pitch, src + (size_t)r * f.row_stride, f.row_bytes, bar);
       }
       src += (size_t)rows * f.row_stride;
       nrows -= rows;
@@ -335,6 +358,21 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
         if (!stream_part(fam, idx, f.w[0] + (size_t)idx * f.task_stride, min(P.tile_lm, P.vocab - idx * P.tile_lm)))
           return false;
         break;
+      case OP_EGU: {
+        // tile -> expert from the table the routing follow-up wrote (visible:
+        // this task was popped after its push, which followed that write)
+        const int tile = idx / P.nt_gu, n = idx - tile * P.nt_gu;
+        const int e = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_e) + tile);
+        const size_t row0 = (size_t)e * P.eff + (size_t)n * P.moe_tn;
+        if (!stream_part(fam, idx, f.w[0] + row0 * f.row_stride, P.moe_tn)) return false;
+        if (!stream_part(fam, idx, f.w[1] + row0 * f.row_stride, P.moe_tn)) return false;
+      } break;
+      case OP_EDOWN: {
+        const int tile = idx / P.nt_d, n = idx - tile * P.nt_d;
+        const int e = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_e) + tile);
+        const size_t row0 = (size_t)e * P.hidden + (size_t)n * P.moe_td;
+        if (!stream_part(fam, idx, f.w[0] + row0 * f.row_stride, P.moe_td)) return false;
+      } break;
       case OP_ATTN: {
         // the chunk's cached (already rotated) keys and values, minus the row
         // this step appends; K rows at the slot start, V rows half a slot in
@@ -462,6 +500,17 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
       n.ctr = ev_ctr(P, EV_LM, 0);
       n.ffam = fam_of(P, OP_LMFIN, -1); n.fop = OP_LMFIN; n.fidx = 0;
       break;
+    case OP_ROUTE:
+      n.ctr = ev_ctr(P, EV_ROUTE, 0);
+      n.ffam = fam_of(P, OP_MINDPTR, -1); n.fop = OP_MINDPTR; n.fidx = 0;
+      break;
+    case OP_MINDPTR: n.ctr = ev_ctr(P, EV_MIDX, 0); break;
+    case OP_EGU: n.ctr = ev_ctr(P, EV_MH, t.idx / P.nt_gu); break;  // the tile's event: set by the routing
+    case OP_EDOWN: n.ctr = ev_ctr(P, EV_MY, 0); break;
+    case OP_COMBINE:
+      n.ctr = ev_ctr(P, EV_MCOMB, 0);
+      n.ffam = fam_of(P, OP_MFIN, -1); n.fop = OP_MFIN; n.fidx = 0;
+      break;
     default: break;
   }
   n.need_old = (n.ctr >= 0 && (n.ffam >= 0 || dyn)) ? 1 : 0;
@@ -489,6 +538,16 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
       if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
       else push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
       break;
+    // MoE: exp_indptr decides how many GroupGEMM tiles run (data-dependent task triggering)
+    case OP_MINDPTR: {
+      const int n_tiles = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile) + P.n_experts);
+      push_range(P, S, ctl, ws, fam_of(P, OP_EGU, -1), 0, n_tiles * P.nt_gu);
+    } break;
+    case OP_EGU: {
+      const int tile = t.idx / P.nt_gu;
+      push_range(P, S, ctl, ws, fam_of(P, OP_EDOWN, -1), tile * P.nt_d, P.nt_d);
+    } break;
+    case OP_EDOWN: push_range(P, S, ctl, ws, fam_of(P, OP_COMBINE, -1), 0, ceil_div(S.B, 8)); break;
     default: break;
   }
 }
@@ -544,7 +603,7 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       }
     }
     if (fired && P.sched == MK_SCHED_DYNAMIC) push_successors(P, S, sm, ctl, ws, t);
-    if (lane < n && t.op == OP_LMFIN && P.sched == MK_SCHED_DYNAMIC)
+    if (lane < n && (t.op == OP_LMFIN || t.op == OP_MFIN) && P.sched == MK_SCHED_DYNAMIC)
       push_range(P, S, ctl, ws, -1, 0, P.n_sm);  // one END per CTA
     unsigned fb = __ballot_sync(0xffffffffu, fired && ni.ffam >= 0);
     if (fb) {
@@ -1240,12 +1299,322 @@ __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S
   out[dd] = O / L;
 }
 
+// ---------------------------------------------------------------- MoE layer
+// (The MoE task bodies are compiled into the MoE instance of the kernel only:
+// see megakernel<kMoE>.)
+// Mixture-of-experts FFN on T tokens ("Event Tensor: A Unified Abstraction for
+// Compiling Dynamic Megakernel", section "Core method": data-dependent event
+// update and data-dependent task triggering).  Rows of the grouped problem
+// are the (token, slot) pairs; expert e owns rows [indptr[e], indptr[e+1]).
+
+// ROUTE: tokens 8*idx .. 8*idx+7.  Phase 1: warp w computes the router
+// logits of experts w, w+8, ... for the 8 tokens, each in one fixed order
+// (lane l sums its products over hidden index 256*i + 8*l + j, i outer, j
+// inner, from +0; then an xor butterfly 16, 8, 4, 2, 1; then the bias), so
+// that the top-k is exact.  Phase 2: warp w takes token w: top-k by logit
+// (ties -> lower expert), softmax over the selected logits, and one
+// histogram atomic per selection whose old value is the pair's rank inside
+// its expert's rows.
+__device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws,
+                                           const TaskDesc& d) {
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
+  const int E = P.n_experts, K = P.top_k, H = P.hidden, T = S.B, nblk = H >> 8;
+  float* lg = sm.xs;  // [8][64] logits of this task's tokens
+  bar_sync(BAR_COMP, kComputeThreads);  // the staging buffer is free
+  const uint4* wr = reinterpret_cast<const uint4*>(P.w_router);
+  const uint4* xr = reinterpret_cast<const uint4*>(S.moe_x);
+  for (int e = w; e < E; e += kComputeWarps) {
+    uint4 wv[kMaxBlk];
+#pragma unroll
+    for (int i = 0; i < kMaxBlk; ++i)
+      if (i < nblk) wv[i] = __ldg(wr + ((size_t)e * H + 256 * i + 8 * lane) / 8);
+    const float bias = P.router_bias ? __ldg(P.router_bias + e) : 0.f;
+    for (int tt = 0; tt < 8; ++tt) {
+      const int t = d.idx * 8 + tt;
+      if (t >= T) break;
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxBlk; ++i)
+        if (i < nblk) {
+          float wf[8], xf[8];
+          bf16x8_to_f32(wv[i], wf);
+          bf16x8_to_f32(__ldg(xr + ((size_t)t * H + 256 * i + 8 * lane) / 8), xf);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc = fmaf(wf[j], xf[j], acc);  // the product is exact in fp32
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc = acc + __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) lg[tt * 64 + e] = acc + bias;
+    }
+  }
+  bar_sync(BAR_COMP, kComputeThreads);
+  const int t = d.idx * 8 + w;
+  if (t >= T) return;
+  const bool has0 = lane < E, has1 = lane + 32 < E;
+  const float v0 = has0 ? lg[w * 64 + lane] : 0.f, v1 = has1 ? lg[w * 64 + lane + 32] : 0.f;
+  if (S.dbg_logits) {
+    if (has0) S.dbg_logits[(size_t)t * E + lane] = v0;
+    if (has1) S.dbg_logits[(size_t)t * E + lane + 32] = v1;
+  }
+  bool av0 = has0, av1 = has1;
+  int sel_e = 0;
+  float sel_v = 0.f;
+  for (int j = 0; j < K; ++j) {
+    const unsigned long long k0 = av0 ? argmax_key(v0, lane) : 0ull, k1 = av1 ? argmax_key(v1, lane + 32) : 0ull;
+    unsigned long long best = k0 > k1 ? k0 : k1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = other > best ? other : best;
+    }
+    const int e = argmax_key_index(best);
+    const float v = __shfl_sync(0xffffffffu, e < 32 ? v0 : v1, e & 31);
+    if (lane == (e & 31)) { if (e < 32) av0 = false; else av1 = false; }
+    if (lane == j) { sel_e = e; sel_v = v; }
+  }
+  const float mx = __shfl_sync(0xffffffffu, sel_v, 0);  // the first selection is the largest
+  const float ex = lane < K ? expf(sel_v - mx) : 0.f;
+  const float sum = warp_sum(ex);
+  if (lane < K) {
+    const float wt = ex / sum;
+    const size_t pi = (size_t)t * K + lane;
+    const int rank = atomicAdd(reinterpret_cast<int*>(ws + P.off_mhist) + sel_e, 1);
+    reinterpret_cast<int*>(ws + P.off_mrank)[pi] = rank;
+    reinterpret_cast<int*>(ws + P.off_midx)[pi] = sel_e;
+    reinterpret_cast<float*>(ws + P.off_mw)[pi] = wt;
+    if (S.dbg_idx) S.dbg_idx[pi] = sel_e;
+    if (S.dbg_w) S.dbg_w[pi] = wt;
+  }
+}
+
+// MINDPTR (follow-up of the routing event, all compute warps): exp_indptr =
+// exclusive prefix sum of the histogram; tile_ptr = exclusive prefix sum of
+// ceil(hist[e] / tm) and the tile -> (expert, m) table the GroupGEMM tasks
+// decode; the run-time count of EV_MY (one per down task); and the row map
+// (pair -> row, row -> pair).
+__device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws) {
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
+  const int E = P.n_experts, K = P.top_k, TMt = P.moe_tm;
+  int* sx = reinterpret_cast<int*>(sm.xs);  // exp_indptr [E + 1]
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (w == 0) {
+    const int* hist = reinterpret_cast<const int*>(ws + P.off_mhist);
+    int* indptr = reinterpret_cast<int*>(ws + P.off_mindptr);
+    int* tptr = reinterpret_cast<int*>(ws + P.off_mtile);
+    int* tile_e = reinterpret_cast<int*>(ws + P.off_mtile_e);
+    int* tile_m = reinterpret_cast<int*>(ws + P.off_mtile_m);
+    const int h0 = lane < E ? __ldcg(hist + lane) : 0, h1 = lane + 32 < E ? __ldcg(hist + lane + 32) : 0;
+    const int c0 = (h0 + TMt - 1) / TMt, c1 = (h1 + TMt - 1) / TMt;
+    int s0 = h0, s1 = h1, u0 = c0, u1 = c1;  // inclusive scans over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a0 = __shfl_up_sync(0xffffffffu, s0, o), a1 = __shfl_up_sync(0xffffffffu, s1, o);
+      const int b0 = __shfl_up_sync(0xffffffffu, u0, o), b1 = __shfl_up_sync(0xffffffffu, u1, o);
+      if (lane >= o) { s0 += a0; s1 += a1; u0 += b0; u1 += b1; }
+    }
+    const int tot_h0 = __shfl_sync(0xffffffffu, s0, 31), tot_c0 = __shfl_sync(0xffffffffu, u0, 31);
+    const int ex0 = s0 - h0, ex1 = tot_h0 + s1 - h1;
+    const int tx0 = u0 - c0, tx1 = tot_c0 + u1 - c1;
+    if (lane < E) {
+      indptr[lane] = ex0; sx[lane] = ex0; tptr[lane] = tx0;
+      for (int m = 0; m < c0; ++m) { tile_e[tx0 + m] = lane; tile_m[tx0 + m] = m; }
+      if (S.dbg_hist) S.dbg_hist[lane] = h0;
+      if (S.dbg_indptr) S.dbg_indptr[lane] = ex0;
+    }
+    if (lane + 32 < E) {
+      indptr[lane + 32] = ex1; sx[lane + 32] = ex1; tptr[lane + 32] = tx1;
+      for (int m = 0; m < c1; ++m) { tile_e[tx1 + m] = lane + 32; tile_m[tx1 + m] = m; }
+      if (S.dbg_hist) S.dbg_hist[lane + 32] = h1;
+      if (S.dbg_indptr) S.dbg_indptr[lane + 32] = ex1;
+    }
+    if (lane == 31) {
+      const int rows = tot_h0 + s1, tiles = tot_c0 + u1;
+      indptr[E] = rows; sx[E] = rows; tptr[E] = tiles;
+      if (S.dbg_indptr) S.dbg_indptr[E] = rows;
+      // data-dependent event count: every down task of every tile notifies EV_MY
+      atomicExch(reinterpret_cast<int*>(ws + P.off_counters) + ev_ctr(P, EV_MY, 0), tiles * P.nt_d);
+    }
+  }
+  bar_sync(BAR_COMP, kComputeThreads);
+  const int* midx = reinterpret_cast<const int*>(ws + P.off_midx);
+  const int* mrank = reinterpret_cast<const int*>(ws + P.off_mrank);
+  int* mrow = reinterpret_cast<int*>(ws + P.off_mrow);
+  int* mperm = reinterpret_cast<int*>(ws + P.off_mperm);
+  const int npairs = S.B * K;
+  for (int p = ct; p < npairs; p += kComputeThreads) {
+    const int row = sx[__ldcg(midx + p)] + __ldcg(mrank + p);
+    mrow[p] = row;
+    mperm[row] = p;
+  }
+}
+
+// A GroupGEMM tile's geometry: expert, first row and row count.
+struct MoeTile { int e, r0, nrows; };
+__device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, unsigned char* ws, int tile) {
+  MoeTile m;
+  m.e = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_e) + tile);
+  const int mi = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_m) + tile);
+  const int h = __ldcg(reinterpret_cast<const int*>(ws + P.off_mhist) + m.e);
+  m.r0 = __ldcg(reinterpret_cast<const int*>(ws + P.off_mindptr) + m.e) + mi * P.moe_tm;
+  m.nrows = min(P.moe_tm, h - mi * P.moe_tm);
+  return m;
+}
+
+// EGU task (tile, n): warp w takes gate row n*tn + w and up row n*tn + w of
+// the tile's expert into registers (freeing its ring slots at once), then
+// runs them over the tile's rows: h[row] = silu(x W_g^T) * (x W_u^T), with x
+// gathered straight from the layer input by the row map.
+__device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
+                                         unsigned char* ws, Control* ctl, const TaskDesc& d) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int H = P.hidden, nblk = H >> 8, K = P.top_k;
+  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
+  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
+  const int rps = P.slot_bytes / (2 * H), spp = (P.moe_tn + rps - 1) / rps;
+  const int ja = w / rps, jb = spp + ja;
+  if (lane < d.nslots && lane != ja && lane != jb) {
+    const int j = s0 + lane;
+    mbar_arrive(&sm.empty[j < R ? j : j - R]);
+  }
+  const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R, sb = s0 + jb < R ? s0 + jb : s0 + jb - R;
+  wait_mbar(&sm.full[sa], s0 + ja < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  wait_mbar(&sm.full[sb], s0 + jb < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  const int roff = (w - ja * rps) * 2 * H;
+  const uint4* ga = reinterpret_cast<const uint4*>(ring + (size_t)sa * P.slot_bytes + roff) + lane;
+  const uint4* ua = reinterpret_cast<const uint4*>(ring + (size_t)sb * P.slot_bytes + roff) + lane;
+  uint4 gw[kMaxBlk], uw[kMaxBlk];
+#pragma unroll
+  for (int i = 0; i < kMaxBlk; ++i)
+    if (i < nblk) { gw[i] = ga[i * 32]; uw[i] = ua[i * 32]; }
+  __syncwarp();
+  if (lane == 0) { mbar_arrive(&sm.empty[sa]); mbar_arrive(&sm.empty[sb]); }
+  const int tile = d.idx / P.nt_gu, n = d.idx - tile * P.nt_gu;
+  const MoeTile mt = moe_tile(P, ws, tile);
+  const int* mperm = reinterpret_cast<const int*>(ws + P.off_mperm);
+  const uint4* xr = reinterpret_cast<const uint4*>(S.moe_x);
+  __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(ws + P.off_mh);
+  const int col = n * P.moe_tn + w;
+  for (int rr = 0; rr < mt.nrows; ++rr) {
+    const int row = mt.r0 + rr;
+    const int t = __ldcg(mperm + row) / K;
+    float ag[2] = {0.f, 0.f}, au[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < kMaxBlk; ++i)
+      if (i < nblk) {
+        float xf[8], gf[8], uf[8];
+        uint4 g4 = gw[i], u4 = uw[i];
+        // keep the weights packed: converting them once outside the row loop
+        // would hold 128 floats and spill
+        asm volatile("" : "+r"(g4.x), "+r"(g4.y), "+r"(g4.z), "+r"(g4.w), "+r"(u4.x), "+r"(u4.y), "+r"(u4.z), "+r"(u4.w));
+        bf16x8_to_f32(__ldg(xr + ((size_t)t * H + 256 * i + 8 * lane) / 8), xf);
+        bf16x8_to_f32(g4, gf);
+        bf16x8_to_f32(u4, uf);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          ag[j & 1] = fmaf(gf[j], xf[j], ag[j & 1]);
+          au[j & 1] = fmaf(uf[j], xf[j], au[j & 1]);
+        }
+      }
+    float g = ag[0] + ag[1], u = au[0] + au[1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      g += __shfl_xor_sync(0xffffffffu, g, o);
+      u += __shfl_xor_sync(0xffffffffu, u, o);
+    }
+    if (lane == 0 && col < P.eff) mh[(size_t)row * P.eff + col] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+  }
+}
+
+// EDOWN task (tile, n): warp w takes down row n*td + w (expert_ffn long, in
+// 8-element chunks c = lane + 32 i) into registers, then runs it over the
+// tile's rows of h: y[row][n*td + w] = h[row] . W_d[n*td + w].
+__device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
+                                           unsigned char* ws, Control* ctl, const TaskDesc& d) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int H = P.hidden, FF = P.eff, nch = FF / 8;
+  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
+  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
+  const int rps = P.slot_bytes / 4096;
+  const int ja = w / rps;
+  if (lane < d.nslots && lane != ja) {
+    const int j = s0 + lane;
+    mbar_arrive(&sm.empty[j < R ? j : j - R]);
+  }
+  const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R;
+  wait_mbar(&sm.full[sa], s0 + ja < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  const uint4* dr = reinterpret_cast<const uint4*>(ring + (size_t)sa * P.slot_bytes + (w - ja * rps) * 4096);
+  uint4 dw[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (lane + 32 * i < nch) dw[i] = dr[lane + 32 * i];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sm.empty[sa]);
+  const int tile = d.idx / P.nt_d, n = d.idx - tile * P.nt_d;
+  const MoeTile mt = moe_tile(P, ws, tile);
+  const uint4* mh = reinterpret_cast<const uint4*>(ws + P.off_mh);
+  float* my = reinterpret_cast<float*>(ws + P.off_my);
+  const int col = n * P.moe_td + w;
+  for (int rr = 0; rr < mt.nrows; ++rr) {
+    const int row = mt.r0 + rr;
+    float acc[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (lane + 32 * i < nch) {
+        float hf[8], wf[8];
+        uint4 d4 = dw[i];
+        asm volatile("" : "+r"(d4.x), "+r"(d4.y), "+r"(d4.z), "+r"(d4.w));  // convert per use (see task_egu)
+        bf16x8_to_f32(__ldcg(mh + ((size_t)row * FF) / 8 + lane + 32 * i), hf);
+        bf16x8_to_f32(d4, wf);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j & 1] = fmaf(wf[j], hf[j], acc[j & 1]);
+      }
+    const float v = warp_sum(acc[0] + acc[1]);
+    if (lane == 0) my[(size_t)row * H + col] = v;
+  }
+}
+
+// COMBINE: warp w takes token 8*idx + w: out[t] = sum_j w[t, j] * y[row(t, j)]
+// in slot order j = 0..k-1, written as bf16.
+__device__ __forceinline__ void task_combine(const DevPlan& P, const StepParams& S, unsigned char* ws,
+                                             const TaskDesc& d) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int H = P.hidden, K = P.top_k, nblk = H >> 8;
+  const int t = d.idx * 8 + w;
+  if (t >= S.B) return;
+  const int* mrow = reinterpret_cast<const int*>(ws + P.off_mrow);
+  const float* mw = reinterpret_cast<const float*>(ws + P.off_mw);
+  const float* my = reinterpret_cast<const float*>(ws + P.off_my);
+  int rows[8];
+  float wts[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < K) { rows[j] = __ldcg(mrow + (size_t)t * K + j); wts[j] = __ldcg(mw + (size_t)t * K + j); }
+  for (int i = 0; i < nblk; ++i) {
+    const int c = 256 * i + 8 * lane;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < K) {
+        const float4* y4 = reinterpret_cast<const float4*>(my + (size_t)rows[j] * H + c);
+        const float4 a = __ldcg(y4), b = __ldcg(y4 + 1);
+        acc[0] = fmaf(wts[j], a.x, acc[0]); acc[1] = fmaf(wts[j], a.y, acc[1]);
+        acc[2] = fmaf(wts[j], a.z, acc[2]); acc[3] = fmaf(wts[j], a.w, acc[3]);
+        acc[4] = fmaf(wts[j], b.x, acc[4]); acc[5] = fmaf(wts[j], b.y, acc[5]);
+        acc[6] = fmaf(wts[j], b.z, acc[6]); acc[7] = fmaf(wts[j], b.w, acc[7]);
+      }
+    __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) o[q] = __float2bfloat16_rn(acc[q]);
+    *reinterpret_cast<uint4*>(S.moe_out + (size_t)t * H + c) = *reinterpret_cast<const uint4*>(o);
+  }
+}
+
+template <bool kMoE>
 __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
                         Control* ctl) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int B = S.B;
   int a_tag = -1;
-  ActRegs av;
   for (uint32_t k = 0;; ++k) {
     // task k: released into cur[k & 1] as phase k >> 1 of go_bar[k & 1]
     if (!wait_mbar(&sm.go_bar[k & 1], (k >> 1) & 1, ctl, P.spin_timeout_ns, -1, -1)) break;
@@ -1254,15 +1623,30 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     uint32_t* trec = (d.rec > 0 && w == 0) ? trace_rec(S, d.rec) : nullptr;
     if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
     GemvSpec g;
-    if (gemv_spec(P, d, g)) {
+    if constexpr (kMoE) {
+      if (d.op == OP_ROUTE) {
+        task_route(P, S, sm, ws, d);
+      } else if (d.op == OP_MINDPTR) {
+        task_mindptr(P, S, sm, ws);
+      } else if (d.op == OP_EGU) {
+        task_egu(P, S, sm, ring, ws, ctl, d);
+      } else if (d.op == OP_EDOWN) {
+        task_edown(P, S, sm, ring, ws, ctl, d);
+      } else if (d.op == OP_COMBINE) {
+        task_combine(P, S, ws, d);
+      }
+    } else if (gemv_spec(P, d, g)) {
       // one pass per batch row (the activation is restaged each pass when
       // B > 1); the ring slots are released after the last pass
       for (int b = 0; b < B; ++b) {
         if (B > 1 || g.tag != a_tag) {
           stage_act(P, ws, sm, g, b);
-          act_to_regs(sm.xs, g.K >> 8, av);
           a_tag = B > 1 ? -1 : g.tag;
         }
+        // the activation's registers live within one task (reloaded from the
+        // staged copy), so no other task body has to keep them
+        ActRegs av;
+        act_to_regs(sm.xs, g.K >> 8, av);
         warp_gemv_task(P, S, sm, ring, ws, ctl, d, g, av, b, trec, b == B - 1);
       }
     } else if (d.op == OP_ATTN) {
@@ -1297,8 +1681,14 @@ __device__ __forceinline__ void arm_events(const DevPlan& P, Smem& sm, const Fam
   }
   const int gtid = blockIdx.x * blockDim.x + tid, gthreads = gridDim.x * blockDim.x;
   for (int i = gtid; i < P.n_counters; i += gthreads) {
+    // the event tensor holding counter i (tensors a plan does not use are empty)
     int e = 0;
-    while (e + 1 < EV_COUNT && i >= P.ev[e + 1].base) ++e;
+    for (; e < EV_COUNT; ++e) {
+      const EventTensorDesc& d = P.ev[e];
+      const int size = d.ndim < 1 ? 0 : d.dims[0] * (d.ndim > 1 ? d.dims[1] : 1) * (d.ndim > 2 ? d.dims[2] : 1);
+      if (i >= d.base && i < d.base + size) break;
+    }
+    if (e == EV_COUNT) continue;
     int lin = i - P.ev[e].base;
     ExprEnv env{B, sm.ctx, {0, 0, 0}};
     for (int dd = P.ev[e].ndim - 1; dd >= 0; --dd) { env.coord[dd] = lin % P.ev[e].dims[dd]; lin /= P.ev[e].dims[dd]; }
@@ -1306,6 +1696,10 @@ __device__ __forceinline__ void arm_events(const DevPlan& P, Smem& sm, const Fam
   }
 }
 
+// One persistent kernel per plan kind: the instances share the interpreter
+// (producer, controller, notifier) and differ in the task bodies compiled in
+// (dense decoder or MoE layer), so each gets its own register allocation.
+template <bool kMoE>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const StepParams S, unsigned char* ws) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring = smem_raw;
@@ -1318,14 +1712,15 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   const int B = S.B;
 
   // ---- prologue: resolve the symbols, arm the Event Tensors, gather embeddings
+  const bool moe = P.kind == MK_MODEL_MOE_LAYER;
   if (tid == 0) {
-    sm.bad = (B < 1 || B > P.max_batch || B > kMaxB) ? 1 : 0;
+    sm.bad = moe ? (B < 1 || B > P.max_tokens) : (B < 1 || B > P.max_batch || B > kMaxB);
     sm.released = 0;
     sm.dq_head = sm.dq_tail = sm.fq_head = sm.fq_tail = sm.notifier_stop = 0;
   }
   if (tid < kComputeWarps * kMaxB) sm.lm_seen[tid / kMaxB][tid % kMaxB] = 0ull;
   __syncthreads();
-  if (!sm.bad && tid < B) {
+  if (!moe && !sm.bad && tid < B) {
     int c = S.ctx[tid], s = S.slots[tid], t = S.tokens[tid];
     sm.ctx[tid] = c; sm.slot[tid] = s; sm.tok[tid] = t;
     if (c < 0 || c >= P.max_ctx || s < 0 || s >= P.n_slots || t < 0 || t >= P.vocab) atomicOr(&sm.bad, 1);
@@ -1350,23 +1745,29 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
       gg.spp = ceil_div(rows_part, rps);
       gg.pairs = pairs;
     };
-    set_geo(OP_QKV, P.hidden, P.tile_qkv / 2, 1);
-    set_geo(OP_OPROJ, P.hidden, P.tile_o, 0);
-    set_geo(OP_GATEUP, P.hidden, P.tile_gu, 1);
-    set_geo(OP_DOWN, P.kseg, P.tile_down, 0);
-    set_geo(OP_LM, P.hidden, P.tile_lm, 0);
-    int run = 0;
-    for (int b = 0; b < B; ++b) {
-      sm.pre[b] = run;
-      sm.nch[b] = ceil_div(sm.ctx[b] + 1, P.chunk);
-      run += sm.nch[b];
+    if (!moe) {
+      set_geo(OP_QKV, P.hidden, P.tile_qkv / 2, 1);
+      set_geo(OP_OPROJ, P.hidden, P.tile_o, 0);
+      set_geo(OP_GATEUP, P.hidden, P.tile_gu, 1);
+      set_geo(OP_DOWN, P.kseg, P.tile_down, 0);
+      set_geo(OP_LM, P.hidden, P.tile_lm, 0);
     }
-    sm.pre[B] = run;
+    if (!moe) {
+      int run = 0;
+      for (int b = 0; b < B; ++b) {
+        sm.pre[b] = run;
+        sm.nch[b] = ceil_div(sm.ctx[b] + 1, P.chunk);
+        run += sm.nch[b];
+      }
+      sm.pre[B] = run;
+    }
   }
   __syncthreads();
   arm_events(P, sm, fams, code, counters, B);
   const int gtid = blockIdx.x * blockDim.x + tid, gthreads = gridDim.x * blockDim.x;
-  {
+  if (moe) {
+    if (blockIdx.x == 0 && tid < P.n_experts) reinterpret_cast<int*>(ws + P.off_mhist)[tid] = 0;
+  } else {
     float* x = reinterpret_cast<float*>(ws + P.off_x);
     const int cpr = P.hidden / 8;
     for (int i = gtid; i < B * cpr; i += gthreads) {
@@ -1384,7 +1785,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   if (blockIdx.x == 0 && tid == 0 && P.sched == MK_SCHED_DYNAMIC) {
     ctl->q_head = 0;
     ctl->q_tail = 0;
-    push_range(P, S, ctl, ws, fam_of(P, OP_QKV, 0), 0, P.n_qkv_tiles);  // EV_IN[0] is armed at zero
+    if (moe) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, -1), 0, ceil_div(B, 8));
+    else push_range(P, S, ctl, ws, fam_of(P, OP_QKV, 0), 0, P.n_qkv_tiles);  // EV_IN[0] is armed at zero
   }
   if (tid == 0) {
     for (int s = 0; s < P.ring_slots; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], kComputeWarps); }
@@ -1417,7 +1819,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   } else if (warp == 2) {
     notifier(P, S, sm, ws, ctl, counters);
   } else {
-    compute(P, S, sm, ring, ws, ctl);
+    compute<kMoE>(P, S, sm, ring, ws, ctl);
   }
 }
 
@@ -1427,6 +1829,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
 #include "launch.hpp"
 
 namespace mk {
+
+static const void* kernel_for(const DevPlan& P) {
+  return P.kind == MK_MODEL_MOE_LAYER ? (const void*)megakernel<true> : (const void*)megakernel<false>;
+}
 
 mk_status dev_query(int* n_sm, int* smem_optin, int* device, std::string& err) {
   int dev = 0;
@@ -1447,10 +1853,11 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
                    std::string& err) {
   cudaStream_t s = (cudaStream_t)stream;
   size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + sizeof(Smem);
-  cudaError_t e = cudaFuncSetAttribute(megakernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const void* kern = kernel_for(p.dp);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) {
     int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, megakernel, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, smem);
     if (e == cudaSuccess && nb < 1) { err = "megakernel does not fit on an SM"; return MK_ERR_UNSUPPORTED; }
   }
   if (e == cudaSuccess)
@@ -1468,7 +1875,7 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
 }
 
 mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& err) {
-  StepParams sp;
+  StepParams sp = StepParams();
   sp.B = a->batch;
   sp.tokens = a->token_ids;
   sp.slots = a->slot_ids;
@@ -1483,7 +1890,7 @@ mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& 
   unsigned char* ws = (unsigned char*)p.ws;
   DevPlan dp = p.dp;
   void* args[] = {(void*)&dp, (void*)&sp, (void*)&ws};
-  cudaError_t e = cudaLaunchCooperativeKernel((const void*)megakernel, dim3(p.dp.n_sm), dim3(kThreads), args,
+  cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(p.dp.n_sm), dim3(kThreads), args,
                                               (size_t)p.dp.smem_bytes, (cudaStream_t)stream);
   if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   p.epoch++;
@@ -1541,10 +1948,10 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   const size_t smem = (size_t)P0.ring_slots * P0.slot_bytes + sizeof(Smem);
   if (st.owner != p.uid) {
     st.owner = 0;
-    e = cudaFuncSetAttribute(megakernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(kernel_for(P0), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess) {
       int nb = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, megakernel, kThreads, smem);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel_for(P0), kThreads, smem);
       if (e == cudaSuccess && nb < 1) { err = "megakernel does not fit on an SM"; return MK_ERR_UNSUPPORTED; }
     }
     // the read-only plan arrays, copied from the plan's own host vectors
@@ -1565,7 +1972,7 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   if (e == cudaSuccess) e = cudaMemsetAsync(ws + P0.off_queue, 0, sizeof(QRange) * (size_t)P0.queue_ranges, s);
   if (e != cudaSuccess) { err = std::string("scratch clear failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
 
-  StepParams sp;
+  StepParams sp = StepParams();
   sp.B = a->batch;
   sp.tokens = a->token_ids;
   sp.slots = a->slot_ids;
@@ -1580,8 +1987,31 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   DevPlan dp = P0;
   dp.smem_bytes = (int)smem;
   void* args[] = {(void*)&dp, (void*)&sp, (void*)&ws};
-  e = cudaLaunchCooperativeKernel((const void*)megakernel, dim3(dp.n_sm), dim3(kThreads), args, smem, s);
+  e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(dp.n_sm), dim3(kThreads), args, smem, s);
   if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
+  return MK_OK;
+}
+
+mk_status dev_launch_moe(Plan& p, const mk_moe_args* a, void* stream, std::string& err) {
+  StepParams sp = StepParams();
+  sp.B = a->n_tokens;
+  sp.moe_x = reinterpret_cast<const __nv_bfloat16*>(a->x);
+  sp.moe_out = reinterpret_cast<__nv_bfloat16*>(a->out);
+  sp.dbg_idx = a->topk_idx;
+  sp.dbg_w = a->topk_w;
+  sp.dbg_hist = a->hist;
+  sp.dbg_indptr = a->indptr;
+  sp.dbg_logits = a->logits;
+  sp.task_counts = a->task_counts;
+  sp.epoch = p.epoch + 1;
+  unsigned char* ws = (unsigned char*)p.ws;
+  DevPlan dp = p.dp;
+  void* args[] = {(void*)&dp, (void*)&sp, (void*)&ws};
+  cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(p.dp.n_sm), dim3(kThreads), args,
+                                              (size_t)p.dp.smem_bytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
+  p.epoch++;
+  p.launches++;
   return MK_OK;
 }
 

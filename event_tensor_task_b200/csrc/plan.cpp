@@ -31,8 +31,8 @@
 
 namespace mk {
 
-static const char* kOpNames[OP_COUNT] = {"end", "qkv", "attn", "merge", "oproj", "gateup",
-                                         "down", "-", "lm", "-", "lmfin"};
+static const char* kOpNames[OP_COUNT] = {"end", "qkv", "attn", "merge", "oproj", "gateup", "down", "-", "lm",
+                                         "-", "lmfin", "route", "mindptr", "egu", "edown", "combine", "mfin"};
 static const int kLayerOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_GATEUP, OP_DOWN};
 static const int kLmOps[] = {OP_LM, OP_LMFIN};
 static constexpr int kFamPerLayer = 6;
@@ -235,10 +235,116 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
 // ---------------------------------------------------------------- build
 static bool pow2_divides(int a, int b) { return a > 0 && b % a == 0; }
 
+// MoE FFN layer ("Event Tensor: A Unified Abstraction for Compiling Dynamic
+// Megakernel", section "Core method", data-dependent dynamism).  The task
+// graph: ROUTE (8 tokens each) -> follow-up MINDPTR (exp_indptr, tile table,
+// row map; arms the count of EV_MY) -> EGU tiles, as many as exp_indptr
+// implies -> per tile, EDOWN tasks -> COMBINE -> follow-up MFIN.  Task counts
+// after ROUTE depend on the routing, so the layer runs on the dynamic queue.
+static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, int smem_bytes,
+                                Plan& p, std::string& err) {
+  const int H = m->hidden, E = m->n_experts, K = m->top_k, FF = m->expert_ffn, TM = m->max_tokens;
+  if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
+  if (E < 1 || E > 64) { err = "n_experts must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
+  if (K < 1 || K > 8 || K > E) { err = "top_k must be in [1, min(8, n_experts)]"; return MK_ERR_UNSUPPORTED; }
+  if (FF < 8 || FF % 8 || FF > 2048) { err = "expert_ffn must be a multiple of 8 in [8, 2048]"; return MK_ERR_UNSUPPORTED; }
+  if (TM < 1 || TM > 4096) { err = "max_tokens must be in [1, 4096]"; return MK_ERR_UNSUPPORTED; }
+  if (o->sched != MK_SCHED_DYNAMIC)
+    { err = "an MoE layer's task counts depend on the routing: use MK_SCHED_DYNAMIC"; return MK_ERR_UNSUPPORTED; }
+  if (n_sm < 1 || n_sm > 1024) { err = "n_sm out of range"; return MK_ERR_INVALID_ARG; }
+  p.m = *m;
+  p.m.layers = nullptr;
+  p.o = *o;
+  p.layer_w.clear();
+  DevPlan& P = p.dp;
+  P = DevPlan();
+  P.kind = MK_MODEL_MOE_LAYER;
+  P.sched = o->sched;
+  P.n_sm = n_sm;
+  P.hidden = H;
+  P.debug_flags = o->debug_flags;
+  P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
+  P.n_experts = E; P.top_k = K; P.eff = FF; P.max_tokens = TM;
+  P.moe_tm = 64;  // routed rows per GroupGEMM tile
+  P.moe_tn = 8;   // one gate/up row pair per compute warp
+  P.moe_td = 8;   // one down row per compute warp
+  P.nt_gu = ceil_div(FF, P.moe_tn);
+  P.nt_d = H / P.moe_td;
+  // sum over experts of ceil(hist_e / tm) <= T*k/tm + (experts with a row)
+  P.max_tiles = ceil_div(TM * K, P.moe_tm) + std::min(E, TM * K);
+  if (FF % P.moe_tn) { err = "expert_ffn must be a multiple of 8"; return MK_ERR_UNSUPPORTED; }
+  P.slot_bytes = 16384;
+  const int reserve = 19 * 1024;
+  P.smem_bytes = smem_bytes;
+  P.ring_slots = std::min(16, (smem_bytes - reserve) / P.slot_bytes);
+  if (P.ring_slots < 5) { err = "not enough shared memory for a 5-slot ring"; return MK_ERR_UNSUPPORTED; }
+
+  p.code.clear();
+  p.fams.clear();
+  p.fam_names.clear();
+  int debug_base = 0;
+  auto add_family = [&](int op, int extent_expr, int max_extent, int followup) {
+    FamilyDesc f{};
+    f.op = op; f.layer = -1; f.extent_expr = extent_expr; f.max_extent = max_extent;
+    f.debug_base = debug_base; f.followup = followup;
+    debug_base += max_extent;
+    P.fam_first_layer[op] = (int)p.fams.size();
+    p.fams.push_back(f);
+    p.fam_names.push_back(kOpNames[op]);
+  };
+  for (int op = 0; op < OP_COUNT; ++op) P.fam_first_layer[op] = -1;
+  const int e_tok8 = Emit(p.code).op(X_B).push(8).op(X_CEILDIV).ret();  // ceil(T / 8); B stands for T
+  add_family(OP_ROUTE, e_tok8, ceil_div(TM, 8), 0);
+  add_family(OP_MINDPTR, emit_const(p.code, 1), 1, 1);
+  // the extents below are set by the routing; the expressions give the maxima
+  add_family(OP_EGU, emit_const(p.code, P.max_tiles * P.nt_gu), P.max_tiles * P.nt_gu, 0);
+  add_family(OP_EDOWN, emit_const(p.code, P.max_tiles * P.nt_d), P.max_tiles * P.nt_d, 0);
+  add_family(OP_COMBINE, e_tok8, ceil_div(TM, 8), 0);
+  add_family(OP_MFIN, emit_const(p.code, 1), 1, 1);
+  P.n_families = (int)p.fams.size();
+  P.debug_slots = debug_base;
+  P.fam_stride = 0;
+
+  int base = 0;
+  const int e_zero = emit_const(p.code, 0);
+  for (int id = 0; id < EV_ROUTE; ++id) {  // the dense decoder's events are empty
+    EventTensorDesc& e = P.ev[id];
+    e.base = 0; e.ndim = 1; e.dims[0] = 0; e.dims[1] = e.dims[2] = 1; e.count_expr = e_zero;
+  }
+  auto add_event = [&](int id, int d0, int count_expr) {
+    EventTensorDesc& e = P.ev[id];
+    e.base = base; e.ndim = 1; e.dims[0] = d0; e.dims[1] = e.dims[2] = 1; e.count_expr = count_expr;
+    base += d0;
+  };
+  add_event(EV_ROUTE, 1, e_tok8);
+  add_event(EV_MIDX, 1, emit_const(p.code, 1));
+  add_event(EV_MH, P.max_tiles, emit_const(p.code, P.nt_gu));
+  add_event(EV_MY, 1, emit_const(p.code, 1 << 30));  // replaced at run time by MINDPTR
+  add_event(EV_MCOMB, 1, e_tok8);
+  P.n_counters = base;
+
+  // no static instructions: one END per CTA
+  P.n_instr_per_sm = 1;
+  p.instr.assign((size_t)n_sm, Instr{-1, 0, 1, 0});
+  // pushes per launch: ROUTE, EGU, one EDOWN range per tile, COMBINE, END
+  P.queue_ranges = P.max_tiles + 8;
+  p.layers.clear();
+  p.rope.clear();
+  P.w_router = m->moe.w_router;
+  P.router_bias = m->moe.router_bias;
+  P.w_egate = m->moe.w_gate;
+  P.w_eup = m->moe.w_up;
+  P.w_edown = m->moe.w_down;
+  std::vector<unsigned char> image;
+  lower_plan(p, image);
+  return MK_OK;
+}
+
 mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, int smem_bytes,
                      Plan& p, std::string& err) {
   if (!m || !o) { err = "null model or options"; return MK_ERR_INVALID_ARG; }
-  if (m->kind != MK_MODEL_DENSE) { err = "only MK_MODEL_DENSE plans are implemented"; return MK_ERR_UNSUPPORTED; }
+  if (m->kind == MK_MODEL_MOE_LAYER) return build_moe_plan(m, o, n_sm, smem_bytes, p, err);
+  if (m->kind != MK_MODEL_DENSE) { err = "unknown model kind"; return MK_ERR_UNSUPPORTED; }
   const int H = m->hidden, D = m->head_dim, Hq = m->n_q_heads, Hkv = m->n_kv_heads, F = m->ffn;
   if (m->n_layers < 1 || m->vocab < 1 || Hkv < 1 || Hq < 1) { err = "non-positive dimension"; return MK_ERR_INVALID_ARG; }
   if (D != 64) { err = "head_dim must be 64"; return MK_ERR_UNSUPPORTED; }
@@ -395,6 +501,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   add_event(EV_O, 1, L, 1, 1, emit_const(p.code, P.n_otiles));
   add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu));
   add_event(EV_LM, 1, 1, 1, 1, emit_const(p.code, P.n_lm_tiles));
+  for (int id = EV_LM + 1; id < EV_COUNT; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // MoE: empty
   P.n_counters = base;
 
   // ---- static schedule: per-SM queues of block instructions in topological
@@ -453,7 +560,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
 // ---------------------------------------------------------------- lowering
 void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   DevPlan& P = p.dp;
-  const int qpg = P.n_q_heads / P.n_kv_heads;
+  const int qpg = P.n_kv_heads > 0 ? P.n_q_heads / P.n_kv_heads : 0;  // 0 for an MoE layer
   long long off = 0;
   auto take = [&](long long bytes) { long long at = off; off += (bytes + 255) / 256 * 256; return at; };
   P.off_control = take(sizeof(Control));
@@ -471,6 +578,21 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_h = take(4LL * P.max_batch * P.ffn);
   P.off_dpart = take(4LL * P.n_kc * P.max_batch * P.hidden);
   P.off_lmbest = take(8LL * P.max_batch);
+  if (P.kind == MK_MODEL_MOE_LAYER) {
+    const long long pairs = (long long)P.max_tokens * P.top_k;
+    P.off_mhist = take(4LL * P.n_experts);
+    P.off_mrank = take(4 * pairs);
+    P.off_midx = take(4 * pairs);
+    P.off_mw = take(4 * pairs);
+    P.off_mindptr = take(4LL * (P.n_experts + 1));
+    P.off_mtile = take(4LL * (P.n_experts + 1));
+    P.off_mtile_e = take(4LL * P.max_tiles);
+    P.off_mtile_m = take(4LL * P.max_tiles);
+    P.off_mperm = take(4 * pairs);
+    P.off_mrow = take(4 * pairs);
+    P.off_mh = take(2 * pairs * P.eff);
+    P.off_my = take(4 * pairs * P.hidden);
+  }
   P.ws_bytes = off;
   // image = [off_families, off_queue): the read-only plan arrays
   image.assign((size_t)(P.off_queue - P.off_families), 0);
@@ -487,6 +609,7 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
 // ---------------------------------------------------------------- bytes
 double step_bytes(const Plan& p, const Binding& bd, bool with_logits) {
   const DevPlan& P = p.dp;
+  if (P.kind != MK_MODEL_DENSE) return -1.0;  // MoE bytes depend on the routing
   double H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads, F = P.ffn;
   double per_layer = ((Hq + 2 * Hkv) * D * H + H * Hq * D + 3 * F * H + 2 * H) * 2.0;
   double w = P.n_layers * per_layer + (double)P.vocab * H * 2.0 + H * 2.0;
@@ -508,6 +631,10 @@ static bool check_binding(const Plan& p, const Binding& bd, std::string& err) {
 }
 
 mk_status validate_plan(const Plan& p, const Binding& bd, std::string& err) {
+  if (p.dp.kind != MK_MODEL_DENSE) {
+    err = "the host task model covers the dense decoder; an MoE layer's graph depends on its routing";
+    return MK_ERR_UNSUPPORTED;
+  }
   if (!check_binding(p, bd, err)) return MK_ERR_INVALID_ARG;
   const DevPlan& P = p.dp;
   std::vector<int> notifiers(P.n_counters, 0);
@@ -778,6 +905,10 @@ mk_status simulate_plan(const Plan& p, const Binding& bd, int n_orders, unsigned
                         int fault_family, mk_sim_report* rep) {
   std::string err;
   std::memset(rep, 0, sizeof(*rep));
+  if (p.dp.kind != MK_MODEL_DENSE) {
+    std::snprintf(rep->first_error, sizeof(rep->first_error), "simulation covers the dense decoder only");
+    return MK_ERR_UNSUPPORTED;
+  }
   if (!check_binding(p, bd, err)) {
     std::snprintf(rep->first_error, sizeof(rep->first_error), "%s", err.c_str());
     return MK_ERR_INVALID_ARG;

@@ -35,7 +35,14 @@ enum Op : int32_t {
   OP_LM = 8,      // final RMSNorm -> vocabulary rows -> logits + running argmax
                   // (9 is unused)
   OP_LMFIN = 10,  // follow-up: the running argmax -> next token
-  OP_COUNT = 11
+  // mixture-of-experts FFN layer (data-dependent task graph, dynamic schedule)
+  OP_ROUTE = 11,    // 8 tokens: router logits -> top-k, weights, per-expert ranks
+  OP_MINDPTR = 12,  // follow-up: exp_indptr, tile table, row map, data-dependent counts
+  OP_EGU = 13,      // GroupGEMM tile: an expert's gate/up rows x its routed rows -> SwiGLU
+  OP_EDOWN = 14,    // GroupGEMM tile: an expert's down rows x its routed rows
+  OP_COMBINE = 15,  // 8 tokens: weighted sum of their top-k expert outputs
+  OP_MFIN = 16,     // follow-up: end of the layer
+  OP_COUNT = 17
 };
 
 // ---------------------------------------------------------------- expressions
@@ -126,7 +133,13 @@ enum EvId : int32_t {
   EV_O = 4,      // [L]          output projection done
   EV_GU = 5,     // [L][n_kc]    SwiGLU outputs of one K segment written
   EV_LM = 6,     // [1]          all LM tiles done
-  EV_COUNT = 7
+  // MoE layer
+  EV_ROUTE = 7,  // [1]          all ROUTE tasks done
+  EV_MIDX = 8,   // [1]          exp_indptr and the tile table written
+  EV_MH = 9,     // [max_tiles]  SwiGLU rows of one GroupGEMM tile written (all its gate/up tasks)
+  EV_MY = 10,    // [1]          all down tasks done (count set at run time from exp_indptr)
+  EV_MCOMB = 11, // [1]          all COMBINE tasks done
+  EV_COUNT = 12
 };
 
 struct EventTensorDesc {
@@ -195,6 +208,18 @@ struct DevPlan {
   // global weights (device)
   const void* embed; const void* lm_head; const void* final_norm;
   void* k_cache; void* v_cache;
+  // MoE layer (kind MK_MODEL_MOE_LAYER)
+  int32_t kind;
+  int32_t n_experts, top_k, eff, max_tokens;
+  int32_t moe_tm;     // routed rows per GroupGEMM tile
+  int32_t moe_tn;     // gate/up row pairs per EGU task
+  int32_t moe_td;     // down rows per EDOWN task
+  int32_t nt_gu, nt_d, max_tiles;
+  int32_t pad2;
+  const void* w_router; const float* router_bias;
+  const void* w_egate; const void* w_eup; const void* w_edown;
+  int64_t off_mhist, off_mrank, off_midx, off_mw, off_mindptr, off_mtile, off_mtile_e, off_mtile_m;
+  int64_t off_mperm, off_mrow, off_mh, off_my;
 };
 
 // Control block at off_control (first 256 bytes of the workspace).

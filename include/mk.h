@@ -49,6 +49,7 @@ typedef int mk_status;
 #define MK_SCHED_DYNAMIC 1  /* shared device queue; a task is pushed when its event fires */
 
 #define MK_MODEL_DENSE 0     /* dense decoder: attention + SwiGLU FFN per layer */
+#define MK_MODEL_MOE_LAYER 1 /* one mixture-of-experts FFN layer (mk_moe_layer); dynamic schedule only */
 
 #define MK_DEBUG_TASK_COUNTS 1u  /* each executed task increments its slot in mk_step_args.task_counts */
 #define MK_DEBUG_TRACE 2u        /* the controller records per-task timestamps in mk_step_args.trace */
@@ -66,11 +67,23 @@ typedef struct mk_layer_weights {
   const void* w_down;     /* [hidden][ffn] */
 } mk_layer_weights;
 
-/* Model description.  Dimensions must satisfy: head_dim == 64,
- * n_q_heads % n_kv_heads == 0, hidden and ffn multiples of 256 with
- * hidden <= 2048, n_q_heads*head_dim == hidden. */
+/* Weights of one mixture-of-experts FFN layer; bf16 row-major, device. */
+typedef struct mk_moe_weights {
+  const void* w_router;      /* [n_experts][hidden] */
+  const float* router_bias;  /* fp32 [n_experts] added to the router logits, or NULL */
+  const void* w_gate;        /* [n_experts][expert_ffn][hidden] */
+  const void* w_up;          /* [n_experts][expert_ffn][hidden] */
+  const void* w_down;        /* [n_experts][hidden][expert_ffn] */
+} mk_moe_weights;
+
+/* Model description.
+ * MK_MODEL_DENSE: head_dim == 64, n_q_heads % n_kv_heads == 0, hidden and
+ *   ffn multiples of 256 with hidden <= 2048, n_q_heads*head_dim == hidden.
+ * MK_MODEL_MOE_LAYER: only hidden (multiple of 256, <= 2048), n_experts
+ *   (<= 64), top_k (<= 8 and <= n_experts), expert_ffn (multiple of 8,
+ *   <= 2048), max_tokens (<= 4096) and moe are read. */
 typedef struct mk_model_desc {
-  int kind;               /* MK_MODEL_DENSE */
+  int kind;               /* MK_MODEL_DENSE or MK_MODEL_MOE_LAYER */
   int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
   float eps;              /* RMSNorm epsilon */
   float rope_theta;       /* rotary base; pair i of a head turns by pos*theta^(-2i/head_dim) */
@@ -83,6 +96,8 @@ typedef struct mk_model_desc {
   const mk_layer_weights* layers; /* host array [n_layers] of device pointers */
   void* k_cache;          /* bf16 [n_layers][n_slots][n_kv_heads][max_ctx][head_dim], device, post-RoPE keys */
   void* v_cache;          /* bf16, same layout as k_cache */
+  int n_experts, top_k, expert_ffn, max_tokens;  /* MK_MODEL_MOE_LAYER */
+  mk_moe_weights moe;     /* MK_MODEL_MOE_LAYER */
 } mk_model_desc;
 
 /* Plan options; zero-initialise and set what you need (0 = default). */
@@ -115,6 +130,20 @@ typedef struct mk_step_args {
   int trace_cap;          /* records per CTA in `trace` */
 } mk_step_args;
 
+/* Arguments of one MoE layer call (MK_MODEL_MOE_LAYER).  All arrays are
+ * device memory; the debug outputs may be NULL. */
+typedef struct mk_moe_args {
+  int n_tokens;           /* T, 1 <= T <= max_tokens */
+  const void* x;          /* bf16 [T][hidden]: the layer input */
+  void* out;              /* bf16 [T][hidden]: sum over the token's top_k experts of weight * expert FFN */
+  int* topk_idx;          /* int32 [T][top_k]: selected experts, largest logit first, ties -> lower id */
+  float* topk_w;          /* fp32 [T][top_k]: softmax of the selected logits */
+  int* hist;              /* int32 [n_experts]: (token, slot) pairs per expert */
+  int* indptr;            /* int32 [n_experts + 1]: exclusive prefix sum of hist */
+  float* logits;          /* fp32 [T][n_experts]: router logits (bias included) */
+  unsigned* task_counts;  /* uint32 [mk_plan_task_slots()] or NULL (MK_DEBUG_TASK_COUNTS); zeroed by the caller */
+} mk_moe_args;
+
 typedef struct mk_device_status {
   int code;               /* MK_OK or MK_ERR_DEVICE_* */
   int family;             /* family index of the task that failed, or -1 */
@@ -140,6 +169,12 @@ typedef struct mk_family_info {
 #define MK_OP_DOWN 6
 #define MK_OP_LM 8
 #define MK_OP_LMFIN 10
+#define MK_OP_ROUTE 11    /* router logits, top-k, softmax weights, per-expert ranks (8 tokens per task) */
+#define MK_OP_MINDPTR 12  /* follow-up: exp_indptr, GroupGEMM tile table, row map, data-dependent event counts */
+#define MK_OP_EGU 13      /* GroupGEMM tile: gate/up rows of one expert x its routed rows -> SwiGLU */
+#define MK_OP_EDOWN 14    /* GroupGEMM tile: down rows of one expert x its routed rows */
+#define MK_OP_COMBINE 15  /* weighted sum of each token's top_k expert outputs (8 tokens per task) */
+#define MK_OP_MFIN 16     /* follow-up: end of the layer */
 
 typedef struct mk_sim_report {
   int orders_run;         /* random interleavings executed */
@@ -212,6 +247,19 @@ mk_status mk_decode_step(mk_plan* p, const mk_step_args* a, void* stream);
  *    workspace to read the code with mk_get_status.
  * Arguments and launch errors as for mk_decode_step. */
 mk_status mk_decode_step_static(mk_plan* p, const mk_step_args* a, void* stream);
+
+/* One mixture-of-experts FFN layer on T tokens: a single launch of the
+ * persistent megakernel on `stream` ("Event Tensor: A Unified Abstraction for
+ * Compiling Dynamic Megakernel", section "Core method", data-dependent
+ * dynamism).  ROUTE tasks compute the router logits, the top_k experts and
+ * their softmax weights and count (token, slot) pairs per expert; the task
+ * that completes the routing event computes exp_indptr and the GroupGEMM tile
+ * table and arms the data-dependent event counts, and the number of gate/up
+ * tiles pushed is the one exp_indptr implies; each tile's down tasks wait on
+ * that tile's event.  Requires a plan of kind MK_MODEL_MOE_LAYER with
+ * MK_SCHED_DYNAMIC and a bound workspace.  Asynchronous; device errors are
+ * read with mk_get_status. */
+mk_status mk_moe_layer(mk_plan* p, const mk_moe_args* a, void* stream);
 
 /* Read the device status word (synchronous copy).  Returns the recorded
  * device code (MK_OK if none).  After a device error, call mk_plan_reset. */

@@ -26,11 +26,11 @@ from .dense import (rms_norm, rope_cos_sin, apply_rope, decode_attention, swiglu
                     bf16_round, DenseOracle)
 from .moe import (router_logits, topk_route, expert_histogram, exp_indptr,
                   moe_ffn, moe_layer)
-from .tasks import expected_dense_tasks, dense_family_extents
+from .tasks import expected_dense_tasks, dense_family_extents, expected_moe_tasks, moe_tiles
 
 __all__ = [
     "rms_norm", "rope_cos_sin", "apply_rope", "decode_attention", "swiglu",
     "bf16_round", "DenseOracle", "router_logits", "topk_route",
     "expert_histogram", "exp_indptr", "moe_ffn", "moe_layer",
-    "expected_dense_tasks", "dense_family_extents",
+    "expected_dense_tasks", "dense_family_extents", "expected_moe_tasks", "moe_tiles",
 ]

@@ -73,3 +73,43 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
     for fam in ("lm", "lmfin"):
         out.update((fam, -1, i) for i in range(ext[fam]))
     return out
+
+
+def moe_tiles(hist, tm: int):
+    """GroupGEMM tiles of an MoE layer: expert ``e``'s ``hist[e]`` rows split
+    into ``ceil(hist[e] / tm)`` tiles of at most ``tm`` rows, numbered expert
+    by expert in increasing expert id ("Event Tensor: A Unified Abstraction
+    for Compiling Dynamic Megakernel", section "Core method": the prefix sum
+    of the per-expert counts decides how many GroupGEMM tiles each expert
+    triggers).  Returns ``[(expert, first row, rows), ...]`` with rows
+    counted from ``exp_indptr[e]``."""
+    tiles, row = [], 0
+    for e, h in enumerate(int(v) for v in hist):
+        for m in range(_ceil(h, tm)):
+            tiles.append((e, row + m * tm, min(tm, h - m * tm)))
+        row += h
+    return tiles
+
+
+def expected_moe_tasks(T: int, hist, hidden: int, expert_ffn: int, tiles: dict) -> set:
+    """The set of ``(family, -1, index)`` one MoE layer call runs exactly once.
+
+    ``route`` and ``combine``: ``ceil(T / 8)`` each (8 tokens per task);
+    ``mindptr`` and ``mfin``: one each; ``egu``: ``tiles * ceil(F / tn)``
+    numbered ``tile * ceil(F / tn) + n``; ``edown``: ``tiles * (H / td)``
+    numbered ``tile * (H / td) + n``.
+    """
+    n_tiles = len(moe_tiles(hist, tiles["tm"]))
+    nt_gu = _ceil(expert_ffn, tiles["tn"])
+    nt_d = hidden // tiles["td"]
+    out = set()
+    for i in range(_ceil(T, 8)):
+        out.add(("route", -1, i))
+        out.add(("combine", -1, i))
+    out.add(("mindptr", -1, 0))
+    out.add(("mfin", -1, 0))
+    for i in range(n_tiles * nt_gu):
+        out.add(("egu", -1, i))
+    for i in range(n_tiles * nt_d):
+        out.add(("edown", -1, i))
+    return out

@@ -414,3 +414,17 @@ def test_task_set_brute_force_attn_numbering():
     # indices are exactly 0..(total-1): a bijection with the (b, g, c) triples
     n = sum(2 * (-(-(c + 1) // 64)) for c in ctx)
     assert attn == list(range(n))
+
+
+def test_moe_tiles_and_task_set_by_hand():
+    # hist = [3, 0, 130, 64], tm = 64: expert 0 -> one tile of 3 rows; expert 2
+    # -> tiles of 64, 64, 2 rows starting at rows 3, 67, 131; expert 3 -> one
+    # tile of 64 rows at row 133.  5 tiles.
+    assert ot.moe_tiles([3, 0, 130, 64], 64) == [(0, 0, 3), (2, 3, 64), (2, 67, 64), (2, 131, 2), (3, 133, 64)]
+    # T = 25 tokens: 4 route + 4 combine tasks; F = 1408, tn = 8 -> 176 gate/up
+    # tasks per tile; H = 2048, td = 8 -> 256 down tasks per tile
+    tasks = ot.expected_moe_tasks(25, [3, 0, 130, 64], 2048, 1408, {"tm": 64, "tn": 8, "td": 8})
+    fams = {}
+    for f, _, i in tasks:
+        fams[f] = fams.get(f, 0) + 1
+    assert fams == {"route": 4, "combine": 4, "mindptr": 1, "mfin": 1, "egu": 5 * 176, "edown": 5 * 256}

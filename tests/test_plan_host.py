@@ -132,3 +132,38 @@ def test_dynamic_queue_capacity_deep_model():
     for B, ctx in [(1, [64]), (2, [300, 5])]:
         code, rep = mk.mk_plan_simulate(d.plan, B, ctx, n_orders=4, seed=5)
         assert code == 0, rep.first_error
+
+
+def test_moe_plan_build_families_and_limits():
+    lay = mk.MoELayer(wl.MOE_64x8, None, max_tokens=512, n_sm=148, host_only=True)
+    names = [f.name.decode() for f in lay.families()]
+    assert names == ["route", "mindptr", "egu", "edown", "combine", "mfin"]
+    fu = {f.name.decode(): f.followup for f in lay.families()}
+    assert fu["mindptr"] == 1 and fu["mfin"] == 1 and fu["egu"] == 0
+    ext = {f.name.decode(): f.max_extent for f in lay.families()}
+    # max tiles = ceil(512 * 8 / 64) + min(64, 4096) = 128; F/8 = 176 and H/8 = 256 tasks per tile
+    assert ext["egu"] == 128 * 176 and ext["edown"] == 128 * 256 and ext["route"] == 64
+    assert mk.mk_plan_workspace_bytes(lay.plan) > 512 * 8 * (1408 * 2 + 2048 * 4)
+    lay.close()
+    for bad in (dict(n_experts=65), dict(top_k=9), dict(expert_ffn=1410), dict(hidden=2304)):
+        shp = wl.MoEShape(**{**dict(hidden=2048, n_experts=64, top_k=8, expert_ffn=1408), **bad})
+        with pytest.raises(mk.MkError):
+            mk.MoELayer(shp, None, max_tokens=64, n_sm=148, host_only=True)
+
+
+def test_moe_plan_requires_dynamic_schedule_and_rejects_dense_calls():
+    d = mk.mk_model_desc()
+    d.kind = mk.MK_MODEL_MOE_LAYER
+    d.hidden, d.n_experts, d.top_k, d.expert_ffn, d.max_tokens = 2048, 64, 8, 1408, 64
+    o = mk.mk_plan_opts()
+    o.sched, o.host_only, o.n_sm = mk.MK_SCHED_STATIC, 1, 148
+    with pytest.raises(mk.MkError) as e:
+        mk.mk_plan_build(d, o)
+    assert e.value.status == mk.MK_ERR_UNSUPPORTED
+    o.sched = mk.MK_SCHED_DYNAMIC
+    plan = mk.mk_plan_build(d, o)
+    a = mk.mk_step_args()
+    a.batch = 1
+    with pytest.raises(mk.MkError):
+        mk.mk_decode_step(plan, a, 0)
+    mk.mk_plan_destroy(plan)
