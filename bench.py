@@ -264,6 +264,55 @@ def torch_baselines(s, w, K, V, max_ctx, tok0, dev, n_steps):
                     "eager and as one captured CUDA graph; device-timed with CUDA events"}
 
 
+def moe_layer_bench(dev, n_iter=10):
+    """The MoE FFN layer (64 experts, top-8, F 1408, hidden 2048) for
+    T in {1, 8, 64, 512} with uniform and Zipf(1.2)-skewed routing: device
+    time per layer call (CUDA events around each call, L2 flushed before
+    it), and the HBM roofline of the bytes the call must read (router, the
+    distinct experts the routing touched, the tokens in and out)."""
+    import torch
+    import event_tensor_task_b200 as mk
+    import workloads as wl
+    shape = wl.MOE_64x8
+    H, E, K, F = shape.hidden, shape.n_experts, shape.top_k, shape.expert_ffn
+    w = {k: v.to(dev) for k, v in wl.moe_weights(shape, seed=0).items()}
+    bias = wl.zipf_bias(E).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # twice the L2
+    peak, peak_kind = peaks()
+    cases = []
+    for regime, b in (("uniform", None), ("zipf", bias)):
+        layer = mk.MoELayer(shape, w, b, max_tokens=512)
+        for T in (1, 8, 64, 512):
+            x = wl.moe_tokens(T, H, seed=0).to(dev)
+            out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+            hist = torch.empty(E, dtype=torch.int32, device=dev)
+            for _ in range(3):
+                layer(x, out, hist=hist)
+            torch.cuda.synchronize()
+            total = 0.0
+            for _ in range(n_iter):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                layer(x, out, hist=hist)
+                e1.record()
+                torch.cuda.synchronize()
+                total += e0.elapsed_time(e1)
+            code, _ = layer.status()
+            if code != 0:
+                raise SystemExit(f"MoE layer device status {code}")
+            us = 1000.0 * total / n_iter
+            touched = int((hist.cpu() > 0).sum())
+            nbytes = E * H * 2 + touched * 3 * F * H * 2 + 2 * T * H * 2
+            gbs = nbytes / (us * 1e-6) / 1e9
+            cases.append({"T": T, "routing": regime, "us_per_layer": us, "experts_touched": touched,
+                          "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak})
+        layer.close()
+    return {"workload": "MoE FFN layer: hidden 2048, 64 experts, top-8, expert FFN 1408, bf16 N(0,0.02) weights, "
+                        "x ~ N(0,1) bf16; L2 flushed before every timed call",
+            "peak_gbs": peak, "peak_kind": peak_kind, "cases": cases}
+
+
 def cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, n_steps):
     """The oracle as it stands: tokens/s over n_steps decode steps after one
     untimed warm-up step (which also widens the weights to fp64 once)."""
@@ -323,6 +372,7 @@ def main():
     ap.add_argument("--sched", default="static", choices=["static", "dynamic"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-torch-baseline", action="store_true")
+    ap.add_argument("--no-moe", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -438,6 +488,10 @@ def main():
         baselines["megakernel_plan_build_and_bind_ms"] = 1000.0 * (time.perf_counter() - t0)
         tmp.close()
 
+    moe = None
+    if world == 1 and not args.no_moe:
+        moe = moe_layer_bench(dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, dt = cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, 2)
@@ -460,6 +514,7 @@ def main():
                      "frac_of_8tbs": achieved / 8000.0, "bytes_per_launch": step_bytes},
         "cpu_baseline": cpu,
         "torch_baselines": baselines,
+        "moe_layer": moe,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 12, "d2h_bytes_per_step": 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),

@@ -1494,34 +1494,50 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
   const uint4* xr = reinterpret_cast<const uint4*>(S.moe_x);
   __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(ws + P.off_mh);
   const int col = n * P.moe_tn + w;
-  for (int rr = 0; rr < mt.nrows; ++rr) {
-    const int row = mt.r0 + rr;
-    const int t = __ldcg(mperm + row) / K;
-    float ag[2] = {0.f, 0.f}, au[2] = {0.f, 0.f};
+  // the tile's row -> token map, one entry per lane (tm <= 64 rows)
+  const int tok0 = lane < mt.nrows ? __ldcg(mperm + mt.r0 + lane) / K : 0;
+  const int tok1 = lane + 32 < mt.nrows ? __ldcg(mperm + mt.r0 + lane + 32) / K : 0;
+  // two rows at a time: both rows' activation loads are in flight together
+  for (int rr = 0; rr < mt.nrows; rr += 2) {
+    const bool two = rr + 1 < mt.nrows;
+    const int ta = __shfl_sync(0xffffffffu, rr < 32 ? tok0 : tok1, rr & 31);
+    const int tb = __shfl_sync(0xffffffffu, rr + 1 < 32 ? tok0 : tok1, (rr + 1) & 31);
+    const uint4* xa = xr + ((size_t)ta * H + 8 * lane) / 8;
+    const uint4* xb = xr + ((size_t)(two ? tb : ta) * H + 8 * lane) / 8;
+    float ag[2] = {0.f, 0.f}, au[2] = {0.f, 0.f}, bg[2] = {0.f, 0.f}, bu[2] = {0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < kMaxBlk; ++i)
       if (i < nblk) {
-        float xf[8], gf[8], uf[8];
+        float xf[8], yf[8], gf[8], uf[8];
         uint4 g4 = gw[i], u4 = uw[i];
         // keep the weights packed: converting them once outside the row loop
         // would hold 128 floats and spill
         asm volatile("" : "+r"(g4.x), "+r"(g4.y), "+r"(g4.z), "+r"(g4.w), "+r"(u4.x), "+r"(u4.y), "+r"(u4.z), "+r"(u4.w));
-        bf16x8_to_f32(__ldg(xr + ((size_t)t * H + 256 * i + 8 * lane) / 8), xf);
+        bf16x8_to_f32(__ldg(xa + 32 * i), xf);
+        bf16x8_to_f32(__ldg(xb + 32 * i), yf);
         bf16x8_to_f32(g4, gf);
         bf16x8_to_f32(u4, uf);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           ag[j & 1] = fmaf(gf[j], xf[j], ag[j & 1]);
           au[j & 1] = fmaf(uf[j], xf[j], au[j & 1]);
+          bg[j & 1] = fmaf(gf[j], yf[j], bg[j & 1]);
+          bu[j & 1] = fmaf(uf[j], yf[j], bu[j & 1]);
         }
       }
-    float g = ag[0] + ag[1], u = au[0] + au[1];
+    float g = ag[0] + ag[1], u = au[0] + au[1], g2 = bg[0] + bg[1], u2 = bu[0] + bu[1];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       g += __shfl_xor_sync(0xffffffffu, g, o);
       u += __shfl_xor_sync(0xffffffffu, u, o);
+      g2 += __shfl_xor_sync(0xffffffffu, g2, o);
+      u2 += __shfl_xor_sync(0xffffffffu, u2, o);
     }
-    if (lane == 0 && col < P.eff) mh[(size_t)row * P.eff + col] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+    if (lane == 0 && col < P.eff) {
+      const int row = mt.r0 + rr;
+      mh[(size_t)row * P.eff + col] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+      if (two) mh[(size_t)(row + 1) * P.eff + col] = __float2bfloat16_rn(g2 / (1.0f + expf(-g2)) * u2);
+    }
   }
 }
 
@@ -1554,22 +1570,38 @@ __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S
   const uint4* mh = reinterpret_cast<const uint4*>(ws + P.off_mh);
   float* my = reinterpret_cast<float*>(ws + P.off_my);
   const int col = n * P.moe_td + w;
-  for (int rr = 0; rr < mt.nrows; ++rr) {
+  // two rows at a time (their loads in flight together)
+  for (int rr = 0; rr < mt.nrows; rr += 2) {
     const int row = mt.r0 + rr;
-    float acc[2] = {0.f, 0.f};
+    const bool two = rr + 1 < mt.nrows;
+    const uint4* ha = mh + ((size_t)row * FF) / 8 + lane;
+    const uint4* hb = mh + ((size_t)(two ? row + 1 : row) * FF) / 8 + lane;
+    float acc[2] = {0.f, 0.f}, bcc[2] = {0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       if (lane + 32 * i < nch) {
-        float hf[8], wf[8];
+        float hf[8], kf[8], wf[8];
         uint4 d4 = dw[i];
         asm volatile("" : "+r"(d4.x), "+r"(d4.y), "+r"(d4.z), "+r"(d4.w));  // convert per use (see task_egu)
-        bf16x8_to_f32(__ldcg(mh + ((size_t)row * FF) / 8 + lane + 32 * i), hf);
+        bf16x8_to_f32(__ldcg(ha + 32 * i), hf);
+        bf16x8_to_f32(__ldcg(hb + 32 * i), kf);
         bf16x8_to_f32(d4, wf);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j & 1] = fmaf(wf[j], hf[j], acc[j & 1]);
+        for (int j = 0; j < 8; ++j) {
+          acc[j & 1] = fmaf(wf[j], hf[j], acc[j & 1]);
+          bcc[j & 1] = fmaf(wf[j], kf[j], bcc[j & 1]);
+        }
       }
-    const float v = warp_sum(acc[0] + acc[1]);
-    if (lane == 0) my[(size_t)row * H + col] = v;
+    float v = acc[0] + acc[1], v2 = bcc[0] + bcc[1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      v += __shfl_xor_sync(0xffffffffu, v, o);
+      v2 += __shfl_xor_sync(0xffffffffu, v2, o);
+    }
+    if (lane == 0) {
+      my[(size_t)row * H + col] = v;
+      if (two) my[(size_t)(row + 1) * H + col] = v2;
+    }
   }
 }
 
