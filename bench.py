@@ -148,16 +148,20 @@ def setup_model(dev, seed=0):
 
 class TorchPerOpDecoder:
     """Same-box comparison point: the same decode step as ordinary per-op
-    PyTorch on the same bf16 weights (cuBLAS bf16 GEMVs with the q/k/v and
-    gate/up weights concatenated, fp32 RMSNorm/RoPE/softmax, a masked GQA
+    PyTorch on the same bf16 weights (cuBLAS bf16 GEMV/GEMM with the q/k/v
+    and gate/up weights concatenated, fp32 RMSNorm/RoPE/softmax, a masked GQA
     attention over the padded cache), run eagerly or replayed as one CUDA
-    graph.  The position and the greedy token advance on the device, so one
-    captured graph serves every step of the decode window."""
+    graph.  B sequences in cache slots 0..B-1 start at contexts ctx0[b]; the
+    positions and the greedy tokens advance on the device, so one captured
+    graph serves every step of the decode window."""
 
     def __init__(self, s, w, K, V, max_ctx, ctx0, window, tok0, dev):
         import torch
-        self.s, self.max_ctx, self.ctx0, self.window = s, max_ctx, ctx0, window
+        self.s, self.max_ctx, self.window = s, max_ctx, window
         L, D = s.n_layers, s.head_dim
+        ctx0 = [int(c) for c in (ctx0 if isinstance(ctx0, (list, tuple)) else [ctx0])]
+        self.B = len(ctx0)
+        self.ctx0 = torch.tensor(ctx0, dtype=torch.long, device=dev)
         self.K, self.V = K.clone(), V.clone()
         self.embed = w["embed"]
         self.final_norm = w["final_norm"].float()
@@ -172,7 +176,8 @@ class TorchPerOpDecoder:
         ang = torch.arange(max_ctx, dtype=torch.float64)[:, None] * s.rope_theta ** (-2.0 * i / D)
         self.cos, self.sin = ang.cos().float().to(dev), ang.sin().float().to(dev)
         self.keypos = torch.arange(max_ctx, device=dev)
-        self.tok = torch.full((1,), tok0, dtype=torch.long, device=dev)
+        self.heads = torch.arange(s.n_kv_heads, device=dev)
+        self.tok = torch.full((self.B,), tok0, dtype=torch.long, device=dev)
         self.counter = torch.zeros((), dtype=torch.long, device=dev)
         self.graph = None
 
@@ -187,26 +192,29 @@ class TorchPerOpDecoder:
         return torch.cat([a * c - b * sn, b * c + a * sn], -1)
 
     def step(self):
-        """One greedy decode step (all on the device, graph-capturable)."""
+        """One greedy decode step for the B sequences (all on the device, graph-capturable)."""
         import torch
-        s = self.s
+        s, B = self.s, self.B
         Hq, Hkv, D = s.n_q_heads, s.n_kv_heads, s.head_dim
-        pos = (self.ctx0 + torch.remainder(self.counter, self.window)).view(1)
-        c, sn = self.cos.index_select(0, pos), self.sin.index_select(0, pos)  # [1, D/2]
-        mask = self.keypos > pos  # keys after the new token's position
-        x = self.embed.index_select(0, self.tok).float()  # [1, H]
+        pos = self.ctx0 + torch.remainder(self.counter, self.window)  # [B]
+        c = self.cos.index_select(0, pos)[:, None, :]
+        sn = self.sin.index_select(0, pos)[:, None, :]
+        mask = (self.keypos[None, :] > pos[:, None])[:, None, None, :]  # keys after each new token
+        rows = ((torch.arange(B, device=pos.device)[:, None] * Hkv + self.heads[None, :]) * self.max_ctx
+                + pos[:, None]).reshape(-1)  # cache rows (slot b, head g, position pos_b)
+        x = self.embed.index_select(0, self.tok).float()  # [B, H]
         for l, lw in enumerate(self.layers):
             h = self._rms(x, lw["attn_norm"]).to(torch.bfloat16)
             qkv = (h @ lw["wqkv"].T).float()
-            q = self._rope(qkv[:, :Hq * D].view(Hq, D), c, sn)
-            k = self._rope(qkv[:, Hq * D:(Hq + Hkv) * D].view(Hkv, D), c, sn)
-            v = qkv[:, (Hq + Hkv) * D:].view(Hkv, D)
-            self.K[l, 0].index_copy_(1, pos, k.to(torch.bfloat16).view(Hkv, 1, D))
-            self.V[l, 0].index_copy_(1, pos, v.to(torch.bfloat16).view(Hkv, 1, D))
-            qg = q.view(Hkv, Hq // Hkv, D)
-            sc = torch.matmul(qg, self.K[l, 0].float().transpose(1, 2)) * (1.0 / math.sqrt(D))
+            q = self._rope(qkv[:, :Hq * D].view(B, Hq, D), c, sn)
+            k = self._rope(qkv[:, Hq * D:(Hq + Hkv) * D].view(B, Hkv, D), c, sn)
+            v = qkv[:, (Hq + Hkv) * D:].view(B, Hkv, D)
+            self.K[l].view(-1, D).index_copy_(0, rows, k.to(torch.bfloat16).reshape(B * Hkv, D))
+            self.V[l].view(-1, D).index_copy_(0, rows, v.to(torch.bfloat16).reshape(B * Hkv, D))
+            qg = q.view(B, Hkv, Hq // Hkv, D)
+            sc = torch.matmul(qg, self.K[l, :B].float().transpose(-1, -2)) * (1.0 / math.sqrt(D))
             sc = sc.masked_fill(mask, float("-inf"))
-            o = torch.matmul(torch.softmax(sc, -1), self.V[l, 0].float()).reshape(1, Hq * D)
+            o = torch.matmul(torch.softmax(sc, -1), self.V[l, :B].float()).reshape(B, Hq * D)
             x = x + (o.to(torch.bfloat16) @ lw["wo"].T).float()
             h = self._rms(x, lw["ffn_norm"]).to(torch.bfloat16)
             gu = (h @ lw["wgu"].T).float()
@@ -262,6 +270,58 @@ def torch_baselines(s, w, K, V, max_ctx, tok0, dev, n_steps):
             "what": "same model, weights and cache on the same GPU: per-op PyTorch (cuBLAS bf16 GEMV, "
                     "fused q/k/v and gate/up weights, masked GQA attention over the padded cache), "
                     "eager and as one captured CUDA graph; device-timed with CUDA events"}
+
+
+def batch_sweep(s, w, dev, n_steps=100, batches=(1, 2, 4)):
+    """Decode steps of the same 1B model at several batch sizes through ONE
+    plan and one compiled kernel (no rebuild, no graph capture), each
+    sequence at its own context drawn uniform in [128, 4096] (seeded), next
+    to the per-op PyTorch CUDA graph captured for that batch size."""
+    import torch
+    import event_tensor_task_b200 as mk
+    import workloads as wl
+    maxB = max(batches)
+    ctx0 = [int(c) for c in wl.context_lengths(maxB, 128, 4096)]
+    max_ctx = max(ctx0) + WINDOW + 32
+    K_cpu, V_cpu = wl.kv_cache(s, maxB, max_ctx, ctx0, seed=0)
+    K, V = K_cpu.to(dev), V_cpu.to(dev)
+    dec = mk.DenseDecoder(s, w, K, V, max_batch=maxB, max_ctx=max_ctx, n_slots=maxB)
+    peak, _ = peaks()
+    slots = torch.arange(maxB, dtype=torch.int32, device=dev)
+    cases = []
+    for B in batches:
+        ctx_tab = torch.tensor([[ctx0[b] + i for b in range(B)] for i in range(WINDOW)], dtype=torch.int32,
+                               device=dev)
+        toks = torch.full((2, B), 5, dtype=torch.int32, device=dev)
+
+        def run(n, start=0):
+            for i in range(start, start + n):
+                dec.step(toks[i % 2], slots[:B], ctx_tab[i % WINDOW], toks[(i + 1) % 2])
+
+        run(5)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run(n_steps, 5)
+        e1.record()
+        torch.cuda.synchronize()
+        code, _ = dec.status()
+        if code != 0:
+            raise SystemExit(f"device status {code} in the batch sweep (B={B})")
+        ms = e0.elapsed_time(e1) / n_steps
+        nbytes = statistics.mean(mk.mk_plan_step_bytes(dec.plan, B, [ctx0[b] + i for b in range(B)])
+                                 for i in range(WINDOW))
+        base = TorchPerOpDecoder(s, w, K, V, max_ctx, ctx0[:B], WINDOW, 5, dev)
+        base.capture()
+        gms = base.timed(n_steps, graph=True)
+        del base
+        cases.append({"B": B, "us_per_step": 1000.0 * ms, "tokens_per_s": B / (ms / 1000.0),
+                      "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                      "frac": nbytes / (ms * 1e-3) / 1e9 / peak,
+                      "torch_cuda_graph_us_per_step": 1000.0 * gms})
+    dec.close()
+    return {"contexts": ctx0, "note": "one plan and one kernel for every B (no rebuild, no graph re-capture); "
+                                      "this build runs B <= 4", "cases": cases}
 
 
 def moe_layer_bench(dev, n_iter=10):
@@ -373,6 +433,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-torch-baseline", action="store_true")
     ap.add_argument("--no-moe", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -491,6 +552,9 @@ def main():
     moe = None
     if world == 1 and not args.no_moe:
         moe = moe_layer_bench(dev)
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        sweep = batch_sweep(s, w, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -515,6 +579,7 @@ def main():
         "cpu_baseline": cpu,
         "torch_baselines": baselines,
         "moe_layer": moe,
+        "batch_sweep": sweep,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 12, "d2h_bytes_per_step": 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),

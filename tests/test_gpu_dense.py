@@ -149,3 +149,19 @@ def test_llama1b_greedy_32_static_vs_dynamic(llama):
         seqs.append((torch.cat(out).cpu(), logits.cpu().clone()))
     assert torch.equal(seqs[0][0], seqs[1][0])
     assert torch.equal(seqs[0][1], seqs[1][1])  # bit-identical final logits
+
+
+def test_llama1b_long_ragged_contexts():
+    # the symbolic-batch workload's context range: three sequences at 128,
+    # 2100 and 4095 cached tokens in one step (33 to 65 key chunks each)
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    ctx = [128, 2100, 4095]
+    case = DenseCase(wl.LLAMA_1B, max_batch=4, max_ctx=4104, n_slots=4, ctx_fill=ctx + [0])
+    tokens = wl.token_ids(3, wl.LLAMA_1B.vocab).tolist()
+    ref, _, _ = _oracle_step(case, tokens, [0, 1, 2], ctx)
+    got = case.gpu_step(tokens, [0, 1, 2], ctx)
+    for b in range(3):
+        assert rel_err(got["logits"][b], ref["logits"][b]) <= TOL
+        check_argmax(got["next_tokens"][b], ref["logits"][b])
+    case.check_task_set(got["task_counts"], 3, ctx)
