@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes as C
 
 from . import _abi
-from ._abi import (MK_MODEL_MOE_LAYER, mk_moe_weights, mk_moe_args, MK_OK, MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_STATIC_SCRATCH_BYTES,
+from ._abi import (MK_MODEL_MOE_LAYER, MK_MODEL_MOE_DECODER, mk_moe_weights, mk_moe_args, MK_OK, MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_STATIC_SCRATCH_BYTES,
                    MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS, MK_DEBUG_TRACE,
                    MK_SIM_FAULT_NONE, MK_SIM_FAULT_DROP_NOTIFY, MK_SIM_FAULT_COUNT_PLUS_ONE,
                    MK_SIM_FAULT_NO_WAIT, OP_NAMES, mk_model_desc, mk_plan_opts, mk_step_args,
@@ -146,7 +146,7 @@ class DenseDecoder:
 
     def __init__(self, shape, weights=None, k_cache=None, v_cache=None, max_batch=1, max_ctx=None,
                  n_slots=None, sched=MK_SCHED_STATIC, n_sm=0, host_only=False, debug=False,
-                 spin_timeout_ns=0, trace=False, workspace=True, **tiles):
+                 spin_timeout_ns=0, trace=False, workspace=True, moe=None, **tiles):
         import torch
         self.shape = shape
         w = weights or {}
@@ -157,12 +157,23 @@ class DenseDecoder:
             p = f"layers.{l}."
             for f in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down"):
                 setattr(self._layers[l], f, _ptr(w.get(p + f)))
+        if moe is not None:
+            # MoE decoder: moe = (MoEShape, [per-layer dict router/w_gate/w_up/w_down], bias or None)
+            mshape, mlayers, mbias = moe
+            self._keep.append(moe)
+            for l in range(L):
+                mw = mlayers[l] if mlayers else {}
+                self._layers[l].moe = mk_moe_weights(_ptr(mw.get("router")), _ptr(mbias), _ptr(mw.get("w_gate")),
+                                                     _ptr(mw.get("w_up")), _ptr(mw.get("w_down")))
+            sched = MK_SCHED_DYNAMIC
         if max_ctx is None:
             max_ctx = k_cache.shape[3]
         if n_slots is None:
             n_slots = k_cache.shape[1] if k_cache is not None else max_batch
         d = mk_model_desc()
-        d.kind = MK_MODEL_DENSE
+        d.kind = MK_MODEL_DENSE if moe is None else MK_MODEL_MOE_DECODER
+        if moe is not None:
+            d.n_experts, d.top_k, d.expert_ffn = moe[0].n_experts, moe[0].top_k, moe[0].expert_ffn
         d.n_layers, d.hidden, d.n_q_heads, d.n_kv_heads = L, shape.hidden, shape.n_q_heads, shape.n_kv_heads
         d.head_dim, d.ffn, d.vocab = shape.head_dim, shape.ffn, shape.vocab
         d.eps, d.rope_theta = shape.eps, shape.rope_theta

@@ -30,20 +30,22 @@ MK_SIM_FAULT_COUNT_PLUS_ONE = 2
 MK_SIM_FAULT_NO_WAIT = 3
 
 MK_MODEL_MOE_LAYER = 1
+MK_MODEL_MOE_DECODER = 2
 
 OP_NAMES = {1: "qkv", 2: "attn", 3: "merge", 4: "oproj", 5: "gateup", 6: "down",
             8: "lm", 10: "lmfin", 11: "route", 12: "mindptr", 13: "egu", 14: "edown", 15: "combine",
             16: "mfin"}
 
 
-class mk_layer_weights(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in
-                ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down")]
-
-
 class mk_moe_weights(C.Structure):
     _fields_ = [("w_router", C.c_void_p), ("router_bias", C.c_void_p), ("w_gate", C.c_void_p),
                 ("w_up", C.c_void_p), ("w_down", C.c_void_p)]
+
+
+class mk_layer_weights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in
+                ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down")] + [
+                    ("moe", mk_moe_weights)]
 
 
 class mk_model_desc(C.Structure):

@@ -102,7 +102,7 @@ mk_status mk_plan_bind_workspace(mk_plan* hp, void* dev_ptr, size_t bytes, void*
 mk_status mk_decode_step(mk_plan* hp, const mk_step_args* a, void* stream) {
   g_err.clear();
   if (!hp || !a) return fail(MK_ERR_INVALID_ARG, "null argument");
-  if (hp->p.dp.kind != MK_MODEL_DENSE) return fail(MK_ERR_INVALID_ARG, "plan is not a dense decoder");
+  if (hp->p.dp.kind == MK_MODEL_MOE_LAYER) return fail(MK_ERR_INVALID_ARG, "plan is an MoE layer (use mk_moe_layer)");
   if (!hp->p.ws) return fail(MK_ERR_WORKSPACE, "no workspace bound");
   if (a->batch < 1 || a->batch > hp->p.dp.max_batch) return fail(MK_ERR_INVALID_ARG, "batch out of [1, max_batch]");
   if (!a->token_ids || !a->slot_ids || !a->ctx_lens || !a->next_tokens)

@@ -183,8 +183,23 @@ __device__ __forceinline__ int ev_ctr(const DevPlan& P, int ev, int c0, int c1 =
   return e.base + lin;
 }
 __device__ __forceinline__ int fam_of(const DevPlan& P, int op, int layer) {
-  return op >= OP_LM ? P.fam_first_layer[op] : P.fam_first_layer[op] + layer * P.fam_stride;
+  return layer < 0 ? P.fam_first_layer[op] : P.fam_first_layer[op] + layer * P.fam_stride;
 }
+// MoE: the scratch block and the weights of an MoE layer (layer -1: the
+// MoE-layer plan's single layer)
+__device__ __forceinline__ unsigned char* moe_block(const DevPlan& P, unsigned char* ws, int layer) {
+  return ws + (layer > 0 ? (size_t)layer * (size_t)P.moe_stride : 0);
+}
+struct MoeW {
+  const void* router; const float* bias; const void* gate; const void* up; const void* down;
+};
+__device__ __forceinline__ MoeW moe_weights(const DevPlan& P, const LayerPtrs* layers, int layer) {
+  if (layer < 0) return MoeW{P.w_router, P.router_bias, P.w_egate, P.w_eup, P.w_edown};
+  const LayerPtrs& l = layers[layer];
+  return MoeW{l.w_router, l.router_bias, l.we_gate, l.we_up, l.we_down};
+}
+__device__ __forceinline__ int moe_li(int layer) { return layer > 0 ? layer : 0; }  // MoE event row
+
 __device__ __forceinline__ bool is_followup(int op) {
   return op == OP_MERGE || op == OP_LMFIN || op == OP_MINDPTR || op == OP_MFIN;
 }
@@ -192,7 +207,9 @@ __device__ __forceinline__ bool is_followup(int op) {
 // Counter a regular task waits on (-1: none).
 __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t, int B) {
   switch (t.op) {
-    case OP_QKV: return ev_ctr(P, EV_IN, t.layer);
+    case OP_QKV:
+      return (P.kind == MK_MODEL_MOE_DECODER && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
+                                                             : ev_ctr(P, EV_IN, t.layer);
     case OP_ATTN: {
       AttnTask a = decode_attn(t.idx, B, P.n_kv_heads, sm.nch, sm.pre);
       return ev_ctr(P, EV_QKV, t.layer, a.g);
@@ -200,10 +217,12 @@ __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t,
     case OP_OPROJ: return ev_ctr(P, EV_ATTN, t.layer);
     case OP_GATEUP: return ev_ctr(P, EV_O, t.layer);
     case OP_DOWN: return ev_ctr(P, EV_GU, t.layer, t.idx / P.n_dtiles);
-    case OP_LM: return ev_ctr(P, EV_IN, P.n_layers);
-    case OP_EDOWN: return ev_ctr(P, EV_MH, t.idx / P.nt_d);
-    case OP_COMBINE: return ev_ctr(P, EV_MY, 0);
-    default: return -1;  // ROUTE; EGU is pushed only once its tile table exists
+    case OP_LM:
+      return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_MCOMB, P.n_layers - 1) : ev_ctr(P, EV_IN, P.n_layers);
+    case OP_ROUTE: return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_O, t.layer) : -1;
+    case OP_EDOWN: return ev_ctr(P, EV_MH, moe_li(t.layer), t.idx / P.nt_d);
+    case OP_COMBINE: return ev_ctr(P, EV_MY, moe_li(t.layer));
+    default: return -1;  // EGU is pushed only once its tile table exists
   }
 }
 
@@ -248,12 +267,13 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, int fam, i
       f.row_bytes = (uint32_t)P.kseg * 2; f.row_stride = (uint32_t)P.ffn * 2; f.row_pitch = f.row_bytes;
       f.rps = P.slot_bytes / (int)f.row_bytes; f.slots_per_part = P.tile_down / f.rps;
       break;
-    case OP_EGU:  // an expert's gate rows, then its up rows (the expert is per task)
-      f.w[0] = (const unsigned char*)P.w_egate; f.w[1] = (const unsigned char*)P.w_eup;
+    case OP_EGU: {  // an expert's gate rows, then its up rows (the expert is per task)
+      const MoeW mw = moe_weights(P, layers, layer);
+      f.w[0] = (const unsigned char*)mw.gate; f.w[1] = (const unsigned char*)mw.up;
       f.parts = 2; f.slots_per_part = ceil_div(P.moe_tn, f.rps);
-      break;
+    } break;
     case OP_EDOWN:  // an expert's down rows (expert_ffn long), placed at a 4 KB pitch
-      f.w[0] = (const unsigned char*)P.w_edown;
+      f.w[0] = (const unsigned char*)moe_weights(P, layers, layer).down;
       f.row_bytes = (uint32_t)P.eff * 2; f.row_stride = f.row_bytes; f.row_pitch = 4096;
       f.rps = P.slot_bytes / 4096; f.slots_per_part = ceil_div(P.moe_td, f.rps);
       break;
@@ -362,14 +382,14 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
         // tile -> expert from the table the routing follow-up wrote (visible:
         // this task was popped after its push, which followed that write)
         const int tile = idx / P.nt_gu, n = idx - tile * P.nt_gu;
-        const int e = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_e) + tile);
+        const int e = __ldcg(reinterpret_cast<const int*>(moe_block(P, ws, layer) + P.off_mtile_e) + tile);
         const size_t row0 = (size_t)e * P.eff + (size_t)n * P.moe_tn;
         if (!stream_part(fam, idx, f.w[0] + row0 * f.row_stride, P.moe_tn)) return false;
         if (!stream_part(fam, idx, f.w[1] + row0 * f.row_stride, P.moe_tn)) return false;
       } break;
       case OP_EDOWN: {
         const int tile = idx / P.nt_d, n = idx - tile * P.nt_d;
-        const int e = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_e) + tile);
+        const int e = __ldcg(reinterpret_cast<const int*>(moe_block(P, ws, layer) + P.off_mtile_e) + tile);
         const size_t row0 = (size_t)e * P.hidden + (size_t)n * P.moe_td;
         if (!stream_part(fam, idx, f.w[0] + row0 * f.row_stride, P.moe_td)) return false;
       } break;
@@ -501,15 +521,15 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
       n.ffam = fam_of(P, OP_LMFIN, -1); n.fop = OP_LMFIN; n.fidx = 0;
       break;
     case OP_ROUTE:
-      n.ctr = ev_ctr(P, EV_ROUTE, 0);
-      n.ffam = fam_of(P, OP_MINDPTR, -1); n.fop = OP_MINDPTR; n.fidx = 0;
+      n.ctr = ev_ctr(P, EV_ROUTE, moe_li(t.layer));
+      n.ffam = fam_of(P, OP_MINDPTR, t.layer); n.fop = OP_MINDPTR; n.flayer = t.layer; n.fidx = 0;
       break;
-    case OP_MINDPTR: n.ctr = ev_ctr(P, EV_MIDX, 0); break;
-    case OP_EGU: n.ctr = ev_ctr(P, EV_MH, t.idx / P.nt_gu); break;  // the tile's event: set by the routing
-    case OP_EDOWN: n.ctr = ev_ctr(P, EV_MY, 0); break;
+    case OP_MINDPTR: n.ctr = ev_ctr(P, EV_MIDX, moe_li(t.layer)); break;
+    case OP_EGU: n.ctr = ev_ctr(P, EV_MH, moe_li(t.layer), t.idx / P.nt_gu); break;  // the tile's event: set by the routing
+    case OP_EDOWN: n.ctr = ev_ctr(P, EV_MY, moe_li(t.layer)); break;
     case OP_COMBINE:
-      n.ctr = ev_ctr(P, EV_MCOMB, 0);
-      n.ffam = fam_of(P, OP_MFIN, -1); n.fop = OP_MFIN; n.fidx = 0;
+      n.ctr = ev_ctr(P, EV_MCOMB, moe_li(t.layer));
+      if (P.kind == MK_MODEL_MOE_LAYER) { n.ffam = fam_of(P, OP_MFIN, -1); n.fop = OP_MFIN; n.fidx = 0; }
       break;
     default: break;
   }
@@ -529,7 +549,10 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
         push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b] + g * sm.nch[b], sm.nch[b]);
     } break;
     case OP_MERGE: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
-    case OP_OPROJ: push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles); break;
+    case OP_OPROJ:
+      if (P.kind == MK_MODEL_MOE_DECODER) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, t.layer), 0, ceil_div(S.B, 8));
+      else push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles);
+      break;
     case OP_GATEUP: {
       int kc = t.idx * P.tile_gu / P.kseg;
       push_range(P, S, ctl, ws, fam_of(P, OP_DOWN, t.layer), kc * P.n_dtiles, P.n_dtiles);
@@ -540,14 +563,20 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
       break;
     // MoE: exp_indptr decides how many GroupGEMM tiles run (data-dependent task triggering)
     case OP_MINDPTR: {
-      const int n_tiles = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile) + P.n_experts);
-      push_range(P, S, ctl, ws, fam_of(P, OP_EGU, -1), 0, n_tiles * P.nt_gu);
+      const int n_tiles = __ldcg(reinterpret_cast<const int*>(moe_block(P, ws, t.layer) + P.off_mtile) + P.n_experts);
+      push_range(P, S, ctl, ws, fam_of(P, OP_EGU, t.layer), 0, n_tiles * P.nt_gu);
     } break;
     case OP_EGU: {
       const int tile = t.idx / P.nt_gu;
-      push_range(P, S, ctl, ws, fam_of(P, OP_EDOWN, -1), tile * P.nt_d, P.nt_d);
+      push_range(P, S, ctl, ws, fam_of(P, OP_EDOWN, t.layer), tile * P.nt_d, P.nt_d);
     } break;
-    case OP_EDOWN: push_range(P, S, ctl, ws, fam_of(P, OP_COMBINE, -1), 0, ceil_div(S.B, 8)); break;
+    case OP_EDOWN: push_range(P, S, ctl, ws, fam_of(P, OP_COMBINE, t.layer), 0, ceil_div(S.B, 8)); break;
+    case OP_COMBINE:  // MoE decoder: the layer's residual is complete
+      if (P.kind == MK_MODEL_MOE_DECODER) {
+        if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
+        else push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
+      }
+      break;
     default: break;
   }
 }
@@ -871,7 +900,8 @@ __device__ __forceinline__ bool gemv_spec(const DevPlan& P, const TaskDesc& d, G
   g.gamma_sel = 0; g.layer = d.layer; g.kc = 0; g.parts = false; g.K = P.hidden;
   switch (d.op) {
     case OP_QKV:
-      g.kind = 0; g.gamma_sel = 0; g.parts = d.layer > 0; g.tag = d.layer * 64; g.rows = P.tile_qkv;
+      g.kind = 0; g.gamma_sel = 0; g.parts = d.layer > 0 && P.kind == MK_MODEL_DENSE; g.tag = d.layer * 64;
+      g.rows = P.tile_qkv;
       return true;
     case OP_OPROJ:
       g.kind = 1; g.tag = d.layer * 64 + 1; g.rows = P.tile_o;
@@ -883,7 +913,7 @@ __device__ __forceinline__ bool gemv_spec(const DevPlan& P, const TaskDesc& d, G
       g.kind = 2; g.kc = d.idx / P.n_dtiles; g.K = P.kseg; g.tag = d.layer * 64 + 8 + g.kc; g.rows = P.tile_down;
       return true;
     case OP_LM:
-      g.kind = 0; g.gamma_sel = 2; g.parts = true; g.tag = 60 * 64;
+      g.kind = 0; g.gamma_sel = 2; g.parts = P.kind == MK_MODEL_DENSE; g.tag = 60 * 64;
       g.rows = min(P.tile_lm, P.vocab - d.idx * P.tile_lm);
       return true;
     default:
@@ -1001,6 +1031,17 @@ __device__ __forceinline__ void act_to_regs(const float* xs, int nblk, ActRegs& 
 // registers, reduced over the warp.
 
 // Ring position of the task's slots.
+// Ring slot release.  A slot's empty barrier expects kComputeWarps arrivals
+// per use; only the warps that READ the slot arrive, each with its share of
+// that count (the first reader adds the remainder).  A warp that reads
+// nothing of a slot never touches its barrier, so no arrival can land in
+// another use's phase (with tasks of up to 8 slots in a 13-slot ring, task
+// k+1's slots can be physical slots that task k still reads).
+__device__ __forceinline__ void release_share(Smem& sm, int slot, int readers, int rank) {
+  const uint32_t share = kComputeWarps / readers + (rank == 0 ? kComputeWarps % readers : 0);
+  mbar_arrive_count(&sm.empty[slot], share);
+}
+
 // Dot products of two rows held in shared memory (bf16, 16-byte chunks per
 // lane, 256 columns per block) with the activation in registers, interleaved
 // for instruction-level parallelism; summed across the warp (every lane gets
@@ -1050,14 +1091,13 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
   const int r0 = w * geo.rpw;                                   // first row of this warp in part 0
   const int n = max(0, min(geo.rpw, g.rows - r0));              // rows (pairs) of this warp
+  if (n == 0) return;  // (reads no slot: see release_share)
   const int ja = r0 >> geo.rps_lg;                              // task slot of part 0's rows
   const int jb = geo.pairs ? geo.spp + ja : -1;                 // task slot of part 1's rows
-  // the task's slots this warp reads none of: released right away, one lane each
-  if (release && lane < d.nslots && lane != ja && lane != jb) {
-    const int j = s0 + lane;
-    mbar_arrive(&sm.empty[j < R ? j : j - R]);
-  }
-  if (n == 0) return;
+  // readers of the slot: the warps whose rows lie in it (rpw divides the rows per slot)
+  const int wps = (1 << geo.rps_lg) / geo.rpw;                  // warps per full slot
+  const int first_w = ja * wps;
+  const int readers = min(wps, (g.rows - first_w * geo.rpw + geo.rpw - 1) / geo.rpw);
   const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R;
   const uint32_t pa = s0 + ja < R ? p0 : p0 ^ 1u;
   wait_mbar(&sm.full[sa], pa, ctl, P.spin_timeout_ns, d.fam, d.idx);
@@ -1088,8 +1128,8 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
   if (release) {
     __syncwarp();
     if (lane == 0) {
-      mbar_arrive(&sm.empty[sa]);
-      if (geo.pairs) mbar_arrive(&sm.empty[sb]);
+      release_share(sm, sa, readers, w - first_w);
+      if (geo.pairs) release_share(sm, sb, readers, w - first_w);  // part 1 has the same readers
     }
   }
   // lane i takes row i (row ops) or pair i (pair ops)
@@ -1140,7 +1180,7 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
       float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
       const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H + col;
       float acc = __ldcg(x + col);
-      if (d.layer > 0)
+      if (d.layer > 0 && P.kind == MK_MODEL_DENSE)
         for (int kc = 0; kc < P.n_kc; ++kc) acc += __ldcg(dp + (size_t)kc * P.max_batch * H);
       x[col] = acc + v0;
     } break;
@@ -1263,7 +1303,7 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
     if (lane == 0) { part[D] = m; part[D + 1] = l; }
   }
   __syncwarp();
-  if (lane == 0) mbar_arrive(&sm.empty[slot]);
+  if (w < qpg && lane == 0) release_share(sm, slot, qpg, w);  // the head warps read the slot
 }
 
 // Merge of a head group's chunk partials, softmax-weighted in chunk order:
@@ -1300,8 +1340,8 @@ __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S
 }
 
 // ---------------------------------------------------------------- MoE layer
-// (The MoE task bodies are compiled into the MoE instance of the kernel only:
-// see megakernel<kMoE>.)
+// (The MoE task bodies are compiled into the MoE instances of the kernel only:
+// see megakernel<kKind>.)
 // Mixture-of-experts FFN on T tokens ("Event Tensor: A Unified Abstraction for
 // Compiling Dynamic Megakernel", section "Core method": data-dependent event
 // update and data-dependent task triggering).  Rows of the grouped problem
@@ -1319,16 +1359,51 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
                                            const TaskDesc& d) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int E = P.n_experts, K = P.top_k, H = P.hidden, T = S.B, nblk = H >> 8;
+  unsigned char* mb = moe_block(P, ws, d.layer);
+  const MoeW mw = moe_weights(P, reinterpret_cast<const LayerPtrs*>(ws + P.off_layers), d.layer);
+  const bool dec = P.kind == MK_MODEL_MOE_DECODER;
+  __nv_bfloat16* xhat = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mxhat);
+  if (dec) {
+    // the layer's FFN input: RMSNorm(x) * ffn_norm of each token's residual row, in bf16
+    const int t = d.idx * 8 + w;
+    if (t < T) {
+      const float* xr32 = reinterpret_cast<const float*>(ws + P.off_x) + (size_t)t * H;
+      const uint4* gam = reinterpret_cast<const uint4*>(reinterpret_cast<const LayerPtrs*>(ws + P.off_layers)[d.layer].ffn_norm);
+      float v[kMaxBlk][8];
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxBlk; ++i)
+        if (i < nblk) {
+          const float4* p4 = reinterpret_cast<const float4*>(xr32 + 256 * i + 8 * lane);
+          const float4 a = __ldcg(p4), b = __ldcg(p4 + 1);
+          v[i][0] = a.x; v[i][1] = a.y; v[i][2] = a.z; v[i][3] = a.w;
+          v[i][4] = b.x; v[i][5] = b.y; v[i][6] = b.z; v[i][7] = b.w;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss += v[i][j] * v[i][j];
+        }
+      const float inv = 1.0f / sqrtf(warp_sum(ss) / (float)H + P.eps);
+#pragma unroll
+      for (int i = 0; i < kMaxBlk; ++i)
+        if (i < nblk) {
+          float gf[8];
+          bf16x8_to_f32(__ldg(gam + (256 * i + 8 * lane) / 8), gf);
+          __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(v[i][j] * inv * gf[j]);
+          *reinterpret_cast<uint4*>(xhat + (size_t)t * H + 256 * i + 8 * lane) = *reinterpret_cast<const uint4*>(o);
+        }
+    }
+  }
   float* lg = sm.xs;  // [8][64] logits of this task's tokens
-  bar_sync(BAR_COMP, kComputeThreads);  // the staging buffer is free
-  const uint4* wr = reinterpret_cast<const uint4*>(P.w_router);
-  const uint4* xr = reinterpret_cast<const uint4*>(S.moe_x);
+  bar_sync(BAR_COMP, kComputeThreads);  // the staging buffer is free (and the FFN inputs are written)
+  const uint4* wr = reinterpret_cast<const uint4*>(mw.router);
+  const uint4* xr = reinterpret_cast<const uint4*>(dec ? xhat : S.moe_x);
   for (int e = w; e < E; e += kComputeWarps) {
     uint4 wv[kMaxBlk];
 #pragma unroll
     for (int i = 0; i < kMaxBlk; ++i)
       if (i < nblk) wv[i] = __ldg(wr + ((size_t)e * H + 256 * i + 8 * lane) / 8);
-    const float bias = P.router_bias ? __ldg(P.router_bias + e) : 0.f;
+    const float bias = mw.bias ? __ldg(mw.bias + e) : 0.f;
     for (int tt = 0; tt < 8; ++tt) {
       const int t = d.idx * 8 + tt;
       if (t >= T) break;
@@ -1338,7 +1413,7 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
         if (i < nblk) {
           float wf[8], xf[8];
           bf16x8_to_f32(wv[i], wf);
-          bf16x8_to_f32(__ldg(xr + ((size_t)t * H + 256 * i + 8 * lane) / 8), xf);
+          bf16x8_to_f32(__ldcg(xr + ((size_t)t * H + 256 * i + 8 * lane) / 8), xf);
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc = fmaf(wf[j], xf[j], acc);  // the product is exact in fp32
         }
@@ -1378,10 +1453,10 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
   if (lane < K) {
     const float wt = ex / sum;
     const size_t pi = (size_t)t * K + lane;
-    const int rank = atomicAdd(reinterpret_cast<int*>(ws + P.off_mhist) + sel_e, 1);
-    reinterpret_cast<int*>(ws + P.off_mrank)[pi] = rank;
-    reinterpret_cast<int*>(ws + P.off_midx)[pi] = sel_e;
-    reinterpret_cast<float*>(ws + P.off_mw)[pi] = wt;
+    const int rank = atomicAdd(reinterpret_cast<int*>(mb + P.off_mhist) + sel_e, 1);
+    reinterpret_cast<int*>(mb + P.off_mrank)[pi] = rank;
+    reinterpret_cast<int*>(mb + P.off_midx)[pi] = sel_e;
+    reinterpret_cast<float*>(mb + P.off_mw)[pi] = wt;
     if (S.dbg_idx) S.dbg_idx[pi] = sel_e;
     if (S.dbg_w) S.dbg_w[pi] = wt;
   }
@@ -1392,17 +1467,19 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
 // ceil(hist[e] / tm) and the tile -> (expert, m) table the GroupGEMM tasks
 // decode; the run-time count of EV_MY (one per down task); and the row map
 // (pair -> row, row -> pair).
-__device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws) {
+__device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws,
+                                             const TaskDesc& d) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int E = P.n_experts, K = P.top_k, TMt = P.moe_tm;
+  unsigned char* mb = moe_block(P, ws, d.layer);
   int* sx = reinterpret_cast<int*>(sm.xs);  // exp_indptr [E + 1]
   bar_sync(BAR_COMP, kComputeThreads);
   if (w == 0) {
-    const int* hist = reinterpret_cast<const int*>(ws + P.off_mhist);
-    int* indptr = reinterpret_cast<int*>(ws + P.off_mindptr);
-    int* tptr = reinterpret_cast<int*>(ws + P.off_mtile);
-    int* tile_e = reinterpret_cast<int*>(ws + P.off_mtile_e);
-    int* tile_m = reinterpret_cast<int*>(ws + P.off_mtile_m);
+    const int* hist = reinterpret_cast<const int*>(mb + P.off_mhist);
+    int* indptr = reinterpret_cast<int*>(mb + P.off_mindptr);
+    int* tptr = reinterpret_cast<int*>(mb + P.off_mtile);
+    int* tile_e = reinterpret_cast<int*>(mb + P.off_mtile_e);
+    int* tile_m = reinterpret_cast<int*>(mb + P.off_mtile_m);
     const int h0 = lane < E ? __ldcg(hist + lane) : 0, h1 = lane + 32 < E ? __ldcg(hist + lane + 32) : 0;
     const int c0 = (h0 + TMt - 1) / TMt, c1 = (h1 + TMt - 1) / TMt;
     int s0 = h0, s1 = h1, u0 = c0, u1 = c1;  // inclusive scans over the lanes
@@ -1432,14 +1509,14 @@ __device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams&
       indptr[E] = rows; sx[E] = rows; tptr[E] = tiles;
       if (S.dbg_indptr) S.dbg_indptr[E] = rows;
       // data-dependent event count: every down task of every tile notifies EV_MY
-      atomicExch(reinterpret_cast<int*>(ws + P.off_counters) + ev_ctr(P, EV_MY, 0), tiles * P.nt_d);
+      atomicExch(reinterpret_cast<int*>(ws + P.off_counters) + ev_ctr(P, EV_MY, moe_li(d.layer)), tiles * P.nt_d);
     }
   }
   bar_sync(BAR_COMP, kComputeThreads);
-  const int* midx = reinterpret_cast<const int*>(ws + P.off_midx);
-  const int* mrank = reinterpret_cast<const int*>(ws + P.off_mrank);
-  int* mrow = reinterpret_cast<int*>(ws + P.off_mrow);
-  int* mperm = reinterpret_cast<int*>(ws + P.off_mperm);
+  const int* midx = reinterpret_cast<const int*>(mb + P.off_midx);
+  const int* mrank = reinterpret_cast<const int*>(mb + P.off_mrank);
+  int* mrow = reinterpret_cast<int*>(mb + P.off_mrow);
+  int* mperm = reinterpret_cast<int*>(mb + P.off_mperm);
   const int npairs = S.B * K;
   for (int p = ct; p < npairs; p += kComputeThreads) {
     const int row = sx[__ldcg(midx + p)] + __ldcg(mrank + p);
@@ -1450,12 +1527,12 @@ __device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams&
 
 // A GroupGEMM tile's geometry: expert, first row and row count.
 struct MoeTile { int e, r0, nrows; };
-__device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, unsigned char* ws, int tile) {
+__device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, const unsigned char* mb, int tile) {
   MoeTile m;
-  m.e = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_e) + tile);
-  const int mi = __ldcg(reinterpret_cast<const int*>(ws + P.off_mtile_m) + tile);
-  const int h = __ldcg(reinterpret_cast<const int*>(ws + P.off_mhist) + m.e);
-  m.r0 = __ldcg(reinterpret_cast<const int*>(ws + P.off_mindptr) + m.e) + mi * P.moe_tm;
+  m.e = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_e) + tile);
+  const int mi = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_m) + tile);
+  const int h = __ldcg(reinterpret_cast<const int*>(mb + P.off_mhist) + m.e);
+  m.r0 = __ldcg(reinterpret_cast<const int*>(mb + P.off_mindptr) + m.e) + mi * P.moe_tm;
   m.nrows = min(P.moe_tm, h - mi * P.moe_tm);
   return m;
 }
@@ -1472,10 +1549,7 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
   const int rps = P.slot_bytes / (2 * H), spp = (P.moe_tn + rps - 1) / rps;
   const int ja = w / rps, jb = spp + ja;
-  if (lane < d.nslots && lane != ja && lane != jb) {
-    const int j = s0 + lane;
-    mbar_arrive(&sm.empty[j < R ? j : j - R]);
-  }
+  const int readers = min(rps, P.moe_tn - ja * rps);  // warps whose rows lie in slot ja (and jb)
   const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R, sb = s0 + jb < R ? s0 + jb : s0 + jb - R;
   wait_mbar(&sm.full[sa], s0 + ja < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
   wait_mbar(&sm.full[sb], s0 + jb < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
@@ -1487,12 +1561,17 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
   for (int i = 0; i < kMaxBlk; ++i)
     if (i < nblk) { gw[i] = ga[i * 32]; uw[i] = ua[i * 32]; }
   __syncwarp();
-  if (lane == 0) { mbar_arrive(&sm.empty[sa]); mbar_arrive(&sm.empty[sb]); }
+  if (lane == 0) {
+    release_share(sm, sa, readers, w - ja * rps);
+    release_share(sm, sb, readers, w - ja * rps);
+  }
   const int tile = d.idx / P.nt_gu, n = d.idx - tile * P.nt_gu;
-  const MoeTile mt = moe_tile(P, ws, tile);
-  const int* mperm = reinterpret_cast<const int*>(ws + P.off_mperm);
-  const uint4* xr = reinterpret_cast<const uint4*>(S.moe_x);
-  __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(ws + P.off_mh);
+  unsigned char* mb = moe_block(P, ws, d.layer);
+  const MoeTile mt = moe_tile(P, mb, tile);
+  const int* mperm = reinterpret_cast<const int*>(mb + P.off_mperm);
+  const uint4* xr = reinterpret_cast<const uint4*>(P.kind == MK_MODEL_MOE_DECODER ? (const void*)(mb + P.off_mxhat)
+                                                                                  : (const void*)S.moe_x);
+  __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mh);
   const int col = n * P.moe_tn + w;
   // the tile's row -> token map, one entry per lane (tm <= 64 rows)
   const int tok0 = lane < mt.nrows ? __ldcg(mperm + mt.r0 + lane) / K : 0;
@@ -1513,8 +1592,8 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
         // keep the weights packed: converting them once outside the row loop
         // would hold 128 floats and spill
         asm volatile("" : "+r"(g4.x), "+r"(g4.y), "+r"(g4.z), "+r"(g4.w), "+r"(u4.x), "+r"(u4.y), "+r"(u4.z), "+r"(u4.w));
-        bf16x8_to_f32(__ldg(xa + 32 * i), xf);
-        bf16x8_to_f32(__ldg(xb + 32 * i), yf);
+        bf16x8_to_f32(__ldcg(xa + 32 * i), xf);
+        bf16x8_to_f32(__ldcg(xb + 32 * i), yf);
         bf16x8_to_f32(g4, gf);
         bf16x8_to_f32(u4, uf);
 #pragma unroll
@@ -1552,10 +1631,7 @@ __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
   const int rps = P.slot_bytes / 4096;
   const int ja = w / rps;
-  if (lane < d.nslots && lane != ja) {
-    const int j = s0 + lane;
-    mbar_arrive(&sm.empty[j < R ? j : j - R]);
-  }
+  const int readers = min(rps, P.moe_td - ja * rps);
   const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R;
   wait_mbar(&sm.full[sa], s0 + ja < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
   const uint4* dr = reinterpret_cast<const uint4*>(ring + (size_t)sa * P.slot_bytes + (w - ja * rps) * 4096);
@@ -1564,11 +1640,12 @@ __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S
   for (int i = 0; i < 8; ++i)
     if (lane + 32 * i < nch) dw[i] = dr[lane + 32 * i];
   __syncwarp();
-  if (lane == 0) mbar_arrive(&sm.empty[sa]);
+  if (lane == 0) release_share(sm, sa, readers, w - ja * rps);
   const int tile = d.idx / P.nt_d, n = d.idx - tile * P.nt_d;
-  const MoeTile mt = moe_tile(P, ws, tile);
-  const uint4* mh = reinterpret_cast<const uint4*>(ws + P.off_mh);
-  float* my = reinterpret_cast<float*>(ws + P.off_my);
+  unsigned char* mb = moe_block(P, ws, d.layer);
+  const MoeTile mt = moe_tile(P, mb, tile);
+  const uint4* mh = reinterpret_cast<const uint4*>(mb + P.off_mh);
+  float* my = reinterpret_cast<float*>(mb + P.off_my);
   const int col = n * P.moe_td + w;
   // two rows at a time (their loads in flight together)
   for (int rr = 0; rr < mt.nrows; rr += 2) {
@@ -1613,9 +1690,12 @@ __device__ __forceinline__ void task_combine(const DevPlan& P, const StepParams&
   const int H = P.hidden, K = P.top_k, nblk = H >> 8;
   const int t = d.idx * 8 + w;
   if (t >= S.B) return;
-  const int* mrow = reinterpret_cast<const int*>(ws + P.off_mrow);
-  const float* mw = reinterpret_cast<const float*>(ws + P.off_mw);
-  const float* my = reinterpret_cast<const float*>(ws + P.off_my);
+  const unsigned char* mb = moe_block(P, ws, d.layer);
+  const int* mrow = reinterpret_cast<const int*>(mb + P.off_mrow);
+  const float* mw = reinterpret_cast<const float*>(mb + P.off_mw);
+  const float* my = reinterpret_cast<const float*>(mb + P.off_my);
+  const bool dec = P.kind == MK_MODEL_MOE_DECODER;
+  float* xres = reinterpret_cast<float*>(ws + P.off_x) + (size_t)t * H;
   int rows[8];
   float wts[8];
 #pragma unroll
@@ -1634,14 +1714,24 @@ __device__ __forceinline__ void task_combine(const DevPlan& P, const StepParams&
         acc[4] = fmaf(wts[j], b.x, acc[4]); acc[5] = fmaf(wts[j], b.y, acc[5]);
         acc[6] = fmaf(wts[j], b.z, acc[6]); acc[7] = fmaf(wts[j], b.w, acc[7]);
       }
-    __align__(16) __nv_bfloat16 o[8];
+    if (dec) {
+      // MoE decoder: the FFN output joins the fp32 residual
+      float4* x4 = reinterpret_cast<float4*>(xres + c);
+      float4 a = __ldcg(x4), b = __ldcg(x4 + 1);
+      a.x += acc[0]; a.y += acc[1]; a.z += acc[2]; a.w += acc[3];
+      b.x += acc[4]; b.y += acc[5]; b.z += acc[6]; b.w += acc[7];
+      x4[0] = a;
+      x4[1] = b;
+    } else {
+      __align__(16) __nv_bfloat16 o[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) o[q] = __float2bfloat16_rn(acc[q]);
-    *reinterpret_cast<uint4*>(S.moe_out + (size_t)t * H + c) = *reinterpret_cast<const uint4*>(o);
+      for (int q = 0; q < 8; ++q) o[q] = __float2bfloat16_rn(acc[q]);
+      *reinterpret_cast<uint4*>(S.moe_out + (size_t)t * H + c) = *reinterpret_cast<const uint4*>(o);
+    }
   }
 }
 
-template <bool kMoE>
+template <int kKind>
 __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
                         Control* ctl) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
@@ -1655,11 +1745,13 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     uint32_t* trec = (d.rec > 0 && w == 0) ? trace_rec(S, d.rec) : nullptr;
     if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
     GemvSpec g;
-    if constexpr (kMoE) {
+    bool moe_task = false;
+    if constexpr (kKind != MK_MODEL_DENSE) {
+      moe_task = d.op >= OP_ROUTE;
       if (d.op == OP_ROUTE) {
         task_route(P, S, sm, ws, d);
       } else if (d.op == OP_MINDPTR) {
-        task_mindptr(P, S, sm, ws);
+        task_mindptr(P, S, sm, ws, d);
       } else if (d.op == OP_EGU) {
         task_egu(P, S, sm, ring, ws, ctl, d);
       } else if (d.op == OP_EDOWN) {
@@ -1667,6 +1759,9 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
       } else if (d.op == OP_COMBINE) {
         task_combine(P, S, ws, d);
       }
+    }
+    if (kKind == MK_MODEL_MOE_LAYER || moe_task) {
+      // (done above)
     } else if (gemv_spec(P, d, g)) {
       // one pass per batch row (the activation is restaged each pass when
       // B > 1); the ring slots are released after the last pass
@@ -1730,8 +1825,9 @@ __device__ __forceinline__ void arm_events(const DevPlan& P, Smem& sm, const Fam
 
 // One persistent kernel per plan kind: the instances share the interpreter
 // (producer, controller, notifier) and differ in the task bodies compiled in
-// (dense decoder or MoE layer), so each gets its own register allocation.
-template <bool kMoE>
+// (dense decoder, MoE layer, or both for the MoE decoder), so each gets its
+// own register allocation.
+template <int kKind>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const StepParams S, unsigned char* ws) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring = smem_raw;
@@ -1797,9 +1893,13 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   __syncthreads();
   arm_events(P, sm, fams, code, counters, B);
   const int gtid = blockIdx.x * blockDim.x + tid, gthreads = gridDim.x * blockDim.x;
-  if (moe) {
-    if (blockIdx.x == 0 && tid < P.n_experts) reinterpret_cast<int*>(ws + P.off_mhist)[tid] = 0;
-  } else {
+  if (P.kind != MK_MODEL_DENSE && blockIdx.x == 0) {
+    // every MoE layer's expert histogram starts at zero
+    const int n_moe = P.kind == MK_MODEL_MOE_DECODER ? P.n_layers : 1;
+    for (int i = tid; i < n_moe * P.n_experts; i += blockDim.x)
+      reinterpret_cast<int*>(moe_block(P, ws, i / P.n_experts) + P.off_mhist)[i % P.n_experts] = 0;
+  }
+  if (!moe) {
     float* x = reinterpret_cast<float*>(ws + P.off_x);
     const int cpr = P.hidden / 8;
     for (int i = gtid; i < B * cpr; i += gthreads) {
@@ -1851,7 +1951,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   } else if (warp == 2) {
     notifier(P, S, sm, ws, ctl, counters);
   } else {
-    compute<kMoE>(P, S, sm, ring, ws, ctl);
+    compute<kKind>(P, S, sm, ring, ws, ctl);
   }
 }
 
@@ -1863,7 +1963,11 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
 namespace mk {
 
 static const void* kernel_for(const DevPlan& P) {
-  return P.kind == MK_MODEL_MOE_LAYER ? (const void*)megakernel<true> : (const void*)megakernel<false>;
+  switch (P.kind) {
+    case MK_MODEL_MOE_LAYER: return (const void*)megakernel<MK_MODEL_MOE_LAYER>;
+    case MK_MODEL_MOE_DECODER: return (const void*)megakernel<MK_MODEL_MOE_DECODER>;
+    default: return (const void*)megakernel<MK_MODEL_DENSE>;
+  }
 }
 
 mk_status dev_query(int* n_sm, int* smem_optin, int* device, std::string& err) {

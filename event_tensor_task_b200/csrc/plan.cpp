@@ -318,7 +318,12 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   };
   add_event(EV_ROUTE, 1, e_tok8);
   add_event(EV_MIDX, 1, emit_const(p.code, 1));
-  add_event(EV_MH, P.max_tiles, emit_const(p.code, P.nt_gu));
+  {
+    EventTensorDesc& e = P.ev[EV_MH];
+    e.base = base; e.ndim = 2; e.dims[0] = 1; e.dims[1] = P.max_tiles; e.dims[2] = 1;
+    e.count_expr = emit_const(p.code, P.nt_gu);
+    base += P.max_tiles;
+  }
   add_event(EV_MY, 1, emit_const(p.code, 1 << 30));  // replaced at run time by MINDPTR
   add_event(EV_MCOMB, 1, e_tok8);
   P.n_counters = base;
@@ -344,14 +349,25 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
                      Plan& p, std::string& err) {
   if (!m || !o) { err = "null model or options"; return MK_ERR_INVALID_ARG; }
   if (m->kind == MK_MODEL_MOE_LAYER) return build_moe_plan(m, o, n_sm, smem_bytes, p, err);
-  if (m->kind != MK_MODEL_DENSE) { err = "unknown model kind"; return MK_ERR_UNSUPPORTED; }
-  const int H = m->hidden, D = m->head_dim, Hq = m->n_q_heads, Hkv = m->n_kv_heads, F = m->ffn;
+  if (m->kind != MK_MODEL_DENSE && m->kind != MK_MODEL_MOE_DECODER) { err = "unknown model kind"; return MK_ERR_UNSUPPORTED; }
+  // MoE decoder: the dense decoder's attention half, then per layer the MoE
+  // FFN families of build_moe_plan on the B tokens (dynamic schedule only)
+  const bool mdec = m->kind == MK_MODEL_MOE_DECODER;
+  const int H = m->hidden, D = m->head_dim, Hq = m->n_q_heads, Hkv = m->n_kv_heads, F = mdec ? 0 : m->ffn;
+  if (mdec) {
+    const int E = m->n_experts, K = m->top_k, FF = m->expert_ffn;
+    if (E < 1 || E > 64) { err = "n_experts must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
+    if (K < 1 || K > 8 || K > E) { err = "top_k must be in [1, min(8, n_experts)]"; return MK_ERR_UNSUPPORTED; }
+    if (FF < 8 || FF % 8 || FF > 2048) { err = "expert_ffn must be a multiple of 8 in [8, 2048]"; return MK_ERR_UNSUPPORTED; }
+    if (o->sched != MK_SCHED_DYNAMIC)
+      { err = "an MoE layer's task counts depend on the routing: use MK_SCHED_DYNAMIC"; return MK_ERR_UNSUPPORTED; }
+  }
   if (m->n_layers < 1 || m->vocab < 1 || Hkv < 1 || Hq < 1) { err = "non-positive dimension"; return MK_ERR_INVALID_ARG; }
   if (D != 64) { err = "head_dim must be 64"; return MK_ERR_UNSUPPORTED; }
   if (Hq % Hkv) { err = "n_q_heads must be a multiple of n_kv_heads"; return MK_ERR_INVALID_ARG; }
   if (Hq * D != H) { err = "n_q_heads * head_dim must equal hidden"; return MK_ERR_UNSUPPORTED; }
   if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
-  if (F % 256) { err = "ffn must be a multiple of 256"; return MK_ERR_UNSUPPORTED; }
+  if (!mdec && (F % 256 || F < 256)) { err = "ffn must be a positive multiple of 256"; return MK_ERR_UNSUPPORTED; }
   if (m->max_batch < 1 || m->max_batch > 4) { err = "max_batch must be in [1, 4] for this build"; return MK_ERR_UNSUPPORTED; }
   if (m->max_ctx < 2 || m->n_slots < m->max_batch) { err = "max_ctx >= 2 and n_slots >= max_batch required"; return MK_ERR_INVALID_ARG; }
   if (o->sched != MK_SCHED_STATIC && o->sched != MK_SCHED_DYNAMIC) { err = "unknown schedule"; return MK_ERR_INVALID_ARG; }
@@ -373,7 +389,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
 
   // K segment of the down projection (split-K), at most 2048 columns
-  int kseg = o->kseg ? o->kseg : std::min(F, 2048);
+  int kseg = mdec ? 2048 : (o->kseg ? o->kseg : std::min(F, 2048));  // (no dense FFN in an MoE decoder)
   while (kseg > 256 && F % kseg) kseg -= 256;
   P.kseg = kseg;
   // rows per 16 KB ring slot of a hidden-wide (and a kseg-wide) row
@@ -463,23 +479,44 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     e_attn = e.start;
   }
   int e_merge = Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret();
+  // MoE decoder: the MoE FFN's geometry (as build_moe_plan) on at most max_batch tokens
+  if (mdec) {
+    P.kind = MK_MODEL_MOE_DECODER;
+    P.n_experts = m->n_experts; P.top_k = m->top_k; P.eff = m->expert_ffn; P.max_tokens = P.max_batch;
+    P.moe_tm = 64; P.moe_tn = 8; P.moe_td = 8;
+    P.nt_gu = ceil_div(P.eff, P.moe_tn);
+    P.nt_d = H / P.moe_td;
+    P.max_tiles = ceil_div(P.max_tokens * P.top_k, P.moe_tm) + std::min(P.n_experts, P.max_tokens * P.top_k);
+  }
+  const int e_tok8 = Emit(p.code).op(X_B).push(8).op(X_CEILDIV).ret();  // ceil(B / 8)
+  static const int kMoeDecOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU, OP_EDOWN,
+                                   OP_COMBINE};
+  const int fam_per_layer = mdec ? 9 : kFamPerLayer;
   for (int l = 0; l < P.n_layers; ++l) {
     add_family(OP_QKV, l, emit_const(p.code, P.n_qkv_tiles), P.n_qkv_tiles, 0);
     add_family(OP_ATTN, l, e_attn, Hkv * P.max_batch * P.max_chunks, 0);
     add_family(OP_MERGE, l, e_merge, Hkv * P.max_batch, 1);
     add_family(OP_OPROJ, l, emit_const(p.code, P.n_otiles), P.n_otiles, 0);
-    add_family(OP_GATEUP, l, emit_const(p.code, P.n_gutiles), P.n_gutiles, 0);
-    add_family(OP_DOWN, l, emit_const(p.code, P.n_dtiles * P.n_kc), P.n_dtiles * P.n_kc, 0);
+    if (mdec) {
+      add_family(OP_ROUTE, l, e_tok8, ceil_div(P.max_tokens, 8), 0);
+      add_family(OP_MINDPTR, l, emit_const(p.code, 1), 1, 1);
+      add_family(OP_EGU, l, emit_const(p.code, P.max_tiles * P.nt_gu), P.max_tiles * P.nt_gu, 0);
+      add_family(OP_EDOWN, l, emit_const(p.code, P.max_tiles * P.nt_d), P.max_tiles * P.nt_d, 0);
+      add_family(OP_COMBINE, l, e_tok8, ceil_div(P.max_tokens, 8), 0);
+    } else {
+      add_family(OP_GATEUP, l, emit_const(p.code, P.n_gutiles), P.n_gutiles, 0);
+      add_family(OP_DOWN, l, emit_const(p.code, P.n_dtiles * P.n_kc), P.n_dtiles * P.n_kc, 0);
+    }
   }
   add_family(OP_LM, -1, emit_const(p.code, P.n_lm_tiles), P.n_lm_tiles, 0);
   add_family(OP_LMFIN, -1, emit_const(p.code, 1), 1, 1);
   P.n_families = (int)p.fams.size();
   if (P.n_families > kMaxFamilies || P.n_layers > 127) { err = "too many task families or layers"; return MK_ERR_UNSUPPORTED; }
   P.debug_slots = debug_base;
-  P.fam_stride = kFamPerLayer;
+  P.fam_stride = fam_per_layer;
   for (int op = 0; op < OP_COUNT; ++op) P.fam_first_layer[op] = -1;
-  for (int k = 0; k < kFamPerLayer; ++k) P.fam_first_layer[kLayerOps[k]] = k;
-  for (int k = 0; k < 2; ++k) P.fam_first_layer[kLmOps[k]] = P.n_layers * kFamPerLayer + k;
+  for (int k = 0; k < fam_per_layer; ++k) P.fam_first_layer[mdec ? kMoeDecOps[k] : kLayerOps[k]] = k;
+  for (int k = 0; k < 2; ++k) P.fam_first_layer[kLmOps[k]] = P.n_layers * fam_per_layer + k;
 
   // ---- event tensors (shapes at the symbols' maxima, wait counts symbolic)
   int base = 0;
@@ -501,7 +538,15 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   add_event(EV_O, 1, L, 1, 1, emit_const(p.code, P.n_otiles));
   add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu));
   add_event(EV_LM, 1, 1, 1, 1, emit_const(p.code, P.n_lm_tiles));
-  for (int id = EV_LM + 1; id < EV_COUNT; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // MoE: empty
+  if (mdec) {  // one element per layer (EV_MH: per layer and GroupGEMM tile)
+    add_event(EV_ROUTE, 1, L, 1, 1, e_tok8);
+    add_event(EV_MIDX, 1, L, 1, 1, emit_const(p.code, 1));
+    add_event(EV_MH, 2, L, P.max_tiles, 1, emit_const(p.code, P.nt_gu));
+    add_event(EV_MY, 1, L, 1, 1, emit_const(p.code, 1 << 30));  // replaced at run time by MINDPTR
+    add_event(EV_MCOMB, 1, L, 1, 1, e_tok8);
+  } else {
+    for (int id = EV_LM + 1; id < EV_COUNT; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // MoE: empty
+  }
   P.n_counters = base;
 
   // ---- static schedule: per-SM queues of block instructions in topological
@@ -509,7 +554,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   // rotation rot_f spreading the blocks that get one task more.
   std::vector<int> regular;
   for (int f = 0; f < P.n_families; ++f)
-    if (!p.fams[f].followup) regular.push_back(f);
+    if (!p.fams[f].followup && !mdec) regular.push_back(f);
   P.n_instr_per_sm = (int)regular.size() + 1;
   p.instr.assign((size_t)n_sm * P.n_instr_per_sm, Instr{});
   Binding typical{1, {std::min(1024, P.max_ctx - 1)}};
@@ -531,14 +576,16 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
 
   // ---- dynamic queue capacity: pushes per step at the symbols' maxima
   // per layer: QKV (1), ATTN (one per sequence and kv head), OPROJ (1),
-  // GATEUP (1), DOWN (one per K segment); then LM (1) and END (1)
-  P.queue_ranges = L * (3 + Hkv * P.max_batch + P.n_kc) + 2;
+  // GATEUP (1), DOWN (one per K segment) -- or for an MoE FFN: ROUTE, EGU,
+  // COMBINE (1 each) and EDOWN (one per tile); then LM (1) and END (1)
+  P.queue_ranges = mdec ? L * (5 + Hkv * P.max_batch + P.max_tiles) + 2 : L * (3 + Hkv * P.max_batch + P.n_kc) + 2;
 
   // ---- layer pointers and the rotary table
   p.layers.resize(L);
   for (int l = 0; l < L; ++l) {
     const mk_layer_weights& w = p.layer_w[l];
-    p.layers[l] = LayerPtrs{w.attn_norm, w.wq, w.wk, w.wv, w.wo, w.ffn_norm, w.w_gate, w.w_up, w.w_down};
+    p.layers[l] = LayerPtrs{w.attn_norm, w.wq, w.wk, w.wv, w.wo, w.ffn_norm, w.w_gate, w.w_up, w.w_down,
+                            w.moe.w_router, w.moe.router_bias, w.moe.w_gate, w.moe.w_up, w.moe.w_down};
   }
   P.embed = m->embed;
   P.lm_head = m->lm_head ? m->lm_head : m->embed;
@@ -578,8 +625,10 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_h = take(4LL * P.max_batch * P.ffn);
   P.off_dpart = take(4LL * P.n_kc * P.max_batch * P.hidden);
   P.off_lmbest = take(8LL * P.max_batch);
-  if (P.kind == MK_MODEL_MOE_LAYER) {
+  if (P.kind != MK_MODEL_DENSE) {
+    // one MoE scratch block per MoE layer (layer 0's offsets; the others follow at moe_stride)
     const long long pairs = (long long)P.max_tokens * P.top_k;
+    const long long block0 = off;
     P.off_mhist = take(4LL * P.n_experts);
     P.off_mrank = take(4 * pairs);
     P.off_midx = take(4 * pairs);
@@ -592,6 +641,10 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
     P.off_mrow = take(4 * pairs);
     P.off_mh = take(2 * pairs * P.eff);
     P.off_my = take(4 * pairs * P.hidden);
+    P.off_mxhat = take(2LL * P.max_tokens * P.hidden);
+    P.moe_stride = off - block0;
+    const int Lm = P.kind == MK_MODEL_MOE_DECODER ? P.n_layers : 1;
+    off += P.moe_stride * (Lm - 1);
   }
   P.ws_bytes = off;
   // image = [off_families, off_queue): the read-only plan arrays

@@ -134,11 +134,12 @@ enum EvId : int32_t {
   EV_GU = 5,     // [L][n_kc]    SwiGLU outputs of one K segment written
   EV_LM = 6,     // [1]          all LM tiles done
   // MoE layer
-  EV_ROUTE = 7,  // [1]          all ROUTE tasks done
-  EV_MIDX = 8,   // [1]          exp_indptr and the tile table written
-  EV_MH = 9,     // [max_tiles]  SwiGLU rows of one GroupGEMM tile written (all its gate/up tasks)
-  EV_MY = 10,    // [1]          all down tasks done (count set at run time from exp_indptr)
-  EV_MCOMB = 11, // [1]          all COMBINE tasks done
+  // (one element per MoE layer: [1] for the MoE-layer plan, [L] for the MoE decoder)
+  EV_ROUTE = 7,  // [Lm]            all ROUTE tasks done
+  EV_MIDX = 8,   // [Lm]            exp_indptr and the tile table written
+  EV_MH = 9,     // [Lm][max_tiles] SwiGLU rows of one GroupGEMM tile written (all its gate/up tasks)
+  EV_MY = 10,    // [Lm]            all down tasks done (count set at run time from exp_indptr)
+  EV_MCOMB = 11, // [Lm]            all COMBINE tasks done (the layer's residual is updated)
   EV_COUNT = 12
 };
 
@@ -178,6 +179,8 @@ MK_HD void instr_range(const Instr& in, int ext, int& lo, int& hi) {
 struct LayerPtrs {
   const void* attn_norm; const void* wq; const void* wk; const void* wv; const void* wo;
   const void* ffn_norm; const void* w_gate; const void* w_up; const void* w_down;
+  // MoE decoder: this layer's MoE FFN
+  const void* w_router; const float* router_bias; const void* we_gate; const void* we_up; const void* we_down;
 };
 
 constexpr int kMaxFamilies = 256;
@@ -208,7 +211,7 @@ struct DevPlan {
   // global weights (device)
   const void* embed; const void* lm_head; const void* final_norm;
   void* k_cache; void* v_cache;
-  // MoE layer (kind MK_MODEL_MOE_LAYER)
+  // MoE layer (kind MK_MODEL_MOE_LAYER) and MoE decoder (MK_MODEL_MOE_DECODER)
   int32_t kind;
   int32_t n_experts, top_k, eff, max_tokens;
   int32_t moe_tm;     // routed rows per GroupGEMM tile
@@ -218,8 +221,11 @@ struct DevPlan {
   int32_t pad2;
   const void* w_router; const float* router_bias;
   const void* w_egate; const void* w_eup; const void* w_edown;
+  // MoE scratch: one block per MoE layer, moe_stride bytes apart; the offsets
+  // below are those of layer 0's block (the MoE-layer plan has one block)
+  int64_t moe_stride;
   int64_t off_mhist, off_mrank, off_midx, off_mw, off_mindptr, off_mtile, off_mtile_e, off_mtile_m;
-  int64_t off_mperm, off_mrow, off_mh, off_my;
+  int64_t off_mperm, off_mrow, off_mh, off_my, off_mxhat;
 };
 
 // Control block at off_control (first 256 bytes of the workspace).

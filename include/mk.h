@@ -50,9 +50,19 @@ typedef int mk_status;
 
 #define MK_MODEL_DENSE 0     /* dense decoder: attention + SwiGLU FFN per layer */
 #define MK_MODEL_MOE_LAYER 1 /* one mixture-of-experts FFN layer (mk_moe_layer); dynamic schedule only */
+#define MK_MODEL_MOE_DECODER 2 /* decoder whose FFNs are MoE layers (mk_decode_step); dynamic schedule only */
 
 #define MK_DEBUG_TASK_COUNTS 1u  /* each executed task increments its slot in mk_step_args.task_counts */
 #define MK_DEBUG_TRACE 2u        /* the controller records per-task timestamps in mk_step_args.trace */
+
+/* Weights of one mixture-of-experts FFN layer; bf16 row-major, device. */
+typedef struct mk_moe_weights {
+  const void* w_router;      /* [n_experts][hidden] */
+  const float* router_bias;  /* fp32 [n_experts] added to the router logits, or NULL */
+  const void* w_gate;        /* [n_experts][expert_ffn][hidden] */
+  const void* w_up;          /* [n_experts][expert_ffn][hidden] */
+  const void* w_down;        /* [n_experts][hidden][expert_ffn] */
+} mk_moe_weights;
 
 /* Per-layer weights of a dense decoder; bf16, row-major [out][in], device. */
 typedef struct mk_layer_weights {
@@ -65,23 +75,21 @@ typedef struct mk_layer_weights {
   const void* w_gate;     /* [ffn][hidden] */
   const void* w_up;       /* [ffn][hidden] */
   const void* w_down;     /* [hidden][ffn] */
+  mk_moe_weights moe;     /* MK_MODEL_MOE_DECODER: this layer's MoE FFN (router, experts) */
 } mk_layer_weights;
 
-/* Weights of one mixture-of-experts FFN layer; bf16 row-major, device. */
-typedef struct mk_moe_weights {
-  const void* w_router;      /* [n_experts][hidden] */
-  const float* router_bias;  /* fp32 [n_experts] added to the router logits, or NULL */
-  const void* w_gate;        /* [n_experts][expert_ffn][hidden] */
-  const void* w_up;          /* [n_experts][expert_ffn][hidden] */
-  const void* w_down;        /* [n_experts][hidden][expert_ffn] */
-} mk_moe_weights;
+
 
 /* Model description.
  * MK_MODEL_DENSE: head_dim == 64, n_q_heads % n_kv_heads == 0, hidden and
  *   ffn multiples of 256 with hidden <= 2048, n_q_heads*head_dim == hidden.
  * MK_MODEL_MOE_LAYER: only hidden (multiple of 256, <= 2048), n_experts
  *   (<= 64), top_k (<= 8 and <= n_experts), expert_ffn (multiple of 8,
- *   <= 2048), max_tokens (<= 4096) and moe are read. */
+ *   <= 2048), max_tokens (<= 4096) and moe are read.
+ * MK_MODEL_MOE_DECODER: the dense fields (ffn, and the dense FFN weights,
+ *   are not used) plus n_experts, top_k, expert_ffn and each layer's moe;
+ *   the FFN of layer l is the MoE layer on the B tokens' RMSNorm'd residual
+ *   rows (ffn_norm gain), added to the residual. */
 typedef struct mk_model_desc {
   int kind;               /* MK_MODEL_DENSE or MK_MODEL_MOE_LAYER */
   int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;

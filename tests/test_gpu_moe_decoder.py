@@ -1,0 +1,84 @@
+"""GPU parity of the MoE decoder (MK_MODEL_MOE_DECODER: each layer's FFN is
+an MoE layer) against the CPU oracle, through mk_decode_step on cuda:0.
+
+Continuous batching: one plan, the batch size and the contexts change every
+step; skewed (Zipf) routing; dynamic schedule.  The oracle's decode step
+takes the MoE FFN on the bf16-rounded normalised residual rows.  Checked:
+logits within max |gpu - oracle| <= 2e-2 * max |oracle| and greedy tokens
+(up to near ties).
+"""
+import pytest
+import torch
+
+import event_tensor_task_b200 as mk
+import oracle
+import workloads as wl
+from gpu_common import rel_err, check_argmax, TOL
+
+pytestmark = pytest.mark.gpu
+
+
+class MoeCase:
+    def __init__(self, shape, mshape, max_batch, max_ctx, ctx_fill):
+        dev = "cuda:0"
+        self.shape, self.mshape = shape, mshape
+        self.w_cpu = wl.dense_weights(shape, seed=0)
+        self.m_cpu = [wl.moe_weights(mshape, seed=0, prefix=f"layers.{l}.moe.") for l in range(shape.n_layers)]
+        self.bias = wl.zipf_bias(mshape.n_experts)
+        self.K_cpu, self.V_cpu = wl.kv_cache(shape, max_batch, max_ctx, ctx_fill, seed=0)
+        self.w = {k: v.to(dev) for k, v in self.w_cpu.items()}
+        self.m = [{k: v.to(dev) for k, v in d.items()} for d in self.m_cpu]
+        self.K, self.V = self.K_cpu.to(dev), self.V_cpu.to(dev)
+        self.dec = mk.DenseDecoder(shape, self.w, self.K, self.V, max_batch=max_batch, max_ctx=max_ctx,
+                                   n_slots=max_batch, moe=(mshape, self.m, self.bias.to(dev)))
+        self.orc = oracle.DenseOracle(shape, self.w_cpu)
+
+    def oracle_moe(self, l, u):
+        return oracle.moe_layer(u.to(torch.bfloat16), self.m_cpu[l], self.mshape.top_k, self.bias)["out"]
+
+    def step(self, K, V, tokens, slots, ctx):
+        dev = "cuda:0"
+        ref = self.orc.step(K, V, tokens, slots, ctx, moe=self.oracle_moe)
+        B = len(tokens)
+        nxt = torch.full((B,), -1, dtype=torch.int32, device=dev)
+        logits = torch.empty(B, self.shape.vocab, dtype=torch.float32, device=dev)
+        self.dec.step(torch.tensor(tokens, dtype=torch.int32, device=dev),
+                      torch.tensor(slots, dtype=torch.int32, device=dev),
+                      torch.tensor(ctx, dtype=torch.int32, device=dev), nxt, logits=logits)
+        torch.cuda.synchronize()
+        code, st = self.dec.status()
+        assert code == 0, f"device status {code} family {st.family} index {st.index} event {st.event}"
+        for b in range(B):
+            assert rel_err(logits[b].cpu(), ref["logits"][b]) <= TOL
+            check_argmax(nxt[b].cpu(), ref["logits"][b])
+        return ref
+
+
+def _walk(case, steps):
+    K, V = case.K_cpu.clone(), case.V_cpu.clone()
+    for tokens, slots, ctx in steps:
+        case.step(K, V, tokens, slots, ctx)
+
+
+def test_tiny_moe_decoder_continuous_batching():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    mshape = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
+    case = MoeCase(wl.TINY, mshape, max_batch=4, max_ctx=320, ctx_fill=[64, 10, 130, 200])
+    _walk(case, [([17], [0], [64]),
+                 ([3, 900, 511], [1, 2, 3], [10, 130, 200]),
+                 ([5, 6, 7, 8], [0, 1, 2, 3], [65, 11, 131, 201]),
+                 ([9, 10], [2, 0], [132, 66])])
+
+
+def test_moe_decoder_1b_attention_64_experts():
+    # two layers of the 1B attention shape, each FFN the 64-expert top-8 layer
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    shape = wl.DenseShape(n_layers=2, hidden=2048, n_q_heads=32, n_kv_heads=8, head_dim=64, ffn=8192,
+                          vocab=128256)
+    case = MoeCase(shape, wl.MOE_64x8, max_batch=4, max_ctx=1100, ctx_fill=[256, 1000, 512, 300])
+    tok = wl.token_ids(4, shape.vocab).tolist()
+    _walk(case, [([tok[0]], [0], [256]),
+                 (tok[:3], [0, 1, 2], [257, 1000, 512]),
+                 (tok, [0, 1, 2, 3], [258, 1001, 513, 300])])
