@@ -324,6 +324,82 @@ def batch_sweep(s, w, dev, n_steps=100, batches=(1, 2, 4)):
                                       "this build runs B <= 4", "cases": cases}
 
 
+def moe_decoder_bench(dev, n_steps=64):
+    """The MoE decoder: 16 layers with the 1B attention shape, each FFN the
+    64-expert top-8 layer (F 1408), vocab 128256, tied embeddings; Zipf(1.2)
+    skewed routing; dynamic schedule; continuous batching with the batch
+    size drawn per step from {1, 2, 3, 4} (this build's B limit) and
+    contexts starting uniform in [256, 4096].  Its 17.7 GB of expert weights
+    are drawn on the device (N(0, 0.02) bf16 from a seeded generator): this
+    leg times the path; parity is tested on a two-layer model whose weights
+    come from the seeded host generators."""
+    import torch
+    import event_tensor_task_b200 as mk
+    import workloads as wl
+    s = wl.DenseShape(n_layers=16, hidden=2048, n_q_heads=32, n_kv_heads=8, head_dim=64, ffn=8192, vocab=128256)
+    ms = wl.MOE_64x8
+    H, D, L = s.hidden, s.head_dim, s.n_layers
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+
+    def rnd(*shape):
+        return (torch.randn(*shape, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+
+    w = {"embed": rnd(s.vocab, H), "final_norm": torch.ones(H, dtype=torch.bfloat16, device=dev)}
+    mlayers = []
+    for l in range(L):
+        p = f"layers.{l}."
+        w[p + "attn_norm"] = torch.ones(H, dtype=torch.bfloat16, device=dev)
+        w[p + "ffn_norm"] = torch.ones(H, dtype=torch.bfloat16, device=dev)
+        w[p + "wq"], w[p + "wk"], w[p + "wv"] = rnd(32 * D, H), rnd(8 * D, H), rnd(8 * D, H)
+        w[p + "wo"] = rnd(H, 32 * D)
+        mlayers.append({"router": rnd(ms.n_experts, H), "w_gate": rnd(ms.n_experts, ms.expert_ffn, H),
+                        "w_up": rnd(ms.n_experts, ms.expert_ffn, H), "w_down": rnd(ms.n_experts, H, ms.expert_ffn)})
+    bias = wl.zipf_bias(ms.n_experts).to(dev)
+    maxB = 4
+    ctx0 = [int(c) for c in wl.context_lengths(maxB, 256, 4096, stream="moe-decoder-ctx")]
+    max_ctx = max(ctx0) + n_steps + 16
+    K = torch.zeros(L, maxB, s.n_kv_heads, max_ctx, D, dtype=torch.bfloat16, device=dev)
+    V = torch.zeros_like(K)
+    for b in range(maxB):
+        K[:, b, :, :ctx0[b]] = torch.randn(L, s.n_kv_heads, ctx0[b], D, generator=gen, device=dev).to(torch.bfloat16)
+        V[:, b, :, :ctx0[b]] = torch.randn(L, s.n_kv_heads, ctx0[b], D, generator=gen, device=dev).to(torch.bfloat16)
+    dec = mk.DenseDecoder(s, w, K, V, max_batch=maxB, max_ctx=max_ctx, n_slots=maxB, moe=(ms, mlayers, bias))
+    sched = wl.batch_schedule(n_steps + 3, [1, 2, 3, 4])
+    ran = [0] * maxB
+    args = []
+    for i, B in enumerate(sched):
+        ctx = [ctx0[b] + ran[b] for b in range(B)]
+        for b in range(B):
+            ran[b] += 1
+        args.append((torch.full((B,), 7, dtype=torch.int32, device=dev), torch.arange(B, dtype=torch.int32, device=dev),
+                     torch.tensor(ctx, dtype=torch.int32, device=dev), torch.empty(B, dtype=torch.int32, device=dev)))
+    for a in args[:3]:
+        dec.step(*a)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_steps + 1)]
+    ev[0].record()
+    for i, a in enumerate(args[3:]):
+        dec.step(*a)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    code, _ = dec.status()
+    if code != 0:
+        raise SystemExit(f"MoE decoder device status {code}")
+    per = {}
+    for i, B in enumerate(sched[3:]):
+        per.setdefault(B, []).append(ev[i].elapsed_time(ev[i + 1]))
+    total_ms = ev[0].elapsed_time(ev[-1])
+    tokens = sum(sched[3:])
+    dec.close()
+    return {"workload": "MoE decoder: 16 layers (1B attention shape), 64 experts top-8 F 1408 per layer, vocab 128256, "
+                        "Zipf(1.2) routing, dynamic schedule, B per step from {1,2,3,4}, contexts from U[256,4096]",
+            "steps": n_steps, "tokens": tokens, "tokens_per_s": tokens / (total_ms / 1000.0),
+            "us_per_step": 1000.0 * total_ms / n_steps,
+            "us_per_step_by_B": {str(B): 1000.0 * statistics.mean(v) for B, v in sorted(per.items())},
+            "weights": "device-drawn N(0,0.02) bf16 (seeded); parity is tested on a two-layer model"}
+
+
 def moe_layer_bench(dev, n_iter=10):
     """The MoE FFN layer (64 experts, top-8, F 1408, hidden 2048) for
     T in {1, 8, 64, 512} with uniform and Zipf(1.2)-skewed routing: device
@@ -434,6 +510,7 @@ def main():
     ap.add_argument("--no-torch-baseline", action="store_true")
     ap.add_argument("--no-moe", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-moe-decoder", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -555,6 +632,9 @@ def main():
     sweep = None
     if world == 1 and not args.no_sweep:
         sweep = batch_sweep(s, w, dev)
+    moe_dec = None
+    if world == 1 and not args.no_moe_decoder:
+        moe_dec = moe_decoder_bench(dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -580,6 +660,7 @@ def main():
         "torch_baselines": baselines,
         "moe_layer": moe,
         "batch_sweep": sweep,
+        "moe_decoder": moe_dec,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 12, "d2h_bytes_per_step": 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
