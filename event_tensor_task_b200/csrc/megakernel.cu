@@ -1537,6 +1537,150 @@ __device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, const unsigned cha
   return m;
 }
 
+// ---- tensor-core tiles (tiles of >= 16 routed rows)
+// Warp-level bf16 MMA m16n8k16 with fp32 accumulation.  K is walked in
+// windows of 32: lane (g = lane / 4, q = lane % 4) loads one 16-byte chunk,
+// columns [8q, 8q + 8) of the window, of each row it needs, and the two MMAs
+// of the window take its halves.  The logical-k -> column map is the same
+// for both operands, so each MMA pairs matching columns and the two MMAs
+// together cover the window's 32 columns once.
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_window(float (&c)[4], const uint4& ua, const uint4& ub, const uint4& wb) {
+  mma_16816(c, ua.x, ub.x, ua.y, ub.y, wb.x, wb.y);
+  mma_16816(c, ua.z, ub.z, ua.w, ub.w, wb.z, wb.w);
+}
+
+// EGU tile on tensor cores: warp w computes the 16 x 8 block (routed rows
+// 16*(w/2) .., gate rows if w is even, up rows if odd) over K = hidden; the
+// up warp hands its block to the gate warp through shared memory for SwiGLU.
+__device__ __forceinline__ void task_egu_mma(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
+                                             unsigned char* mb, Control* ctl, const TaskDesc& d, const MoeTile& mt,
+                                             int n) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int g = lane >> 2, q = lane & 3;
+  const int H = P.hidden, K = P.top_k;
+  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
+  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
+  const int rps = P.slot_bytes / (2 * H), spp = (P.moe_tn + rps - 1) / rps;
+  const int mbk = w >> 1, nb = w & 1;  // m block; part 0 (gate) or 1 (up)
+  const int n_mb = (mt.nrows + 15) >> 4;
+  const bool active = mbk < n_mb;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+    for (int j = 0; j < spp; ++j) {
+      const int js = s0 + nb * spp + j;
+      wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    }
+    const int jg = s0 + nb * spp + g / rps;
+    const unsigned char* brow = ring + (size_t)(jg < R ? jg : jg - R) * P.slot_bytes + (size_t)(g % rps) * 2 * H;
+    const int* mperm = reinterpret_cast<const int*>(mb + P.off_mperm);
+    const __nv_bfloat16* xsrc = P.kind == MK_MODEL_MOE_DECODER
+                                    ? reinterpret_cast<const __nv_bfloat16*>(mb + P.off_mxhat) : S.moe_x;
+    const int rlo = mbk * 16 + g, rhi = rlo + 8;
+    const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
+    const uint4* alo = vlo ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rlo) / K) * H) : nullptr;
+    const uint4* ahi = vhi ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rhi) / K) * H) : nullptr;
+    const uint4* bp = reinterpret_cast<const uint4*>(brow);
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 4
+    for (int k0 = 0; k0 < H; k0 += 32) {
+      const int c = (k0 >> 3) + q;  // 16-byte chunk of the row
+      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
+      mma_window(acc, ua, ub, bp[c]);
+    }
+    __syncwarp();
+    if (lane == 0)
+      for (int j = 0; j < spp; ++j) {
+        const int js = s0 + nb * spp + j;
+        release_share(sm, js < R ? js : js - R, n_mb, mbk);  // the part's slots are read by its n_mb warps
+      }
+  }
+  // up -> gate hand-over (the staging buffer as scratch)
+  float* xch = sm.xs;
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (active && nb == 1)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xch[(mbk * 32 + lane) * 4 + i] = acc[i];
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (active && nb == 0) {
+    __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mh);
+    const int col = n * P.moe_tn + 2 * q;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = mbk * 16 + g + (i >> 1) * 8;
+      const float gt = acc[i], up = xch[(mbk * 32 + lane) * 4 + i];
+      if (r < mt.nrows && col + (i & 1) < P.eff)
+        mh[(size_t)(mt.r0 + r) * P.eff + col + (i & 1)] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
+    }
+  }
+}
+
+// EDOWN tile on tensor cores: warp w computes the 16 x 8 block of routed rows
+// 16*(w/2) .. and the task's 8 down rows over half of K (even warps the first
+// half of the windows, odd warps the second); the halves are added through
+// shared memory.
+__device__ __forceinline__ void task_edown_mma(const DevPlan& P, Smem& sm, unsigned char* ring, unsigned char* mb,
+                                               Control* ctl, const TaskDesc& d, const MoeTile& mt, int n) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int g = lane >> 2, q = lane & 3;
+  const int H = P.hidden, FF = P.eff;
+  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
+  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
+  const int rps = P.slot_bytes / 4096, nsl = (P.moe_td + rps - 1) / rps;
+  const int mbk = w >> 1, kh = w & 1;
+  const int n_mb = (mt.nrows + 15) >> 4;
+  const bool active = mbk < n_mb;
+  const int nwin = FF >> 5, w0 = kh ? nwin / 2 : 0, w1 = kh ? nwin : nwin / 2;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+    for (int j = 0; j < nsl; ++j) {
+      const int js = s0 + j;
+      wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    }
+    const int jg = s0 + g / rps;
+    const uint4* bp = reinterpret_cast<const uint4*>(ring + (size_t)(jg < R ? jg : jg - R) * P.slot_bytes +
+                                                     (size_t)(g % rps) * 4096);
+    const uint4* mh = reinterpret_cast<const uint4*>(mb + P.off_mh);
+    const int rlo = mbk * 16 + g, rhi = rlo + 8;
+    const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
+    const uint4* alo = mh + ((size_t)(mt.r0 + (vlo ? rlo : 0)) * FF) / 8;
+    const uint4* ahi = mh + ((size_t)(mt.r0 + (vhi ? rhi : 0)) * FF) / 8;
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 4
+    for (int wi = w0; wi < w1; ++wi) {
+      const int c = wi * 4 + q;
+      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
+      mma_window(acc, ua, ub, bp[c]);
+    }
+    __syncwarp();
+    if (lane == 0)
+      for (int j = 0; j < nsl; ++j) {
+        const int js = s0 + j;
+        release_share(sm, js < R ? js : js - R, 2 * n_mb, w);  // all active warps read every slot
+      }
+  }
+  float* xch = sm.xs;
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (active && kh == 1)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xch[(mbk * 32 + lane) * 4 + i] = acc[i];
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (active && kh == 0) {
+    float* my = reinterpret_cast<float*>(mb + P.off_my);
+    const int col = n * P.moe_td + 2 * q;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = mbk * 16 + g + (i >> 1) * 8;
+      if (r < mt.nrows) my[(size_t)(mt.r0 + r) * H + col + (i & 1)] = acc[i] + xch[(mbk * 32 + lane) * 4 + i];
+    }
+  }
+}
+
 // EGU task (tile, n): warp w takes gate row n*tn + w and up row n*tn + w of
 // the tile's expert into registers (freeing its ring slots at once), then
 // runs them over the tile's rows: h[row] = silu(x W_g^T) * (x W_u^T), with x
@@ -1545,6 +1689,15 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
                                          unsigned char* ws, Control* ctl, const TaskDesc& d) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int H = P.hidden, nblk = H >> 8, K = P.top_k;
+  {
+    const int tile = d.idx / P.nt_gu;
+    unsigned char* mb = moe_block(P, ws, d.layer);
+    const MoeTile mt = moe_tile(P, mb, tile);
+    if (mt.nrows >= 16) {  // a real contraction: tensor cores
+      task_egu_mma(P, S, sm, ring, mb, ctl, d, mt, d.idx - tile * P.nt_gu);
+      return;
+    }
+  }
   const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
   const int rps = P.slot_bytes / (2 * H), spp = (P.moe_tn + rps - 1) / rps;
@@ -1627,6 +1780,15 @@ __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S
                                            unsigned char* ws, Control* ctl, const TaskDesc& d) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int H = P.hidden, FF = P.eff, nch = FF / 8;
+  {
+    const int tile = d.idx / P.nt_d;
+    unsigned char* mb = moe_block(P, ws, d.layer);
+    const MoeTile mt = moe_tile(P, mb, tile);
+    if (mt.nrows >= 16 && FF % 64 == 0) {  // a real contraction: tensor cores (K in windows of 32, split in two)
+      task_edown_mma(P, sm, ring, mb, ctl, d, mt, d.idx - tile * P.nt_d);
+      return;
+    }
+  }
   const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
   const int rps = P.slot_bytes / 4096;
@@ -1761,7 +1923,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
       }
     }
     if (kKind == MK_MODEL_MOE_LAYER || moe_task) {
-      // (done above)
+      a_tag = -1;  // MoE tasks use the staging buffer as scratch
     } else if (gemv_spec(P, d, g)) {
       // one pass per batch row (the activation is restaged each pass when
       // B > 1); the ring slots are released after the last pass
