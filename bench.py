@@ -324,6 +324,24 @@ def batch_sweep(s, w, dev, n_steps=100, batches=(1, 2, 4)):
                                       "this build runs B <= 4", "cases": cases}
 
 
+def profile_moe(T):
+    """Four calls of the 64-expert top-8 MoE layer on T tokens (uniform routing)."""
+    import torch
+    import event_tensor_task_b200 as mk
+    import workloads as wl
+    dev = "cuda:0"
+    w = {k: v.to(dev) for k, v in wl.moe_weights(wl.MOE_64x8, seed=0).items()}
+    layer = mk.MoELayer(wl.MOE_64x8, w, None, max_tokens=max(T, 8))
+    x = wl.moe_tokens(T, wl.MOE_64x8.hidden, seed=0).to(dev)
+    out = torch.empty(T, wl.MOE_64x8.hidden, dtype=torch.bfloat16, device=dev)
+    for _ in range(4):
+        layer(x, out)
+    torch.cuda.synchronize()
+    code, _ = layer.status()
+    if code != 0:
+        raise SystemExit(f"MoE layer device status {code}")
+
+
 def moe_decoder_bench(dev, n_steps=64):
     """The MoE decoder: 16 layers with the 1B attention shape, each FFN the
     64-expert top-8 layer (F 1408), vocab 128256, tied embeddings; Zipf(1.2)
@@ -511,6 +529,8 @@ def main():
     ap.add_argument("--no-moe", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-moe-decoder", action="store_true")
+    ap.add_argument("--profile-moe", type=int, default=0, metavar="T",
+                    help="only run 4 MoE-layer calls on T tokens (a short command for ncu) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -519,6 +539,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.profile_moe:
+        profile_moe(args.profile_moe)
         return
 
     import torch
