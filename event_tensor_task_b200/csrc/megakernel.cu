@@ -1555,292 +1555,185 @@ __device__ __forceinline__ void mma_window(float (&c)[4], const uint4& ua, const
   mma_16816(c, ua.z, ub.z, ua.w, ub.w, wb.z, wb.w);
 }
 
-// EGU tile on tensor cores: warp w computes the 16 x 8 block (routed rows
-// 16*(w/2) .., gate rows if w is even, up rows if odd) over K = hidden; the
-// up warp hands its block to the gate warp through shared memory for SwiGLU.
-__device__ __forceinline__ void task_egu_mma(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
-                                             unsigned char* mb, Control* ctl, const TaskDesc& d, const MoeTile& mt,
-                                             int n) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int H = P.hidden, K = P.top_k;
-  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
-  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int rps = P.slot_bytes / (2 * H), spp = (P.moe_tn + rps - 1) / rps;
-  const int mbk = w >> 1, nb = w & 1;  // m block; part 0 (gate) or 1 (up)
-  const int n_mb = (mt.nrows + 15) >> 4;
-  const bool active = mbk < n_mb;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (active) {
-    for (int j = 0; j < spp; ++j) {
-      const int js = s0 + nb * spp + j;
-      wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-    }
-    const int jg = s0 + nb * spp + g / rps;
-    const unsigned char* brow = ring + (size_t)(jg < R ? jg : jg - R) * P.slot_bytes + (size_t)(g % rps) * 2 * H;
-    const int* mperm = reinterpret_cast<const int*>(mb + P.off_mperm);
-    const __nv_bfloat16* xsrc = P.kind == MK_MODEL_MOE_DECODER
-                                    ? reinterpret_cast<const __nv_bfloat16*>(mb + P.off_mxhat) : S.moe_x;
-    const int rlo = mbk * 16 + g, rhi = rlo + 8;
-    const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
-    const uint4* alo = vlo ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rlo) / K) * H) : nullptr;
-    const uint4* ahi = vhi ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rhi) / K) * H) : nullptr;
-    const uint4* bp = reinterpret_cast<const uint4*>(brow);
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 4
-    for (int k0 = 0; k0 < H; k0 += 32) {
-      const int c = (k0 >> 3) + q;  // 16-byte chunk of the row
-      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
-      mma_window(acc, ua, ub, bp[c]);
-    }
-    __syncwarp();
-    if (lane == 0)
-      for (int j = 0; j < spp; ++j) {
-        const int js = s0 + nb * spp + j;
-        release_share(sm, js < R ? js : js - R, n_mb, mbk);  // the part's slots are read by its n_mb warps
-      }
-  }
-  // up -> gate hand-over (the staging buffer as scratch)
-  float* xch = sm.xs;
-  bar_sync(BAR_COMP, kComputeThreads);
-  if (active && nb == 1)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) xch[(mbk * 32 + lane) * 4 + i] = acc[i];
-  bar_sync(BAR_COMP, kComputeThreads);
-  if (active && nb == 0) {
-    __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mh);
-    const int col = n * P.moe_tn + 2 * q;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = mbk * 16 + g + (i >> 1) * 8;
-      const float gt = acc[i], up = xch[(mbk * 32 + lane) * 4 + i];
-      if (r < mt.nrows && col + (i & 1) < P.eff)
-        mh[(size_t)(mt.r0 + r) * P.eff + col + (i & 1)] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
-    }
-  }
+// Readers of the ring slots of an n x (rows of 8) block layout: the slots of
+// one part hold rows [j*rps, (j+1)*rps) of its 16 rows; the warps (m block
+// mb, half nh) read the slots holding rows [8*nh, 8*nh + 8).  Returns the
+// number of readers of slot j and this warp's rank among them.
+__device__ __forceinline__ void half_readers(int j, int rps, int n_mb, int mb, int nh, int& readers, int& rank) {
+  const int lo = j * rps, hi = min((j + 1) * rps, 16);
+  const bool h0 = lo < 8, h1 = hi > 8;
+  readers = n_mb * ((h0 ? 1 : 0) + (h1 ? 1 : 0));
+  rank = (nh == 1 && h0 ? n_mb : 0) + mb;
 }
 
-// EDOWN tile on tensor cores: warp w computes the 16 x 8 block of routed rows
-// 16*(w/2) .. and the task's 8 down rows over half of K (even warps the first
-// half of the windows, odd warps the second); the halves are added through
-// shared memory.
-__device__ __forceinline__ void task_edown_mma(const DevPlan& P, Smem& sm, unsigned char* ring, unsigned char* mb,
-                                               Control* ctl, const TaskDesc& d, const MoeTile& mt, int n) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int H = P.hidden, FF = P.eff;
-  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
-  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int rps = P.slot_bytes / 4096, nsl = (P.moe_td + rps - 1) / rps;
-  const int mbk = w >> 1, kh = w & 1;
-  const int n_mb = (mt.nrows + 15) >> 4;
-  const bool active = mbk < n_mb;
-  const int nwin = FF >> 5, w0 = kh ? nwin / 2 : 0, w1 = kh ? nwin : nwin / 2;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (active) {
-    for (int j = 0; j < nsl; ++j) {
-      const int js = s0 + j;
-      wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-    }
-    const int jg = s0 + g / rps;
-    const uint4* bp = reinterpret_cast<const uint4*>(ring + (size_t)(jg < R ? jg : jg - R) * P.slot_bytes +
-                                                     (size_t)(g % rps) * 4096);
-    const uint4* mh = reinterpret_cast<const uint4*>(mb + P.off_mh);
-    const int rlo = mbk * 16 + g, rhi = rlo + 8;
-    const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
-    const uint4* alo = mh + ((size_t)(mt.r0 + (vlo ? rlo : 0)) * FF) / 8;
-    const uint4* ahi = mh + ((size_t)(mt.r0 + (vhi ? rhi : 0)) * FF) / 8;
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 4
-    for (int wi = w0; wi < w1; ++wi) {
-      const int c = wi * 4 + q;
-      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
-      mma_window(acc, ua, ub, bp[c]);
-    }
-    __syncwarp();
-    if (lane == 0)
-      for (int j = 0; j < nsl; ++j) {
-        const int js = s0 + j;
-        release_share(sm, js < R ? js : js - R, 2 * n_mb, w);  // all active warps read every slot
-      }
-  }
-  float* xch = sm.xs;
-  bar_sync(BAR_COMP, kComputeThreads);
-  if (active && kh == 1)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) xch[(mbk * 32 + lane) * 4 + i] = acc[i];
-  bar_sync(BAR_COMP, kComputeThreads);
-  if (active && kh == 0) {
-    float* my = reinterpret_cast<float*>(mb + P.off_my);
-    const int col = n * P.moe_td + 2 * q;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = mbk * 16 + g + (i >> 1) * 8;
-      if (r < mt.nrows) my[(size_t)(mt.r0 + r) * H + col + (i & 1)] = acc[i] + xch[(mbk * 32 + lane) * 4 + i];
-    }
-  }
-}
-
-// EGU task (tile, n): warp w takes gate row n*tn + w and up row n*tn + w of
-// the tile's expert into registers (freeing its ring slots at once), then
-// runs them over the tile's rows: h[row] = silu(x W_g^T) * (x W_u^T), with x
-// gathered straight from the layer input by the row map.
+// EGU task (tile, n) on tensor cores: gate rows and up rows 16n .. 16n+15 of
+// the tile's expert against its routed rows (<= 64, gathered straight from
+// the layer input by the row map).  Warp w computes the 16 x 8 blocks of
+// routed rows 16*(w/2) .. for gate and up columns 8*(w%2) .. of the task, so
+// SwiGLU is applied in registers.
 __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                          unsigned char* ws, Control* ctl, const TaskDesc& d) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int H = P.hidden, nblk = H >> 8, K = P.top_k;
-  {
-    const int tile = d.idx / P.nt_gu;
-    unsigned char* mb = moe_block(P, ws, d.layer);
-    const MoeTile mt = moe_tile(P, mb, tile);
-    if (mt.nrows >= 16) {  // a real contraction: tensor cores
-      task_egu_mma(P, S, sm, ring, mb, ctl, d, mt, d.idx - tile * P.nt_gu);
-      return;
-    }
-  }
+  const int g = lane >> 2, q = lane & 3;
+  const int H = P.hidden, K = P.top_k, TN = P.moe_tn;
   const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int rps = P.slot_bytes / (2 * H), spp = (P.moe_tn + rps - 1) / rps;
-  const int ja = w / rps, jb = spp + ja;
-  const int readers = min(rps, P.moe_tn - ja * rps);  // warps whose rows lie in slot ja (and jb)
-  const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R, sb = s0 + jb < R ? s0 + jb : s0 + jb - R;
-  wait_mbar(&sm.full[sa], s0 + ja < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  wait_mbar(&sm.full[sb], s0 + jb < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  const int roff = (w - ja * rps) * 2 * H;
-  const uint4* ga = reinterpret_cast<const uint4*>(ring + (size_t)sa * P.slot_bytes + roff) + lane;
-  const uint4* ua = reinterpret_cast<const uint4*>(ring + (size_t)sb * P.slot_bytes + roff) + lane;
-  uint4 gw[kMaxBlk], uw[kMaxBlk];
-#pragma unroll
-  for (int i = 0; i < kMaxBlk; ++i)
-    if (i < nblk) { gw[i] = ga[i * 32]; uw[i] = ua[i * 32]; }
-  __syncwarp();
-  if (lane == 0) {
-    release_share(sm, sa, readers, w - ja * rps);
-    release_share(sm, sb, readers, w - ja * rps);
-  }
   const int tile = d.idx / P.nt_gu, n = d.idx - tile * P.nt_gu;
   unsigned char* mb = moe_block(P, ws, d.layer);
   const MoeTile mt = moe_tile(P, mb, tile);
+  const int rps = P.slot_bytes / (2 * H), spp = (TN + rps - 1) / rps;
+  // warp pairs (w / 2) take the m blocks; when there are fewer than 4, the
+  // spare pairs split K with them (ks parts, added through shared memory)
+  const int n_mb = (mt.nrows + 15) >> 4;
+  const int ks = n_mb == 1 ? 4 : (n_mb == 2 ? 2 : 1);
+  const int pair = w >> 1, nh = w & 1;
+  const int mbk = pair % n_mb, kp = pair / n_mb;
+  const int n_act = n_mb * ks;  // active warp pairs
+  const bool active = pair < n_act;
+  const int nwin = H >> 5, win0 = kp * nwin / ks, win1 = (kp + 1) * nwin / ks;
+  const int jlo = (8 * nh) / rps, jhi = (8 * nh + 7) / rps;  // this warp's slots within each part
+  float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+  for (int part = 0; part < 2; ++part)
+    for (int j = jlo; j <= jhi; ++j) {
+      const int js = s0 + part * spp + j;
+      wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    }
+  const int row = 8 * nh + g;  // weight row of this lane within each part
+  const int jg = s0 + row / rps, ju = s0 + spp + row / rps;
+  const size_t roff = (size_t)(row % rps) * 2 * H;
+  const uint4* bg = reinterpret_cast<const uint4*>(ring + (size_t)(jg < R ? jg : jg - R) * P.slot_bytes + roff);
+  const uint4* bu = reinterpret_cast<const uint4*>(ring + (size_t)(ju < R ? ju : ju - R) * P.slot_bytes + roff);
   const int* mperm = reinterpret_cast<const int*>(mb + P.off_mperm);
-  const uint4* xr = reinterpret_cast<const uint4*>(P.kind == MK_MODEL_MOE_DECODER ? (const void*)(mb + P.off_mxhat)
-                                                                                  : (const void*)S.moe_x);
-  __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mh);
-  const int col = n * P.moe_tn + w;
-  // the tile's row -> token map, one entry per lane (tm <= 64 rows)
-  const int tok0 = lane < mt.nrows ? __ldcg(mperm + mt.r0 + lane) / K : 0;
-  const int tok1 = lane + 32 < mt.nrows ? __ldcg(mperm + mt.r0 + lane + 32) / K : 0;
-  // two rows at a time: both rows' activation loads are in flight together
-  for (int rr = 0; rr < mt.nrows; rr += 2) {
-    const bool two = rr + 1 < mt.nrows;
-    const int ta = __shfl_sync(0xffffffffu, rr < 32 ? tok0 : tok1, rr & 31);
-    const int tb = __shfl_sync(0xffffffffu, rr + 1 < 32 ? tok0 : tok1, (rr + 1) & 31);
-    const uint4* xa = xr + ((size_t)ta * H + 8 * lane) / 8;
-    const uint4* xb = xr + ((size_t)(two ? tb : ta) * H + 8 * lane) / 8;
-    float ag[2] = {0.f, 0.f}, au[2] = {0.f, 0.f}, bg[2] = {0.f, 0.f}, bu[2] = {0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < kMaxBlk; ++i)
-      if (i < nblk) {
-        float xf[8], yf[8], gf[8], uf[8];
-        uint4 g4 = gw[i], u4 = uw[i];
-        // keep the weights packed: converting them once outside the row loop
-        // would hold 128 floats and spill
-        asm volatile("" : "+r"(g4.x), "+r"(g4.y), "+r"(g4.z), "+r"(g4.w), "+r"(u4.x), "+r"(u4.y), "+r"(u4.z), "+r"(u4.w));
-        bf16x8_to_f32(__ldcg(xa + 32 * i), xf);
-        bf16x8_to_f32(__ldcg(xb + 32 * i), yf);
-        bf16x8_to_f32(g4, gf);
-        bf16x8_to_f32(u4, uf);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          ag[j & 1] = fmaf(gf[j], xf[j], ag[j & 1]);
-          au[j & 1] = fmaf(uf[j], xf[j], au[j & 1]);
-          bg[j & 1] = fmaf(gf[j], yf[j], bg[j & 1]);
-          bu[j & 1] = fmaf(uf[j], yf[j], bu[j & 1]);
-        }
+  const __nv_bfloat16* xsrc = P.kind == MK_MODEL_MOE_DECODER
+                                  ? reinterpret_cast<const __nv_bfloat16*>(mb + P.off_mxhat) : S.moe_x;
+  const int rlo = mbk * 16 + g, rhi = rlo + 8;
+  const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
+  const uint4* alo = vlo ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rlo) / K) * H) : nullptr;
+  const uint4* ahi = vhi ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rhi) / K) * H) : nullptr;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 4
+  for (int wi = win0; wi < win1; ++wi) {
+    const int c = wi * 4 + q;  // 16-byte chunk of the row
+    const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
+    mma_window(ag, ua, ub, bg[c]);
+    mma_window(au, ua, ub, bu[c]);
+  }
+  __syncwarp();
+  if (lane == 0)
+    for (int part = 0; part < 2; ++part)
+      for (int j = jlo; j <= jhi; ++j) {
+        int readers, rank;
+        half_readers(j, rps, n_act, pair, nh, readers, rank);
+        const int js = s0 + part * spp + j;
+        release_share(sm, js < R ? js : js - R, readers, rank);
       }
-    float g = ag[0] + ag[1], u = au[0] + au[1], g2 = bg[0] + bg[1], u2 = bu[0] + bu[1];
+  }
+  if (ks > 1) {
+    // K parts 1.. hand their sums to part 0 (the staging buffer as scratch)
+    float* xch = sm.xs;
+    bar_sync(BAR_COMP, kComputeThreads);
+    // entry e = ((kp - 1) * n_mb + mbk) * 2 + nh < (ks - 1) * n_mb * 2 <= 6, 256 floats each (<= 1536 of 2048)
+    if (active && kp > 0) {
+      float* e = xch + ((((kp - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 8;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      g += __shfl_xor_sync(0xffffffffu, g, o);
-      u += __shfl_xor_sync(0xffffffffu, u, o);
-      g2 += __shfl_xor_sync(0xffffffffu, g2, o);
-      u2 += __shfl_xor_sync(0xffffffffu, u2, o);
+      for (int i = 0; i < 4; ++i) { e[i] = ag[i]; e[4 + i] = au[i]; }
     }
-    if (lane == 0 && col < P.eff) {
-      const int row = mt.r0 + rr;
-      mh[(size_t)row * P.eff + col] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
-      if (two) mh[(size_t)(row + 1) * P.eff + col] = __float2bfloat16_rn(g2 / (1.0f + expf(-g2)) * u2);
-    }
+    bar_sync(BAR_COMP, kComputeThreads);
+    if (active && kp == 0)
+      for (int o = 1; o < ks; ++o) {
+        const float* e = xch + ((((o - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { ag[i] += e[i]; au[i] += e[4 + i]; }
+      }
+  }
+  if (!active || kp > 0) return;
+  __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mh);
+  const int col = n * TN + 8 * nh + 2 * q;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = mbk * 16 + g + (i >> 1) * 8;
+    const float gt = ag[i];
+    if (r < mt.nrows) mh[(size_t)(mt.r0 + r) * P.eff + col + (i & 1)] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * au[i]);
   }
 }
 
-// EDOWN task (tile, n): warp w takes down row n*td + w (expert_ffn long, in
-// 8-element chunks c = lane + 32 i) into registers, then runs it over the
-// tile's rows of h: y[row][n*td + w] = h[row] . W_d[n*td + w].
+// EDOWN task (tile, n) on tensor cores: down rows 16n .. 16n+15 of the tile's
+// expert (expert_ffn long, at a 4 KB pitch in the ring) against the tile's
+// rows of h.  Warp w computes the 16 x 8 block of routed rows 16*(w/2) .. and
+// down rows 8*(w%2) .. over the whole of K.
 __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                            unsigned char* ws, Control* ctl, const TaskDesc& d) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int H = P.hidden, FF = P.eff, nch = FF / 8;
-  {
-    const int tile = d.idx / P.nt_d;
-    unsigned char* mb = moe_block(P, ws, d.layer);
-    const MoeTile mt = moe_tile(P, mb, tile);
-    if (mt.nrows >= 16 && FF % 64 == 0) {  // a real contraction: tensor cores (K in windows of 32, split in two)
-      task_edown_mma(P, sm, ring, mb, ctl, d, mt, d.idx - tile * P.nt_d);
-      return;
-    }
-  }
+  const int g = lane >> 2, q = lane & 3;
+  const int H = P.hidden, FF = P.eff, TD = P.moe_td;
   const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int rps = P.slot_bytes / 4096;
-  const int ja = w / rps;
-  const int readers = min(rps, P.moe_td - ja * rps);
-  const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R;
-  wait_mbar(&sm.full[sa], s0 + ja < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  const uint4* dr = reinterpret_cast<const uint4*>(ring + (size_t)sa * P.slot_bytes + (w - ja * rps) * 4096);
-  uint4 dw[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (lane + 32 * i < nch) dw[i] = dr[lane + 32 * i];
-  __syncwarp();
-  if (lane == 0) release_share(sm, sa, readers, w - ja * rps);
   const int tile = d.idx / P.nt_d, n = d.idx - tile * P.nt_d;
   unsigned char* mb = moe_block(P, ws, d.layer);
   const MoeTile mt = moe_tile(P, mb, tile);
+  const int rps = P.slot_bytes / 4096;
+  const int n_mb = (mt.nrows + 15) >> 4;
+  const int ks = n_mb == 1 ? 4 : (n_mb == 2 ? 2 : 1);  // spare warp pairs split K (see task_egu)
+  const int pair = w >> 1, nh = w & 1;
+  const int mbk = pair % n_mb, kp = pair / n_mb;
+  const int n_act = n_mb * ks;
+  const bool active = pair < n_act;
+  const int nwin = FF >> 5, win0 = kp * nwin / ks, win1 = (kp + 1) * nwin / ks;
+  const int jlo = (8 * nh) / rps, jhi = (8 * nh + 7) / rps;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+  for (int j = jlo; j <= jhi; ++j) {
+    const int js = s0 + j;
+    wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  }
+  const int row = 8 * nh + g, jr = s0 + row / rps;
+  const uint4* bp = reinterpret_cast<const uint4*>(ring + (size_t)(jr < R ? jr : jr - R) * P.slot_bytes +
+                                                   (size_t)(row % rps) * 4096);
   const uint4* mh = reinterpret_cast<const uint4*>(mb + P.off_mh);
-  float* my = reinterpret_cast<float*>(mb + P.off_my);
-  const int col = n * P.moe_td + w;
-  // two rows at a time (their loads in flight together)
-  for (int rr = 0; rr < mt.nrows; rr += 2) {
-    const int row = mt.r0 + rr;
-    const bool two = rr + 1 < mt.nrows;
-    const uint4* ha = mh + ((size_t)row * FF) / 8 + lane;
-    const uint4* hb = mh + ((size_t)(two ? row + 1 : row) * FF) / 8 + lane;
-    float acc[2] = {0.f, 0.f}, bcc[2] = {0.f, 0.f};
+  const int rlo = mbk * 16 + g, rhi = rlo + 8;
+  const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
+  const uint4* alo = mh + ((size_t)(mt.r0 + (vlo ? rlo : 0)) * FF) / 8;
+  const uint4* ahi = mh + ((size_t)(mt.r0 + (vhi ? rhi : 0)) * FF) / 8;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 4
+  for (int wi = win0; wi < win1; ++wi) {
+    const int c = wi * 4 + q;
+    const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
+    mma_window(acc, ua, ub, bp[c]);
+  }
+  __syncwarp();
+  if (lane == 0)
+    for (int j = jlo; j <= jhi; ++j) {
+      int readers, rank;
+      half_readers(j, rps, n_act, pair, nh, readers, rank);
+      const int js = s0 + j;
+      release_share(sm, js < R ? js : js - R, readers, rank);
+    }
+  }
+  if (ks > 1) {
+    float* xch = sm.xs;  // entries as in task_egu, 4 floats per lane
+    bar_sync(BAR_COMP, kComputeThreads);
+    if (active && kp > 0) {
+      float* e = xch + ((((kp - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 4;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (lane + 32 * i < nch) {
-        float hf[8], kf[8], wf[8];
-        uint4 d4 = dw[i];
-        asm volatile("" : "+r"(d4.x), "+r"(d4.y), "+r"(d4.z), "+r"(d4.w));  // convert per use (see task_egu)
-        bf16x8_to_f32(__ldcg(ha + 32 * i), hf);
-        bf16x8_to_f32(__ldcg(hb + 32 * i), kf);
-        bf16x8_to_f32(d4, wf);
+      for (int i = 0; i < 4; ++i) e[i] = acc[i];
+    }
+    bar_sync(BAR_COMP, kComputeThreads);
+    if (active && kp == 0)
+      for (int o = 1; o < ks; ++o) {
+        const float* e = xch + ((((o - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 4;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          acc[j & 1] = fmaf(wf[j], hf[j], acc[j & 1]);
-          bcc[j & 1] = fmaf(wf[j], kf[j], bcc[j & 1]);
-        }
+        for (int i = 0; i < 4; ++i) acc[i] += e[i];
       }
-    float v = acc[0] + acc[1], v2 = bcc[0] + bcc[1];
+  }
+  if (!active || kp > 0) return;
+  float* my = reinterpret_cast<float*>(mb + P.off_my);
+  const int col = n * TD + 8 * nh + 2 * q;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      v += __shfl_xor_sync(0xffffffffu, v, o);
-      v2 += __shfl_xor_sync(0xffffffffu, v2, o);
-    }
-    if (lane == 0) {
-      my[(size_t)row * H + col] = v;
-      if (two) my[(size_t)(row + 1) * H + col] = v2;
-    }
+  for (int i = 0; i < 4; ++i) {
+    const int r = mbk * 16 + g + (i >> 1) * 8;
+    if (r < mt.nrows) my[(size_t)(mt.r0 + r) * H + col + (i & 1)] = acc[i];
   }
 }
 

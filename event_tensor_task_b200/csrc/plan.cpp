@@ -247,7 +247,7 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
   if (E < 1 || E > 64) { err = "n_experts must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
   if (K < 1 || K > 8 || K > E) { err = "top_k must be in [1, min(8, n_experts)]"; return MK_ERR_UNSUPPORTED; }
-  if (FF < 8 || FF % 8 || FF > 2048) { err = "expert_ffn must be a multiple of 8 in [8, 2048]"; return MK_ERR_UNSUPPORTED; }
+  if (FF < 32 || FF % 32 || FF > 2048) { err = "expert_ffn must be a multiple of 32 in [32, 2048]"; return MK_ERR_UNSUPPORTED; }
   if (TM < 1 || TM > 4096) { err = "max_tokens must be in [1, 4096]"; return MK_ERR_UNSUPPORTED; }
   if (o->sched != MK_SCHED_DYNAMIC)
     { err = "an MoE layer's task counts depend on the routing: use MK_SCHED_DYNAMIC"; return MK_ERR_UNSUPPORTED; }
@@ -266,13 +266,13 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
   P.n_experts = E; P.top_k = K; P.eff = FF; P.max_tokens = TM;
   P.moe_tm = 64;  // routed rows per GroupGEMM tile
-  P.moe_tn = 8;   // one gate/up row pair per compute warp
-  P.moe_td = 8;   // one down row per compute warp
+  P.moe_tn = 16;  // gate/up rows per EGU task (16 + 16: 8 ring slots at hidden 2048)
+  P.moe_td = 16;  // down rows per EDOWN task
   P.nt_gu = ceil_div(FF, P.moe_tn);
   P.nt_d = H / P.moe_td;
   // sum over experts of ceil(hist_e / tm) <= T*k/tm + (experts with a row)
   P.max_tiles = ceil_div(TM * K, P.moe_tm) + std::min(E, TM * K);
-  if (FF % P.moe_tn) { err = "expert_ffn must be a multiple of 8"; return MK_ERR_UNSUPPORTED; }
+  if (FF % P.moe_tn) { err = "expert_ffn must be a multiple of 16"; return MK_ERR_UNSUPPORTED; }
   P.slot_bytes = 16384;
   const int reserve = 19 * 1024;
   P.smem_bytes = smem_bytes;
@@ -358,7 +358,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     const int E = m->n_experts, K = m->top_k, FF = m->expert_ffn;
     if (E < 1 || E > 64) { err = "n_experts must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
     if (K < 1 || K > 8 || K > E) { err = "top_k must be in [1, min(8, n_experts)]"; return MK_ERR_UNSUPPORTED; }
-    if (FF < 8 || FF % 8 || FF > 2048) { err = "expert_ffn must be a multiple of 8 in [8, 2048]"; return MK_ERR_UNSUPPORTED; }
+    if (FF < 32 || FF % 32 || FF > 2048) { err = "expert_ffn must be a multiple of 32 in [32, 2048]"; return MK_ERR_UNSUPPORTED; }
     if (o->sched != MK_SCHED_DYNAMIC)
       { err = "an MoE layer's task counts depend on the routing: use MK_SCHED_DYNAMIC"; return MK_ERR_UNSUPPORTED; }
   }
@@ -483,7 +483,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (mdec) {
     P.kind = MK_MODEL_MOE_DECODER;
     P.n_experts = m->n_experts; P.top_k = m->top_k; P.eff = m->expert_ffn; P.max_tokens = P.max_batch;
-    P.moe_tm = 64; P.moe_tn = 8; P.moe_td = 8;
+    P.moe_tm = 64; P.moe_tn = 16; P.moe_td = 16;
     P.nt_gu = ceil_div(P.eff, P.moe_tn);
     P.nt_d = H / P.moe_td;
     P.max_tiles = ceil_div(P.max_tokens * P.top_k, P.moe_tm) + std::min(P.n_experts, P.max_tokens * P.top_k);

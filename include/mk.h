@@ -84,7 +84,7 @@ typedef struct mk_layer_weights {
  * MK_MODEL_DENSE: head_dim == 64, n_q_heads % n_kv_heads == 0, hidden and
  *   ffn multiples of 256 with hidden <= 2048, n_q_heads*head_dim == hidden.
  * MK_MODEL_MOE_LAYER: only hidden (multiple of 256, <= 2048), n_experts
- *   (<= 64), top_k (<= 8 and <= n_experts), expert_ffn (multiple of 8,
+ *   (<= 64), top_k (<= 8 and <= n_experts), expert_ffn (multiple of 32,
  *   <= 2048), max_tokens (<= 4096) and moe are read.
  * MK_MODEL_MOE_DECODER: the dense fields (ffn, and the dense FFN weights,
  *   are not used) plus n_experts, top_k, expert_ffn and each layer's moe;

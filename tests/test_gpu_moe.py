@@ -18,7 +18,7 @@ from gpu_common import rel_err, TOL
 
 pytestmark = pytest.mark.gpu
 
-TILES = {"tm": 64, "tn": 8, "td": 8}  # the plan's GroupGEMM tile sizes
+TILES = {"tm": 64, "tn": 16, "td": 16}  # the plan's GroupGEMM tile sizes
 TINY_MOE = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
 
 

@@ -141,11 +141,11 @@ def test_moe_plan_build_families_and_limits():
     fu = {f.name.decode(): f.followup for f in lay.families()}
     assert fu["mindptr"] == 1 and fu["mfin"] == 1 and fu["egu"] == 0
     ext = {f.name.decode(): f.max_extent for f in lay.families()}
-    # max tiles = ceil(512 * 8 / 64) + min(64, 4096) = 128; F/8 = 176 and H/8 = 256 tasks per tile
-    assert ext["egu"] == 128 * 176 and ext["edown"] == 128 * 256 and ext["route"] == 64
+    # max tiles = ceil(512 * 8 / 64) + min(64, 4096) = 128; F/16 = 88 and H/16 = 128 tasks per tile
+    assert ext["egu"] == 128 * 88 and ext["edown"] == 128 * 128 and ext["route"] == 64
     assert mk.mk_plan_workspace_bytes(lay.plan) > 512 * 8 * (1408 * 2 + 2048 * 4)
     lay.close()
-    for bad in (dict(n_experts=65), dict(top_k=9), dict(expert_ffn=1410), dict(hidden=2304)):
+    for bad in (dict(n_experts=65), dict(top_k=9), dict(expert_ffn=1400), dict(hidden=2304)):
         shp = wl.MoEShape(**{**dict(hidden=2048, n_experts=64, top_k=8, expert_ffn=1408), **bad})
         with pytest.raises(mk.MkError):
             mk.MoELayer(shp, None, max_tokens=64, n_sm=148, host_only=True)
