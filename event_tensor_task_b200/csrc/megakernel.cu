@@ -52,6 +52,7 @@ constexpr int kDoneQ = 32;    // controller -> notifier
 constexpr int kFollowQ = 16;  // notifier -> controller
 constexpr int kMaxB = 4;      // batch rows per step on this path
 constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
+constexpr int kActPitch = 2048 + 8;  // bf16 elements per staged activation row (16-byte bank offset per row)
 constexpr int kDynLookahead = 2;
 
 struct StepParams {
@@ -85,13 +86,11 @@ struct TaskDesc {
 
 // Ring geometry of a GEMV op's tasks, fixed for the plan: the producer copies
 // part 0's rows (and, for the rotate-half and gate/up pair ops, part 1's rows
-// from a fresh slot) into consecutive ring slots, rps rows per slot.  Compute
-// warp w owns rows [w * rpw, (w + 1) * rpw) of each part.
+// from a fresh slot) into consecutive ring slots, rps rows per slot.
 struct OpGeo {
-  int nblk;       // 256-column blocks per row (K / 256)
+  int rows_part;  // rows of a part (a multiple of 16)
   int row_bytes;  // 2 K
   int rps_lg;     // log2(rows per slot)
-  int rpw;        // rows per warp per part
   int spp;        // slots per part
   int pairs;      // 1: two parts (rotate-half or gate/up pairs)
 };
@@ -113,18 +112,27 @@ struct Smem {
   int fam_ext[kMaxFamilies];
   signed char fam_op[kMaxFamilies], fam_layer[kMaxFamilies];
   // activation staging: one batch row, loaded once per CTA for all warps
-  alignas(16) float xs[2048];  // read and written as float4
-  float red8[kComputeWarps];
+  // staging buffer: the GEMV activation rows (bf16, row b at b * kActPitch);
+  // other tasks use it as fp32 scratch (xs)
+  union {
+    alignas(16) float xs[2048];
+    alignas(16) __nv_bfloat16 xa[kMaxB * kActPitch];
+  };
+  alignas(16) float gred[2][kComputeWarps][16][4];  // GEMV partial tiles (double-buffered)
+  float red8[kMaxB][kComputeWarps];
   OpGeo geo[OP_COUNT];  // GEMV geometry per op, set in the prologue
   unsigned long long lm_seen[kComputeWarps][kMaxB];  // per compute warp: best argmax key it has published
   uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
-  // attention scratch, one row per head warp
-  float qs[4][64], ps[4][64], newk[4][64], newv[4][64];
+  // attention scratch: the group's queries, the chunk's scores, the new
+  // K and V rows (bf16, as in the cache) and the warps' exp-sums
+  float aq[4][64], asc[4][64];
+  uint4 anew[16];
+  float alsum[kComputeWarps][4];
   volatile int released;  // regular tasks the controller has handed to compute
   volatile int dq_head, dq_tail, fq_head, fq_tail, notifier_stop;
   int bad;
 };
-static_assert(sizeof(Smem) <= 19 * 1024, "fixed shared-memory area exceeds its reserve");
+static_assert(sizeof(Smem) <= kSmemReserve, "fixed shared-memory area exceeds its reserve");
 static_assert(offsetof(Smem, xs) % 16 == 0, "vector accesses to the staging buffer need 16-byte alignment");
 static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, fifo_full) % 8 == 0, "mbarriers need 8-byte alignment");
 constexpr int BAR_COMP = 3;  // named barrier of the 8 compute warps
@@ -928,15 +936,16 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Activation row b of a GEMV family into shared memory (sm.xs, fp32): the 8
-// compute warps load it once for the CTA (adding the previous layer's down
-// partials to x when asked), reduce its sum of squares and apply the RMSNorm
-// in place.  Called by all compute warps for the same task (the tag sequence
-// is the same for all warps).
-__device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int b) {
+// Activation rows 0..B-1 of a GEMV family into shared memory, bf16 (the
+// tensor-core operand type), row b at sm.xa + b * kActPitch: the compute
+// warps load them once for the CTA (adding the previous layer's down
+// partials to x when asked), reduce each row's sum of squares and apply the
+// RMSNorm.  Called by all compute warps for the same task (the tag sequence
+// is the same for all warps).  Thread t stages columns [8t, 8t + 8).
+__device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int B) {
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
-  const int K = g.K;  // at most 8 * kComputeThreads: each thread stages one 8-column chunk
+  const int K = g.K;  // at most 8 * kComputeThreads
   const int c = ct * 8;
   const bool has = c < K;
   const float* src;
@@ -945,228 +954,257 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
   else if (g.kind == 1) { src = reinterpret_cast<const float*>(ws + P.off_attn); rstride = (size_t)P.n_q_heads * P.head_dim; }
   else { src = reinterpret_cast<const float*>(ws + P.off_h) + (size_t)g.kc * P.kseg; rstride = P.ffn; }
   const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
-  // every load of the chunk (activation, split-K partials, norm gain) is
-  // issued before the first use, so staging costs one round trip to L2
-  float4 u = make_float4(0.f, 0.f, 0.f, 0.f), v = u;
-  float4 du[4], dv[4];
+  const int nq = g.parts ? P.n_kc : 0;
+  // every load of the chunk (all rows, split-K partials, norm gain) is issued
+  // before the first use, so staging costs about one round trip to L2
+  float4 u[kMaxB], v[kMaxB];
   uint4 graw = make_uint4(0u, 0u, 0u, 0u);
-  const int nq = g.parts ? min(P.n_kc, 4) : 0;
-  if (has) {
-    const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
-    u = __ldcg(p4);
-    v = __ldcg(p4 + 1);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (q < nq) {
-        const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
-        du[q] = __ldcg(d4);
-        dv[q] = __ldcg(d4 + 1);
-      }
-    if (g.kind == 0) {
-      const void* gp = g.gamma_sel == 2 ? P.final_norm
-                                        : (g.gamma_sel == 1 ? layers[g.layer].ffn_norm : layers[g.layer].attn_norm);
-      graw = __ldg(reinterpret_cast<const uint4*>(gp) + c / 8);
+  for (int b = 0; b < kMaxB; ++b) {
+    u[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+    v[b] = u[b];
+    if (has && b < B) {
+      const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
+      u[b] = __ldcg(p4);
+      v[b] = __ldcg(p4 + 1);
     }
   }
-  bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the previous activation
-  float ss = 0.f;
-  if (has) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (q < nq) {
-        u.x += du[q].x; u.y += du[q].y; u.z += du[q].z; u.w += du[q].w;
-        v.x += dv[q].x; v.y += dv[q].y; v.z += dv[q].z; v.w += dv[q].w;
-      }
-    if (g.parts)
-      for (int q = 4; q < P.n_kc; ++q) {
-        const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
-        float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
-        u.x += a4.x; u.y += a4.y; u.z += a4.z; u.w += a4.w;
-        v.x += b4.x; v.y += b4.y; v.z += b4.z; v.w += b4.w;
-      }
-    ss = u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w + v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  if (has && g.kind == 0) {
+    const void* gp = g.gamma_sel == 2 ? P.final_norm
+                                      : (g.gamma_sel == 1 ? layers[g.layer].ffn_norm : layers[g.layer].attn_norm);
+    graw = __ldg(reinterpret_cast<const uint4*>(gp) + c / 8);
   }
+  if (has)
+#pragma unroll 4
+    for (int q = 0; q < nq; ++q) {
+#pragma unroll
+      for (int b = 0; b < kMaxB; ++b)
+        if (b < B) {
+          const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
+          const float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
+          u[b].x += a4.x; u[b].y += a4.y; u[b].z += a4.z; u[b].w += a4.w;
+          v[b].x += b4.x; v[b].y += b4.y; v[b].z += b4.z; v[b].w += b4.w;
+        }
+    }
+  float inv[kMaxB];
+#pragma unroll
+  for (int b = 0; b < kMaxB; ++b) inv[b] = 1.f;
   if (g.kind == 0) {
-    ss = warp_sum(ss);
-    if (lane == 0) sm.red8[w] = ss;
-    bar_sync(BAR_COMP, kComputeThreads);
-    float tot = 0.f;
 #pragma unroll
-    for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[q];
-    const float inv = 1.0f / sqrtf(tot / (float)K + P.eps);
-    float gf[8];
-    bf16x8_to_f32(graw, gf);
-    u.x *= inv * gf[0]; u.y *= inv * gf[1]; u.z *= inv * gf[2]; u.w *= inv * gf[3];
-    v.x *= inv * gf[4]; v.y *= inv * gf[5]; v.z *= inv * gf[6]; v.w *= inv * gf[7];
+    for (int b = 0; b < kMaxB; ++b) {
+      float ss = u[b].x * u[b].x + u[b].y * u[b].y + u[b].z * u[b].z + u[b].w * u[b].w + v[b].x * v[b].x +
+                 v[b].y * v[b].y + v[b].z * v[b].z + v[b].w * v[b].w;
+      ss = warp_sum(ss);
+      if (lane == 0) sm.red8[b][w] = ss;
+    }
+    bar_sync(BAR_COMP, kComputeThreads);  // (also: every warp is done with the previous activation)
+#pragma unroll
+    for (int b = 0; b < kMaxB; ++b) {
+      float tot = 0.f;
+#pragma unroll
+      for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[b][q];
+      inv[b] = 1.0f / sqrtf(tot / (float)K + P.eps);
+    }
+  } else {
+    bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the previous activation
   }
   if (has) {
-    *reinterpret_cast<float4*>(&sm.xs[c]) = u;
-    *reinterpret_cast<float4*>(&sm.xs[c + 4]) = v;
+    float gf[8];
+    if (g.kind == 0) bf16x8_to_f32(graw, gf);
+#pragma unroll
+    for (int b = 0; b < kMaxB; ++b)
+      if (b < B) {
+        float f[8] = {u[b].x, u[b].y, u[b].z, u[b].w, v[b].x, v[b].y, v[b].z, v[b].w};
+        __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(g.kind == 0 ? f[j] * inv[b] * gf[j] : f[j]);
+        *reinterpret_cast<uint4*>(&sm.xa[b * kActPitch + c]) = *reinterpret_cast<const uint4*>(o);
+      }
   }
   bar_sync(BAR_COMP, kComputeThreads);  // the activation is complete
 }
 
-// A lane holds columns 256*i + 8*lane + j (i < K/256, j < 8) of the staged
-// activation row in registers, so the dot products read only weights from
-// shared memory.
-typedef float ActRegs[kMaxBlk][8];
-
-__device__ __forceinline__ void act_to_regs(const float* xs, int nblk, ActRegs& av) {
-  const int lane = threadIdx.x & 31;
-  const float4* a4 = reinterpret_cast<const float4*>(xs) + 2 * lane;
-#pragma unroll
-  for (int i = 0; i < kMaxBlk; ++i) {
-    if (i < nblk) {
-      const float4 u = a4[i * 64], v = a4[i * 64 + 1];
-      av[i][0] = u.x; av[i][1] = u.y; av[i][2] = u.z; av[i][3] = u.w;
-      av[i][4] = v.x; av[i][5] = v.y; av[i][6] = v.z; av[i][7] = v.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) av[i][j] = 0.f;
-    }
-  }
-}
-
-// Dot product of one weight row (bf16, in a ring slot) with the activation
-// registers, reduced over the warp.
-
-// Ring position of the task's slots.
 // Ring slot release.  A slot's empty barrier expects kComputeWarps arrivals
 // per use; only the warps that READ the slot arrive, each with its share of
-// that count (the first reader adds the remainder).  A warp that reads
-// nothing of a slot never touches its barrier, so no arrival can land in
-// another use's phase (with tasks of up to 8 slots in a 13-slot ring, task
-// k+1's slots can be physical slots that task k still reads).
+// that count (the first reader adds the remainder).  A warp arrives only
+// after it has waited for the slot's data, so no arrival can land in
+// another use's phase (with tasks of up to 8 slots in the ring, task k+1's
+// slots can be physical slots that task k still reads).
 __device__ __forceinline__ void release_share(Smem& sm, int slot, int readers, int rank) {
   const uint32_t share = kComputeWarps / readers + (rank == 0 ? kComputeWarps % readers : 0);
   mbar_arrive_count(&sm.empty[slot], share);
 }
 
-// Dot products of two rows held in shared memory (bf16, 16-byte chunks per
-// lane, 256 columns per block) with the activation in registers, interleaved
-// for instruction-level parallelism; summed across the warp (every lane gets
-// both sums).
-__device__ __forceinline__ void warp_dot2(const unsigned char* ra, const unsigned char* rb, int nblk,
-                                          const ActRegs& av, float& sa, float& sb) {
-  const int lane = threadIdx.x & 31;
-  const uint4* a4 = reinterpret_cast<const uint4*>(ra) + lane;
-  const uint4* b4 = reinterpret_cast<const uint4*>(rb) + lane;
-  float acc_a[2] = {0.f, 0.f}, acc_b[2] = {0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < kMaxBlk; ++i) {
-    if (i < nblk) {
-      float wa[8], wb[8];
-      bf16x8_to_f32(a4[i * 32], wa);
-      bf16x8_to_f32(b4[i * 32], wb);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        acc_a[j & 1] = fmaf(wa[j], av[i][j], acc_a[j & 1]);
-        acc_b[j & 1] = fmaf(wb[j], av[i][j], acc_b[j & 1]);
-      }
-    }
-  }
-  float va = acc_a[0] + acc_a[1], vb = acc_b[0] + acc_b[1];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    va += __shfl_xor_sync(0xffffffffu, va, o);
-    vb += __shfl_xor_sync(0xffffffffu, vb, o);
-  }
-  sa = va;
-  sb = vb;
+// ---- tensor-core tiles
+// Warp-level bf16 MMA m16n8k16 with fp32 accumulation.  K is walked in
+// windows of 32: lane (g = lane / 4, q = lane % 4) loads one 16-byte chunk,
+// columns [8q, 8q + 8) of the window, of each row it needs, and the two MMAs
+// of the window take its halves.  The logical-k -> column map is the same
+// for both operands, so each MMA pairs matching columns and the two MMAs
+// together cover the window's 32 columns once.
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_window(float (&c)[4], const uint4& ua, const uint4& ub, const uint4& wb) {
+  mma_16816(c, ua.x, ub.x, ua.y, ub.y, wb.x, wb.y);
+  mma_16816(c, ua.z, ub.z, ua.w, ub.w, wb.z, wb.w);
 }
 
-// One warp's share of a GEMV task for batch row b.  The warp owns a
-// contiguous block of rows (row ops) or of row pairs (rotate-half q/k pairs,
-// gate/up pairs), so it waits on one ring slot (two for pair ops) and
-// releases every other slot of the task at once.  Its row sums end up in all
-// lanes; lane i then runs the epilogue of its row (or pair) i.
-__device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
-                                               unsigned char* ws, Control* ctl, const TaskDesc& d,
-                                               const GemvSpec& g, const ActRegs& av, int b, uint32_t* trec,
-                                               bool release) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+// Epilogue item of thread ct in a GEMV task: batch row b and row (pair ops:
+// pair) r of the task; items are B x RI with RI the rows (pairs) of the task.
+struct GemvItem { int b, r; bool on; };
+__device__ __forceinline__ GemvItem gemv_item(const OpGeo& geo, int B) {
+  const int ct = threadIdx.x - kComputeBase;
+  const int RI = geo.rows_part;
+  GemvItem it;
+  it.b = ct / RI;
+  it.r = ct - it.b * RI;
+  it.on = it.b < B;
+  return it;
+}
+
+// Epilogue operands that do not depend on the task's products, loaded before
+// them so that their round trip to L2 overlaps the staging and the math: a
+// QKV item takes (cos, sin) of the rotary table for its column; an
+// O-projection item the residual terms of its column (x and up to four of
+// the previous layer's down-projection partials).
+struct EpiAhead { float a[5]; };
+__device__ __forceinline__ void gemv_epilogue_ahead(const DevPlan& P, const Smem& sm, unsigned char* ws,
+                                                    const TaskDesc& d, const GemvItem& it, EpiAhead& e) {
+#pragma unroll
+  for (int i = 0; i < 5; ++i) e.a[i] = 0.f;
+  if (!it.on) return;
+  if (d.op == OP_QKV) {
+    const QkvTile q = decode_qkv(P, d.idx);
+    if (q.kind != 2) {
+      const float2 cs = __ldg(reinterpret_cast<const float2*>(ws + P.off_rope) + (size_t)sm.ctx[it.b] * 32 +
+                              q.j0 + it.r);
+      e.a[0] = cs.x;
+      e.a[1] = cs.y;
+    }
+  } else if (d.op == OP_OPROJ) {
+    const size_t col = (size_t)d.idx * P.tile_o + it.r;
+    const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)it.b * P.hidden + col;
+    e.a[0] = __ldcg(reinterpret_cast<const float*>(ws + P.off_x) + (size_t)it.b * P.hidden + col);
+    if (d.layer > 0 && P.kind == MK_MODEL_DENSE)
+#pragma unroll
+      for (int kc = 0; kc < 4; ++kc)
+        if (kc < P.n_kc) e.a[1 + kc] = __ldcg(dp + (size_t)kc * P.max_batch * P.hidden);
+  }
+}
+
+// A GEMV task on tensor cores: Y[rows x B] = W[rows x K] . A[B x K]^T, W
+// the task's rows in its ring slots (bf16), A the staged activation rows.
+// The task's rows form nrb = rows / 16 row blocks (pair ops: part 0's blocks,
+// then part 1's); warp w takes row block w / kp over K part w % kp (kp = 8 /
+// nrb) with the activation rows as the MMA's n = 8 columns (column n reads
+// row min(n, B - 1)).  Each warp leaves its 16 x 4 partial tile in
+// sm.gred[buf]; after a barrier, thread ct sums the kp partials of its item
+// (batch row b, row or pair r) and runs the op's epilogue.  Every warp waits
+// for every slot of the task and then releases each with a share of 1.
+__device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
+                                          unsigned char* ws, Control* ctl, const TaskDesc& d, const GemvSpec& g,
+                                          int B, int buf, const EpiAhead& ea, const GemvItem& it, uint32_t* trec) {
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const OpGeo geo = sm.geo[d.op];
   const int R = P.ring_slots;
   const int s0 = d.slot_ph & 0xffff;
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int r0 = w * geo.rpw;                                   // first row of this warp in part 0
-  const int n = max(0, min(geo.rpw, g.rows - r0));              // rows (pairs) of this warp
-  if (n == 0) return;  // (reads no slot: see release_share)
-  const int ja = r0 >> geo.rps_lg;                              // task slot of part 0's rows
-  const int jb = geo.pairs ? geo.spp + ja : -1;                 // task slot of part 1's rows
-  // readers of the slot: the warps whose rows lie in it (rpw divides the rows per slot)
-  const int wps = (1 << geo.rps_lg) / geo.rpw;                  // warps per full slot
-  const int first_w = ja * wps;
-  const int readers = min(wps, (g.rows - first_w * geo.rpw + geo.rpw - 1) / geo.rpw);
-  const int sa = s0 + ja < R ? s0 + ja : s0 + ja - R;
-  const uint32_t pa = s0 + ja < R ? p0 : p0 ^ 1u;
-  wait_mbar(&sm.full[sa], pa, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  int sb = sa;
-  if (geo.pairs) {
-    sb = s0 + jb < R ? s0 + jb : s0 + jb - R;
-    wait_mbar(&sm.full[sb], s0 + jb < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  const int nparts = geo.pairs ? 2 : 1;
+  const int nslots = d.nslots;
+  for (int j = 0; j < nslots; ++j) {
+    const int sj = s0 + j < R ? s0 + j : s0 + j - R;
+    wait_mbar(&sm.full[sj], s0 + j < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
   }
   if (trec && lane == 0) {
     trec[TR_DATA] = (uint32_t)global_ns();
-    trec[TR_ISSUE] = sm.slot_t[sa];
+    trec[TR_ISSUE] = sm.slot_t[s0];
   }
-  const int roff = (r0 & ((1 << geo.rps_lg) - 1)) * geo.row_bytes;
-  const unsigned char* base_a = ring + (size_t)sa * P.slot_bytes + roff;
-  const unsigned char* base_b = ring + (size_t)sb * P.slot_bytes + roff;
-  // y[2t], y[2t+1]: pair ops: part-0 and part-1 row of pair t; row ops: rows 2t, 2t+1
-  float y[8];
+  // this warp's row block and K part
+  const int rows_total = nparts * geo.rows_part;
+  const int nrb = rows_total >> 4;
+  const int kp = kComputeWarps / nrb;
+  const int rb = w / kp, kpi = w - rb * kp;
+  const int rbp = geo.rows_part >> 4;         // row blocks per part
+  const int part = rb / rbp;
+  const int valid = geo.pairs ? geo.rows_part : g.rows;  // valid rows of the part
+  const int g8 = lane >> 2, q = lane & 3;
+  int ra = (rb - part * rbp) * 16 + g8, rbb = ra + 8;
+  ra = min(ra, valid - 1);
+  rbb = min(rbb, valid - 1);
+  auto row_ptr = [&](int r) -> const unsigned char* {
+    const int j = part * geo.spp + (r >> geo.rps_lg);
+    const int sj = s0 + j < R ? s0 + j : s0 + j - R;
+    return ring + (size_t)sj * P.slot_bytes + (size_t)(r & ((1 << geo.rps_lg) - 1)) * geo.row_bytes;
+  };
+  const int kw = g.K / kp;  // columns of this warp
+  const int kbase = kpi * kw;
+  const uint4* pa = reinterpret_cast<const uint4*>(row_ptr(ra) + (size_t)kbase * 2) + q;
+  const uint4* pb = reinterpret_cast<const uint4*>(row_ptr(rbb) + (size_t)kbase * 2) + q;
+  const uint4* px = reinterpret_cast<const uint4*>(&sm.xa[min(g8, B - 1) * kActPitch + kbase]) + q;
+  const int nwin = kw >> 5;
+  float c[4][4];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    y[2 * t] = y[2 * t + 1] = 0.f;
-    if (geo.pairs) {
-      if (t < n) warp_dot2(base_a + t * geo.row_bytes, base_b + t * geo.row_bytes, geo.nblk, av, y[2 * t], y[2 * t + 1]);
-    } else if (2 * t < n) {
-      const int t1 = 2 * t + 1 < n ? 2 * t + 1 : 2 * t;  // an odd last row is paired with itself
-      warp_dot2(base_a + 2 * t * geo.row_bytes, base_a + t1 * geo.row_bytes, geo.nblk, av, y[2 * t], y[2 * t + 1]);
-    }
+  for (int u = 0; u < 4; ++u) c[u][0] = c[u][1] = c[u][2] = c[u][3] = 0.f;
+  for (int w4 = 0; w4 < nwin; w4 += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (w4 + u < nwin) {
+        const int o = (w4 + u) * 4;  // 16-byte chunks per 32-column window
+        mma_window(c[u], pa[o], pb[o], px[o]);
+      }
   }
-  if (release) {
-    __syncwarp();
-    if (lane == 0) {
-      release_share(sm, sa, readers, w - first_w);
-      if (geo.pairs) release_share(sm, sb, readers, w - first_w);  // part 1 has the same readers
+  __syncwarp();
+  if (lane == 0)
+    for (int j = 0; j < nslots; ++j) {
+      const int sj = s0 + j < R ? s0 + j : s0 + j - R;
+      release_share(sm, sj, kComputeWarps, w);
     }
+  // partial tile: lane (g8, q < 2) holds rows g8, g8 + 8 at batch columns 2q, 2q + 1
+  float (*red)[16][4] = sm.gred[buf];
+  if (q < 2) {
+    const float d0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]), d1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
+    const float d2 = (c[0][2] + c[1][2]) + (c[2][2] + c[3][2]), d3 = (c[0][3] + c[1][3]) + (c[2][3] + c[3][3]);
+    *reinterpret_cast<float2*>(&red[w][g8][2 * q]) = make_float2(d0, d1);
+    *reinterpret_cast<float2*>(&red[w][g8 + 8][2 * q]) = make_float2(d2, d3);
   }
-  // lane i takes row i (row ops) or pair i (pair ops)
+  bar_sync(BAR_COMP, kComputeThreads);
+  // epilogue: item (b, r); v0 = row r (pair ops: part 0 row r), v1 = part 1 row r
+  const int b = it.b, r = it.r;
+  const bool mine = it.on && r < (geo.pairs ? geo.rows_part : g.rows);
   float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    if (geo.pairs) {
-      if (t < 4 && lane == t) { v0 = y[2 * t]; v1 = y[2 * t + 1]; }
-    } else if (lane == t) {
-      v0 = y[t];
-    }
+  if (mine) {
+    const int rb0 = r >> 4, rr = r & 15;
+    for (int k = 0; k < kp; ++k) v0 += red[rb0 * kp + k][rr][b];
+    if (geo.pairs)
+      for (int k = 0; k < kp; ++k) v1 += red[(rbp + rb0) * kp + k][rr][b];
   }
   const int H = P.hidden;
-  const bool mine = lane < n;
   switch (d.op) {
     case OP_QKV: {
       // RoPE on q and k (rotate-half pairs j, j + D/2), then q -> buffer, k/v -> cache
       if (!mine) break;
-      QkvTile q = decode_qkv(P, d.idx);
+      QkvTile qt = decode_qkv(P, d.idx);
       const int pos = sm.ctx[b];
-      const int j = q.j0 + r0 + lane;
-      if (q.kind == 2) {
-        size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
+      const int j = qt.j0 + r;
+      if (qt.kind == 2) {
+        size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + qt.head) * P.max_ctx + pos;
         __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * P.head_dim;
         vc[j] = __float2bfloat16_rn(v0);
         vc[j + 32] = __float2bfloat16_rn(v1);
       } else {
-        const float* rope = reinterpret_cast<const float*>(ws + P.off_rope) + ((size_t)pos * 32 + j) * 2;
-        const float c = __ldg(rope), sn = __ldg(rope + 1);
-        const float x0 = v0 * c - v1 * sn, x1 = v1 * c + v0 * sn;
-        if (q.kind == 0) {
+        const float cs = ea.a[0], sn = ea.a[1];  // (cos, sin) of (pos, j), loaded before the products
+        const float x0 = v0 * cs - v1 * sn, x1 = v1 * cs + v0 * sn;
+        if (qt.kind == 0) {
           float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * P.head_dim +
-                      q.head * P.head_dim;
+                      qt.head * P.head_dim;
           qb[j] = x0;
           qb[j + 32] = x1;
         } else {
-          size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + q.head) * P.max_ctx + pos;
+          size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + qt.head) * P.max_ctx + pos;
           __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * P.head_dim;
           kc[j] = __float2bfloat16_rn(x0);
           kc[j + 32] = __float2bfloat16_rn(x1);
@@ -1176,41 +1214,44 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
     case OP_OPROJ: {
       // residual: x = (x + previous layer's down partials) + o W_o^T
       if (!mine) break;
-      const size_t col = (size_t)d.idx * P.tile_o + r0 + lane;
+      const size_t col = (size_t)d.idx * P.tile_o + r;
       float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
-      const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H + col;
-      float acc = __ldcg(x + col);
-      if (d.layer > 0 && P.kind == MK_MODEL_DENSE)
-        for (int kc = 0; kc < P.n_kc; ++kc) acc += __ldcg(dp + (size_t)kc * P.max_batch * H);
+      float acc = ea.a[0];
+      if (d.layer > 0 && P.kind == MK_MODEL_DENSE) {
+        acc += (ea.a[1] + ea.a[2]) + (ea.a[3] + ea.a[4]);
+        const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H + col;
+        for (int kc = 4; kc < P.n_kc; ++kc) acc += __ldcg(dp + (size_t)kc * P.max_batch * H);
+      }
       x[col] = acc + v0;
     } break;
     case OP_GATEUP: {
       if (!mine) break;
-      float* h = reinterpret_cast<float*>(ws + P.off_h) + (size_t)b * P.ffn + (size_t)d.idx * P.tile_gu + r0;
-      h[lane] = v0 / (1.0f + expf(-v0)) * v1;
+      float* h = reinterpret_cast<float*>(ws + P.off_h) + (size_t)b * P.ffn + (size_t)d.idx * P.tile_gu + r;
+      *h = v0 / (1.0f + expf(-v0)) * v1;
     } break;
     case OP_DOWN: {
       if (!mine) break;
       const int nt = d.idx - g.kc * P.n_dtiles;
-      float* part = reinterpret_cast<float*>(ws + P.off_dpart) + ((size_t)g.kc * P.max_batch + b) * H +
-                    (size_t)nt * P.tile_down + r0;
-      part[lane] = v0;
+      float* dpart = reinterpret_cast<float*>(ws + P.off_dpart) + ((size_t)g.kc * P.max_batch + b) * H +
+                     (size_t)nt * P.tile_down + r;
+      *dpart = v0;
     } break;
     case OP_LM: {
-      // logits, then the warp's best (logit, id) key; published with an atomic
-      // max only when it beats what this warp published before (order independent)
-      const int r = d.idx * P.tile_lm + r0 + lane;
+      // logits, then the warp's best (logit, id) key (the warp's items share
+      // one batch row); published with an atomic max only when it beats what
+      // this warp published before (order independent)
+      const int row = d.idx * P.tile_lm + r;
       unsigned long long key = 0ull;
       if (mine) {
-        if (S.logits) S.logits[(size_t)b * P.vocab + r] = v0;
-        key = argmax_key(v0, r);
+        if (S.logits) S.logits[(size_t)b * P.vocab + row] = v0;
+        key = argmax_key(v0, row);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
         key = other > key ? other : key;
       }
-      if (lane == 0 && key > sm.lm_seen[w][b]) {
+      if (lane == 0 && it.on && key > sm.lm_seen[w][b]) {
         sm.lm_seen[w][b] = key;
         atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, key);
       }
@@ -1219,96 +1260,140 @@ __device__ __forceinline__ void warp_gemv_task(const DevPlan& P, const StepParam
   }
 }
 
+// One chunk of split-K decode attention for the qpg query heads of a GQA
+// group (flash-decoding partial: unnormalised output, running max, sum).
+// All 8 compute warps share the chunk: warp w scores keys [8w, 8w + 8) for
+// every head of the group (each K row is read from shared memory once; a
+// lane holds one 16-byte slice of a row and the matching 8 query values of
+// each head in registers), then accumulates those keys' V rows for every
+// head; the 8 warps' partial outputs are summed through the staging buffer.
+// The new key (position ctx) is read from the cache in global memory: the
+// ring copy of its chunk may predate this step's append.
 __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                        unsigned char* ws, Control* ctl, const TaskDesc& d) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, D = P.head_dim, CH = P.chunk;
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
+  const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, CH = P.chunk;
+  constexpr int D = 64;  // head_dim (the plan builder accepts 64 only)
   const int slot = d.slot_ph & 0xffff;
   const uint32_t par = (uint32_t)d.slot_ph >> 16;
-  if (w < qpg) {
-    // warp w: query head g*qpg + w over this chunk's keys
-    AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
-    const int p = sm.ctx[a.b];
-    const int n_old = max(0, min(CH, p - a.c * CH));
-    const bool has_new = (p - a.c * CH) < CH;
-    const int n_keys = n_old + (has_new ? 1 : 0);
-    float* qs = sm.qs[w];
-    float* ps = sm.ps[w];
-    const float* q = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D +
-                     (size_t)(a.g * qpg + w) * D;
-    qs[lane] = __ldcg(q + lane) * 0.125f;  // 1/sqrt(64)
-    qs[lane + 32] = __ldcg(q + lane + 32) * 0.125f;
-    if (has_new) {
-      size_t row = (((size_t)d.layer * P.n_slots + sm.slot[a.b]) * Hkv + a.g) * P.max_ctx + p;
-      const unsigned short* kn = reinterpret_cast<const unsigned short*>(P.k_cache) + row * D;
-      const unsigned short* vn = reinterpret_cast<const unsigned short*>(P.v_cache) + row * D;
-      sm.newk[w][lane] = bf16_bits_to_f32(__ldcg(kn + lane));
-      sm.newk[w][lane + 32] = bf16_bits_to_f32(__ldcg(kn + lane + 32));
-      sm.newv[w][lane] = bf16_bits_to_f32(__ldcg(vn + lane));
-      sm.newv[w][lane + 32] = bf16_bits_to_f32(__ldcg(vn + lane + 32));
-    }
-    __syncwarp();
-    wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
-    const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
-    const unsigned char* vbase = kbase + (size_t)CH * D * 2;
-    // scores of keys lane and lane + 32
-    float sc[2];
+  const AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
+  const int p = sm.ctx[a.b];
+  const int n_old = max(0, min(CH, p - a.c * CH));
+  const bool has_new = (p - a.c * CH) < CH;
+  const int n_keys = n_old + (has_new ? 1 : 0);
+  // queries of the group (scaled by 1/sqrt(64)) and the new K/V rows
+  const float* q = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D +
+                   (size_t)a.g * qpg * D;
+  if (ct < qpg * D) sm.aq[ct >> 6][ct & 63] = __ldcg(q + ct) * 0.125f;
+  if (has_new && ct < 16) {
+    const size_t row = (((size_t)d.layer * P.n_slots + sm.slot[a.b]) * Hkv + a.g) * P.max_ctx + p;
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(ct < 8 ? P.k_cache : P.v_cache) + row * D * 2;
+    sm.anew[ct] = __ldcg(reinterpret_cast<const uint4*>(src) + (ct & 7));
+  }
+  bar_sync(BAR_COMP, kComputeThreads);
+  wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
+  const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
+  const unsigned char* vbase = kbase + (size_t)CH * D * 2;
+  const unsigned char* knew = reinterpret_cast<const unsigned char*>(&sm.anew[0]);
+  const unsigned char* vnew = reinterpret_cast<const unsigned char*>(&sm.anew[8]);
+  // scores: lane = (key kq of 4, 16-byte column slice ci of 8)
+  {
+    const int kq = lane >> 3, ci = lane & 7;
+    float qr[4][8];
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      const int kk = lane + 32 * h2;
-      float s = -INFINITY;
-      if (kk < n_old) {
-        s = 0.f;
-        const uint4* kr = reinterpret_cast<const uint4*>(kbase + (size_t)kk * D * 2);
+    for (int h = 0; h < 4; ++h)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int ci = (i + kk) & 7;  // rotate the start so the lanes' rows hit distinct banks
-          float kf[8];
-          bf16x8_to_f32(kr[ci], kf);
+      for (int j = 0; j < 8; ++j) qr[h][j] = h < qpg ? sm.aq[h][ci * 8 + j] : 0.f;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) s = fmaf(kf[j], qs[ci * 8 + j], s);
-        }
-      } else if (kk < n_keys) {
-        s = 0.f;
-        for (int j = 0; j < D; ++j) s = fmaf(sm.newk[w][j], qs[j], s);
+    for (int pass = 0; pass < 2; ++pass) {
+      const int kk = 8 * w + 4 * pass + kq;
+      const unsigned char* row = (has_new && kk == n_old) ? knew : kbase + (size_t)kk * D * 2;
+      float kf[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + ci * 16), kf);
+      float s[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc = fmaf(kf[j], qr[h][j], acc);
+        s[h] = acc;
       }
-      sc[h2] = s;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+        for (int h = 0; h < 4; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], o);
+      const float mine = ci == 0 ? s[0] : ci == 1 ? s[1] : ci == 2 ? s[2] : s[3];
+      if (ci < qpg) sm.asc[ci][kk] = kk < n_keys ? mine : -INFINITY;
     }
-    float m = fmaxf(sc[0], sc[1]);
+  }
+  bar_sync(BAR_COMP, kComputeThreads);
+  // softmax statistics of the chunk, per head (every warp computes them)
+  float M[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    float m = -INFINITY;
+    if (h < qpg) m = fmaxf(sm.asc[h][lane], sm.asc[h][lane + 32]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float e0 = lane < n_keys ? expf(sc[0] - m) : 0.f;
-    const float e1 = lane + 32 < n_keys ? expf(sc[1] - m) : 0.f;
-    const float l = warp_sum(e0 + e1);
-    ps[lane] = e0;
-    ps[lane + 32] = e1;
-    __syncwarp();
-    float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int kk = 0; kk < n_old; ++kk) {
-      const unsigned short* vr = reinterpret_cast<const unsigned short*>(vbase + (size_t)kk * D * 2);
-      const float pk = ps[kk];
-      o0[kk & 3] = fmaf(pk, bf16_bits_to_f32(vr[lane]), o0[kk & 3]);
-      o1[kk & 3] = fmaf(pk, bf16_bits_to_f32(vr[lane + 32]), o1[kk & 3]);
+    M[h] = m;
+  }
+  // lane = (head hp, key j of this warp's 8): its probability
+  const int hp = lane >> 3, j = lane & 7;
+  const float Mh = hp == 0 ? M[0] : hp == 1 ? M[1] : hp == 2 ? M[2] : M[3];
+  float pl = (hp < qpg && 8 * w + j < n_keys) ? expf(sm.asc[hp][8 * w + j] - Mh) : 0.f;
+  float ls = pl;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  if (j == 0 && hp < qpg) sm.alsum[w][hp] = ls;
+  // P.V over this warp's keys: lane = output columns 2*lane, 2*lane + 1
+  float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int kk = 8 * w + jj;
+    if (kk < n_keys) {
+      const unsigned char* row = (has_new && kk == n_old) ? vnew : vbase + (size_t)kk * D * 2;
+      const uint32_t v2 = *reinterpret_cast<const uint32_t*>(row + lane * 4);
+      const float va = __uint_as_float(v2 << 16), vb = __uint_as_float(v2 & 0xffff0000u);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float ph = __shfl_sync(0xffffffffu, pl, h * 8 + jj);
+        o0[h] = fmaf(ph, va, o0[h]);
+        o1[h] = fmaf(ph, vb, o1[h]);
+      }
     }
-    float r0 = (o0[0] + o0[1]) + (o0[2] + o0[3]), r1 = (o1[0] + o1[1]) + (o1[2] + o1[3]);
-    if (has_new) {
-      r0 = fmaf(ps[n_old], sm.newv[w][lane], r0);
-      r1 = fmaf(ps[n_old], sm.newv[w][lane + 32], r1);
-    }
-    float* part = reinterpret_cast<float*>(ws + P.off_apart) +
-                  (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2)) + w * (D + 2);
-    part[lane] = r0;
-    part[lane + 32] = r1;
-    if (lane == 0) { part[D] = m; part[D + 1] = l; }
   }
   __syncwarp();
-  if (w < qpg && lane == 0) release_share(sm, slot, qpg, w);  // the head warps read the slot
+  if (lane == 0) release_share(sm, slot, kComputeWarps, w);  // every warp has read its K and V rows
+  // the 8 warps' partial outputs, [w][h][64] in the staging buffer
+  float* ob = sm.xs;
+#pragma unroll
+  for (int h = 0; h < 4; ++h)
+    if (h < qpg) *reinterpret_cast<float2*>(ob + (w * 4 + h) * D + 2 * lane) = make_float2(o0[h], o1[h]);
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (ct < qpg * D) {
+    const int h = ct >> 6, dd = ct & 63;  // h is uniform in a warp
+    float O = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < kComputeWarps; ++ww) O += ob[(ww * 4 + h) * D + dd];
+    float* part = reinterpret_cast<float*>(ws + P.off_apart) +
+                  (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2)) + h * (D + 2);
+    part[dd] = O;
+    if (dd == 0) {
+      float L = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < kComputeWarps; ++ww) L += sm.alsum[ww][h];
+      part[D] = h == 0 ? M[0] : h == 1 ? M[1] : h == 2 ? M[2] : M[3];
+      part[D + 1] = L;
+    }
+  }
 }
 
-// Merge of a head group's chunk partials, softmax-weighted in chunk order:
-// the chunk maxima and weights are computed lane-parallel (lane c holds chunk
-// c, c + 32, ...), then each lane sums its output dimension over the chunks.
+// Merge of the chunk partials of one (sequence, GQA group): the output of
+// head h is sum_c e^(m_c - M) o_c / sum_c e^(m_c - M) l_c.  Warp pair
+// (2h, 2h + 1) takes head h, 32 output columns each; a batch of up to 16
+// chunks is loaded in one round trip (lane c: m and l of chunk c; every lane:
+// its column of all the batch's chunk outputs), with an online rescale across
+// batches.
 __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws,
                                         const TaskDesc& d) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
@@ -1320,20 +1405,28 @@ __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S
   const size_t cs = (size_t)qpg * (D + 2);
   const float* part = reinterpret_cast<const float*>(ws + P.off_apart) + ((size_t)b * Hkv + g) * P.max_chunks * cs +
                       h * (D + 2);
-  float M = -INFINITY;
-  for (int c = lane; c < nch; c += 32) M = fmaxf(M, __ldcg(part + c * cs + D));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float L = 0.f, O = 0.f;
-  for (int c0 = 0; c0 < nch; c0 += 32) {
+  float M = -INFINITY, L = 0.f, O = 0.f;
+  for (int c0 = 0; c0 < nch; c0 += 16) {
+    const int n = min(16, nch - c0);
     const int c = c0 + lane;
-    const float e = c < nch ? expf(__ldcg(part + c * cs + D) - M) : 0.f;
-    L += warp_sum(c < nch ? __ldcg(part + c * cs + D + 1) * e : 0.f);
-    const int n = min(32, nch - c0);
+    const bool in = lane < n;  // lane c - c0 of the batch
+    const float mc = in ? __ldcg(part + c * cs + D) : -INFINITY;
+    const float lc = in ? __ldcg(part + c * cs + D + 1) : 0.f;
+    float ov[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) ov[q] = q < n ? __ldcg(part + (c0 + q) * cs + dd) : 0.f;
+    float mb = mc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const float Mn = fmaxf(M, mb);
+    const float sc = expf(M - Mn);  // 0 on the first batch (M = -inf, Mn finite)
+    const float e = in ? expf(mc - Mn) : 0.f;
+    L = L * sc + warp_sum(lc * e);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int q = 0; q < n; ++q) acc[q & 3] = fmaf(__ldcg(part + (c0 + q) * cs + dd), __shfl_sync(0xffffffffu, e, q), acc[q & 3]);
-    O += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) acc[q & 3] = fmaf(ov[q], __shfl_sync(0xffffffffu, e, q), acc[q & 3]);
+    O = O * sc + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    M = Mn;
   }
   float* out = reinterpret_cast<float*>(ws + P.off_attn) + (size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D;
   out[dd] = O / L;
@@ -1537,23 +1630,7 @@ __device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, const unsigned cha
   return m;
 }
 
-// ---- tensor-core tiles (tiles of >= 16 routed rows)
-// Warp-level bf16 MMA m16n8k16 with fp32 accumulation.  K is walked in
-// windows of 32: lane (g = lane / 4, q = lane % 4) loads one 16-byte chunk,
-// columns [8q, 8q + 8) of the window, of each row it needs, and the two MMAs
-// of the window take its halves.  The logical-k -> column map is the same
-// for both operands, so each MMA pairs matching columns and the two MMAs
-// together cover the window's 32 columns once.
-__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_window(float (&c)[4], const uint4& ua, const uint4& ub, const uint4& wb) {
-  mma_16816(c, ua.x, ub.x, ua.y, ub.y, wb.x, wb.y);
-  mma_16816(c, ua.z, ub.z, ua.w, ub.w, wb.z, wb.w);
-}
+// ---- MoE tensor-core tiles (tiles of >= 16 routed rows): mma_window above
 
 // Readers of the ring slots of an n x (rows of 8) block layout: the slots of
 // one part hold rows [j*rps, (j+1)*rps) of its 16 rows; the warps (m block
@@ -1792,6 +1869,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int B = S.B;
   int a_tag = -1;
+  int gbuf = 0;  // GEMV partial-tile buffer of the next GEMV task
   for (uint32_t k = 0;; ++k) {
     // task k: released into cur[k & 1] as phase k >> 1 of go_bar[k & 1]
     if (!wait_mbar(&sm.go_bar[k & 1], (k >> 1) & 1, ctl, P.spin_timeout_ns, -1, -1)) break;
@@ -1818,21 +1896,19 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     if (kKind == MK_MODEL_MOE_LAYER || moe_task) {
       a_tag = -1;  // MoE tasks use the staging buffer as scratch
     } else if (gemv_spec(P, d, g)) {
-      // one pass per batch row (the activation is restaged each pass when
-      // B > 1); the ring slots are released after the last pass
-      for (int b = 0; b < B; ++b) {
-        if (B > 1 || g.tag != a_tag) {
-          stage_act(P, ws, sm, g, b);
-          a_tag = B > 1 ? -1 : g.tag;
-        }
-        // the activation's registers live within one task (reloaded from the
-        // staged copy), so no other task body has to keep them
-        ActRegs av;
-        act_to_regs(sm.xs, g.K >> 8, av);
-        warp_gemv_task(P, S, sm, ring, ws, ctl, d, g, av, b, trec, b == B - 1);
+      // all B activation rows are staged together; an unchanged tag reuses them
+      const GemvItem it = gemv_item(sm.geo[d.op], B);
+      EpiAhead ea;
+      gemv_epilogue_ahead(P, sm, ws, d, it, ea);
+      if (g.tag != a_tag) {
+        stage_act(P, ws, sm, g, B);
+        a_tag = g.tag;
       }
+      gemv_task(P, S, sm, ring, ws, ctl, d, g, B, gbuf, ea, it, trec);
+      gbuf ^= 1;
     } else if (d.op == OP_ATTN) {
       task_attn(P, S, sm, ring, ws, ctl, d);
+      a_tag = -1;  // the staging buffer held the warps' partial outputs
     } else if (d.op == OP_MERGE) {
       task_merge(P, S, sm, ws, d);
     } else if (d.op == OP_LMFIN) {
@@ -1921,10 +1997,9 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     auto set_geo = [&](int op, int K, int rows_part, int pairs) {
       OpGeo& gg = sm.geo[op];
       const int rps = P.slot_bytes / (2 * K);
-      gg.nblk = K >> 8;
+      gg.rows_part = rows_part;
       gg.row_bytes = 2 * K;
       gg.rps_lg = __ffs(rps) - 1;
-      gg.rpw = rows_part / kComputeWarps;
       gg.spp = ceil_div(rows_part, rps);
       gg.pairs = pairs;
     };

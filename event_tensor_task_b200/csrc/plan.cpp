@@ -274,7 +274,7 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   P.max_tiles = ceil_div(TM * K, P.moe_tm) + std::min(E, TM * K);
   if (FF % P.moe_tn) { err = "expert_ffn must be a multiple of 16"; return MK_ERR_UNSUPPORTED; }
   P.slot_bytes = 16384;
-  const int reserve = 19 * 1024;
+  const int reserve = kSmemReserve;
   P.smem_bytes = smem_bytes;
   P.ring_slots = std::min(16, (smem_bytes - reserve) / P.slot_bytes);
   if (P.ring_slots < 5) { err = "not enough shared memory for a 5-slot ring"; return MK_ERR_UNSUPPORTED; }
@@ -426,13 +426,19 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (P.tile_qkv / rows_per_slot_h > 8 || P.tile_o / rows_per_slot_h > 8 || 2 * P.tile_gu / rows_per_slot_h > 8 ||
       P.tile_down / rows_per_slot_k > 8 || ceil_div(P.tile_lm, rows_per_slot_h) > 8)
     { err = "a tile spans more than 8 ring slots"; return MK_ERR_UNSUPPORTED; }
-  // each compute warp owns a contiguous block of rows (row pairs) of a task,
-  // inside one ring slot: at most 8 rows or 4 pairs, and no more than a slot holds
-  if (P.tile_qkv / 2 > 32 || P.tile_o > 64 || P.tile_gu > 32 || P.tile_down > 64 || P.tile_lm > 64)
-    { err = "a tile gives a warp more than 8 rows"; return MK_ERR_UNSUPPORTED; }
-  if (P.tile_qkv / 16 > rows_per_slot_h || P.tile_o / 8 > rows_per_slot_h || P.tile_gu / 8 > rows_per_slot_h ||
-      P.tile_down / 8 > rows_per_slot_k || P.tile_lm / 8 > rows_per_slot_h)
-    { err = "a tile gives a warp more rows than one ring slot holds"; return MK_ERR_UNSUPPORTED; }
+  // tensor-core GEMV tiles: whole 16-row blocks per part, 1, 2, 4 or 8 blocks
+  // per task (the 8 compute warps split them evenly), at most 256 epilogue
+  // items (rows or pairs x batch rows) and LM items of one batch row per warp
+  auto blocks_ok = [](int rows_part, int parts) {
+    if (rows_part % 16) return false;
+    const int nrb = parts * rows_part / 16;
+    return nrb == 1 || nrb == 2 || nrb == 4 || nrb == 8;
+  };
+  if (!blocks_ok(P.tile_qkv / 2, 2) || !blocks_ok(P.tile_o, 1) || !blocks_ok(P.tile_gu, 2) ||
+      !blocks_ok(P.tile_down, 1) || !blocks_ok(P.tile_lm, 1) || P.tile_lm % 32)
+    { err = "GEMV tiles must be whole 16-row blocks (1, 2, 4 or 8 per task; tile_lm a multiple of 32)"; return MK_ERR_UNSUPPORTED; }
+  if (P.tile_qkv / 2 > 64 || P.tile_o > 64 || P.tile_gu > 64 || P.tile_down > 64 || P.tile_lm > 64)
+    { err = "a GEMV tile has more than 64 rows (pairs) per part"; return MK_ERR_UNSUPPORTED; }
   P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
   P.n_otiles = H / P.tile_o;
   P.n_gutiles = F / P.tile_gu;
@@ -442,7 +448,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.max_chunks = ceil_div(P.max_ctx, P.chunk);
 
   // shared memory: ring of 16 KB slots plus a fixed control area
-  const int reserve = 19 * 1024;  // fixed shared-memory area of the kernel
+  const int reserve = kSmemReserve;  // fixed shared-memory area of the kernel
   P.smem_bytes = smem_bytes;
   P.ring_slots = std::min(16, (smem_bytes - reserve) / P.slot_bytes);
   if (P.ring_slots < 3) { err = "not enough shared memory for a 3-slot ring"; return MK_ERR_UNSUPPORTED; }

@@ -184,6 +184,7 @@ struct LayerPtrs {
 };
 
 constexpr int kMaxFamilies = 256;
+constexpr int kSmemReserve = 29 * 1024;  // the kernel's fixed shared-memory area; the ring takes the rest
 constexpr int kMaxBatch = 128;
 
 // Fixed header of the plan; passed to the kernel by value.  Offsets are in
