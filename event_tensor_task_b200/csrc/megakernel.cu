@@ -31,9 +31,11 @@
 // Every spin is bounded by the plan's timeout; on expiry the kernel records an
 // error in the control block, raises an abort flag that every spin polls,
 // drains its in-flight copies and exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/mk.h"
@@ -84,14 +86,13 @@ struct TaskDesc {
   uint32_t t_issue;  // trace: when the producer queued the task (low 32 bits of ns)
 };
 
-// Ring geometry of a GEMV op's tasks, fixed for the plan: the producer copies
-// part 0's rows (and, for the rotate-half and gate/up pair ops, part 1's rows
-// from a fresh slot) into consecutive ring slots, rps rows per slot.
+// Ring geometry of a GEMV op's tasks, fixed for the plan: the task's rows
+// (part 0's, then for the rotate-half and gate/up pair ops part 1's) arrive
+// in kGemvSlots consecutive ring slots by column: slot j holds columns
+// [j cw, (j + 1) cw) of every row, row after row (cw * 2 bytes each).
 struct OpGeo {
-  int rows_part;  // rows of a part (a multiple of 16)
-  int row_bytes;  // 2 K
-  int rps_lg;     // log2(rows per slot)
-  int spp;        // slots per part
+  int rows_part;  // rows of a part (16 or 32)
+  int cw;         // columns per slot (K / kGemvSlots)
   int pairs;      // 1: two parts (rotate-half or gate/up pairs)
 };
 
@@ -118,7 +119,7 @@ struct Smem {
     alignas(16) float xs[2048];
     alignas(16) __nv_bfloat16 xa[kMaxB * kActPitch];
   };
-  alignas(16) float gred[2][kComputeWarps][16][4];  // GEMV partial tiles (double-buffered)
+  alignas(16) float gred[2][kComputeWarps][32][4];  // GEMV partial tiles (double-buffered)
   float red8[kMaxB][kComputeWarps];
   OpGeo geo[OP_COUNT];  // GEMV geometry per op, set in the prologue
   unsigned long long lm_seen[kComputeWarps][kMaxB];  // per compute warp: best argmax key it has published
@@ -247,11 +248,23 @@ struct ProdFam {
   int slots_per_part;
   int parts;
   size_t task_stride;         // bytes between consecutive tasks' first rows
+  const void* tm[3];          // GEMV ops: tensor maps of the parts' matrices (QKV: q, k, v)
 };
 
-__device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, int fam, int op, int layer, ProdFam& f) {
+__device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsigned char* tmaps, int fam, int op,
+                           int layer, ProdFam& f) {
   const uint32_t H2 = (uint32_t)P.hidden * 2;
   f.fam = fam; f.op = op; f.layer = layer;
+  auto tmap = [&](int l, int m) -> const void* { return tmaps + (size_t)tmap_index(l, m) * kTmapBytes; };
+  f.tm[0] = f.tm[1] = f.tm[2] = nullptr;
+  switch (op) {
+    case OP_QKV: f.tm[0] = tmap(layer, TM_WQ); f.tm[1] = tmap(layer, TM_WK); f.tm[2] = tmap(layer, TM_WV); break;
+    case OP_OPROJ: f.tm[0] = tmap(layer, TM_WO); break;
+    case OP_GATEUP: f.tm[0] = tmap(layer, TM_GATE); f.tm[1] = tmap(layer, TM_UP); break;
+    case OP_DOWN: f.tm[0] = tmap(layer, TM_DOWN); break;
+    case OP_LM: f.tm[0] = tmap(P.n_layers, 0); break;
+    default: break;
+  }
   f.row_bytes = H2; f.row_stride = H2; f.row_pitch = H2; f.rps = P.slot_bytes / (int)H2; f.parts = 1;
   f.w[0] = f.w[1] = f.w[2] = nullptr;
   f.task_stride = 0;
@@ -296,7 +309,7 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, int fam, i
 __device__ __forceinline__ int task_slots(const DevPlan& P, const ProdFam& f, int idx) {
   if (f.op == OP_ATTN) return 1;
   if (f.op == OP_ROUTE || f.op == OP_COMBINE || f.op == OP_MINDPTR || f.op == OP_MFIN) return 0;
-  if (f.op == OP_LM) return ceil_div(min(P.tile_lm, P.vocab - idx * P.tile_lm), f.rps);
+  if (f.op == OP_QKV || f.op == OP_OPROJ || f.op == OP_GATEUP || f.op == OP_DOWN || f.op == OP_LM) return kGemvSlots;
   return f.parts * f.slots_per_part;
 }
 
@@ -343,12 +356,29 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     return true;
   };
 
+  // a GEMV task's rows by column slices: slot j gets columns [x0 + j cw,
+  // x0 + (j + 1) cw) of part 0's rows (from row y0 of map tm0), then of part
+  // 1's rows (row y1 of tm1), as one TMA box each
+  auto stream_tiles = [&](int fam, int idx, int rows_part, int cw, int x0, const void* tm0, int y0, const void* tm1,
+                          int y1) -> bool {
+    const uint32_t part_bytes = (uint32_t)rows_part * cw * 2;
+    for (int j = 0; j < kGemvSlots; ++j) {
+      unsigned char* dst;
+      uint64_t* bar;
+      if (!next_slot(fam, idx, dst, bar)) return false;
+      mbar_arrive_expect_tx(bar, tm1 ? 2 * part_bytes : part_bytes);
+      tma_load_2d(dst, tm0, x0 + j * cw, y0, bar);
+      if (tm1) tma_load_2d(dst + part_bytes, tm1, x0 + j * cw, y1, bar);
+    }
+    return true;
+  };
+
   auto emit = [&](int fam, int idx) -> bool {
     int op = OP_END, layer = -1;
     if (fam >= 0) {
       op = sm.fam_op[fam];
       layer = sm.fam_layer[fam];
-      if (fam != f.fam) prod_setup(P, layers, fam, op, layer, f);
+      if (fam != f.fam) prod_setup(P, layers, ws + P.off_tmap, fam, op, layer, f);
     }
     TaskDesc d;
     d.fam = fam; d.idx = idx; d.op = op; d.layer = layer;
@@ -364,26 +394,30 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     if (fam < 0) return true;
     switch (op) {
       case OP_QKV: {
+        // rotate-half pairs: rows j0.. of the head, then rows j0 + D/2.. of it
         QkvTile q = decode_qkv(P, idx);
-        const unsigned char* base = f.w[q.kind] + ((size_t)q.head * P.head_dim + q.j0) * f.row_stride;
-        const int half = P.tile_qkv / 2;
-        if (!stream_part(fam, idx, base, half)) return false;
-        if (!stream_part(fam, idx, base + (size_t)(P.head_dim / 2) * f.row_stride, half)) return false;
+        const int y = q.head * P.head_dim + q.j0, half = P.tile_qkv / 2;
+        if (!stream_tiles(fam, idx, half, P.hidden / kGemvSlots, 0, f.tm[q.kind], y, f.tm[q.kind],
+                          y + P.head_dim / 2))
+          return false;
       } break;
       case OP_OPROJ:
-        if (!stream_part(fam, idx, f.w[0] + (size_t)idx * f.task_stride, P.tile_o)) return false;
+        if (!stream_tiles(fam, idx, P.tile_o, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_o, nullptr, 0))
+          return false;
         break;
       case OP_GATEUP:
-        if (!stream_part(fam, idx, f.w[0] + (size_t)idx * f.task_stride, P.tile_gu)) return false;
-        if (!stream_part(fam, idx, f.w[1] + (size_t)idx * f.task_stride, P.tile_gu)) return false;
+        if (!stream_tiles(fam, idx, P.tile_gu, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_gu, f.tm[1],
+                          idx * P.tile_gu))
+          return false;
         break;
       case OP_DOWN: {
-        int kc = idx / P.n_dtiles, n = idx - kc * P.n_dtiles;
-        const unsigned char* base = f.w[0] + (size_t)n * P.tile_down * f.row_stride + (size_t)kc * f.row_bytes;
-        if (!stream_part(fam, idx, base, P.tile_down)) return false;
+        const int kc = idx / P.n_dtiles, n = idx - kc * P.n_dtiles;
+        if (!stream_tiles(fam, idx, P.tile_down, P.kseg / kGemvSlots, kc * P.kseg, f.tm[0], n * P.tile_down, nullptr,
+                          0))
+          return false;
       } break;
-      case OP_LM:
-        if (!stream_part(fam, idx, f.w[0] + (size_t)idx * f.task_stride, min(P.tile_lm, P.vocab - idx * P.tile_lm)))
+      case OP_LM:  // the last tile's rows past the vocabulary read as zeros
+        if (!stream_tiles(fam, idx, P.tile_lm, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_lm, nullptr, 0))
           return false;
         break;
       case OP_EGU: {
@@ -1097,14 +1131,14 @@ __device__ __forceinline__ void gemv_epilogue_ahead(const DevPlan& P, const Smem
 }
 
 // A GEMV task on tensor cores: Y[rows x B] = W[rows x K] . A[B x K]^T, W
-// the task's rows in its ring slots (bf16), A the staged activation rows.
-// The task's rows form nrb = rows / 16 row blocks (pair ops: part 0's blocks,
-// then part 1's); warp w takes row block w / kp over K part w % kp (kp = 8 /
-// nrb) with the activation rows as the MMA's n = 8 columns (column n reads
-// row min(n, B - 1)).  Each warp leaves its 16 x 4 partial tile in
-// sm.gred[buf]; after a barrier, thread ct sums the kp partials of its item
-// (batch row b, row or pair r) and runs the op's epilogue.  Every warp waits
-// for every slot of the task and then releases each with a share of 1.
+// the task's (at most 32) rows in its kGemvSlots ring slots (bf16, by column
+// slice), A the staged activation rows.  Warp w reads only slot w: every row
+// block (16 rows) of the task over columns [w cw, (w + 1) cw), with the
+// activation rows as the MMA's n = 8 columns (column n reads row min(n, B -
+// 1)); it waits for that slot alone and releases it (the slot's only reader)
+// as soon as its products are done.  Each warp leaves its rows x 4 partial
+// tile in sm.gred[buf]; after a barrier, thread ct sums the 8 partials of its
+// item (batch row b, row or pair r) and runs the op's epilogue.
 __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                           unsigned char* ws, Control* ctl, const TaskDesc& d, const GemvSpec& g,
                                           int B, int buf, const EpiAhead& ea, const GemvItem& it, uint32_t* trec) {
@@ -1113,74 +1147,71 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   const int R = P.ring_slots;
   const int s0 = d.slot_ph & 0xffff;
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int nparts = geo.pairs ? 2 : 1;
-  const int nslots = d.nslots;
-  for (int j = 0; j < nslots; ++j) {
-    const int sj = s0 + j < R ? s0 + j : s0 + j - R;
-    wait_mbar(&sm.full[sj], s0 + j < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  }
+  const int sw = s0 + w < R ? s0 + w : s0 + w - R;  // this warp's slot
+  wait_mbar(&sm.full[sw], s0 + w < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
   if (trec && lane == 0) {
     trec[TR_DATA] = (uint32_t)global_ns();
     trec[TR_ISSUE] = sm.slot_t[s0];
   }
-  // this warp's row block and K part
-  const int rows_total = nparts * geo.rows_part;
-  const int nrb = rows_total >> 4;
-  const int kp = kComputeWarps / nrb;
-  const int rb = w / kp, kpi = w - rb * kp;
-  const int rbp = geo.rows_part >> 4;         // row blocks per part
-  const int part = rb / rbp;
-  const int valid = geo.pairs ? geo.rows_part : g.rows;  // valid rows of the part
+  const int nrb = (geo.pairs ? 2 : 1) * geo.rows_part >> 4;  // row blocks: 1 or 2
   const int g8 = lane >> 2, q = lane & 3;
-  int ra = (rb - part * rbp) * 16 + g8, rbb = ra + 8;
-  ra = min(ra, valid - 1);
-  rbb = min(rbb, valid - 1);
-  auto row_ptr = [&](int r) -> const unsigned char* {
-    const int j = part * geo.spp + (r >> geo.rps_lg);
-    const int sj = s0 + j < R ? s0 + j : s0 + j - R;
-    return ring + (size_t)sj * P.slot_bytes + (size_t)(r & ((1 << geo.rps_lg) - 1)) * geo.row_bytes;
-  };
-  const int kw = g.K / kp;  // columns of this warp
-  const int kbase = kpi * kw;
-  const uint4* pa = reinterpret_cast<const uint4*>(row_ptr(ra) + (size_t)kbase * 2) + q;
-  const uint4* pb = reinterpret_cast<const uint4*>(row_ptr(rbb) + (size_t)kbase * 2) + q;
-  const uint4* px = reinterpret_cast<const uint4*>(&sm.xa[min(g8, B - 1) * kActPitch + kbase]) + q;
-  const int nwin = kw >> 5;
-  float c[4][4];
+  const int pitch = geo.cw * 2;  // bytes per row in the slot
+  const unsigned char* slot = ring + (size_t)sw * P.slot_bytes;
+  const uint4* pa0 = reinterpret_cast<const uint4*>(slot + (size_t)g8 * pitch) + q;
+  const uint4* pb0 = reinterpret_cast<const uint4*>(slot + (size_t)(g8 + 8) * pitch) + q;
+  const uint4* pa1 = reinterpret_cast<const uint4*>(slot + (size_t)(g8 + 16) * pitch) + q;
+  const uint4* pb1 = reinterpret_cast<const uint4*>(slot + (size_t)(g8 + 24) * pitch) + q;
+  const uint4* px = reinterpret_cast<const uint4*>(&sm.xa[min(g8, B - 1) * kActPitch + w * geo.cw]) + q;
+  const int nwin = geo.cw >> 5;
+  float c0[2][4], c1[2][4];  // row blocks 0 and 1, two accumulators each
 #pragma unroll
-  for (int u = 0; u < 4; ++u) c[u][0] = c[u][1] = c[u][2] = c[u][3] = 0.f;
-  for (int w4 = 0; w4 < nwin; w4 += 4) {
+  for (int u = 0; u < 2; ++u)
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (w4 + u < nwin) {
-        const int o = (w4 + u) * 4;  // 16-byte chunks per 32-column window
-        mma_window(c[u], pa[o], pb[o], px[o]);
+    for (int i = 0; i < 4; ++i) c0[u][i] = c1[u][i] = 0.f;
+  // windows in pairs, alternating accumulators (16-byte chunks: 4 per window)
+  if (nrb == 2) {
+    for (int win = 0; win < nwin; win += 2) {
+      const int o = win * 4;
+      const uint4 xb = px[o];
+      mma_window(c0[0], pa0[o], pb0[o], xb);
+      mma_window(c1[0], pa1[o], pb1[o], xb);
+      if (win + 1 < nwin) {
+        const uint4 xb1 = px[o + 4];
+        mma_window(c0[1], pa0[o + 4], pb0[o + 4], xb1);
+        mma_window(c1[1], pa1[o + 4], pb1[o + 4], xb1);
       }
+    }
+  } else {
+    for (int win = 0; win < nwin; win += 2) {
+      const int o = win * 4;
+      mma_window(c0[0], pa0[o], pb0[o], px[o]);
+      if (win + 1 < nwin) mma_window(c0[1], pa0[o + 4], pb0[o + 4], px[o + 4]);
+    }
   }
   __syncwarp();
-  if (lane == 0)
-    for (int j = 0; j < nslots; ++j) {
-      const int sj = s0 + j < R ? s0 + j : s0 + j - R;
-      release_share(sm, sj, kComputeWarps, w);
-    }
-  // partial tile: lane (g8, q < 2) holds rows g8, g8 + 8 at batch columns 2q, 2q + 1
-  float (*red)[16][4] = sm.gred[buf];
+  if (lane == 0) release_share(sm, sw, 1, 0);  // the slot's only reader
+  // partial tile: lane (g8, q < 2) holds rows g8, g8 + 8 (+ 16 for block 1)
+  // at batch columns 2q, 2q + 1
+  float (*red)[32][4] = sm.gred[buf];
   if (q < 2) {
-    const float d0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]), d1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
-    const float d2 = (c[0][2] + c[1][2]) + (c[2][2] + c[3][2]), d3 = (c[0][3] + c[1][3]) + (c[2][3] + c[3][3]);
-    *reinterpret_cast<float2*>(&red[w][g8][2 * q]) = make_float2(d0, d1);
-    *reinterpret_cast<float2*>(&red[w][g8 + 8][2 * q]) = make_float2(d2, d3);
+    *reinterpret_cast<float2*>(&red[w][g8][2 * q]) = make_float2(c0[0][0] + c0[1][0], c0[0][1] + c0[1][1]);
+    *reinterpret_cast<float2*>(&red[w][g8 + 8][2 * q]) = make_float2(c0[0][2] + c0[1][2], c0[0][3] + c0[1][3]);
+    if (nrb == 2) {
+      *reinterpret_cast<float2*>(&red[w][g8 + 16][2 * q]) = make_float2(c1[0][0] + c1[1][0], c1[0][1] + c1[1][1]);
+      *reinterpret_cast<float2*>(&red[w][g8 + 24][2 * q]) = make_float2(c1[0][2] + c1[1][2], c1[0][3] + c1[1][3]);
+    }
   }
   bar_sync(BAR_COMP, kComputeThreads);
   // epilogue: item (b, r); v0 = row r (pair ops: part 0 row r), v1 = part 1 row r
   const int b = it.b, r = it.r;
-  const bool mine = it.on && r < (geo.pairs ? geo.rows_part : g.rows);
+  const bool mine = it.on && (geo.pairs || d.op != OP_LM || d.idx * P.tile_lm + r < P.vocab);
   float v0 = 0.f, v1 = 0.f;
   if (mine) {
-    const int rb0 = r >> 4, rr = r & 15;
-    for (int k = 0; k < kp; ++k) v0 += red[rb0 * kp + k][rr][b];
+#pragma unroll
+    for (int k = 0; k < kComputeWarps; ++k) v0 += red[k][r][b];
     if (geo.pairs)
-      for (int k = 0; k < kp; ++k) v1 += red[(rbp + rb0) * kp + k][rr][b];
+#pragma unroll
+      for (int k = 0; k < kComputeWarps; ++k) v1 += red[k][geo.rows_part + r][b];
   }
   const int H = P.hidden;
   switch (d.op) {
@@ -1996,11 +2027,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     // GEMV geometry of each op (see OpGeo)
     auto set_geo = [&](int op, int K, int rows_part, int pairs) {
       OpGeo& gg = sm.geo[op];
-      const int rps = P.slot_bytes / (2 * K);
       gg.rows_part = rows_part;
-      gg.row_bytes = 2 * K;
-      gg.rps_lg = __ffs(rps) - 1;
-      gg.spp = ceil_div(rows_part, rps);
+      gg.cw = K / kGemvSlots;
       gg.pairs = pairs;
     };
     if (!moe) {
@@ -2115,9 +2143,72 @@ mk_status dev_query(int* n_sm, int* smem_optin, int* device, std::string& err) {
 
 int smem_fixed_bytes() { return (int)((sizeof(Smem) + 1023) / 1024 * 1024); }
 
-mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vector<unsigned char>& image,
+// The driver's tensor-map encoder, looked up once through the runtime (no
+// link-time dependency on the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// Tensor maps of the dense weight matrices, written into the plan image: a
+// bf16 [rows][cols] matrix with a row stride, read in boxes of (cols / 8)
+// columns x box_rows rows (one box per ring slot and part); rows past the
+// end read as zeros.
+static bool encode_weight_maps(const DevPlan& P, std::vector<unsigned char>& image, std::string& err) {
+  if (P.kind == MK_MODEL_MOE_LAYER) return true;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) { err = "cuTensorMapEncodeTiled is not available"; return false; }
+  const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(image.data() + (P.off_layers - P.off_families));
+  auto put = [&](int index, const void* w, long long rows, long long cols, long long stride_elems, int box_cols,
+                 int box_rows, const char* what) -> bool {
+    if (!w) return true;  // (an MoE decoder has no dense FFN)
+    if (reinterpret_cast<uintptr_t>(w) & 15) { err = std::string(what) + " must be 16-byte aligned"; return false; }
+    CUtensorMap m;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)stride_elems * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) { err = std::string("tensor map of ") + what + " rejected by the driver"; return false; }
+    std::memcpy(image.data() + (P.off_tmap - P.off_families) + (size_t)index * kTmapBytes, &m, sizeof(m));
+    return true;
+  };
+  static_assert(sizeof(CUtensorMap) == kTmapBytes, "tensor map size");
+  const int H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads, F = P.ffn;
+  for (int l = 0; l < P.n_layers; ++l) {
+    const LayerPtrs& lp = layers[l];
+    const int bh = H / kGemvSlots;  // columns per slot of a hidden-wide row
+    if (!put(tmap_index(l, TM_WQ), lp.wq, (long long)Hq * D, H, H, bh, P.tile_qkv / 2, "wq") ||
+        !put(tmap_index(l, TM_WK), lp.wk, (long long)Hkv * D, H, H, bh, P.tile_qkv / 2, "wk") ||
+        !put(tmap_index(l, TM_WV), lp.wv, (long long)Hkv * D, H, H, bh, P.tile_qkv / 2, "wv") ||
+        !put(tmap_index(l, TM_WO), lp.wo, H, (long long)Hq * D, (long long)Hq * D, bh, P.tile_o, "wo"))
+      return false;
+    if (P.kind == MK_MODEL_DENSE &&
+        (!put(tmap_index(l, TM_GATE), lp.w_gate, F, H, H, bh, P.tile_gu, "w_gate") ||
+         !put(tmap_index(l, TM_UP), lp.w_up, F, H, H, bh, P.tile_gu, "w_up") ||
+         !put(tmap_index(l, TM_DOWN), lp.w_down, H, F, F, P.kseg / kGemvSlots, P.tile_down, "w_down")))
+      return false;
+  }
+  return put(tmap_index(P.n_layers, 0), P.lm_head, P.vocab, H, H, H / kGemvSlots, P.tile_lm, "lm_head");
+}
+
+mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vector<unsigned char>& image_in,
                    std::string& err) {
   cudaStream_t s = (cudaStream_t)stream;
+  std::vector<unsigned char> image = image_in;
+  if (!encode_weight_maps(p.dp, image, err)) return MK_ERR_INVALID_ARG;
   size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + sizeof(Smem);
   const void* kern = kernel_for(p.dp);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -2193,9 +2284,6 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
     err = "plan scratch exceeds MK_STATIC_SCRATCH_BYTES";
     return MK_ERR_WORKSPACE;
   }
-  // the plan arrays below are exactly what the workspace image holds
-  const long long rope_end = P0.off_rope + (4LL * (long long)p.rope.size() + 255) / 256 * 256;
-  if (rope_end != P0.off_queue) { err = "plan arrays do not match the workspace layout"; return MK_ERR_PLAN; }
 
   std::lock_guard<std::mutex> lock(g_static_mu);
   StaticScratchState& st = g_static[dev];
@@ -2220,15 +2308,12 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel_for(P0), kThreads, smem);
       if (e == cudaSuccess && nb < 1) { err = "megakernel does not fit on an SM"; return MK_ERR_UNSUPPORTED; }
     }
-    // the read-only plan arrays, copied from the plan's own host vectors
-    auto put = [&](long long off, const void* src, size_t n) {
-      if (e == cudaSuccess && n) e = cudaMemcpyAsync(ws + off, src, n, cudaMemcpyHostToDevice, s);
-    };
-    put(P0.off_families, p.fams.data(), sizeof(FamilyDesc) * p.fams.size());
-    put(P0.off_expr, p.code.data(), 4 * p.code.size());
-    put(P0.off_instr, p.instr.data(), sizeof(Instr) * p.instr.size());
-    put(P0.off_layers, p.layers.data(), sizeof(LayerPtrs) * p.layers.size());
-    put(P0.off_rope, p.rope.data(), 4 * p.rope.size());
+    // the read-only plan arrays and the weights' tensor maps (host memory only)
+    std::vector<unsigned char> image;
+    lower_plan(p, image);
+    if (!encode_weight_maps(P0, image, err)) return MK_ERR_INVALID_ARG;
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(ws + P0.off_families, image.data(), image.size(), cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) { err = std::string("plan upload failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
     st.owner = p.uid;
   }

@@ -233,7 +233,6 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
 }
 
 // ---------------------------------------------------------------- build
-static bool pow2_divides(int a, int b) { return a > 0 && b % a == 0; }
 
 // MoE FFN layer ("Event Tensor: A Unified Abstraction for Compiling Dynamic
 // Megakernel", section "Core method", data-dependent dynamism).  The task
@@ -392,53 +391,30 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   int kseg = mdec ? 2048 : (o->kseg ? o->kseg : std::min(F, 2048));  // (no dense FFN in an MoE decoder)
   while (kseg > 256 && F % kseg) kseg -= 256;
   P.kseg = kseg;
-  // rows per 16 KB ring slot of a hidden-wide (and a kseg-wide) row
-  const int rps_h = 8192 / H, rps_k = 8192 / kseg;
-  // tiles split evenly over the 8 compute warps (QKV and gate/up tiles hand
-  // each warp whole row pairs, the others whole rows).  Defaults: the largest
-  // legal tiles up to 8 ring slots per task (gate/up: 4 + 4; down: 8; O: 4
-  // slots, as O sits on the critical path), which amortise the fixed
-  // per-task cost best on the 1B shape
-  P.tile_qkv = o->tile_qkv ? o->tile_qkv : std::max(16, std::min(D, 8 * rps_h));
-  P.tile_o = o->tile_o ? o->tile_o : std::max(8, std::min(64, 4 * rps_h));
-  P.tile_gu = o->tile_gu ? o->tile_gu : std::max(8, std::min(32, 4 * rps_h));
-  P.tile_down = o->tile_down ? o->tile_down : std::max(8, std::min(64, 8 * rps_k));
-  P.tile_lm = o->tile_lm ? o->tile_lm : std::max(16, std::min(64, 8 * rps_h));
+  // GEMV tiles on tensor cores: 16 or 32 rows per task in whole 16-row
+  // blocks (QKV: 16 rotate-half pairs; gate/up: 16 gate + 16 up rows), spread
+  // over 8 ring slots by column: slot j holds columns [j K/8, (j+1) K/8) of
+  // every row of the task.  Defaults: the 32-row tasks, O at 16 rows (it sits
+  // on the critical path; more tasks than SMs)
+  P.tile_qkv = o->tile_qkv ? o->tile_qkv : 32;
+  P.tile_o = o->tile_o ? o->tile_o : 16;
+  P.tile_gu = o->tile_gu ? o->tile_gu : 16;
+  P.tile_down = o->tile_down ? o->tile_down : 32;
+  P.tile_lm = o->tile_lm ? o->tile_lm : 32;
   P.chunk = o->attn_chunk ? o->attn_chunk : 64;
   P.slot_bytes = 16384;
-  const int rows_per_slot_h = P.slot_bytes / (2 * H);
-  const int rows_per_slot_k = P.slot_bytes / (2 * kseg);
   if (!(P.kseg % 256 == 0 && F % P.kseg == 0 && P.kseg >= 1024 && P.kseg <= 2048))
     { err = "kseg must be a multiple of 256 in [1024, 2048] dividing ffn"; return MK_ERR_INVALID_ARG; }
   if (Hq / Hkv > 4) { err = "at most 4 query heads per kv head"; return MK_ERR_UNSUPPORTED; }
-  if (!(pow2_divides(P.tile_qkv, D) && P.tile_qkv % 16 == 0 && (P.tile_qkv / 2) % rows_per_slot_h == 0))
-    { err = "tile_qkv must be a multiple of 16 dividing head_dim, whole ring slots per half"; return MK_ERR_INVALID_ARG; }
-  if (!(pow2_divides(P.tile_o, H) && P.tile_o % rows_per_slot_h == 0 && P.tile_o % 8 == 0))
-    { err = "tile_o must divide hidden and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
-  if (!(pow2_divides(P.tile_gu, P.kseg) && P.tile_gu % rows_per_slot_h == 0 && P.tile_gu % 8 == 0))
-    { err = "tile_gu must divide kseg and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
-  if (!(pow2_divides(P.tile_down, H) && P.tile_down % rows_per_slot_k == 0 && P.tile_down % 8 == 0))
-    { err = "tile_down must divide hidden and fill whole ring slots"; return MK_ERR_INVALID_ARG; }
-  if (!(P.tile_lm > 0 && P.tile_lm % rows_per_slot_h == 0 && P.tile_lm % 8 == 0))
-    { err = "tile_lm must be a multiple of 8 filling whole ring slots"; return MK_ERR_INVALID_ARG; }
+  if (P.tile_qkv != 32) { err = "tile_qkv must be 32 (16 rotate-half pairs)"; return MK_ERR_UNSUPPORTED; }
+  if (!((P.tile_o == 16 || P.tile_o == 32) && H % P.tile_o == 0))
+    { err = "tile_o must be 16 or 32 and divide hidden"; return MK_ERR_UNSUPPORTED; }
+  if (P.tile_gu != 16 || P.kseg % P.tile_gu)
+    { err = "tile_gu must be 16 (16 gate + 16 up rows)"; return MK_ERR_UNSUPPORTED; }
+  if (!((P.tile_down == 16 || P.tile_down == 32) && H % P.tile_down == 0))
+    { err = "tile_down must be 16 or 32 and divide hidden"; return MK_ERR_UNSUPPORTED; }
+  if (P.tile_lm != 32) { err = "tile_lm must be 32"; return MK_ERR_UNSUPPORTED; }
   if (P.chunk != 64) { err = "attn_chunk must be 64"; return MK_ERR_UNSUPPORTED; }
-  // a task spans at most 8 ring slots
-  if (P.tile_qkv / rows_per_slot_h > 8 || P.tile_o / rows_per_slot_h > 8 || 2 * P.tile_gu / rows_per_slot_h > 8 ||
-      P.tile_down / rows_per_slot_k > 8 || ceil_div(P.tile_lm, rows_per_slot_h) > 8)
-    { err = "a tile spans more than 8 ring slots"; return MK_ERR_UNSUPPORTED; }
-  // tensor-core GEMV tiles: whole 16-row blocks per part, 1, 2, 4 or 8 blocks
-  // per task (the 8 compute warps split them evenly), at most 256 epilogue
-  // items (rows or pairs x batch rows) and LM items of one batch row per warp
-  auto blocks_ok = [](int rows_part, int parts) {
-    if (rows_part % 16) return false;
-    const int nrb = parts * rows_part / 16;
-    return nrb == 1 || nrb == 2 || nrb == 4 || nrb == 8;
-  };
-  if (!blocks_ok(P.tile_qkv / 2, 2) || !blocks_ok(P.tile_o, 1) || !blocks_ok(P.tile_gu, 2) ||
-      !blocks_ok(P.tile_down, 1) || !blocks_ok(P.tile_lm, 1) || P.tile_lm % 32)
-    { err = "GEMV tiles must be whole 16-row blocks (1, 2, 4 or 8 per task; tile_lm a multiple of 32)"; return MK_ERR_UNSUPPORTED; }
-  if (P.tile_qkv / 2 > 64 || P.tile_o > 64 || P.tile_gu > 64 || P.tile_down > 64 || P.tile_lm > 64)
-    { err = "a GEMV tile has more than 64 rows (pairs) per part"; return MK_ERR_UNSUPPORTED; }
   P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
   P.n_otiles = H / P.tile_o;
   P.n_gutiles = F / P.tile_gu;
@@ -623,6 +599,8 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_instr = take((long long)sizeof(Instr) * (long long)p.instr.size());
   P.off_layers = take((long long)sizeof(LayerPtrs) * P.n_layers);
   P.off_rope = take(4LL * (long long)p.rope.size());
+  // tensor maps of the dense weights (encoded when the workspace is bound)
+  P.off_tmap = take(P.kind == MK_MODEL_MOE_LAYER ? 0 : (long long)kTmapBytes * (P.n_layers * kTmapPerLayer + 1));
   P.off_queue = take((long long)sizeof(QRange) * P.queue_ranges);
   P.off_x = take(4LL * P.max_batch * P.hidden);
   P.off_q = take(4LL * P.max_batch * P.n_q_heads * P.head_dim);

@@ -184,7 +184,15 @@ struct LayerPtrs {
 };
 
 constexpr int kMaxFamilies = 256;
-constexpr int kSmemReserve = 29 * 1024;  // the kernel's fixed shared-memory area; the ring takes the rest
+constexpr int kSmemReserve = 33 * 1024;  // the kernel's fixed shared-memory area; the ring takes the rest
+// A GEMV task's weights arrive in kGemvSlots ring slots, slot j holding columns
+// [j K / 8, (j + 1) K / 8) of all the task's rows (one 2-D TMA box per part),
+// through one tensor map per dense weight matrix: matrix m of layer l at
+// index l * kTmapPerLayer + m, the LM head after the last layer.
+constexpr int kGemvSlots = 8;
+constexpr int kTmapBytes = 128;
+enum TmapMatrix : int { TM_WQ = 0, TM_WK, TM_WV, TM_WO, TM_GATE, TM_UP, TM_DOWN, kTmapPerLayer };
+MK_HD int tmap_index(int layer, int m) { return layer * kTmapPerLayer + m; }
 constexpr int kMaxBatch = 128;
 
 // Fixed header of the plan; passed to the kernel by value.  Offsets are in
@@ -208,6 +216,7 @@ struct DevPlan {
   // workspace offsets
   int64_t off_control, off_counters, off_families, off_expr, off_instr, off_layers, off_rope;
   int64_t off_queue, off_x, off_q, off_apart, off_attn, off_h, off_dpart, off_lmbest;
+  int64_t off_tmap;  // TMA tensor maps of the dense weights (kTmapBytes each, see tmap_index)
   int64_t ws_bytes;
   // global weights (device)
   const void* embed; const void* lm_head; const void* final_norm;

@@ -45,10 +45,14 @@ def test_plan_build_and_tiles():
 
 
 def test_plan_rejects_oversized_tiles():
-    # more than 8 ring slots per task, or more rows per warp than one slot holds
-    for bad in (dict(tile_gu=32), dict(tile_lm=64), dict(tile_o=64), dict(tile_down=64)):
+    # a GEMV task is at most 32 rows (two 16-row tensor-core blocks) spread
+    # over 8 column slices; tiles that are not whole 16-row blocks are refused
+    for bad in (dict(tile_gu=32), dict(tile_lm=64), dict(tile_o=64), dict(tile_down=64), dict(tile_o=8),
+                dict(tile_down=24), dict(tile_qkv=16), dict(tile_lm=16)):
         with pytest.raises(mk.MkError):
             _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148, **bad)
+    for ok in (dict(tile_o=32), dict(tile_down=16)):
+        _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148, **ok).close()
 
 
 def test_plan_rejects_bad_shapes():
@@ -90,7 +94,7 @@ def test_simulator_clean(sched, B, ctx):
     assert rep.nonzero_counters == 0 and rep.static_dynamic_mismatch == 0
     t = d.tiles()
     tiles = {k: t[k] for k in ("tile_qkv", "chunk", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm")}
-    assert tiles == dict(tile_qkv=64, chunk=64, tile_o=64, tile_gu=32, tile_down=64, kseg=1024, tile_lm=64)
+    assert tiles == dict(tile_qkv=32, chunk=64, tile_o=16, tile_gu=16, tile_down=32, kseg=1024, tile_lm=32)
     assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, tiles))
 
 
