@@ -175,6 +175,8 @@ __device__ __forceinline__ bool wait_mbar(uint64_t* bar, uint32_t parity, Contro
 enum TraceField : int {
   TR_FAM = 0, TR_IDX = 1, TR_POP = 2, TR_READY = 3, TR_GO = 4, TR_DONE = 5, TR_NOTIFIED = 6,
   TR_CSTART = 7, TR_CEND = 8, TR_ISSUE = 9, TR_DATA = 10,
+  // GEMV tasks: activation staged, products done, partial tiles summed
+  TR_STAGED = 11, TR_MATH = 12, TR_RED = 13,
   // header fields
   TRH_RECORDS = 0, TRH_BATCHES = 1, TRH_NOTIFIED = 2, TRH_FENCE_NS = 3
 };
@@ -257,6 +259,13 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsi
   f.fam = fam; f.op = op; f.layer = layer;
   auto tmap = [&](int l, int m) -> const void* { return tmaps + (size_t)tmap_index(l, m) * kTmapBytes; };
   f.tm[0] = f.tm[1] = f.tm[2] = nullptr;
+  // the RMSNorm gain this family's staging reads (one 2H-byte row, not
+  // otherwise L2-resident after a step's weight stream) goes to L2 now, long
+  // before the family's first task runs
+  const void* gain = op == OP_QKV ? layers[layer].attn_norm
+                     : op == OP_GATEUP ? layers[layer].ffn_norm
+                     : op == OP_LM ? P.final_norm : nullptr;
+  if (gain) bulk_prefetch_l2(gain, H2);
   switch (op) {
     case OP_QKV: f.tm[0] = tmap(layer, TM_WQ); f.tm[1] = tmap(layer, TM_WK); f.tm[2] = tmap(layer, TM_WV); break;
     case OP_OPROJ: f.tm[0] = tmap(layer, TM_WO); break;
@@ -367,8 +376,14 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       uint64_t* bar;
       if (!next_slot(fam, idx, dst, bar)) return false;
       mbar_arrive_expect_tx(bar, tm1 ? 2 * part_bytes : part_bytes);
-      tma_load_2d(dst, tm0, x0 + j * cw, y0, bar);
-      if (tm1) tma_load_2d(dst + part_bytes, tm1, x0 + j * cw, y1, bar);
+      if (cw >= 64) {  // swizzled [rows][cw / 64][64] boxes
+        const int xc = (x0 + j * cw) >> 6;
+        tma_load_3d(dst, tm0, 0, xc, y0, bar);
+        if (tm1) tma_load_3d(dst + part_bytes, tm1, 0, xc, y1, bar);
+      } else {
+        tma_load_2d(dst, tm0, x0 + j * cw, y0, bar);
+        if (tm1) tma_load_2d(dst + part_bytes, tm1, x0 + j * cw, y1, bar);
+      }
     }
     return true;
   };
@@ -623,10 +638,12 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
   }
 }
 
-// Notifier warp: drains up to kFollowQ entries of the done queue at a time,
-// orders all their outputs with ONE gpu-scope release fence, then decrements
-// the counters (one lane per task; result-free decrements of the same counter
-// are combined into one add).
+// Notifier warp: drains up to kFollowQ entries of the done queue at a time
+// and decrements their counters with gpu-scope release operations (one lane
+// per distinct counter; decrements of the same counter are combined into one
+// add).  The release covers every output of the batch's tasks: the compute
+// warps' writes precede the done barrier, the controller's queue hand-off
+// and this warp's reads in CTA order, and release is cumulative.
 __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, Control* ctl,
                          int* counters) {
   const int lane = threadIdx.x & 31;
@@ -650,9 +667,7 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       ni = notify_info(P, S, sm, t);
     }
     __syncwarp();
-    unsigned long long tf0 = trace ? global_ns() : 0;
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    if (trace) { fence_ns += global_ns() - tf0; n_batches++; }
+    if (trace) n_batches++;
     // one atomic per distinct counter of the batch: the lowest lane of each
     // group subtracts the group's size; when the old value is needed, the
     // counter reached zero iff it equalled that size (the follow-up and the
@@ -670,7 +685,7 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
         if (old < cnt) record_error(ctl, MK_ERR_DEVICE_BOUNDS, t.fam, t.idx, key);
         fired = old == cnt;
       } else {
-        asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(counters + key), "r"(-cnt) : "memory");
+        asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(counters + key), "r"(-cnt) : "memory");
       }
     }
     if (fired && P.sched == MK_SCHED_DYNAMIC) push_successors(P, S, sm, ctl, ws, t);
@@ -989,56 +1004,73 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
   else { src = reinterpret_cast<const float*>(ws + P.off_h) + (size_t)g.kc * P.kseg; rstride = P.ffn; }
   const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
   const int nq = g.parts ? P.n_kc : 0;
-  // every load of the chunk (all rows, split-K partials, norm gain) is issued
-  // before the first use, so staging costs about one round trip to L2
+  // every load of a row's chunk (x or the activation, up to four split-K
+  // partials) is issued before the first use, rows one after another, so
+  // staging costs about one round trip to L2 per row at most
   float4 u[kMaxB], v[kMaxB];
   uint4 graw = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-  for (int b = 0; b < kMaxB; ++b) {
-    u[b] = make_float4(0.f, 0.f, 0.f, 0.f);
-    v[b] = u[b];
-    if (has && b < B) {
-      const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
-      u[b] = __ldcg(p4);
-      v[b] = __ldcg(p4 + 1);
-    }
-  }
   if (has && g.kind == 0) {
     const void* gp = g.gamma_sel == 2 ? P.final_norm
                                       : (g.gamma_sel == 1 ? layers[g.layer].ffn_norm : layers[g.layer].attn_norm);
     graw = __ldg(reinterpret_cast<const uint4*>(gp) + c / 8);
   }
-  if (has)
-#pragma unroll 4
-    for (int q = 0; q < nq; ++q) {
 #pragma unroll
-      for (int b = 0; b < kMaxB; ++b)
-        if (b < B) {
+  for (int b = 0; b < kMaxB; ++b) {
+    u[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+    v[b] = u[b];
+    if (has && b < B) {
+      float4 t[5][2];
+      const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
+      t[0][0] = __ldcg(p4);
+      t[0][1] = __ldcg(p4 + 1);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        t[q + 1][0] = t[q + 1][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (q < nq) {
           const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
-          const float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
-          u[b].x += a4.x; u[b].y += a4.y; u[b].z += a4.z; u[b].w += a4.w;
-          v[b].x += b4.x; v[b].y += b4.y; v[b].z += b4.z; v[b].w += b4.w;
+          t[q + 1][0] = __ldcg(d4);
+          t[q + 1][1] = __ldcg(d4 + 1);
         }
+      }
+      auto sum5 = [&](int h) {
+        float4 r;
+        r.x = t[0][h].x + ((t[1][h].x + t[2][h].x) + (t[3][h].x + t[4][h].x));
+        r.y = t[0][h].y + ((t[1][h].y + t[2][h].y) + (t[3][h].y + t[4][h].y));
+        r.z = t[0][h].z + ((t[1][h].z + t[2][h].z) + (t[3][h].z + t[4][h].z));
+        r.w = t[0][h].w + ((t[1][h].w + t[2][h].w) + (t[3][h].w + t[4][h].w));
+        return r;
+      };
+      u[b] = sum5(0);
+      v[b] = sum5(1);
+      for (int q = 4; q < nq; ++q) {  // (more than four K segments)
+        const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
+        const float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
+        u[b].x += a4.x; u[b].y += a4.y; u[b].z += a4.z; u[b].w += a4.w;
+        v[b].x += b4.x; v[b].y += b4.y; v[b].z += b4.z; v[b].w += b4.w;
+      }
     }
+  }
   float inv[kMaxB];
 #pragma unroll
   for (int b = 0; b < kMaxB; ++b) inv[b] = 1.f;
   if (g.kind == 0) {
 #pragma unroll
-    for (int b = 0; b < kMaxB; ++b) {
-      float ss = u[b].x * u[b].x + u[b].y * u[b].y + u[b].z * u[b].z + u[b].w * u[b].w + v[b].x * v[b].x +
-                 v[b].y * v[b].y + v[b].z * v[b].z + v[b].w * v[b].w;
-      ss = warp_sum(ss);
-      if (lane == 0) sm.red8[b][w] = ss;
-    }
+    for (int b = 0; b < kMaxB; ++b)
+      if (b < B) {
+        float ss = u[b].x * u[b].x + u[b].y * u[b].y + u[b].z * u[b].z + u[b].w * u[b].w + v[b].x * v[b].x +
+                   v[b].y * v[b].y + v[b].z * v[b].z + v[b].w * v[b].w;
+        ss = warp_sum(ss);
+        if (lane == 0) sm.red8[b][w] = ss;
+      }
     bar_sync(BAR_COMP, kComputeThreads);  // (also: every warp is done with the previous activation)
 #pragma unroll
-    for (int b = 0; b < kMaxB; ++b) {
-      float tot = 0.f;
+    for (int b = 0; b < kMaxB; ++b)
+      if (b < B) {
+        float tot = 0.f;
 #pragma unroll
-      for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[b][q];
-      inv[b] = 1.0f / sqrtf(tot / (float)K + P.eps);
-    }
+        for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[b][q];
+        inv[b] = 1.0f / sqrtf(tot / (float)K + P.eps);
+      }
   } else {
     bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the previous activation
   }
@@ -1157,10 +1189,14 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   const int g8 = lane >> 2, q = lane & 3;
   const int pitch = geo.cw * 2;  // bytes per row in the slot
   const unsigned char* slot = ring + (size_t)sw * P.slot_bytes;
-  const uint4* pa0 = reinterpret_cast<const uint4*>(slot + (size_t)g8 * pitch) + q;
-  const uint4* pb0 = reinterpret_cast<const uint4*>(slot + (size_t)(g8 + 8) * pitch) + q;
-  const uint4* pa1 = reinterpret_cast<const uint4*>(slot + (size_t)(g8 + 16) * pitch) + q;
-  const uint4* pb1 = reinterpret_cast<const uint4*>(slot + (size_t)(g8 + 24) * pitch) + q;
+  // 16-byte chunk (window win, lane chunk q) of slot row r: with cw >= 64 the
+  // rows are 128-byte lines under the 128-byte swizzle (chunk c of line n at
+  // c ^ (n & 7)), which puts the 8 rows a quarter-warp reads on distinct banks
+  const bool swz = geo.cw >= 64;
+  auto chunk = [&](int r, int win) -> const uint4* {
+    const int o = r * pitch + (win * 4 + q) * 16;
+    return reinterpret_cast<const uint4*>(slot + (swz ? (o ^ (((o >> 7) & 7) << 4)) : o));
+  };
   const uint4* px = reinterpret_cast<const uint4*>(&sm.xa[min(g8, B - 1) * kActPitch + w * geo.cw]) + q;
   const int nwin = geo.cw >> 5;
   float c0[2][4], c1[2][4];  // row blocks 0 and 1, two accumulators each
@@ -1171,25 +1207,24 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   // windows in pairs, alternating accumulators (16-byte chunks: 4 per window)
   if (nrb == 2) {
     for (int win = 0; win < nwin; win += 2) {
-      const int o = win * 4;
-      const uint4 xb = px[o];
-      mma_window(c0[0], pa0[o], pb0[o], xb);
-      mma_window(c1[0], pa1[o], pb1[o], xb);
+      const uint4 xb = px[win * 4];
+      mma_window(c0[0], *chunk(g8, win), *chunk(g8 + 8, win), xb);
+      mma_window(c1[0], *chunk(g8 + 16, win), *chunk(g8 + 24, win), xb);
       if (win + 1 < nwin) {
-        const uint4 xb1 = px[o + 4];
-        mma_window(c0[1], pa0[o + 4], pb0[o + 4], xb1);
-        mma_window(c1[1], pa1[o + 4], pb1[o + 4], xb1);
+        const uint4 xb1 = px[win * 4 + 4];
+        mma_window(c0[1], *chunk(g8, win + 1), *chunk(g8 + 8, win + 1), xb1);
+        mma_window(c1[1], *chunk(g8 + 16, win + 1), *chunk(g8 + 24, win + 1), xb1);
       }
     }
   } else {
     for (int win = 0; win < nwin; win += 2) {
-      const int o = win * 4;
-      mma_window(c0[0], pa0[o], pb0[o], px[o]);
-      if (win + 1 < nwin) mma_window(c0[1], pa0[o + 4], pb0[o + 4], px[o + 4]);
+      mma_window(c0[0], *chunk(g8, win), *chunk(g8 + 8, win), px[win * 4]);
+      if (win + 1 < nwin) mma_window(c0[1], *chunk(g8, win + 1), *chunk(g8 + 8, win + 1), px[win * 4 + 4]);
     }
   }
   __syncwarp();
   if (lane == 0) release_share(sm, sw, 1, 0);  // the slot's only reader
+  if (trec && lane == 0) trec[TR_MATH] = (uint32_t)global_ns();
   // partial tile: lane (g8, q < 2) holds rows g8, g8 + 8 (+ 16 for block 1)
   // at batch columns 2q, 2q + 1
   float (*red)[32][4] = sm.gred[buf];
@@ -1202,6 +1237,7 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
     }
   }
   bar_sync(BAR_COMP, kComputeThreads);
+  if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
   // epilogue: item (b, r); v0 = row r (pair ops: part 0 row r), v1 = part 1 row r
   const int b = it.b, r = it.r;
   const bool mine = it.on && (geo.pairs || d.op != OP_LM || d.idx * P.tile_lm + r < P.vocab);
@@ -1935,6 +1971,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
         stage_act(P, ws, sm, g, B);
         a_tag = g.tag;
       }
+      if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
       gemv_task(P, S, sm, ring, ws, ctl, d, g, B, gbuf, ea, it, trec);
       gbuf ^= 1;
     } else if (d.op == OP_ATTN) {
@@ -2174,18 +2211,35 @@ static bool encode_weight_maps(const DevPlan& P, std::vector<unsigned char>& ima
     if (!w) return true;  // (an MoE decoder has no dense FFN)
     if (reinterpret_cast<uintptr_t>(w) & 15) { err = std::string(what) + " must be 16-byte aligned"; return false; }
     CUtensorMap m;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)stride_elems * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r;
+    if (box_cols >= 64) {
+      // [rows][cols / 64][64] with the 128-byte swizzle: a box lands as rows of
+      // box_cols / 64 128-byte lines, 16-byte chunk c of line n at c ^ (n & 7)
+      const cuuint64_t dims[3] = {64, (cuuint64_t)cols / 64, (cuuint64_t)rows};
+      const cuuint64_t strides[2] = {128, (cuuint64_t)stride_elems * 2};
+      const cuuint32_t box[3] = {64, (cuuint32_t)box_cols / 64, (cuuint32_t)box_rows};
+      r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+      const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+      const cuuint64_t strides[1] = {(cuuint64_t)stride_elems * 2};
+      const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+      r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     if (r != CUDA_SUCCESS) { err = std::string("tensor map of ") + what + " rejected by the driver"; return false; }
     std::memcpy(image.data() + (P.off_tmap - P.off_families) + (size_t)index * kTmapBytes, &m, sizeof(m));
     return true;
   };
   static_assert(sizeof(CUtensorMap) == kTmapBytes, "tensor map size");
+  // the norm gains are prefetched into L2 with bulk copies: 16-byte aligned
+  for (int l = 0; l < P.n_layers; ++l)
+    if ((reinterpret_cast<uintptr_t>(layers[l].attn_norm) | reinterpret_cast<uintptr_t>(layers[l].ffn_norm)) & 15)
+      { err = "norm gains must be 16-byte aligned"; return false; }
+  if (reinterpret_cast<uintptr_t>(P.final_norm) & 15) { err = "final_norm must be 16-byte aligned"; return false; }
   const int H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads, F = P.ffn;
   for (int l = 0; l < P.n_layers; ++l) {
     const LayerPtrs& lp = layers[l];

@@ -8,14 +8,16 @@ timer in ns.  ``t_issue``: the producer issued the task's copies; ``t_pop``:
 the controller took it; ``t_ready``: its event had fired; ``t_go``: it was
 released; ``t_cstart``/``t_cend``: the compute warps started / finished it;
 ``t_data``: its first ring slot was full; ``t_done``: the controller saw it
-finish; ``t_notified``: its event counter was decremented.
+finish; ``t_notified``: its event counter was decremented.  GEMV tasks also
+record ``t_staged`` (activation staged), ``t_math`` (compute warp 0's
+products done) and ``t_red`` (partial tiles summed, epilogue starts).
 """
 from __future__ import annotations
 
 import json
 
 FIELDS = ["family", "index", "pop", "ready", "go", "done", "notified", "cstart", "cend", "issue", "data",
-          "lastdata", "math", "red", "epi"]
+          "staged", "math", "red"]
 
 
 def records(trace, fam_names):
