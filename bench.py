@@ -272,7 +272,7 @@ def torch_baselines(s, w, K, V, max_ctx, tok0, dev, n_steps):
                     "eager and as one captured CUDA graph; device-timed with CUDA events"}
 
 
-def batch_sweep(s, w, dev, n_steps=100, batches=(1, 2, 4)):
+def batch_sweep(s, w, dev, n_steps=100, batches=(1, 2, 4, 8)):
     """Decode steps of the same 1B model at several batch sizes through ONE
     plan and one compiled kernel (no rebuild, no graph capture), each
     sequence at its own context drawn uniform in [128, 4096] (seeded), next
@@ -321,7 +321,7 @@ def batch_sweep(s, w, dev, n_steps=100, batches=(1, 2, 4)):
                       "torch_cuda_graph_us_per_step": 1000.0 * gms})
     dec.close()
     return {"contexts": ctx0, "note": "one plan and one kernel for every B (no rebuild, no graph re-capture); "
-                                      "this build runs B <= 4", "cases": cases}
+                                      "this build runs B <= 8", "cases": cases}
 
 
 def profile_moe(T):
@@ -346,7 +346,7 @@ def moe_decoder_bench(dev, n_steps=64):
     """The MoE decoder: 16 layers with the 1B attention shape, each FFN the
     64-expert top-8 layer (F 1408), vocab 128256, tied embeddings; Zipf(1.2)
     skewed routing; dynamic schedule; continuous batching with the batch
-    size drawn per step from {1, 2, 3, 4} (this build's B limit) and
+    size drawn per step from {1, ..., 8} (this build's B limit) and
     contexts starting uniform in [256, 4096].  Its 17.7 GB of expert weights
     are drawn on the device (N(0, 0.02) bf16 from a seeded generator): this
     leg times the path; parity is tested on a two-layer model whose weights
@@ -374,7 +374,7 @@ def moe_decoder_bench(dev, n_steps=64):
         mlayers.append({"router": rnd(ms.n_experts, H), "w_gate": rnd(ms.n_experts, ms.expert_ffn, H),
                         "w_up": rnd(ms.n_experts, ms.expert_ffn, H), "w_down": rnd(ms.n_experts, H, ms.expert_ffn)})
     bias = wl.zipf_bias(ms.n_experts).to(dev)
-    maxB = 4
+    maxB = 8
     ctx0 = [int(c) for c in wl.context_lengths(maxB, 256, 4096, stream="moe-decoder-ctx")]
     max_ctx = max(ctx0) + n_steps + 16
     K = torch.zeros(L, maxB, s.n_kv_heads, max_ctx, D, dtype=torch.bfloat16, device=dev)
@@ -383,7 +383,7 @@ def moe_decoder_bench(dev, n_steps=64):
         K[:, b, :, :ctx0[b]] = torch.randn(L, s.n_kv_heads, ctx0[b], D, generator=gen, device=dev).to(torch.bfloat16)
         V[:, b, :, :ctx0[b]] = torch.randn(L, s.n_kv_heads, ctx0[b], D, generator=gen, device=dev).to(torch.bfloat16)
     dec = mk.DenseDecoder(s, w, K, V, max_batch=maxB, max_ctx=max_ctx, n_slots=maxB, moe=(ms, mlayers, bias))
-    sched = wl.batch_schedule(n_steps + 3, [1, 2, 3, 4])
+    sched = wl.batch_schedule(n_steps + 3, list(range(1, maxB + 1)))
     ran = [0] * maxB
     args = []
     for i, B in enumerate(sched):
@@ -411,7 +411,7 @@ def moe_decoder_bench(dev, n_steps=64):
     tokens = sum(sched[3:])
     dec.close()
     return {"workload": "MoE decoder: 16 layers (1B attention shape), 64 experts top-8 F 1408 per layer, vocab 128256, "
-                        "Zipf(1.2) routing, dynamic schedule, B per step from {1,2,3,4}, contexts from U[256,4096]",
+                        "Zipf(1.2) routing, dynamic schedule, B per step from {1..8}, contexts from U[256,4096]",
             "steps": n_steps, "tokens": tokens, "tokens_per_s": tokens / (total_ms / 1000.0),
             "us_per_step": 1000.0 * total_ms / n_steps,
             "us_per_step_by_B": {str(B): 1000.0 * statistics.mean(v) for B, v in sorted(per.items())},

@@ -52,9 +52,8 @@ constexpr int kFifo = 16;
 constexpr int kMaxSlots = 16;
 constexpr int kDoneQ = 32;    // controller -> notifier
 constexpr int kFollowQ = 16;  // notifier -> controller
-constexpr int kMaxB = 4;      // batch rows per step on this path
+constexpr int kMaxB = kMaxBatchRows;  // batch rows per step on this path
 constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
-constexpr int kActPitch = 2048 + 8;  // bf16 elements per staged activation row (16-byte bank offset per row)
 constexpr int kDynLookahead = 2;
 
 struct StepParams {
@@ -112,14 +111,15 @@ struct Smem {
   int ctx[kSmemBatch], slot[kSmemBatch], tok[kSmemBatch], nch[kSmemBatch], pre[kSmemBatch + 1];
   int fam_ext[kMaxFamilies];
   signed char fam_op[kMaxFamilies], fam_layer[kMaxFamilies];
-  // activation staging: one batch row, loaded once per CTA for all warps
-  // staging buffer: the GEMV activation rows (bf16, row b at b * kActPitch);
-  // other tasks use it as fp32 scratch (xs)
-  union {
-    alignas(16) float xs[2048];
-    alignas(16) __nv_bfloat16 xa[kMaxB * kActPitch];
-  };
-  alignas(16) float gred[2][kComputeWarps][32][4];  // GEMV partial tiles (double-buffered)
+  // the staging buffer, kSmemFixed bytes past this struct's start: the GEMV
+  // activation rows (bf16, row b at b * kActPitch), or fp32 scratch (xs) for
+  // the other task bodies; then the GEMV partial tiles (two buffers of
+  // [8 warps][32 rows][gbatch]).  Addresses derived from `this`, so the
+  // compiler keeps them in the shared window (shared-memory instructions).
+  __device__ __forceinline__ unsigned char* stage() { return reinterpret_cast<unsigned char*>(this) + kSmemFixed; }
+  __device__ __forceinline__ float* xs() { return reinterpret_cast<float*>(stage()); }
+  __device__ __forceinline__ __nv_bfloat16* xa() { return reinterpret_cast<__nv_bfloat16*>(stage()); }
+  __device__ __forceinline__ float* gred(int act_bytes) { return reinterpret_cast<float*>(stage() + act_bytes); }
   float red8[kMaxB][kComputeWarps];
   OpGeo geo[OP_COUNT];  // GEMV geometry per op, set in the prologue
   unsigned long long lm_seen[kComputeWarps][kMaxB];  // per compute warp: best argmax key it has published
@@ -133,8 +133,8 @@ struct Smem {
   volatile int dq_head, dq_tail, fq_head, fq_tail, notifier_stop;
   int bad;
 };
-static_assert(sizeof(Smem) <= kSmemReserve, "fixed shared-memory area exceeds its reserve");
-static_assert(offsetof(Smem, xs) % 16 == 0, "vector accesses to the staging buffer need 16-byte alignment");
+static_assert(sizeof(Smem) <= kSmemFixed, "fixed shared-memory area exceeds its reserve");
+static_assert(kSmemFixed % 128 == 0, "the staging buffer needs 128-byte alignment");
 static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, fifo_full) % 8 == 0, "mbarriers need 8-byte alignment");
 constexpr int BAR_COMP = 3;  // named barrier of the 8 compute warps
 
@@ -986,11 +986,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Activation rows 0..B-1 of a GEMV family into shared memory, bf16 (the
-// tensor-core operand type), row b at sm.xa + b * kActPitch: the compute
+// tensor-core operand type), row b at sm.xa() + b * kActPitch: the compute
 // warps load them once for the CTA (adding the previous layer's down
 // partials to x when asked), reduce each row's sum of squares and apply the
-// RMSNorm.  Called by all compute warps for the same task (the tag sequence
-// is the same for all warps).  Thread t stages columns [8t, 8t + 8).
+// RMSNorm.  Rows go in groups of four (one round trip to L2 per group: every
+// load of a group is issued before the first use).  Called by all compute
+// warps for the same task (the tag sequence is the same for all warps).
+// Thread t stages columns [8t, 8t + 8).
 __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int B) {
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
@@ -1004,88 +1006,88 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
   else { src = reinterpret_cast<const float*>(ws + P.off_h) + (size_t)g.kc * P.kseg; rstride = P.ffn; }
   const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart);
   const int nq = g.parts ? P.n_kc : 0;
-  // every load of a row's chunk (x or the activation, up to four split-K
-  // partials) is issued before the first use, rows one after another, so
-  // staging costs about one round trip to L2 per row at most
-  float4 u[kMaxB], v[kMaxB];
+  // (the gain stays raw until its first use, so its load overlaps the rows')
   uint4 graw = make_uint4(0u, 0u, 0u, 0u);
   if (has && g.kind == 0) {
     const void* gp = g.gamma_sel == 2 ? P.final_norm
                                       : (g.gamma_sel == 1 ? layers[g.layer].ffn_norm : layers[g.layer].attn_norm);
     graw = __ldg(reinterpret_cast<const uint4*>(gp) + c / 8);
   }
+  for (int b0 = 0; b0 < B; b0 += 4) {
+    float4 u[4], v[4];
 #pragma unroll
-  for (int b = 0; b < kMaxB; ++b) {
-    u[b] = make_float4(0.f, 0.f, 0.f, 0.f);
-    v[b] = u[b];
-    if (has && b < B) {
-      float4 t[5][2];
-      const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
-      t[0][0] = __ldcg(p4);
-      t[0][1] = __ldcg(p4 + 1);
+    for (int i = 0; i < 4; ++i) {
+      const int b = b0 + i;
+      u[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      v[i] = u[i];
+      if (has && b < B) {
+        float4 t[5][2];
+        const float4* p4 = reinterpret_cast<const float4*>(src + (size_t)b * rstride + c);
+        t[0][0] = __ldcg(p4);
+        t[0][1] = __ldcg(p4 + 1);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        t[q + 1][0] = t[q + 1][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (q < nq) {
+        for (int q = 0; q < 4; ++q) {
+          t[q + 1][0] = t[q + 1][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (q < nq) {
+            const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
+            t[q + 1][0] = __ldcg(d4);
+            t[q + 1][1] = __ldcg(d4 + 1);
+          }
+        }
+        auto sum5 = [&](int h) {
+          float4 r;
+          r.x = t[0][h].x + ((t[1][h].x + t[2][h].x) + (t[3][h].x + t[4][h].x));
+          r.y = t[0][h].y + ((t[1][h].y + t[2][h].y) + (t[3][h].y + t[4][h].y));
+          r.z = t[0][h].z + ((t[1][h].z + t[2][h].z) + (t[3][h].z + t[4][h].z));
+          r.w = t[0][h].w + ((t[1][h].w + t[2][h].w) + (t[3][h].w + t[4][h].w));
+          return r;
+        };
+        u[i] = sum5(0);
+        v[i] = sum5(1);
+        for (int q = 4; q < nq; ++q) {  // (more than four K segments)
           const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
-          t[q + 1][0] = __ldcg(d4);
-          t[q + 1][1] = __ldcg(d4 + 1);
+          const float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
+          u[i].x += a4.x; u[i].y += a4.y; u[i].z += a4.z; u[i].w += a4.w;
+          v[i].x += b4.x; v[i].y += b4.y; v[i].z += b4.z; v[i].w += b4.w;
         }
       }
-      auto sum5 = [&](int h) {
-        float4 r;
-        r.x = t[0][h].x + ((t[1][h].x + t[2][h].x) + (t[3][h].x + t[4][h].x));
-        r.y = t[0][h].y + ((t[1][h].y + t[2][h].y) + (t[3][h].y + t[4][h].y));
-        r.z = t[0][h].z + ((t[1][h].z + t[2][h].z) + (t[3][h].z + t[4][h].z));
-        r.w = t[0][h].w + ((t[1][h].w + t[2][h].w) + (t[3][h].w + t[4][h].w));
-        return r;
-      };
-      u[b] = sum5(0);
-      v[b] = sum5(1);
-      for (int q = 4; q < nq; ++q) {  // (more than four K segments)
-        const float4* d4 = reinterpret_cast<const float4*>(dp + ((size_t)q * P.max_batch + b) * P.hidden + c);
-        const float4 a4 = __ldcg(d4), b4 = __ldcg(d4 + 1);
-        u[b].x += a4.x; u[b].y += a4.y; u[b].z += a4.z; u[b].w += a4.w;
-        v[b].x += b4.x; v[b].y += b4.y; v[b].z += b4.z; v[b].w += b4.w;
-      }
     }
-  }
-  float inv[kMaxB];
+    float inv[4] = {1.f, 1.f, 1.f, 1.f};
+    if (g.kind == 0) {
 #pragma unroll
-  for (int b = 0; b < kMaxB; ++b) inv[b] = 1.f;
-  if (g.kind == 0) {
+      for (int i = 0; i < 4; ++i)
+        if (b0 + i < B) {
+          float ss = u[i].x * u[i].x + u[i].y * u[i].y + u[i].z * u[i].z + u[i].w * u[i].w + v[i].x * v[i].x +
+                     v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+          ss = warp_sum(ss);
+          if (lane == 0) sm.red8[b0 + i][w] = ss;
+        }
+    }
+    // (the first group's barrier also means every warp is done with the previous activation)
+    bar_sync(BAR_COMP, kComputeThreads);
+    if (g.kind == 0) {
 #pragma unroll
-    for (int b = 0; b < kMaxB; ++b)
-      if (b < B) {
-        float ss = u[b].x * u[b].x + u[b].y * u[b].y + u[b].z * u[b].z + u[b].w * u[b].w + v[b].x * v[b].x +
-                   v[b].y * v[b].y + v[b].z * v[b].z + v[b].w * v[b].w;
-        ss = warp_sum(ss);
-        if (lane == 0) sm.red8[b][w] = ss;
-      }
-    bar_sync(BAR_COMP, kComputeThreads);  // (also: every warp is done with the previous activation)
+      for (int i = 0; i < 4; ++i)
+        if (b0 + i < B) {
+          float tot = 0.f;
 #pragma unroll
-    for (int b = 0; b < kMaxB; ++b)
-      if (b < B) {
-        float tot = 0.f;
+          for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[b0 + i][q];
+          inv[i] = 1.0f / sqrtf(tot / (float)K + P.eps);
+        }
+    }
+    if (has) {
+      float gf[8];
+      bf16x8_to_f32(graw, gf);
 #pragma unroll
-        for (int q = 0; q < kComputeWarps; ++q) tot += sm.red8[b][q];
-        inv[b] = 1.0f / sqrtf(tot / (float)K + P.eps);
-      }
-  } else {
-    bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the previous activation
-  }
-  if (has) {
-    float gf[8];
-    if (g.kind == 0) bf16x8_to_f32(graw, gf);
+      for (int i = 0; i < 4; ++i)
+        if (b0 + i < B) {
+          const float f[8] = {u[i].x, u[i].y, u[i].z, u[i].w, v[i].x, v[i].y, v[i].z, v[i].w};
+          __align__(16) __nv_bfloat16 o[8];
 #pragma unroll
-    for (int b = 0; b < kMaxB; ++b)
-      if (b < B) {
-        float f[8] = {u[b].x, u[b].y, u[b].z, u[b].w, v[b].x, v[b].y, v[b].z, v[b].w};
-        __align__(16) __nv_bfloat16 o[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(g.kind == 0 ? f[j] * inv[b] * gf[j] : f[j]);
-        *reinterpret_cast<uint4*>(&sm.xa[b * kActPitch + c]) = *reinterpret_cast<const uint4*>(o);
-      }
+          for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(g.kind == 0 ? f[j] * inv[i] * gf[j] : f[j]);
+          *reinterpret_cast<uint4*>(&sm.xa()[(b0 + i) * kActPitch + c]) = *reinterpret_cast<const uint4*>(o);
+        }
+    }
   }
   bar_sync(BAR_COMP, kComputeThreads);  // the activation is complete
 }
@@ -1169,7 +1171,7 @@ __device__ __forceinline__ void gemv_epilogue_ahead(const DevPlan& P, const Smem
 // activation rows as the MMA's n = 8 columns (column n reads row min(n, B -
 // 1)); it waits for that slot alone and releases it (the slot's only reader)
 // as soon as its products are done.  Each warp leaves its rows x 4 partial
-// tile in sm.gred[buf]; after a barrier, thread ct sums the 8 partials of its
+// tile in buffer buf of sm.gred(); after a barrier, thread ct sums the 8 partials of its
 // item (batch row b, row or pair r) and runs the op's epilogue.
 __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                           unsigned char* ws, Control* ctl, const TaskDesc& d, const GemvSpec& g,
@@ -1197,7 +1199,7 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
     const int o = r * pitch + (win * 4 + q) * 16;
     return reinterpret_cast<const uint4*>(slot + (swz ? (o ^ (((o >> 7) & 7) << 4)) : o));
   };
-  const uint4* px = reinterpret_cast<const uint4*>(&sm.xa[min(g8, B - 1) * kActPitch + w * geo.cw]) + q;
+  const uint4* px = reinterpret_cast<const uint4*>(&sm.xa()[min(g8, B - 1) * kActPitch + w * geo.cw]) + q;
   const int nwin = geo.cw >> 5;
   float c0[2][4], c1[2][4];  // row blocks 0 and 1, two accumulators each
 #pragma unroll
@@ -1225,16 +1227,22 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   __syncwarp();
   if (lane == 0) release_share(sm, sw, 1, 0);  // the slot's only reader
   if (trec && lane == 0) trec[TR_MATH] = (uint32_t)global_ns();
-  // partial tile: lane (g8, q < 2) holds rows g8, g8 + 8 (+ 16 for block 1)
-  // at batch columns 2q, 2q + 1
-  float (*red)[32][4] = sm.gred[buf];
-  if (q < 2) {
-    *reinterpret_cast<float2*>(&red[w][g8][2 * q]) = make_float2(c0[0][0] + c0[1][0], c0[0][1] + c0[1][1]);
-    *reinterpret_cast<float2*>(&red[w][g8 + 8][2 * q]) = make_float2(c0[0][2] + c0[1][2], c0[0][3] + c0[1][3]);
-    if (nrb == 2) {
-      *reinterpret_cast<float2*>(&red[w][g8 + 16][2 * q]) = make_float2(c1[0][0] + c1[1][0], c1[0][1] + c1[1][1]);
-      *reinterpret_cast<float2*>(&red[w][g8 + 24][2 * q]) = make_float2(c1[0][2] + c1[1][2], c1[0][3] + c1[1][3]);
+  // partial tile: lane (g8, q) holds rows g8, g8 + 8 (+ 16 for block 1) at
+  // batch columns 2q, 2q + 1; kept as [w][column][32 rows] for the columns
+  // of the batch (column-major, so the epilogue's reads are consecutive)
+  float* red = sm.gred(P.act_bytes) + (size_t)buf * (kComputeWarps * kMaxB * 32);
+  auto put = [&](int row, float x0, float x1) {
+    if (2 * q < B) {
+      float* e = red + ((size_t)w * kMaxB + 2 * q) * 32 + row;
+      e[0] = x0;
+      e[32] = x1;
     }
+  };
+  put(g8, c0[0][0] + c0[1][0], c0[0][1] + c0[1][1]);
+  put(g8 + 8, c0[0][2] + c0[1][2], c0[0][3] + c0[1][3]);
+  if (nrb == 2) {
+    put(g8 + 16, c1[0][0] + c1[1][0], c1[0][1] + c1[1][1]);
+    put(g8 + 24, c1[0][2] + c1[1][2], c1[0][3] + c1[1][3]);
   }
   bar_sync(BAR_COMP, kComputeThreads);
   if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
@@ -1244,10 +1252,10 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   float v0 = 0.f, v1 = 0.f;
   if (mine) {
 #pragma unroll
-    for (int k = 0; k < kComputeWarps; ++k) v0 += red[k][r][b];
+    for (int k = 0; k < kComputeWarps; ++k) v0 += red[(k * kMaxB + b) * 32 + r];
     if (geo.pairs)
 #pragma unroll
-      for (int k = 0; k < kComputeWarps; ++k) v1 += red[k][geo.rows_part + r][b];
+      for (int k = 0; k < kComputeWarps; ++k) v1 += red[(k * kMaxB + b) * 32 + geo.rows_part + r];
   }
   const int H = P.hidden;
   switch (d.op) {
@@ -1432,7 +1440,7 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
   __syncwarp();
   if (lane == 0) release_share(sm, slot, kComputeWarps, w);  // every warp has read its K and V rows
   // the 8 warps' partial outputs, [w][h][64] in the staging buffer
-  float* ob = sm.xs;
+  float* ob = sm.xs();
 #pragma unroll
   for (int h = 0; h < 4; ++h)
     if (h < qpg) *reinterpret_cast<float2*>(ob + (w * 4 + h) * D + 2 * lane) = make_float2(o0[h], o1[h]);
@@ -1554,7 +1562,7 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
         }
     }
   }
-  float* lg = sm.xs;  // [8][64] logits of this task's tokens
+  float* lg = sm.xs();  // [8][64] logits of this task's tokens
   bar_sync(BAR_COMP, kComputeThreads);  // the staging buffer is free (and the FFN inputs are written)
   const uint4* wr = reinterpret_cast<const uint4*>(mw.router);
   const uint4* xr = reinterpret_cast<const uint4*>(dec ? xhat : S.moe_x);
@@ -1632,7 +1640,7 @@ __device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams&
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int E = P.n_experts, K = P.top_k, TMt = P.moe_tm;
   unsigned char* mb = moe_block(P, ws, d.layer);
-  int* sx = reinterpret_cast<int*>(sm.xs);  // exp_indptr [E + 1]
+  int* sx = reinterpret_cast<int*>(sm.xs());  // exp_indptr [E + 1]
   bar_sync(BAR_COMP, kComputeThreads);
   if (w == 0) {
     const int* hist = reinterpret_cast<const int*>(mb + P.off_mhist);
@@ -1775,7 +1783,7 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
   }
   if (ks > 1) {
     // K parts 1.. hand their sums to part 0 (the staging buffer as scratch)
-    float* xch = sm.xs;
+    float* xch = sm.xs();
     bar_sync(BAR_COMP, kComputeThreads);
     // entry e = ((kp - 1) * n_mb + mbk) * 2 + nh < (ks - 1) * n_mb * 2 <= 6, 256 floats each (<= 1536 of 2048)
     if (active && kp > 0) {
@@ -1856,7 +1864,7 @@ __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S
     }
   }
   if (ks > 1) {
-    float* xch = sm.xs;  // entries as in task_egu, 4 floats per lane
+    float* xch = sm.xs();  // entries as in task_egu, 4 floats per lane
     bar_sync(BAR_COMP, kComputeThreads);
     if (active && kp > 0) {
       float* e = xch + ((((kp - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 4;
@@ -2178,7 +2186,7 @@ mk_status dev_query(int* n_sm, int* smem_optin, int* device, std::string& err) {
   return MK_OK;
 }
 
-int smem_fixed_bytes() { return (int)((sizeof(Smem) + 1023) / 1024 * 1024); }
+int smem_fixed_bytes() { return kSmemFixed; }
 
 // The driver's tensor-map encoder, looked up once through the runtime (no
 // link-time dependency on the driver library).
@@ -2263,7 +2271,7 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
   cudaStream_t s = (cudaStream_t)stream;
   std::vector<unsigned char> image = image_in;
   if (!encode_weight_maps(p.dp, image, err)) return MK_ERR_INVALID_ARG;
-  size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + sizeof(Smem);
+  size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + kSmemFixed + p.dp.act_bytes + p.dp.gred_bytes;
   const void* kern = kernel_for(p.dp);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) {
@@ -2353,7 +2361,7 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   }
   cudaStream_t s = (cudaStream_t)stream;
   unsigned char* ws = st.addr;
-  const size_t smem = (size_t)P0.ring_slots * P0.slot_bytes + sizeof(Smem);
+  const size_t smem = (size_t)P0.ring_slots * P0.slot_bytes + kSmemFixed + P0.act_bytes + P0.gred_bytes;
   if (st.owner != p.uid) {
     st.owner = 0;
     e = cudaFuncSetAttribute(kernel_for(P0), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -234,6 +234,17 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
 
 // ---------------------------------------------------------------- build
 
+// Shared-memory split of a CTA (see kSmemFixed): the staging buffer sized for
+// `rows` batch rows, the partial tiles (for the dense GEMV tasks; none for
+// rows = 0), the rest to 16 KB ring slots.
+static void smem_layout(DevPlan& P, int rows, int smem_bytes) {
+  P.gbatch = kMaxBatchRows;
+  P.act_bytes = std::max(8192, (rows * kActPitch * 2 + 127) / 128 * 128);
+  P.gred_bytes = rows > 0 ? 2 * 8 * 32 * P.gbatch * 4 : 0;
+  P.smem_bytes = smem_bytes;
+  P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - P.gred_bytes) / P.slot_bytes);
+}
+
 // MoE FFN layer ("Event Tensor: A Unified Abstraction for Compiling Dynamic
 // Megakernel", section "Core method", data-dependent dynamism).  The task
 // graph: ROUTE (8 tokens each) -> follow-up MINDPTR (exp_indptr, tile table,
@@ -273,9 +284,7 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   P.max_tiles = ceil_div(TM * K, P.moe_tm) + std::min(E, TM * K);
   if (FF % P.moe_tn) { err = "expert_ffn must be a multiple of 16"; return MK_ERR_UNSUPPORTED; }
   P.slot_bytes = 16384;
-  const int reserve = kSmemReserve;
-  P.smem_bytes = smem_bytes;
-  P.ring_slots = std::min(16, (smem_bytes - reserve) / P.slot_bytes);
+  smem_layout(P, 0, smem_bytes);
   if (P.ring_slots < 5) { err = "not enough shared memory for a 5-slot ring"; return MK_ERR_UNSUPPORTED; }
 
   p.code.clear();
@@ -367,7 +376,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (Hq * D != H) { err = "n_q_heads * head_dim must equal hidden"; return MK_ERR_UNSUPPORTED; }
   if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
   if (!mdec && (F % 256 || F < 256)) { err = "ffn must be a positive multiple of 256"; return MK_ERR_UNSUPPORTED; }
-  if (m->max_batch < 1 || m->max_batch > 4) { err = "max_batch must be in [1, 4] for this build"; return MK_ERR_UNSUPPORTED; }
+  if (m->max_batch < 1 || m->max_batch > kMaxBatchRows) { err = "max_batch must be in [1, 8] for this build"; return MK_ERR_UNSUPPORTED; }
   if (m->max_ctx < 2 || m->n_slots < m->max_batch) { err = "max_ctx >= 2 and n_slots >= max_batch required"; return MK_ERR_INVALID_ARG; }
   if (o->sched != MK_SCHED_STATIC && o->sched != MK_SCHED_DYNAMIC) { err = "unknown schedule"; return MK_ERR_INVALID_ARG; }
   if (n_sm < 1 || n_sm > 1024) { err = "n_sm out of range"; return MK_ERR_INVALID_ARG; }
@@ -424,9 +433,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.max_chunks = ceil_div(P.max_ctx, P.chunk);
 
   // shared memory: ring of 16 KB slots plus a fixed control area
-  const int reserve = kSmemReserve;  // fixed shared-memory area of the kernel
-  P.smem_bytes = smem_bytes;
-  P.ring_slots = std::min(16, (smem_bytes - reserve) / P.slot_bytes);
+  smem_layout(P, P.max_batch, smem_bytes);
   if (P.ring_slots < 3) { err = "not enough shared memory for a 3-slot ring"; return MK_ERR_UNSUPPORTED; }
 
   // ---- expressions and families

@@ -184,7 +184,15 @@ struct LayerPtrs {
 };
 
 constexpr int kMaxFamilies = 256;
-constexpr int kSmemReserve = 33 * 1024;  // the kernel's fixed shared-memory area; the ring takes the rest
+// Dynamic shared memory of a CTA: the ring (ring_slots x slot_bytes), the
+// kernel's fixed control area (at most kSmemFixed bytes), the staging buffer
+// (act_bytes: the GEMV activation rows in bf16, kActPitch elements per batch
+// row, or 8 KB of fp32 scratch for the other task bodies) and the GEMV
+// partial tiles (gred_bytes: two buffers of 8 warps x gbatch = 8 columns x 32
+// rows of fp32).
+constexpr int kSmemFixed = 9 * 1024;
+constexpr int kActPitch = 2048 + 8;  // bf16 elements per staged activation row (16-byte bank offset per row)
+constexpr int kMaxBatchRows = 8;     // batch rows of a dense step (the GEMV's MMA n = 8 columns)
 // A GEMV task's weights arrive in kGemvSlots ring slots, slot j holding columns
 // [j K / 8, (j + 1) K / 8) of all the task's rows (one 2-D TMA box per part),
 // through one tensor map per dense weight matrix: matrix m of layer l at
@@ -205,6 +213,7 @@ struct DevPlan {
   int32_t tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, chunk;
   int32_t n_qkv_tiles, n_otiles, n_gutiles, n_dtiles, n_kc, n_lm_tiles, max_chunks;
   int32_t ring_slots, slot_bytes, smem_bytes;
+  int32_t act_bytes, gred_bytes, gbatch, pad3;  // shared-memory staging buffer and partial tiles
   int32_t n_counters, debug_slots, queue_ranges;
   uint32_t debug_flags;
   int32_t pad0;

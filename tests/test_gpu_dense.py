@@ -153,7 +153,7 @@ def test_llama1b_greedy_32_static_vs_dynamic(llama):
 
 def test_llama1b_long_ragged_contexts():
     # the symbolic-batch workload's context range: three sequences at 128,
-    # 2100 and 4095 cached tokens in one step (33 to 65 key chunks each)
+    # 2100 and 4095 cached tokens in one step (3 to 65 key chunks each)
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     ctx = [128, 2100, 4095]
@@ -165,3 +165,38 @@ def test_llama1b_long_ragged_contexts():
         assert rel_err(got["logits"][b], ref["logits"][b]) <= TOL
         check_argmax(got["next_tokens"][b], ref["logits"][b])
     case.check_task_set(got["task_counts"], 3, ctx)
+
+
+@pytest.mark.parametrize("sched", [mk.MK_SCHED_STATIC, mk.MK_SCHED_DYNAMIC])
+def test_tiny_batch_of_eight(sched):
+    # B up to 8: every column of the GEMV's MMA n = 8 carries a batch row;
+    # one plan steps B = 8, 5 and 1 with ragged contexts
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    fill = [64, 0, 70, 190, 5, 127, 128, 300]
+    case = DenseCase(wl.TINY, max_batch=8, max_ctx=320, n_slots=8, ctx_fill=fill, sched=sched)
+    K, V = case.K_cpu.clone(), case.V_cpu.clone()
+    tok = wl.token_ids(8, wl.TINY.vocab).tolist()
+    for tokens, slots, ctx in [(tok, list(range(8)), fill),
+                               (tok[:5], [7, 1, 3, 0, 5], [301, 1, 191, 65, 128]),
+                               (tok[:1], [6], [129])]:
+        ref = case.oracle.step(K, V, tokens, slots, ctx)
+        got = case.gpu_step(tokens, slots, ctx)
+        for b in range(len(tokens)):
+            assert rel_err(got["logits"][b], ref["logits"][b]) <= TOL
+            check_argmax(got["next_tokens"][b], ref["logits"][b])
+        case.check_task_set(got["task_counts"], len(tokens), ctx)
+
+
+def test_llama1b_batch_of_eight():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    ctx = [128, 700, 1500, 2100, 64, 0, 999, 4095]
+    case = DenseCase(wl.LLAMA_1B, max_batch=8, max_ctx=4104, n_slots=8, ctx_fill=ctx)
+    tokens = wl.token_ids(8, wl.LLAMA_1B.vocab).tolist()
+    ref, _, _ = _oracle_step(case, tokens, list(range(8)), ctx)
+    got = case.gpu_step(tokens, list(range(8)), ctx)
+    for b in range(8):
+        assert rel_err(got["logits"][b], ref["logits"][b]) <= TOL
+        check_argmax(got["next_tokens"][b], ref["logits"][b])
+    case.check_task_set(got["task_counts"], 8, ctx)
