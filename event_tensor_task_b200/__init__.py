@@ -75,6 +75,13 @@ def mk_moe_layer(plan: int, args: mk_moe_args, stream: int = 0):
     _check(lib().mk_moe_layer(plan, C.byref(args), stream))
 
 
+def mk_get_stats(plan: int) -> dict:
+    """Plan and runtime counters (mk_get_stats) as a dict."""
+    st = _abi.mk_stats()
+    _check(lib().mk_get_stats(plan, C.byref(st)))
+    return {name: getattr(st, name) for name, _ in st._fields_}
+
+
 def mk_get_status(plan: int):
     st = mk_device_status()
     code = lib().mk_get_status(plan, C.byref(st))
@@ -220,6 +227,9 @@ class DenseDecoder:
 
     def status(self):
         return mk_get_status(self.plan)
+
+    def stats(self):
+        return mk_get_stats(self.plan)
 
     def reset(self):
         import torch

@@ -89,6 +89,13 @@ class mk_device_status(C.Structure):
     _fields_ = [("code", C.c_int), ("family", C.c_int), ("index", C.c_int), ("event", C.c_int), ("sm", C.c_int)]
 
 
+class mk_stats(C.Structure):
+    _fields_ = [("launches", C.c_longlong), ("build_ms", C.c_double), ("n_families", C.c_int),
+                ("n_counters", C.c_int), ("ring_slots", C.c_int), ("n_sm", C.c_int),
+                ("workspace_bytes", C.c_longlong), ("queue_ranges_cap", C.c_int), ("last_queue_ranges", C.c_int),
+                ("last_queue_tasks", C.c_longlong), ("last_queue_pops", C.c_longlong)]
+
+
 class mk_family_info(C.Structure):
     _fields_ = [("op", C.c_int), ("layer", C.c_int), ("debug_base", C.c_int), ("max_extent", C.c_int),
                 ("followup", C.c_int), ("name", C.c_char * 16)]
@@ -110,6 +117,7 @@ PROTOTYPES = {
     "mk_decode_step_static": (C.c_int, [C.c_void_p, C.POINTER(mk_step_args), C.c_void_p]),
     "mk_moe_layer": (C.c_int, [C.c_void_p, C.POINTER(mk_moe_args), C.c_void_p]),
     "mk_get_status": (C.c_int, [C.c_void_p, C.POINTER(mk_device_status)]),
+    "mk_get_stats": (C.c_int, [C.c_void_p, C.POINTER(mk_stats)]),
     "mk_plan_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
     "mk_plan_task_slots": (C.c_int, [C.c_void_p]),
     "mk_plan_num_families": (C.c_int, [C.c_void_p]),

@@ -1,7 +1,10 @@
 // api.cpp — the extern "C" boundary of libmk.so (declared in include/mk.h).
 // No exception crosses it; every failure returns an mk_status and leaves a
 // message for mk_last_error().
+#include <cuda_runtime.h>
+
 #include <atomic>
+#include <chrono>
 #include <cstring>
 #include <new>
 #include <string>
@@ -36,6 +39,7 @@ const char* mk_last_error(void) { return g_err.c_str(); }
 
 mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_plan** out) {
   g_err.clear();
+  const auto t_build0 = std::chrono::steady_clock::now();
   if (!m || !opts || !out) return fail(MK_ERR_INVALID_ARG, "null argument");
   *out = nullptr;
   try {
@@ -67,6 +71,7 @@ mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_pla
     static std::atomic<unsigned long long> next_uid{1};
     hp->p.device = device;
     hp->p.uid = next_uid++;
+    hp->p.build_ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t_build0).count();
     *out = hp;
     return MK_OK;
   } catch (const std::bad_alloc&) {
@@ -144,6 +149,32 @@ mk_status mk_moe_layer(mk_plan* hp, const mk_moe_args* a, void* stream) {
   std::string err;
   mk_status s = mk::dev_launch_moe(hp->p, a, stream, err);
   return s == MK_OK ? MK_OK : fail(s, err);
+}
+
+mk_status mk_get_stats(mk_plan* hp, mk_stats* st) {
+  g_err.clear();
+  if (!hp || !st) return fail(MK_ERR_INVALID_ARG, "null argument");
+  const mk::DevPlan& P = hp->p.dp;
+  st->launches = hp->p.launches;
+  st->build_ms = hp->p.build_ms;
+  st->n_families = P.n_families;
+  st->n_counters = P.n_counters;
+  st->ring_slots = P.ring_slots;
+  st->n_sm = P.n_sm;
+  st->workspace_bytes = P.ws_bytes;
+  st->queue_ranges_cap = P.sched == MK_SCHED_DYNAMIC ? P.queue_ranges : 0;
+  st->last_queue_ranges = -1;
+  st->last_queue_tasks = -1;
+  st->last_queue_pops = -1;
+  if (hp->p.ws && hp->p.launches > 0 && P.sched == MK_SCHED_DYNAMIC) {
+    mk::Control c;
+    cudaError_t e = cudaMemcpy(&c, (unsigned char*)hp->p.ws + P.off_control, sizeof(c), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(MK_ERR_CUDA, std::string("control block read failed: ") + cudaGetErrorString(e));
+    st->last_queue_ranges = (int)(c.q_tail >> 40);
+    st->last_queue_tasks = (long long)(c.q_tail & ((1ull << 40) - 1));
+    st->last_queue_pops = (long long)c.q_head;
+  }
+  return MK_OK;
 }
 
 mk_status mk_get_status(mk_plan* hp, mk_device_status* st) {

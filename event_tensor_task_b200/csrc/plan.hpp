@@ -60,6 +60,7 @@ struct Plan {
   size_t ws_bound = 0;
   unsigned epoch = 0;
   long long launches = 0;
+  double build_ms = 0.0;             // host time of mk_plan_build
 
   // host model of the task graph
   int fam_index(int op, int layer) const;

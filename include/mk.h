@@ -95,7 +95,7 @@ typedef struct mk_model_desc {
   int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
   float eps;              /* RMSNorm epsilon */
   float rope_theta;       /* rotary base; pair i of a head turns by pos*theta^(-2i/head_dim) */
-  int max_batch;          /* largest B a step may use */
+  int max_batch;          /* largest B a step may use (at most 8 for the dense and MoE decoder kinds) */
   int max_ctx;            /* cache capacity in positions (ctx_lens[b] < max_ctx) */
   int n_slots;            /* sequences the KV cache holds */
   const void* embed;      /* [vocab][hidden] bf16, device */
@@ -272,6 +272,29 @@ mk_status mk_moe_layer(mk_plan* p, const mk_moe_args* a, void* stream);
 /* Read the device status word (synchronous copy).  Returns the recorded
  * device code (MK_OK if none).  After a device error, call mk_plan_reset. */
 mk_status mk_get_status(mk_plan* p, mk_device_status* st);
+
+/* Plan and runtime counters.  The last_* fields describe the last launch
+ * through mk_decode_step / mk_moe_layer and are read from the device control
+ * block with a synchronous copy (call after the stream has synchronised);
+ * they are -1 when no workspace is bound, nothing has launched yet, or the
+ * plan runs the static schedule. */
+typedef struct mk_stats {
+  long long launches;          /* kernel launches through this plan, every entry point */
+  double build_ms;             /* host time mk_plan_build took */
+  int n_families;              /* task families of the plan */
+  int n_counters;              /* Event Tensor counters (sum of all event tensors' sizes) */
+  int ring_slots;              /* shared-memory ring slots per CTA */
+  int n_sm;                    /* CTAs of the persistent kernel */
+  long long workspace_bytes;   /* mk_plan_workspace_bytes */
+  int queue_ranges_cap;        /* dynamic queue capacity in task ranges (0: static schedule) */
+  int last_queue_ranges;       /* ranges pushed during the last launch */
+  long long last_queue_tasks;  /* tasks pushed during the last launch (one END per CTA included) */
+  long long last_queue_pops;   /* queue pops during the last launch */
+} mk_stats;
+
+/* Fill *st.  MK_ERR_INVALID_ARG for null arguments, MK_ERR_CUDA if the
+ * control-block copy fails. */
+mk_status mk_get_stats(mk_plan* p, mk_stats* st);
 
 /* Clear the device control block (status, barrier and queue counters) and the
  * dynamic queue's entries. */

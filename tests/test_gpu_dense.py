@@ -10,6 +10,7 @@ import torch
 import event_tensor_task_b200 as mk
 import workloads as wl
 from gpu_common import DenseCase, rel_err, check_argmax, TOL
+from oracle import tasks as ot
 
 pytestmark = pytest.mark.gpu
 
@@ -69,6 +70,14 @@ def test_tiny_static_equals_dynamic_bitwise(tiny):
     assert torch.equal(a["logits"], b["logits"])
     assert torch.equal(a["next_tokens"], b["next_tokens"])
     dyn.check_task_set(b["task_counts"], 3, ctx)
+    # the dynamic queue of that launch: every task except the follow-ups
+    # (MERGE, LMFIN run where their event fired) was pushed once, plus one
+    # END per CTA, and every push was popped
+    want = ot.expected_dense_tasks(wl.TINY, 3, ctx, dyn.tiles_for_oracle())
+    st = dyn.dec.stats()
+    pushed = sum(1 for f, _, _ in want if f not in ("merge", "lmfin")) + st["n_sm"]
+    assert st["last_queue_tasks"] == pushed and st["last_queue_pops"] == pushed
+    assert 0 < st["last_queue_ranges"] <= st["queue_ranges_cap"] and st["launches"] == 1
 
 
 def test_tiny_dynamic_steps_after_reset(tiny):

@@ -171,3 +171,16 @@ def test_moe_plan_requires_dynamic_schedule_and_rejects_dense_calls():
     with pytest.raises(mk.MkError):
         mk.mk_decode_step(plan, a, 0)
     mk.mk_plan_destroy(plan)
+
+
+def test_stats_without_a_device():
+    # mk_get_stats on a host-only plan: the plan's figures, no launch yet
+    d = _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148)
+    st = d.stats()
+    assert st["launches"] == 0 and st["build_ms"] > 0.0
+    assert st["n_families"] == len(d.families()) and st["n_sm"] == 148
+    assert st["ring_slots"] == d.tiles()["ring_slots"]
+    assert st["workspace_bytes"] == mk.mk_plan_workspace_bytes(d.plan)
+    assert st["queue_ranges_cap"] == 0  # static schedule
+    assert st["last_queue_tasks"] == -1 and st["last_queue_pops"] == -1
+    d.close()
