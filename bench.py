@@ -486,6 +486,25 @@ def cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, n_steps):
     return n_steps / dt, torch.get_num_threads(), dt
 
 
+def max_over_ranks(x, device):
+    """Max of x over the ranks of the default process group (x itself when no
+    group is initialised): the timed region of a multi-GPU run is the slowest
+    rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, items_per_rank, max_ms):
+    """Items per second over all ranks (replicas: every rank does the same
+    work) for a timed region of max_ms, the max over ranks."""
+    return world * items_per_rank / (max_ms / 1000.0)
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
@@ -592,13 +611,9 @@ def main():
     code, st = dec.status()
     if code != 0:
         raise SystemExit(f"device status {code} in the timed region")
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     ms_step = ms / args.steps
-    tokens = world * 1 * args.steps
-    value = tokens / (ms / 1000.0)
+    value = whole_job_rate(world, 1 * args.steps, ms)
 
     # algorithmic bytes per launch (mean over the context window)
     step_bytes = statistics.mean(mk.mk_plan_step_bytes(dec.plan, 1, [CTX0 + (i % WINDOW)])
@@ -633,12 +648,8 @@ def main():
     e2e_steps(n_e2e, args.warmup)
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e_value = world * n_e2e / (e_ms / 1000.0)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = whole_job_rate(world, n_e2e, e_ms)
 
     baselines = None
     if world == 1 and not args.no_torch_baseline:
