@@ -71,6 +71,18 @@ def test_tiny_moe_decoder_continuous_batching():
                  ([9, 10], [2, 0], [132, 66])])
 
 
+def test_tiny_moe_decoder_batch_of_eight():
+    # B up to 8: the MoE FFN on 8 tokens (ROUTE in one task, ragged per-expert
+    # rows) after attention over eight ragged contexts
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    mshape = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
+    fill = [64, 10, 130, 200, 0, 77, 250, 5]
+    case = MoeCase(wl.TINY, mshape, max_batch=8, max_ctx=320, ctx_fill=fill)
+    _walk(case, [(list(range(11, 19)), list(range(8)), fill),
+                 ([19, 20, 21, 22, 23], [7, 0, 4, 2, 5], [6, 65, 1, 131, 78])])
+
+
 def test_moe_decoder_1b_attention_64_experts():
     # two layers of the 1B attention shape, each FFN the 64-expert top-8 layer
     if not torch.cuda.is_available():
