@@ -34,6 +34,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstddef>
 #include <cstring>
 #include <mutex>
@@ -318,7 +319,10 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsi
 __device__ __forceinline__ int task_slots(const DevPlan& P, const ProdFam& f, int idx) {
   if (f.op == OP_ATTN) return 1;
   if (f.op == OP_ROUTE || f.op == OP_COMBINE || f.op == OP_MINDPTR || f.op == OP_MFIN) return 0;
-  if (f.op == OP_QKV || f.op == OP_OPROJ || f.op == OP_GATEUP || f.op == OP_DOWN || f.op == OP_LM) return kGemvSlots;
+  if (f.op == OP_QKV || f.op == OP_OPROJ) return kGemvSlots;
+  if (f.op == OP_GATEUP) return P.tile_gu > 16 ? 2 * kGemvSlots : kGemvSlots;
+  if (f.op == OP_DOWN) return P.tile_down > 32 ? 2 * kGemvSlots : kGemvSlots;
+  if (f.op == OP_LM) return P.tile_lm > 32 ? 2 * kGemvSlots : kGemvSlots;
   return f.parts * f.slots_per_part;
 }
 
@@ -421,19 +425,27 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
           return false;
         break;
       case OP_GATEUP:
-        if (!stream_tiles(fam, idx, P.tile_gu, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_gu, f.tm[1],
-                          idx * P.tile_gu))
-          return false;
+        if (P.tile_gu <= 16) {  // one half: 16 gate + 16 up rows per slot
+          if (!stream_tiles(fam, idx, P.tile_gu, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_gu, f.tm[1],
+                            idx * P.tile_gu))
+            return false;
+        } else {  // two halves of 8 slots: the gate rows, then the up rows
+          if (!stream_tiles(fam, idx, P.tile_gu, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_gu, nullptr, 0) ||
+              !stream_tiles(fam, idx, P.tile_gu, P.hidden / kGemvSlots, 0, f.tm[1], idx * P.tile_gu, nullptr, 0))
+            return false;
+        }
         break;
       case OP_DOWN: {
         const int kc = idx / P.n_dtiles, n = idx - kc * P.n_dtiles;
-        if (!stream_tiles(fam, idx, P.tile_down, P.kseg / kGemvSlots, kc * P.kseg, f.tm[0], n * P.tile_down, nullptr,
-                          0))
-          return false;
+        for (int r0 = 0; r0 < P.tile_down; r0 += 32)  // halves of at most 32 rows
+          if (!stream_tiles(fam, idx, min(32, P.tile_down), P.kseg / kGemvSlots, kc * P.kseg, f.tm[0],
+                            n * P.tile_down + r0, nullptr, 0))
+            return false;
       } break;
       case OP_LM:  // the last tile's rows past the vocabulary read as zeros
-        if (!stream_tiles(fam, idx, P.tile_lm, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_lm, nullptr, 0))
-          return false;
+        for (int r0 = 0; r0 < P.tile_lm; r0 += 32)
+          if (!stream_tiles(fam, idx, 32, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_lm + r0, nullptr, 0))
+            return false;
         break;
       case OP_EGU: {
         // tile -> expert from the table the routing follow-up wrote (visible:
@@ -1121,15 +1133,14 @@ __device__ __forceinline__ void mma_window(float (&c)[4], const uint4& ua, const
   mma_16816(c, ua.z, ub.z, ua.w, ub.w, wb.z, wb.w);
 }
 
-// Epilogue item of thread ct in a GEMV task: batch row b and row (pair ops:
-// pair) r of the task; items are B x RI with RI the rows (pairs) of the task.
+// Epilogue item i of a GEMV task: batch row b and row (pair ops: pair) r of
+// the task; items are B x RI with RI the rows (pairs) of the task.
 struct GemvItem { int b, r; bool on; };
-__device__ __forceinline__ GemvItem gemv_item(const OpGeo& geo, int B) {
-  const int ct = threadIdx.x - kComputeBase;
+__device__ __forceinline__ GemvItem gemv_item(const OpGeo& geo, int B, int i) {
   const int RI = geo.rows_part;
   GemvItem it;
-  it.b = ct / RI;
-  it.r = ct - it.b * RI;
+  it.b = i / RI;
+  it.r = i - it.b * RI;
   it.on = it.b < B;
   return it;
 }
@@ -1165,174 +1176,200 @@ __device__ __forceinline__ void gemv_epilogue_ahead(const DevPlan& P, const Smem
 }
 
 // A GEMV task on tensor cores: Y[rows x B] = W[rows x K] . A[B x K]^T, W
-// the task's (at most 32) rows in its kGemvSlots ring slots (bf16, by column
-// slice), A the staged activation rows.  Warp w reads only slot w: every row
-// block (16 rows) of the task over columns [w cw, (w + 1) cw), with the
-// activation rows as the MMA's n = 8 columns (column n reads row min(n, B -
-// 1)); it waits for that slot alone and releases it (the slot's only reader)
-// as soon as its products are done.  Each warp leaves its rows x 4 partial
-// tile in buffer buf of sm.gred(); after a barrier, thread ct sums the 8 partials of its
-// item (batch row b, row or pair r) and runs the op's epilogue.
+// the task's rows (16, 32 or 64) in its ring slots (bf16, by column slice),
+// A the staged activation rows.  The rows arrive in halves of at most 32 rows
+// and 8 slots each (pair ops with 32 + 32 rows: the part-0 half, then the
+// part-1 half); product warp w reads slot w of each half: every 16-row block
+// of the half over columns [w cw, (w + 1) cw), with the activation rows as
+// the MMA's n = 8 columns (column n reads row min(n, B - 1)).  It waits for
+// that slot alone and releases it (its only reader) as soon as its products
+// are done.  Each warp leaves its partial tile in sm.gred() ([w][column][64
+// rows]); after a barrier, the threads sum the 8 partials of their items
+// (batch row b, row or pair r; 256 items at a time) and run the op's
+// epilogue; a last barrier frees the partial tiles for the next task.
 __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                           unsigned char* ws, Control* ctl, const TaskDesc& d, const GemvSpec& g,
-                                          int B, int buf, const EpiAhead& ea, const GemvItem& it, uint32_t* trec) {
+                                          int B, const EpiAhead& ea0, uint32_t* trec) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const OpGeo geo = sm.geo[d.op];
   const int R = P.ring_slots;
   const int s0 = d.slot_ph & 0xffff;
   const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int sw = s0 + w < R ? s0 + w : s0 + w - R;  // this warp's slot
-  wait_mbar(&sm.full[sw], s0 + w < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  if (trec && lane == 0) {
-    trec[TR_DATA] = (uint32_t)global_ns();
-    trec[TR_ISSUE] = sm.slot_t[s0];
-  }
-  const int nrb = (geo.pairs ? 2 : 1) * geo.rows_part >> 4;  // row blocks: 1 or 2
+  const int rows_total = (geo.pairs ? 2 : 1) * geo.rows_part;
+  const int nh = rows_total > 32 ? 2 : 1;        // halves of 8 slots
+  const int nrb = (rows_total > 32 ? 32 : rows_total) >> 4;  // 16-row blocks per half: 1 or 2
   const int g8 = lane >> 2, q = lane & 3;
-  const int pitch = geo.cw * 2;  // bytes per row in the slot
-  const unsigned char* slot = ring + (size_t)sw * P.slot_bytes;
+  const int pitch = geo.cw * 2;  // bytes per row in a slot
   // 16-byte chunk (window win, lane chunk q) of slot row r: with cw >= 64 the
   // rows are 128-byte lines under the 128-byte swizzle (chunk c of line n at
   // c ^ (n & 7)), which puts the 8 rows a quarter-warp reads on distinct banks
   const bool swz = geo.cw >= 64;
-  auto chunk = [&](int r, int win) -> const uint4* {
-    const int o = r * pitch + (win * 4 + q) * 16;
-    return reinterpret_cast<const uint4*>(slot + (swz ? (o ^ (((o >> 7) & 7) << 4)) : o));
-  };
   const uint4* px = reinterpret_cast<const uint4*>(&sm.xa()[min(g8, B - 1) * kActPitch + w * geo.cw]) + q;
   const int nwin = geo.cw >> 5;
-  float c0[2][4], c1[2][4];  // row blocks 0 and 1, two accumulators each
-#pragma unroll
-  for (int u = 0; u < 2; ++u)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) c0[u][i] = c1[u][i] = 0.f;
-  // windows in pairs, alternating accumulators (16-byte chunks: 4 per window)
-  if (nrb == 2) {
-    for (int win = 0; win < nwin; win += 2) {
-      const uint4 xb = px[win * 4];
-      mma_window(c0[0], *chunk(g8, win), *chunk(g8 + 8, win), xb);
-      mma_window(c1[0], *chunk(g8 + 16, win), *chunk(g8 + 24, win), xb);
-      if (win + 1 < nwin) {
-        const uint4 xb1 = px[win * 4 + 4];
-        mma_window(c0[1], *chunk(g8, win + 1), *chunk(g8 + 8, win + 1), xb1);
-        mma_window(c1[1], *chunk(g8 + 16, win + 1), *chunk(g8 + 24, win + 1), xb1);
-      }
-    }
-  } else {
-    for (int win = 0; win < nwin; win += 2) {
-      mma_window(c0[0], *chunk(g8, win), *chunk(g8 + 8, win), px[win * 4]);
-      if (win + 1 < nwin) mma_window(c0[1], *chunk(g8, win + 1), *chunk(g8 + 8, win + 1), px[win * 4 + 4]);
-    }
-  }
-  __syncwarp();
-  if (lane == 0) release_share(sm, sw, 1, 0);  // the slot's only reader
-  if (trec && lane == 0) trec[TR_MATH] = (uint32_t)global_ns();
-  // partial tile: lane (g8, q) holds rows g8, g8 + 8 (+ 16 for block 1) at
-  // batch columns 2q, 2q + 1; kept as [w][column][32 rows] for the columns
-  // of the batch (column-major, so the epilogue's reads are consecutive)
-  float* red = sm.gred(P.act_bytes) + (size_t)buf * (kComputeWarps * kMaxB * 32);
-  auto put = [&](int row, float x0, float x1) {
+  float* red = sm.gred(P.act_bytes);
+  auto put = [&](int row, float x0, float x1) {  // partial tile: [w][column][64 rows]
     if (2 * q < B) {
-      float* e = red + ((size_t)w * kMaxB + 2 * q) * 32 + row;
+      float* e = red + ((size_t)w * kMaxB + 2 * q) * 64 + row;
       e[0] = x0;
-      e[32] = x1;
+      e[64] = x1;
     }
   };
-  put(g8, c0[0][0] + c0[1][0], c0[0][1] + c0[1][1]);
-  put(g8 + 8, c0[0][2] + c0[1][2], c0[0][3] + c0[1][3]);
-  if (nrb == 2) {
-    put(g8 + 16, c1[0][0] + c1[1][0], c1[0][1] + c1[1][1]);
-    put(g8 + 24, c1[0][2] + c1[1][2], c1[0][3] + c1[1][3]);
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
-  // epilogue: item (b, r); v0 = row r (pair ops: part 0 row r), v1 = part 1 row r
-  const int b = it.b, r = it.r;
-  const bool mine = it.on && (geo.pairs || d.op != OP_LM || d.idx * P.tile_lm + r < P.vocab);
-  float v0 = 0.f, v1 = 0.f;
-  if (mine) {
+  for (int h = 0; h < nh; ++h) {
+    const int j = kGemvSlots * h + w;  // this warp's slot of the task
+    const int wrap = (s0 + j) / R;
+    const int sw = s0 + j - wrap * R;
+    if (j >= R) {
+      // The ring position also held slot j - R of this task.  A parity wait
+      // on the full barrier cannot tell that use's phase from this one's, so
+      // first wait until slot j - R has been released (the empty barrier's
+      // phase for that use: it cannot move on before this warp releases slot
+      // j); the full barrier is then at most one phase behind slot j.
+      const int wrap_prev = (s0 + j - R) / R;
+      wait_mbar(&sm.empty[sw], p0 ^ ((uint32_t)wrap_prev & 1u), ctl, P.spin_timeout_ns, d.fam, d.idx);
+    }
+    wait_mbar(&sm.full[sw], p0 ^ ((uint32_t)wrap & 1u), ctl, P.spin_timeout_ns, d.fam, d.idx);
+    if (trec && lane == 0 && h == 0) {
+      trec[TR_DATA] = (uint32_t)global_ns();
+      trec[TR_ISSUE] = sm.slot_t[s0];
+    }
+    const unsigned char* slot = ring + (size_t)sw * P.slot_bytes;
+    auto chunk = [&](int r, int win) -> const uint4* {
+      const int o = r * pitch + (win * 4 + q) * 16;
+      return reinterpret_cast<const uint4*>(slot + (swz ? (o ^ (((o >> 7) & 7) << 4)) : o));
+    };
+    float c0[2][4], c1[2][4];  // row blocks 0 and 1, two accumulators each
 #pragma unroll
-    for (int k = 0; k < kComputeWarps; ++k) v0 += red[(k * kMaxB + b) * 32 + r];
-    if (geo.pairs)
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int k = 0; k < kComputeWarps; ++k) v1 += red[(k * kMaxB + b) * 32 + geo.rows_part + r];
-  }
-  const int H = P.hidden;
-  switch (d.op) {
-    case OP_QKV: {
-      // RoPE on q and k (rotate-half pairs j, j + D/2), then q -> buffer, k/v -> cache
-      if (!mine) break;
-      QkvTile qt = decode_qkv(P, d.idx);
-      const int pos = sm.ctx[b];
-      const int j = qt.j0 + r;
-      if (qt.kind == 2) {
-        size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + qt.head) * P.max_ctx + pos;
-        __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * P.head_dim;
-        vc[j] = __float2bfloat16_rn(v0);
-        vc[j + 32] = __float2bfloat16_rn(v1);
-      } else {
-        const float cs = ea.a[0], sn = ea.a[1];  // (cos, sin) of (pos, j), loaded before the products
-        const float x0 = v0 * cs - v1 * sn, x1 = v1 * cs + v0 * sn;
-        if (qt.kind == 0) {
-          float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * P.head_dim +
-                      qt.head * P.head_dim;
-          qb[j] = x0;
-          qb[j + 32] = x1;
-        } else {
-          size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + qt.head) * P.max_ctx + pos;
-          __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * P.head_dim;
-          kc[j] = __float2bfloat16_rn(x0);
-          kc[j + 32] = __float2bfloat16_rn(x1);
+      for (int i = 0; i < 4; ++i) c0[u][i] = c1[u][i] = 0.f;
+    // windows in pairs, alternating accumulators (16-byte chunks: 4 per window)
+    if (nrb == 2) {
+      for (int win = 0; win < nwin; win += 2) {
+        const uint4 xb = px[win * 4];
+        mma_window(c0[0], *chunk(g8, win), *chunk(g8 + 8, win), xb);
+        mma_window(c1[0], *chunk(g8 + 16, win), *chunk(g8 + 24, win), xb);
+        if (win + 1 < nwin) {
+          const uint4 xb1 = px[win * 4 + 4];
+          mma_window(c0[1], *chunk(g8, win + 1), *chunk(g8 + 8, win + 1), xb1);
+          mma_window(c1[1], *chunk(g8 + 16, win + 1), *chunk(g8 + 24, win + 1), xb1);
         }
       }
-    } break;
-    case OP_OPROJ: {
-      // residual: x = (x + previous layer's down partials) + o W_o^T
-      if (!mine) break;
-      const size_t col = (size_t)d.idx * P.tile_o + r;
-      float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
-      float acc = ea.a[0];
-      if (d.layer > 0 && P.kind == MK_MODEL_DENSE) {
-        acc += (ea.a[1] + ea.a[2]) + (ea.a[3] + ea.a[4]);
-        const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H + col;
-        for (int kc = 4; kc < P.n_kc; ++kc) acc += __ldcg(dp + (size_t)kc * P.max_batch * H);
+    } else {
+      for (int win = 0; win < nwin; win += 2) {
+        mma_window(c0[0], *chunk(g8, win), *chunk(g8 + 8, win), px[win * 4]);
+        if (win + 1 < nwin) mma_window(c0[1], *chunk(g8, win + 1), *chunk(g8 + 8, win + 1), px[win * 4 + 4]);
       }
-      x[col] = acc + v0;
-    } break;
-    case OP_GATEUP: {
-      if (!mine) break;
-      float* h = reinterpret_cast<float*>(ws + P.off_h) + (size_t)b * P.ffn + (size_t)d.idx * P.tile_gu + r;
-      *h = v0 / (1.0f + expf(-v0)) * v1;
-    } break;
-    case OP_DOWN: {
-      if (!mine) break;
-      const int nt = d.idx - g.kc * P.n_dtiles;
-      float* dpart = reinterpret_cast<float*>(ws + P.off_dpart) + ((size_t)g.kc * P.max_batch + b) * H +
-                     (size_t)nt * P.tile_down + r;
-      *dpart = v0;
-    } break;
-    case OP_LM: {
-      // logits, then the warp's best (logit, id) key (the warp's items share
-      // one batch row); published with an atomic max only when it beats what
-      // this warp published before (order independent)
-      const int row = d.idx * P.tile_lm + r;
-      unsigned long long key = 0ull;
-      if (mine) {
-        if (S.logits) S.logits[(size_t)b * P.vocab + row] = v0;
-        key = argmax_key(v0, row);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
-        key = other > key ? other : key;
-      }
-      if (lane == 0 && it.on && key > sm.lm_seen[w][b]) {
-        sm.lm_seen[w][b] = key;
-        atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, key);
-      }
-    } break;
-    default: break;
+    }
+    __syncwarp();
+    if (lane == 0) release_share(sm, sw, 1, 0);  // the slot's only reader
+    // lane (g8, q) holds rows g8, g8 + 8 (+ 16 for block 1) of the half at
+    // batch columns 2q, 2q + 1
+    const int rh = 32 * h;
+    put(rh + g8, c0[0][0] + c0[1][0], c0[0][1] + c0[1][1]);
+    put(rh + g8 + 8, c0[0][2] + c0[1][2], c0[0][3] + c0[1][3]);
+    if (nrb == 2) {
+      put(rh + g8 + 16, c1[0][0] + c1[1][0], c1[0][1] + c1[1][1]);
+      put(rh + g8 + 24, c1[0][2] + c1[1][2], c1[0][3] + c1[1][3]);
+    }
   }
+  if (trec && lane == 0) trec[TR_MATH] = (uint32_t)global_ns();
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
+  const int n_items = B * geo.rows_part;
+  for (int i0 = 0; i0 < n_items; i0 += kComputeThreads) {
+    // item (b, r); v0 = row r (pair ops: part 0 row r), v1 = part 1 row r
+    const GemvItem it = gemv_item(geo, B, i0 + ct);
+    EpiAhead ea;
+    if (i0 == 0) ea = ea0;
+    else gemv_epilogue_ahead(P, sm, ws, d, it, ea);
+    const int b = it.b, r = it.r;
+    const bool mine = it.on && (geo.pairs || d.op != OP_LM || d.idx * P.tile_lm + r < P.vocab);
+    float v0 = 0.f, v1 = 0.f;
+    if (mine) {
+#pragma unroll
+      for (int k = 0; k < kComputeWarps; ++k) v0 += red[(k * kMaxB + b) * 64 + r];
+      if (geo.pairs)
+#pragma unroll
+        for (int k = 0; k < kComputeWarps; ++k) v1 += red[(k * kMaxB + b) * 64 + geo.rows_part + r];
+    }
+    const int H = P.hidden;
+    switch (d.op) {
+      case OP_QKV: {
+        // RoPE on q and k (rotate-half pairs j, j + D/2), then q -> buffer, k/v -> cache
+        if (!mine) break;
+        QkvTile qt = decode_qkv(P, d.idx);
+        const int pos = sm.ctx[b];
+        const int j = qt.j0 + r;
+        if (qt.kind == 2) {
+          size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + qt.head) * P.max_ctx + pos;
+          __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * P.head_dim;
+          vc[j] = __float2bfloat16_rn(v0);
+          vc[j + 32] = __float2bfloat16_rn(v1);
+        } else {
+          const float cs = ea.a[0], sn = ea.a[1];  // (cos, sin) of (pos, j), loaded before the products
+          const float x0 = v0 * cs - v1 * sn, x1 = v1 * cs + v0 * sn;
+          if (qt.kind == 0) {
+            float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * P.head_dim +
+                        qt.head * P.head_dim;
+            qb[j] = x0;
+            qb[j + 32] = x1;
+          } else {
+            size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + qt.head) * P.max_ctx + pos;
+            __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * P.head_dim;
+            kc[j] = __float2bfloat16_rn(x0);
+            kc[j + 32] = __float2bfloat16_rn(x1);
+          }
+        }
+      } break;
+      case OP_OPROJ: {
+        // residual: x = (x + previous layer's down partials) + o W_o^T
+        if (!mine) break;
+        const size_t col = (size_t)d.idx * P.tile_o + r;
+        float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
+        float acc = ea.a[0];
+        if (d.layer > 0 && P.kind == MK_MODEL_DENSE) {
+          acc += (ea.a[1] + ea.a[2]) + (ea.a[3] + ea.a[4]);
+          const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H + col;
+          for (int kc = 4; kc < P.n_kc; ++kc) acc += __ldcg(dp + (size_t)kc * P.max_batch * H);
+        }
+        x[col] = acc + v0;
+      } break;
+      case OP_GATEUP: {
+        if (!mine) break;
+        float* h = reinterpret_cast<float*>(ws + P.off_h) + (size_t)b * P.ffn + (size_t)d.idx * P.tile_gu + r;
+        *h = v0 / (1.0f + expf(-v0)) * v1;
+      } break;
+      case OP_DOWN: {
+        if (!mine) break;
+        const int nt = d.idx - g.kc * P.n_dtiles;
+        float* dpart = reinterpret_cast<float*>(ws + P.off_dpart) + ((size_t)g.kc * P.max_batch + b) * H +
+                       (size_t)nt * P.tile_down + r;
+        *dpart = v0;
+      } break;
+      case OP_LM: {
+        // logits, then the warp's best (logit, id) key (the warp's items share
+        // one batch row); published with an atomic max only when it beats what
+        // this warp published before (order independent)
+        const int row = d.idx * P.tile_lm + r;
+        unsigned long long key = 0ull;
+        if (mine) {
+          if (S.logits) S.logits[(size_t)b * P.vocab + row] = v0;
+          key = argmax_key(v0, row);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+          key = other > key ? other : key;
+        }
+        if (lane == 0 && it.on && key > sm.lm_seen[w][b]) {
+          sm.lm_seen[w][b] = key;
+          atomicMax(reinterpret_cast<unsigned long long*>(ws + P.off_lmbest) + b, key);
+        }
+      } break;
+      default: break;
+    }
+  }
+  bar_sync(BAR_COMP, kComputeThreads);  // the partial tiles are free for the next task
 }
 
 // One chunk of split-K decode attention for the qpg query heads of a GQA
@@ -1944,7 +1981,6 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int B = S.B;
   int a_tag = -1;
-  int gbuf = 0;  // GEMV partial-tile buffer of the next GEMV task
   for (uint32_t k = 0;; ++k) {
     // task k: released into cur[k & 1] as phase k >> 1 of go_bar[k & 1]
     if (!wait_mbar(&sm.go_bar[k & 1], (k >> 1) & 1, ctl, P.spin_timeout_ns, -1, -1)) break;
@@ -1972,7 +2008,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
       a_tag = -1;  // MoE tasks use the staging buffer as scratch
     } else if (gemv_spec(P, d, g)) {
       // all B activation rows are staged together; an unchanged tag reuses them
-      const GemvItem it = gemv_item(sm.geo[d.op], B);
+      const GemvItem it = gemv_item(sm.geo[d.op], B, threadIdx.x - kComputeBase);
       EpiAhead ea;
       gemv_epilogue_ahead(P, sm, ws, d, it, ea);
       if (g.tag != a_tag) {
@@ -1980,8 +2016,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
         a_tag = g.tag;
       }
       if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
-      gemv_task(P, S, sm, ring, ws, ctl, d, g, B, gbuf, ea, it, trec);
-      gbuf ^= 1;
+      gemv_task(P, S, sm, ring, ws, ctl, d, g, B, ea, trec);
     } else if (d.op == OP_ATTN) {
       task_attn(P, S, sm, ring, ws, ctl, d);
       a_tag = -1;  // the staging buffer held the warps' partial outputs
@@ -2258,12 +2293,32 @@ static bool encode_weight_maps(const DevPlan& P, std::vector<unsigned char>& ima
         !put(tmap_index(l, TM_WO), lp.wo, H, (long long)Hq * D, (long long)Hq * D, bh, P.tile_o, "wo"))
       return false;
     if (P.kind == MK_MODEL_DENSE &&
-        (!put(tmap_index(l, TM_GATE), lp.w_gate, F, H, H, bh, P.tile_gu, "w_gate") ||
-         !put(tmap_index(l, TM_UP), lp.w_up, F, H, H, bh, P.tile_gu, "w_up") ||
-         !put(tmap_index(l, TM_DOWN), lp.w_down, H, F, F, P.kseg / kGemvSlots, P.tile_down, "w_down")))
+        (!put(tmap_index(l, TM_GATE), lp.w_gate, F, H, H, bh, std::min(32, P.tile_gu), "w_gate") ||
+         !put(tmap_index(l, TM_UP), lp.w_up, F, H, H, bh, std::min(32, P.tile_gu), "w_up") ||
+         !put(tmap_index(l, TM_DOWN), lp.w_down, H, F, F, P.kseg / kGemvSlots, std::min(32, P.tile_down), "w_down")))
       return false;
   }
-  return put(tmap_index(P.n_layers, 0), P.lm_head, P.vocab, H, H, H / kGemvSlots, P.tile_lm, "lm_head");
+  return put(tmap_index(P.n_layers, 0), P.lm_head, P.vocab, H, H, H / kGemvSlots, 32, "lm_head");
+}
+
+// The dynamic shared-memory limit is an attribute of the kernel function, and
+// plans of one kernel instance may need different sizes (the staging buffer
+// depends on max_batch): set it for the plan being launched when another plan
+// left a different value (one table entry per device and instance).
+static cudaError_t ensure_smem_attr(int device, const void* kern, int smem) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<int, const void*>, int>> set;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& e : set)
+    if (e.first.first == device && e.first.second == kern) {
+      if (e.second == smem) return cudaSuccess;
+      cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (r == cudaSuccess) e.second = smem;
+      return r;
+    }
+  cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (r == cudaSuccess) set.push_back({{device, kern}, smem});
+  return r;
 }
 
 mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vector<unsigned char>& image_in,
@@ -2273,7 +2328,7 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
   if (!encode_weight_maps(p.dp, image, err)) return MK_ERR_INVALID_ARG;
   size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + kSmemFixed + p.dp.act_bytes + p.dp.gred_bytes;
   const void* kern = kernel_for(p.dp);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_attr(p.device, kern, (int)smem);
   if (e == cudaSuccess) {
     int nb = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, smem);
@@ -2309,8 +2364,10 @@ mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& 
   unsigned char* ws = (unsigned char*)p.ws;
   DevPlan dp = p.dp;
   void* args[] = {(void*)&dp, (void*)&sp, (void*)&ws};
-  cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(p.dp.n_sm), dim3(kThreads), args,
-                                              (size_t)p.dp.smem_bytes, (cudaStream_t)stream);
+  cudaError_t e = ensure_smem_attr(p.device, kernel_for(p.dp), p.dp.smem_bytes);
+  if (e == cudaSuccess)
+    e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(p.dp.n_sm), dim3(kThreads), args,
+                                    (size_t)p.dp.smem_bytes, (cudaStream_t)stream);
   if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   p.epoch++;
   p.launches++;
@@ -2364,7 +2421,7 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   const size_t smem = (size_t)P0.ring_slots * P0.slot_bytes + kSmemFixed + P0.act_bytes + P0.gred_bytes;
   if (st.owner != p.uid) {
     st.owner = 0;
-    e = cudaFuncSetAttribute(kernel_for(P0), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = ensure_smem_attr(p.device, kernel_for(P0), (int)smem);
     if (e == cudaSuccess) {
       int nb = 0;
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel_for(P0), kThreads, smem);
@@ -2400,7 +2457,8 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   DevPlan dp = P0;
   dp.smem_bytes = (int)smem;
   void* args[] = {(void*)&dp, (void*)&sp, (void*)&ws};
-  e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(dp.n_sm), dim3(kThreads), args, smem, s);
+  e = ensure_smem_attr(p.device, kernel_for(p.dp), (int)smem);
+  if (e == cudaSuccess) e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(dp.n_sm), dim3(kThreads), args, smem, s);
   if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   return MK_OK;
 }
@@ -2420,7 +2478,9 @@ mk_status dev_launch_moe(Plan& p, const mk_moe_args* a, void* stream, std::strin
   unsigned char* ws = (unsigned char*)p.ws;
   DevPlan dp = p.dp;
   void* args[] = {(void*)&dp, (void*)&sp, (void*)&ws};
-  cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(p.dp.n_sm), dim3(kThreads), args,
+  cudaError_t e = ensure_smem_attr(p.device, kernel_for(p.dp), p.dp.smem_bytes);
+  if (e == cudaSuccess)
+    e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(p.dp.n_sm), dim3(kThreads), args,
                                               (size_t)p.dp.smem_bytes, (cudaStream_t)stream);
   if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
   p.epoch++;

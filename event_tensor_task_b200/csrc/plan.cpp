@@ -240,7 +240,7 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
 static void smem_layout(DevPlan& P, int rows, int smem_bytes) {
   P.gbatch = kMaxBatchRows;
   P.act_bytes = std::max(8192, (rows * kActPitch * 2 + 127) / 128 * 128);
-  P.gred_bytes = rows > 0 ? 2 * 8 * 32 * P.gbatch * 4 : 0;
+  P.gred_bytes = rows > 0 ? 8 * P.gbatch * 64 * 4 : 0;
   P.smem_bytes = smem_bytes;
   P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - P.gred_bytes) / P.slot_bytes);
 }
@@ -400,17 +400,16 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   int kseg = mdec ? 2048 : (o->kseg ? o->kseg : std::min(F, 2048));  // (no dense FFN in an MoE decoder)
   while (kseg > 256 && F % kseg) kseg -= 256;
   P.kseg = kseg;
-  // GEMV tiles on tensor cores: 16 or 32 rows per task in whole 16-row
-  // blocks (QKV: 16 rotate-half pairs; gate/up: 16 gate + 16 up rows), spread
-  // over 8 ring slots by column: slot j holds columns [j K/8, (j+1) K/8) of
-  // every row of the task.  Defaults: 32 rows everywhere (fewer, larger
-  // tasks: the per-task cost dominates; a 1B step with 16-row O tasks took 3%
-  // longer)
+  // GEMV tiles on tensor cores: 16, 32 or 64 rows per task in whole 16-row
+  // blocks (QKV: 16 rotate-half pairs; gate/up: 16 + 16 or 32 + 32 rows), in
+  // halves of at most 32 rows spread over 8 ring slots by column: slot j of a
+  // half holds columns [j K/8, (j+1) K/8) of the half's rows.  Defaults: the
+  // largest tiles (the per-task cost dominates the B=1 step)
   P.tile_qkv = o->tile_qkv ? o->tile_qkv : 32;
   P.tile_o = o->tile_o ? o->tile_o : 32;
-  P.tile_gu = o->tile_gu ? o->tile_gu : 16;
-  P.tile_down = o->tile_down ? o->tile_down : 32;
-  P.tile_lm = o->tile_lm ? o->tile_lm : 32;
+  P.tile_gu = o->tile_gu ? o->tile_gu : 32;
+  P.tile_down = o->tile_down ? o->tile_down : 64;
+  P.tile_lm = o->tile_lm ? o->tile_lm : 64;
   P.chunk = o->attn_chunk ? o->attn_chunk : 64;
   P.slot_bytes = 16384;
   if (!(P.kseg % 256 == 0 && F % P.kseg == 0 && P.kseg >= 1024 && P.kseg <= 2048))
@@ -419,11 +418,11 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (P.tile_qkv != 32) { err = "tile_qkv must be 32 (16 rotate-half pairs)"; return MK_ERR_UNSUPPORTED; }
   if (!((P.tile_o == 16 || P.tile_o == 32) && H % P.tile_o == 0))
     { err = "tile_o must be 16 or 32 and divide hidden"; return MK_ERR_UNSUPPORTED; }
-  if (P.tile_gu != 16 || P.kseg % P.tile_gu)
-    { err = "tile_gu must be 16 (16 gate + 16 up rows)"; return MK_ERR_UNSUPPORTED; }
-  if (!((P.tile_down == 16 || P.tile_down == 32) && H % P.tile_down == 0))
-    { err = "tile_down must be 16 or 32 and divide hidden"; return MK_ERR_UNSUPPORTED; }
-  if (P.tile_lm != 32) { err = "tile_lm must be 32"; return MK_ERR_UNSUPPORTED; }
+  if (!((P.tile_gu == 16 || P.tile_gu == 32) && P.kseg % P.tile_gu == 0))
+    { err = "tile_gu must be 16 or 32 (gate + up rows each)"; return MK_ERR_UNSUPPORTED; }
+  if (!((P.tile_down == 16 || P.tile_down == 32 || P.tile_down == 64) && H % P.tile_down == 0))
+    { err = "tile_down must be 16, 32 or 64 and divide hidden"; return MK_ERR_UNSUPPORTED; }
+  if (P.tile_lm != 32 && P.tile_lm != 64) { err = "tile_lm must be 32 or 64"; return MK_ERR_UNSUPPORTED; }
   if (P.chunk != 64) { err = "attn_chunk must be 64"; return MK_ERR_UNSUPPORTED; }
   P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
   P.n_otiles = H / P.tile_o;

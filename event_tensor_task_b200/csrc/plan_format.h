@@ -188,8 +188,7 @@ constexpr int kMaxFamilies = 256;
 // kernel's fixed control area (at most kSmemFixed bytes), the staging buffer
 // (act_bytes: the GEMV activation rows in bf16, kActPitch elements per batch
 // row, or 8 KB of fp32 scratch for the other task bodies) and the GEMV
-// partial tiles (gred_bytes: two buffers of 8 warps x gbatch = 8 columns x 32
-// rows of fp32).
+// partial tiles (gred_bytes: 8 warps x gbatch = 8 columns x 64 rows of fp32).
 constexpr int kSmemFixed = 9 * 1024;
 constexpr int kActPitch = 2048 + 8;  // bf16 elements per staged activation row (16-byte bank offset per row)
 constexpr int kMaxBatchRows = 8;     // batch rows of a dense step (the GEMV's MMA n = 8 columns)

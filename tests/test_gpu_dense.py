@@ -209,3 +209,18 @@ def test_llama1b_batch_of_eight():
         assert rel_err(got["logits"][b], ref["logits"][b]) <= TOL
         check_argmax(got["next_tokens"][b], ref["logits"][b])
     case.check_task_set(got["task_counts"], 8, ctx)
+
+
+@pytest.mark.parametrize("sched", [mk.MK_SCHED_STATIC, mk.MK_SCHED_DYNAMIC])
+def test_llama1b_many_steps_ring_reuse(llama, sched):
+    # 64-row tasks take 16 ring slots, so a task reuses ring positions of its
+    # own first slots: many steps in a row must neither stall nor change the
+    # result (the last step is compared with a fresh single step)
+    case = llama if sched == mk.MK_SCHED_STATIC else DenseCase(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_slots=1,
+                                                              ctx_fill=[1024], sched=sched)
+    assert case.dec.tiles()["ring_slots"] < 16 and case.dec.tiles()["tile_lm"] == 64
+    tokens, slots, ctx = [77], [0], [1024]
+    first = case.gpu_step(tokens, slots, ctx)
+    for _ in range(150):
+        last = case.gpu_step(tokens, slots, ctx, counts=False)
+    assert torch.equal(first["logits"], last["logits"])

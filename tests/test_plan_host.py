@@ -35,8 +35,8 @@ def _host(shape, max_batch=4, max_ctx=320, sched=mk.MK_SCHED_STATIC, n_sm=16, **
 def test_plan_build_and_tiles():
     d = _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148)
     t = d.tiles()
-    assert t["tile_qkv"] == 32 and t["tile_o"] == 32 and t["tile_gu"] == 16 and t["tile_down"] == 32
-    assert t["kseg"] == 2048 and t["tile_lm"] == 32 and t["chunk"] == 64 and t["n_sm"] == 148
+    assert t["tile_qkv"] == 32 and t["tile_o"] == 32 and t["tile_gu"] == 32 and t["tile_down"] == 64
+    assert t["kseg"] == 2048 and t["tile_lm"] == 64 and t["chunk"] == 64 and t["n_sm"] == 148
     fams = d.families()
     assert len(fams) == 16 * 6 + 2
     assert [f.name.decode() for f in fams[:6]] == ["qkv.0", "attn.0", "merge.0", "oproj.0", "gateup.0",
@@ -45,13 +45,13 @@ def test_plan_build_and_tiles():
 
 
 def test_plan_rejects_oversized_tiles():
-    # a GEMV task is at most 32 rows (two 16-row tensor-core blocks) spread
-    # over 8 column slices; tiles that are not whole 16-row blocks are refused
-    for bad in (dict(tile_gu=32), dict(tile_lm=64), dict(tile_o=64), dict(tile_down=64), dict(tile_o=8),
-                dict(tile_down=24), dict(tile_qkv=16), dict(tile_lm=16)):
+    # a GEMV task is at most 64 rows (two halves of up to 32 rows, each over
+    # 8 column slices); tiles that are not whole 16-row blocks are refused
+    for bad in (dict(tile_gu=64), dict(tile_lm=128), dict(tile_o=64), dict(tile_down=128), dict(tile_o=8),
+                dict(tile_down=24), dict(tile_qkv=16), dict(tile_lm=16), dict(tile_gu=8)):
         with pytest.raises(mk.MkError):
             _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148, **bad)
-    for ok in (dict(tile_o=16), dict(tile_down=16)):
+    for ok in (dict(tile_o=16), dict(tile_down=16), dict(tile_down=32), dict(tile_gu=16), dict(tile_lm=32)):
         _host(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_sm=148, **ok).close()
 
 
@@ -94,7 +94,7 @@ def test_simulator_clean(sched, B, ctx):
     assert rep.nonzero_counters == 0 and rep.static_dynamic_mismatch == 0
     t = d.tiles()
     tiles = {k: t[k] for k in ("tile_qkv", "chunk", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm")}
-    assert tiles == dict(tile_qkv=32, chunk=64, tile_o=32, tile_gu=16, tile_down=32, kseg=1024, tile_lm=32)
+    assert tiles == dict(tile_qkv=32, chunk=64, tile_o=32, tile_gu=32, tile_down=64, kseg=1024, tile_lm=64)
     assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, tiles))
 
 
