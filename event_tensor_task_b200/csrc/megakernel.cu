@@ -1094,10 +1094,19 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
       for (int i = 0; i < 4; ++i)
         if (b0 + i < B) {
           const float f[8] = {u[i].x, u[i].y, u[i].z, u[i].w, v[i].x, v[i].y, v[i].z, v[i].w};
-          __align__(16) __nv_bfloat16 o[8];
+          __align__(16) __nv_bfloat16 o[8], lo[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(g.kind == 0 ? f[j] * inv[i] * gf[j] : f[j]);
-          *reinterpret_cast<uint4*>(&sm.xa()[(b0 + i) * kActPitch + c]) = *reinterpret_cast<const uint4*>(o);
+          for (int j = 0; j < 8; ++j) {
+            const float a = g.kind == 0 ? f[j] * inv[i] * gf[j] : f[j];
+            o[j] = __float2bfloat16_rn(a);
+            lo[j] = __float2bfloat16_rn(a - __bfloat162float(o[j]));  // what bf16 left out
+          }
+          if (2 * B <= kMaxB) {  // split rows: row 2b holds row b in bf16, row 2b + 1 what bf16 left out
+            *reinterpret_cast<uint4*>(&sm.xa()[2 * (b0 + i) * kActPitch + c]) = *reinterpret_cast<const uint4*>(o);
+            *reinterpret_cast<uint4*>(&sm.xa()[(2 * (b0 + i) + 1) * kActPitch + c]) = *reinterpret_cast<const uint4*>(lo);
+          } else {
+            *reinterpret_cast<uint4*>(&sm.xa()[(b0 + i) * kActPitch + c]) = *reinterpret_cast<const uint4*>(o);
+          }
         }
     }
   }
@@ -1204,11 +1213,18 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   // rows are 128-byte lines under the 128-byte swizzle (chunk c of line n at
   // c ^ (n & 7)), which puts the 8 rows a quarter-warp reads on distinct banks
   const bool swz = geo.cw >= 64;
-  const uint4* px = reinterpret_cast<const uint4*>(&sm.xa()[min(g8, B - 1) * kActPitch + w * geo.cw]) + q;
+  // activation rows staged: B, or 2B when 2B <= 8 (row 2b + 1 carries the
+  // bf16 remainder of row b, so the products see ~16-bit activations; lane q
+  // then holds batch row q's two halves in its two columns and adds them)
+  const bool split = 2 * B <= kMaxB;
+  const int ncol = split ? 2 * B : B;
+  const uint4* px = reinterpret_cast<const uint4*>(&sm.xa()[min(g8, ncol - 1) * kActPitch + w * geo.cw]) + q;
   const int nwin = geo.cw >> 5;
   float* red = sm.gred(P.act_bytes);
   auto put = [&](int row, float x0, float x1) {  // partial tile: [w][column][64 rows]
-    if (2 * q < B) {
+    if (split) {
+      if (q < B) red[((size_t)w * kMaxB + q) * 64 + row] = x0 + x1;
+    } else if (2 * q < ncol) {
       float* e = red + ((size_t)w * kMaxB + 2 * q) * 64 + row;
       e[0] = x0;
       e[64] = x1;

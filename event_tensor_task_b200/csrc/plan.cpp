@@ -239,7 +239,8 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
 // rows = 0), the rest to 16 KB ring slots.
 static void smem_layout(DevPlan& P, int rows, int smem_bytes) {
   P.gbatch = kMaxBatchRows;
-  P.act_bytes = std::max(8192, (rows * kActPitch * 2 + 127) / 128 * 128);
+  // (B <= 4 stages 2B rows: each row's bf16 value and its bf16 remainder)
+  P.act_bytes = std::max(8192, (std::min(2 * rows, kMaxBatchRows) * kActPitch * 2 + 127) / 128 * 128);
   P.gred_bytes = rows > 0 ? 8 * P.gbatch * 64 * 4 : 0;
   P.smem_bytes = smem_bytes;
   P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - P.gred_bytes) / P.slot_bytes);
