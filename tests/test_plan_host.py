@@ -184,3 +184,18 @@ def test_stats_without_a_device():
     assert st["queue_ranges_cap"] == 0  # static schedule
     assert st["last_queue_tasks"] == -1 and st["last_queue_pops"] == -1
     d.close()
+
+
+def test_shared_memory_split_per_max_batch():
+    # the staging buffer holds 2 x max_batch bf16 rows (value and remainder)
+    # up to 8 rows, the rest of 227 KB goes to 16 KB ring slots after the 9 KB
+    # fixed area and the 16 KB of GEMV partial tiles
+    rows = {1: 2, 2: 4, 4: 8, 8: 8}
+    for mb, want in ((1, 12), (2, 11), (4, 10), (8, 10)):
+        act = max(8192, (rows[mb] * (2048 + 8) * 2 + 127) // 128 * 128)
+        assert (232448 - 9 * 1024 - act - 16384) // 16384 == want
+        d = _host(wl.LLAMA_1B, max_batch=mb, max_ctx=1088, n_sm=148)
+        assert d.tiles()["ring_slots"] == want
+        d.close()
+    with pytest.raises(mk.MkError):
+        _host(wl.LLAMA_1B, max_batch=9, max_ctx=1088, n_sm=148)
