@@ -45,7 +45,7 @@ def _rank(rank, world, port, out):
 def test_two_replicas_max_over_ranks_and_rate():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:  # (no fork of a threaded process)
         out = mgr.dict()
         mp.start_processes(_rank, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
         res = dict(out)
