@@ -12,22 +12,26 @@
 //
 // Warp roles inside a CTA (352 threads):
 //   warp 0     producer   walks the task stream ahead of execution and streams
-//                         each task's weights (and cached KV rows) into a ring
-//                         of 16 KB shared-memory slots with bulk async copies;
-//                         it never waits on events, so weight traffic runs
-//                         ahead of synchronisation.
+//                         each task's weights into a ring of 16 KB shared-
+//                         memory slots: GEMV rows by 2-D/3-D TMA boxes (one
+//                         tensor map per weight matrix, 128-byte swizzle, a
+//                         task's rows in column slices), cached KV rows and
+//                         expert rows by bulk async copies; it never waits on
+//                         events, so weight traffic runs ahead of
+//                         synchronisation.
 //   warp 1     controller takes tasks in order, waits on their events and
 //                         releases them to the compute warps through a
 //                         two-deep buffer (the next task is staged while the
 //                         current one runs).
-//   warp 2     notifier   publishes finished tasks: one gpu-scope release
-//                         fence per batch, then the counter decrements; the
+//   warp 2     notifier   publishes finished tasks with gpu-scope release
+//                         decrements, one per distinct counter of a batch; the
 //                         decrement that takes a counter to zero queues the
 //                         event's follow-up task and, in dynamic mode, pushes
 //                         the consumer tasks.
-//   warps 3-10 compute    each warp works through whole weight rows of a task
-//                         (dot products reduced inside the warp, no block
-//                         barriers), or one attention head of a key chunk.
+//   warps 3-10 compute    GEMV tasks on tensor cores (warp MMA m16n8k16 bf16,
+//                         the batch rows as the n = 8 columns; warp j reads
+//                         only slot j of each half of a task), attention
+//                         chunks, merges and the MoE task bodies.
 // Every spin is bounded by the plan's timeout; on expiry the kernel records an
 // error in the control block, raises an abort flag that every spin polls,
 // drains its in-flight copies and exits.
