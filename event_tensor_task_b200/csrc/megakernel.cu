@@ -59,6 +59,7 @@ constexpr int kDoneQ = 32;    // controller -> notifier
 constexpr int kFollowQ = 16;  // notifier -> controller
 constexpr int kMaxB = kMaxBatchRows;  // batch rows per step on this path
 constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
+constexpr int kMoeStageRows = 2;  // MoE tiles with at most this many routed rows stage them in shared memory
 constexpr int kDynLookahead = 2;
 
 struct StepParams {
@@ -1802,6 +1803,23 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
   const int nwin = H >> 5, win0 = kp * nwin / ks, win1 = (kp + 1) * nwin / ks;
   const int jlo = (8 * nh) / rps, jhi = (8 * nh + 7) / rps;  // this warp's slots within each part
   float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
+  const int* mperm = reinterpret_cast<const int*>(mb + P.off_mperm);
+  const __nv_bfloat16* xsrc = P.kind == MK_MODEL_MOE_DECODER
+                                  ? reinterpret_cast<const __nv_bfloat16*>(mb + P.off_mxhat) : S.moe_x;
+  // a tile of at most kMoeStageRows routed rows (small T) stages their A
+  // operand in the staging buffer once, instead of reading it from L2 inside
+  // the K loop
+  const int cpr = H / 8;  // 16-byte chunks per row
+  const bool staged = mt.nrows <= kMoeStageRows;
+  if (staged) {
+    bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the staging buffer
+    for (int i = threadIdx.x - kComputeBase; i < mt.nrows * cpr; i += kComputeThreads) {
+      const int r = i / cpr, c = i - r * cpr;
+      reinterpret_cast<uint4*>(sm.xs())[i] =
+          __ldcg(reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + r) / K) * H) + c);
+    }
+    bar_sync(BAR_COMP, kComputeThreads);
+  }
   if (active) {
   for (int part = 0; part < 2; ++part)
     for (int j = jlo; j <= jhi; ++j) {
@@ -1813,20 +1831,29 @@ __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, 
   const size_t roff = (size_t)(row % rps) * 2 * H;
   const uint4* bg = reinterpret_cast<const uint4*>(ring + (size_t)(jg < R ? jg : jg - R) * P.slot_bytes + roff);
   const uint4* bu = reinterpret_cast<const uint4*>(ring + (size_t)(ju < R ? ju : ju - R) * P.slot_bytes + roff);
-  const int* mperm = reinterpret_cast<const int*>(mb + P.off_mperm);
-  const __nv_bfloat16* xsrc = P.kind == MK_MODEL_MOE_DECODER
-                                  ? reinterpret_cast<const __nv_bfloat16*>(mb + P.off_mxhat) : S.moe_x;
   const int rlo = mbk * 16 + g, rhi = rlo + 8;
   const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
-  const uint4* alo = vlo ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rlo) / K) * H) : nullptr;
+  const uint4* alo = !vlo ? nullptr
+                     : staged ? reinterpret_cast<const uint4*>(sm.xs()) + (size_t)rlo * cpr
+                              : reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rlo) / K) * H);
   const uint4* ahi = vhi ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rhi) / K) * H) : nullptr;
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  if (staged) {  // (rows g + 8 lie past the tile's rows)
 #pragma unroll 4
-  for (int wi = win0; wi < win1; ++wi) {
-    const int c = wi * 4 + q;  // 16-byte chunk of the row
-    const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
-    mma_window(ag, ua, ub, bg[c]);
-    mma_window(au, ua, ub, bu[c]);
+    for (int wi = win0; wi < win1; ++wi) {
+      const int c = wi * 4 + q;
+      const uint4 ua = vlo ? alo[c] : z;
+      mma_window(ag, ua, z, bg[c]);
+      mma_window(au, ua, z, bu[c]);
+    }
+  } else {
+#pragma unroll 4
+    for (int wi = win0; wi < win1; ++wi) {
+      const int c = wi * 4 + q;  // 16-byte chunk of the row
+      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
+      mma_window(ag, ua, ub, bg[c]);
+      mma_window(au, ua, ub, bu[c]);
+    }
   }
   __syncwarp();
   if (lane == 0)
@@ -1891,6 +1918,15 @@ __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S
   const int nwin = FF >> 5, win0 = kp * nwin / ks, win1 = (kp + 1) * nwin / ks;
   const int jlo = (8 * nh) / rps, jhi = (8 * nh + 7) / rps;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint4* mh = reinterpret_cast<const uint4*>(mb + P.off_mh);
+  const int cpr = FF / 8;  // 16-byte chunks per row
+  const bool staged = mt.nrows <= kMoeStageRows;  // as in task_egu
+  if (staged) {
+    bar_sync(BAR_COMP, kComputeThreads);
+    for (int i = threadIdx.x - kComputeBase; i < mt.nrows * cpr; i += kComputeThreads)
+      reinterpret_cast<uint4*>(sm.xs())[i] = __ldcg(mh + (size_t)mt.r0 * cpr + i);  // rows r0 .. r0 + nrows - 1
+    bar_sync(BAR_COMP, kComputeThreads);
+  }
   if (active) {
   for (int j = jlo; j <= jhi; ++j) {
     const int js = s0 + j;
@@ -1899,17 +1935,25 @@ __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S
   const int row = 8 * nh + g, jr = s0 + row / rps;
   const uint4* bp = reinterpret_cast<const uint4*>(ring + (size_t)(jr < R ? jr : jr - R) * P.slot_bytes +
                                                    (size_t)(row % rps) * 4096);
-  const uint4* mh = reinterpret_cast<const uint4*>(mb + P.off_mh);
   const int rlo = mbk * 16 + g, rhi = rlo + 8;
   const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
   const uint4* alo = mh + ((size_t)(mt.r0 + (vlo ? rlo : 0)) * FF) / 8;
   const uint4* ahi = mh + ((size_t)(mt.r0 + (vhi ? rhi : 0)) * FF) / 8;
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  if (staged) {  // (rows g + 8 lie past the tile's rows)
+    const uint4* slo = reinterpret_cast<const uint4*>(sm.xs()) + (size_t)(vlo ? rlo : 0) * cpr;
 #pragma unroll 4
-  for (int wi = win0; wi < win1; ++wi) {
-    const int c = wi * 4 + q;
-    const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
-    mma_window(acc, ua, ub, bp[c]);
+    for (int wi = win0; wi < win1; ++wi) {
+      const int c = wi * 4 + q;
+      mma_window(acc, vlo ? slo[c] : z, z, bp[c]);
+    }
+  } else {
+#pragma unroll 4
+    for (int wi = win0; wi < win1; ++wi) {
+      const int c = wi * 4 + q;
+      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
+      mma_window(acc, ua, ub, bp[c]);
+    }
   }
   __syncwarp();
   if (lane == 0)
