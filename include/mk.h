@@ -104,8 +104,8 @@ typedef struct mk_model_desc {
   const mk_layer_weights* layers; /* host array [n_layers] of device pointers */
   void* k_cache;          /* bf16 [n_layers][n_slots][n_kv_heads][max_ctx][head_dim], device, post-RoPE keys */
   void* v_cache;          /* bf16, same layout as k_cache */
-  int n_experts, top_k, expert_ffn, max_tokens;  /* MK_MODEL_MOE_LAYER */
-  mk_moe_weights moe;     /* MK_MODEL_MOE_LAYER */
+  int n_experts, top_k, expert_ffn, max_tokens;  /* MK_MODEL_MOE_LAYER and MK_MODEL_MOE_DECODER */
+  mk_moe_weights moe;     /* MK_MODEL_MOE_LAYER (the decoder's per-layer experts are in layers[l].moe) */
 } mk_model_desc;
 
 /* Plan options; zero-initialise and set what you need (0 = default). */
@@ -114,6 +114,12 @@ typedef struct mk_plan_opts {
   int n_sm;               /* CTAs of the persistent kernel; 0 = SMs of the current device */
   int host_only;          /* 1: build without touching a GPU (validation/simulation only) */
   int smem_bytes;         /* dynamic shared memory per CTA; 0 = device opt-in maximum */
+  /* GEMV task tiles in rows (0 = default): tile_qkv 32 (16 rotate-half
+   * pairs); tile_o 16 or 32 (default 32); tile_gu 16 or 32 gate rows plus as
+   * many up rows (default 32); tile_down 16, 32 or 64 (default 64); tile_lm 32
+   * or 64 (default 64).  kseg: down-projection K segment, a multiple of 256 in
+   * [1024, 2048] dividing ffn.  attn_chunk: 64 keys.  Other values are
+   * refused with MK_ERR_UNSUPPORTED or MK_ERR_INVALID_ARG. */
   int tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, attn_chunk;
   long long spin_timeout_ns; /* device spin-wait limit; 0 = 2 s */
   unsigned debug_flags;   /* MK_DEBUG_* bits */
@@ -216,7 +222,11 @@ mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_pla
 size_t mk_plan_workspace_bytes(const mk_plan* p);
 
 /* Bind caller-allocated device workspace and upload the lowered plan into it
- * (asynchronous on `stream`).  Must be called before mk_decode_step. */
+ * (synchronises `stream`).  Must be called before mk_decode_step.  The dense
+ * weight matrices are read through TMA tensor maps encoded here: every weight
+ * matrix and norm gain must be 16-byte aligned (MK_ERR_INVALID_ARG
+ * otherwise, also when the driver rejects a map); MK_ERR_WORKSPACE for a
+ * missing, short or misaligned workspace. */
 mk_status mk_plan_bind_workspace(mk_plan* p, void* dev_ptr, size_t bytes, void* stream);
 
 /* One decode step: a single launch of the persistent megakernel on `stream`.
