@@ -264,6 +264,93 @@ def test_zero_mixing_predicts_input_token():
         assert int(r["next_tokens"][0]) == t
 
 
+def test_argmax_ties_golden():
+    # hand-worked rows with tied maxima (tests/golden/argmax_ties.txt)
+    for row in read_golden("argmax_ties.txt"):
+        assert row[0] == "case"
+        arrow = row.index("->")
+        vals = torch.tensor([float(v) for v in row[1:arrow]], dtype=F64)
+        assert od.argmax_lowest(vals) == int(row[arrow + 1]), row
+
+
+def test_decode_step_tied_logits_pick_lowest_id():
+    # two identical rows of the tied embedding give two identical logits; when
+    # they are the maximum the step returns the lower id
+    s = wl.TINY
+    w = wl.dense_weights(s)
+    K, V = wl.kv_cache(s, 1, 80, [64])
+    tok = 500
+    best = int(od.DenseOracle(s, w).step(K.clone(), V.clone(), [tok], [0], [64])["next_tokens"][0])
+    low = 0 if best != 0 else 1
+    assert tok != low  # (the input row itself is unchanged)
+    w2 = dict(w)
+    e = w["embed"].clone()
+    e[low] = e[best]
+    w2["embed"] = e
+    r = od.DenseOracle(s, w2).step(K.clone(), V.clone(), [tok], [0], [64])
+    lg = r["logits"][0]
+    assert float(lg[low]) == float(lg[best]) and float(lg[best]) == float(lg.max())
+    assert int(r["next_tokens"][0]) == min(low, best)
+
+
+# ---------------------------------------------------------------- MoE decoder block
+def _dense_ffn_hook(w, s, round_input=False):
+    """The dense FFN of each layer as a replacement FFN callable (fp64)."""
+    def hook(l, u):
+        P = f"layers.{l}."
+        if round_input:
+            u = od.bf16_round(u)
+        return od.swiglu(u @ w[P + "w_gate"].double().T, u @ w[P + "w_up"].double().T) @ w[P + "w_down"].double().T
+    return hook
+
+
+def test_decoder_ffn_hook_reproduces_dense_step():
+    # the replacement-FFN path (the MoE decoder's block) must see the
+    # ffn-normed residual u and add its output to the residual: with the dense
+    # FFN as the hook the step equals the dense step, residual captures included
+    w, K, V, ctx = _micro_inputs()
+    o = od.DenseOracle(MICRO, w)
+    ref = o.step(K.clone(), V.clone(), [5, 17], [0, 1], ctx, capture=True)
+    got = o.step(K.clone(), V.clone(), [5, 17], [0, 1], ctx, moe=_dense_ffn_hook(w, MICRO), capture=True)
+    assert torch.allclose(got["logits"], ref["logits"], rtol=0, atol=1e-12)
+    for a, b in zip(got["residual"], ref["residual"]):
+        assert torch.allclose(a, b, rtol=0, atol=1e-12)
+    # a hook fed x instead of u, or a dropped residual add, changes the result
+    def bad_input(l, u):
+        return _dense_ffn_hook(w, MICRO)(l, u * 2.0)
+    bad = o.step(K.clone(), V.clone(), [5, 17], [0, 1], ctx, moe=bad_input)
+    assert not torch.allclose(bad["logits"], ref["logits"], atol=1e-6)
+
+
+def _moe_from_dense(w, s, l, E):
+    """E identical experts, each the dense FFN of layer l; router zeros."""
+    P = f"layers.{l}."
+    return {"router": torch.zeros(E, s.hidden, dtype=torch.bfloat16),
+            "w_gate": w[P + "w_gate"][None].expand(E, -1, -1).contiguous(),
+            "w_up": w[P + "w_up"][None].expand(E, -1, -1).contiguous(),
+            "w_down": w[P + "w_down"][None].expand(E, -1, -1).contiguous()}
+
+
+@pytest.mark.parametrize("E,k", [(1, 1), (4, 2)])
+def test_decoder_moe_block_equals_dense_on_rounded_input(E, k):
+    # the MoE decoder block as the GPU tests build it (MoE layer on the
+    # bf16-rounded normalised residual): E = k = 1 with the dense FFN as the
+    # expert, and E identical experts with top-k > 1 (weights sum to one), both
+    # equal the dense FFN applied to the rounded input
+    s = wl.DenseShape(n_layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=64, vocab=40)
+    w = wl.dense_weights(s, seed=3)
+    K, V = wl.kv_cache(s, 2, 16, [5, 9], seed=3)
+    o = od.DenseOracle(s, w)
+    experts = [_moe_from_dense(w, s, l, E) for l in range(s.n_layers)]
+    hook = lambda l, u: om.moe_layer(u.to(torch.bfloat16), experts[l], k)["out"]
+    got = o.step(K.clone(), V.clone(), [3, 11], [0, 1], [5, 9], moe=hook, capture=True)
+    ref = o.step(K.clone(), V.clone(), [3, 11], [0, 1], [5, 9], moe=_dense_ffn_hook(w, s, round_input=True),
+                 capture=True)
+    assert torch.allclose(got["logits"], ref["logits"], rtol=0, atol=1e-12)
+    for a, b in zip(got["residual"], ref["residual"]):
+        assert torch.allclose(a, b, rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- MoE router
 def test_router_order_golden():
     rows = read_golden("router_order.txt")
