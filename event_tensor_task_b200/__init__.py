@@ -11,10 +11,12 @@ from __future__ import annotations
 import ctypes as C
 
 from . import _abi
-from ._abi import (MK_MODEL_MOE_LAYER, MK_MODEL_MOE_DECODER, mk_moe_weights, mk_moe_args, MK_OK, MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_STATIC_SCRATCH_BYTES,
+from ._abi import (MK_MODEL_MOE_LAYER, MK_MODEL_MOE_DECODER, mk_moe_weights, mk_moe_args, MK_OK, MK_ERR_INVALID_ARG,
+                   MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_ERR_CUDA, MK_ERR_DEVICE_TIMEOUT, MK_ERR_DEVICE_BOUNDS,
+                   MK_ERR_PLAN, MK_STATIC_SCRATCH_BYTES,
                    MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS, MK_DEBUG_TRACE,
                    MK_SIM_FAULT_NONE, MK_SIM_FAULT_DROP_NOTIFY, MK_SIM_FAULT_COUNT_PLUS_ONE,
-                   MK_SIM_FAULT_NO_WAIT, OP_NAMES, mk_model_desc, mk_plan_opts, mk_step_args,
+                   MK_SIM_FAULT_NO_WAIT, MK_SIM_FAULT_COUNT_MINUS_ONE, OP_NAMES, mk_model_desc, mk_plan_opts, mk_step_args,
                    mk_layer_weights, mk_device_status, mk_family_info, mk_sim_report)
 
 _lib = None
@@ -40,6 +42,8 @@ def _check(status: int):
 
 
 def _ints(vals):
+    if vals is None:
+        return None
     vals = [int(v) for v in vals]
     return (C.c_int * len(vals))(*vals)
 
@@ -107,10 +111,18 @@ def mk_plan_family_info(plan: int, f: int) -> mk_family_info:
 
 
 def mk_plan_tiles(plan: int) -> dict:
-    out = (C.c_int * 9)()
+    out = (C.c_int * 11)()
     _check(lib().mk_plan_tiles(plan, out))
-    keys = ("tile_qkv", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm", "chunk", "n_sm", "ring_slots")
+    keys = ("tile_qkv", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm", "chunk", "n_sm", "ring_slots",
+            "attn_split", "wide")
     return dict(zip(keys, list(out)))
+
+
+def mk_plan_counter_region(plan: int):
+    """(byte offset in the workspace, number of int32 counters) of the Event Tensor counters."""
+    off, n = C.c_longlong(), C.c_int()
+    _check(lib().mk_plan_counter_region(plan, C.byref(off), C.byref(n)))
+    return int(off.value), int(n.value)
 
 
 def mk_plan_validate(plan: int, batch: int, ctx_lens) -> None:
@@ -212,13 +224,19 @@ class DenseDecoder:
         return mk_plan_tiles(self.plan)
 
     def step(self, token_ids, slot_ids, ctx_lens, next_tokens, logits=None, task_counts=None, stream=None,
-             trace=None, static_scratch=False):
+             trace=None, static_scratch=False, capture=None):
         """One decode step on ``stream`` (default: torch's current stream);
-        through mk_decode_step_static when ``static_scratch``."""
+        through mk_decode_step_static when ``static_scratch``.  ``capture``
+        maps ``resid``, ``moe_in``, ``topk``, ``hist``, ``indptr`` to device
+        tensors that receive the step's debug captures (mk_step_args)."""
         import torch
         a = mk_step_args()
         if trace is not None:
             a.trace, a.trace_cap = _ptr(trace), int(trace.shape[1])
+        if capture:
+            a.capture_resid, a.capture_moe_in = _ptr(capture.get("resid")), _ptr(capture.get("moe_in"))
+            a.capture_topk, a.capture_hist = _ptr(capture.get("topk")), _ptr(capture.get("hist"))
+            a.capture_indptr = _ptr(capture.get("indptr"))
         a.batch = int(token_ids.numel())
         a.token_ids, a.slot_ids, a.ctx_lens = _ptr(token_ids), _ptr(slot_ids), _ptr(ctx_lens)
         a.logits, a.next_tokens, a.task_counts = _ptr(logits), _ptr(next_tokens), _ptr(task_counts)
@@ -227,6 +245,13 @@ class DenseDecoder:
 
     def status(self):
         return mk_get_status(self.plan)
+
+    def counters(self):
+        """The Event Tensor counters in the bound workspace (int32 tensor on the device)."""
+        import torch
+        off, n = mk_plan_counter_region(self.plan)
+        base = (_ptr(self.ws) + 255) // 256 * 256 - _ptr(self.ws)
+        return self.ws[base + off: base + off + 4 * n].view(torch.int32)
 
     def stats(self):
         return mk_get_stats(self.plan)
@@ -298,6 +323,13 @@ class MoELayer:
 
     def status(self):
         return mk_get_status(self.plan)
+
+    def counters(self):
+        """The Event Tensor counters in the bound workspace (int32 tensor on the device)."""
+        import torch
+        off, n = mk_plan_counter_region(self.plan)
+        base = (_ptr(self.ws) + 255) // 256 * 256 - _ptr(self.ws)
+        return self.ws[base + off: base + off + 4 * n].view(torch.int32)
 
     def close(self):
         if self.plan:

@@ -28,13 +28,14 @@ MK_SIM_FAULT_NONE = 0
 MK_SIM_FAULT_DROP_NOTIFY = 1
 MK_SIM_FAULT_COUNT_PLUS_ONE = 2
 MK_SIM_FAULT_NO_WAIT = 3
+MK_SIM_FAULT_COUNT_MINUS_ONE = 4
 
 MK_MODEL_MOE_LAYER = 1
 MK_MODEL_MOE_DECODER = 2
 
-OP_NAMES = {1: "qkv", 2: "attn", 3: "merge", 4: "oproj", 5: "gateup", 6: "down",
-            8: "lm", 10: "lmfin", 11: "route", 12: "mindptr", 13: "egu", 14: "edown", 15: "combine",
-            16: "mfin"}
+OP_NAMES = {1: "qkv", 2: "attn", 3: "merge", 4: "oproj", 5: "gateup", 6: "down", 7: "norm",
+            8: "lm", 9: "norm2", 10: "lmfin", 11: "route", 12: "mindptr", 13: "egu", 14: "edown", 15: "combine",
+            16: "mfin", 17: "normf"}
 
 
 class mk_moe_weights(C.Structure):
@@ -73,7 +74,8 @@ class mk_plan_opts(C.Structure):
         ("sched", C.c_int), ("n_sm", C.c_int), ("host_only", C.c_int), ("smem_bytes", C.c_int),
         ("tile_qkv", C.c_int), ("tile_o", C.c_int), ("tile_gu", C.c_int), ("tile_down", C.c_int),
         ("kseg", C.c_int), ("tile_lm", C.c_int), ("attn_chunk", C.c_int),
-        ("spin_timeout_ns", C.c_longlong), ("debug_flags", C.c_uint),
+        ("spin_timeout_ns", C.c_longlong), ("debug_flags", C.c_uint), ("fault", C.c_int),
+        ("fault_family", C.c_int), ("attn_split", C.c_int),
     ]
 
 
@@ -82,6 +84,8 @@ class mk_step_args(C.Structure):
         ("batch", C.c_int), ("token_ids", C.c_void_p), ("slot_ids", C.c_void_p), ("ctx_lens", C.c_void_p),
         ("logits", C.c_void_p), ("next_tokens", C.c_void_p), ("task_counts", C.c_void_p),
         ("trace", C.c_void_p), ("trace_cap", C.c_int),
+        ("capture_resid", C.c_void_p), ("capture_moe_in", C.c_void_p), ("capture_topk", C.c_void_p),
+        ("capture_hist", C.c_void_p), ("capture_indptr", C.c_void_p),
     ]
 
 
@@ -123,6 +127,7 @@ PROTOTYPES = {
     "mk_plan_num_families": (C.c_int, [C.c_void_p]),
     "mk_plan_family_info": (C.c_int, [C.c_void_p, C.c_int, C.POINTER(mk_family_info)]),
     "mk_plan_tiles": (C.c_int, [C.c_void_p, C.POINTER(C.c_int)]),
+    "mk_plan_counter_region": (C.c_int, [C.c_void_p, C.POINTER(C.c_longlong), C.POINTER(C.c_int)]),
     "mk_plan_validate": (C.c_int, [C.c_void_p, C.c_int, C.POINTER(C.c_int)]),
     "mk_plan_simulate": (C.c_int, [C.c_void_p, C.c_int, C.POINTER(C.c_int), C.c_int, C.c_uint, C.c_int,
                                    C.c_int, C.POINTER(mk_sim_report)]),

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <stdexcept>
 #include <chrono>
 #include <cstring>
 #include <new>
@@ -26,8 +27,14 @@ mk_status fail(mk_status s, const std::string& msg) {
 }
 
 bool binding_from(const mk_plan* hp, int batch, const int* ctx, mk::Binding& bd) {
-  if (!hp || batch < 1 || batch > hp->p.dp.max_batch || !ctx) return false;
+  if (!hp || batch < 1) return false;
   bd.B = batch;
+  if (hp->p.dp.kind == MK_MODEL_MOE_LAYER) {  // batch = tokens; no contexts
+    if (batch > hp->p.dp.max_tokens) return false;
+    bd.ctx.assign(batch, 0);
+    return true;
+  }
+  if (batch > hp->p.dp.max_batch || !ctx) return false;
   bd.ctx.assign(ctx, ctx + batch);
   return true;
 }
@@ -58,10 +65,13 @@ mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_pla
     }
     mk_plan* hp = new mk_plan();
     mk_status s = mk::build_plan(m, opts, n_sm, smem, hp->p, err);
-    if (s == MK_OK && hp->p.dp.kind == MK_MODEL_DENSE) {
+    if (s == MK_OK) {
       // the plan must validate on a small binding of the symbols before use
-      std::vector<int> ctx(hp->p.dp.max_batch, std::min(hp->p.dp.max_ctx - 1, 3 * hp->p.dp.chunk - 1));
-      mk::Binding bd{hp->p.dp.max_batch, ctx};
+      // (MoE plans: on a routing drawn from a fixed seed)
+      const bool layer = hp->p.dp.kind == MK_MODEL_MOE_LAYER;
+      const int B = layer ? std::min(hp->p.dp.max_tokens, 16) : hp->p.dp.max_batch;
+      std::vector<int> ctx(B, layer ? 0 : std::min(hp->p.dp.max_ctx - 1, 3 * hp->p.dp.chunk - 1));
+      mk::Binding bd{B, ctx, {}};
       s = mk::validate_plan(hp->p, bd, err);
     }
     if (s != MK_OK) {
@@ -76,6 +86,8 @@ mk_status mk_plan_build(const mk_model_desc* m, const mk_plan_opts* opts, mk_pla
     return MK_OK;
   } catch (const std::bad_alloc&) {
     return fail(MK_ERR_INVALID_ARG, "out of host memory");
+  } catch (const std::exception& e) {
+    return fail(MK_ERR_PLAN, std::string("unexpected error while building the plan: ") + e.what());
   } catch (...) {
     return fail(MK_ERR_PLAN, "unexpected error while building the plan");
   }
@@ -214,11 +226,20 @@ mk_status mk_plan_family_info(const mk_plan* hp, int f, mk_family_info* out) {
   return MK_OK;
 }
 
+mk_status mk_plan_counter_region(const mk_plan* hp, long long* byte_offset, int* n_counters) {
+  g_err.clear();
+  if (!hp || !byte_offset || !n_counters) return fail(MK_ERR_INVALID_ARG, "null argument");
+  *byte_offset = hp->p.dp.off_counters;
+  *n_counters = hp->p.dp.n_counters;
+  return MK_OK;
+}
+
 mk_status mk_plan_tiles(const mk_plan* hp, int* o) {
   g_err.clear();
   if (!hp || !o) return fail(MK_ERR_INVALID_ARG, "null argument");
   const mk::DevPlan& P = hp->p.dp;
-  int v[9] = {P.tile_qkv, P.tile_o, P.tile_gu, P.tile_down, P.kseg, P.tile_lm, P.chunk, P.n_sm, P.ring_slots};
+  int v[11] = {P.tile_qkv, P.tile_o, P.tile_gu, P.tile_down, P.kseg, P.tile_lm, P.chunk, P.n_sm, P.ring_slots,
+               P.attn_split, P.wide};
   std::memcpy(o, v, sizeof(v));
   return MK_OK;
 }

@@ -59,7 +59,6 @@ constexpr int kDoneQ = 32;    // controller -> notifier
 constexpr int kFollowQ = 16;  // notifier -> controller
 constexpr int kMaxB = kMaxBatchRows;  // batch rows per step on this path
 constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
-constexpr int kMoeStageRows = 2;  // MoE tiles with at most this many routed rows stage them in shared memory
 constexpr int kDynLookahead = 2;
 
 struct StepParams {
@@ -81,6 +80,8 @@ struct StepParams {
   uint32_t* trace;
   int trace_cap;
   unsigned epoch;
+  float* cap_resid;      // [L][B][H] residual after each layer (or null)
+  __nv_bfloat16* cap_moe_in;  // MoE decoder: [L][B][H] router input (or null)
 };
 
 struct TaskDesc {
@@ -109,6 +110,10 @@ struct Smem {
   uint64_t full[kMaxSlots], empty[kMaxSlots];
   uint64_t go_bar[2];    // controller -> compute: task k is in cur[k & 1] (count 1)
   uint64_t done_bar[2];  // compute -> controller: task k finished (one arrive per warp)
+  uint64_t acc_bar;      // tcgen05: the current GroupGEMM task's accumulator is complete (count 1)
+  uint64_t bfull[kBStages], bempty[kBStages];  // wide batch: activation chunks (B operand) in the staging buffer
+  uint32_t tmem_base;    // tcgen05: this CTA's tensor-memory allocation (MoE plans)
+  uint32_t pad_tm;
   uint64_t fifo_full[kFifo], fifo_empty[kFifo];
   TaskDesc fifo[kFifo];
   TaskDesc cur[2];
@@ -175,14 +180,29 @@ __device__ __forceinline__ bool wait_mbar(uint64_t* bar, uint32_t parity, Contro
   }
 }
 
+// A wait on an event inside the CTA that always completes (the controller's
+// next release, the tensor cores' accumulator): bounded by three spin limits,
+// but not ended by the abort flag, so that every compute warp sees the same
+// sequence of tasks and no MMA is still running when its TMEM is read or
+// freed (see compute).
+__device__ __forceinline__ bool wait_local(uint64_t* bar, uint32_t parity, long long timeout_ns) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (int it = 0;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63) == 63 && (long long)(global_ns() - t0) > 3 * timeout_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------- trace
 // MK_DEBUG_TRACE: per CTA, records of 16 uint32 (low 32 bits of the global
 // timer in ns); record 0 is the CTA's header.
 enum TraceField : int {
   TR_FAM = 0, TR_IDX = 1, TR_POP = 2, TR_READY = 3, TR_GO = 4, TR_DONE = 5, TR_NOTIFIED = 6,
   TR_CSTART = 7, TR_CEND = 8, TR_ISSUE = 9, TR_DATA = 10,
-  // GEMV tasks: activation staged, products done, partial tiles summed
-  TR_STAGED = 11, TR_MATH = 12, TR_RED = 13,
+  // GEMV tasks: activation staged, products done, partial tiles summed,
+  // epilogue items written, the staging's first loads consumed
+  TR_STAGED = 11, TR_MATH = 12, TR_RED = 13, TR_EPI = 14, TR_LOADS = 15,
   // header fields
   TRH_RECORDS = 0, TRH_BATCHES = 1, TRH_NOTIFIED = 2, TRH_FENCE_NS = 3
 };
@@ -224,17 +244,23 @@ __device__ __forceinline__ bool is_followup(int op) {
 // Counter a regular task waits on (-1: none).
 __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t, int B) {
   switch (t.op) {
+    case OP_NORM: return ev_ctr(P, EV_IN, t.layer);
+    case OP_NORM2: return ev_ctr(P, EV_O, t.layer);
+    case OP_NORMF: return ev_ctr(P, EV_IN, P.n_layers);
     case OP_QKV:
+      if (P.wide) return ev_ctr(P, EV_N1, t.layer);
       return (P.kind == MK_MODEL_MOE_DECODER && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
                                                              : ev_ctr(P, EV_IN, t.layer);
     case OP_ATTN: {
+      if (P.wide) return ev_ctr(P, EV_QKV, t.layer, 0);
       AttnTask a = decode_attn(t.idx, B, P.n_kv_heads, sm.nch, sm.pre);
       return ev_ctr(P, EV_QKV, t.layer, a.g);
     }
     case OP_OPROJ: return ev_ctr(P, EV_ATTN, t.layer);
-    case OP_GATEUP: return ev_ctr(P, EV_O, t.layer);
+    case OP_GATEUP: return P.wide ? ev_ctr(P, EV_N2, t.layer) : ev_ctr(P, EV_O, t.layer);
     case OP_DOWN: return ev_ctr(P, EV_GU, t.layer, t.idx / P.n_dtiles);
     case OP_LM:
+      if (P.wide) return ev_ctr(P, EV_NF, 0);
       return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_MCOMB, P.n_layers - 1) : ev_ctr(P, EV_IN, P.n_layers);
     case OP_ROUTE: return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_O, t.layer) : -1;
     case OP_EDOWN: return ev_ctr(P, EV_MH, moe_li(t.layer), t.idx / P.nt_d);
@@ -256,15 +282,16 @@ struct ProdFam {
   int slots_per_part;
   int parts;
   size_t task_stride;         // bytes between consecutive tasks' first rows
-  const void* tm[3];          // GEMV ops: tensor maps of the parts' matrices (QKV: q, k, v)
+  const void* tm[4];          // tensor maps: GEMV parts (QKV: q, k, v); EGU: gate, up, routed rows (16-,
+                              // 64-row boxes); EDOWN: down, SwiGLU rows (16-, 64-row boxes)
 };
 
 __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsigned char* tmaps, int fam, int op,
                            int layer, ProdFam& f) {
   const uint32_t H2 = (uint32_t)P.hidden * 2;
   f.fam = fam; f.op = op; f.layer = layer;
-  auto tmap = [&](int l, int m) -> const void* { return tmaps + (size_t)tmap_index(l, m) * kTmapBytes; };
-  f.tm[0] = f.tm[1] = f.tm[2] = nullptr;
+  auto tmap = [&](int l, int m) -> const void* { return tmaps + (size_t)tmap_index(l < 0 ? 0 : l, m) * kTmapBytes; };
+  f.tm[0] = f.tm[1] = f.tm[2] = f.tm[3] = nullptr;
   // the RMSNorm gain this family's staging reads (one 2H-byte row, not
   // otherwise L2-resident after a step's weight stream) goes to L2 now, long
   // before the family's first task runs
@@ -277,7 +304,12 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsi
     case OP_OPROJ: f.tm[0] = tmap(layer, TM_WO); break;
     case OP_GATEUP: f.tm[0] = tmap(layer, TM_GATE); f.tm[1] = tmap(layer, TM_UP); break;
     case OP_DOWN: f.tm[0] = tmap(layer, TM_DOWN); break;
-    case OP_LM: f.tm[0] = tmap(P.n_layers, 0); break;
+    case OP_LM: f.tm[0] = tmaps + (size_t)(P.n_layers * kTmapPerLayer + TMG_LM) * kTmapBytes; break;
+    case OP_EGU:
+      f.tm[0] = tmap(layer, TM_GATE); f.tm[1] = tmap(layer, TM_UP);
+      f.tm[2] = tmap(layer, TM_XG16); f.tm[3] = tmap(layer, TM_XG64);
+      break;
+    case OP_EDOWN: f.tm[0] = tmap(layer, TM_DOWN); f.tm[1] = tmap(layer, TM_HG16); f.tm[2] = tmap(layer, TM_HG64); break;
     default: break;
   }
   f.row_bytes = H2; f.row_stride = H2; f.row_pitch = H2; f.rps = P.slot_bytes / (int)H2; f.parts = 1;
@@ -303,16 +335,7 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsi
       f.row_bytes = (uint32_t)P.kseg * 2; f.row_stride = (uint32_t)P.ffn * 2; f.row_pitch = f.row_bytes;
       f.rps = P.slot_bytes / (int)f.row_bytes; f.slots_per_part = P.tile_down / f.rps;
       break;
-    case OP_EGU: {  // an expert's gate rows, then its up rows (the expert is per task)
-      const MoeW mw = moe_weights(P, layers, layer);
-      f.w[0] = (const unsigned char*)mw.gate; f.w[1] = (const unsigned char*)mw.up;
-      f.parts = 2; f.slots_per_part = ceil_div(P.moe_tn, f.rps);
-    } break;
-    case OP_EDOWN:  // an expert's down rows (expert_ffn long), placed at a 4 KB pitch
-      f.w[0] = (const unsigned char*)moe_weights(P, layers, layer).down;
-      f.row_bytes = (uint32_t)P.eff * 2; f.row_stride = f.row_bytes; f.row_pitch = 4096;
-      f.rps = P.slot_bytes / 4096; f.slots_per_part = ceil_div(P.moe_td, f.rps);
-      break;
+
     case OP_LM:
       f.w[0] = (const unsigned char*)P.lm_head;
       f.slots_per_part = ceil_div(P.tile_lm, f.rps); f.task_stride = (size_t)P.tile_lm * H2;
@@ -322,14 +345,34 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsi
 }
 
 __device__ __forceinline__ int task_slots(const DevPlan& P, const ProdFam& f, int idx) {
-  if (f.op == OP_ATTN) return 1;
+  if (f.op == OP_ATTN) return P.attn_split;  // (at most; the task's chunks)
+  if (P.wide && (f.op == OP_QKV || f.op == OP_OPROJ || f.op == OP_LM)) return P.hidden / 64;
+  if (P.wide && f.op == OP_GATEUP) return 2 * (P.hidden / 64);
+  if (P.wide && f.op == OP_DOWN) return P.kseg / 64;
+  if (f.op == OP_NORM || f.op == OP_NORM2 || f.op == OP_NORMF) return 0;
   if (f.op == OP_ROUTE || f.op == OP_COMBINE || f.op == OP_MINDPTR || f.op == OP_MFIN) return 0;
   if (f.op == OP_QKV || f.op == OP_OPROJ) return kGemvSlots;
   if (f.op == OP_GATEUP) return P.tile_gu > 16 ? 2 * kGemvSlots : kGemvSlots;
   if (f.op == OP_DOWN) return P.tile_down > 32 ? 2 * kGemvSlots : kGemvSlots;
   if (f.op == OP_LM) return P.tile_lm > 32 ? 2 * kGemvSlots : kGemvSlots;
+  if (f.op == OP_EGU) return 3 * (P.hidden / 64);  // per 64-column chunk: gate rows, up rows, routed rows
+  if (f.op == OP_EDOWN) return 2 * (P.eff / 64);   // per 64-column chunk: down rows, SwiGLU rows
   return f.parts * f.slots_per_part;
 }
+
+// A GroupGEMM tile's geometry: expert, m block, first compact row and row count.
+struct MoeTile { int e, m, r0, nrows; };
+__device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, const unsigned char* mb, int tile) {
+  MoeTile t;
+  t.e = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_e) + tile);
+  t.m = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_m) + tile);
+  const int h = __ldcg(reinterpret_cast<const int*>(mb + P.off_mhist) + t.e);
+  t.r0 = __ldcg(reinterpret_cast<const int*>(mb + P.off_mindptr) + t.e) + t.m * P.moe_tm;
+  t.nrows = min(P.moe_tm, h - t.m * P.moe_tm);
+  return t;
+}
+// rows of the B operand a tile loads (its TMA box): 16 for small tiles, else the tile size
+__device__ __forceinline__ int moe_tile_n(int nrows) { return nrows <= 16 ? 16 : kMoeTileRows; }
 
 __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                          unsigned char* ws, Control* ctl) {
@@ -355,25 +398,6 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     if (++slot == P.ring_slots) { slot = 0; phase ^= 1; }
     return true;
   };
-  // rows [0, nrows) of a part starting at src into consecutive slots
-  auto stream_part = [&](int fam, int idx, const unsigned char* src, int nrows) -> bool {
-    while (nrows > 0) {
-      unsigned char* dst;
-      uint64_t* bar;
-      if (!next_slot(fam, idx, dst, bar)) return false;
-      int rows = min(nrows, f.rps);
-      mbar_arrive_expect_tx(bar, (uint32_t)rows * f.row_bytes);
-      if (f.row_stride == f.row_bytes && f.row_pitch == f.row_bytes) {
-        bulk_g2s(dst, src, (uint32_t)rows * f.row_bytes, bar);
-      } else {
-        for (int r = 0; r < rows; ++r) bulk_g2s(dst + r * f.row_pitch, src + (size_t)r * f.row_stride, f.row_bytes, bar);
-      }
-      src += (size_t)rows * f.row_stride;
-      nrows -= rows;
-    }
-    return true;
-  };
-
   // a GEMV task's rows by column slices: slot j gets columns [x0 + j cw,
   // x0 + (j + 1) cw) of part 0's rows (from row y0 of map tm0), then of part
   // 1's rows (row y1 of tm1), as one TMA box each
@@ -416,6 +440,35 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     mbar_arrive(&sm.fifo_full[k]);
     fifo_seq++;
     if (fam < 0) return true;
+    if (P.wide && (op == OP_QKV || op == OP_OPROJ || op == OP_GATEUP || op == OP_DOWN || op == OP_LM)) {
+      // wide batch: the task's 128 weight rows in 64-column chunks, one slot
+      // per chunk and part (gate/up: the gate rows, then the up rows); the
+      // activation (the B operand) is loaded by the MMA-issuing thread once
+      // the task's event has fired (see gemm_issue_wide)
+      int row = idx * kWideRows, x0 = 0, nk = P.hidden / 64;
+      const void* m0 = f.tm[0];
+      if (op == OP_QKV) {
+        const int nq = P.n_q_heads * P.head_dim / kWideRows, nkv = P.n_kv_heads * P.head_dim / kWideRows;
+        const int kind = idx < nq ? 0 : idx < nq + nkv ? 1 : 2;
+        m0 = f.tm[kind];
+        row = (idx - (kind == 0 ? 0 : kind == 1 ? nq : nq + nkv)) * kWideRows;
+      } else if (op == OP_DOWN) {
+        const int kc = idx / P.n_dtiles;
+        row = (idx - kc * P.n_dtiles) * kWideRows;
+        x0 = kc * P.kseg;
+        nk = P.kseg / 64;
+      }
+      for (int c = 0; c < nk; ++c)
+        for (int part = 0; part < (op == OP_GATEUP ? 2 : 1); ++part) {
+          unsigned char* dst;
+          uint64_t* bar;
+          if (!next_slot(fam, idx, dst, bar)) return false;
+          mbar_arrive_expect_tx(bar, (uint32_t)kWideRows * 128u);
+          tma_load_2d(dst, part ? f.tm[1] : m0, x0 + c * 64, row, bar);
+        }
+      emitted++;
+      return true;
+    }
     switch (op) {
       case OP_QKV: {
         // rotate-half pairs: rows j0.. of the head, then rows j0 + D/2.. of it
@@ -452,38 +505,63 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
           if (!stream_tiles(fam, idx, 32, P.hidden / kGemvSlots, 0, f.tm[0], idx * P.tile_lm + r0, nullptr, 0))
             return false;
         break;
-      case OP_EGU: {
-        // tile -> expert from the table the routing follow-up wrote (visible:
-        // this task was popped after its push, which followed that write)
-        const int tile = idx / P.nt_gu, n = idx - tile * P.nt_gu;
-        const int e = __ldcg(reinterpret_cast<const int*>(moe_block(P, ws, layer) + P.off_mtile_e) + tile);
-        const size_t row0 = (size_t)e * P.eff + (size_t)n * P.moe_tn;
-        if (!stream_part(fam, idx, f.w[0] + row0 * f.row_stride, P.moe_tn)) return false;
-        if (!stream_part(fam, idx, f.w[1] + row0 * f.row_stride, P.moe_tn)) return false;
-      } break;
+      case OP_EGU:
       case OP_EDOWN: {
-        const int tile = idx / P.nt_d, n = idx - tile * P.nt_d;
-        const int e = __ldcg(reinterpret_cast<const int*>(moe_block(P, ws, layer) + P.off_mtile_e) + tile);
-        const size_t row0 = (size_t)e * P.hidden + (size_t)n * P.moe_td;
-        if (!stream_part(fam, idx, f.w[0] + row0 * f.row_stride, P.moe_td)) return false;
+        // GroupGEMM tile (tcgen05): per 64-column chunk of K, the task's 128
+        // weight rows (gate/up: the gate rows, then the up rows, one slot
+        // each) and the tile's routed rows as the B operand, each a 2-D TMA
+        // box under the 128-byte swizzle.  The tile's expert and rows come
+        // from the tables the routing follow-up wrote, and the B rows were
+        // written by other SMs' generic stores (routing tasks: the token rows;
+        // gate/up tasks: the SwiGLU rows).  This task was popped after its
+        // push, which followed those writes; the proxy fence orders them
+        // before this thread's TMA reads.
+        const unsigned char* mb = moe_block(P, ws, layer);
+        const bool gu = op == OP_EGU;
+        const int per = gu ? P.nt_gu : P.nt_d;
+        const int tile = idx / per, n = idx - tile * per;
+        const MoeTile mt = moe_tile(P, mb, tile);
+        const int nb = moe_tile_n(mt.nrows);
+        const uint32_t bbytes = (uint32_t)nb * 128;
+        fence_proxy_async_global();
+        const int wrow = mt.e * (gu ? P.eff : P.hidden) + n * kMoeTaskRows;
+        const int brow = gu ? mt.e * P.moe_cap + mt.m * P.moe_tm : mt.r0;
+        const void* bmap = gu ? f.tm[nb == 16 ? 2 : 3] : f.tm[nb == 16 ? 1 : 2];
+        const int nk = (gu ? P.hidden : P.eff) / 64;
+        for (int c = 0; c < nk; ++c) {
+          unsigned char* dst;
+          uint64_t* bar;
+          for (int part = 0; part < (gu ? 2 : 1); ++part) {
+            if (!next_slot(fam, idx, dst, bar)) return false;
+            mbar_arrive_expect_tx(bar, 128u * 128u);
+            tma_load_2d(dst, f.tm[part], c * 64, wrow, bar);
+          }
+          if (!next_slot(fam, idx, dst, bar)) return false;
+          mbar_arrive_expect_tx(bar, bbytes);
+          tma_load_2d(dst, bmap, c * 64, brow, bar);
+        }
       } break;
       case OP_ATTN: {
+        // the task's key chunks (attn_split of them at most), one slot each:
         // the chunk's cached (already rotated) keys and values, minus the row
         // this step appends; K rows at the slot start, V rows half a slot in
         AttnTask a = decode_attn(idx, S.B, P.n_kv_heads, sm.nch, sm.pre);
-        int p = sm.ctx[a.b];
-        int n_old = max(0, min(P.chunk, p - a.c * P.chunk));
-        unsigned char* dst;
-        uint64_t* bar;
-        if (!next_slot(fam, idx, dst, bar)) return false;
-        uint32_t bytes = (uint32_t)n_old * P.head_dim * 2;
-        mbar_arrive_expect_tx(bar, 2 * bytes);
-        if (n_old > 0) {
-          size_t row0 = (((size_t)layer * P.n_slots + sm.slot[a.b]) * P.n_kv_heads + a.g) * P.max_ctx +
-                        (size_t)a.c * P.chunk;
-          bulk_g2s(dst, (const unsigned char*)P.k_cache + row0 * P.head_dim * 2, bytes, bar);
-          bulk_g2s(dst + (size_t)P.chunk * P.head_dim * 2, (const unsigned char*)P.v_cache + row0 * P.head_dim * 2,
-                   bytes, bar);
+        const int p = sm.ctx[a.b];
+        const int c0 = a.c * P.attn_split, c1 = min(c0 + P.attn_split, ceil_div(p + 1, P.chunk));
+        for (int cc = c0; cc < c1; ++cc) {
+          const int n_old = max(0, min(P.chunk, p - cc * P.chunk));
+          unsigned char* dst;
+          uint64_t* bar;
+          if (!next_slot(fam, idx, dst, bar)) return false;
+          const uint32_t bytes = (uint32_t)n_old * P.head_dim * 2;
+          mbar_arrive_expect_tx(bar, 2 * bytes);
+          if (n_old > 0) {
+            const size_t row0 = (((size_t)layer * P.n_slots + sm.slot[a.b]) * P.n_kv_heads + a.g) * P.max_ctx +
+                                (size_t)cc * P.chunk;
+            bulk_g2s(dst, (const unsigned char*)P.k_cache + row0 * P.head_dim * 2, bytes, bar);
+            bulk_g2s(dst + (size_t)P.chunk * P.head_dim * 2, (const unsigned char*)P.v_cache + row0 * P.head_dim * 2,
+                     bytes, bar);
+          }
         }
       } break;
       default: break;
@@ -580,7 +658,10 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
   NotifyInfo n;
   n.ctr = -1; n.ffam = -1; n.fop = 0; n.flayer = -1; n.fidx = 0; n.need_old = 0;
   switch (t.op) {
-    case OP_QKV: n.ctr = ev_ctr(P, EV_QKV, t.layer, decode_qkv(P, t.idx).group); break;
+    case OP_NORM: n.ctr = ev_ctr(P, EV_N1, t.layer); break;
+    case OP_NORM2: n.ctr = ev_ctr(P, EV_N2, t.layer); break;
+    case OP_NORMF: n.ctr = ev_ctr(P, EV_NF, 0); break;
+    case OP_QKV: n.ctr = ev_ctr(P, EV_QKV, t.layer, P.wide ? 0 : decode_qkv(P, t.idx).group); break;
     case OP_ATTN: {
       AttnTask a = decode_attn(t.idx, S.B, Hkv, sm.nch, sm.pre);
       n.ctr = ev_ctr(P, EV_CHUNK, t.layer, a.b, a.g);
@@ -617,7 +698,15 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
                                 unsigned char* ws, const TaskDesc& t) {
   const int Hkv = P.n_kv_heads;
   switch (t.op) {
+    case OP_NORM: push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer), 0, P.n_qkv_tiles); break;
+    case OP_NORM2: push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles); break;
+    case OP_NORMF: push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles); break;
     case OP_QKV: {
+      if (P.wide) {  // (one event per layer: every kv head's tasks of a sequence in one range)
+        for (int b = 0; b < S.B; ++b)
+          push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b], Hkv * sm.nch[b]);
+        break;
+      }
       int g = decode_qkv(P, t.idx).group;
       for (int b = 0; b < S.B; ++b)
         push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b] + g * sm.nch[b], sm.nch[b]);
@@ -625,6 +714,7 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
     case OP_MERGE: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
     case OP_OPROJ:
       if (P.kind == MK_MODEL_MOE_DECODER) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, t.layer), 0, ceil_div(S.B, 8));
+      else if (P.wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM2, t.layer), 0, ceil_div(S.B, 8));
       else push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles);
       break;
     case OP_GATEUP: {
@@ -632,8 +722,14 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
       push_range(P, S, ctl, ws, fam_of(P, OP_DOWN, t.layer), kc * P.n_dtiles, P.n_dtiles);
     } break;
     case OP_DOWN:
-      if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
-      else push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
+      if (P.wide) {
+        if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, ceil_div(S.B, 8));
+        else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, ceil_div(S.B, 8));
+      } else if (t.layer + 1 < P.n_layers) {
+        push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
+      } else {
+        push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
+      }
       break;
     // MoE: exp_indptr decides how many GroupGEMM tiles run (data-dependent task triggering)
     case OP_MINDPTR: {
@@ -959,6 +1055,13 @@ __device__ void controller(const DevPlan& P, const StepParams& S, Smem& sm, unsi
 }
 
 // ---------------------------------------------------------------- compute
+// Ring slot i of a task (its first slot and phase in slot_ph).
+__device__ __forceinline__ int task_slot(const TaskDesc& d, int i, int R, uint32_t& parity) {
+  const int pos = (d.slot_ph & 0xffff) + i, wrap = pos / R;
+  parity = ((uint32_t)d.slot_ph >> 16) ^ ((uint32_t)wrap & 1u);
+  return pos - wrap * R;
+}
+
 struct GemvSpec {
   int kind;           // 0: RMSNorm(x) * gamma, 1: attention output, 2: SwiGLU segment
   int gamma_sel;      // kind 0: 0 attention-norm gain of `layer`, 1 FFN-norm gain, 2 final-norm gain
@@ -996,6 +1099,9 @@ __device__ __forceinline__ bool gemv_spec(const DevPlan& P, const TaskDesc& d, G
 }
 
 
+// TMEM address of lane quadrant q (lanes 32q .. 32q + 31), column 0.
+__device__ __forceinline__ uint32_t S_tmem_lane(uint32_t base, int q) { return base + ((uint32_t)(32 * q) << 16); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -1010,7 +1116,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 // load of a group is issued before the first use).  Called by all compute
 // warps for the same task (the tag sequence is the same for all warps).
 // Thread t stages columns [8t, 8t + 8).
-__device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int B) {
+__device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, Smem& sm, const GemvSpec& g, int B,
+                                          uint32_t* trec, float* cap) {
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int K = g.K;  // at most 8 * kComputeThreads
@@ -1067,6 +1174,11 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
           u[i].x += a4.x; u[i].y += a4.y; u[i].z += a4.z; u[i].w += a4.w;
           v[i].x += b4.x; v[i].y += b4.y; v[i].z += b4.z; v[i].w += b4.w;
         }
+        if (cap) {  // debug capture of the residual row this staging reduced
+          float4* c4 = reinterpret_cast<float4*>(cap + (size_t)b * K + c);
+          c4[0] = u[i];
+          c4[1] = v[i];
+        }
       }
     }
     float inv[4] = {1.f, 1.f, 1.f, 1.f};
@@ -1080,6 +1192,7 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
           if (lane == 0) sm.red8[b0 + i][w] = ss;
         }
     }
+    if (trec && lane == 0 && b0 == 0) trec[TR_LOADS] = (uint32_t)global_ns();
     // (the first group's barrier also means every warp is done with the previous activation)
     bar_sync(BAR_COMP, kComputeThreads);
     if (g.kind == 0) {
@@ -1118,16 +1231,13 @@ __device__ __forceinline__ void stage_act(const DevPlan& P, unsigned char* ws, S
   bar_sync(BAR_COMP, kComputeThreads);  // the activation is complete
 }
 
-// Ring slot release.  A slot's empty barrier expects kComputeWarps arrivals
-// per use; only the warps that READ the slot arrive, each with its share of
-// that count (the first reader adds the remainder).  A warp arrives only
-// after it has waited for the slot's data, so no arrival can land in
-// another use's phase (with tasks of up to 8 slots in the ring, task k+1's
-// slots can be physical slots that task k still reads).
-__device__ __forceinline__ void release_share(Smem& sm, int slot, int readers, int rank) {
-  const uint32_t share = kComputeWarps / readers + (rank == 0 ? kComputeWarps % readers : 0);
-  mbar_arrive_count(&sm.empty[slot], share);
-}
+// Ring slot release.  A slot's empty barrier expects one arrival per use,
+// made after every read of the slot: by the slot's only reader (a GEMV
+// product warp), by one thread after a barrier of all readers (attention),
+// or by tcgen05.commit once the MMAs reading it completed (GroupGEMM tiles).
+// Nobody arrives before it has waited for the slot's data, so no arrival can
+// land in another use's phase (task k+1's slots can be physical slots that
+// task k still reads).
 
 // ---- tensor-core tiles
 // Warp-level bf16 MMA m16n8k16 with fp32 accumulation.  K is walked in
@@ -1282,7 +1392,7 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
       }
     }
     __syncwarp();
-    if (lane == 0) release_share(sm, sw, 1, 0);  // the slot's only reader
+    if (lane == 0) mbar_arrive(&sm.empty[sw]);  // the slot's only reader
     // lane (g8, q) holds rows g8, g8 + 8 (+ 16 for block 1) of the half at
     // batch columns 2q, 2q + 1
     const int rh = 32 * h;
@@ -1390,118 +1500,135 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
       default: break;
     }
   }
+  if (trec && lane == 0) trec[TR_EPI] = (uint32_t)global_ns();
   bar_sync(BAR_COMP, kComputeThreads);  // the partial tiles are free for the next task
 }
 
-// One chunk of split-K decode attention for the qpg query heads of a GQA
-// group (flash-decoding partial: unnormalised output, running max, sum).
-// All 8 compute warps share the chunk: warp w scores keys [8w, 8w + 8) for
-// every head of the group (each K row is read from shared memory once; a
-// lane holds one 16-byte slice of a row and the matching 8 query values of
-// each head in registers), then accumulates those keys' V rows for every
-// head; the 8 warps' partial outputs are summed through the staging buffer.
-// The new key (position ctx) is read from the cache in global memory: the
-// ring copy of its chunk may predate this step's append.
+// One task of split-KV decode attention for the qpg query heads of a GQA
+// group: up to attn_split consecutive 64-key chunks of one sequence, one ring
+// slot each (flash-decoding partial: unnormalised output, running max, sum).
+// All 8 compute warps share a chunk: warp w scores keys [8w, 8w + 8) for
+// every head of the group (each K row is read from shared memory once; a lane
+// holds one 16-byte slice of a row and the matching 8 query values of each
+// head in registers), then accumulates those keys' V rows for every head
+// with an online rescale across the task's chunks (every warp derives the
+// same running maximum from the chunk's scores); the 8 warps' partial
+// outputs are summed through the staging buffer at the end.  The new key
+// (position ctx) is read from the cache in global memory: the ring copy of
+// its chunk may predate this step's append.
 __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                        unsigned char* ws, Control* ctl, const TaskDesc& d) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, CH = P.chunk;
   constexpr int D = 64;  // head_dim (the plan builder accepts 64 only)
-  const int slot = d.slot_ph & 0xffff;
-  const uint32_t par = (uint32_t)d.slot_ph >> 16;
   const AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
   const int p = sm.ctx[a.b];
-  const int n_old = max(0, min(CH, p - a.c * CH));
-  const bool has_new = (p - a.c * CH) < CH;
-  const int n_keys = n_old + (has_new ? 1 : 0);
+  const int n_chunks = ceil_div(p + 1, CH);
+  const int c0 = a.c * P.attn_split, c1 = min(c0 + P.attn_split, n_chunks);
+  const bool task_new = c1 == n_chunks;  // the task's last chunk holds the new key
   // queries of the group (scaled by 1/sqrt(64)) and the new K/V rows
   const float* q = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D +
                    (size_t)a.g * qpg * D;
   if (ct < qpg * D) sm.aq[ct >> 6][ct & 63] = __ldcg(q + ct) * 0.125f;
-  if (has_new && ct < 16) {
+  if (task_new && ct < 16) {
     const size_t row = (((size_t)d.layer * P.n_slots + sm.slot[a.b]) * Hkv + a.g) * P.max_ctx + p;
     const unsigned char* src = reinterpret_cast<const unsigned char*>(ct < 8 ? P.k_cache : P.v_cache) + row * D * 2;
     sm.anew[ct] = __ldcg(reinterpret_cast<const uint4*>(src) + (ct & 7));
   }
   bar_sync(BAR_COMP, kComputeThreads);
-  wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
-  const unsigned char* vbase = kbase + (size_t)CH * D * 2;
   const unsigned char* knew = reinterpret_cast<const unsigned char*>(&sm.anew[0]);
   const unsigned char* vnew = reinterpret_cast<const unsigned char*>(&sm.anew[8]);
-  // scores: lane = (key kq of 4, 16-byte column slice ci of 8)
-  {
-    const int kq = lane >> 3, ci = lane & 7;
-    float qr[4][8];
+  const int kq = lane >> 3, ci = lane & 7;  // scores: lane = (key kq of 4, 16-byte column slice ci of 8)
+  float qr[4][8];
 #pragma unroll
-    for (int h = 0; h < 4; ++h)
+  for (int h = 0; h < 4; ++h)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) qr[h][j] = h < qpg ? sm.aq[h][ci * 8 + j] : 0.f;
+    for (int j = 0; j < 8; ++j) qr[h][j] = h < qpg ? sm.aq[h][ci * 8 + j] : 0.f;
+  const int hp = lane >> 3, j8 = lane & 7;  // probabilities: lane = (head hp, key j8 of this warp's 8)
+  float M[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running maximum per head (same in every warp)
+  float L[4] = {0.f, 0.f, 0.f, 0.f};                          // this warp's running exp-sum per head
+  float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int cc = c0; cc < c1; ++cc) {
+    uint32_t par;
+    const int slot = task_slot(d, cc - c0, P.ring_slots, par);
+    const int n_old = max(0, min(CH, p - cc * CH));
+    const bool has_new = (p - cc * CH) < CH;
+    const int n_keys = n_old + (has_new ? 1 : 0);
+    wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
+    const unsigned char* vbase = kbase + (size_t)CH * D * 2;
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       const int kk = 8 * w + 4 * pass + kq;
       const unsigned char* row = (has_new && kk == n_old) ? knew : kbase + (size_t)kk * D * 2;
       float kf[8];
       bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + ci * 16), kf);
-      float s[4];
+      float sc[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         float acc = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc = fmaf(kf[j], qr[h][j], acc);
-        s[h] = acc;
+        sc[h] = acc;
       }
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1)
 #pragma unroll
-        for (int h = 0; h < 4; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], o);
-      const float mine = ci == 0 ? s[0] : ci == 1 ? s[1] : ci == 2 ? s[2] : s[3];
+        for (int h = 0; h < 4; ++h) sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], o);
+      const float mine = ci == 0 ? sc[0] : ci == 1 ? sc[1] : ci == 2 ? sc[2] : sc[3];
       if (ci < qpg) sm.asc[ci][kk] = kk < n_keys ? mine : -INFINITY;
     }
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  // softmax statistics of the chunk, per head (every warp computes them)
-  float M[4];
+    bar_sync(BAR_COMP, kComputeThreads);
+    // the chunk's maximum per head joins the running maximum; earlier sums rescale
+    float scale[4];
 #pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    float m = -INFINITY;
-    if (h < qpg) m = fmaxf(sm.asc[h][lane], sm.asc[h][lane + 32]);
+    for (int h = 0; h < 4; ++h) {
+      float m = -INFINITY;
+      if (h < qpg) m = fmaxf(sm.asc[h][lane], sm.asc[h][lane + 32]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    M[h] = m;
-  }
-  // lane = (head hp, key j of this warp's 8): its probability
-  const int hp = lane >> 3, j = lane & 7;
-  const float Mh = hp == 0 ? M[0] : hp == 1 ? M[1] : hp == 2 ? M[2] : M[3];
-  float pl = (hp < qpg && 8 * w + j < n_keys) ? expf(sm.asc[hp][8 * w + j] - Mh) : 0.f;
-  float ls = pl;
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const float mn = fmaxf(M[h], m);
+      scale[h] = h < qpg ? expf(M[h] - mn) : 0.f;  // 0 on the first chunk (M = -inf, mn finite)
+      M[h] = mn;
+    }
+    const float Mh = hp == 0 ? M[0] : hp == 1 ? M[1] : hp == 2 ? M[2] : M[3];
+    const float pl = (hp < qpg && 8 * w + j8 < n_keys) ? expf(sm.asc[hp][8 * w + j8] - Mh) : 0.f;
+    float ls = pl;
 #pragma unroll
-  for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-  if (j == 0 && hp < qpg) sm.alsum[w][hp] = ls;
-  // P.V over this warp's keys: lane = output columns 2*lane, 2*lane + 1
-  float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    const int kk = 8 * w + jj;
-    if (kk < n_keys) {
-      const unsigned char* row = (has_new && kk == n_old) ? vnew : vbase + (size_t)kk * D * 2;
-      const uint32_t v2 = *reinterpret_cast<const uint32_t*>(row + lane * 4);
-      const float va = __uint_as_float(v2 << 16), vb = __uint_as_float(v2 & 0xffff0000u);
+    for (int h = 0; h < 4; ++h) {
+      L[h] = L[h] * scale[h] + __shfl_sync(0xffffffffu, ls, 8 * h);
+      o0[h] *= scale[h];
+      o1[h] *= scale[h];
+    }
+    // P.V over this warp's keys: lane = output columns 2*lane, 2*lane + 1
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float ph = __shfl_sync(0xffffffffu, pl, h * 8 + jj);
-        o0[h] = fmaf(ph, va, o0[h]);
-        o1[h] = fmaf(ph, vb, o1[h]);
+    for (int jj = 0; jj < 8; ++jj) {
+      const int kk = 8 * w + jj;
+      if (kk < n_keys) {
+        const unsigned char* row = (has_new && kk == n_old) ? vnew : vbase + (size_t)kk * D * 2;
+        const uint32_t v2 = *reinterpret_cast<const uint32_t*>(row + lane * 4);
+        const float va = __uint_as_float(v2 << 16), vb = __uint_as_float(v2 & 0xffff0000u);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float ph = __shfl_sync(0xffffffffu, pl, h * 8 + jj);
+          o0[h] = fmaf(ph, va, o0[h]);
+          o1[h] = fmaf(ph, vb, o1[h]);
+        }
       }
     }
+    bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the scores and the slot's K and V rows
+    if (ct == 0) mbar_arrive(&sm.empty[slot]);
   }
-  __syncwarp();
-  if (lane == 0) release_share(sm, slot, kComputeWarps, w);  // every warp has read its K and V rows
-  // the 8 warps' partial outputs, [w][h][64] in the staging buffer
+  // the 8 warps' partial outputs, [w][h][64] in the staging buffer, and sums
   float* ob = sm.xs();
 #pragma unroll
   for (int h = 0; h < 4; ++h)
-    if (h < qpg) *reinterpret_cast<float2*>(ob + (w * 4 + h) * D + 2 * lane) = make_float2(o0[h], o1[h]);
+    if (h < qpg) {
+      *reinterpret_cast<float2*>(ob + (w * 4 + h) * D + 2 * lane) = make_float2(o0[h], o1[h]);
+      if (lane == 0) sm.alsum[w][h] = L[h];
+    }
   bar_sync(BAR_COMP, kComputeThreads);
   if (ct < qpg * D) {
     const int h = ct >> 6, dd = ct & 63;  // h is uniform in a warp
@@ -1512,11 +1639,11 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
                   (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2)) + h * (D + 2);
     part[dd] = O;
     if (dd == 0) {
-      float L = 0.f;
+      float Ls = 0.f;
 #pragma unroll
-      for (int ww = 0; ww < kComputeWarps; ++ww) L += sm.alsum[ww][h];
+      for (int ww = 0; ww < kComputeWarps; ++ww) Ls += sm.alsum[ww][h];
       part[D] = h == 0 ? M[0] : h == 1 ? M[1] : h == 2 ? M[2] : M[3];
-      part[D + 1] = L;
+      part[D + 1] = Ls;
     }
   }
 }
@@ -1563,6 +1690,278 @@ __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S
   }
   float* out = reinterpret_cast<float*>(ws + P.off_attn) + (size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D;
   out[dd] = O / L;
+  if (P.wide)  // the O projection's B operand
+    reinterpret_cast<__nv_bfloat16*>(ws + P.off_attn_bf)[(size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D + dd] =
+        __float2bfloat16_rn(O / L);
+}
+
+// ---------------------------------------------------------------- wide batch
+// (max_batch > 8.)  The normalised activations are materialised in bf16 by
+// NORM tasks, and every projection is a tcgen05 GEMM task: 128 weight rows
+// (the MMA's M) x the batch (N = B rounded up to 16) over K in 64-column
+// chunks.  The weight chunks stream through the ring from the producer, ahead
+// of the task's event; the activation chunks are loaded by the MMA-issuing
+// thread itself, after the event fired (the controller released the task),
+// into kBStages stages of the staging buffer.
+
+// NORM / NORM2 / NORMF: warp w takes batch row 8 idx + w: the residual (NORM
+// and NORMF add the previous layer's down-projection partials in a fixed
+// order; NORM stores the sum back as the residual), then RMSNorm times the
+// gain, stored as bf16 for the GEMM tasks.
+__device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S, unsigned char* ws,
+                                          const TaskDesc& d) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int b = d.idx * 8 + w, H = P.hidden, nblk = H >> 8;
+  if (b >= S.B) return;
+  const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
+  const int lx = d.op == OP_NORMF ? P.n_layers : d.layer;
+  const bool parts = d.op != OP_NORM2 && lx > 0;
+  const void* gp = d.op == OP_NORM ? layers[d.layer].attn_norm : d.op == OP_NORM2 ? layers[d.layer].ffn_norm
+                                                                                   : P.final_norm;
+  float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
+  const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H;
+  float v[kMaxBlk][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxBlk; ++i)
+    if (i < nblk) {
+      const int c = 256 * i + 8 * lane;
+      float4 a = __ldcg(reinterpret_cast<const float4*>(x + c)), e = __ldcg(reinterpret_cast<const float4*>(x + c) + 1);
+      if (parts)
+        for (int kc = 0; kc < P.n_kc; ++kc) {
+          const float4* d4 = reinterpret_cast<const float4*>(dp + (size_t)kc * P.max_batch * H + c);
+          const float4 p0 = __ldcg(d4), p1 = __ldcg(d4 + 1);
+          a.x += p0.x; a.y += p0.y; a.z += p0.z; a.w += p0.w;
+          e.x += p1.x; e.y += p1.y; e.z += p1.z; e.w += p1.w;
+        }
+      v[i][0] = a.x; v[i][1] = a.y; v[i][2] = a.z; v[i][3] = a.w;
+      v[i][4] = e.x; v[i][5] = e.y; v[i][6] = e.z; v[i][7] = e.w;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss += v[i][j] * v[i][j];
+      if (d.op == OP_NORM && parts) {
+        reinterpret_cast<float4*>(x + c)[0] = a;
+        reinterpret_cast<float4*>(x + c)[1] = e;
+      }
+      // debug capture: the residual after layer lx - 1
+      if (S.cap_resid && lx > 0) {
+        float4* c4 = reinterpret_cast<float4*>(S.cap_resid + ((size_t)(lx - 1) * S.B + b) * H + c);
+        c4[0] = a;
+        c4[1] = e;
+      }
+    }
+  const float inv = 1.0f / sqrtf(warp_sum(ss) / (float)H + P.eps);
+  __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + P.off_xn) + (size_t)b * H;
+#pragma unroll
+  for (int i = 0; i < kMaxBlk; ++i)
+    if (i < nblk) {
+      const int c = 256 * i + 8 * lane;
+      float gf[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(gp) + c / 8), gf);
+      __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(v[i][j] * inv * gf[j]);
+      *reinterpret_cast<uint4*>(xn + c) = *reinterpret_cast<const uint4*>(o);
+    }
+}
+
+// MMA issue of a wide-batch GEMM task (one thread): per chunk c the task's
+// weight slots (parts of them) from the ring and activation chunk c (act_rows
+// rows x 64 columns, columns x0 + 64c of the activation buffer) from stage
+// (bq + c) % kBStages of the staging buffer; the chunk for c + kBStages - 1
+// is loaded once the MMAs of chunk c - 1 released its stage.
+__device__ __forceinline__ void gemm_issue_wide(const DevPlan& P, Smem& sm, unsigned char* ring, Control* ctl,
+                                                const TaskDesc& d, const void* bmap, int x0, int nk, int parts,
+                                                int N, uint32_t& bq) {
+  const int R = P.ring_slots;
+  const uint32_t idesc = umma_idesc_bf16(kWideRows, N);
+  const uint32_t tm = sm.tmem_base;
+  const uint32_t bbytes = (uint32_t)P.act_rows * 128u;
+  unsigned char* stages = sm.stage();
+  const uint32_t u0 = bq;
+  auto load_b = [&](int c) {
+    const uint32_t u = u0 + (uint32_t)c;
+    const int st = (int)(u % kBStages);
+    if (u >= kBStages) wait_local(&sm.bempty[st], ((u / kBStages) - 1) & 1u, P.spin_timeout_ns);
+    mbar_arrive_expect_tx(&sm.bfull[st], bbytes);
+    tma_load_2d(stages + (size_t)st * bbytes, bmap, x0 + c * 64, 0, &sm.bfull[st]);
+  };
+  // the activation was written by other SMs' generic stores, ordered before
+  // this thread by the task's event (the controller's acquire, then the
+  // release to the compute warps); order that view before the TMA reads
+  fence_proxy_async_global();
+  for (int c = 0; c < min(kBStages - 1, nk); ++c) load_b(c);
+  for (int c = 0; c < nk; ++c) {
+    if (c + kBStages - 1 < nk) load_b(c + kBStages - 1);
+    int sl[2];
+    for (int q = 0; q < parts; ++q) {
+      uint32_t par;
+      sl[q] = task_slot(d, parts * c + q, R, par);
+      wait_mbar(&sm.full[sl[q]], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    }
+    const uint32_t u = u0 + (uint32_t)c;
+    const int st = (int)(u % kBStages);
+    wait_mbar(&sm.bfull[st], (u / kBStages) & 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    tc_fence_after();
+    const uint64_t b = umma_desc_sw128(stages + (size_t)st * bbytes);
+    for (int q = 0; q < parts; ++q) {
+      const uint64_t a = umma_desc_sw128(ring + (size_t)sl[q] * P.slot_bytes);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) umma_bf16(tm + 128u * q, a + 2u * k, b + 2u * k, idesc, (c | k) ? 1u : 0u);
+    }
+    for (int q = 0; q < parts; ++q) umma_commit(&sm.empty[sl[q]]);
+    umma_commit(&sm.bempty[st]);
+  }
+  bq = u0 + (uint32_t)nk;
+  umma_commit(&sm.acc_bar);
+}
+
+// A wide-batch GEMM task: QKV (+ RoPE, KV append), O projection (+ residual),
+// gate/up (+ SwiGLU), down (K segment partial) or LM head (+ logits and
+// running argmax).  Lane quadrant q of the accumulator = weight rows 32q ..
+// 32q + 31 of the tile; the two warps of a quadrant split the batch columns.
+__device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
+                                               unsigned char* ws, Control* ctl, const TaskDesc& d, uint32_t& tc_n,
+                                               uint32_t& bq) {
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
+  const int B = S.B, H = P.hidden, D = P.head_dim;
+  const int N = ceil_div(B, 16) * 16;
+  const unsigned char* gmaps = ws + P.off_tmap + (size_t)P.n_layers * kTmapPerLayer * kTmapBytes;
+  const void* xn_map = gmaps + (size_t)TMG_XN * kTmapBytes;
+  int x0 = 0, nk = H / 64, parts = 1;
+  const void* bmap = xn_map;
+  if (d.op == OP_OPROJ) bmap = gmaps + (size_t)TMG_ATTN * kTmapBytes;
+  if (d.op == OP_GATEUP) parts = 2;
+  if (d.op == OP_DOWN) {
+    bmap = gmaps + (size_t)TMG_H * kTmapBytes;
+    x0 = (d.idx / P.n_dtiles) * P.kseg;
+    nk = P.kseg / 64;
+  }
+  if (w == 0) {
+    if (lane == 0) gemm_issue_wide(P, sm, ring, ctl, d, bmap, x0, nk, parts, N, bq);
+    __syncwarp();
+  }
+  wait_local(&sm.acc_bar, tc_n & 1u, P.spin_timeout_ns);
+  tc_n++;
+  tc_fence_after();
+  const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant = weight rows 32q .. 32q + 31
+  const int r = 32 * q + lane;           // this lane's row of the tile
+  const uint32_t ta = S_tmem_lane(sm.tmem_base, q);
+  const int cb0 = (w >> 2) * (N / 2), cb1 = cb0 + N / 2;  // this warp's batch columns
+  switch (d.op) {
+    case OP_QKV: {
+      // a tile is two heads (q, k or v rows); rotate-half pairs (j, j + 32)
+      // of a head sit in quadrants (0, 1) and (2, 3): the odd quadrants hand
+      // their values over through the staging buffer
+      const int nq = P.n_q_heads * D / kWideRows, nkv = P.n_kv_heads * D / kWideRows;
+      const int kind = d.idx < nq ? 0 : d.idx < nq + nkv ? 1 : 2;
+      const int h0 = 2 * (d.idx - (kind == 0 ? 0 : kind == 1 ? nq : nq + nkv));
+      float* xch = sm.xs();  // [64][act_rows]
+      if (q & 1)
+        for (int c8 = cb0; c8 < cb1; c8 += 8) {
+          float v[8];
+          tmem_ld8(ta + (uint32_t)c8, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) xch[((q >> 1) * 32 + lane) * P.act_rows + c8 + i] = v[i];
+        }
+      tc_fence_before();
+      bar_sync(BAR_COMP, kComputeThreads);
+      if (!(q & 1)) {
+        const int hh = h0 + (q >> 1), j = lane;
+        for (int c8 = cb0; c8 < cb1; c8 += 8) {
+          float v[8];
+          tmem_ld8(ta + (uint32_t)c8, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int b = c8 + i;
+            if (b >= B) break;
+            const float v0 = v[i], v1 = xch[((q >> 1) * 32 + lane) * P.act_rows + b];
+            const int pos = sm.ctx[b];
+            if (kind == 2) {
+              const size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + hh) * P.max_ctx + pos;
+              __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(P.v_cache) + row * D;
+              vc[j] = __float2bfloat16_rn(v0);
+              vc[j + 32] = __float2bfloat16_rn(v1);
+            } else {
+              const float2 cs = __ldg(reinterpret_cast<const float2*>(ws + P.off_rope) + (size_t)pos * 32 + j);
+              const float x0r = v0 * cs.x - v1 * cs.y, x1r = v1 * cs.x + v0 * cs.y;
+              if (kind == 0) {
+                float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * D + hh * D;
+                qb[j] = x0r;
+                qb[j + 32] = x1r;
+              } else {
+                const size_t row = (((size_t)d.layer * P.n_slots + sm.slot[b]) * P.n_kv_heads + hh) * P.max_ctx + pos;
+                __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(P.k_cache) + row * D;
+                kc[j] = __float2bfloat16_rn(x0r);
+                kc[j + 32] = __float2bfloat16_rn(x1r);
+              }
+            }
+          }
+        }
+      }
+    } break;
+    case OP_OPROJ: {
+      float* x = reinterpret_cast<float*>(ws + P.off_x);
+      const int col = d.idx * kWideRows + r;
+      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+        float v[8];
+        tmem_ld8(ta + (uint32_t)c8, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (c8 + i < B) x[(size_t)(c8 + i) * H + col] += v[i];
+      }
+    } break;
+    case OP_GATEUP: {
+      __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_h_bf);
+      const int col = d.idx * kWideRows + r;
+      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+        float g[8], u[8];
+        tmem_ld8(ta + (uint32_t)c8, g);
+        tmem_ld8(ta + 128u + (uint32_t)c8, u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (c8 + i < B) hb[(size_t)(c8 + i) * P.ffn + col] = __float2bfloat16_rn(g[i] / (1.0f + expf(-g[i])) * u[i]);
+      }
+    } break;
+    case OP_DOWN: {
+      const int kc = d.idx / P.n_dtiles, col = (d.idx - kc * P.n_dtiles) * kWideRows + r;
+      float* dp = reinterpret_cast<float*>(ws + P.off_dpart) + (size_t)kc * P.max_batch * H;
+      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+        float v[8];
+        tmem_ld8(ta + (uint32_t)c8, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (c8 + i < B) dp[(size_t)(c8 + i) * H + col] = v[i];
+      }
+    } break;
+    case OP_LM: {
+      // logits of vocabulary row `row`; per batch column the warp's best
+      // (logit, id) key, published with an atomic max when it beats the
+      // running maximum (order independent)
+      const int row = d.idx * kWideRows + r;
+      const bool in = row < P.vocab;
+      unsigned long long* best = reinterpret_cast<unsigned long long*>(ws + P.off_lmbest);
+      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+        float v[8];
+        tmem_ld8(ta + (uint32_t)c8, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int b = c8 + i;
+          if (b >= B) break;
+          if (S.logits && in) S.logits[(size_t)b * P.vocab + row] = v[i];
+          unsigned long long key = in ? argmax_key(v[i], row) : 0ull;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+            key = other > key ? other : key;
+          }
+          if (lane == 0 && key > __ldcg(best + b)) atomicMax(best + b, key);
+        }
+      }
+    } break;
+    default: break;
+  }
+  tc_fence_before();
+  bar_sync(BAR_COMP, kComputeThreads);  // the accumulator and the staging buffer are free for the next task
 }
 
 // ---------------------------------------------------------------- MoE layer
@@ -1617,6 +2016,9 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
 #pragma unroll
           for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(v[i][j] * inv * gf[j]);
           *reinterpret_cast<uint4*>(xhat + (size_t)t * H + 256 * i + 8 * lane) = *reinterpret_cast<const uint4*>(o);
+          if (S.cap_moe_in)
+            *reinterpret_cast<uint4*>(S.cap_moe_in + ((size_t)d.layer * T + t) * H + 256 * i + 8 * lane) =
+                *reinterpret_cast<const uint4*>(o);
         }
     }
   }
@@ -1653,9 +2055,11 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
   if (t >= T) return;
   const bool has0 = lane < E, has1 = lane + 32 < E;
   const float v0 = has0 ? lg[w * 64 + lane] : 0.f, v1 = has1 ? lg[w * 64 + lane + 32] : 0.f;
+  // debug outputs: the MoE decoder's hold one block per layer
+  const size_t lblk = dec ? (size_t)d.layer : 0;
   if (S.dbg_logits) {
-    if (has0) S.dbg_logits[(size_t)t * E + lane] = v0;
-    if (has1) S.dbg_logits[(size_t)t * E + lane + 32] = v1;
+    if (has0) S.dbg_logits[(lblk * T + t) * E + lane] = v0;
+    if (has1) S.dbg_logits[(lblk * T + t) * E + lane + 32] = v1;
   }
   bool av0 = has0, av1 = has1;
   int sel_e = 0;
@@ -1676,15 +2080,25 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
   const float mx = __shfl_sync(0xffffffffu, sel_v, 0);  // the first selection is the largest
   const float ex = lane < K ? expf(sel_v - mx) : 0.f;
   const float sum = warp_sum(ex);
+  int rank = 0;
   if (lane < K) {
     const float wt = ex / sum;
     const size_t pi = (size_t)t * K + lane;
-    const int rank = atomicAdd(reinterpret_cast<int*>(mb + P.off_mhist) + sel_e, 1);
+    rank = atomicAdd(reinterpret_cast<int*>(mb + P.off_mhist) + sel_e, 1);
     reinterpret_cast<int*>(mb + P.off_mrank)[pi] = rank;
     reinterpret_cast<int*>(mb + P.off_midx)[pi] = sel_e;
     reinterpret_cast<float*>(mb + P.off_mw)[pi] = wt;
-    if (S.dbg_idx) S.dbg_idx[pi] = sel_e;
-    if (S.dbg_w) S.dbg_w[pi] = wt;
+    if (S.dbg_idx) S.dbg_idx[lblk * T * K + pi] = sel_e;
+    if (S.dbg_w) S.dbg_w[lblk * T * K + pi] = wt;
+  }
+  // grouping: the token's row goes to each selected expert's rows of the
+  // routed-row buffer, at the pair's rank there (each GroupGEMM tile then
+  // loads its B operand as one box of consecutive rows)
+  uint4* xg = reinterpret_cast<uint4*>(mb + P.off_mxg);
+  const size_t dst_row = lane < K ? ((size_t)sel_e * P.moe_cap + rank) * (H / 8) : 0;  // lane j: pair j's row
+  for (int i = 0; i < nblk; ++i) {
+    const uint4 v = __ldcg(xr + (size_t)t * (H / 8) + 32 * i + lane);
+    for (int j = 0; j < K; ++j) xg[__shfl_sync(0xffffffffu, dst_row, j) + 32 * i + lane] = v;
   }
 }
 
@@ -1698,7 +2112,10 @@ __device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams&
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int E = P.n_experts, K = P.top_k, TMt = P.moe_tm;
   unsigned char* mb = moe_block(P, ws, d.layer);
-  int* sx = reinterpret_cast<int*>(sm.xs());  // exp_indptr [E + 1]
+  int* sx = reinterpret_cast<int*>(sm.xs());  // exp_indptr [E + 1], then the tile count
+  const size_t lblk = P.kind == MK_MODEL_MOE_DECODER ? (size_t)d.layer : 0;
+  int* dbg_hist = S.dbg_hist ? S.dbg_hist + lblk * E : nullptr;
+  int* dbg_indptr = S.dbg_indptr ? S.dbg_indptr + lblk * (E + 1) : nullptr;
   bar_sync(BAR_COMP, kComputeThreads);
   if (w == 0) {
     const int* hist = reinterpret_cast<const int*>(mb + P.off_mhist);
@@ -1721,24 +2138,31 @@ __device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams&
     if (lane < E) {
       indptr[lane] = ex0; sx[lane] = ex0; tptr[lane] = tx0;
       for (int m = 0; m < c0; ++m) { tile_e[tx0 + m] = lane; tile_m[tx0 + m] = m; }
-      if (S.dbg_hist) S.dbg_hist[lane] = h0;
-      if (S.dbg_indptr) S.dbg_indptr[lane] = ex0;
+      if (dbg_hist) dbg_hist[lane] = h0;
+      if (dbg_indptr) dbg_indptr[lane] = ex0;
     }
     if (lane + 32 < E) {
       indptr[lane + 32] = ex1; sx[lane + 32] = ex1; tptr[lane + 32] = tx1;
       for (int m = 0; m < c1; ++m) { tile_e[tx1 + m] = lane + 32; tile_m[tx1 + m] = m; }
-      if (S.dbg_hist) S.dbg_hist[lane + 32] = h1;
-      if (S.dbg_indptr) S.dbg_indptr[lane + 32] = ex1;
+      if (dbg_hist) dbg_hist[lane + 32] = h1;
+      if (dbg_indptr) dbg_indptr[lane + 32] = ex1;
     }
     if (lane == 31) {
       const int rows = tot_h0 + s1, tiles = tot_c0 + u1;
-      indptr[E] = rows; sx[E] = rows; tptr[E] = tiles;
-      if (S.dbg_indptr) S.dbg_indptr[E] = rows;
+      indptr[E] = rows; sx[E] = rows; tptr[E] = tiles; sx[E + 1] = tiles;
+      if (dbg_indptr) dbg_indptr[E] = rows;
       // data-dependent event count: every down task of every tile notifies EV_MY
       atomicExch(reinterpret_cast<int*>(ws + P.off_counters) + ev_ctr(P, EV_MY, moe_li(d.layer)), tiles * P.nt_d);
     }
   }
   bar_sync(BAR_COMP, kComputeThreads);
+  // data-dependent event update: the tiles the routing created wait for their
+  // gate/up tasks (the elements past them stay armed at zero); the GroupGEMM
+  // tasks are pushed only after this task's notify, which releases these writes
+  {
+    int* ctr = reinterpret_cast<int*>(ws + P.off_counters);
+    for (int t = ct; t < sx[E + 1]; t += kComputeThreads) atomicExch(ctr + ev_ctr(P, EV_MH, moe_li(d.layer), t), P.nt_gu);
+  }
   const int* midx = reinterpret_cast<const int*>(mb + P.off_midx);
   const int* mrank = reinterpret_cast<const int*>(mb + P.off_mrank);
   int* mrow = reinterpret_cast<int*>(mb + P.off_mrow);
@@ -1751,243 +2175,111 @@ __device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams&
   }
 }
 
-// A GroupGEMM tile's geometry: expert, first row and row count.
-struct MoeTile { int e, r0, nrows; };
-__device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, const unsigned char* mb, int tile) {
-  MoeTile m;
-  m.e = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_e) + tile);
-  const int mi = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_m) + tile);
-  const int h = __ldcg(reinterpret_cast<const int*>(mb + P.off_mhist) + m.e);
-  m.r0 = __ldcg(reinterpret_cast<const int*>(mb + P.off_mindptr) + m.e) + mi * P.moe_tm;
-  m.nrows = min(P.moe_tm, h - mi * P.moe_tm);
-  return m;
+// ---- GroupGEMM tiles on tcgen05 (5th-generation tensor cores, TMEM accumulators)
+// A tile is up to kMoeTileRows routed rows of one expert; a task multiplies
+// kMoeTaskRows weight rows of that expert (the MMA's M = 128) by the tile's
+// rows (N = 16 or 64, the B operand) over K in 64-column chunks that the
+// producer streams into the ring (see emit).  Compute warp 0's lane 0 issues
+// the MMAs (M 128 x N x 16, bf16 in, fp32 accumulate in TMEM) as the chunks
+// land and releases each slot with tcgen05.commit; the accumulator's
+// completion arrives on acc_bar.  The epilogue reads TMEM: warp quadrant q
+// (hardware warp % 4) owns lanes 32q .. 32q + 31, i.e. weight rows; the two
+// compute warps of a quadrant split the N columns (routed rows).
+
+// Issue the MMAs of one GroupGEMM task (one thread).  Per chunk c of K the
+// task's slots are [A0, (A1,) B]: A0 (and A1 for gate/up, its up rows) are
+// 128 weight rows x 64 columns, B is the tile's N rows x 64 columns.  D0 at
+// TMEM column 0 accumulates A0 . B^T, D1 at column 128 accumulates A1 . B^T.
+__device__ __forceinline__ void moe_issue_mma(const DevPlan& P, Smem& sm, unsigned char* ring, Control* ctl,
+                                              const TaskDesc& d, int nk, int parts, int N) {
+  const int R = P.ring_slots;
+  const uint32_t idesc = umma_idesc_bf16(kMoeTaskRows, N);
+  const uint32_t tm = sm.tmem_base;
+  for (int c = 0; c < nk; ++c) {
+    int sl[3];
+    for (int q = 0; q <= parts; ++q) {
+      uint32_t par;
+      sl[q] = task_slot(d, (parts + 1) * c + q, R, par);
+      wait_mbar(&sm.full[sl[q]], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    }
+    tc_fence_after();
+    const uint64_t b = umma_desc_sw128(ring + (size_t)sl[parts] * P.slot_bytes);
+    for (int q = 0; q < parts; ++q) {
+      const uint64_t a = umma_desc_sw128(ring + (size_t)sl[q] * P.slot_bytes);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) umma_bf16(tm + 128u * q, a + 2u * k, b + 2u * k, idesc, (c | k) ? 1u : 0u);
+    }
+    for (int q = 0; q <= parts; ++q) umma_commit(&sm.empty[sl[q]]);
+  }
+  umma_commit(&sm.acc_bar);
 }
 
-// ---- MoE tensor-core tiles (tiles of >= 16 routed rows): mma_window above
-
-// Readers of the ring slots of an n x (rows of 8) block layout: the slots of
-// one part hold rows [j*rps, (j+1)*rps) of its 16 rows; the warps (m block
-// mb, half nh) read the slots holding rows [8*nh, 8*nh + 8).  Returns the
-// number of readers of slot j and this warp's rank among them.
-__device__ __forceinline__ void half_readers(int j, int rps, int n_mb, int mb, int nh, int& readers, int& rank) {
-  const int lo = j * rps, hi = min((j + 1) * rps, 16);
-  const bool h0 = lo < 8, h1 = hi > 8;
-  readers = n_mb * ((h0 ? 1 : 0) + (h1 ? 1 : 0));
-  rank = (nh == 1 && h0 ? n_mb : 0) + mb;
-}
-
-// EGU task (tile, n) on tensor cores: gate rows and up rows 16n .. 16n+15 of
-// the tile's expert against its routed rows (<= 64, gathered straight from
-// the layer input by the row map).  Warp w computes the 16 x 8 blocks of
-// routed rows 16*(w/2) .. for gate and up columns 8*(w%2) .. of the task, so
-// SwiGLU is applied in registers.
+// EGU task (tile, n): gate rows and up rows n*128 .. n*128 + 127 of the
+// tile's expert against its routed rows (gathered by the routing tasks into
+// the expert's rows of the routed-row buffer) -> SwiGLU, stored as bf16 at the
+// tile's compact rows of the SwiGLU buffer.
 __device__ __forceinline__ void task_egu(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
-                                         unsigned char* ws, Control* ctl, const TaskDesc& d) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int H = P.hidden, K = P.top_k, TN = P.moe_tn;
-  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
-  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int tile = d.idx / P.nt_gu, n = d.idx - tile * P.nt_gu;
+                                         unsigned char* ws, Control* ctl, const TaskDesc& d, uint32_t& tc_n) {
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   unsigned char* mb = moe_block(P, ws, d.layer);
+  const int tile = d.idx / P.nt_gu, n = d.idx - tile * P.nt_gu;
   const MoeTile mt = moe_tile(P, mb, tile);
-  const int rps = P.slot_bytes / (2 * H), spp = (TN + rps - 1) / rps;
-  // warp pairs (w / 2) take the m blocks; when there are fewer than 4, the
-  // spare pairs split K with them (ks parts, added through shared memory)
-  const int n_mb = (mt.nrows + 15) >> 4;
-  const int ks = n_mb == 1 ? 4 : (n_mb == 2 ? 2 : 1);
-  const int pair = w >> 1, nh = w & 1;
-  const int mbk = pair % n_mb, kp = pair / n_mb;
-  const int n_act = n_mb * ks;  // active warp pairs
-  const bool active = pair < n_act;
-  const int nwin = H >> 5, win0 = kp * nwin / ks, win1 = (kp + 1) * nwin / ks;
-  const int jlo = (8 * nh) / rps, jhi = (8 * nh + 7) / rps;  // this warp's slots within each part
-  float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-  const int* mperm = reinterpret_cast<const int*>(mb + P.off_mperm);
-  const __nv_bfloat16* xsrc = P.kind == MK_MODEL_MOE_DECODER
-                                  ? reinterpret_cast<const __nv_bfloat16*>(mb + P.off_mxhat) : S.moe_x;
-  // a tile of at most kMoeStageRows routed rows (small T) stages their A
-  // operand in the staging buffer once, instead of reading it from L2 inside
-  // the K loop
-  const int cpr = H / 8;  // 16-byte chunks per row
-  const bool staged = mt.nrows <= kMoeStageRows;
-  if (staged) {
-    bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the staging buffer
-    for (int i = threadIdx.x - kComputeBase; i < mt.nrows * cpr; i += kComputeThreads) {
-      const int r = i / cpr, c = i - r * cpr;
-      reinterpret_cast<uint4*>(sm.xs())[i] =
-          __ldcg(reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + r) / K) * H) + c);
-    }
-    bar_sync(BAR_COMP, kComputeThreads);
+  const int N = moe_tile_n(mt.nrows);
+  if (w == 0) {
+    if (lane == 0) moe_issue_mma(P, sm, ring, ctl, d, P.hidden / 64, 2, N);
+    __syncwarp();
   }
-  if (active) {
-  for (int part = 0; part < 2; ++part)
-    for (int j = jlo; j <= jhi; ++j) {
-      const int js = s0 + part * spp + j;
-      wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-    }
-  const int row = 8 * nh + g;  // weight row of this lane within each part
-  const int jg = s0 + row / rps, ju = s0 + spp + row / rps;
-  const size_t roff = (size_t)(row % rps) * 2 * H;
-  const uint4* bg = reinterpret_cast<const uint4*>(ring + (size_t)(jg < R ? jg : jg - R) * P.slot_bytes + roff);
-  const uint4* bu = reinterpret_cast<const uint4*>(ring + (size_t)(ju < R ? ju : ju - R) * P.slot_bytes + roff);
-  const int rlo = mbk * 16 + g, rhi = rlo + 8;
-  const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
-  const uint4* alo = !vlo ? nullptr
-                     : staged ? reinterpret_cast<const uint4*>(sm.xs()) + (size_t)rlo * cpr
-                              : reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rlo) / K) * H);
-  const uint4* ahi = vhi ? reinterpret_cast<const uint4*>(xsrc + (size_t)(__ldcg(mperm + mt.r0 + rhi) / K) * H) : nullptr;
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  if (staged) {  // (rows g + 8 lie past the tile's rows)
-#pragma unroll 4
-    for (int wi = win0; wi < win1; ++wi) {
-      const int c = wi * 4 + q;
-      const uint4 ua = vlo ? alo[c] : z;
-      mma_window(ag, ua, z, bg[c]);
-      mma_window(au, ua, z, bu[c]);
-    }
-  } else {
-#pragma unroll 4
-    for (int wi = win0; wi < win1; ++wi) {
-      const int c = wi * 4 + q;  // 16-byte chunk of the row
-      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
-      mma_window(ag, ua, ub, bg[c]);
-      mma_window(au, ua, ub, bu[c]);
-    }
-  }
-  __syncwarp();
-  if (lane == 0)
-    for (int part = 0; part < 2; ++part)
-      for (int j = jlo; j <= jhi; ++j) {
-        int readers, rank;
-        half_readers(j, rps, n_act, pair, nh, readers, rank);
-        const int js = s0 + part * spp + j;
-        release_share(sm, js < R ? js : js - R, readers, rank);
-      }
-  }
-  if (ks > 1) {
-    // K parts 1.. hand their sums to part 0 (the staging buffer as scratch)
-    float* xch = sm.xs();
-    bar_sync(BAR_COMP, kComputeThreads);
-    // entry e = ((kp - 1) * n_mb + mbk) * 2 + nh < (ks - 1) * n_mb * 2 <= 6, 256 floats each (<= 1536 of 2048)
-    if (active && kp > 0) {
-      float* e = xch + ((((kp - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 8;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { e[i] = ag[i]; e[4 + i] = au[i]; }
-    }
-    bar_sync(BAR_COMP, kComputeThreads);
-    if (active && kp == 0)
-      for (int o = 1; o < ks; ++o) {
-        const float* e = xch + ((((o - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 8;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { ag[i] += e[i]; au[i] += e[4 + i]; }
-      }
-  }
-  if (!active || kp > 0) return;
+  wait_local(&sm.acc_bar, tc_n & 1u, P.spin_timeout_ns);
+  tc_n++;
+  tc_fence_after();
+  const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
+  const int col = n * kMoeTaskRows + 32 * q + lane;  // this lane's gate/up row = SwiGLU column
+  const bool ok = col < P.eff;
   __nv_bfloat16* mh = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mh);
-  const int col = n * TN + 8 * nh + 2 * q;
+  const uint32_t ta = S_tmem_lane(sm.tmem_base, q);
+  for (int c8 = (w >> 2) * (N / 2); c8 < ((w >> 2) + 1) * (N / 2); c8 += 8) {
+    float g[8], u[8];
+    tmem_ld8(ta + (uint32_t)c8, g);
+    tmem_ld8(ta + 128u + (uint32_t)c8, u);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = mbk * 16 + g + (i >> 1) * 8;
-    const float gt = ag[i];
-    if (r < mt.nrows) mh[(size_t)(mt.r0 + r) * P.eff + col + (i & 1)] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * au[i]);
+    for (int i = 0; i < 8; ++i)
+      if (ok && c8 + i < mt.nrows)
+        mh[(size_t)(mt.r0 + c8 + i) * P.eff + col] = __float2bfloat16_rn(g[i] / (1.0f + expf(-g[i])) * u[i]);
   }
+  tc_fence_before();
+  bar_sync(BAR_COMP, kComputeThreads);  // the accumulator is free for the next task
 }
 
-// EDOWN task (tile, n) on tensor cores: down rows 16n .. 16n+15 of the tile's
-// expert (expert_ffn long, at a 4 KB pitch in the ring) against the tile's
-// rows of h.  Warp w computes the 16 x 8 block of routed rows 16*(w/2) .. and
-// down rows 8*(w%2) .. over the whole of K.
+// EDOWN task (tile, n): down rows n*128 .. n*128 + 127 of the tile's expert
+// against the tile's SwiGLU rows -> fp32 at the tile's compact rows, columns
+// n*128 .. n*128 + 127, of the expert-output buffer.
 __device__ __forceinline__ void task_edown(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
-                                           unsigned char* ws, Control* ctl, const TaskDesc& d) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int H = P.hidden, FF = P.eff, TD = P.moe_td;
-  const int R = P.ring_slots, s0 = d.slot_ph & 0xffff;
-  const uint32_t p0 = (uint32_t)d.slot_ph >> 16;
-  const int tile = d.idx / P.nt_d, n = d.idx - tile * P.nt_d;
+                                           unsigned char* ws, Control* ctl, const TaskDesc& d, uint32_t& tc_n) {
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   unsigned char* mb = moe_block(P, ws, d.layer);
+  const int tile = d.idx / P.nt_d, n = d.idx - tile * P.nt_d;
   const MoeTile mt = moe_tile(P, mb, tile);
-  const int rps = P.slot_bytes / 4096;
-  const int n_mb = (mt.nrows + 15) >> 4;
-  const int ks = n_mb == 1 ? 4 : (n_mb == 2 ? 2 : 1);  // spare warp pairs split K (see task_egu)
-  const int pair = w >> 1, nh = w & 1;
-  const int mbk = pair % n_mb, kp = pair / n_mb;
-  const int n_act = n_mb * ks;
-  const bool active = pair < n_act;
-  const int nwin = FF >> 5, win0 = kp * nwin / ks, win1 = (kp + 1) * nwin / ks;
-  const int jlo = (8 * nh) / rps, jhi = (8 * nh + 7) / rps;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint4* mh = reinterpret_cast<const uint4*>(mb + P.off_mh);
-  const int cpr = FF / 8;  // 16-byte chunks per row
-  const bool staged = mt.nrows <= kMoeStageRows;  // as in task_egu
-  if (staged) {
-    bar_sync(BAR_COMP, kComputeThreads);
-    for (int i = threadIdx.x - kComputeBase; i < mt.nrows * cpr; i += kComputeThreads)
-      reinterpret_cast<uint4*>(sm.xs())[i] = __ldcg(mh + (size_t)mt.r0 * cpr + i);  // rows r0 .. r0 + nrows - 1
-    bar_sync(BAR_COMP, kComputeThreads);
+  const int N = moe_tile_n(mt.nrows);
+  if (w == 0) {
+    if (lane == 0) moe_issue_mma(P, sm, ring, ctl, d, P.eff / 64, 1, N);
+    __syncwarp();
   }
-  if (active) {
-  for (int j = jlo; j <= jhi; ++j) {
-    const int js = s0 + j;
-    wait_mbar(&sm.full[js < R ? js : js - R], js < R ? p0 : p0 ^ 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
-  }
-  const int row = 8 * nh + g, jr = s0 + row / rps;
-  const uint4* bp = reinterpret_cast<const uint4*>(ring + (size_t)(jr < R ? jr : jr - R) * P.slot_bytes +
-                                                   (size_t)(row % rps) * 4096);
-  const int rlo = mbk * 16 + g, rhi = rlo + 8;
-  const bool vlo = rlo < mt.nrows, vhi = rhi < mt.nrows;
-  const uint4* alo = mh + ((size_t)(mt.r0 + (vlo ? rlo : 0)) * FF) / 8;
-  const uint4* ahi = mh + ((size_t)(mt.r0 + (vhi ? rhi : 0)) * FF) / 8;
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  if (staged) {  // (rows g + 8 lie past the tile's rows)
-    const uint4* slo = reinterpret_cast<const uint4*>(sm.xs()) + (size_t)(vlo ? rlo : 0) * cpr;
-#pragma unroll 4
-    for (int wi = win0; wi < win1; ++wi) {
-      const int c = wi * 4 + q;
-      mma_window(acc, vlo ? slo[c] : z, z, bp[c]);
-    }
-  } else {
-#pragma unroll 4
-    for (int wi = win0; wi < win1; ++wi) {
-      const int c = wi * 4 + q;
-      const uint4 ua = vlo ? __ldcg(alo + c) : z, ub = vhi ? __ldcg(ahi + c) : z;
-      mma_window(acc, ua, ub, bp[c]);
-    }
-  }
-  __syncwarp();
-  if (lane == 0)
-    for (int j = jlo; j <= jhi; ++j) {
-      int readers, rank;
-      half_readers(j, rps, n_act, pair, nh, readers, rank);
-      const int js = s0 + j;
-      release_share(sm, js < R ? js : js - R, readers, rank);
-    }
-  }
-  if (ks > 1) {
-    float* xch = sm.xs();  // entries as in task_egu, 4 floats per lane
-    bar_sync(BAR_COMP, kComputeThreads);
-    if (active && kp > 0) {
-      float* e = xch + ((((kp - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 4;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) e[i] = acc[i];
-    }
-    bar_sync(BAR_COMP, kComputeThreads);
-    if (active && kp == 0)
-      for (int o = 1; o < ks; ++o) {
-        const float* e = xch + ((((o - 1) * n_mb + mbk) * 2 + nh) * 32 + lane) * 4;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += e[i];
-      }
-  }
-  if (!active || kp > 0) return;
+  wait_local(&sm.acc_bar, tc_n & 1u, P.spin_timeout_ns);
+  tc_n++;
+  tc_fence_after();
+  const int q = (threadIdx.x >> 5) & 3;
+  const int col = n * kMoeTaskRows + 32 * q + lane;  // output column (< hidden)
   float* my = reinterpret_cast<float*>(mb + P.off_my);
-  const int col = n * TD + 8 * nh + 2 * q;
+  const uint32_t ta = S_tmem_lane(sm.tmem_base, q);
+  for (int c8 = (w >> 2) * (N / 2); c8 < ((w >> 2) + 1) * (N / 2); c8 += 8) {
+    float v[8];
+    tmem_ld8(ta + (uint32_t)c8, v);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = mbk * 16 + g + (i >> 1) * 8;
-    if (r < mt.nrows) my[(size_t)(mt.r0 + r) * H + col + (i & 1)] = acc[i];
+    for (int i = 0; i < 8; ++i)
+      if (c8 + i < mt.nrows) my[(size_t)(mt.r0 + c8 + i) * P.hidden + col] = v[i];
   }
+  tc_fence_before();
+  bar_sync(BAR_COMP, kComputeThreads);
 }
 
 // COMBINE: warp w takes token 8*idx + w: out[t] = sum_j w[t, j] * y[row(t, j)]
@@ -2039,44 +2331,72 @@ __device__ __forceinline__ void task_combine(const DevPlan& P, const StepParams&
   }
 }
 
+// Kernel instances: the plan kinds (MK_MODEL_*), and the dense decoder's
+// wide-batch path as an instance of its own.
+constexpr int kKindDenseWide = 3;
+
 template <int kKind>
 __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
                         Control* ctl) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int B = S.B;
   int a_tag = -1;
+  uint32_t tc_n = 0;  // tcgen05 tasks run (the phase of acc_bar)
+  uint32_t bq = 0;    // wide batch: activation chunks the MMA issuer loaded (stage and phase)
+  constexpr bool kWide = kKind == kKindDenseWide;
+  constexpr bool tc = kKind != MK_MODEL_DENSE;
+  if constexpr (tc) {
+    // tensor memory for the tcgen05 accumulators, held for the kernel's lifetime
+    if (w == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc_fence_before();
+    bar_sync(BAR_COMP, kComputeThreads);
+    tc_fence_after();
+  }
   for (uint32_t k = 0;; ++k) {
-    // task k: released into cur[k & 1] as phase k >> 1 of go_bar[k & 1]
-    if (!wait_mbar(&sm.go_bar[k & 1], (k >> 1) & 1, ctl, P.spin_timeout_ns, -1, -1)) break;
+    // task k: released into cur[k & 1] as phase k >> 1 of go_bar[k & 1].  An
+    // abort does not end this wait: the controller always releases either
+    // the task or an END (its own waits are bounded), and every compute warp
+    // must see the same sequence, since the task bodies meet at barriers.
+    if (!wait_local(&sm.go_bar[k & 1], (k >> 1) & 1, P.spin_timeout_ns)) break;
     const TaskDesc d = sm.cur[k & 1];
     if (d.op == OP_END) break;
     uint32_t* trec = (d.rec > 0 && w == 0) ? trace_rec(S, d.rec) : nullptr;
     if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
     GemvSpec g;
     bool moe_task = false;
-    if constexpr (kKind != MK_MODEL_DENSE) {
+    if constexpr (kKind == MK_MODEL_MOE_LAYER || kKind == MK_MODEL_MOE_DECODER) {
       moe_task = d.op >= OP_ROUTE;
       if (d.op == OP_ROUTE) {
         task_route(P, S, sm, ws, d);
       } else if (d.op == OP_MINDPTR) {
         task_mindptr(P, S, sm, ws, d);
       } else if (d.op == OP_EGU) {
-        task_egu(P, S, sm, ring, ws, ctl, d);
+        task_egu(P, S, sm, ring, ws, ctl, d, tc_n);
       } else if (d.op == OP_EDOWN) {
-        task_edown(P, S, sm, ring, ws, ctl, d);
+        task_edown(P, S, sm, ring, ws, ctl, d, tc_n);
       } else if (d.op == OP_COMBINE) {
         task_combine(P, S, ws, d);
       }
     }
     if (kKind == MK_MODEL_MOE_LAYER || moe_task) {
       a_tag = -1;  // MoE tasks use the staging buffer as scratch
-    } else if (gemv_spec(P, d, g)) {
+    } else if (kWide && (d.op == OP_QKV || d.op == OP_OPROJ || d.op == OP_GATEUP || d.op == OP_DOWN ||
+                         d.op == OP_LM)) {
+      if constexpr (kWide) task_gemm_wide(P, S, sm, ring, ws, ctl, d, tc_n, bq);
+    } else if (kWide && (d.op == OP_NORM || d.op == OP_NORM2 || d.op == OP_NORMF)) {
+      if constexpr (kWide) task_norm(P, S, ws, d);
+    } else if (!kWide && gemv_spec(P, d, g)) {
       // all B activation rows are staged together; an unchanged tag reuses them
       const GemvItem it = gemv_item(sm.geo[d.op], B, threadIdx.x - kComputeBase);
       EpiAhead ea;
       gemv_epilogue_ahead(P, sm, ws, d, it, ea);
       if (g.tag != a_tag) {
-        stage_act(P, ws, sm, g, B);
+        // debug capture: the residual after layer l is what QKV of layer l + 1
+        // (the LM head after the last layer) reduces; task 0 of the family writes it
+        float* cap = nullptr;
+        if (S.cap_resid && d.idx == 0 && ((d.op == OP_QKV && d.layer > 0) || d.op == OP_LM))
+          cap = S.cap_resid + (size_t)(d.op == OP_LM ? P.n_layers - 1 : d.layer - 1) * B * P.hidden;
+        stage_act(P, ws, sm, g, B, trec, cap);
         a_tag = g.tag;
       }
       if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
@@ -2087,15 +2407,22 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     } else if (d.op == OP_MERGE) {
       task_merge(P, S, sm, ws, d);
     } else if (d.op == OP_LMFIN) {
-      if (w < B && lane == 0) {
-        unsigned long long k = __ldcg(reinterpret_cast<const unsigned long long*>(ws + P.off_lmbest) + w);
-        S.next_tokens[w] = argmax_key_index(k);
+      for (int b = threadIdx.x - kComputeBase; b < B; b += kComputeThreads) {
+        unsigned long long k = __ldcg(reinterpret_cast<const unsigned long long*>(ws + P.off_lmbest) + b);
+        S.next_tokens[b] = argmax_key_index(k);
       }
     }
     if (trec && lane == 0) trec[TR_CEND] = (uint32_t)global_ns();
     // every lane of the warp has finished its writes before lane 0 arrives
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.done_bar[k & 1]);
+  }
+  if constexpr (tc) {
+    // every MMA completed (each task waited for its accumulator): free the TMEM
+    tc_fence_before();
+    bar_sync(BAR_COMP, kComputeThreads);
+    tc_fence_after();
+    if (w == 0) tmem_dealloc(sm.tmem_base, kTmemCols);
   }
 }
 
@@ -2125,7 +2452,7 @@ __device__ __forceinline__ void arm_events(const DevPlan& P, Smem& sm, const Fam
     int lin = i - P.ev[e].base;
     ExprEnv env{B, sm.ctx, {0, 0, 0}};
     for (int dd = P.ev[e].ndim - 1; dd >= 0; --dd) { env.coord[dd] = lin % P.ev[e].dims[dd]; lin /= P.ev[e].dims[dd]; }
-    counters[i] = expr_eval(code, P.ev[e].count_expr, env);
+    counters[i] = expr_eval(code, P.ev[e].count_expr, env) + (i == P.fault_ctr ? 1 : 0);
   }
 }
 
@@ -2148,7 +2475,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   // ---- prologue: resolve the symbols, arm the Event Tensors, gather embeddings
   const bool moe = P.kind == MK_MODEL_MOE_LAYER;
   if (tid == 0) {
-    sm.bad = moe ? (B < 1 || B > P.max_tokens) : (B < 1 || B > P.max_batch || B > kMaxB);
+    sm.bad = moe ? (B < 1 || B > P.max_tokens) : (B < 1 || B > P.max_batch || B > (P.wide ? kMaxWideBatch : kMaxB));
+    // the ring's slots hold 128-byte-swizzled TMA boxes and tcgen05 operands,
+    // whose swizzle pattern assumes 1024-byte-aligned slots
+    if (smem_u32(smem_raw) & 1023u) sm.bad = 1;
     sm.released = 0;
     sm.dq_head = sm.dq_tail = sm.fq_head = sm.fq_tail = sm.notifier_stop = 0;
   }
@@ -2175,7 +2505,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
       gg.cw = K / kGemvSlots;
       gg.pairs = pairs;
     };
-    if (!moe) {
+    if (!moe && !P.wide) {
       set_geo(OP_QKV, P.hidden, P.tile_qkv / 2, 1);
       set_geo(OP_OPROJ, P.hidden, P.tile_o, 0);
       set_geo(OP_GATEUP, P.hidden, P.tile_gu, 1);
@@ -2184,9 +2514,9 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     }
     if (!moe) {
       int run = 0;
-      for (int b = 0; b < B; ++b) {
+      for (int b = 0; b < B; ++b) {  // attention tasks of sequence b: its key chunks, attn_split at a time
         sm.pre[b] = run;
-        sm.nch[b] = ceil_div(sm.ctx[b] + 1, P.chunk);
+        sm.nch[b] = ceil_div(ceil_div(sm.ctx[b] + 1, P.chunk), P.attn_split);
         run += sm.nch[b];
       }
       sm.pre[B] = run;
@@ -2220,11 +2550,14 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     ctl->q_head = 0;
     ctl->q_tail = 0;
     if (moe) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, -1), 0, ceil_div(B, 8));
+    else if (P.wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, 0), 0, ceil_div(B, 8));  // EV_IN[0] armed at zero
     else push_range(P, S, ctl, ws, fam_of(P, OP_QKV, 0), 0, P.n_qkv_tiles);  // EV_IN[0] is armed at zero
   }
   if (tid == 0) {
-    for (int s = 0; s < P.ring_slots; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], kComputeWarps); }
+    for (int s = 0; s < P.ring_slots; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
     for (int j = 0; j < 2; ++j) { mbar_init(&sm.go_bar[j], 1); mbar_init(&sm.done_bar[j], kComputeWarps); }
+    mbar_init(&sm.acc_bar, 1);
+    for (int j = 0; j < kBStages; ++j) { mbar_init(&sm.bfull[j], 1); mbar_init(&sm.bempty[j], 1); }
     for (int k = 0; k < kFifo; ++k) { mbar_init(&sm.fifo_full[k], 1); mbar_init(&sm.fifo_empty[k], 1); }
     fence_proxy_async_smem();
   }
@@ -2268,7 +2601,7 @@ static const void* kernel_for(const DevPlan& P) {
   switch (P.kind) {
     case MK_MODEL_MOE_LAYER: return (const void*)megakernel<MK_MODEL_MOE_LAYER>;
     case MK_MODEL_MOE_DECODER: return (const void*)megakernel<MK_MODEL_MOE_DECODER>;
-    default: return (const void*)megakernel<MK_MODEL_DENSE>;
+    default: return P.wide ? (const void*)megakernel<kKindDenseWide> : (const void*)megakernel<MK_MODEL_DENSE>;
   }
 }
 
@@ -2308,11 +2641,53 @@ static EncodeTiledFn encode_tiled_fn() {
 // bf16 [rows][cols] matrix with a row stride, read in boxes of (cols / 8)
 // columns x box_rows rows (one box per ring slot and part); rows past the
 // end read as zeros.
-static bool encode_weight_maps(const DevPlan& P, std::vector<unsigned char>& image, std::string& err) {
-  if (P.kind == MK_MODEL_MOE_LAYER) return true;
+static bool encode_weight_maps(const DevPlan& P, const unsigned char* ws, std::vector<unsigned char>& image,
+                               std::string& err) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) { err = "cuTensorMapEncodeTiled is not available"; return false; }
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(image.data() + (P.off_layers - P.off_families));
+  // a bf16 [rows][cols] row-major matrix read in boxes of 64 columns x box_rows
+  // rows under the 128-byte swizzle (the K-major layout of a tcgen05 operand);
+  // rows past the end read as zeros
+  auto put_sw128 = [&](int index, const void* w, long long rows, long long cols, int box_rows,
+                       const char* what) -> bool {
+    if (reinterpret_cast<uintptr_t>(w) & 15) { err = std::string(what) + " must be 16-byte aligned"; return false; }
+    CUtensorMap m;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) { err = std::string("tensor map of ") + what + " rejected by the driver"; return false; }
+    std::memcpy(image.data() + (P.off_tmap - P.off_families) + (size_t)index * kTmapBytes, &m, sizeof(m));
+    return true;
+  };
+  if (P.kind != MK_MODEL_DENSE) {
+    // GroupGEMM operands of every MoE layer: the expert matrices and the
+    // layer's routed-row and SwiGLU buffers in the workspace
+    const int Lm = P.kind == MK_MODEL_MOE_DECODER ? P.n_layers : 1;
+    const long long E = P.n_experts, F = P.eff, H = P.hidden, cap = P.moe_cap, K = P.top_k;
+    for (int l = 0; l < Lm; ++l) {
+      const bool dec = P.kind == MK_MODEL_MOE_DECODER;
+      const void* g = dec ? layers[l].we_gate : P.w_egate;
+      const void* u = dec ? layers[l].we_up : P.w_eup;
+      const void* dn = dec ? layers[l].we_down : P.w_edown;
+      if (!g || !u || !dn) { err = "MoE expert weights missing"; return false; }
+      const unsigned char* blk = ws + P.off_mxg + (size_t)l * P.moe_stride;
+      const unsigned char* hblk = ws + P.off_mh + (size_t)l * P.moe_stride;
+      if (!put_sw128(tmap_index(l, TM_GATE), g, E * F, H, kMoeTaskRows, "expert w_gate") ||
+          !put_sw128(tmap_index(l, TM_UP), u, E * F, H, kMoeTaskRows, "expert w_up") ||
+          !put_sw128(tmap_index(l, TM_DOWN), dn, E * H, F, kMoeTaskRows, "expert w_down") ||
+          !put_sw128(tmap_index(l, TM_XG16), blk, E * cap, H, 16, "routed rows") ||
+          !put_sw128(tmap_index(l, TM_XG64), blk, E * cap, H, kMoeTileRows, "routed rows") ||
+          !put_sw128(tmap_index(l, TM_HG16), hblk, cap * K, F, 16, "SwiGLU rows") ||
+          !put_sw128(tmap_index(l, TM_HG64), hblk, cap * K, F, kMoeTileRows, "SwiGLU rows"))
+        return false;
+    }
+    if (P.kind == MK_MODEL_MOE_LAYER) return true;
+  }
   auto put = [&](int index, const void* w, long long rows, long long cols, long long stride_elems, int box_cols,
                  int box_rows, const char* what) -> bool {
     if (!w) return true;  // (an MoE decoder has no dense FFN)
@@ -2348,6 +2723,26 @@ static bool encode_weight_maps(const DevPlan& P, std::vector<unsigned char>& ima
       { err = "norm gains must be 16-byte aligned"; return false; }
   if (reinterpret_cast<uintptr_t>(P.final_norm) & 15) { err = "final_norm must be 16-byte aligned"; return false; }
   const int H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads, F = P.ffn;
+  if (P.wide) {
+    // wide batch: every matrix in boxes of 64 columns x 128 rows (a tcgen05
+    // A operand per box), the activations in boxes of 64 columns x act_rows
+    const int g0 = P.n_layers * kTmapPerLayer;
+    for (int l = 0; l < P.n_layers; ++l) {
+      const LayerPtrs& lp = layers[l];
+      if (!put_sw128(tmap_index(l, TM_WQ), lp.wq, (long long)Hq * D, H, kWideRows, "wq") ||
+          !put_sw128(tmap_index(l, TM_WK), lp.wk, (long long)Hkv * D, H, kWideRows, "wk") ||
+          !put_sw128(tmap_index(l, TM_WV), lp.wv, (long long)Hkv * D, H, kWideRows, "wv") ||
+          !put_sw128(tmap_index(l, TM_WO), lp.wo, H, (long long)Hq * D, kWideRows, "wo") ||
+          !put_sw128(tmap_index(l, TM_GATE), lp.w_gate, F, H, kWideRows, "w_gate") ||
+          !put_sw128(tmap_index(l, TM_UP), lp.w_up, F, H, kWideRows, "w_up") ||
+          !put_sw128(tmap_index(l, TM_DOWN), lp.w_down, H, F, kWideRows, "w_down"))
+        return false;
+    }
+    return put_sw128(g0 + TMG_LM, P.lm_head, P.vocab, H, kWideRows, "lm_head") &&
+           put_sw128(g0 + TMG_XN, ws + P.off_xn, P.act_rows, H, P.act_rows, "normalised activations") &&
+           put_sw128(g0 + TMG_ATTN, ws + P.off_attn_bf, P.act_rows, H, P.act_rows, "attention output") &&
+           put_sw128(g0 + TMG_H, ws + P.off_h_bf, P.act_rows, F, P.act_rows, "SwiGLU output");
+  }
   for (int l = 0; l < P.n_layers; ++l) {
     const LayerPtrs& lp = layers[l];
     const int bh = H / kGemvSlots;  // columns per slot of a hidden-wide row
@@ -2389,7 +2784,7 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
                    std::string& err) {
   cudaStream_t s = (cudaStream_t)stream;
   std::vector<unsigned char> image = image_in;
-  if (!encode_weight_maps(p.dp, image, err)) return MK_ERR_INVALID_ARG;
+  if (!encode_weight_maps(p.dp, (const unsigned char*)ws, image, err)) return MK_ERR_INVALID_ARG;
   size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + kSmemFixed + p.dp.act_bytes + p.dp.gred_bytes;
   const void* kern = kernel_for(p.dp);
   cudaError_t e = ensure_smem_attr(p.device, kern, (int)smem);
@@ -2412,6 +2807,16 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
   return MK_OK;
 }
 
+// the decode step's debug captures (the MoE decoder's routing captures use the
+// MoE layer's debug outputs, one block per layer)
+static void set_captures(StepParams& sp, const mk_step_args* a) {
+  sp.cap_resid = a->capture_resid;
+  sp.cap_moe_in = reinterpret_cast<__nv_bfloat16*>(a->capture_moe_in);
+  sp.dbg_idx = a->capture_topk;
+  sp.dbg_hist = a->capture_hist;
+  sp.dbg_indptr = a->capture_indptr;
+}
+
 mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& err) {
   StepParams sp = StepParams();
   sp.B = a->batch;
@@ -2424,6 +2829,7 @@ mk_status dev_launch(Plan& p, const mk_step_args* a, void* stream, std::string& 
   sp.trace = (p.dp.debug_flags & MK_DEBUG_TRACE) ? (uint32_t*)a->trace : nullptr;
   sp.trace_cap = a->trace_cap;
   if (sp.trace && sp.trace_cap < 2) sp.trace = nullptr;
+  set_captures(sp, a);
   sp.epoch = p.epoch + 1;
   unsigned char* ws = (unsigned char*)p.ws;
   DevPlan dp = p.dp;
@@ -2470,15 +2876,18 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
 
   std::lock_guard<std::mutex> lock(g_static_mu);
   StaticScratchState& st = g_static[dev];
-  if (!st.addr) {
-    // first call on this device: resolve the array's address with the device current
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
-    if (e != cudaSuccess) {
-      err = std::string("cudaGetSymbolAddress of the static scratch failed: ") + cudaGetErrorString(e);
-      return MK_ERR_CUDA;
-    }
+  // the array's address in this device's context, resolved on every call (a
+  // reset of the context reloads the module, possibly at another address, and
+  // then the plan arrays must be uploaded again)
+  void* ptr = nullptr;
+  e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+  if (e != cudaSuccess) {
+    err = std::string("cudaGetSymbolAddress of the static scratch failed: ") + cudaGetErrorString(e);
+    return MK_ERR_CUDA;
+  }
+  if (st.addr != static_cast<unsigned char*>(ptr)) {
     st.addr = static_cast<unsigned char*>(ptr);
+    st.owner = 0;
   }
   cudaStream_t s = (cudaStream_t)stream;
   unsigned char* ws = st.addr;
@@ -2494,7 +2903,7 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
     // the read-only plan arrays and the weights' tensor maps (host memory only)
     std::vector<unsigned char> image;
     lower_plan(p, image);
-    if (!encode_weight_maps(P0, image, err)) return MK_ERR_INVALID_ARG;
+    if (!encode_weight_maps(P0, ws, image, err)) return MK_ERR_INVALID_ARG;
     if (e == cudaSuccess)
       e = cudaMemcpyAsync(ws + P0.off_families, image.data(), image.size(), cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) { err = std::string("plan upload failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
@@ -2517,6 +2926,7 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   sp.trace = (P0.debug_flags & MK_DEBUG_TRACE) ? (uint32_t*)a->trace : nullptr;
   sp.trace_cap = a->trace_cap;
   if (sp.trace && sp.trace_cap < 2) sp.trace = nullptr;
+  set_captures(sp, a);
   sp.epoch = 1;
   DevPlan dp = P0;
   dp.smem_bytes = (int)smem;
@@ -2524,6 +2934,7 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   e = ensure_smem_attr(p.device, kernel_for(p.dp), (int)smem);
   if (e == cudaSuccess) e = cudaLaunchCooperativeKernel(kernel_for(p.dp), dim3(dp.n_sm), dim3(kThreads), args, smem, s);
   if (e != cudaSuccess) { err = std::string("launch failed: ") + cudaGetErrorString(e); return MK_ERR_CUDA; }
+  p.launches++;
   return MK_OK;
 }
 

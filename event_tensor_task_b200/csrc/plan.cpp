@@ -31,8 +31,9 @@
 
 namespace mk {
 
-static const char* kOpNames[OP_COUNT] = {"end", "qkv", "attn", "merge", "oproj", "gateup", "down", "-", "lm",
-                                         "-", "lmfin", "route", "mindptr", "egu", "edown", "combine", "mfin"};
+static const char* kOpNames[OP_COUNT] = {"end", "qkv", "attn", "merge", "oproj", "gateup", "down", "norm", "lm",
+                                         "norm2", "lmfin", "route", "mindptr", "egu", "edown", "combine", "mfin",
+                                         "normf"};
 static const int kLayerOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_GATEUP, OP_DOWN};
 static const int kLmOps[] = {OP_LM, OP_LMFIN};
 static constexpr int kFamPerLayer = 6;
@@ -52,11 +53,56 @@ int emit_const(std::vector<int32_t>& code, int v) { return Emit(code).push(v).re
 }  // namespace
 
 int Plan::fam_index(int op, int layer) const {
-  if (op == OP_LM) return dp.n_layers * kFamPerLayer;
-  if (op == OP_LMFIN) return dp.n_layers * kFamPerLayer + 1;
-  for (int k = 0; k < kFamPerLayer; ++k)
-    if (kLayerOps[k] == op) return layer * kFamPerLayer + k;
-  return -1;
+  // (as the device's fam_of: the family of (op, layer 0) plus the layer stride)
+  const int f0 = dp.fam_first_layer[op];
+  if (f0 < 0) return -1;
+  return layer < 0 ? f0 : f0 + layer * dp.fam_stride;
+}
+
+int Plan::actual_extent(int f, const Binding& bd) const {
+  const int op = fams[f].op;
+  if (op == OP_EGU || op == OP_EDOWN) {
+    const int li = fams[f].layer < 0 ? 0 : fams[f].layer;
+    if (li >= (int)bd.route.size()) return 0;
+    return bd.route[li].tiles * (op == OP_EGU ? dp.nt_gu : dp.nt_d);
+  }
+  return family_extent(f, bd);
+}
+
+void draw_routing(const Plan& p, Binding& bd, unsigned seed, double skew) {
+  const DevPlan& P = p.dp;
+  bd.route.clear();
+  if (P.kind == MK_MODEL_DENSE) return;
+  const int Lm = P.kind == MK_MODEL_MOE_DECODER ? P.n_layers : 1;
+  const int E = P.n_experts, K = P.top_k, T = bd.B;
+  std::mt19937 rng(seed * 2654435761u + 17u);
+  for (int l = 0; l < Lm; ++l) {
+    MoeRoute r;
+    std::vector<int> perm(E);
+    for (int e = 0; e < E; ++e) perm[e] = e;
+    std::shuffle(perm.begin(), perm.end(), rng);
+    std::vector<double> wt(E);
+    for (int i = 0; i < E; ++i) wt[perm[i]] = skew > 0 ? std::pow((double)(i + 1), -skew) : 1.0;
+    r.idx.resize((size_t)T * K);
+    for (int t = 0; t < T; ++t) {
+      std::vector<double> w = wt;
+      for (int j = 0; j < K; ++j) {  // k distinct experts, drawn by weight without replacement
+        std::discrete_distribution<int> pick(w.begin(), w.end());
+        const int e = pick(rng);
+        r.idx[(size_t)t * K + j] = e;
+        w[e] = 0.0;
+      }
+    }
+    r.hist.assign(E, 0);
+    r.rank.resize(r.idx.size());
+    for (size_t q = 0; q < r.idx.size(); ++q) r.rank[q] = r.hist[r.idx[q]]++;
+    r.indptr.assign(E + 1, 0);
+    for (int e = 0; e < E; ++e) r.indptr[e + 1] = r.indptr[e] + r.hist[e];
+    for (int e = 0; e < E; ++e)
+      for (int m = 0; m < ceil_div(r.hist[e], P.moe_tm); ++m) { r.tile_e.push_back(e); r.tile_m.push_back(m); }
+    r.tiles = (int)r.tile_e.size();
+    bd.route.push_back(std::move(r));
+  }
 }
 
 int Plan::counter(int ev, int c0, int c1, int c2) const {
@@ -85,21 +131,75 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
   t.idx = idx;
   int op = fams[f].op, l = fams[f].layer;
   int B = bd.B, H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads;
-  int qpg = Hq / Hkv, F = P.ffn;
+  int qpg = Hkv > 0 ? Hq / Hkv : 0, F = P.ffn;  // (no attention in an MoE layer plan)
   long long QD = (long long)Hq * D;
   auto kv_row = [&](int layer, int slot, int g, int pos) -> long long {
     return ((((long long)layer * P.n_slots + slot) * Hkv + g) * P.max_ctx + pos) * D;
   };
   // sequence b uses slot b in the host model (slots are distinct by contract)
+  const bool mdec = P.kind == MK_MODEL_MOE_DECODER;
+  // MoE: this family's layer block, its routing and a tile's rows
+  const int li = l < 0 ? 0 : l;
+  const long long maxT = P.max_tokens, Kk = P.top_k;
+  const MoeRoute* rt = (P.kind != MK_MODEL_DENSE && li < (int)bd.route.size()) ? &bd.route[li] : nullptr;
+  auto tile_rows = [&](int tile, int& r0, int& nr) {
+    const int e = rt->tile_e[tile], m = rt->tile_m[tile];
+    r0 = rt->indptr[e] + m * P.moe_tm;
+    nr = std::min(P.moe_tm, rt->hist[e] - m * P.moe_tm);
+  };
+  const bool wide = P.wide != 0;
+  auto nsplit = [&](int b) { return ceil_div(ceil_div(bd.ctx[b] + 1, P.chunk), P.attn_split); };
+  auto rows8 = [&](int i, int& b0, int& b1) { b0 = 8 * i; b1 = std::min(B, 8 * i + 8); };
+  if (wide && op == OP_QKV) {
+    // a 128-row tile of [Wq; Wk; Wv]: two heads of q, k or v rows
+    const int nq = Hq * D / kWideRows, nk = Hkv * D / kWideRows;
+    const int kind = idx < nq ? 0 : idx < nq + nk ? 1 : 2;
+    const int h0 = 2 * (idx - (kind == 0 ? 0 : kind == 1 ? nq : nq + nk));
+    t.wait_ev = counter(EV_N1, l);
+    t.notify_ev = counter(EV_QKV, l, 0);
+    for (int b = 0; b < B; ++b) {
+      t.reads.push_back({BUF_XN, (long long)b * H, (long long)(b + 1) * H});
+      for (int hh = h0; hh < h0 + 2; ++hh) {
+        if (kind == 0) {
+          const long long base = b * QD + (long long)hh * D;
+          t.writes.push_back({BUF_Q, base, base + D});
+        } else {
+          const long long base = kv_row(l, b, hh, bd.ctx[b]);
+          t.writes.push_back({kind == 1 ? BUF_KC : BUF_VC, base, base + D});
+        }
+      }
+    }
+    return;
+  }
   switch (op) {
+    case OP_NORM:
+    case OP_NORM2:
+    case OP_NORMF: {
+      // wide batch: rows 8 idx .. of the residual -> normalised bf16 rows
+      int b0, b1;
+      rows8(idx, b0, b1);
+      const int lx = op == OP_NORMF ? P.n_layers : l;
+      t.wait_ev = op == OP_NORM2 ? counter(EV_O, l) : counter(EV_IN, lx);
+      t.notify_ev = op == OP_NORM ? counter(EV_N1, l) : op == OP_NORM2 ? counter(EV_N2, l) : counter(EV_NF, 0);
+      for (int b = b0; b < b1; ++b) {
+        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        if (op != OP_NORM2 && lx > 0)
+          for (int kc = 0; kc < P.n_kc; ++kc) {
+            const long long pb = ((long long)kc * P.max_batch + b) * H;
+            t.reads.push_back({BUF_DPART, pb, pb + H});
+          }
+        if (op == OP_NORM) t.writes.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        t.writes.push_back({BUF_XN, (long long)b * H, (long long)(b + 1) * H});
+      }
+    } break;
     case OP_QKV: {
       QkvTile q = decode_qkv(P, idx);
-      t.wait_ev = counter(EV_IN, l);
+      t.wait_ev = (mdec && l > 0) ? counter(EV_MCOMB, l - 1) : counter(EV_IN, l);
       t.notify_ev = counter(EV_QKV, l, q.group);
       int half = P.tile_qkv / 2;
       for (int b = 0; b < B; ++b) {
         t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
-        if (l > 0)
+        if (l > 0 && !mdec)
           for (int kc = 0; kc < P.n_kc; ++kc) {
             long long pb = ((long long)kc * P.max_batch + b) * H;
             t.reads.push_back({BUF_DPART, pb, pb + H});
@@ -117,16 +217,17 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       }
     } break;
     case OP_ATTN: {
-      std::vector<int> nch(B), pre(B + 1, 0);
-      for (int b = 0; b < B; ++b) { nch[b] = ceil_div(bd.ctx[b] + 1, P.chunk); pre[b + 1] = pre[b] + nch[b]; }
-      AttnTask a = decode_attn(idx, B, Hkv, nch.data(), pre.data());
-      t.wait_ev = counter(EV_QKV, l, a.g);
+      // task c of (b, g): key chunks c * attn_split .. of the sequence
+      std::vector<int> nsp(B), pre(B + 1, 0);
+      for (int b = 0; b < B; ++b) { nsp[b] = nsplit(b); pre[b + 1] = pre[b] + nsp[b]; }
+      AttnTask a = decode_attn(idx, B, Hkv, nsp.data(), pre.data());
+      t.wait_ev = counter(EV_QKV, l, wide ? 0 : a.g);
       t.notify_ev = counter(EV_CHUNK, l, a.b, a.g);
       t.follow_fam = fam_index(OP_MERGE, l);
       t.follow_idx = a.b * Hkv + a.g;
       long long qb = a.b * QD + (long long)a.g * qpg * D;
       t.reads.push_back({BUF_Q, qb, qb + (long long)qpg * D});
-      int p0 = a.c * P.chunk, p1 = std::min(p0 + P.chunk, bd.ctx[a.b] + 1);
+      int p0 = a.c * P.attn_split * P.chunk, p1 = std::min(p0 + P.attn_split * P.chunk, bd.ctx[a.b] + 1);
       long long kb = kv_row(l, a.b, a.g, p0);
       t.reads.push_back({BUF_KC, kb, kb + (long long)(p1 - p0) * D});
       t.reads.push_back({BUF_VC, kb, kb + (long long)(p1 - p0) * D});
@@ -135,7 +236,7 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
     } break;
     case OP_MERGE: {
       int b = idx / Hkv, g = idx % Hkv;
-      int nch = ceil_div(bd.ctx[b] + 1, P.chunk);
+      int nch = nsplit(b);
       long long pb = ((long long)b * Hkv + g) * P.max_chunks;
       t.reads.push_back({BUF_APART, pb, pb + nch});
       long long ob = b * QD + (long long)g * qpg * D;
@@ -149,7 +250,7 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
         t.reads.push_back({BUF_ATTN, b * QD, (b + 1) * QD});
         long long xb = (long long)b * H + (long long)idx * P.tile_o;
         t.reads.push_back({BUF_X, xb, xb + P.tile_o});
-        if (l > 0)
+        if (l > 0 && !mdec && !wide)
           for (int kc = 0; kc < P.n_kc; ++kc) {
             long long pb = ((long long)kc * P.max_batch + b) * H + (long long)idx * P.tile_o;
             t.reads.push_back({BUF_DPART, pb, pb + P.tile_o});
@@ -158,10 +259,10 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       }
     } break;
     case OP_GATEUP: {
-      t.wait_ev = counter(EV_O, l);
+      t.wait_ev = wide ? counter(EV_N2, l) : counter(EV_O, l);
       t.notify_ev = counter(EV_GU, l, idx * P.tile_gu / P.kseg);
       for (int b = 0; b < B; ++b) {
-        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        t.reads.push_back({wide ? BUF_XN : BUF_X, (long long)b * H, (long long)(b + 1) * H});
         long long hb = (long long)b * F + (long long)idx * P.tile_gu;
         t.writes.push_back({BUF_H, hb, hb + P.tile_gu});
       }
@@ -178,14 +279,14 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       }
     } break;
     case OP_LM: {
-      t.wait_ev = counter(EV_IN, P.n_layers);
+      t.wait_ev = mdec ? counter(EV_MCOMB, P.n_layers - 1) : wide ? counter(EV_NF, 0) : counter(EV_IN, P.n_layers);
       t.notify_ev = counter(EV_LM, 0);
       t.follow_fam = fam_index(OP_LMFIN, -1);
       t.follow_idx = 0;
       int r0 = idx * P.tile_lm, r1 = std::min(P.vocab, r0 + P.tile_lm);
       for (int b = 0; b < B; ++b) {
-        t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
-        for (int kc = 0; kc < P.n_kc; ++kc) {
+        t.reads.push_back({wide ? BUF_XN : BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        for (int kc = 0; kc < (mdec || wide ? 0 : P.n_kc); ++kc) {
           long long pb = ((long long)kc * P.max_batch + b) * H;
           t.reads.push_back({BUF_DPART, pb, pb + H});
         }
@@ -195,7 +296,79 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
     case OP_LMFIN: {
       for (int b = 0; b < B; ++b) t.writes.push_back({BUF_NEXT, b, b + 1});
     } break;
-    default: break;
+    // ---- MoE FFN (T = B tokens; per-layer scratch blocks)
+    case OP_ROUTE: {
+      t.wait_ev = mdec ? counter(EV_O, l) : -1;
+      t.notify_ev = counter(EV_ROUTE, li);
+      t.follow_fam = fam_index(OP_MINDPTR, l);
+      t.follow_idx = 0;
+      for (int tok = 8 * idx; tok < std::min(B, 8 * idx + 8); ++tok) {
+        if (mdec) {
+          t.reads.push_back({BUF_X, (long long)tok * H, (long long)(tok + 1) * H});
+          t.writes.push_back({BUF_MXHAT, (li * maxT + tok) * H, (li * maxT + tok + 1) * H});
+        }
+        t.writes.push_back({BUF_MPAIR, (li * maxT + tok) * Kk, (li * maxT + tok + 1) * Kk});
+        for (int j = 0; j < P.top_k; ++j) {  // the token's row copy in each selected expert's rows
+          const size_t q = (size_t)tok * P.top_k + j;
+          const long long row = ((long long)li * P.n_experts + rt->idx[q]) * P.moe_cap + rt->rank[q];
+          t.writes.push_back({BUF_MXG, row * H, (row + 1) * H});
+        }
+      }
+    } break;
+    case OP_MINDPTR: {
+      t.notify_ev = counter(EV_MIDX, li);
+      t.reads.push_back({BUF_MPAIR, li * maxT * Kk, li * maxT * Kk + (long long)B * Kk});
+      t.writes.push_back({BUF_MTAB, li, li + 1});
+    } break;
+    case OP_EGU: {
+      const int tile = idx / P.nt_gu, n = idx % P.nt_gu;
+      int r0, nr;
+      tile_rows(tile, r0, nr);
+      t.notify_ev = counter(EV_MH, li, tile);
+      t.reads.push_back({BUF_MTAB, li, li + 1});
+      {  // the tile's routed token rows
+        const long long row = ((long long)li * P.n_experts + rt->tile_e[tile]) * P.moe_cap + rt->tile_m[tile] * P.moe_tm;
+        t.reads.push_back({BUF_MXG, row * H, (row + nr) * H});
+      }
+      const long long c0 = (long long)n * P.moe_tn, c1 = std::min<long long>(P.eff, c0 + P.moe_tn);
+      for (int r = r0; r < r0 + nr; ++r) {
+        const long long rb = (li * maxT * Kk + r) * P.eff;
+        t.writes.push_back({BUF_MH, rb + c0, rb + c1});
+      }
+    } break;
+    case OP_EDOWN: {
+      const int tile = idx / P.nt_d, n = idx % P.nt_d;
+      int r0, nr;
+      tile_rows(tile, r0, nr);
+      t.wait_ev = counter(EV_MH, li, tile);
+      t.notify_ev = counter(EV_MY, li);
+      t.reads.push_back({BUF_MTAB, li, li + 1});
+      t.reads.push_back({BUF_MH, (li * maxT * Kk + r0) * P.eff, (li * maxT * Kk + r0 + nr) * P.eff});
+      for (int r = r0; r < r0 + nr; ++r) {
+        const long long rb = (li * maxT * Kk + r) * H + (long long)n * P.moe_td;
+        t.writes.push_back({BUF_MY, rb, rb + P.moe_td});
+      }
+    } break;
+    case OP_COMBINE: {
+      t.wait_ev = counter(EV_MY, li);
+      t.notify_ev = counter(EV_MCOMB, li);
+      if (!mdec) { t.follow_fam = fam_index(OP_MFIN, -1); t.follow_idx = 0; }
+      t.reads.push_back({BUF_MTAB, li, li + 1});
+      for (int tok = 8 * idx; tok < std::min(B, 8 * idx + 8); ++tok) {
+        t.reads.push_back({BUF_MPAIR, (li * maxT + tok) * Kk, (li * maxT + tok + 1) * Kk});
+        for (int j = 0; j < P.top_k; ++j) {  // the segment of the pair's expert (its row lies in it)
+          const int e = rt->idx[(size_t)tok * P.top_k + j];
+          t.reads.push_back({BUF_MY, (li * maxT * Kk + rt->indptr[e]) * H, (li * maxT * Kk + rt->indptr[e + 1]) * H});
+        }
+        if (mdec) {
+          t.reads.push_back({BUF_X, (long long)tok * H, (long long)(tok + 1) * H});
+          t.writes.push_back({BUF_X, (long long)tok * H, (long long)(tok + 1) * H});
+        } else {
+          t.writes.push_back({BUF_MOUT, (long long)tok * H, (long long)(tok + 1) * H});
+        }
+      }
+    } break;
+    default: break;  // MFIN: end of the layer call
   }
 }
 
@@ -212,23 +385,50 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
   int c[3] = {0, 0, 0};
   for (int d = dp.ev[ev].ndim - 1; d >= 0; --d) { c[d] = lin % dp.ev[ev].dims[d]; lin /= dp.ev[ev].dims[d]; }
   auto add = [&](int f, int lo, int n) { if (n > 0) { out.push_back(f); out.push_back(lo); out.push_back(n); } };
+  const bool mdec = dp.kind == MK_MODEL_MOE_DECODER;
+  const int ml = dp.kind == MK_MODEL_MOE_LAYER ? -1 : c[0];  // the MoE event's layer
+  const bool wide = dp.wide != 0;
+  const int n8 = ceil_div(bd.B, 8);
   switch (ev) {
     case EV_IN:
-      if (c[0] < dp.n_layers) add(fam_index(OP_QKV, c[0]), 0, dp.n_qkv_tiles);
+      if (mdec) break;  // (the MoE decoder's layers chain through EV_MCOMB)
+      if (wide) {
+        if (c[0] < dp.n_layers) add(fam_index(OP_NORM, c[0]), 0, n8);
+        else add(fam_index(OP_NORMF, -1), 0, n8);
+      } else if (c[0] < dp.n_layers) {
+        add(fam_index(OP_QKV, c[0]), 0, dp.n_qkv_tiles);
+      } else {
+        add(fam_index(OP_LM, -1), 0, dp.n_lm_tiles);
+      }
+      break;
+    case EV_N1: add(fam_index(OP_QKV, c[0]), 0, dp.n_qkv_tiles); break;
+    case EV_N2: add(fam_index(OP_GATEUP, c[0]), 0, dp.n_gutiles); break;
+    case EV_NF: add(fam_index(OP_LM, -1), 0, dp.n_lm_tiles); break;
+    case EV_MIDX: add(fam_index(OP_EGU, ml), 0, bd.route[c[0]].tiles * dp.nt_gu); break;
+    case EV_MH: add(fam_index(OP_EDOWN, ml), c[1] * dp.nt_d, dp.nt_d); break;
+    case EV_MY: add(fam_index(OP_COMBINE, ml), 0, ceil_div(bd.B, 8)); break;
+    case EV_MCOMB:
+      if (!mdec) break;  // (the MoE layer's end is a follow-up)
+      if (c[0] + 1 < dp.n_layers) add(fam_index(OP_QKV, c[0] + 1), 0, dp.n_qkv_tiles);
       else add(fam_index(OP_LM, -1), 0, dp.n_lm_tiles);
       break;
     case EV_QKV: {
       int pre = 0;
       for (int b = 0; b < bd.B; ++b) {
-        int nch = ceil_div(bd.ctx[b] + 1, dp.chunk);
-        add(fam_index(OP_ATTN, c[0]), dp.n_kv_heads * pre + c[1] * nch, nch);
-        pre += nch;
+        const int ns = ceil_div(ceil_div(bd.ctx[b] + 1, dp.chunk), dp.attn_split);
+        if (wide) add(fam_index(OP_ATTN, c[0]), dp.n_kv_heads * pre, dp.n_kv_heads * ns);  // every kv head
+        else add(fam_index(OP_ATTN, c[0]), dp.n_kv_heads * pre + c[1] * ns, ns);
+        pre += ns;
       }
     } break;
     case EV_ATTN: add(fam_index(OP_OPROJ, c[0]), 0, dp.n_otiles); break;
-    case EV_O: add(fam_index(OP_GATEUP, c[0]), 0, dp.n_gutiles); break;
+    case EV_O:
+      if (mdec) add(fam_index(OP_ROUTE, c[0]), 0, n8);
+      else if (wide) add(fam_index(OP_NORM2, c[0]), 0, n8);
+      else add(fam_index(OP_GATEUP, c[0]), 0, dp.n_gutiles);
+      break;
     case EV_GU: add(fam_index(OP_DOWN, c[0]), c[1] * dp.n_dtiles, dp.n_dtiles); break;
-    default: break;  // EV_CHUNK and EV_LM trigger follow-ups
+    default: break;  // EV_CHUNK, EV_LM and EV_ROUTE trigger follow-ups
   }
 }
 
@@ -246,6 +446,7 @@ static void smem_layout(DevPlan& P, int rows, int smem_bytes) {
   P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - P.gred_bytes) / P.slot_bytes);
 }
 
+
 // MoE FFN layer ("Event Tensor: A Unified Abstraction for Compiling Dynamic
 // Megakernel", section "Core method", data-dependent dynamism).  The task
 // graph: ROUTE (8 tokens each) -> follow-up MINDPTR (exp_indptr, tile table,
@@ -258,7 +459,7 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
   if (E < 1 || E > 64) { err = "n_experts must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
   if (K < 1 || K > 8 || K > E) { err = "top_k must be in [1, min(8, n_experts)]"; return MK_ERR_UNSUPPORTED; }
-  if (FF < 32 || FF % 32 || FF > 2048) { err = "expert_ffn must be a multiple of 32 in [32, 2048]"; return MK_ERR_UNSUPPORTED; }
+  if (FF < 64 || FF % 64 || FF > 2048) { err = "expert_ffn must be a multiple of 64 in [64, 2048]"; return MK_ERR_UNSUPPORTED; }
   if (TM < 1 || TM > 4096) { err = "max_tokens must be in [1, 4096]"; return MK_ERR_UNSUPPORTED; }
   if (o->sched != MK_SCHED_DYNAMIC)
     { err = "an MoE layer's task counts depend on the routing: use MK_SCHED_DYNAMIC"; return MK_ERR_UNSUPPORTED; }
@@ -275,15 +476,17 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   P.hidden = H;
   P.debug_flags = o->debug_flags;
   P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
+  P.fault_ctr = -1;
+  if (o->fault != 0) { err = "fault injection is available for decoder plans only"; return MK_ERR_INVALID_ARG; }
   P.n_experts = E; P.top_k = K; P.eff = FF; P.max_tokens = TM;
-  P.moe_tm = 64;  // routed rows per GroupGEMM tile
-  P.moe_tn = 16;  // gate/up rows per EGU task (16 + 16: 8 ring slots at hidden 2048)
-  P.moe_td = 16;  // down rows per EDOWN task
+  P.moe_tm = kMoeTileRows;  // routed rows per GroupGEMM tile
+  P.moe_tn = kMoeTaskRows;  // gate rows (and as many up rows) per EGU task
+  P.moe_td = kMoeTaskRows;  // down rows per EDOWN task
   P.nt_gu = ceil_div(FF, P.moe_tn);
   P.nt_d = H / P.moe_td;
+  P.moe_cap = TM;
   // sum over experts of ceil(hist_e / tm) <= T*k/tm + (experts with a row)
   P.max_tiles = ceil_div(TM * K, P.moe_tm) + std::min(E, TM * K);
-  if (FF % P.moe_tn) { err = "expert_ffn must be a multiple of 16"; return MK_ERR_UNSUPPORTED; }
   P.slot_bytes = 16384;
   smem_layout(P, 0, smem_bytes);
   if (P.ring_slots < 5) { err = "not enough shared memory for a 5-slot ring"; return MK_ERR_UNSUPPORTED; }
@@ -330,7 +533,7 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   {
     EventTensorDesc& e = P.ev[EV_MH];
     e.base = base; e.ndim = 2; e.dims[0] = 1; e.dims[1] = P.max_tiles; e.dims[2] = 1;
-    e.count_expr = emit_const(p.code, P.nt_gu);
+    e.count_expr = emit_const(p.code, 0);  // armed at run time by MINDPTR for the tiles the routing made
     base += P.max_tiles;
   }
   add_event(EV_MY, 1, emit_const(p.code, 1 << 30));  // replaced at run time by MINDPTR
@@ -367,7 +570,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     const int E = m->n_experts, K = m->top_k, FF = m->expert_ffn;
     if (E < 1 || E > 64) { err = "n_experts must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
     if (K < 1 || K > 8 || K > E) { err = "top_k must be in [1, min(8, n_experts)]"; return MK_ERR_UNSUPPORTED; }
-    if (FF < 32 || FF % 32 || FF > 2048) { err = "expert_ffn must be a multiple of 32 in [32, 2048]"; return MK_ERR_UNSUPPORTED; }
+    if (FF < 64 || FF % 64 || FF > 2048) { err = "expert_ffn must be a multiple of 64 in [64, 2048]"; return MK_ERR_UNSUPPORTED; }
     if (o->sched != MK_SCHED_DYNAMIC)
       { err = "an MoE layer's task counts depend on the routing: use MK_SCHED_DYNAMIC"; return MK_ERR_UNSUPPORTED; }
   }
@@ -377,7 +580,10 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (Hq * D != H) { err = "n_q_heads * head_dim must equal hidden"; return MK_ERR_UNSUPPORTED; }
   if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
   if (!mdec && (F % 256 || F < 256)) { err = "ffn must be a positive multiple of 256"; return MK_ERR_UNSUPPORTED; }
-  if (m->max_batch < 1 || m->max_batch > kMaxBatchRows) { err = "max_batch must be in [1, 8] for this build"; return MK_ERR_UNSUPPORTED; }
+  // above kMaxBatchRows the dense decoder runs the wide-batch path
+  const bool wide = !mdec && m->max_batch > kMaxBatchRows;
+  if (m->max_batch < 1 || m->max_batch > (mdec ? kMaxBatchRows : kMaxWideBatch))
+    { err = mdec ? "max_batch must be in [1, 8] for an MoE decoder" : "max_batch must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
   if (m->max_ctx < 2 || m->n_slots < m->max_batch) { err = "max_ctx >= 2 and n_slots >= max_batch required"; return MK_ERR_INVALID_ARG; }
   if (o->sched != MK_SCHED_STATIC && o->sched != MK_SCHED_DYNAMIC) { err = "unknown schedule"; return MK_ERR_INVALID_ARG; }
   if (n_sm < 1 || n_sm > 1024) { err = "n_sm out of range"; return MK_ERR_INVALID_ARG; }
@@ -396,6 +602,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.n_slots = m->n_slots; P.eps = m->eps;
   P.debug_flags = o->debug_flags;
   P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
+  P.fault_ctr = -1;
 
   // K segment of the down projection (split-K), at most 2048 columns
   int kseg = mdec ? 2048 : (o->kseg ? o->kseg : std::min(F, 2048));  // (no dense FFN in an MoE decoder)
@@ -413,17 +620,30 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.tile_lm = o->tile_lm ? o->tile_lm : 64;
   P.chunk = o->attn_chunk ? o->attn_chunk : 64;
   P.slot_bytes = 16384;
+  P.wide = wide ? 1 : 0;
+  P.attn_split = o->attn_split ? o->attn_split : (wide ? 8 : 1);
+  if (P.attn_split < 1 || P.attn_split > 16) { err = "attn_split must be in [1, 16]"; return MK_ERR_INVALID_ARG; }
+  if (wide) {
+    // tcgen05 GEMM tasks: kWideRows weight rows each (the MMA's M), every
+    // weight matrix read in 64-column chunks, the batch as the MMA's N
+    if (o->tile_qkv || o->tile_o || o->tile_gu || o->tile_down || o->tile_lm)
+      { err = "the wide-batch path takes no GEMV tile options"; return MK_ERR_INVALID_ARG; }
+    P.tile_qkv = P.tile_o = P.tile_gu = P.tile_down = P.tile_lm = kWideRows;
+    if (H % kWideRows || F % kWideRows) { err = "wide batch: hidden and ffn must be multiples of 128"; return MK_ERR_UNSUPPORTED; }
+    if (Hq / Hkv < 2 || (Hq / Hkv) % 2) { err = "wide batch: an even number of query heads per kv head"; return MK_ERR_UNSUPPORTED; }
+  }
+  P.act_rows = ceil_div(P.max_batch, 16) * 16;
   if (!(P.kseg % 256 == 0 && F % P.kseg == 0 && P.kseg >= 1024 && P.kseg <= 2048))
     { err = "kseg must be a multiple of 256 in [1024, 2048] dividing ffn"; return MK_ERR_INVALID_ARG; }
   if (Hq / Hkv > 4) { err = "at most 4 query heads per kv head"; return MK_ERR_UNSUPPORTED; }
-  if (P.tile_qkv != 32) { err = "tile_qkv must be 32 (16 rotate-half pairs)"; return MK_ERR_UNSUPPORTED; }
-  if (!((P.tile_o == 16 || P.tile_o == 32) && H % P.tile_o == 0))
+  if (!wide && P.tile_qkv != 32) { err = "tile_qkv must be 32 (16 rotate-half pairs)"; return MK_ERR_UNSUPPORTED; }
+  if (!wide && !((P.tile_o == 16 || P.tile_o == 32) && H % P.tile_o == 0))
     { err = "tile_o must be 16 or 32 and divide hidden"; return MK_ERR_UNSUPPORTED; }
-  if (!((P.tile_gu == 16 || P.tile_gu == 32) && P.kseg % P.tile_gu == 0))
+  if (!wide && !((P.tile_gu == 16 || P.tile_gu == 32) && P.kseg % P.tile_gu == 0))
     { err = "tile_gu must be 16 or 32 (gate + up rows each)"; return MK_ERR_UNSUPPORTED; }
-  if (!((P.tile_down == 16 || P.tile_down == 32 || P.tile_down == 64) && H % P.tile_down == 0))
+  if (!wide && !((P.tile_down == 16 || P.tile_down == 32 || P.tile_down == 64) && H % P.tile_down == 0))
     { err = "tile_down must be 16, 32 or 64 and divide hidden"; return MK_ERR_UNSUPPORTED; }
-  if (P.tile_lm != 32 && P.tile_lm != 64) { err = "tile_lm must be 32 or 64"; return MK_ERR_UNSUPPORTED; }
+  if (!wide && P.tile_lm != 32 && P.tile_lm != 64) { err = "tile_lm must be 32 or 64"; return MK_ERR_UNSUPPORTED; }
   if (P.chunk != 64) { err = "attn_chunk must be 64"; return MK_ERR_UNSUPPORTED; }
   P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
   P.n_otiles = H / P.tile_o;
@@ -433,8 +653,19 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.n_lm_tiles = ceil_div(P.vocab, P.tile_lm);
   P.max_chunks = ceil_div(P.max_ctx, P.chunk);
 
-  // shared memory: ring of 16 KB slots plus a fixed control area
-  smem_layout(P, P.max_batch, smem_bytes);
+  // shared memory: ring of 16 KB slots plus a fixed control area (wide
+  // batch: the staging buffer holds the activation chunks of the GEMM tasks'
+  // MMA issuer, kBStages x act_rows x 128 bytes, and afterwards the QKV
+  // tiles' rotate-half exchange, 64 rows x act_rows fp32; no GEMV partial tiles)
+  if (wide) {
+    P.gbatch = 0;
+    P.act_bytes = std::max(std::max(8192, 64 * P.act_rows * 4), kBStages * P.act_rows * 128);
+    P.gred_bytes = 0;
+    P.smem_bytes = smem_bytes;
+    P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes) / P.slot_bytes);
+  } else {
+    smem_layout(P, P.max_batch, smem_bytes);
+  }
   if (P.ring_slots < 3) { err = "not enough shared memory for a 3-slot ring"; return MK_ERR_UNSUPPORTED; }
 
   // ---- expressions and families
@@ -462,6 +693,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     p.code.push_back(X_VAR); p.code.push_back(X_CTX_AT);
     p.code.push_back(X_PUSH); p.code.push_back(1); p.code.push_back(X_ADD);
     p.code.push_back(X_PUSH); p.code.push_back(P.chunk); p.code.push_back(X_CEILDIV);
+    p.code.push_back(X_PUSH); p.code.push_back(P.attn_split); p.code.push_back(X_CEILDIV);
     p.code.push_back(X_RET);
     p.code[len_at] = (int)(p.code.size() - body);
     p.code.push_back(X_MUL);
@@ -473,20 +705,25 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (mdec) {
     P.kind = MK_MODEL_MOE_DECODER;
     P.n_experts = m->n_experts; P.top_k = m->top_k; P.eff = m->expert_ffn; P.max_tokens = P.max_batch;
-    P.moe_tm = 64; P.moe_tn = 16; P.moe_td = 16;
+    P.moe_tm = kMoeTileRows; P.moe_tn = kMoeTaskRows; P.moe_td = kMoeTaskRows;
     P.nt_gu = ceil_div(P.eff, P.moe_tn);
     P.nt_d = H / P.moe_td;
+    P.moe_cap = P.max_tokens;
     P.max_tiles = ceil_div(P.max_tokens * P.top_k, P.moe_tm) + std::min(P.n_experts, P.max_tokens * P.top_k);
-  }
+    }
   const int e_tok8 = Emit(p.code).op(X_B).push(8).op(X_CEILDIV).ret();  // ceil(B / 8)
   static const int kMoeDecOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU, OP_EDOWN,
                                    OP_COMBINE};
-  const int fam_per_layer = mdec ? 9 : kFamPerLayer;
+  static const int kWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_NORM2, OP_GATEUP, OP_DOWN};
+  const int fam_per_layer = mdec ? 9 : wide ? 8 : kFamPerLayer;
+  const int max_tasks_attn = Hkv * P.max_batch * ceil_div(P.max_chunks, P.attn_split);
   for (int l = 0; l < P.n_layers; ++l) {
+    if (wide) add_family(OP_NORM, l, e_tok8, ceil_div(P.max_batch, 8), 0);
     add_family(OP_QKV, l, emit_const(p.code, P.n_qkv_tiles), P.n_qkv_tiles, 0);
-    add_family(OP_ATTN, l, e_attn, Hkv * P.max_batch * P.max_chunks, 0);
+    add_family(OP_ATTN, l, e_attn, max_tasks_attn, 0);
     add_family(OP_MERGE, l, e_merge, Hkv * P.max_batch, 1);
     add_family(OP_OPROJ, l, emit_const(p.code, P.n_otiles), P.n_otiles, 0);
+    if (wide) add_family(OP_NORM2, l, e_tok8, ceil_div(P.max_batch, 8), 0);
     if (mdec) {
       add_family(OP_ROUTE, l, e_tok8, ceil_div(P.max_tokens, 8), 0);
       add_family(OP_MINDPTR, l, emit_const(p.code, 1), 1, 1);
@@ -498,6 +735,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
       add_family(OP_DOWN, l, emit_const(p.code, P.n_dtiles * P.n_kc), P.n_dtiles * P.n_kc, 0);
     }
   }
+  if (wide) add_family(OP_NORMF, -1, e_tok8, ceil_div(P.max_batch, 8), 0);
   add_family(OP_LM, -1, emit_const(p.code, P.n_lm_tiles), P.n_lm_tiles, 0);
   add_family(OP_LMFIN, -1, emit_const(p.code, 1), 1, 1);
   P.n_families = (int)p.fams.size();
@@ -505,8 +743,12 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.debug_slots = debug_base;
   P.fam_stride = fam_per_layer;
   for (int op = 0; op < OP_COUNT; ++op) P.fam_first_layer[op] = -1;
-  for (int k = 0; k < fam_per_layer; ++k) P.fam_first_layer[mdec ? kMoeDecOps[k] : kLayerOps[k]] = k;
-  for (int k = 0; k < 2; ++k) P.fam_first_layer[kLmOps[k]] = P.n_layers * fam_per_layer + k;
+  for (int k = 0; k < fam_per_layer; ++k) P.fam_first_layer[mdec ? kMoeDecOps[k] : wide ? kWideOps[k] : kLayerOps[k]] = k;
+  {
+    int g0 = P.n_layers * fam_per_layer;
+    if (wide) P.fam_first_layer[OP_NORMF] = g0++;
+    for (int k = 0; k < 2; ++k) P.fam_first_layer[kLmOps[k]] = g0 + k;
+  }
 
   // ---- event tensors (shapes at the symbols' maxima, wait counts symbolic)
   int base = 0;
@@ -520,10 +762,11 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   const int qkv_per_group = (Hq / Hkv + 2) * (D / P.tile_qkv);
   add_event(EV_IN, 1, L + 1, 1, 1,
             Emit(p.code).push(0).coord(0).op(X_LT).push(P.n_dtiles * P.n_kc).op(X_MUL).ret());
-  add_event(EV_QKV, 2, L, Hkv, 1, emit_const(p.code, qkv_per_group));
+  if (wide) add_event(EV_QKV, 2, L, 1, 1, emit_const(p.code, P.n_qkv_tiles));  // (a tile spans two kv heads)
+  else add_event(EV_QKV, 2, L, Hkv, 1, emit_const(p.code, qkv_per_group));
   add_event(EV_CHUNK, 3, L, P.max_batch, Hkv,
             Emit(p.code).coord(1).op(X_B).op(X_LT).coord(1).op(X_CTX_AT).push(1).op(X_ADD)
-                .push(P.chunk).op(X_CEILDIV).op(X_MUL).ret());
+                .push(P.chunk).op(X_CEILDIV).push(P.attn_split).op(X_CEILDIV).op(X_MUL).ret());
   add_event(EV_ATTN, 1, L, 1, 1, Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret());
   add_event(EV_O, 1, L, 1, 1, emit_const(p.code, P.n_otiles));
   add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu));
@@ -531,11 +774,18 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (mdec) {  // one element per layer (EV_MH: per layer and GroupGEMM tile)
     add_event(EV_ROUTE, 1, L, 1, 1, e_tok8);
     add_event(EV_MIDX, 1, L, 1, 1, emit_const(p.code, 1));
-    add_event(EV_MH, 2, L, P.max_tiles, 1, emit_const(p.code, P.nt_gu));
+    add_event(EV_MH, 2, L, P.max_tiles, 1, emit_const(p.code, 0));  // armed at run time by MINDPTR
     add_event(EV_MY, 1, L, 1, 1, emit_const(p.code, 1 << 30));  // replaced at run time by MINDPTR
     add_event(EV_MCOMB, 1, L, 1, 1, e_tok8);
   } else {
-    for (int id = EV_LM + 1; id < EV_COUNT; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // MoE: empty
+    for (int id = EV_LM + 1; id <= EV_MCOMB; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // MoE: empty
+  }
+  if (wide) {
+    add_event(EV_N1, 1, L, 1, 1, e_tok8);
+    add_event(EV_N2, 1, L, 1, 1, e_tok8);
+    add_event(EV_NF, 1, 1, 1, 1, e_tok8);
+  } else {
+    for (int id = EV_N1; id < EV_COUNT; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // wide only: empty
   }
   P.n_counters = base;
 
@@ -568,7 +818,11 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   // per layer: QKV (1), ATTN (one per sequence and kv head), OPROJ (1),
   // GATEUP (1), DOWN (one per K segment) -- or for an MoE FFN: ROUTE, EGU,
   // COMBINE (1 each) and EDOWN (one per tile); then LM (1) and END (1)
-  P.queue_ranges = mdec ? L * (5 + Hkv * P.max_batch + P.max_tiles) + 2 : L * (3 + Hkv * P.max_batch + P.n_kc) + 2;
+  // wide batch: NORM, QKV, OPROJ, NORM2, GATEUP (1 each), ATTN (one per
+  // sequence), DOWN (one per K segment); then NORMF, LM and END
+  P.queue_ranges = mdec ? L * (5 + Hkv * P.max_batch + P.max_tiles) + 2
+                   : wide ? L * (5 + P.max_batch + P.n_kc) + 3
+                          : L * (3 + Hkv * P.max_batch + P.n_kc) + 2;
 
   // ---- layer pointers and the rotary table
   p.layers.resize(L);
@@ -589,6 +843,19 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
       p.rope[((size_t)pos * (D / 2) + i) * 2 + 0] = (float)std::cos(ang);
       p.rope[((size_t)pos * (D / 2) + i) * 2 + 1] = (float)std::sin(ang);
     }
+  // ---- device fault injection: one event armed one above its notifies
+  if (o->fault == MK_SIM_FAULT_COUNT_PLUS_ONE) {
+    const int f = o->fault_family;
+    const int op = (f >= 0 && f < P.n_families) ? p.fams[f].op : -1;
+    if (op != OP_QKV && op != OP_OPROJ && op != OP_GATEUP && op != OP_DOWN && op != OP_LM)
+      { err = "fault_family must be a qkv, oproj, gateup, down or lm family"; return MK_ERR_INVALID_ARG; }
+    TaskRec t;
+    p.task(f, 0, Binding{1, {0}}, t);  // these families notify the same counter at every binding
+    P.fault_ctr = t.notify_ev;
+  } else if (o->fault != 0) {
+    err = "unknown fault kind";
+    return MK_ERR_INVALID_ARG;
+  }
   std::vector<unsigned char> image;
   lower_plan(p, image);
   return MK_OK;
@@ -607,8 +874,8 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_instr = take((long long)sizeof(Instr) * (long long)p.instr.size());
   P.off_layers = take((long long)sizeof(LayerPtrs) * P.n_layers);
   P.off_rope = take(4LL * (long long)p.rope.size());
-  // tensor maps of the dense weights (encoded when the workspace is bound)
-  P.off_tmap = take(P.kind == MK_MODEL_MOE_LAYER ? 0 : (long long)kTmapBytes * (P.n_layers * kTmapPerLayer + 1));
+  // tensor maps of the weights and activation buffers (encoded when the workspace is bound)
+  P.off_tmap = take((long long)kTmapBytes * (std::max(P.n_layers, 1) * kTmapPerLayer + kTmapGlobal));
   P.off_queue = take((long long)sizeof(QRange) * P.queue_ranges);
   P.off_x = take(4LL * P.max_batch * P.hidden);
   P.off_q = take(4LL * P.max_batch * P.n_q_heads * P.head_dim);
@@ -617,6 +884,12 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_h = take(4LL * P.max_batch * P.ffn);
   P.off_dpart = take(4LL * P.n_kc * P.max_batch * P.hidden);
   P.off_lmbest = take(8LL * P.max_batch);
+  // wide batch: the bf16 activations the GEMM tasks load by TMA (act_rows rows
+  // each, so that a box of act_rows rows stays inside the buffer)
+  const long long ar = P.wide ? P.act_rows : 0;
+  P.off_xn = take(2LL * ar * P.hidden);
+  P.off_attn_bf = take(2LL * ar * P.hidden);
+  P.off_h_bf = take(2LL * ar * P.ffn);
   if (P.kind != MK_MODEL_DENSE) {
     // one MoE scratch block per MoE layer (layer 0's offsets; the others follow at moe_stride)
     const long long pairs = (long long)P.max_tokens * P.top_k;
@@ -634,6 +907,7 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
     P.off_mh = take(2 * pairs * P.eff);
     P.off_my = take(4 * pairs * P.hidden);
     P.off_mxhat = take(2LL * P.max_tokens * P.hidden);
+    P.off_mxg = take(2LL * P.n_experts * P.moe_cap * P.hidden);
     P.moe_stride = off - block0;
     const int Lm = P.kind == MK_MODEL_MOE_DECODER ? P.n_layers : 1;
     off += P.moe_stride * (Lm - 1);
@@ -668,6 +942,10 @@ double step_bytes(const Plan& p, const Binding& bd, bool with_logits) {
 
 // ---------------------------------------------------------------- validation
 static bool check_binding(const Plan& p, const Binding& bd, std::string& err) {
+  if (p.dp.kind == MK_MODEL_MOE_LAYER) {  // B is the token count; no contexts
+    if (bd.B < 1 || bd.B > p.dp.max_tokens) { err = "token count out of range"; return false; }
+    return true;
+  }
   if (bd.B < 1 || bd.B > p.dp.max_batch) { err = "batch out of range"; return false; }
   if ((int)bd.ctx.size() < bd.B) { err = "ctx_lens shorter than batch"; return false; }
   for (int b = 0; b < bd.B; ++b)
@@ -675,12 +953,20 @@ static bool check_binding(const Plan& p, const Binding& bd, std::string& err) {
   return true;
 }
 
-mk_status validate_plan(const Plan& p, const Binding& bd, std::string& err) {
-  if (p.dp.kind != MK_MODEL_DENSE) {
-    err = "the host task model covers the dense decoder; an MoE layer's graph depends on its routing";
-    return MK_ERR_UNSUPPORTED;
-  }
-  if (!check_binding(p, bd, err)) return MK_ERR_INVALID_ARG;
+// Wait count of a counter for a binding: the armed expression, or for the
+// MoE events armed at run time by the routing follow-up (EV_MY: one per down
+// task; EV_MH: one per gate/up task of a tile the routing made) their value
+// after that arming.
+static int runtime_count(const Plan& p, int ev, int c0, int c1, int c2, const Binding& bd) {
+  if (ev == EV_MY && c0 < (int)bd.route.size()) return bd.route[c0].tiles * p.dp.nt_d;
+  if (ev == EV_MH && c0 < (int)bd.route.size()) return c1 < bd.route[c0].tiles ? p.dp.nt_gu : 0;
+  return p.event_count(ev, c0, c1, c2, bd);
+}
+
+mk_status validate_plan(const Plan& p, const Binding& bd_in, std::string& err) {
+  if (!check_binding(p, bd_in, err)) return MK_ERR_INVALID_ARG;
+  Binding bd = bd_in;
+  if (p.dp.kind != MK_MODEL_DENSE && bd.route.empty()) draw_routing(p, bd, 0, 0.0);
   const DevPlan& P = p.dp;
   std::vector<int> notifiers(P.n_counters, 0);
   std::vector<int> last_notifier_fam(P.n_counters, -1);
@@ -689,7 +975,7 @@ mk_status validate_plan(const Plan& p, const Binding& bd, std::string& err) {
   TaskRec t;
   std::vector<int> followups_seen(P.n_families, 0);
   for (int f = 0; f < P.n_families; ++f) {
-    int n = p.family_extent(f, bd);
+    int n = p.actual_extent(f, bd);
     if (n < 0 || n > p.fams[f].max_extent) {
       err = "family " + p.fam_names[f] + " extent exceeds its reserved maximum";
       return MK_ERR_PLAN;
@@ -715,7 +1001,7 @@ mk_status validate_plan(const Plan& p, const Binding& bd, std::string& err) {
       for (int b = 0; b < d1; ++b)
         for (int c = 0; c < d2; ++c) {
           int ci = p.counter(e, a, b, c);
-          int cnt = p.event_count(e, a, b, c, bd);
+          int cnt = runtime_count(p, e, a, b, c, bd);
           if (cnt != notifiers[ci]) {
             err = "event " + std::to_string(e) + " element (" + std::to_string(a) + "," + std::to_string(b) +
                   "," + std::to_string(c) + ") waits for " + std::to_string(cnt) + " but has " +
@@ -806,6 +1092,8 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
   sim.evc.assign(P.n_counters, VC{std::vector<unsigned>(nw, 0)});
   sim.counters.assign(P.n_counters, 0);
   bool fault_done = false;
+  // clock of each event when its counter reached zero (armed at zero: none)
+  std::vector<VC> fired(P.n_counters, VC{std::vector<unsigned>(nw, 0)});
   for (int e = 0; e < EV_COUNT; ++e) {
     const EventTensorDesc& d = P.ev[e];
     int d1 = d.ndim > 1 ? d.dims[1] : 1, d2 = d.ndim > 2 ? d.dims[2] : 1;
@@ -813,15 +1101,19 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
       for (int b = 0; b < d1; ++b)
         for (int c = 0; c < d2; ++c) sim.counters[p.counter(e, a, b, c)] = p.event_count(e, a, b, c, bd);
   }
-  if (fault == MK_SIM_FAULT_COUNT_PLUS_ONE && fault_family >= 0 && fault_family < P.n_families) {
-    TaskRec t0;
-    if (p.family_extent(fault_family, bd) > 0) {
-      p.task(fault_family, 0, bd, t0);
-      if (t0.notify_ev >= 0) sim.counters[t0.notify_ev] += 1;
-    }
-  }
   std::vector<int> ext(P.n_families);
-  for (int f = 0; f < P.n_families; ++f) ext[f] = p.family_extent(f, bd);
+  for (int f = 0; f < P.n_families; ++f) ext[f] = p.actual_extent(f, bd);
+  // wrong wait counts: the event task 0 of the fault family notifies, armed
+  // one above or one below its notifies (again after a run-time arming)
+  int fault_ctr = -1, fault_delta = 0;
+  if ((fault == MK_SIM_FAULT_COUNT_PLUS_ONE || fault == MK_SIM_FAULT_COUNT_MINUS_ONE) && fault_family >= 0 &&
+      fault_family < P.n_families && ext[fault_family] > 0) {
+    TaskRec t0;
+    p.task(fault_family, 0, bd, t0);
+    fault_ctr = t0.notify_ev;
+    fault_delta = fault == MK_SIM_FAULT_COUNT_PLUS_ONE ? 1 : -1;
+    if (fault_ctr >= 0) sim.counters[fault_ctr] += fault_delta;
+  }
 
   // per-worker task sources
   std::vector<std::vector<Work>> local(nw);   // static: own queue; both: follow-ups
@@ -846,15 +1138,12 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
       std::stable_sort(local[w].begin(), local[w].end(),
                        [](const Work& a, const Work& b) { return a.fam < b.fam; });
   } else {
-    std::vector<int> succ;
-    for (int ci = 0; ci < P.n_counters; ++ci)
-      if (sim.counters[ci] == 0) {
-        succ.clear();
-        p.successors(ci, bd, succ);
-        ranges_pushed += (int)succ.size() / 3;
-        for (size_t k = 0; k < succ.size(); k += 3)
-          for (int i = 0; i < succ[k + 2]; ++i) shared.push_back({succ[k], succ[k + 1] + i, std::vector<unsigned>(nw, 0)});
-      }
+    // the launch's first push, as on the device: the routing tasks of an MoE
+    // layer call, or the QKV tiles of layer 0 of a decoder
+    const int f0 = P.kind == MK_MODEL_MOE_LAYER ? p.fam_index(OP_ROUTE, -1)
+                   : P.wide ? p.fam_index(OP_NORM, 0) : p.fam_index(OP_QKV, 0);
+    ranges_pushed += 1;
+    for (int i = 0; i < ext[f0]; ++i) shared.push_back({f0, i, std::vector<unsigned>(nw, 0)});
   }
   TaskRec t;
   int executed = 0;
@@ -864,28 +1153,45 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
     p.task(wk.fam, wk.idx, bd, t);
     if (!wk.vc.empty()) { VC v{wk.vc}; me.join(v); }
     bool skip_wait = fault == MK_SIM_FAULT_NO_WAIT && wk.fam == fault_family;
-    if (t.wait_ev >= 0 && !skip_wait) me.join(sim.evc[t.wait_ev]);
+    // the wait synchronises with the notifies that took the counter to zero
+    // (a later, surplus notify is not ordered before the waiter)
+    if (t.wait_ev >= 0 && !skip_wait) me.join(fired[t.wait_ev]);
     for (auto& r : t.reads) sim.access(w, r, false);
     for (auto& r : t.writes) sim.access(w, r, true);
     exec_count[p.fams[wk.fam].debug_base + wk.idx]++;
     executed++;
+    if (p.fams[wk.fam].op == OP_MINDPTR) {
+      // data-dependent event update: the routing follow-up arms the down
+      // count and the gate/up count of every tile the routing made
+      const int li = p.fams[wk.fam].layer < 0 ? 0 : p.fams[wk.fam].layer;
+      const int cmy = p.counter(EV_MY, li);
+      sim.counters[cmy] = bd.route[li].tiles * P.nt_d + (cmy == fault_ctr ? fault_delta : 0);
+      for (int tl = 0; tl < bd.route[li].tiles; ++tl) {
+        const int cmh = p.counter(EV_MH, li, tl);
+        sim.counters[cmh] = P.nt_gu + (cmh == fault_ctr ? fault_delta : 0);
+      }
+    }
     if (t.notify_ev >= 0) {
       if (fault == MK_SIM_FAULT_DROP_NOTIFY && wk.fam == fault_family && !fault_done) { fault_done = true; return; }
       sim.evc[t.notify_ev].join(me);
       int old = sim.counters[t.notify_ev]--;
+      auto push_succ = [&]() {
+        std::vector<int> succ;
+        p.successors(t.notify_ev, bd, succ);
+        ranges_pushed += (int)succ.size() / 3;
+        for (size_t k = 0; k < succ.size(); k += 3)
+          for (int i = 0; i < succ[k + 2]; ++i) shared.push_back({succ[k], succ[k + 1] + i, me.c});
+      };
       if (old == 1) {
+        fired[t.notify_ev] = sim.evc[t.notify_ev];
         me.join(sim.evc[t.notify_ev]);  // the last notifier acquires every release
         if (t.follow_fam >= 0) follow[w].push_back({t.follow_fam, t.follow_idx, {}});
-        if (dynamic) {
-          std::vector<int> succ;
-          p.successors(t.notify_ev, bd, succ);
-          ranges_pushed += (int)succ.size() / 3;
-          for (size_t k = 0; k < succ.size(); k += 3)
-            for (int i = 0; i < succ[k + 2]; ++i) shared.push_back({succ[k], succ[k + 1] + i, me.c});
-        }
+        if (dynamic) push_succ();
       }
     }
   };
+  std::vector<Work> held(nw);
+  std::vector<char> held_ok(nw, 0);
   auto ready = [&](int w) -> int {  // 1 follow-up, 2 regular, 0 blocked
     if (!follow[w].empty()) return 1;
     if (!dynamic) {
@@ -896,7 +1202,19 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
       if (tr.wait_ev >= 0 && sim.counters[tr.wait_ev] != 0 && !skip_wait) return 0;
       return 2;
     }
-    return shared_head < shared.size() ? 2 : 0;
+    // dynamic: a worker pops the queue head into its held slot and runs it
+    // once its event has fired (the device's controller waits on the counter
+    // of a popped task as well)
+    if (!held_ok[w]) {
+      if (shared_head >= shared.size()) return 0;
+      held[w] = shared[shared_head++];
+      held_ok[w] = true;
+    }
+    TaskRec tr;
+    p.task(held[w].fam, held[w].idx, bd, tr);
+    bool skip_wait = fault == MK_SIM_FAULT_NO_WAIT && held[w].fam == fault_family;
+    if (tr.wait_ev >= 0 && sim.counters[tr.wait_ev] > 0 && !skip_wait) return 0;
+    return 2;
   };
   std::vector<int> cand;
   for (;;) {
@@ -914,8 +1232,8 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
     } else if (!dynamic) {
       exec(w, local[w][pos[w]++]);
     } else {
-      Work wk = shared[shared_head++];
-      exec(w, wk);
+      held_ok[w] = false;
+      exec(w, held[w]);
     }
   }
   if (dynamic) {
@@ -931,8 +1249,10 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
   for (int w = 0; w < nw; ++w)
     if ((!dynamic && pos[w] < local[w].size()) || !follow[w].empty()) left = true;
   if (dynamic && shared_head < shared.size()) left = true;
+  for (int w = 0; w < nw; ++w)
+    if (held_ok[w]) left = true;
   // a plan that stops before the final task has deadlocked
-  int fin = p.fam_index(OP_LMFIN, -1);
+  int fin = p.fam_index(P.kind == MK_MODEL_MOE_LAYER ? OP_MFIN : OP_LMFIN, -1);
   if (exec_count[p.fams[fin].debug_base] == 0) left = true;
   if (left) rep->deadlocks++;
   for (int ci = 0; ci < P.n_counters; ++ci)
@@ -946,25 +1266,25 @@ static int run_order(const Plan& p, const Binding& bd, bool dynamic, std::mt1993
   return executed;
 }
 
-mk_status simulate_plan(const Plan& p, const Binding& bd, int n_orders, unsigned seed, int fault,
+mk_status simulate_plan(const Plan& p, const Binding& bd_in, int n_orders, unsigned seed, int fault,
                         int fault_family, mk_sim_report* rep) {
   std::string err;
   std::memset(rep, 0, sizeof(*rep));
-  if (p.dp.kind != MK_MODEL_DENSE) {
-    std::snprintf(rep->first_error, sizeof(rep->first_error), "simulation covers the dense decoder only");
-    return MK_ERR_UNSUPPORTED;
-  }
-  if (!check_binding(p, bd, err)) {
+  if (!check_binding(p, bd_in, err)) {
     std::snprintf(rep->first_error, sizeof(rep->first_error), "%s", err.c_str());
     return MK_ERR_INVALID_ARG;
   }
+  // MoE plans: a routing drawn from the seed (odd seeds skewed), dynamic orders only
+  Binding bd = bd_in;
+  const bool moe = p.dp.kind != MK_MODEL_DENSE;
+  if (moe) draw_routing(p, bd, seed, (seed & 1u) ? 1.2 : 0.0);
   std::mt19937 rng(seed);
   std::vector<int> want(p.dp.debug_slots, 0);
   for (int f = 0; f < p.dp.n_families; ++f)
-    for (int i = 0; i < p.family_extent(f, bd); ++i) want[p.fams[f].debug_base + i] = 1;
+    for (int i = 0; i < p.actual_extent(f, bd); ++i) want[p.fams[f].debug_base + i] = 1;
   std::vector<int> first_set;
   for (int k = 0; k < n_orders; ++k) {
-    bool dynamic = (k % 2) == 1;
+    bool dynamic = moe || (k % 2) == 1;
     std::vector<int> exec_count(p.dp.debug_slots, 0);
     run_order(p, bd, dynamic, rng, fault, fault_family, exec_count, rep);
     rep->orders_run++;

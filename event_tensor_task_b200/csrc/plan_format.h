@@ -31,9 +31,9 @@ enum Op : int32_t {
   OP_OPROJ = 4,   // output projection rows + residual
   OP_GATEUP = 5,  // RMSNorm -> gate and up rows -> SwiGLU
   OP_DOWN = 6,    // down projection rows over one K segment -> partial
-                  // (7 is unused)
+  OP_NORM = 7,    // wide batch: 8 rows: residual (x + down partials) -> x, RMSNorm(x) * attn gain -> bf16
   OP_LM = 8,      // final RMSNorm -> vocabulary rows -> logits + running argmax
-                  // (9 is unused)
+  OP_NORM2 = 9,   // wide batch: 8 rows: RMSNorm(x) * FFN gain -> bf16
   OP_LMFIN = 10,  // follow-up: the running argmax -> next token
   // mixture-of-experts FFN layer (data-dependent task graph, dynamic schedule)
   OP_ROUTE = 11,    // 8 tokens: router logits -> top-k, weights, per-expert ranks
@@ -42,7 +42,8 @@ enum Op : int32_t {
   OP_EDOWN = 14,    // GroupGEMM tile: an expert's down rows x its routed rows
   OP_COMBINE = 15,  // 8 tokens: weighted sum of their top-k expert outputs
   OP_MFIN = 16,     // follow-up: end of the layer
-  OP_COUNT = 17
+  OP_NORMF = 17,    // wide batch: 8 rows: final residual, RMSNorm * final gain -> bf16
+  OP_COUNT = 18
 };
 
 // ---------------------------------------------------------------- expressions
@@ -140,7 +141,11 @@ enum EvId : int32_t {
   EV_MH = 9,     // [Lm][max_tiles] SwiGLU rows of one GroupGEMM tile written (all its gate/up tasks)
   EV_MY = 10,    // [Lm]            all down tasks done (count set at run time from exp_indptr)
   EV_MCOMB = 11, // [Lm]            all COMBINE tasks done (the layer's residual is updated)
-  EV_COUNT = 12
+  // wide batch (max_batch > 8): the normalised activations are materialised
+  EV_N1 = 12,    // [L]  layer input normalised (bf16) and the residual materialised
+  EV_N2 = 13,    // [L]  FFN input normalised
+  EV_NF = 14,    // [1]  final norm done
+  EV_COUNT = 15
 };
 
 struct EventTensorDesc {
@@ -191,16 +196,36 @@ constexpr int kMaxFamilies = 256;
 // partial tiles (gred_bytes: 8 warps x gbatch = 8 columns x 64 rows of fp32).
 constexpr int kSmemFixed = 9 * 1024;
 constexpr int kActPitch = 2048 + 8;  // bf16 elements per staged activation row (16-byte bank offset per row)
-constexpr int kMaxBatchRows = 8;     // batch rows of a dense step (the GEMV's MMA n = 8 columns)
+constexpr int kMaxBatchRows = 8;     // batch rows of a narrow step (the GEMV's MMA n = 8 columns)
+constexpr int kMaxWideBatch = 64;    // batch rows of a wide step (tcgen05 GEMM tiles, N up to 64)
+// wide batch: GEMM tasks of kWideRows weight rows (the tcgen05 MMA's M); the
+// global tensor maps after the per-layer ones: the LM head, then the
+// normalised activations, the attention output and the SwiGLU output (bf16)
+constexpr int kWideRows = 128;
+constexpr int kBStages = 3;  // wide batch: activation-chunk stages of the MMA issuer (in the staging buffer)
+enum TmapGlobal : int { TMG_LM = 0, TMG_XN, TMG_ATTN, TMG_H, kTmapGlobal };
 // A GEMV task's weights arrive in kGemvSlots ring slots, slot j holding columns
 // [j K / 8, (j + 1) K / 8) of all the task's rows (one 2-D TMA box per part),
 // through one tensor map per dense weight matrix: matrix m of layer l at
 // index l * kTmapPerLayer + m, the LM head after the last layer.
 constexpr int kGemvSlots = 8;
 constexpr int kTmapBytes = 128;
-enum TmapMatrix : int { TM_WQ = 0, TM_WK, TM_WV, TM_WO, TM_GATE, TM_UP, TM_DOWN, kTmapPerLayer };
+// Per layer: the dense matrices; in MoE plans TM_GATE / TM_UP / TM_DOWN map
+// the layer's expert matrices ([E * F][H] and [E * H][F], boxes of 64 columns
+// x 128 rows) and TM_XG / TM_HG the GroupGEMM activation buffers (the routed
+// token rows per expert, the SwiGLU rows) in boxes of 64 columns x 16 or 64
+// rows (the MoE-layer plan uses layer 0's entries).
+enum TmapMatrix : int {
+  TM_WQ = 0, TM_WK, TM_WV, TM_WO, TM_GATE, TM_UP, TM_DOWN, TM_XG16, TM_XG64, TM_HG16, TM_HG64, kTmapPerLayer
+};
 MK_HD int tmap_index(int layer, int m) { return layer * kTmapPerLayer + m; }
 constexpr int kMaxBatch = 128;
+// MoE GroupGEMM on tcgen05: a tile is kMoeTileRows routed rows of one expert;
+// a task covers kMoeTaskRows weight rows (gate/up: that many gate rows and as
+// many up rows; down: that many output rows), the MMA's M
+constexpr int kMoeTileRows = 64;
+constexpr int kMoeTaskRows = 128;
+constexpr int kTmemCols = 256;  // TMEM columns a CTA of an MoE plan allocates
 
 // Fixed header of the plan; passed to the kernel by value.  Offsets are in
 // bytes from the workspace base.
@@ -215,7 +240,7 @@ struct DevPlan {
   int32_t act_bytes, gred_bytes, gbatch, pad3;  // shared-memory staging buffer and partial tiles
   int32_t n_counters, debug_slots, queue_ranges;
   uint32_t debug_flags;
-  int32_t pad0;
+  int32_t fault_ctr;  // fault injection: this counter is armed one above its count (-1: none)
   int64_t spin_timeout_ns;
   EventTensorDesc ev[EV_COUNT];
   int32_t fam_first_layer[OP_COUNT];  // family index of (op, layer 0), or of the op for LM families
@@ -244,6 +269,14 @@ struct DevPlan {
   int64_t moe_stride;
   int64_t off_mhist, off_mrank, off_midx, off_mw, off_mindptr, off_mtile, off_mtile_e, off_mtile_m;
   int64_t off_mperm, off_mrow, off_mh, off_my, off_mxhat;
+  int64_t off_mxg;  // routed token rows, bf16 [E][moe_cap][H] (row = the pair's rank in its expert)
+  int32_t moe_cap;  // rows per expert in off_mxg (the plan's token maximum)
+  // wide batch: tcgen05 GEMM tasks on materialised bf16 activations
+  int32_t wide;       // 1: max_batch > kMaxBatchRows
+  int32_t attn_split; // key chunks per attention task
+  int32_t act_rows;   // rows of the activation buffers' TMA boxes (max_batch rounded up to 16)
+  int32_t pad4;
+  int64_t off_xn, off_attn_bf, off_h_bf;  // bf16 [max_batch][H], [max_batch][H], [max_batch][F]
 };
 
 // Control block at off_control (first 256 bytes of the workspace).
@@ -282,8 +315,9 @@ MK_HD QkvTile decode_qkv(const DevPlan& P, int i) {
   return t;
 }
 
-// ATTN task i -> (b, g, c) given per-sequence chunk counts nch[] and their
-// exclusive prefix pre[] (index = Hkv * pre[b] + g * nch[b] + c).
+// ATTN task i -> (b, g, c) given per-sequence task counts nch[] (key chunks
+// grouped attn_split at a time) and their exclusive prefix pre[] (index =
+// Hkv * pre[b] + g * nch[b] + c).
 struct AttnTask { int b, g, c; };
 MK_HD AttnTask decode_attn(int i, int B, int Hkv, const int* nch, const int* pre) {
   int lo = 0, hi = B - 1;

@@ -10,14 +10,16 @@ released; ``t_cstart``/``t_cend``: the compute warps started / finished it;
 ``t_data``: its first ring slot was full; ``t_done``: the controller saw it
 finish; ``t_notified``: its event counter was decremented.  GEMV tasks also
 record ``t_staged`` (activation staged), ``t_math`` (compute warp 0's
-products done) and ``t_red`` (partial tiles summed, epilogue starts).
+products done), ``t_red`` (partial tiles summed, epilogue starts),
+``t_epi`` (compute warp 0's epilogue items written) and ``t_loads`` (the
+staging's first rows loaded).
 """
 from __future__ import annotations
 
 import json
 
 FIELDS = ["family", "index", "pop", "ready", "go", "done", "notified", "cstart", "cend", "issue", "data",
-          "staged", "math", "red"]
+          "staged", "math", "red", "epi", "loads"]
 
 
 def records(trace, fam_names):

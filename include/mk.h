@@ -95,7 +95,9 @@ typedef struct mk_model_desc {
   int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
   float eps;              /* RMSNorm epsilon */
   float rope_theta;       /* rotary base; pair i of a head turns by pos*theta^(-2i/head_dim) */
-  int max_batch;          /* largest B a step may use (at most 8 for the dense and MoE decoder kinds) */
+  int max_batch;          /* largest B a step may use: dense decoder at most 64 (above 8 the plan runs
+                             the wide-batch path: materialised bf16 activations and tcgen05 GEMM
+                             tasks of 128 weight rows), MoE decoder at most 8 */
   int max_ctx;            /* cache capacity in positions (ctx_lens[b] < max_ctx) */
   int n_slots;            /* sequences the KV cache holds */
   const void* embed;      /* [vocab][hidden] bf16, device */
@@ -123,6 +125,21 @@ typedef struct mk_plan_opts {
   int tile_qkv, tile_o, tile_gu, tile_down, kseg, tile_lm, attn_chunk;
   long long spin_timeout_ns; /* device spin-wait limit; 0 = 2 s */
   unsigned debug_flags;   /* MK_DEBUG_* bits */
+  /* Fault injection for failure-detection tests (0 = none).  With
+   * MK_SIM_FAULT_COUNT_PLUS_ONE the device plan arms the event that task 0 of
+   * family `fault_family` notifies with one wait more than it will ever
+   * receive, so the tasks waiting on it run into the spin-wait limit: the
+   * kernel records MK_ERR_DEVICE_TIMEOUT (mk_get_status names the waiting
+   * task and the counter), every CTA drains its copies and exits, and the
+   * CUDA context stays usable.  Only families whose notified event does not
+   * depend on the step's symbols (qkv, oproj, gateup, down, lm) are accepted;
+   * other values are refused with MK_ERR_INVALID_ARG. */
+  int fault;
+  int fault_family;
+  /* Key chunks (attn_chunk keys each) per attention task: 0 = default (1 for
+   * max_batch <= 8, 8 above), at most 16.  A task streams its chunks through
+   * the ring with an online softmax and leaves one partial for the merge. */
+  int attn_split;
 } mk_plan_opts;
 
 typedef struct mk_plan mk_plan;
@@ -139,9 +156,18 @@ typedef struct mk_step_args {
   unsigned* trace;        /* uint32 [n_sm][trace_cap][16] or NULL (MK_DEBUG_TRACE): per CTA, record 0
                              is a header {records, notifier batches, notified tasks, fence ns} and
                              records 1.. are tasks {family, index, t_pop, t_ready, t_go, t_done,
-                             t_notified, t_compute_start, t_compute_end, t_issue, t_data, 0...};
+                             t_notified, t_compute_start, t_compute_end, t_issue, t_data, and for
+                             GEMV tasks t_staged, t_math, t_red, t_epi, t_loads};
                              times are the low 32 bits of %globaltimer in ns */
   int trace_cap;          /* records per CTA in `trace` */
+  /* Debug captures (device memory; each NULL to skip, written only when set;
+   * B is this step's batch): */
+  float* capture_resid;   /* fp32 [n_layers][B][hidden]: the residual stream after each layer */
+  void* capture_moe_in;   /* MoE decoder: bf16 [n_layers][B][hidden], each layer's MoE input
+                             (RMSNorm of the residual times the ffn_norm gain, as the router reads it) */
+  int* capture_topk;      /* MoE decoder: int32 [n_layers][B][top_k], each layer's selected experts */
+  int* capture_hist;      /* MoE decoder: int32 [n_layers][n_experts], each layer's expert histogram */
+  int* capture_indptr;    /* MoE decoder: int32 [n_layers][n_experts + 1], each layer's exp_indptr */
 } mk_step_args;
 
 /* Arguments of one MoE layer call (MK_MODEL_MOE_LAYER).  All arrays are
@@ -189,6 +215,9 @@ typedef struct mk_family_info {
 #define MK_OP_EDOWN 14    /* GroupGEMM tile: down rows of one expert x its routed rows */
 #define MK_OP_COMBINE 15  /* weighted sum of each token's top_k expert outputs (8 tokens per task) */
 #define MK_OP_MFIN 16     /* follow-up: end of the layer */
+#define MK_OP_NORM 7      /* wide batch, 8 rows: residual materialised, RMSNorm * attention gain -> bf16 */
+#define MK_OP_NORM2 9     /* wide batch, 8 rows: RMSNorm * FFN gain -> bf16 */
+#define MK_OP_NORMF 17    /* wide batch, 8 rows: final residual, RMSNorm * final gain -> bf16 */
 
 typedef struct mk_sim_report {
   int orders_run;         /* random interleavings executed */
@@ -206,6 +235,8 @@ typedef struct mk_sim_report {
 #define MK_SIM_FAULT_DROP_NOTIFY 1   /* one task of `fault_family` skips its notify */
 #define MK_SIM_FAULT_COUNT_PLUS_ONE 2 /* the wait count of one event of `fault_family` is one too high */
 #define MK_SIM_FAULT_NO_WAIT 3       /* tasks of `fault_family` do not wait on their event */
+#define MK_SIM_FAULT_COUNT_MINUS_ONE 4 /* the wait count of that event is one too low (also when the
+                                        count is armed at run time, as the MoE routing arms its tiles) */
 
 /* Last error message of the calling thread ("" if none). */
 const char* mk_last_error(void);
@@ -250,11 +281,12 @@ mk_status mk_decode_step(mk_plan* p, const mk_step_args* a, void* stream);
  *  - The plan must have been built on the current device (not host_only); a
  *    plan needing more scratch than MK_STATIC_SCRATCH_BYTES is rejected with
  *    MK_ERR_WORKSPACE.  mk_plan_bind_workspace is not needed.
- *  - The first call on a device resolves the array's address with
- *    cudaGetSymbolAddress (which may load the module), and the first call
+ *  - Every call resolves the array's address with cudaGetSymbolAddress
+ *    (the first call on a device may load the module), and the first call
  *    with a plan uploads that plan's arrays with cudaMemcpyAsync from host
- *    memory: make both before any stream capture.  No graph capture of this
- *    call is supported.
+ *    memory, again after a context reset moved the array: make the first
+ *    call before any stream capture.  No graph capture of this call is
+ *    supported.
  *  - The array is shared by every plan and every call on the device and keeps
  *    the last call's contents; each call clears the control block and task
  *    queue (cudaMemsetAsync) and starts at launch epoch 1.  Calls that overlap
@@ -315,14 +347,23 @@ int mk_plan_task_slots(const mk_plan* p);
 int mk_plan_num_families(const mk_plan* p);
 mk_status mk_plan_family_info(const mk_plan* p, int family, mk_family_info* out);
 
-/* Tile sizes the plan chose, in this order: tile_qkv, tile_o, tile_gu,
- * tile_down, kseg, tile_lm, attn_chunk, n_sm, ring_slots. */
-mk_status mk_plan_tiles(const mk_plan* p, int* out9);
+/* Where the Event Tensor counters live in the bound workspace: their byte
+ * offset from the workspace start and their number (int32 each).  After a
+ * step that completed, every counter reads zero: each wait count was met by
+ * exactly its number of notifies.  MK_ERR_INVALID_ARG for null arguments. */
+mk_status mk_plan_counter_region(const mk_plan* p, long long* byte_offset, int* n_counters);
+
+/* Tile sizes the plan chose, written to out[11] in this order: tile_qkv,
+ * tile_o, tile_gu, tile_down, kseg, tile_lm, attn_chunk, n_sm, ring_slots,
+ * attn_split (key chunks per attention task), wide (1: the wide-batch path). */
+mk_status mk_plan_tiles(const mk_plan* p, int* out);
 
 /* Host validation for one binding of the symbols (B, ctx_lens host array):
  * every event's wait count equals its number of notifiers, every wait
  * targets an event notified only by tasks earlier in the topological order,
- * and the static queues are deadlock-free.  MK_OK or MK_ERR_PLAN. */
+ * and the static queues are deadlock-free.  MoE plans are checked on a
+ * routing drawn from a fixed seed (the data-dependent counts taken as the
+ * routing follow-up arms them).  MK_OK or MK_ERR_PLAN. */
 mk_status mk_plan_validate(const mk_plan* p, int batch, const int* ctx_lens_host);
 
 /* Plan simulator (race detector): executes the lowered plan on the host in
@@ -330,7 +371,13 @@ mk_status mk_plan_validate(const mk_plan* p, int batch, const int* ctx_lens_host
  * bodies that only record the memory regions they read and write.  Checks
  * that every conflicting access pair is ordered by events (vector clocks),
  * that every task runs exactly once, that every counter ends at zero, and
- * that the static and dynamic schedules run the same task set. */
+ * that the static and dynamic schedules run the same task set.  For MoE
+ * plans (batch = tokens of the layer call; ctx_lens may be NULL for
+ * MK_MODEL_MOE_LAYER) every MoE layer gets a routing drawn from `seed` (top_k
+ * distinct experts per token, uniform for even seeds, Zipf(1.2)-weighted for
+ * odd ones); the routing follow-up then arms the data-dependent event counts
+ * and pushes as many GroupGEMM tasks as the routing's exp_indptr implies,
+ * and every order runs the dynamic schedule. */
 mk_status mk_plan_simulate(const mk_plan* p, int batch, const int* ctx_lens_host,
                            int n_orders, unsigned seed, int fault, int fault_family,
                            mk_sim_report* report);

@@ -22,8 +22,16 @@ Task families of one dense layer, in the order a layer runs them:
 After the last layer: ``lm`` (``tile_lm`` vocabulary rows each) and
 ``lmfin`` (one: the greedy token from the LM tiles' running maximum).
 
-Linear index of an ``attn`` task: ``Hkv * sum_{b'<b} nch_{b'} + g * nch_b + c``.
-``down`` tasks are numbered K-segment-major: ``kc * (H / tile_down) + n``.
+An attention task may take ``split`` consecutive key chunks (``tiles["split"]``,
+default 1): sequence b then has ``nch_b = ceil(ceil((ctx_b + 1) / chunk) /
+split)`` attention tasks per kv head.  Linear index of an ``attn`` task:
+``Hkv * sum_{b'<b} nch_{b'} + g * nch_b + c``.  ``down`` tasks are numbered
+K-segment-major: ``kc * (H / tile_down) + n``.
+
+With ``tiles["wide"]`` (the wide-batch layout, where the normalised
+activations are materialised) a layer also runs ``norm`` before ``qkv`` and
+``norm2`` before ``gateup``, and ``normf`` runs before ``lm``: one task per 8
+batch rows each.
 """
 from __future__ import annotations
 
@@ -36,9 +44,11 @@ def dense_family_extents(shape, B: int, ctx, tiles: dict) -> dict:
     """Number of tasks of each family in one layer (and after the last)."""
     H, D = shape.hidden, shape.head_dim
     Hq, Hkv = shape.n_q_heads, shape.n_kv_heads
-    nch = [_ceil(int(ctx[b]) + 1, tiles["chunk"]) for b in range(B)]
+    nch = [_ceil(_ceil(int(ctx[b]) + 1, tiles["chunk"]), tiles.get("split", 1)) for b in range(B)]
     n_lm = _ceil(shape.vocab, tiles["tile_lm"])
+    norms = {"norm": _ceil(B, 8), "norm2": _ceil(B, 8), "normf": _ceil(B, 8)} if tiles.get("wide") else {}
     return {
+        **norms,
         "qkv": (Hq + 2 * Hkv) * D // tiles["tile_qkv"],
         "attn": Hkv * sum(nch),
         "merge": Hkv * B,
@@ -59,18 +69,19 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
     """
     ext = dense_family_extents(shape, B, ctx, tiles)
     Hkv = shape.n_kv_heads
+    wide = bool(tiles.get("wide"))
     out = set()
     for l in range(shape.n_layers):
-        for fam in ("qkv", "merge", "oproj", "gateup", "down"):
+        for fam in ("qkv", "merge", "oproj", "gateup", "down") + (("norm", "norm2") if wide else ()):
             out.update((fam, l, i) for i in range(ext[fam]))
         base = 0
         for b in range(B):
-            nch = _ceil(int(ctx[b]) + 1, tiles["chunk"])
+            nch = _ceil(_ceil(int(ctx[b]) + 1, tiles["chunk"]), tiles.get("split", 1))
             for g in range(Hkv):
                 for c in range(nch):
                     out.add(("attn", l, Hkv * base + g * nch + c))
             base += nch
-    for fam in ("lm", "lmfin"):
+    for fam in ("lm", "lmfin") + (("normf",) if wide else ()):
         out.update((fam, -1, i) for i in range(ext[fam]))
     return out
 

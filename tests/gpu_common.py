@@ -10,9 +10,20 @@ TOL = 2e-2  # max |gpu - ref| <= TOL * max |ref| per compared tensor
 
 
 def rel_err(got, ref):
+    """max |got - ref| / max |ref| (recorded for the session's margin report)."""
+    from conftest import record_margin
     got = got.double().cpu()
     ref = ref.double().cpu()
-    return float((got - ref).abs().max() / ref.abs().max().clamp_min(1e-30))
+    e = float((got - ref).abs().max() / ref.abs().max().clamp_min(1e-30))
+    record_margin(e)
+    return e
+
+
+def counters_at_zero(dec):
+    """Every Event Tensor counter of the plan reads zero after a finished step."""
+    ctr = dec.counters().cpu()
+    nz = torch.nonzero(ctr).flatten().tolist()
+    assert not nz, f"{len(nz)} event counters not at zero after the step (first {nz[:5]}: {ctr[nz[:5]].tolist()})"
 
 
 def to_dev(w, dev="cuda:0"):
@@ -38,23 +49,38 @@ class DenseCase:
     def tiles_for_oracle(self):
         t = self.dec.tiles()
         return dict(tile_qkv=t["tile_qkv"], chunk=t["chunk"], tile_o=t["tile_o"], tile_gu=t["tile_gu"],
-                    tile_down=t["tile_down"], kseg=t["kseg"], tile_lm=t["tile_lm"])
+                    tile_down=t["tile_down"], kseg=t["kseg"], tile_lm=t["tile_lm"], split=t["attn_split"],
+                    wide=bool(t["wide"]))
 
-    def gpu_step(self, tokens, slots, ctx, with_logits=True, counts=True):
+    def gpu_step(self, tokens, slots, ctx, with_logits=True, counts=True, capture=False):
+        """One step through mk_decode_step; with ``capture`` also the residual
+        after every layer.  Checks the device status and that every event
+        counter ended at zero."""
         dev = "cuda:0"
         B = len(tokens)
+        cap = None
+        if capture:
+            cap = {"resid": torch.full((self.shape.n_layers, B, self.shape.hidden), float("nan"), device=dev)}
         tok = torch.tensor(tokens, dtype=torch.int32, device=dev)
         sl = torch.tensor(slots, dtype=torch.int32, device=dev)
         cx = torch.tensor(ctx, dtype=torch.int32, device=dev)
         nxt = torch.full((B,), -1, dtype=torch.int32, device=dev)
         logits = torch.empty(B, self.shape.vocab, dtype=torch.float32, device=dev) if with_logits else None
         tc = torch.zeros(mk.mk_plan_task_slots(self.dec.plan), dtype=torch.int32, device=dev) if counts else None
-        self.dec.step(tok, sl, cx, nxt, logits=logits, task_counts=tc)
+        self.dec.step(tok, sl, cx, nxt, logits=logits, task_counts=tc, capture=cap)
         torch.cuda.synchronize()
         code, st = self.dec.status()
         assert code == 0, f"device status {code} family {st.family} index {st.index} event {st.event}"
+        counters_at_zero(self.dec)
         return {"next_tokens": nxt.cpu(), "logits": None if logits is None else logits.cpu(),
-                "task_counts": None if tc is None else tc.cpu()}
+                "task_counts": None if tc is None else tc.cpu(),
+                "resid": None if cap is None else cap["resid"].cpu()}
+
+    def check_hidden(self, got, ref):
+        """The residual after every layer against the oracle's captures."""
+        for l in range(self.shape.n_layers):
+            for b in range(got["resid"].shape[1]):
+                assert rel_err(got["resid"][l, b], ref["residual"][l][b]) <= TOL, f"layer {l} row {b}"
 
     def check_task_set(self, counts, B, ctx):
         """Every task of the step ran exactly once; nothing else ran."""
@@ -79,4 +105,6 @@ def check_argmax(gpu_tok, ref_logits, tol=TOL):
         return True
     margin = float(ref[best] - ref[int(gpu_tok)])
     assert margin <= tol * float(ref.abs().max()), f"token {int(gpu_tok)} vs {best}, margin {margin}"
+    from conftest import record_margin
+    record_margin(near_tie=True)
     return False

@@ -22,9 +22,9 @@ def tiny():
     return DenseCase(wl.TINY, max_batch=4, max_ctx=320, n_slots=4, ctx_fill=[64, 0, 70, 190])
 
 
-def _oracle_step(case, tokens, slots, ctx):
+def _oracle_step(case, tokens, slots, ctx, capture=False):
     K, V = case.K_cpu.clone(), case.V_cpu.clone()
-    return case.oracle.step(K, V, tokens, slots, ctx), K, V
+    return case.oracle.step(K, V, tokens, slots, ctx, capture=capture), K, V
 
 
 def test_tiny_single_step_parity(tiny):
@@ -41,10 +41,12 @@ def test_tiny_single_step_parity(tiny):
 
 
 def test_tiny_ragged_batch_parity(tiny):
-    # sequences at context 0 (empty cache), 70 and 190 in slots 1..3
+    # sequences at context 0 (empty cache), 70 and 190 in slots 1..3; the
+    # residual after every layer is compared too
     tokens, slots, ctx = [3, 900, 511], [1, 2, 3], [0, 70, 190]
-    ref, _, _ = _oracle_step(tiny, tokens, slots, ctx)
-    got = tiny.gpu_step(tokens, slots, ctx)
+    ref, _, _ = _oracle_step(tiny, tokens, slots, ctx, capture=True)
+    got = tiny.gpu_step(tokens, slots, ctx, capture=True)
+    tiny.check_hidden(got, ref)
     for b in range(3):
         assert rel_err(got["logits"][b], ref["logits"][b]) <= TOL
         check_argmax(got["next_tokens"][b], ref["logits"][b])
@@ -118,15 +120,23 @@ def llama():
     return DenseCase(wl.LLAMA_1B, max_batch=1, max_ctx=1088, n_slots=1, ctx_fill=[1024])
 
 
-def test_llama1b_decode_parity_and_task_set(llama):
+def test_llama1b_greedy_32_steps_parity(llama):
+    # the 32-step greedy window from context 1024 against the oracle, both
+    # sides continuing from the oracle's token; task set at the first step,
+    # the residual after every layer at the first and the last step
     tokens = wl.token_ids(1, wl.LLAMA_1B.vocab).tolist()
+    llama.K.copy_(llama.K_cpu.to("cuda:0"))
+    llama.V.copy_(llama.V_cpu.to("cuda:0"))
     K, V = llama.K_cpu.clone(), llama.V_cpu.clone()
     tok, pos = tokens[0], 1024
-    for step in range(3):
-        ref = llama.oracle.step(K, V, [tok], [0], [pos])
-        got = llama.gpu_step([tok], [0], [pos], counts=(step == 0))
+    for step in range(32):
+        edge = step in (0, 31)
+        ref = llama.oracle.step(K, V, [tok], [0], [pos], capture=edge)
+        got = llama.gpu_step([tok], [0], [pos], counts=(step == 0), capture=edge)
         assert rel_err(got["logits"], ref["logits"]) <= TOL
         check_argmax(got["next_tokens"][0], ref["logits"][0])
+        if edge:
+            llama.check_hidden(got, ref)
         if step == 0:
             llama.check_task_set(got["task_counts"], 1, [pos])
         tok = int(ref["next_tokens"][0])
@@ -203,8 +213,9 @@ def test_llama1b_batch_of_eight():
     ctx = [128, 700, 1500, 2100, 64, 0, 999, 4095]
     case = DenseCase(wl.LLAMA_1B, max_batch=8, max_ctx=4104, n_slots=8, ctx_fill=ctx)
     tokens = wl.token_ids(8, wl.LLAMA_1B.vocab).tolist()
-    ref, _, _ = _oracle_step(case, tokens, list(range(8)), ctx)
-    got = case.gpu_step(tokens, list(range(8)), ctx)
+    ref, _, _ = _oracle_step(case, tokens, list(range(8)), ctx, capture=True)
+    got = case.gpu_step(tokens, list(range(8)), ctx, capture=True)
+    case.check_hidden(got, ref)
     for b in range(8):
         assert rel_err(got["logits"][b], ref["logits"][b]) <= TOL
         check_argmax(got["next_tokens"][b], ref["logits"][b])

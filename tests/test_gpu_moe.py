@@ -14,11 +14,11 @@ import event_tensor_task_b200 as mk
 import oracle
 import workloads as wl
 from oracle import tasks as ot
-from gpu_common import rel_err, TOL
+from gpu_common import rel_err, counters_at_zero, TOL
 
 pytestmark = pytest.mark.gpu
 
-TILES = {"tm": 64, "tn": 16, "td": 16}  # the plan's GroupGEMM tile sizes
+TILES = {"tm": 64, "tn": 128, "td": 128}  # the plan's GroupGEMM tile sizes (routed rows, weight rows per task)
 TINY_MOE = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
 
 
@@ -53,6 +53,7 @@ def _check(shape, layer, w_cpu, bias_cpu, T, seed=0):
     torch.cuda.synchronize()
     code, st = layer.status()
     assert code == 0, f"device status {code} family {st.family} index {st.index} event {st.event}"
+    counters_at_zero(layer)
     assert torch.equal(logits.cpu(), ref["logits"]), "router logits differ (the summation order is fixed)"
     assert torch.equal(idx.cpu(), ref["idx"])
     assert torch.equal(hist.cpu(), ref["hist"])

@@ -3,9 +3,15 @@ an MoE layer) against the CPU oracle, through mk_decode_step on cuda:0.
 
 Continuous batching: one plan, the batch size and the contexts change every
 step; skewed (Zipf) routing; dynamic schedule.  The oracle's decode step
-takes the MoE FFN on the bf16-rounded normalised residual rows.  Checked:
-logits within max |gpu - oracle| <= 2e-2 * max |oracle| and greedy tokens
-(up to near ties).
+takes the MoE FFN on the bf16-rounded normalised residual rows (the MoE
+layer's input is a stored bf16 tensor).  Checked per step:
+  - logits and the residual after every layer within max |gpu - oracle| <=
+    2e-2 * max |oracle|, greedy tokens (up to near ties);
+  - layer-local routing, exact: each layer's top-k ids, expert histogram and
+    exp_indptr equal the oracle's MoE layer run on the bf16 router input the
+    GPU captured for that layer (floating-point drift across layers cannot
+    flip a comparison there);
+  - every event counter at zero after the step.
 """
 import pytest
 import torch
@@ -13,7 +19,7 @@ import torch
 import event_tensor_task_b200 as mk
 import oracle
 import workloads as wl
-from gpu_common import rel_err, check_argmax, TOL
+from gpu_common import rel_err, check_argmax, counters_at_zero, TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -38,19 +44,35 @@ class MoeCase:
 
     def step(self, K, V, tokens, slots, ctx):
         dev = "cuda:0"
-        ref = self.orc.step(K, V, tokens, slots, ctx, moe=self.oracle_moe)
+        ref = self.orc.step(K, V, tokens, slots, ctx, moe=self.oracle_moe, capture=True)
         B = len(tokens)
+        L, H, E, k = self.shape.n_layers, self.shape.hidden, self.mshape.n_experts, self.mshape.top_k
         nxt = torch.full((B,), -1, dtype=torch.int32, device=dev)
         logits = torch.empty(B, self.shape.vocab, dtype=torch.float32, device=dev)
+        cap = {"resid": torch.full((L, B, H), float("nan"), device=dev),
+               "moe_in": torch.zeros(L, B, H, dtype=torch.bfloat16, device=dev),
+               "topk": torch.full((L, B, k), -1, dtype=torch.int32, device=dev),
+               "hist": torch.full((L, E), -1, dtype=torch.int32, device=dev),
+               "indptr": torch.full((L, E + 1), -1, dtype=torch.int32, device=dev)}
         self.dec.step(torch.tensor(tokens, dtype=torch.int32, device=dev),
                       torch.tensor(slots, dtype=torch.int32, device=dev),
-                      torch.tensor(ctx, dtype=torch.int32, device=dev), nxt, logits=logits)
+                      torch.tensor(ctx, dtype=torch.int32, device=dev), nxt, logits=logits, capture=cap)
         torch.cuda.synchronize()
         code, st = self.dec.status()
         assert code == 0, f"device status {code} family {st.family} index {st.index} event {st.event}"
+        counters_at_zero(self.dec)
         for b in range(B):
             assert rel_err(logits[b].cpu(), ref["logits"][b]) <= TOL
             check_argmax(nxt[b].cpu(), ref["logits"][b])
+        cap = {n: t.cpu() for n, t in cap.items()}
+        for l in range(L):
+            for b in range(B):
+                assert rel_err(cap["resid"][l, b], ref["residual"][l][b]) <= TOL, f"layer {l} row {b}"
+            # layer-local routing on the GPU's own bf16 router input
+            r = oracle.moe_layer(cap["moe_in"][l], self.m_cpu[l], k, self.bias)
+            assert torch.equal(cap["topk"][l], r["idx"]), f"layer {l}: top-k ids"
+            assert torch.equal(cap["hist"][l], r["hist"]), f"layer {l}: expert histogram"
+            assert torch.equal(cap["indptr"][l], r["indptr"]), f"layer {l}: exp_indptr"
         return ref
 
 

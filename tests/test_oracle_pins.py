@@ -503,6 +503,27 @@ def test_task_set_brute_force_attn_numbering():
     assert attn == list(range(n))
 
 
+def test_task_set_wide_layout_by_hand():
+    # TINY (2 layers, H 256, 4 q / 2 kv heads, F 1024, V 1024), wide layout,
+    # 128-row tiles, kseg 1024, split 8; B = 9 at contexts 0..8 except one at
+    # 600 (ceil(601 / 64) = 10 chunks -> 2 tasks), the others 1 task each.
+    # Per layer: norm 2, qkv (4 + 4) * 64 / 128 = 4, attn 2 * (8 + 2) = 20,
+    # merge 18, oproj 2, norm2 2, gateup 8, down 2; then normf 2, lm 8, lmfin 1.
+    tiles = dict(tile_qkv=128, chunk=64, tile_o=128, tile_gu=128, tile_down=128, kseg=1024, tile_lm=128,
+                 split=8, wide=True)
+    ctx = [0, 1, 2, 3, 4, 5, 6, 7, 600]
+    tasks = ot.expected_dense_tasks(wl.TINY, 9, ctx, tiles)
+    fams = {}
+    for f, l, i in tasks:
+        fams[(f, l)] = fams.get((f, l), 0) + 1
+    for l in range(2):
+        assert {k[0]: v for k, v in fams.items() if k[1] == l} == {
+            "norm": 2, "qkv": 4, "attn": 20, "merge": 18, "oproj": 2, "norm2": 2, "gateup": 8, "down": 2}
+    assert fams[("normf", -1)] == 2 and fams[("lm", -1)] == 8 and fams[("lmfin", -1)] == 1
+    # the last sequence's two tasks per kv head: Hkv * 8 + g * 2 + c
+    assert {i for f, l, i in tasks if f == "attn" and l == 0 and i >= 16} == {16, 17, 18, 19}
+
+
 def test_moe_tiles_and_task_set_by_hand():
     # hist = [3, 0, 130, 64], tm = 64: expert 0 -> one tile of 3 rows; expert 2
     # -> tiles of 64, 64, 2 rows starting at rows 3, 67, 131; expert 3 -> one

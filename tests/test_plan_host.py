@@ -63,7 +63,9 @@ def test_plan_rejects_bad_shapes():
     with pytest.raises(mk.MkError):
         _host(wl.TINY, tile_qkv=24)
     with pytest.raises(mk.MkError):
-        _host(wl.TINY, max_batch=9)
+        _host(wl.TINY, max_batch=65)
+    with pytest.raises(mk.MkError):  # the wide-batch path takes no GEMV tile options
+        _host(wl.TINY, max_batch=16, tile_o=16)
 
 
 def test_step_bytes_matches_hand_count():
@@ -145,11 +147,12 @@ def test_moe_plan_build_families_and_limits():
     fu = {f.name.decode(): f.followup for f in lay.families()}
     assert fu["mindptr"] == 1 and fu["mfin"] == 1 and fu["egu"] == 0
     ext = {f.name.decode(): f.max_extent for f in lay.families()}
-    # max tiles = ceil(512 * 8 / 64) + min(64, 4096) = 128; F/16 = 88 and H/16 = 128 tasks per tile
-    assert ext["egu"] == 128 * 88 and ext["edown"] == 128 * 128 and ext["route"] == 64
+    # max tiles = ceil(512 * 8 / 64) + min(64, 4096) = 128; per tile ceil(F/128) = 11 gate/up tasks
+    # and H/128 = 16 down tasks (128 weight rows each, the tcgen05 MMA's M)
+    assert ext["egu"] == 128 * 11 and ext["edown"] == 128 * 16 and ext["route"] == 64
     assert mk.mk_plan_workspace_bytes(lay.plan) > 512 * 8 * (1408 * 2 + 2048 * 4)
     lay.close()
-    for bad in (dict(n_experts=65), dict(top_k=9), dict(expert_ffn=1400), dict(hidden=2304)):
+    for bad in (dict(n_experts=65), dict(top_k=9), dict(expert_ffn=1400), dict(expert_ffn=1376), dict(hidden=2304)):
         shp = wl.MoEShape(**{**dict(hidden=2048, n_experts=64, top_k=8, expert_ffn=1408), **bad})
         with pytest.raises(mk.MkError):
             mk.MoELayer(shp, None, max_tokens=64, n_sm=148, host_only=True)
@@ -197,5 +200,105 @@ def test_shared_memory_split_per_max_batch():
         d = _host(wl.LLAMA_1B, max_batch=mb, max_ctx=1088, n_sm=148)
         assert d.tiles()["ring_slots"] == want
         d.close()
+    # above 8 rows the wide-batch path: no partial tiles; the staging buffer
+    # holds the MMA issuer's activation chunks (3 x rows x 128 B, rows = B
+    # rounded up to 16) or the QKV exchange (64 x rows fp32)
+    for mb, act in ((9, 8192), (64, 3 * 64 * 128)):
+        d = _host(wl.LLAMA_1B, max_batch=mb, max_ctx=1088, n_sm=148)
+        t = d.tiles()
+        assert t["tile_qkv"] == t["tile_o"] == t["tile_gu"] == t["tile_down"] == t["tile_lm"] == 128
+        assert t["ring_slots"] == (232448 - 9 * 1024 - act) // 16384
+        d.close()
     with pytest.raises(mk.MkError):
-        _host(wl.LLAMA_1B, max_batch=9, max_ctx=1088, n_sm=148)
+        _host(wl.LLAMA_1B, max_batch=65, max_ctx=1088, n_sm=148)
+
+
+# ---------------------------------------------------------------- MoE graphs in the simulator
+TINY_MOE = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
+
+
+def _moe_layer_host(n_sm=16, max_tokens=512):
+    return mk.MoELayer(wl.MOE_64x8, None, max_tokens=max_tokens, n_sm=n_sm, host_only=True)
+
+
+def _moe_decoder_host(n_sm=8, max_batch=4):
+    return mk.DenseDecoder(wl.TINY, max_batch=max_batch, max_ctx=320, n_slots=max_batch, n_sm=n_sm,
+                           host_only=True, moe=(TINY_MOE, None, None))
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 200])
+@pytest.mark.parametrize("seed", [2, 3])  # uniform and Zipf-skewed routing
+def test_moe_layer_simulator_clean(T, seed):
+    # data-dependent arming and triggering: the routing follow-up arms the
+    # down count and one gate/up count per tile, and pushes as many GroupGEMM
+    # tasks as exp_indptr implies; every order must be race-free, run each
+    # task once and leave every counter at zero
+    lay = _moe_layer_host()
+    code, rep = mk.mk_plan_simulate(lay.plan, T, None, n_orders=6, seed=seed)
+    assert code == 0, rep.first_error
+    assert rep.races == 0 and rep.deadlocks == 0 and rep.exactly_once_violations == 0 and rep.nonzero_counters == 0
+    # route + combine (ceil(T/8) each), mindptr, mfin, and per tile ceil(F/128) gate/up + H/128 down tasks
+    fixed = 2 * ((T + 7) // 8) + 2
+    assert (rep.tasks_per_order - fixed) % (11 + 16) == 0 and rep.tasks_per_order > fixed
+    mk.mk_plan_validate(lay.plan, T, None)
+
+
+def test_moe_layer_simulator_one_token_touches_eight_tiles():
+    # T = 1 with top-8 routing: 8 experts with one row each -> 8 tiles
+    lay = _moe_layer_host()
+    code, rep = mk.mk_plan_simulate(lay.plan, 1, None, n_orders=2, seed=4)
+    assert code == 0 and rep.tasks_per_order == 2 + 2 + 8 * (11 + 16), rep.first_error
+
+
+@pytest.mark.parametrize("B,ctx", [(1, [64]), (3, [5, 70, 130]), (4, [0, 1, 63, 64])])
+def test_moe_decoder_simulator_clean(B, ctx):
+    d = _moe_decoder_host()
+    for seed in (1, 2):
+        code, rep = mk.mk_plan_simulate(d.plan, B, ctx, n_orders=20, seed=seed)
+        assert code == 0, rep.first_error
+        assert rep.races == 0 and rep.deadlocks == 0 and rep.nonzero_counters == 0
+    mk.mk_plan_validate(d.plan, B, ctx)
+
+
+@pytest.mark.parametrize("fam,fault,want", [
+    ("egu", mk.MK_SIM_FAULT_DROP_NOTIFY, "deadlock"),
+    ("route", mk.MK_SIM_FAULT_COUNT_PLUS_ONE, "deadlock"),
+    ("edown", mk.MK_SIM_FAULT_DROP_NOTIFY, "deadlock"),
+    # a tile armed with one gate/up task too few: its down tasks read a
+    # SwiGLU row block that is still being written
+    ("egu", mk.MK_SIM_FAULT_COUNT_MINUS_ONE, "race"),
+    # the down count armed one too low: the combine reads unfinished rows
+    ("edown", mk.MK_SIM_FAULT_COUNT_MINUS_ONE, "race"),
+    # the routing event one too low: exp_indptr built before every pair is counted
+    ("route", mk.MK_SIM_FAULT_COUNT_MINUS_ONE, "race"),
+])
+def test_moe_layer_simulator_detects_faults(fam, fault, want):
+    # (MoE plans run the dynamic schedule only: a task is pushed when its
+    # event fires, so the data-dependent counts the routing arms are what
+    # orders the GroupGEMM tiles)
+    lay = _moe_layer_host()
+    f = [x.name.decode() for x in lay.families()].index(fam)
+    code, rep = mk.mk_plan_simulate(lay.plan, 24, None, 6, 5, fault, f)
+    assert code != 0
+    if want == "deadlock":
+        assert rep.deadlocks == rep.orders_run
+    elif want == "race":
+        assert rep.races > 0, rep.first_error
+
+
+@pytest.mark.parametrize("fam,want", [("oproj.1", "race"), ("edown.0", "race"), ("egu.1", "deadlock"),
+                                      ("combine.0", "deadlock")])
+def test_moe_decoder_count_minus_one(fam, want):
+    # ROUTE reads the residual the O projection wrote, COMBINE the rows of
+    # every down task: one notify too few releases them early.  With B = 3
+    # the layer has one COMBINE task, and with F = 64 a tile has one gate/up
+    # task, so those events armed at zero never fire (their consumers are
+    # pushed by the notify that reaches zero)
+    d = _moe_decoder_host()
+    f = [x.name.decode() for x in d.families()].index(fam)
+    code, rep = mk.mk_plan_simulate(d.plan, 3, [5, 70, 130], 20, 3, mk.MK_SIM_FAULT_COUNT_MINUS_ONE, f)
+    assert code != 0
+    if want == "race":
+        assert rep.races > 0, rep.first_error
+    else:
+        assert rep.deadlocks == rep.orders_run

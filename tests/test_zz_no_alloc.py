@@ -96,6 +96,26 @@ def test_static_scratch_switches_back_to_an_earlier_plan(gpu):
 
 
 @pytest.mark.gpu
+def test_static_scratch_dynamic_plans_back_to_back(gpu):
+    # two dynamic plans of different max_batch (so different queue and
+    # control offsets in the shared array): the larger one first, then the
+    # smaller, each bitwise equal to its workspace twin
+    dyn = mk.MK_SCHED_DYNAMIC
+    calls_b = [([9, 10, 11], [0, 1, 2], [64, 10, 130]), ([1, 2, 3], [0, 1, 2], [65, 11, 131])]
+    calls_a = [([5, 6], [0, 1], [64, 10]), ([7, 8], [0, 1], [65, 11])]
+    ref_b, _, _ = _case(wl.TINY, 4, 320, [64, 10, 130, 200], dyn, workspace=True)
+    ref_a, _, _ = _case(wl.TINY, 2, 256, [64, 10], dyn, workspace=True)
+    sta_b, _, _ = _case(wl.TINY, 4, 320, [64, 10, 130, 200], dyn, workspace=False)
+    sta_a, _, _ = _case(wl.TINY, 2, 256, [64, 10], dyn, workspace=False)
+    want = _two_calls(ref_b, calls_b, static_scratch=False) + _two_calls(ref_a, calls_a, static_scratch=False)
+    got = _two_calls(sta_b, calls_b, static_scratch=True) + _two_calls(sta_a, calls_a, static_scratch=True)
+    for (lw, nw), (lg, ng) in zip(want, got):
+        assert torch.equal(nw, ng) and torch.equal(lw, lg)
+    # every entry point counts its launches
+    assert sta_b.stats()["launches"] == 2 and sta_a.stats()["launches"] == 2
+
+
+@pytest.mark.gpu
 def test_static_scratch_rejects_a_plan_above_its_size(gpu):
     # a 32768-long context makes the rope table alone 8 MiB
     shape = wl.TINY
