@@ -64,6 +64,15 @@ def ncu_traffic(summary="megakernel_llama1b_b1_ncu.md"):
     return int(tr.group(1))
 
 
+def bf16_peak():
+    """Measured dense bf16 TFLOP/s (burst) of this machine's B200s, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -149,11 +158,12 @@ def setup_model(dev, seed=0):
 class TorchPerOpDecoder:
     """Same-box comparison point: the same decode step as ordinary per-op
     PyTorch on the same bf16 weights (cuBLAS bf16 GEMV/GEMM with the q/k/v
-    and gate/up weights concatenated, fp32 RMSNorm/RoPE/softmax, a masked GQA
-    attention over the padded cache), run eagerly or replayed as one CUDA
-    graph.  B sequences in cache slots 0..B-1 start at contexts ctx0[b]; the
-    positions and the greedy tokens advance on the device, so one captured
-    graph serves every step of the decode window."""
+    and gate/up weights concatenated, fp32 RMSNorm/RoPE, bf16 scaled-dot-
+    product attention with a length mask over the cache padded to the
+    window's last position), run eagerly or replayed as one CUDA graph.  B
+    sequences in cache slots 0..B-1 start at contexts ctx0[b]; the positions
+    and the greedy tokens advance on the device, so one captured graph serves
+    every step of the decode window."""
 
     def __init__(self, s, w, K, V, max_ctx, ctx0, window, tok0, dev):
         import torch
@@ -175,7 +185,10 @@ class TorchPerOpDecoder:
         i = torch.arange(D // 2, dtype=torch.float64)
         ang = torch.arange(max_ctx, dtype=torch.float64)[:, None] * s.rope_theta ** (-2.0 * i / D)
         self.cos, self.sin = ang.cos().float().to(dev), ang.sin().float().to(dev)
-        self.keypos = torch.arange(max_ctx, device=dev)
+        # attention reads the cache up to the longest context of the window
+        # (padded: a captured graph has static shapes), in bf16
+        self.T = min(max_ctx, int(max(ctx0)) + window)
+        self.keypos = torch.arange(self.T, device=dev)
         self.heads = torch.arange(s.n_kv_heads, device=dev)
         self.tok = torch.full((self.B,), tok0, dtype=torch.long, device=dev)
         self.counter = torch.zeros((), dtype=torch.long, device=dev)
@@ -211,10 +224,10 @@ class TorchPerOpDecoder:
             v = qkv[:, (Hq + Hkv) * D:].view(B, Hkv, D)
             self.K[l].view(-1, D).index_copy_(0, rows, k.to(torch.bfloat16).reshape(B * Hkv, D))
             self.V[l].view(-1, D).index_copy_(0, rows, v.to(torch.bfloat16).reshape(B * Hkv, D))
-            qg = q.view(B, Hkv, Hq // Hkv, D)
-            sc = torch.matmul(qg, self.K[l, :B].float().transpose(-1, -2)) * (1.0 / math.sqrt(D))
-            sc = sc.masked_fill(mask, float("-inf"))
-            o = torch.matmul(torch.softmax(sc, -1), self.V[l, :B].float()).reshape(B, Hq * D)
+            qg = q.view(B, Hkv, Hq // Hkv, D).to(torch.bfloat16)  # the group's query heads as the query rows
+            o = torch.nn.functional.scaled_dot_product_attention(
+                qg, self.K[l, :B, :, :self.T], self.V[l, :B, :, :self.T], attn_mask=~mask,
+                scale=1.0 / math.sqrt(D)).float().reshape(B, Hq * D)
             x = x + (o.to(torch.bfloat16) @ lw["wo"].T).float()
             h = self._rms(x, lw["ffn_norm"]).to(torch.bfloat16)
             gu = (h @ lw["wgu"].T).float()
@@ -272,56 +285,98 @@ def torch_baselines(s, w, K, V, max_ctx, tok0, dev, n_steps):
                     "eager and as one captured CUDA graph; device-timed with CUDA events"}
 
 
-def batch_sweep(s, w, dev, n_steps=100, batches=(1, 2, 4, 8)):
-    """Decode steps of the same 1B model at several batch sizes through ONE
-    plan and one compiled kernel (no rebuild, no graph capture), each
-    sequence at its own context drawn uniform in [128, 4096] (seeded), next
-    to the per-op PyTorch CUDA graph captured for that batch size."""
+def device_kv_cache(s, n_slots, max_ctx, ctx, dev, seed=0):
+    """A bf16 N(0, 1) cache drawn on the device (seeded), zero past each
+    sequence's context: the symbolic-batch sweep's 64-sequence cache is too
+    large to draw on the host in a bench run (parity tests use the host
+    generator on smaller cases)."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    shape = (s.n_layers, n_slots, s.n_kv_heads, max_ctx, s.head_dim)
+    K = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    V = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    for l in range(s.n_layers):
+        for b in range(len(ctx)):
+            K[l, b, :, :ctx[b]] = torch.randn(s.n_kv_heads, ctx[b], s.head_dim, generator=gen, device=dev).to(torch.bfloat16)
+            V[l, b, :, :ctx[b]] = torch.randn(s.n_kv_heads, ctx[b], s.head_dim, generator=gen, device=dev).to(torch.bfloat16)
+    return K, V
+
+
+def percentiles(ms_list):
+    """p10 / p50 / p90 of per-step device times (ms) in us."""
+    v = sorted(ms_list)
+    pick = lambda q: v[min(len(v) - 1, int(q * (len(v) - 1) + 0.5))]
+    return {"p10_us": 1000.0 * pick(0.1), "p50_us": 1000.0 * pick(0.5), "p90_us": 1000.0 * pick(0.9)}
+
+
+def timed_steps(run, n, start):
+    """Run steps start .. start + n - 1 with a CUDA event after each; returns
+    (mean ms, per-step ms list)."""
+    import torch
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    ev[0].record()
+    for i in range(n):
+        run(1, start + i)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+    return ev[0].elapsed_time(ev[n]) / n, per
+
+
+def batch_sweep(s, w, dev, n_steps=100, plans=((8, (1, 2, 4, 8)), (64, (1, 2, 4, 8, 16, 32, 64)))):
+    """Decode steps of the same 1B model at several batch sizes, each plan
+    ONE plan and one compiled kernel for all its batch sizes (no rebuild, no
+    graph capture), each sequence at its own context drawn uniform in [128,
+    4096] (seeded), next to the per-op PyTorch CUDA graph captured for that
+    batch size.  Plans: max_batch 8 (the small-batch GEMV path) and
+    max_batch 64 (the wide-batch path: tcgen05 GEMM tasks)."""
     import torch
     import event_tensor_task_b200 as mk
     import workloads as wl
-    maxB = max(batches)
+    maxB = max(mb for mb, _ in plans)
     ctx0 = [int(c) for c in wl.context_lengths(maxB, 128, 4096)]
     max_ctx = max(ctx0) + WINDOW + 32
-    K_cpu, V_cpu = wl.kv_cache(s, maxB, max_ctx, ctx0, seed=0)
-    K, V = K_cpu.to(dev), V_cpu.to(dev)
-    dec = mk.DenseDecoder(s, w, K, V, max_batch=maxB, max_ctx=max_ctx, n_slots=maxB)
+    K, V = device_kv_cache(s, maxB, max_ctx, ctx0, dev)
     peak, _ = peaks()
     slots = torch.arange(maxB, dtype=torch.int32, device=dev)
-    cases = []
-    for B in batches:
-        ctx_tab = torch.tensor([[ctx0[b] + i for b in range(B)] for i in range(WINDOW)], dtype=torch.int32,
-                               device=dev)
-        toks = torch.full((2, B), 5, dtype=torch.int32, device=dev)
+    out = {"contexts": ctx0, "plans": []}
+    graph_us = {}
+    for mb, batches in plans:
+        dec = mk.DenseDecoder(s, w, K, V, max_batch=mb, max_ctx=max_ctx, n_slots=maxB)
+        cases = []
+        for B in batches:
+            ctx_tab = torch.tensor([[ctx0[b] + i for b in range(B)] for i in range(WINDOW)], dtype=torch.int32,
+                                   device=dev)
+            toks = torch.full((2, B), 5, dtype=torch.int32, device=dev)
 
-        def run(n, start=0):
-            for i in range(start, start + n):
-                dec.step(toks[i % 2], slots[:B], ctx_tab[i % WINDOW], toks[(i + 1) % 2])
+            def run(n, start=0):
+                for i in range(start, start + n):
+                    dec.step(toks[i % 2], slots[:B], ctx_tab[i % WINDOW], toks[(i + 1) % 2])
 
-        run(5)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        run(n_steps, 5)
-        e1.record()
-        torch.cuda.synchronize()
-        code, _ = dec.status()
-        if code != 0:
-            raise SystemExit(f"device status {code} in the batch sweep (B={B})")
-        ms = e0.elapsed_time(e1) / n_steps
-        nbytes = statistics.mean(mk.mk_plan_step_bytes(dec.plan, B, [ctx0[b] + i for b in range(B)])
-                                 for i in range(WINDOW))
-        base = TorchPerOpDecoder(s, w, K, V, max_ctx, ctx0[:B], WINDOW, 5, dev)
-        base.capture()
-        gms = base.timed(n_steps, graph=True)
-        del base
-        cases.append({"B": B, "us_per_step": 1000.0 * ms, "tokens_per_s": B / (ms / 1000.0),
-                      "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
-                      "frac": nbytes / (ms * 1e-3) / 1e9 / peak,
-                      "torch_cuda_graph_us_per_step": 1000.0 * gms})
-    dec.close()
-    return {"contexts": ctx0, "note": "one plan and one kernel for every B (no rebuild, no graph re-capture); "
-                                      "this build runs B <= 8", "cases": cases}
+            run(5)
+            torch.cuda.synchronize()
+            ms, per = timed_steps(run, n_steps, 5)
+            code, _ = dec.status()
+            if code != 0:
+                raise SystemExit(f"device status {code} in the batch sweep (max_batch {mb}, B={B})")
+            nbytes = statistics.mean(mk.mk_plan_step_bytes(dec.plan, B, [ctx0[b] + i for b in range(B)])
+                                     for i in range(WINDOW))
+            if B not in graph_us:
+                base = TorchPerOpDecoder(s, w, K, V, max_ctx, ctx0[:B], WINDOW, 5, dev)
+                base.capture()
+                graph_us[B] = 1000.0 * base.timed(n_steps, graph=True)
+                del base
+            cases.append({"B": B, "us_per_step": 1000.0 * ms, **percentiles(per), "tokens_per_s": B / (ms / 1000.0),
+                          "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                          "frac": nbytes / (ms * 1e-3) / 1e9 / peak,
+                          "torch_cuda_graph_us_per_step": graph_us[B],
+                          "speedup_vs_graph": graph_us[B] / (1000.0 * ms)})
+        out["plans"].append({"max_batch": mb, "wide": bool(dec.tiles()["wide"]),
+                             "note": "one plan and one kernel for every B of this list (no rebuild, no re-capture)",
+                             "cases": cases})
+        dec.close()
+    return out
 
 
 def profile_moe(T):
@@ -346,8 +401,9 @@ def moe_decoder_bench(dev, n_steps=64):
     """The MoE decoder: 16 layers with the 1B attention shape, each FFN the
     64-expert top-8 layer (F 1408), vocab 128256, tied embeddings; Zipf(1.2)
     skewed routing; dynamic schedule; continuous batching with the batch
-    size drawn per step from {1, ..., 8} (this build's B limit) and
-    contexts starting uniform in [256, 4096].  Its 17.7 GB of expert weights
+    size drawn per step from {1, ..., 128} (one plan of max_batch 128: the
+    wide-batch attention half and LM head) and contexts starting uniform in
+    [256, 4096].  Its 17.7 GB of expert weights
     are drawn on the device (N(0, 0.02) bf16 from a seeded generator): this
     leg times the path; parity is tested on a two-layer model whose weights
     come from the seeded host generators."""
@@ -374,7 +430,7 @@ def moe_decoder_bench(dev, n_steps=64):
         mlayers.append({"router": rnd(ms.n_experts, H), "w_gate": rnd(ms.n_experts, ms.expert_ffn, H),
                         "w_up": rnd(ms.n_experts, ms.expert_ffn, H), "w_down": rnd(ms.n_experts, H, ms.expert_ffn)})
     bias = wl.zipf_bias(ms.n_experts).to(dev)
-    maxB = 8
+    maxB = 128
     ctx0 = [int(c) for c in wl.context_lengths(maxB, 256, 4096, stream="moe-decoder-ctx")]
     max_ctx = max(ctx0) + n_steps + 16
     K = torch.zeros(L, maxB, s.n_kv_heads, max_ctx, D, dtype=torch.bfloat16, device=dev)
@@ -405,16 +461,49 @@ def moe_decoder_bench(dev, n_steps=64):
     if code != 0:
         raise SystemExit(f"MoE decoder device status {code}")
     per = {}
+    step_ms = []
     for i, B in enumerate(sched[3:]):
         per.setdefault(B, []).append(ev[i].elapsed_time(ev[i + 1]))
+        step_ms.append(ev[i].elapsed_time(ev[i + 1]))
     total_ms = ev[0].elapsed_time(ev[-1])
     tokens = sum(sched[3:])
+    # algorithmic bytes of each timed step from its run-time routing: the
+    # steps are replayed (same inputs, so the same cache rows and routing) with
+    # the per-layer histogram captured, and each layer reads its router and
+    # the experts its histogram touched (17.3 MB each)
+    E, F = ms.n_experts, ms.expert_ffn
+    attn_w = L * ((32 + 2 * 8) * D * H + H * 32 * D) * 2.0
+    lm = s.vocab * H * 2.0
+    nbytes = []
+    hist = torch.empty(L, E, dtype=torch.int32, device=dev)
+    for i, a in enumerate(args[3:]):
+        B = sched[3 + i]
+        dec.step(*a, capture={"hist": hist})
+        torch.cuda.synchronize()
+        touched = int((hist > 0).sum())
+        ctx_sum = float(a[2].sum())
+        nbytes.append(attn_w + lm + L * E * H * 2.0 + touched * 3.0 * F * H * 2.0 + B * H * 2.0 +
+                      L * s.n_kv_heads * D * 2 * 2.0 * (ctx_sum + B))
+    code, _ = dec.status()
+    if code != 0:
+        raise SystemExit(f"MoE decoder device status {code} in the byte replay")
+    peak, _ = peaks()
+    achieved = statistics.mean(nbytes) / (total_ms / n_steps * 1e-3) / 1e9
     dec.close()
+    buckets = {}
+    for B, v in per.items():
+        key = "1-8" if B <= 8 else "9-32" if B <= 32 else "33-64" if B <= 64 else "65-128"
+        buckets.setdefault(key, []).extend(v)
     return {"workload": "MoE decoder: 16 layers (1B attention shape), 64 experts top-8 F 1408 per layer, vocab 128256, "
-                        "Zipf(1.2) routing, dynamic schedule, B per step from {1..8}, contexts from U[256,4096]",
+                        "Zipf(1.2) routing, dynamic schedule, B per step from {1..128}, contexts from U[256,4096]",
+            "us_per_step_by_B_bucket": {k: 1000.0 * statistics.mean(v) for k, v in sorted(buckets.items())},
             "steps": n_steps, "tokens": tokens, "tokens_per_s": tokens / (total_ms / 1000.0),
             "us_per_step": 1000.0 * total_ms / n_steps,
-            "us_per_step_by_B": {str(B): 1000.0 * statistics.mean(v) for B, v in sorted(per.items())},
+
+            **percentiles(step_ms),
+            "algorithmic_bytes_per_step": statistics.mean(nbytes), "achieved_gbs": achieved, "frac": achieved / peak,
+            "bytes_rule": "attention and router weights + the experts each layer's run-time histogram touched "
+                          "(3 x 1408 x 2048 bf16 each) + LM head + KV reads and appends + embedding rows",
             "weights": "device-drawn N(0,0.02) bf16 (seeded); parity is tested on a two-layer model"}
 
 
@@ -434,37 +523,101 @@ def moe_layer_bench(dev, n_iter=10):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # twice the L2
     peak, peak_kind = peaks()
     cases = []
+    def timed_call(layer, x, out, hist):
+        for _ in range(3):
+            layer(x, out, hist=hist)
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(n_iter):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            layer(x, out, hist=hist)
+            e1.record()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        code, _ = layer.status()
+        if code != 0:
+            raise SystemExit(f"MoE layer device status {code}")
+        return 1000.0 * total / n_iter
+
     for regime, b in (("uniform", None), ("zipf", bias)):
         layer = mk.MoELayer(shape, w, b, max_tokens=512)
+        fixed = mk.MoELayer(shape, w, b, max_tokens=512, moe_tiles=2)  # (fixed 64-row tiles, for comparison)
         for T in (1, 8, 64, 512):
             x = wl.moe_tokens(T, H, seed=0).to(dev)
             out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
             hist = torch.empty(E, dtype=torch.int32, device=dev)
-            for _ in range(3):
-                layer(x, out, hist=hist)
-            torch.cuda.synchronize()
-            total = 0.0
-            for _ in range(n_iter):
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                layer(x, out, hist=hist)
-                e1.record()
-                torch.cuda.synchronize()
-                total += e0.elapsed_time(e1)
-            code, _ = layer.status()
-            if code != 0:
-                raise SystemExit(f"MoE layer device status {code}")
-            us = 1000.0 * total / n_iter
+            us_fixed = timed_call(fixed, x, out, hist)
+            us = timed_call(layer, x, out, hist)
             touched = int((hist.cpu() > 0).sum())
             nbytes = E * H * 2 + touched * 3 * F * H * 2 + 2 * T * H * 2
             gbs = nbytes / (us * 1e-6) / 1e9
-            cases.append({"T": T, "routing": regime, "us_per_layer": us, "experts_touched": touched,
-                          "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak})
+            flops = 2.0 * T * K * 3 * F * H  # the GroupGEMM: (gate, up, down) x every routed row
+            tfs = flops / (us * 1e-6) / 1e12
+            cases.append({"T": T, "routing": regime, "us_per_layer": us, "us_fixed_64_row_tiles": us_fixed,
+                          "experts_touched": touched,
+                          "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak,
+                          "groupgemm_tflops": tfs, "frac_of_bf16_peak": tfs / bf16_peak()})
         layer.close()
+        fixed.close()
     return {"workload": "MoE FFN layer: hidden 2048, 64 experts, top-8, expert FFN 1408, bf16 N(0,0.02) weights, "
                         "x ~ N(0,1) bf16; L2 flushed before every timed call",
             "peak_gbs": peak, "peak_kind": peak_kind, "cases": cases}
+
+
+def interpreter_bench(s, w, K, V, max_ctx, dev, n_steps=200):
+    """The interpreter alone: the 1B plan at B=1 (context 1024) with empty
+    tasks (MK_DEBUG_EMPTY_TASKS: every task keeps its events, waits,
+    notifies and queue pushes, but streams no data and runs no body), static
+    and dynamic schedule.  Reports the step time, the dispatch rate (tasks
+    per microsecond over the whole GPU) and, from one traced step, the
+    notify -> wait latency between SMs: per dependency hop of a layer, the
+    first consumer's event-ready time minus the last producer's notify time."""
+    import collections
+    import torch
+    import event_tensor_task_b200 as mk
+    from event_tensor_task_b200 import trace as mtr
+    out = {}
+    hops = (("qkv", "attn"), ("merge", "oproj"), ("oproj", "gateup"), ("gateup", "down"))
+    for name, sched in (("static", mk.MK_SCHED_STATIC), ("dynamic", mk.MK_SCHED_DYNAMIC)):
+        dec = mk.DenseDecoder(s, w, K, V, max_batch=1, max_ctx=max_ctx, n_slots=1, sched=sched, empty_tasks=True,
+                              trace=True)
+        tok = torch.full((1,), 5, dtype=torch.int32, device=dev)
+        slot = torch.zeros(1, dtype=torch.int32, device=dev)
+        ctx = torch.tensor([CTX0], dtype=torch.int32, device=dev)
+        nxt = torch.empty(1, dtype=torch.int32, device=dev)
+
+        def run(n, start=0):
+            for _ in range(n):
+                dec.step(tok, slot, ctx, nxt)
+
+        run(5)
+        torch.cuda.synchronize()
+        ms, per = timed_steps(run, n_steps, 0)
+        tr = torch.zeros(148, 400, 16, dtype=torch.int32, device=dev)
+        dec.step(tok, slot, ctx, nxt, trace=tr)
+        torch.cuda.synchronize()
+        code, _ = dec.status()
+        if code != 0:
+            raise SystemExit(f"device status {code} in the interpreter bench")
+        recs = mtr.records(tr, [f.name.decode() for f in dec.families()])
+        byfam = collections.defaultdict(list)
+        for r in recs:
+            byfam[r["family"]].append(r)
+        lat = []
+        for l in range(s.n_layers):
+            for a, b in hops:
+                prod = [r["notified"] for r in byfam.get(f"{a}.{l}", []) if r["notified"] is not None]
+                cons = [r["ready"] for r in byfam.get(f"{b}.{l}", []) if r["ready"] is not None]
+                if prod and cons:
+                    lat.append((min(cons) - max(prod)) / 1000.0)
+        out[name] = {"us_per_step": 1000.0 * ms, **percentiles(per), "tasks_per_step": len(recs),
+                     "tasks_per_us": len(recs) / (1000.0 * ms),
+                     "notify_to_ready_us": {"median": statistics.median(lat) if lat else None,
+                                            "max": max(lat) if lat else None, "hops": len(lat)}}
+        dec.close()
+    return out
 
 
 def cpu_oracle_rate(s, w_cpu, K_cpu, V_cpu, n_steps):
@@ -548,6 +701,7 @@ def main():
     ap.add_argument("--no-moe", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-moe-decoder", action="store_true")
+    ap.add_argument("--no-interp", action="store_true")
     ap.add_argument("--profile-moe", type=int, default=0, metavar="T",
                     help="only run 4 MoE-layer calls on T tokens (a short command for ncu) and exit")
     args = ap.parse_args()
@@ -595,19 +749,22 @@ def main():
     if code != 0:
         raise SystemExit(f"device status {code} after warm-up (family {st.family} index {st.index})")
 
-    # ---- device-timed region: K steps, inputs resident in HBM
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- device-timed region: K steps, inputs resident in HBM (an event
+    # after every step gives the per-step percentiles)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with ClockSampler(torch.cuda.current_device() if world == 1 else local) as clk:
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        ev0.record(stream)
-        run(args.steps, args.warmup)
-        ev1.record(stream)
+        evs[0].record(stream)
+        for i in range(args.steps):
+            run(1, args.warmup + i)
+            evs[i + 1].record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-    ms = ev0.elapsed_time(ev1)
+    ms = evs[0].elapsed_time(evs[-1])
+    step_pct = percentiles([evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)])
     code, st = dec.status()
     if code != 0:
         raise SystemExit(f"device status {code} in the timed region")
@@ -660,6 +817,9 @@ def main():
         baselines["megakernel_plan_build_and_bind_ms"] = 1000.0 * (time.perf_counter() - t0)
         tmp.close()
 
+    interp = None
+    if world == 1 and not args.no_interp:
+        interp = interpreter_bench(s, w, K, V, max_ctx, dev)
     moe = None
     if world == 1 and not args.no_moe:
         moe = moe_layer_bench(dev)
@@ -684,7 +844,7 @@ def main():
         return
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "us_per_step": 1000.0 * ms_step,
+        "warmup": args.warmup, "ms_per_step": ms_step, "us_per_step": 1000.0 * ms_step, **step_pct,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) KV cache)", "config": workload_config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -695,6 +855,7 @@ def main():
         "moe_layer": moe,
         "batch_sweep": sweep,
         "moe_decoder": moe_dec,
+        "interpreter": interp,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 12, "d2h_bytes_per_step": 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),

@@ -15,6 +15,7 @@ from ._abi import (MK_MODEL_MOE_LAYER, MK_MODEL_MOE_DECODER, mk_moe_weights, mk_
                    MK_ERR_UNSUPPORTED, MK_ERR_WORKSPACE, MK_ERR_CUDA, MK_ERR_DEVICE_TIMEOUT, MK_ERR_DEVICE_BOUNDS,
                    MK_ERR_PLAN, MK_STATIC_SCRATCH_BYTES,
                    MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_MODEL_DENSE, MK_DEBUG_TASK_COUNTS, MK_DEBUG_TRACE,
+                   MK_DEBUG_EMPTY_TASKS,
                    MK_SIM_FAULT_NONE, MK_SIM_FAULT_DROP_NOTIFY, MK_SIM_FAULT_COUNT_PLUS_ONE,
                    MK_SIM_FAULT_NO_WAIT, MK_SIM_FAULT_COUNT_MINUS_ONE, OP_NAMES, mk_model_desc, mk_plan_opts, mk_step_args,
                    mk_layer_weights, mk_device_status, mk_family_info, mk_sim_report)
@@ -165,7 +166,7 @@ class DenseDecoder:
 
     def __init__(self, shape, weights=None, k_cache=None, v_cache=None, max_batch=1, max_ctx=None,
                  n_slots=None, sched=MK_SCHED_STATIC, n_sm=0, host_only=False, debug=False,
-                 spin_timeout_ns=0, trace=False, workspace=True, moe=None, **tiles):
+                 spin_timeout_ns=0, trace=False, workspace=True, moe=None, empty_tasks=False, **tiles):
         import torch
         self.shape = shape
         w = weights or {}
@@ -205,7 +206,8 @@ class DenseDecoder:
         o = mk_plan_opts()
         o.sched, o.n_sm, o.host_only = sched, n_sm, int(host_only)
         o.spin_timeout_ns = spin_timeout_ns
-        o.debug_flags = (MK_DEBUG_TASK_COUNTS if debug else 0) | (MK_DEBUG_TRACE if trace else 0)
+        o.debug_flags = ((MK_DEBUG_TASK_COUNTS if debug else 0) | (MK_DEBUG_TRACE if trace else 0) |
+                         (MK_DEBUG_EMPTY_TASKS if empty_tasks else 0))
         for k, v in tiles.items():
             setattr(o, k, int(v))
         self.desc, self.opts = d, o
@@ -282,7 +284,7 @@ class MoELayer:
     """
 
     def __init__(self, shape, weights, bias=None, max_tokens=512, n_sm=0, debug=False, spin_timeout_ns=0,
-                 host_only=False):
+                 host_only=False, moe_tiles=0):
         import torch
         self.shape = shape
         self._keep = [weights, bias]
@@ -297,6 +299,7 @@ class MoELayer:
         o.sched, o.n_sm, o.host_only = MK_SCHED_DYNAMIC, n_sm, int(host_only)
         o.spin_timeout_ns = spin_timeout_ns
         o.debug_flags = MK_DEBUG_TASK_COUNTS if debug else 0
+        o.moe_tiles = moe_tiles
         self.desc, self.opts = d, o
         self.plan = mk_plan_build(d, o)
         self.ws = None

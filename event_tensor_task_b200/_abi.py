@@ -22,6 +22,7 @@ MK_SCHED_DYNAMIC = 1
 MK_MODEL_DENSE = 0
 MK_DEBUG_TASK_COUNTS = 1
 MK_DEBUG_TRACE = 2
+MK_DEBUG_EMPTY_TASKS = 4
 MK_STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 MK_SIM_FAULT_NONE = 0
@@ -75,7 +76,7 @@ class mk_plan_opts(C.Structure):
         ("tile_qkv", C.c_int), ("tile_o", C.c_int), ("tile_gu", C.c_int), ("tile_down", C.c_int),
         ("kseg", C.c_int), ("tile_lm", C.c_int), ("attn_chunk", C.c_int),
         ("spin_timeout_ns", C.c_longlong), ("debug_flags", C.c_uint), ("fault", C.c_int),
-        ("fault_family", C.c_int), ("attn_split", C.c_int),
+        ("fault_family", C.c_int), ("attn_split", C.c_int), ("moe_tiles", C.c_int),
     ]
 
 

@@ -102,9 +102,6 @@ struct OpGeo {
   int pairs;      // 1: two parts (rotate-half or gate/up pairs)
 };
 
-// batch rows the per-CTA sequence tables hold (the kernel runs B <= kMaxB)
-constexpr int kSmemBatch = 64;
-static_assert(kMaxB <= kSmemBatch, "sequence tables too small");
 
 struct Smem {
   uint64_t full[kMaxSlots], empty[kMaxSlots];
@@ -119,7 +116,9 @@ struct Smem {
   TaskDesc cur[2];
   TaskDesc doneq[kDoneQ];
   TaskDesc followq[kFollowQ];
-  int ctx[kSmemBatch], slot[kSmemBatch], tok[kSmemBatch], nch[kSmemBatch], pre[kSmemBatch + 1];
+  // per-sequence tables of the step (max_batch entries each, pre one more),
+  // in the dynamic region after the staging buffer and the partial tiles
+  int *ctx, *slot, *tok, *nch, *pre;
   int fam_ext[kMaxFamilies];
   signed char fam_op[kMaxFamilies], fam_layer[kMaxFamilies];
   // the staging buffer, kSmemFixed bytes past this struct's start: the GEMV
@@ -244,9 +243,12 @@ __device__ __forceinline__ bool is_followup(int op) {
 // Counter a regular task waits on (-1: none).
 __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t, int B) {
   switch (t.op) {
-    case OP_NORM: return ev_ctr(P, EV_IN, t.layer);
+    case OP_NORM:  // (the MoE decoder's layers chain through the combine of the layer before)
+      return (P.kind == MK_MODEL_MOE_DECODER && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
+                                                             : ev_ctr(P, EV_IN, t.layer);
     case OP_NORM2: return ev_ctr(P, EV_O, t.layer);
-    case OP_NORMF: return ev_ctr(P, EV_IN, P.n_layers);
+    case OP_NORMF:
+      return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_MCOMB, P.n_layers - 1) : ev_ctr(P, EV_IN, P.n_layers);
     case OP_QKV:
       if (P.wide) return ev_ctr(P, EV_N1, t.layer);
       return (P.kind == MK_MODEL_MOE_DECODER && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
@@ -284,6 +286,8 @@ struct ProdFam {
   size_t task_stride;         // bytes between consecutive tasks' first rows
   const void* tm[4];          // tensor maps: GEMV parts (QKV: q, k, v); EGU: gate, up, routed rows (16-,
                               // 64-row boxes); EDOWN: down, SwiGLU rows (16-, 64-row boxes)
+  const void* xg128;          // EGU / EDOWN: the 128-row boxes of the routed and the SwiGLU rows
+  const void* hg128;
 };
 
 __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsigned char* tmaps, int fam, int op,
@@ -310,6 +314,13 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsi
       f.tm[2] = tmap(layer, TM_XG16); f.tm[3] = tmap(layer, TM_XG64);
       break;
     case OP_EDOWN: f.tm[0] = tmap(layer, TM_DOWN); f.tm[1] = tmap(layer, TM_HG16); f.tm[2] = tmap(layer, TM_HG64); break;
+    default: break;
+  }
+  f.xg128 = nullptr;
+  f.hg128 = nullptr;
+  switch (op) {
+    case OP_EGU: f.xg128 = tmap(layer, TM_XG128); break;
+    case OP_EDOWN: f.hg128 = tmap(layer, TM_HG128); break;
     default: break;
   }
   f.row_bytes = H2; f.row_stride = H2; f.row_pitch = H2; f.rps = P.slot_bytes / (int)H2; f.parts = 1;
@@ -361,18 +372,20 @@ __device__ __forceinline__ int task_slots(const DevPlan& P, const ProdFam& f, in
 }
 
 // A GroupGEMM tile's geometry: expert, m block, first compact row and row count.
-struct MoeTile { int e, m, r0, nrows; };
+struct MoeTile { int e, m, r0, nrows, tm; };
 __device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, const unsigned char* mb, int tile) {
   MoeTile t;
   t.e = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_e) + tile);
   t.m = __ldcg(reinterpret_cast<const int*>(mb + P.off_mtile_m) + tile);
   const int h = __ldcg(reinterpret_cast<const int*>(mb + P.off_mhist) + t.e);
-  t.r0 = __ldcg(reinterpret_cast<const int*>(mb + P.off_mindptr) + t.e) + t.m * P.moe_tm;
-  t.nrows = min(P.moe_tm, h - t.m * P.moe_tm);
+  const int tm = moe_tile_rows(h, P.moe_tm, P.moe_big);
+  t.r0 = __ldcg(reinterpret_cast<const int*>(mb + P.off_mindptr) + t.e) + t.m * tm;
+  t.tm = tm;
+  t.nrows = min(tm, h - t.m * tm);
   return t;
 }
-// rows of the B operand a tile loads (its TMA box): 16 for small tiles, else the tile size
-__device__ __forceinline__ int moe_tile_n(int nrows) { return nrows <= 16 ? 16 : kMoeTileRows; }
+// rows of the B operand a tile loads (its TMA box and the MMA's N): 16, 64 or 128
+__device__ __forceinline__ int moe_tile_n(int nrows) { return nrows <= 16 ? 16 : nrows <= kMoeTileRows ? kMoeTileRows : kMoeBigTileRows; }
 
 __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                          unsigned char* ws, Control* ctl) {
@@ -430,7 +443,8 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     }
     TaskDesc d;
     d.fam = fam; d.idx = idx; d.op = op; d.layer = layer;
-    d.nslots = fam >= 0 ? task_slots(P, f, idx) : 0;
+    const bool empty = (P.debug_flags & MK_DEBUG_EMPTY_TASKS) != 0;  // scheduling only: no copies
+    d.nslots = (fam >= 0 && !empty) ? task_slots(P, f, idx) : 0;
     d.slot_ph = slot | (int)(phase << 16);
     d.rec = 0;
     int k = fifo_seq % kFifo;
@@ -440,6 +454,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     mbar_arrive(&sm.fifo_full[k]);
     fifo_seq++;
     if (fam < 0) return true;
+    if (empty) { emitted++; return true; }
     if (P.wide && (op == OP_QKV || op == OP_OPROJ || op == OP_GATEUP || op == OP_DOWN || op == OP_LM)) {
       // wide batch: the task's 128 weight rows in 64-column chunks, one slot
       // per chunk and part (gate/up: the gate rows, then the up rows); the
@@ -525,8 +540,9 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
         const uint32_t bbytes = (uint32_t)nb * 128;
         fence_proxy_async_global();
         const int wrow = mt.e * (gu ? P.eff : P.hidden) + n * kMoeTaskRows;
-        const int brow = gu ? mt.e * P.moe_cap + mt.m * P.moe_tm : mt.r0;
-        const void* bmap = gu ? f.tm[nb == 16 ? 2 : 3] : f.tm[nb == 16 ? 1 : 2];
+        const int brow = gu ? mt.e * P.moe_cap + mt.m * mt.tm : mt.r0;
+        const void* bmap = gu ? (nb == 16 ? f.tm[2] : nb == kMoeTileRows ? f.tm[3] : f.xg128)
+                              : (nb == 16 ? f.tm[1] : nb == kMoeTileRows ? f.tm[2] : f.hg128);
         const int nk = (gu ? P.hidden : P.eff) / 64;
         for (int c = 0; c < nk; ++c) {
           unsigned char* dst;
@@ -743,8 +759,14 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
     case OP_EDOWN: push_range(P, S, ctl, ws, fam_of(P, OP_COMBINE, t.layer), 0, ceil_div(S.B, 8)); break;
     case OP_COMBINE:  // MoE decoder: the layer's residual is complete
       if (P.kind == MK_MODEL_MOE_DECODER) {
-        if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
-        else push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
+        if (P.wide) {
+          if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, ceil_div(S.B, 8));
+          else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, ceil_div(S.B, 8));
+        } else if (t.layer + 1 < P.n_layers) {
+          push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
+        } else {
+          push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles);
+        }
       }
       break;
     default: break;
@@ -1548,9 +1570,11 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
   float M[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running maximum per head (same in every warp)
   float L[4] = {0.f, 0.f, 0.f, 0.f};                          // this warp's running exp-sum per head
   float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+  int last_slot = 0;
   for (int cc = c0; cc < c1; ++cc) {
     uint32_t par;
     const int slot = task_slot(d, cc - c0, P.ring_slots, par);
+    last_slot = slot;
     const int n_old = max(0, min(CH, p - cc * CH));
     const bool has_new = (p - cc * CH) < CH;
     const int n_keys = n_old + (has_new ? 1 : 0);
@@ -1618,8 +1642,10 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
         }
       }
     }
-    bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the scores and the slot's K and V rows
-    if (ct == 0) mbar_arrive(&sm.empty[slot]);
+    if (cc + 1 < c1) {  // (the last chunk's slot is released after the final barrier below)
+      bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the scores and the slot's K and V rows
+      if (ct == 0) mbar_arrive(&sm.empty[slot]);
+    }
   }
   // the 8 warps' partial outputs, [w][h][64] in the staging buffer, and sums
   float* ob = sm.xs();
@@ -1630,6 +1656,7 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
       if (lane == 0) sm.alsum[w][h] = L[h];
     }
   bar_sync(BAR_COMP, kComputeThreads);
+  if (ct == 0) mbar_arrive(&sm.empty[last_slot]);  // every warp has read the last chunk's K and V rows
   if (ct < qpg * D) {
     const int h = ct >> 6, dd = ct & 63;  // h is uniform in a warp
     float O = 0.f;
@@ -1715,7 +1742,7 @@ __device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S,
   if (b >= S.B) return;
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int lx = d.op == OP_NORMF ? P.n_layers : d.layer;
-  const bool parts = d.op != OP_NORM2 && lx > 0;
+  const bool parts = P.kind == MK_MODEL_DENSE && d.op != OP_NORM2 && lx > 0;  // (an MoE decoder's x is complete)
   const void* gp = d.op == OP_NORM ? layers[d.layer].attn_norm : d.op == OP_NORM2 ? layers[d.layer].ffn_norm
                                                                                    : P.final_norm;
   float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
@@ -1742,8 +1769,8 @@ __device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S,
         reinterpret_cast<float4*>(x + c)[0] = a;
         reinterpret_cast<float4*>(x + c)[1] = e;
       }
-      // debug capture: the residual after layer lx - 1
-      if (S.cap_resid && lx > 0) {
+      // debug capture: the residual after layer lx - 1 (what NORM and NORMF reduce)
+      if (S.cap_resid && lx > 0 && d.op != OP_NORM2) {
         float4* c4 = reinterpret_cast<float4*>(S.cap_resid + ((size_t)(lx - 1) * S.B + b) * H + c);
         c4[0] = a;
         c4[1] = e;
@@ -2124,7 +2151,9 @@ __device__ __forceinline__ void task_mindptr(const DevPlan& P, const StepParams&
     int* tile_e = reinterpret_cast<int*>(mb + P.off_mtile_e);
     int* tile_m = reinterpret_cast<int*>(mb + P.off_mtile_m);
     const int h0 = lane < E ? __ldcg(hist + lane) : 0, h1 = lane + 32 < E ? __ldcg(hist + lane + 32) : 0;
-    const int c0 = (h0 + TMt - 1) / TMt, c1 = (h1 + TMt - 1) / TMt;
+    // tiles per expert, from its routed rows (routing-aware tile heights)
+    const int t0 = moe_tile_rows(h0, TMt, P.moe_big), t1 = moe_tile_rows(h1, TMt, P.moe_big);
+    const int c0 = (h0 + t0 - 1) / t0, c1 = (h1 + t1 - 1) / t1;
     int s0 = h0, s1 = h1, u0 = c0, u1 = c1;  // inclusive scans over the lanes
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -2334,6 +2363,7 @@ __device__ __forceinline__ void task_combine(const DevPlan& P, const StepParams&
 // Kernel instances: the plan kinds (MK_MODEL_*), and the dense decoder's
 // wide-batch path as an instance of its own.
 constexpr int kKindDenseWide = 3;
+constexpr int kKindMoeDecWide = 4;  // the MoE decoder above 8 rows: wide attention half, MoE FFN
 
 template <int kKind>
 __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
@@ -2343,7 +2373,8 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
   int a_tag = -1;
   uint32_t tc_n = 0;  // tcgen05 tasks run (the phase of acc_bar)
   uint32_t bq = 0;    // wide batch: activation chunks the MMA issuer loaded (stage and phase)
-  constexpr bool kWide = kKind == kKindDenseWide;
+  constexpr bool kWide = kKind == kKindDenseWide || kKind == kKindMoeDecWide;
+  constexpr bool kMoe = kKind == MK_MODEL_MOE_LAYER || kKind == MK_MODEL_MOE_DECODER || kKind == kKindMoeDecWide;
   constexpr bool tc = kKind != MK_MODEL_DENSE;
   if constexpr (tc) {
     // tensor memory for the tcgen05 accumulators, held for the kernel's lifetime
@@ -2364,8 +2395,14 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
     GemvSpec g;
     bool moe_task = false;
-    if constexpr (kKind == MK_MODEL_MOE_LAYER || kKind == MK_MODEL_MOE_DECODER) {
-      moe_task = d.op >= OP_ROUTE;
+    if (P.debug_flags & MK_DEBUG_EMPTY_TASKS) {  // interpreter measurement: no body
+      if (trec && lane == 0) trec[TR_CEND] = (uint32_t)global_ns();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.done_bar[k & 1]);
+      continue;
+    }
+    if constexpr (kMoe) {
+      moe_task = d.op >= OP_ROUTE && d.op <= OP_MFIN;
       if (d.op == OP_ROUTE) {
         task_route(P, S, sm, ws, d);
       } else if (d.op == OP_MINDPTR) {
@@ -2475,7 +2512,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   // ---- prologue: resolve the symbols, arm the Event Tensors, gather embeddings
   const bool moe = P.kind == MK_MODEL_MOE_LAYER;
   if (tid == 0) {
-    sm.bad = moe ? (B < 1 || B > P.max_tokens) : (B < 1 || B > P.max_batch || B > (P.wide ? kMaxWideBatch : kMaxB));
+    int* seq = reinterpret_cast<int*>(sm.stage() + P.act_bytes + P.gred_bytes);
+    const int mb = P.max_batch > 0 ? P.max_batch : 1;
+    sm.ctx = seq; sm.slot = seq + mb; sm.tok = seq + 2 * mb; sm.nch = seq + 3 * mb; sm.pre = seq + 4 * mb;
+    sm.bad = moe ? (B < 1 || B > P.max_tokens) : (B < 1 || B > P.max_batch || B > (P.wide ? kMaxBatch : kMaxB));
     // the ring's slots hold 128-byte-swizzled TMA boxes and tcgen05 operands,
     // whose swizzle pattern assumes 1024-byte-aligned slots
     if (smem_u32(smem_raw) & 1023u) sm.bad = 1;
@@ -2600,7 +2640,8 @@ namespace mk {
 static const void* kernel_for(const DevPlan& P) {
   switch (P.kind) {
     case MK_MODEL_MOE_LAYER: return (const void*)megakernel<MK_MODEL_MOE_LAYER>;
-    case MK_MODEL_MOE_DECODER: return (const void*)megakernel<MK_MODEL_MOE_DECODER>;
+    case MK_MODEL_MOE_DECODER:
+      return P.wide ? (const void*)megakernel<kKindMoeDecWide> : (const void*)megakernel<MK_MODEL_MOE_DECODER>;
     default: return P.wide ? (const void*)megakernel<kKindDenseWide> : (const void*)megakernel<MK_MODEL_DENSE>;
   }
 }
@@ -2683,7 +2724,9 @@ static bool encode_weight_maps(const DevPlan& P, const unsigned char* ws, std::v
           !put_sw128(tmap_index(l, TM_XG16), blk, E * cap, H, 16, "routed rows") ||
           !put_sw128(tmap_index(l, TM_XG64), blk, E * cap, H, kMoeTileRows, "routed rows") ||
           !put_sw128(tmap_index(l, TM_HG16), hblk, cap * K, F, 16, "SwiGLU rows") ||
-          !put_sw128(tmap_index(l, TM_HG64), hblk, cap * K, F, kMoeTileRows, "SwiGLU rows"))
+          !put_sw128(tmap_index(l, TM_HG64), hblk, cap * K, F, kMoeTileRows, "SwiGLU rows") ||
+          !put_sw128(tmap_index(l, TM_XG128), blk, E * cap, H, kMoeBigTileRows, "routed rows") ||
+          !put_sw128(tmap_index(l, TM_HG128), hblk, cap * K, F, kMoeBigTileRows, "SwiGLU rows"))
         return false;
     }
     if (P.kind == MK_MODEL_MOE_LAYER) return true;
@@ -2732,16 +2775,19 @@ static bool encode_weight_maps(const DevPlan& P, const unsigned char* ws, std::v
       if (!put_sw128(tmap_index(l, TM_WQ), lp.wq, (long long)Hq * D, H, kWideRows, "wq") ||
           !put_sw128(tmap_index(l, TM_WK), lp.wk, (long long)Hkv * D, H, kWideRows, "wk") ||
           !put_sw128(tmap_index(l, TM_WV), lp.wv, (long long)Hkv * D, H, kWideRows, "wv") ||
-          !put_sw128(tmap_index(l, TM_WO), lp.wo, H, (long long)Hq * D, kWideRows, "wo") ||
-          !put_sw128(tmap_index(l, TM_GATE), lp.w_gate, F, H, kWideRows, "w_gate") ||
-          !put_sw128(tmap_index(l, TM_UP), lp.w_up, F, H, kWideRows, "w_up") ||
-          !put_sw128(tmap_index(l, TM_DOWN), lp.w_down, H, F, kWideRows, "w_down"))
+          !put_sw128(tmap_index(l, TM_WO), lp.wo, H, (long long)Hq * D, kWideRows, "wo"))
+        return false;
+      if (P.kind == MK_MODEL_DENSE &&  // (an MoE decoder's entries hold its expert maps)
+          (!put_sw128(tmap_index(l, TM_GATE), lp.w_gate, F, H, kWideRows, "w_gate") ||
+           !put_sw128(tmap_index(l, TM_UP), lp.w_up, F, H, kWideRows, "w_up") ||
+           !put_sw128(tmap_index(l, TM_DOWN), lp.w_down, H, F, kWideRows, "w_down")))
         return false;
     }
     return put_sw128(g0 + TMG_LM, P.lm_head, P.vocab, H, kWideRows, "lm_head") &&
            put_sw128(g0 + TMG_XN, ws + P.off_xn, P.act_rows, H, P.act_rows, "normalised activations") &&
            put_sw128(g0 + TMG_ATTN, ws + P.off_attn_bf, P.act_rows, H, P.act_rows, "attention output") &&
-           put_sw128(g0 + TMG_H, ws + P.off_h_bf, P.act_rows, F, P.act_rows, "SwiGLU output");
+           (P.kind != MK_MODEL_DENSE ||
+            put_sw128(g0 + TMG_H, ws + P.off_h_bf, P.act_rows, F, P.act_rows, "SwiGLU output"));
   }
   for (int l = 0; l < P.n_layers; ++l) {
     const LayerPtrs& lp = layers[l];
@@ -2785,7 +2831,8 @@ mk_status dev_bind(Plan& p, void* ws, size_t bytes, void* stream, const std::vec
   cudaStream_t s = (cudaStream_t)stream;
   std::vector<unsigned char> image = image_in;
   if (!encode_weight_maps(p.dp, (const unsigned char*)ws, image, err)) return MK_ERR_INVALID_ARG;
-  size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + kSmemFixed + p.dp.act_bytes + p.dp.gred_bytes;
+  size_t smem = (size_t)p.dp.ring_slots * p.dp.slot_bytes + kSmemFixed + p.dp.act_bytes + p.dp.gred_bytes +
+                seq_table_bytes(p.dp);
   const void* kern = kernel_for(p.dp);
   cudaError_t e = ensure_smem_attr(p.device, kern, (int)smem);
   if (e == cudaSuccess) {
@@ -2891,7 +2938,8 @@ mk_status dev_launch_static(Plan& p, const mk_step_args* a, void* stream, std::s
   }
   cudaStream_t s = (cudaStream_t)stream;
   unsigned char* ws = st.addr;
-  const size_t smem = (size_t)P0.ring_slots * P0.slot_bytes + kSmemFixed + P0.act_bytes + P0.gred_bytes;
+  const size_t smem = (size_t)P0.ring_slots * P0.slot_bytes + kSmemFixed + P0.act_bytes + P0.gred_bytes +
+                      seq_table_bytes(P0);
   if (st.owner != p.uid) {
     st.owner = 0;
     e = ensure_smem_attr(p.device, kernel_for(P0), (int)smem);

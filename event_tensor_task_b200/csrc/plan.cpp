@@ -98,8 +98,10 @@ void draw_routing(const Plan& p, Binding& bd, unsigned seed, double skew) {
     for (size_t q = 0; q < r.idx.size(); ++q) r.rank[q] = r.hist[r.idx[q]]++;
     r.indptr.assign(E + 1, 0);
     for (int e = 0; e < E; ++e) r.indptr[e + 1] = r.indptr[e] + r.hist[e];
-    for (int e = 0; e < E; ++e)
-      for (int m = 0; m < ceil_div(r.hist[e], P.moe_tm); ++m) { r.tile_e.push_back(e); r.tile_m.push_back(m); }
+    for (int e = 0; e < E; ++e) {
+      const int tm = moe_tile_rows(r.hist[e], P.moe_tm, P.moe_big);
+      for (int m = 0; m < ceil_div(r.hist[e], tm); ++m) { r.tile_e.push_back(e); r.tile_m.push_back(m); }
+    }
     r.tiles = (int)r.tile_e.size();
     bd.route.push_back(std::move(r));
   }
@@ -144,8 +146,9 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
   const MoeRoute* rt = (P.kind != MK_MODEL_DENSE && li < (int)bd.route.size()) ? &bd.route[li] : nullptr;
   auto tile_rows = [&](int tile, int& r0, int& nr) {
     const int e = rt->tile_e[tile], m = rt->tile_m[tile];
-    r0 = rt->indptr[e] + m * P.moe_tm;
-    nr = std::min(P.moe_tm, rt->hist[e] - m * P.moe_tm);
+    const int tm = moe_tile_rows(rt->hist[e], P.moe_tm, P.moe_big);
+    r0 = rt->indptr[e] + m * tm;
+    nr = std::min(tm, rt->hist[e] - m * tm);
   };
   const bool wide = P.wide != 0;
   auto nsplit = [&](int b) { return ceil_div(ceil_div(bd.ctx[b] + 1, P.chunk), P.attn_split); };
@@ -179,16 +182,19 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       int b0, b1;
       rows8(idx, b0, b1);
       const int lx = op == OP_NORMF ? P.n_layers : l;
-      t.wait_ev = op == OP_NORM2 ? counter(EV_O, l) : counter(EV_IN, lx);
+      if (mdec)  // (the MoE decoder's layers chain through the combine of the layer before)
+        t.wait_ev = lx > 0 ? counter(EV_MCOMB, lx - 1) : counter(EV_IN, 0);
+      else
+        t.wait_ev = op == OP_NORM2 ? counter(EV_O, l) : counter(EV_IN, lx);
       t.notify_ev = op == OP_NORM ? counter(EV_N1, l) : op == OP_NORM2 ? counter(EV_N2, l) : counter(EV_NF, 0);
       for (int b = b0; b < b1; ++b) {
         t.reads.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
-        if (op != OP_NORM2 && lx > 0)
+        if (op != OP_NORM2 && lx > 0 && !mdec)
           for (int kc = 0; kc < P.n_kc; ++kc) {
             const long long pb = ((long long)kc * P.max_batch + b) * H;
             t.reads.push_back({BUF_DPART, pb, pb + H});
           }
-        if (op == OP_NORM) t.writes.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        if (op == OP_NORM && !mdec) t.writes.push_back({BUF_X, (long long)b * H, (long long)(b + 1) * H});
         t.writes.push_back({BUF_XN, (long long)b * H, (long long)(b + 1) * H});
       }
     } break;
@@ -279,7 +285,7 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       }
     } break;
     case OP_LM: {
-      t.wait_ev = mdec ? counter(EV_MCOMB, P.n_layers - 1) : wide ? counter(EV_NF, 0) : counter(EV_IN, P.n_layers);
+      t.wait_ev = wide ? counter(EV_NF, 0) : mdec ? counter(EV_MCOMB, P.n_layers - 1) : counter(EV_IN, P.n_layers);
       t.notify_ev = counter(EV_LM, 0);
       t.follow_fam = fam_index(OP_LMFIN, -1);
       t.follow_idx = 0;
@@ -327,7 +333,9 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       t.notify_ev = counter(EV_MH, li, tile);
       t.reads.push_back({BUF_MTAB, li, li + 1});
       {  // the tile's routed token rows
-        const long long row = ((long long)li * P.n_experts + rt->tile_e[tile]) * P.moe_cap + rt->tile_m[tile] * P.moe_tm;
+        const int e = rt->tile_e[tile];
+        const long long row = ((long long)li * P.n_experts + e) * P.moe_cap +
+                              (long long)rt->tile_m[tile] * moe_tile_rows(rt->hist[e], P.moe_tm, P.moe_big);
         t.reads.push_back({BUF_MXG, row * H, (row + nr) * H});
       }
       const long long c0 = (long long)n * P.moe_tn, c1 = std::min<long long>(P.eff, c0 + P.moe_tn);
@@ -409,8 +417,14 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
     case EV_MY: add(fam_index(OP_COMBINE, ml), 0, ceil_div(bd.B, 8)); break;
     case EV_MCOMB:
       if (!mdec) break;  // (the MoE layer's end is a follow-up)
-      if (c[0] + 1 < dp.n_layers) add(fam_index(OP_QKV, c[0] + 1), 0, dp.n_qkv_tiles);
-      else add(fam_index(OP_LM, -1), 0, dp.n_lm_tiles);
+      if (wide) {
+        if (c[0] + 1 < dp.n_layers) add(fam_index(OP_NORM, c[0] + 1), 0, n8);
+        else add(fam_index(OP_NORMF, -1), 0, n8);
+      } else if (c[0] + 1 < dp.n_layers) {
+        add(fam_index(OP_QKV, c[0] + 1), 0, dp.n_qkv_tiles);
+      } else {
+        add(fam_index(OP_LM, -1), 0, dp.n_lm_tiles);
+      }
       break;
     case EV_QKV: {
       int pre = 0;
@@ -443,7 +457,8 @@ static void smem_layout(DevPlan& P, int rows, int smem_bytes) {
   P.act_bytes = std::max(8192, (std::min(2 * rows, kMaxBatchRows) * kActPitch * 2 + 127) / 128 * 128);
   P.gred_bytes = rows > 0 ? 8 * P.gbatch * 64 * 4 : 0;
   P.smem_bytes = smem_bytes;
-  P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - P.gred_bytes) / P.slot_bytes);
+  P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - P.gred_bytes - seq_table_bytes(P)) /
+                                  P.slot_bytes);
 }
 
 
@@ -478,6 +493,8 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
   P.fault_ctr = -1;
   if (o->fault != 0) { err = "fault injection is available for decoder plans only"; return MK_ERR_INVALID_ARG; }
+  if (o->debug_flags & MK_DEBUG_EMPTY_TASKS)
+    { err = "empty tasks: an MoE layer's task graph depends on its routing"; return MK_ERR_INVALID_ARG; }
   P.n_experts = E; P.top_k = K; P.eff = FF; P.max_tokens = TM;
   P.moe_tm = kMoeTileRows;  // routed rows per GroupGEMM tile
   P.moe_tn = kMoeTaskRows;  // gate rows (and as many up rows) per EGU task
@@ -485,6 +502,8 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   P.nt_gu = ceil_div(FF, P.moe_tn);
   P.nt_d = H / P.moe_td;
   P.moe_cap = TM;
+  if (o->moe_tiles < 0 || o->moe_tiles > 2) { err = "moe_tiles must be 0, 1 or 2"; return MK_ERR_INVALID_ARG; }
+  P.moe_big = o->moe_tiles != 2;
   // sum over experts of ceil(hist_e / tm) <= T*k/tm + (experts with a row)
   P.max_tiles = ceil_div(TM * K, P.moe_tm) + std::min(E, TM * K);
   P.slot_bytes = 16384;
@@ -566,6 +585,8 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   // FFN families of build_moe_plan on the B tokens (dynamic schedule only)
   const bool mdec = m->kind == MK_MODEL_MOE_DECODER;
   const int H = m->hidden, D = m->head_dim, Hq = m->n_q_heads, Hkv = m->n_kv_heads, F = mdec ? 0 : m->ffn;
+  if (mdec && (o->debug_flags & MK_DEBUG_EMPTY_TASKS))
+    { err = "empty tasks: an MoE layer's task graph depends on its routing"; return MK_ERR_INVALID_ARG; }
   if (mdec) {
     const int E = m->n_experts, K = m->top_k, FF = m->expert_ffn;
     if (E < 1 || E > 64) { err = "n_experts must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
@@ -581,9 +602,12 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (H % 256 || H > 2048 || H < 256) { err = "hidden must be a multiple of 256 in [256, 2048]"; return MK_ERR_UNSUPPORTED; }
   if (!mdec && (F % 256 || F < 256)) { err = "ffn must be a positive multiple of 256"; return MK_ERR_UNSUPPORTED; }
   // above kMaxBatchRows the dense decoder runs the wide-batch path
-  const bool wide = !mdec && m->max_batch > kMaxBatchRows;
-  if (m->max_batch < 1 || m->max_batch > (mdec ? kMaxBatchRows : kMaxWideBatch))
-    { err = mdec ? "max_batch must be in [1, 8] for an MoE decoder" : "max_batch must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
+  // (an MoE decoder above 8 rows runs the wide-batch attention half and LM
+  // head; its FFN is the MoE layer either way)
+  const bool wide = m->max_batch > kMaxBatchRows;
+  const bool dwide = wide && !mdec;
+  if (m->max_batch < 1 || m->max_batch > (mdec ? kMaxBatch : kMaxWideBatch))
+    { err = mdec ? "max_batch must be in [1, 128] for an MoE decoder" : "max_batch must be in [1, 64]"; return MK_ERR_UNSUPPORTED; }
   if (m->max_ctx < 2 || m->n_slots < m->max_batch) { err = "max_ctx >= 2 and n_slots >= max_batch required"; return MK_ERR_INVALID_ARG; }
   if (o->sched != MK_SCHED_STATIC && o->sched != MK_SCHED_DYNAMIC) { err = "unknown schedule"; return MK_ERR_INVALID_ARG; }
   if (n_sm < 1 || n_sm > 1024) { err = "n_sm out of range"; return MK_ERR_INVALID_ARG; }
@@ -630,6 +654,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
       { err = "the wide-batch path takes no GEMV tile options"; return MK_ERR_INVALID_ARG; }
     P.tile_qkv = P.tile_o = P.tile_gu = P.tile_down = P.tile_lm = kWideRows;
     if (H % kWideRows || F % kWideRows) { err = "wide batch: hidden and ffn must be multiples of 128"; return MK_ERR_UNSUPPORTED; }
+    if (P.vocab < 1) { err = "non-positive vocabulary"; return MK_ERR_INVALID_ARG; }
     if (Hq / Hkv < 2 || (Hq / Hkv) % 2) { err = "wide batch: an even number of query heads per kv head"; return MK_ERR_UNSUPPORTED; }
   }
   P.act_rows = ceil_div(P.max_batch, 16) * 16;
@@ -662,7 +687,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     P.act_bytes = std::max(std::max(8192, 64 * P.act_rows * 4), kBStages * P.act_rows * 128);
     P.gred_bytes = 0;
     P.smem_bytes = smem_bytes;
-    P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes) / P.slot_bytes);
+    P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - seq_table_bytes(P)) / P.slot_bytes);
   } else {
     smem_layout(P, P.max_batch, smem_bytes);
   }
@@ -709,13 +734,18 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     P.nt_gu = ceil_div(P.eff, P.moe_tn);
     P.nt_d = H / P.moe_td;
     P.moe_cap = P.max_tokens;
+    if (o->moe_tiles < 0 || o->moe_tiles > 2) { err = "moe_tiles must be 0, 1 or 2"; return MK_ERR_INVALID_ARG; }
+    P.moe_big = o->moe_tiles != 2;
     P.max_tiles = ceil_div(P.max_tokens * P.top_k, P.moe_tm) + std::min(P.n_experts, P.max_tokens * P.top_k);
     }
   const int e_tok8 = Emit(p.code).op(X_B).push(8).op(X_CEILDIV).ret();  // ceil(B / 8)
   static const int kMoeDecOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU, OP_EDOWN,
                                    OP_COMBINE};
   static const int kWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_NORM2, OP_GATEUP, OP_DOWN};
-  const int fam_per_layer = mdec ? 9 : wide ? 8 : kFamPerLayer;
+  static const int kMoeDecWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU,
+                                       OP_EDOWN, OP_COMBINE};
+  const int fam_per_layer = mdec ? (wide ? 10 : 9) : wide ? 8 : kFamPerLayer;
+  const int* layer_ops = mdec ? (wide ? kMoeDecWideOps : kMoeDecOps) : wide ? kWideOps : kLayerOps;
   const int max_tasks_attn = Hkv * P.max_batch * ceil_div(P.max_chunks, P.attn_split);
   for (int l = 0; l < P.n_layers; ++l) {
     if (wide) add_family(OP_NORM, l, e_tok8, ceil_div(P.max_batch, 8), 0);
@@ -723,7 +753,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     add_family(OP_ATTN, l, e_attn, max_tasks_attn, 0);
     add_family(OP_MERGE, l, e_merge, Hkv * P.max_batch, 1);
     add_family(OP_OPROJ, l, emit_const(p.code, P.n_otiles), P.n_otiles, 0);
-    if (wide) add_family(OP_NORM2, l, e_tok8, ceil_div(P.max_batch, 8), 0);
+    if (dwide) add_family(OP_NORM2, l, e_tok8, ceil_div(P.max_batch, 8), 0);
     if (mdec) {
       add_family(OP_ROUTE, l, e_tok8, ceil_div(P.max_tokens, 8), 0);
       add_family(OP_MINDPTR, l, emit_const(p.code, 1), 1, 1);
@@ -743,7 +773,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.debug_slots = debug_base;
   P.fam_stride = fam_per_layer;
   for (int op = 0; op < OP_COUNT; ++op) P.fam_first_layer[op] = -1;
-  for (int k = 0; k < fam_per_layer; ++k) P.fam_first_layer[mdec ? kMoeDecOps[k] : wide ? kWideOps[k] : kLayerOps[k]] = k;
+  for (int k = 0; k < fam_per_layer; ++k) P.fam_first_layer[layer_ops[k]] = k;
   {
     int g0 = P.n_layers * fam_per_layer;
     if (wide) P.fam_first_layer[OP_NORMF] = g0++;
@@ -782,7 +812,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   }
   if (wide) {
     add_event(EV_N1, 1, L, 1, 1, e_tok8);
-    add_event(EV_N2, 1, L, 1, 1, e_tok8);
+    add_event(EV_N2, 1, dwide ? L : 0, 1, 1, e_tok8);
     add_event(EV_NF, 1, 1, 1, 1, e_tok8);
   } else {
     for (int id = EV_N1; id < EV_COUNT; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // wide only: empty
@@ -820,7 +850,9 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   // COMBINE (1 each) and EDOWN (one per tile); then LM (1) and END (1)
   // wide batch: NORM, QKV, OPROJ, NORM2, GATEUP (1 each), ATTN (one per
   // sequence), DOWN (one per K segment); then NORMF, LM and END
-  P.queue_ranges = mdec ? L * (5 + Hkv * P.max_batch + P.max_tiles) + 2
+  // (MoE decoder, wide: NORM, QKV, OPROJ, ROUTE, EGU, COMBINE, ATTN per
+  // sequence, EDOWN per tile; then NORMF, LM, END)
+  P.queue_ranges = mdec ? (wide ? L * (6 + P.max_batch + P.max_tiles) + 3 : L * (5 + Hkv * P.max_batch + P.max_tiles) + 2)
                    : wide ? L * (5 + P.max_batch + P.n_kc) + 3
                           : L * (3 + Hkv * P.max_batch + P.n_kc) + 2;
 

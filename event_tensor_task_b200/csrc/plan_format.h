@@ -189,6 +189,10 @@ struct LayerPtrs {
 };
 
 constexpr int kMaxFamilies = 256;
+struct DevPlan;
+// bytes of the per-sequence tables (ctx, slot, token, attention tasks and
+// their prefix; max_batch ints each, one more for the prefix)
+MK_HD int seq_table_bytes_for(int max_batch) { return ((5 * (max_batch > 0 ? max_batch : 1) + 1) * 4 + 127) / 128 * 128; }
 // Dynamic shared memory of a CTA: the ring (ring_slots x slot_bytes), the
 // kernel's fixed control area (at most kSmemFixed bytes), the staging buffer
 // (act_bytes: the GEMV activation rows in bf16, kActPitch elements per batch
@@ -216,7 +220,8 @@ constexpr int kTmapBytes = 128;
 // token rows per expert, the SwiGLU rows) in boxes of 64 columns x 16 or 64
 // rows (the MoE-layer plan uses layer 0's entries).
 enum TmapMatrix : int {
-  TM_WQ = 0, TM_WK, TM_WV, TM_WO, TM_GATE, TM_UP, TM_DOWN, TM_XG16, TM_XG64, TM_HG16, TM_HG64, kTmapPerLayer
+  TM_WQ = 0, TM_WK, TM_WV, TM_WO, TM_GATE, TM_UP, TM_DOWN, TM_XG16, TM_XG64, TM_HG16, TM_HG64,
+  TM_XG128, TM_HG128, kTmapPerLayer
 };
 MK_HD int tmap_index(int layer, int m) { return layer * kTmapPerLayer + m; }
 constexpr int kMaxBatch = 128;
@@ -225,6 +230,11 @@ constexpr int kMaxBatch = 128;
 // many up rows; down: that many output rows), the MMA's M
 constexpr int kMoeTileRows = 64;
 constexpr int kMoeTaskRows = 128;
+constexpr int kMoeBigTileRows = 128;  // routing-aware tiles: experts with more rows than kMoeTileRows
+// Rows per GroupGEMM tile of an expert with h routed rows: with routing-aware
+// tiles (moe_big), an expert holding more than kMoeTileRows rows gets tiles of
+// kMoeBigTileRows, so its weights stream once per 128 rows instead of 64.
+MK_HD int moe_tile_rows(int h, int tm, int big) { return (big && h > tm) ? kMoeBigTileRows : tm; }
 constexpr int kTmemCols = 256;  // TMEM columns a CTA of an MoE plan allocates
 
 // Fixed header of the plan; passed to the kernel by value.  Offsets are in
@@ -271,6 +281,8 @@ struct DevPlan {
   int64_t off_mperm, off_mrow, off_mh, off_my, off_mxhat;
   int64_t off_mxg;  // routed token rows, bf16 [E][moe_cap][H] (row = the pair's rank in its expert)
   int32_t moe_cap;  // rows per expert in off_mxg (the plan's token maximum)
+  int32_t moe_big;  // routing-aware tiles (see moe_tile_rows)
+  int32_t pad5;
   // wide batch: tcgen05 GEMM tasks on materialised bf16 activations
   int32_t wide;       // 1: max_batch > kMaxBatchRows
   int32_t attn_split; // key chunks per attention task
@@ -278,6 +290,8 @@ struct DevPlan {
   int32_t pad4;
   int64_t off_xn, off_attn_bf, off_h_bf;  // bf16 [max_batch][H], [max_batch][H], [max_batch][F]
 };
+
+MK_HD int seq_table_bytes(const DevPlan& P) { return seq_table_bytes_for(P.max_batch); }
 
 // Control block at off_control (first 256 bytes of the workspace).
 struct Control {

@@ -54,6 +54,9 @@ typedef int mk_status;
 
 #define MK_DEBUG_TASK_COUNTS 1u  /* each executed task increments its slot in mk_step_args.task_counts */
 #define MK_DEBUG_TRACE 2u        /* the controller records per-task timestamps in mk_step_args.trace */
+#define MK_DEBUG_EMPTY_TASKS 4u  /* interpreter measurement (dense plans only): every task keeps its events,
+                                    queue pushes and pops but streams no data and runs no body, so a
+                                    step times the scheduling alone (its outputs are not computed) */
 
 /* Weights of one mixture-of-experts FFN layer; bf16 row-major, device. */
 typedef struct mk_moe_weights {
@@ -140,6 +143,12 @@ typedef struct mk_plan_opts {
    * max_batch <= 8, 8 above), at most 16.  A task streams its chunks through
    * the ring with an online softmax and leaves one partial for the merge. */
   int attn_split;
+  /* MoE GroupGEMM tiles, chosen per expert from the run-time histogram
+   * (0 = default: routing-aware; 1 = routing-aware; 2 = fixed): an expert
+   * with more than 64 routed rows gets tiles of 128 rows (its weights stream
+   * once per 128 rows), the others tiles of 64 (16 when a tile has at most
+   * 16 rows, as the MMA's N). */
+  int moe_tiles;
 } mk_plan_opts;
 
 typedef struct mk_plan mk_plan;

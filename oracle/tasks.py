@@ -86,18 +86,22 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
     return out
 
 
-def moe_tiles(hist, tm: int):
+def moe_tiles(hist, tm: int, big: int = 0):
     """GroupGEMM tiles of an MoE layer: expert ``e``'s ``hist[e]`` rows split
-    into ``ceil(hist[e] / tm)`` tiles of at most ``tm`` rows, numbered expert
-    by expert in increasing expert id ("Event Tensor: A Unified Abstraction
-    for Compiling Dynamic Megakernel", section "Core method": the prefix sum
-    of the per-expert counts decides how many GroupGEMM tiles each expert
-    triggers).  Returns ``[(expert, first row, rows), ...]`` with rows
-    counted from ``exp_indptr[e]``."""
+    into ``ceil(hist[e] / tm_e)`` tiles of at most ``tm_e`` rows, numbered
+    expert by expert in increasing expert id ("Event Tensor: A Unified
+    Abstraction for Compiling Dynamic Megakernel", section "Core method": the
+    prefix sum of the per-expert counts decides how many GroupGEMM tiles each
+    expert triggers).  ``tm_e = tm``, or with routing-aware tiles (``big`` > 0;
+    "RaMP: Runtime-Aware Megakernel Polymorphism for Mixture-of-Experts": the
+    tile configuration follows the run-time histogram) ``tm_e = big`` for an
+    expert with more than ``tm`` rows.  Returns ``[(expert, first row, rows),
+    ...]`` with rows counted from ``exp_indptr[e]``."""
     tiles, row = [], 0
     for e, h in enumerate(int(v) for v in hist):
-        for m in range(_ceil(h, tm)):
-            tiles.append((e, row + m * tm, min(tm, h - m * tm)))
+        te = big if (big and h > tm) else tm
+        for m in range(_ceil(h, te)):
+            tiles.append((e, row + m * te, min(te, h - m * te)))
         row += h
     return tiles
 
@@ -110,7 +114,7 @@ def expected_moe_tasks(T: int, hist, hidden: int, expert_ffn: int, tiles: dict) 
     numbered ``tile * ceil(F / tn) + n``; ``edown``: ``tiles * (H / td)``
     numbered ``tile * (H / td) + n``.
     """
-    n_tiles = len(moe_tiles(hist, tiles["tm"]))
+    n_tiles = len(moe_tiles(hist, tiles["tm"], tiles.get("big", 0)))
     nt_gu = _ceil(expert_ffn, tiles["tn"])
     nt_d = hidden // tiles["td"]
     out = set()

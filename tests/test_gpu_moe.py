@@ -18,7 +18,9 @@ from gpu_common import rel_err, counters_at_zero, TOL
 
 pytestmark = pytest.mark.gpu
 
-TILES = {"tm": 64, "tn": 128, "td": 128}  # the plan's GroupGEMM tile sizes (routed rows, weight rows per task)
+# the plan's GroupGEMM tiles: routed rows per tile (128 for experts with more
+# than 64 rows: routing-aware), weight rows per task
+TILES = {"tm": 64, "big": 128, "tn": 128, "td": 128}
 TINY_MOE = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
 
 

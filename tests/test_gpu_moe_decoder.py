@@ -61,18 +61,18 @@ class MoeCase:
         code, st = self.dec.status()
         assert code == 0, f"device status {code} family {st.family} index {st.index} event {st.event}"
         counters_at_zero(self.dec)
-        for b in range(B):
-            assert rel_err(logits[b].cpu(), ref["logits"][b]) <= TOL
-            check_argmax(nxt[b].cpu(), ref["logits"][b])
         cap = {n: t.cpu() for n, t in cap.items()}
-        for l in range(L):
-            for b in range(B):
-                assert rel_err(cap["resid"][l, b], ref["residual"][l][b]) <= TOL, f"layer {l} row {b}"
+        for l in range(L):  # (layer by layer first: a failure names the layer)
             # layer-local routing on the GPU's own bf16 router input
             r = oracle.moe_layer(cap["moe_in"][l], self.m_cpu[l], k, self.bias)
             assert torch.equal(cap["topk"][l], r["idx"]), f"layer {l}: top-k ids"
             assert torch.equal(cap["hist"][l], r["hist"]), f"layer {l}: expert histogram"
             assert torch.equal(cap["indptr"][l], r["indptr"]), f"layer {l}: exp_indptr"
+            for b in range(B):
+                assert rel_err(cap["resid"][l, b], ref["residual"][l][b]) <= TOL, f"layer {l} row {b}"
+        for b in range(B):
+            assert rel_err(logits[b].cpu(), ref["logits"][b]) <= TOL, f"logits row {b}"
+            check_argmax(nxt[b].cpu(), ref["logits"][b])
         return ref
 
 
@@ -116,3 +116,45 @@ def test_moe_decoder_1b_attention_64_experts():
     _walk(case, [([tok[0]], [0], [256]),
                  (tok[:3], [0, 1, 2], [257, 1000, 512]),
                  (tok, [0, 1, 2, 3], [258, 1001, 513, 300])])
+
+
+def test_tiny_moe_decoder_wide_batch():
+    # above 8 rows the decoder's attention half and LM head run the wide-batch
+    # path (tcgen05 GEMM tasks on materialised bf16 activations); its FFN is
+    # the MoE layer on the B tokens: one plan for B = 16, 9 and 12
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    mshape = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
+    fill = [64, 10, 130, 200, 0, 77, 250, 5, 1, 2, 3, 100, 64, 65, 129, 33]
+    case = MoeCase(wl.TINY, mshape, max_batch=16, max_ctx=320, ctx_fill=fill)
+    assert case.dec.tiles()["wide"] == 1
+    tok = wl.token_ids(16, wl.TINY.vocab).tolist()
+    _walk(case, [(tok, list(range(16)), fill),
+                 (tok[:9], [15, 0, 4, 2, 5, 7, 9, 11, 13], [34, 65, 1, 131, 78, 6, 3, 101, 65]),
+                 (tok[:12], list(range(12)), [65, 11, 131, 201, 1, 79, 251, 7, 2, 4, 4, 102])])
+
+
+def test_tiny_moe_decoder_batch_128():
+    # the widest plan (max_batch 128: activation boxes and MMA N of 128 rows)
+    # on the tiny shape, B = 128 and 70
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    mshape = wl.MoEShape(hidden=256, n_experts=8, top_k=2, expert_ffn=64)
+    fill = [int(c) for c in wl.context_lengths(128, 0, 300, stream="tiny-128")]
+    case = MoeCase(wl.TINY, mshape, max_batch=128, max_ctx=320, ctx_fill=fill)
+    tok = wl.token_ids(128, wl.TINY.vocab).tolist()
+    _walk(case, [(tok, list(range(128)), fill),
+                 (tok[:70], list(range(70)), [c + 1 for c in fill[:70]])])
+
+
+def test_moe_decoder_1b_attention_batch_128():
+    # the MoE decoder workload's width: two layers of the 1B attention shape,
+    # 64 experts top-8 per layer, B = 128 with contexts uniform in [256, 4096]
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    shape = wl.DenseShape(n_layers=2, hidden=2048, n_q_heads=32, n_kv_heads=8, head_dim=64, ffn=8192,
+                          vocab=128256)
+    ctx = [int(c) for c in wl.context_lengths(128, 256, 4096, stream="moe-decoder-ctx")]
+    case = MoeCase(shape, wl.MOE_64x8, max_batch=128, max_ctx=4104, ctx_fill=ctx)
+    tok = wl.token_ids(128, shape.vocab).tolist()
+    _walk(case, [(tok, list(range(128)), ctx)])

@@ -529,6 +529,9 @@ def test_moe_tiles_and_task_set_by_hand():
     # -> tiles of 64, 64, 2 rows starting at rows 3, 67, 131; expert 3 -> one
     # tile of 64 rows at row 133.  5 tiles.
     assert ot.moe_tiles([3, 0, 130, 64], 64) == [(0, 0, 3), (2, 3, 64), (2, 67, 64), (2, 131, 2), (3, 133, 64)]
+    # routing-aware heights: expert 2 (130 > 64 rows) -> tiles of 128, 2 rows;
+    # expert 3 (exactly 64) keeps one 64-row tile
+    assert ot.moe_tiles([3, 0, 130, 64], 64, big=128) == [(0, 0, 3), (2, 3, 128), (2, 131, 2), (3, 133, 64)]
     # T = 25 tokens: 4 route + 4 combine tasks; F = 1408, tn = 8 -> 176 gate/up
     # tasks per tile; H = 2048, td = 8 -> 256 down tasks per tile
     tasks = ot.expected_moe_tasks(25, [3, 0, 130, 64], 2048, 1408, {"tm": 64, "tn": 8, "td": 8})
