@@ -76,7 +76,7 @@ class mk_plan_opts(C.Structure):
         ("tile_qkv", C.c_int), ("tile_o", C.c_int), ("tile_gu", C.c_int), ("tile_down", C.c_int),
         ("kseg", C.c_int), ("tile_lm", C.c_int), ("attn_chunk", C.c_int),
         ("spin_timeout_ns", C.c_longlong), ("debug_flags", C.c_uint), ("fault", C.c_int),
-        ("fault_family", C.c_int), ("attn_split", C.c_int), ("moe_tiles", C.c_int),
+        ("fault_family", C.c_int), ("attn_split", C.c_int), ("moe_tiles", C.c_int), ("act_split", C.c_int),
     ]
 
 

@@ -61,6 +61,19 @@ constexpr int kMaxB = kMaxBatchRows;  // batch rows per step on this path
 constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
 constexpr int kDynLookahead = 2;
 
+// Kernel instances: the plan kinds (MK_MODEL_*) and the wide-batch layouts
+// (max_batch > 8) of the dense and the MoE decoder, each with only the code
+// paths its plans take (the interpreter roles included).
+constexpr int kKindDenseWide = 3;
+constexpr int kKindMoeDecWide = 4;  // the MoE decoder above 8 rows: wide attention half, MoE FFN
+template <int K>
+struct Kind {
+  static constexpr bool wide = K == kKindDenseWide || K == kKindMoeDecWide;
+  static constexpr bool moe_layer = K == MK_MODEL_MOE_LAYER;
+  static constexpr bool moe_dec = K == MK_MODEL_MOE_DECODER || K == kKindMoeDecWide;
+  static constexpr bool moe = moe_layer || moe_dec;
+};
+
 struct StepParams {
   int B;                 // batch size; the token count T for an MoE layer
   // MoE layer
@@ -136,7 +149,8 @@ struct Smem {
   uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
   // attention scratch: the group's queries, the chunk's scores, the new
   // K and V rows (bf16, as in the cache) and the warps' exp-sums
-  float aq[4][64], asc[4][64];
+  alignas(16) float aq[4][64];
+  float asc[4][64];
   uint4 anew[16];
   float alsum[kComputeWarps][4];
   volatile int released;  // regular tasks the controller has handed to compute
@@ -241,30 +255,32 @@ __device__ __forceinline__ bool is_followup(int op) {
 }
 
 // Counter a regular task waits on (-1: none).
+template <int kKind>
 __device__ int wait_counter(const DevPlan& P, const Smem& sm, const TaskDesc& t, int B) {
+  constexpr bool kW = Kind<kKind>::wide, kMD = Kind<kKind>::moe_dec;
   switch (t.op) {
     case OP_NORM:  // (the MoE decoder's layers chain through the combine of the layer before)
-      return (P.kind == MK_MODEL_MOE_DECODER && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
+      return (kMD && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
                                                              : ev_ctr(P, EV_IN, t.layer);
     case OP_NORM2: return ev_ctr(P, EV_O, t.layer);
     case OP_NORMF:
-      return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_MCOMB, P.n_layers - 1) : ev_ctr(P, EV_IN, P.n_layers);
+      return kMD ? ev_ctr(P, EV_MCOMB, P.n_layers - 1) : ev_ctr(P, EV_IN, P.n_layers);
     case OP_QKV:
-      if (P.wide) return ev_ctr(P, EV_N1, t.layer);
-      return (P.kind == MK_MODEL_MOE_DECODER && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
+      if (kW) return ev_ctr(P, EV_N1, t.layer);
+      return (kMD && t.layer > 0) ? ev_ctr(P, EV_MCOMB, t.layer - 1)
                                                              : ev_ctr(P, EV_IN, t.layer);
     case OP_ATTN: {
-      if (P.wide) return ev_ctr(P, EV_QKV, t.layer, 0);
+      if (kW) return ev_ctr(P, EV_QKV, t.layer, 0);
       AttnTask a = decode_attn(t.idx, B, P.n_kv_heads, sm.nch, sm.pre);
       return ev_ctr(P, EV_QKV, t.layer, a.g);
     }
     case OP_OPROJ: return ev_ctr(P, EV_ATTN, t.layer);
-    case OP_GATEUP: return P.wide ? ev_ctr(P, EV_N2, t.layer) : ev_ctr(P, EV_O, t.layer);
+    case OP_GATEUP: return kW ? ev_ctr(P, EV_N2, t.layer) : ev_ctr(P, EV_O, t.layer);
     case OP_DOWN: return ev_ctr(P, EV_GU, t.layer, t.idx / P.n_dtiles);
     case OP_LM:
-      if (P.wide) return ev_ctr(P, EV_NF, 0);
-      return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_MCOMB, P.n_layers - 1) : ev_ctr(P, EV_IN, P.n_layers);
-    case OP_ROUTE: return P.kind == MK_MODEL_MOE_DECODER ? ev_ctr(P, EV_O, t.layer) : -1;
+      if (kW) return ev_ctr(P, EV_NF, 0);
+      return kMD ? ev_ctr(P, EV_MCOMB, P.n_layers - 1) : ev_ctr(P, EV_IN, P.n_layers);
+    case OP_ROUTE: return kMD ? ev_ctr(P, EV_O, t.layer) : -1;
     case OP_EDOWN: return ev_ctr(P, EV_MH, moe_li(t.layer), t.idx / P.nt_d);
     case OP_COMBINE: return ev_ctr(P, EV_MY, moe_li(t.layer));
     default: return -1;  // EGU is pushed only once its tile table exists
@@ -355,11 +371,12 @@ __device__ void prod_setup(const DevPlan& P, const LayerPtrs* layers, const unsi
   }
 }
 
+template <int kKind>
 __device__ __forceinline__ int task_slots(const DevPlan& P, const ProdFam& f, int idx) {
   if (f.op == OP_ATTN) return P.attn_split;  // (at most; the task's chunks)
-  if (P.wide && (f.op == OP_QKV || f.op == OP_OPROJ || f.op == OP_LM)) return P.hidden / 64;
-  if (P.wide && f.op == OP_GATEUP) return 2 * (P.hidden / 64);
-  if (P.wide && f.op == OP_DOWN) return P.kseg / 64;
+  if (Kind<kKind>::wide && (f.op == OP_QKV || f.op == OP_OPROJ || f.op == OP_LM)) return P.hidden / 64;
+  if (Kind<kKind>::wide && f.op == OP_GATEUP) return 2 * (P.hidden / 64);
+  if (Kind<kKind>::wide && f.op == OP_DOWN) return P.kseg / 64;
   if (f.op == OP_NORM || f.op == OP_NORM2 || f.op == OP_NORMF) return 0;
   if (f.op == OP_ROUTE || f.op == OP_COMBINE || f.op == OP_MINDPTR || f.op == OP_MFIN) return 0;
   if (f.op == OP_QKV || f.op == OP_OPROJ) return kGemvSlots;
@@ -387,6 +404,7 @@ __device__ __forceinline__ MoeTile moe_tile(const DevPlan& P, const unsigned cha
 // rows of the B operand a tile loads (its TMA box and the MMA's N): 16, 64 or 128
 __device__ __forceinline__ int moe_tile_n(int nrows) { return nrows <= 16 ? 16 : nrows <= kMoeTileRows ? kMoeTileRows : kMoeBigTileRows; }
 
+template <int kKind>
 __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                          unsigned char* ws, Control* ctl) {
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
@@ -444,7 +462,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     TaskDesc d;
     d.fam = fam; d.idx = idx; d.op = op; d.layer = layer;
     const bool empty = (P.debug_flags & MK_DEBUG_EMPTY_TASKS) != 0;  // scheduling only: no copies
-    d.nslots = (fam >= 0 && !empty) ? task_slots(P, f, idx) : 0;
+    d.nslots = (fam >= 0 && !empty) ? task_slots<kKind>(P, f, idx) : 0;
     d.slot_ph = slot | (int)(phase << 16);
     d.rec = 0;
     int k = fifo_seq % kFifo;
@@ -455,7 +473,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     fifo_seq++;
     if (fam < 0) return true;
     if (empty) { emitted++; return true; }
-    if (P.wide && (op == OP_QKV || op == OP_OPROJ || op == OP_GATEUP || op == OP_DOWN || op == OP_LM)) {
+    if (Kind<kKind>::wide && (op == OP_QKV || op == OP_OPROJ || op == OP_GATEUP || op == OP_DOWN || op == OP_LM)) {
       // wide batch: the task's 128 weight rows in 64-column chunks, one slot
       // per chunk and part (gate/up: the gate rows, then the up rows); the
       // activation (the B operand) is loaded by the MMA-issuing thread once
@@ -521,7 +539,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
             return false;
         break;
       case OP_EGU:
-      case OP_EDOWN: {
+      case OP_EDOWN: if constexpr (Kind<kKind>::moe) {
         // GroupGEMM tile (tcgen05): per 64-column chunk of K, the task's 128
         // weight rows (gate/up: the gate rows, then the up rows, one slot
         // each) and the tile's routed rows as the B operand, each a 2-D TMA
@@ -668,6 +686,7 @@ struct NotifyInfo {
   int ctr, ffam, fop, flayer, fidx, need_old;
 };
 
+template <int kKind>
 __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const Smem& sm, const TaskDesc& t) {
   const int Hkv = P.n_kv_heads;
   const bool dyn = P.sched == MK_SCHED_DYNAMIC;
@@ -677,7 +696,7 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
     case OP_NORM: n.ctr = ev_ctr(P, EV_N1, t.layer); break;
     case OP_NORM2: n.ctr = ev_ctr(P, EV_N2, t.layer); break;
     case OP_NORMF: n.ctr = ev_ctr(P, EV_NF, 0); break;
-    case OP_QKV: n.ctr = ev_ctr(P, EV_QKV, t.layer, P.wide ? 0 : decode_qkv(P, t.idx).group); break;
+    case OP_QKV: n.ctr = ev_ctr(P, EV_QKV, t.layer, Kind<kKind>::wide ? 0 : decode_qkv(P, t.idx).group); break;
     case OP_ATTN: {
       AttnTask a = decode_attn(t.idx, S.B, Hkv, sm.nch, sm.pre);
       n.ctr = ev_ctr(P, EV_CHUNK, t.layer, a.b, a.g);
@@ -700,7 +719,7 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
     case OP_EDOWN: n.ctr = ev_ctr(P, EV_MY, moe_li(t.layer)); break;
     case OP_COMBINE:
       n.ctr = ev_ctr(P, EV_MCOMB, moe_li(t.layer));
-      if (P.kind == MK_MODEL_MOE_LAYER) { n.ffam = fam_of(P, OP_MFIN, -1); n.fop = OP_MFIN; n.fidx = 0; }
+      if (Kind<kKind>::moe_layer) { n.ffam = fam_of(P, OP_MFIN, -1); n.fop = OP_MFIN; n.fidx = 0; }
       break;
     default: break;
   }
@@ -710,6 +729,7 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
 
 // Dynamic mode: the notifier whose decrement took a counter to zero pushes
 // the tasks that wait on it.
+template <int kKind>
 __device__ void push_successors(const DevPlan& P, const StepParams& S, const Smem& sm, Control* ctl,
                                 unsigned char* ws, const TaskDesc& t) {
   const int Hkv = P.n_kv_heads;
@@ -718,7 +738,7 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
     case OP_NORM2: push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles); break;
     case OP_NORMF: push_range(P, S, ctl, ws, fam_of(P, OP_LM, -1), 0, P.n_lm_tiles); break;
     case OP_QKV: {
-      if (P.wide) {  // (one event per layer: every kv head's tasks of a sequence in one range)
+      if (Kind<kKind>::wide) {  // (one event per layer: every kv head's tasks of a sequence in one range)
         for (int b = 0; b < S.B; ++b)
           push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b], Hkv * sm.nch[b]);
         break;
@@ -729,8 +749,8 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
     } break;
     case OP_MERGE: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
     case OP_OPROJ:
-      if (P.kind == MK_MODEL_MOE_DECODER) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, t.layer), 0, ceil_div(S.B, 8));
-      else if (P.wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM2, t.layer), 0, ceil_div(S.B, 8));
+      if (Kind<kKind>::moe_dec) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, t.layer), 0, ceil_div(S.B, 8));
+      else if (Kind<kKind>::wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM2, t.layer), 0, ceil_div(S.B, 8));
       else push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles);
       break;
     case OP_GATEUP: {
@@ -738,7 +758,7 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
       push_range(P, S, ctl, ws, fam_of(P, OP_DOWN, t.layer), kc * P.n_dtiles, P.n_dtiles);
     } break;
     case OP_DOWN:
-      if (P.wide) {
+      if (Kind<kKind>::wide) {
         if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, ceil_div(S.B, 8));
         else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, ceil_div(S.B, 8));
       } else if (t.layer + 1 < P.n_layers) {
@@ -748,18 +768,18 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
       }
       break;
     // MoE: exp_indptr decides how many GroupGEMM tiles run (data-dependent task triggering)
-    case OP_MINDPTR: {
+    case OP_MINDPTR: if constexpr (Kind<kKind>::moe) {
       const int n_tiles = __ldcg(reinterpret_cast<const int*>(moe_block(P, ws, t.layer) + P.off_mtile) + P.n_experts);
       push_range(P, S, ctl, ws, fam_of(P, OP_EGU, t.layer), 0, n_tiles * P.nt_gu);
     } break;
-    case OP_EGU: {
+    case OP_EGU: if constexpr (Kind<kKind>::moe) {
       const int tile = t.idx / P.nt_gu;
       push_range(P, S, ctl, ws, fam_of(P, OP_EDOWN, t.layer), tile * P.nt_d, P.nt_d);
     } break;
     case OP_EDOWN: push_range(P, S, ctl, ws, fam_of(P, OP_COMBINE, t.layer), 0, ceil_div(S.B, 8)); break;
     case OP_COMBINE:  // MoE decoder: the layer's residual is complete
-      if (P.kind == MK_MODEL_MOE_DECODER) {
-        if (P.wide) {
+      if (Kind<kKind>::moe_dec) {
+        if (Kind<kKind>::wide) {
           if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, ceil_div(S.B, 8));
           else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, ceil_div(S.B, 8));
         } else if (t.layer + 1 < P.n_layers) {
@@ -779,6 +799,7 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
 // add).  The release covers every output of the batch's tasks: the compute
 // warps' writes precede the done barrier, the controller's queue hand-off
 // and this warp's reads in CTA order, and release is cumulative.
+template <int kKind>
 __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, Control* ctl,
                          int* counters) {
   const int lane = threadIdx.x & 31;
@@ -799,7 +820,7 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     ni.ctr = -1; ni.need_old = 0; ni.ffam = -1;
     if (lane < n) {
       t = sm.doneq[(tail + lane) % kDoneQ];
-      ni = notify_info(P, S, sm, t);
+      ni = notify_info<kKind>(P, S, sm, t);
     }
     __syncwarp();
     if (trace) n_batches++;
@@ -823,7 +844,7 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
         asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(counters + key), "r"(-cnt) : "memory");
       }
     }
-    if (fired && P.sched == MK_SCHED_DYNAMIC) push_successors(P, S, sm, ctl, ws, t);
+    if (fired && P.sched == MK_SCHED_DYNAMIC) push_successors<kKind>(P, S, sm, ctl, ws, t);
     if (lane < n && (t.op == OP_LMFIN || t.op == OP_MFIN) && P.sched == MK_SCHED_DYNAMIC)
       push_range(P, S, ctl, ws, -1, 0, P.n_sm);  // one END per CTA
     unsigned fb = __ballot_sync(0xffffffffu, fired && ni.ffam >= 0);
@@ -871,6 +892,7 @@ __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsign
 // goes to cur[k & 1] and completes phase k >> 1 of go_bar[k & 1]; the warps
 // report it done on done_bar[k & 1].  Per-buffer barriers keep every barrier
 // at most one phase ahead of any warp.
+template <int kKind>
 __device__ void controller(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, Control* ctl,
                            int* counters) {
   const int lane = threadIdx.x & 31;
@@ -1022,7 +1044,7 @@ __device__ void controller(const DevPlan& P, const StepParams& S, Smem& sm, unsi
       break;
     }
     if (!is_followup(t.op)) {
-      int w = wait_counter(P, sm, t, S.B);
+      int w = wait_counter<kKind>(P, sm, t, S.B);
       if (w >= 0 && w != known) {
         int st = 0;  // 1 fired, 2 follow-up, 3 dead
         unsigned long long t0 = global_ns();
@@ -1539,7 +1561,7 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
 // (position ctx) is read from the cache in global memory: the ring copy of
 // its chunk may predate this step's append.
 __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
-                                       unsigned char* ws, Control* ctl, const TaskDesc& d) {
+                                       unsigned char* ws, Control* ctl, const TaskDesc& d, uint32_t* trec) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, CH = P.chunk;
   constexpr int D = 64;  // head_dim (the plan builder accepts 64 only)
@@ -1558,14 +1580,10 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
     sm.anew[ct] = __ldcg(reinterpret_cast<const uint4*>(src) + (ct & 7));
   }
   bar_sync(BAR_COMP, kComputeThreads);
+  if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
   const unsigned char* knew = reinterpret_cast<const unsigned char*>(&sm.anew[0]);
   const unsigned char* vnew = reinterpret_cast<const unsigned char*>(&sm.anew[8]);
   const int kq = lane >> 3, ci = lane & 7;  // scores: lane = (key kq of 4, 16-byte column slice ci of 8)
-  float qr[4][8];
-#pragma unroll
-  for (int h = 0; h < 4; ++h)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) qr[h][j] = h < qpg ? sm.aq[h][ci * 8 + j] : 0.f;
   const int hp = lane >> 3, j8 = lane & 7;  // probabilities: lane = (head hp, key j8 of this warp's 8)
   float M[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running maximum per head (same in every warp)
   float L[4] = {0.f, 0.f, 0.f, 0.f};                          // this warp's running exp-sum per head
@@ -1579,8 +1597,19 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
     const bool has_new = (p - cc * CH) < CH;
     const int n_keys = n_old + (has_new ? 1 : 0);
     wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    if (trec && lane == 0 && cc == c0) trec[TR_DATA] = (uint32_t)global_ns();
     const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
     const unsigned char* vbase = kbase + (size_t)CH * D * 2;
+    // the group's queries at this lane's 8 columns (from shared memory per
+    // chunk, so that they hold no registers across the chunk loop)
+    float qr[4][8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&sm.aq[h][ci * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sm.aq[h][ci * 8 + 4]);
+      qr[h][0] = a0.x; qr[h][1] = a0.y; qr[h][2] = a0.z; qr[h][3] = a0.w;
+      qr[h][4] = a1.x; qr[h][5] = a1.y; qr[h][6] = a1.z; qr[h][7] = a1.w;
+    }
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       const int kk = 8 * w + 4 * pass + kq;
@@ -1647,6 +1676,7 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
       if (ct == 0) mbar_arrive(&sm.empty[slot]);
     }
   }
+  if (trec && lane == 0) trec[TR_MATH] = (uint32_t)global_ns();
   // the 8 warps' partial outputs, [w][h][64] in the staging buffer, and sums
   float* ob = sm.xs();
 #pragma unroll
@@ -1657,6 +1687,7 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
     }
   bar_sync(BAR_COMP, kComputeThreads);
   if (ct == 0) mbar_arrive(&sm.empty[last_slot]);  // every warp has read the last chunk's K and V rows
+  if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
   if (ct < qpg * D) {
     const int h = ct >> 6, dd = ct & 63;  // h is uniform in a warp
     float O = 0.f;
@@ -1672,6 +1703,28 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
       part[D] = h == 0 ? M[0] : h == 1 ? M[1] : h == 2 ? M[2] : M[3];
       part[D + 1] = Ls;
     }
+  }
+}
+
+// wide batch: store v at column c of batch row b of an activation buffer with
+// ld columns (its bf16 value, and with the split its bf16 remainder)
+__device__ __forceinline__ void store_act(const DevPlan& P, __nv_bfloat16* buf, size_t ld, int b, size_t c, float v) {
+  const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+  buf[(size_t)act_buf_row(P.act_split, b, 0) * ld + c] = hv;
+  if (P.act_split) buf[(size_t)act_buf_row(P.act_split, b, 1) * ld + c] = __float2bfloat16_rn(v - __bfloat162float(hv));
+}
+
+// wide batch: accumulator columns of batch rows 8 g8 .. 8 g8 + 7 from TMEM
+// address ta (value plus remainder products with the split)
+__device__ __forceinline__ void acc_rows8(uint32_t ta, int split, int g8, float (&v)[8]) {
+  if (split) {
+    float r[8];
+    tmem_ld8(ta + 16u * (uint32_t)g8, v);
+    tmem_ld8(ta + 16u * (uint32_t)g8 + 8u, r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] += r[i];
+  } else {
+    tmem_ld8(ta + 8u * (uint32_t)g8, v);
   }
 }
 
@@ -1718,8 +1771,8 @@ __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S
   float* out = reinterpret_cast<float*>(ws + P.off_attn) + (size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D;
   out[dd] = O / L;
   if (P.wide)  // the O projection's B operand
-    reinterpret_cast<__nv_bfloat16*>(ws + P.off_attn_bf)[(size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D + dd] =
-        __float2bfloat16_rn(O / L);
+    store_act(P, reinterpret_cast<__nv_bfloat16*>(ws + P.off_attn_bf), (size_t)P.n_q_heads * D, b,
+              (size_t)(g * qpg + h) * D + dd, O / L);
 }
 
 // ---------------------------------------------------------------- wide batch
@@ -1777,22 +1830,29 @@ __device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S,
       }
     }
   const float inv = 1.0f / sqrtf(warp_sum(ss) / (float)H + P.eps);
-  __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + P.off_xn) + (size_t)b * H;
+  __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + P.off_xn);
+  __nv_bfloat16* xv = xn + (size_t)act_buf_row(P.act_split, b, 0) * H;
+  __nv_bfloat16* xr = xn + (size_t)act_buf_row(P.act_split, b, 1) * H;
 #pragma unroll
   for (int i = 0; i < kMaxBlk; ++i)
     if (i < nblk) {
       const int c = 256 * i + 8 * lane;
       float gf[8];
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(gp) + c / 8), gf);
-      __align__(16) __nv_bfloat16 o[8];
+      __align__(16) __nv_bfloat16 o[8], rm[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(v[i][j] * inv * gf[j]);
-      *reinterpret_cast<uint4*>(xn + c) = *reinterpret_cast<const uint4*>(o);
+      for (int j = 0; j < 8; ++j) {
+        const float y = v[i][j] * inv * gf[j];
+        o[j] = __float2bfloat16_rn(y);
+        rm[j] = __float2bfloat16_rn(y - __bfloat162float(o[j]));
+      }
+      *reinterpret_cast<uint4*>(xv + c) = *reinterpret_cast<const uint4*>(o);
+      if (P.act_split) *reinterpret_cast<uint4*>(xr + c) = *reinterpret_cast<const uint4*>(rm);
     }
 }
 
 // MMA issue of a wide-batch GEMM task (one thread): per chunk c the task's
-// weight slots (parts of them) from the ring and activation chunk c (act_rows
+// weight slots (parts of them) from the ring and activation chunk c (all buffer
 // rows x 64 columns, columns x0 + 64c of the activation buffer) from stage
 // (bq + c) % kBStages of the staging buffer; the chunk for c + kBStages - 1
 // is loaded once the MMAs of chunk c - 1 released its stage.
@@ -1802,7 +1862,7 @@ __device__ __forceinline__ void gemm_issue_wide(const DevPlan& P, Smem& sm, unsi
   const int R = P.ring_slots;
   const uint32_t idesc = umma_idesc_bf16(kWideRows, N);
   const uint32_t tm = sm.tmem_base;
-  const uint32_t bbytes = (uint32_t)P.act_rows * 128u;
+  const uint32_t bbytes = (uint32_t)act_buf_rows(P.act_split, P.act_rows) * 128u;
   unsigned char* stages = sm.stage();
   const uint32_t u0 = bq;
   auto load_b = [&](int c) {
@@ -1851,7 +1911,8 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
                                                uint32_t& bq) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int B = S.B, H = P.hidden, D = P.head_dim;
-  const int N = ceil_div(B, 16) * 16;
+  const int N = P.act_split ? 16 * ceil_div(B, 8) : ceil_div(B, 16) * 16;  // MMA N (see act_buf_row)
+  const int sp = P.act_split;
   const unsigned char* gmaps = ws + P.off_tmap + (size_t)P.n_layers * kTmapPerLayer * kTmapBytes;
   const void* xn_map = gmaps + (size_t)TMG_XN * kTmapBytes;
   int x0 = 0, nk = H / 64, parts = 1;
@@ -1873,7 +1934,8 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
   const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant = weight rows 32q .. 32q + 31
   const int r = 32 * q + lane;           // this lane's row of the tile
   const uint32_t ta = S_tmem_lane(sm.tmem_base, q);
-  const int cb0 = (w >> 2) * (N / 2), cb1 = cb0 + N / 2;  // this warp's batch columns
+  const int ng = ceil_div(ceil_div(B, 8), 2);  // groups of 8 batch rows per warpgroup
+  const int gb0 = (w >> 2) * ng, gb1 = min(gb0 + ng, ceil_div(B, 8));  // this warp's groups
   switch (d.op) {
     case OP_QKV: {
       // a tile is two heads (q, k or v rows); rotate-half pairs (j, j + 32)
@@ -1884,9 +1946,10 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
       const int h0 = 2 * (d.idx - (kind == 0 ? 0 : kind == 1 ? nq : nq + nkv));
       float* xch = sm.xs();  // [64][act_rows]
       if (q & 1)
-        for (int c8 = cb0; c8 < cb1; c8 += 8) {
+        for (int g8 = gb0; g8 < gb1; ++g8) {
+          const int c8 = 8 * g8;
           float v[8];
-          tmem_ld8(ta + (uint32_t)c8, v);
+          acc_rows8(ta, sp, g8, v);
 #pragma unroll
           for (int i = 0; i < 8; ++i) xch[((q >> 1) * 32 + lane) * P.act_rows + c8 + i] = v[i];
         }
@@ -1894,9 +1957,10 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
       bar_sync(BAR_COMP, kComputeThreads);
       if (!(q & 1)) {
         const int hh = h0 + (q >> 1), j = lane;
-        for (int c8 = cb0; c8 < cb1; c8 += 8) {
+        for (int g8 = gb0; g8 < gb1; ++g8) {
+          const int c8 = 8 * g8;
           float v[8];
-          tmem_ld8(ta + (uint32_t)c8, v);
+          acc_rows8(ta, sp, g8, v);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int b = c8 + i;
@@ -1929,9 +1993,10 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
     case OP_OPROJ: {
       float* x = reinterpret_cast<float*>(ws + P.off_x);
       const int col = d.idx * kWideRows + r;
-      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+      for (int g8 = gb0; g8 < gb1; ++g8) {
+        const int c8 = 8 * g8;
         float v[8];
-        tmem_ld8(ta + (uint32_t)c8, v);
+        acc_rows8(ta, sp, g8, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           if (c8 + i < B) x[(size_t)(c8 + i) * H + col] += v[i];
@@ -1940,21 +2005,23 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
     case OP_GATEUP: {
       __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_h_bf);
       const int col = d.idx * kWideRows + r;
-      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+      for (int g8 = gb0; g8 < gb1; ++g8) {
+        const int c8 = 8 * g8;
         float g[8], u[8];
-        tmem_ld8(ta + (uint32_t)c8, g);
-        tmem_ld8(ta + 128u + (uint32_t)c8, u);
+        acc_rows8(ta, sp, g8, g);
+        acc_rows8(ta + 128u, sp, g8, u);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          if (c8 + i < B) hb[(size_t)(c8 + i) * P.ffn + col] = __float2bfloat16_rn(g[i] / (1.0f + expf(-g[i])) * u[i]);
+          if (c8 + i < B) store_act(P, hb, P.ffn, c8 + i, col, g[i] / (1.0f + expf(-g[i])) * u[i]);
       }
     } break;
     case OP_DOWN: {
       const int kc = d.idx / P.n_dtiles, col = (d.idx - kc * P.n_dtiles) * kWideRows + r;
       float* dp = reinterpret_cast<float*>(ws + P.off_dpart) + (size_t)kc * P.max_batch * H;
-      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+      for (int g8 = gb0; g8 < gb1; ++g8) {
+        const int c8 = 8 * g8;
         float v[8];
-        tmem_ld8(ta + (uint32_t)c8, v);
+        acc_rows8(ta, sp, g8, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           if (c8 + i < B) dp[(size_t)(c8 + i) * H + col] = v[i];
@@ -1967,9 +2034,10 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
       const int row = d.idx * kWideRows + r;
       const bool in = row < P.vocab;
       unsigned long long* best = reinterpret_cast<unsigned long long*>(ws + P.off_lmbest);
-      for (int c8 = cb0; c8 < cb1; c8 += 8) {
+      for (int g8 = gb0; g8 < gb1; ++g8) {
+        const int c8 = 8 * g8;
         float v[8];
-        tmem_ld8(ta + (uint32_t)c8, v);
+        acc_rows8(ta, sp, g8, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int b = c8 + i;
@@ -2362,9 +2430,6 @@ __device__ __forceinline__ void task_combine(const DevPlan& P, const StepParams&
 
 // Kernel instances: the plan kinds (MK_MODEL_*), and the dense decoder's
 // wide-batch path as an instance of its own.
-constexpr int kKindDenseWide = 3;
-constexpr int kKindMoeDecWide = 4;  // the MoE decoder above 8 rows: wide attention half, MoE FFN
-
 template <int kKind>
 __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring, unsigned char* ws,
                         Control* ctl) {
@@ -2439,7 +2504,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
       if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
       gemv_task(P, S, sm, ring, ws, ctl, d, g, B, ea, trec);
     } else if (d.op == OP_ATTN) {
-      task_attn(P, S, sm, ring, ws, ctl, d);
+      task_attn(P, S, sm, ring, ws, ctl, d, trec);
       a_tag = -1;  // the staging buffer held the warps' partial outputs
     } else if (d.op == OP_MERGE) {
       task_merge(P, S, sm, ws, d);
@@ -2620,11 +2685,11 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
 
   // ---- interpreter roles
   if (warp == 0) {
-    if ((tid & 31) == 0) producer(P, S, sm, ring, ws, ctl);
+    if ((tid & 31) == 0) producer<kKind>(P, S, sm, ring, ws, ctl);
   } else if (warp == 1) {
-    controller(P, S, sm, ws, ctl, counters);
+    controller<kKind>(P, S, sm, ws, ctl, counters);
   } else if (warp == 2) {
-    notifier(P, S, sm, ws, ctl, counters);
+    notifier<kKind>(P, S, sm, ws, ctl, counters);
   } else {
     compute<kKind>(P, S, sm, ring, ws, ctl);
   }
@@ -2768,7 +2833,7 @@ static bool encode_weight_maps(const DevPlan& P, const unsigned char* ws, std::v
   const int H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads, F = P.ffn;
   if (P.wide) {
     // wide batch: every matrix in boxes of 64 columns x 128 rows (a tcgen05
-    // A operand per box), the activations in boxes of 64 columns x act_rows
+    // A operand per box), the activations in boxes of 64 columns x all their rows
     const int g0 = P.n_layers * kTmapPerLayer;
     for (int l = 0; l < P.n_layers; ++l) {
       const LayerPtrs& lp = layers[l];
@@ -2783,11 +2848,11 @@ static bool encode_weight_maps(const DevPlan& P, const unsigned char* ws, std::v
            !put_sw128(tmap_index(l, TM_DOWN), lp.w_down, H, F, kWideRows, "w_down")))
         return false;
     }
+    const int ar = act_buf_rows(P.act_split, P.act_rows);  // (value and remainder rows with the split)
     return put_sw128(g0 + TMG_LM, P.lm_head, P.vocab, H, kWideRows, "lm_head") &&
-           put_sw128(g0 + TMG_XN, ws + P.off_xn, P.act_rows, H, P.act_rows, "normalised activations") &&
-           put_sw128(g0 + TMG_ATTN, ws + P.off_attn_bf, P.act_rows, H, P.act_rows, "attention output") &&
-           (P.kind != MK_MODEL_DENSE ||
-            put_sw128(g0 + TMG_H, ws + P.off_h_bf, P.act_rows, F, P.act_rows, "SwiGLU output"));
+           put_sw128(g0 + TMG_XN, ws + P.off_xn, ar, H, ar, "normalised activations") &&
+           put_sw128(g0 + TMG_ATTN, ws + P.off_attn_bf, ar, H, ar, "attention output") &&
+           (P.kind != MK_MODEL_DENSE || put_sw128(g0 + TMG_H, ws + P.off_h_bf, ar, F, ar, "SwiGLU output"));
   }
   for (int l = 0; l < P.n_layers; ++l) {
     const LayerPtrs& lp = layers[l];

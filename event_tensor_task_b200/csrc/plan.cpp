@@ -658,6 +658,12 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     if (Hq / Hkv < 2 || (Hq / Hkv) % 2) { err = "wide batch: an even number of query heads per kv head"; return MK_ERR_UNSUPPORTED; }
   }
   P.act_rows = ceil_div(P.max_batch, 16) * 16;
+  // wide batch: activations as value + remainder (near-fp32 products) while
+  // both MMA operand rows fit (2 x 64 columns per accumulator)
+  if (o->act_split < 0 || o->act_split > 2) { err = "act_split must be 0, 1 or 2"; return MK_ERR_INVALID_ARG; }
+  P.act_split = wide && o->act_split != 2 && P.act_rows <= kMaxWideBatch;
+  if (wide && o->act_split == 1 && !P.act_split)
+    { err = "act_split: value + remainder rows need max_batch <= 64"; return MK_ERR_UNSUPPORTED; }
   if (!(P.kseg % 256 == 0 && F % P.kseg == 0 && P.kseg >= 1024 && P.kseg <= 2048))
     { err = "kseg must be a multiple of 256 in [1024, 2048] dividing ffn"; return MK_ERR_INVALID_ARG; }
   if (Hq / Hkv > 4) { err = "at most 4 query heads per kv head"; return MK_ERR_UNSUPPORTED; }
@@ -684,7 +690,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   // tiles' rotate-half exchange, 64 rows x act_rows fp32; no GEMV partial tiles)
   if (wide) {
     P.gbatch = 0;
-    P.act_bytes = std::max(std::max(8192, 64 * P.act_rows * 4), kBStages * P.act_rows * 128);
+    P.act_bytes = std::max(std::max(8192, 64 * P.act_rows * 4), kBStages * act_buf_rows(P.act_split, P.act_rows) * 128);
     P.gred_bytes = 0;
     P.smem_bytes = smem_bytes;
     P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - seq_table_bytes(P)) / P.slot_bytes);
@@ -918,7 +924,7 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_lmbest = take(8LL * P.max_batch);
   // wide batch: the bf16 activations the GEMM tasks load by TMA (act_rows rows
   // each, so that a box of act_rows rows stays inside the buffer)
-  const long long ar = P.wide ? P.act_rows : 0;
+  const long long ar = P.wide ? act_buf_rows(P.act_split, P.act_rows) : 0;
   P.off_xn = take(2LL * ar * P.hidden);
   P.off_attn_bf = take(2LL * ar * P.hidden);
   P.off_h_bf = take(2LL * ar * P.ffn);

@@ -234,6 +234,15 @@ constexpr int kMoeBigTileRows = 128;  // routing-aware tiles: experts with more 
 // Rows per GroupGEMM tile of an expert with h routed rows: with routing-aware
 // tiles (moe_big), an expert holding more than kMoeTileRows rows gets tiles of
 // kMoeBigTileRows, so its weights stream once per 128 rows instead of 64.
+// wide batch: buffer row of batch row b's bf16 value (part 0) or of its bf16
+// remainder v - value (part 1).  With the split, rows come in groups of 16:
+// the values of batch rows 8g .. 8g + 7, then their remainders, so that one
+// MMA with N = 16 * ceil(B / 8) columns multiplies both and the epilogue adds
+// column pairs (8g + i, 16g + 8 + i -> batch row 8g + i).
+MK_HD int act_buf_row(int split, int b, int part) { return split ? (b >> 3) * 16 + part * 8 + (b & 7) : b; }
+// rows of an activation buffer (and of its TMA box)
+MK_HD int act_buf_rows(int split, int act_rows) { return split ? 2 * act_rows : act_rows; }
+
 MK_HD int moe_tile_rows(int h, int tm, int big) { return (big && h > tm) ? kMoeBigTileRows : tm; }
 constexpr int kTmemCols = 256;  // TMEM columns a CTA of an MoE plan allocates
 
@@ -286,8 +295,8 @@ struct DevPlan {
   // wide batch: tcgen05 GEMM tasks on materialised bf16 activations
   int32_t wide;       // 1: max_batch > kMaxBatchRows
   int32_t attn_split; // key chunks per attention task
-  int32_t act_rows;   // rows of the activation buffers' TMA boxes (max_batch rounded up to 16)
-  int32_t pad4;
+  int32_t act_rows;   // batch rows of the activation buffers (max_batch rounded up to 16)
+  int32_t act_split;  // 1: each activation row stored as its bf16 value and its bf16 remainder (see act_buf_row)
   int64_t off_xn, off_attn_bf, off_h_bf;  // bf16 [max_batch][H], [max_batch][H], [max_batch][F]
 };
 

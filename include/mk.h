@@ -149,6 +149,14 @@ typedef struct mk_plan_opts {
    * once per 128 rows), the others tiles of 64 (16 when a tile has at most
    * 16 rows, as the MMA's N). */
   int moe_tiles;
+  /* Wide batch (max_batch > 8): how the GEMM tasks' activation operand is
+   * stored (0 = default: split when max_batch <= 64; 1 = split; 2 = plain).
+   * Split: each row as its bf16 value plus a second row with the bf16
+   * remainder (v - value), both multiplied in one MMA and added in the
+   * epilogue, so the products see about 16 significant bits of the
+   * activation; plain: the bf16 value only.  1 with max_batch > 64 is
+   * refused with MK_ERR_UNSUPPORTED. */
+  int act_split;
 } mk_plan_opts;
 
 typedef struct mk_plan mk_plan;
@@ -362,9 +370,10 @@ mk_status mk_plan_family_info(const mk_plan* p, int family, mk_family_info* out)
  * exactly its number of notifies.  MK_ERR_INVALID_ARG for null arguments. */
 mk_status mk_plan_counter_region(const mk_plan* p, long long* byte_offset, int* n_counters);
 
-/* Tile sizes the plan chose, written to out[11] in this order: tile_qkv,
+/* Tile sizes the plan chose, written to out[12] in this order: tile_qkv,
  * tile_o, tile_gu, tile_down, kseg, tile_lm, attn_chunk, n_sm, ring_slots,
- * attn_split (key chunks per attention task), wide (1: the wide-batch path). */
+ * attn_split (key chunks per attention task), wide (1: the wide-batch path),
+ * act_split (1: wide-batch activations as value + remainder rows). */
 mk_status mk_plan_tiles(const mk_plan* p, int* out);
 
 /* Host validation for one binding of the symbols (B, ctx_lens host array):

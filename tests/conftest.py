@@ -32,14 +32,16 @@ def read_golden(name):
 MARGINS = {}
 
 
-def record_margin(err=None, near_tie=False):
+def record_margin(err=None, near_tie=False, route_tie=False):
     test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
-    m = MARGINS.setdefault(test, {"max_rel_err": 0.0, "compared": 0, "near_ties": 0})
+    m = MARGINS.setdefault(test, {"max_rel_err": 0.0, "compared": 0, "near_ties": 0, "route_ties": 0})
     if err is not None:
         m["max_rel_err"] = max(m["max_rel_err"], float(err))
         m["compared"] += 1
     if near_tie:
         m["near_ties"] += 1
+    if route_tie:
+        m["route_ties"] += 1
 
 
 def pytest_terminal_summary(terminalreporter):
@@ -48,4 +50,4 @@ def pytest_terminal_summary(terminalreporter):
     terminalreporter.write_line("parity margins (max |gpu - ref| / max |ref| per test; tolerance 2e-2):")
     for test, m in sorted(MARGINS.items()):
         terminalreporter.write_line(f"  {m['max_rel_err']:.3e}  over {m['compared']:4d} tensors, "
-                                    f"{m['near_ties']} near-tie argmax  {test}")
+                                    f"{m['near_ties']} near-tie argmax, {m['route_ties']} near-tie routings  {test}")

@@ -7,6 +7,11 @@ takes the MoE FFN on the bf16-rounded normalised residual rows (the MoE
 layer's input is a stored bf16 tensor).  Checked per step:
   - logits and the residual after every layer within max |gpu - oracle| <=
     2e-2 * max |oracle|, greedy tokens (up to near ties);
+  - the expert set of every token equal to the oracle's own routing, or a
+    near tie (the experts that differ lie within 2e-2 * max |logit| of the
+    top-k boundary); a row routed across a near tie leaves the comparison
+    from that layer on (its later values follow another, equally valid
+    routing), at most one row in eight;
   - layer-local routing, exact: each layer's top-k ids, expert histogram and
     exp_indptr equal the oracle's MoE layer run on the bf16 router input the
     GPU captured for that layer (floating-point drift across layers cannot
@@ -19,7 +24,10 @@ import torch
 import event_tensor_task_b200 as mk
 import oracle
 import workloads as wl
+from conftest import record_margin
 from gpu_common import rel_err, check_argmax, counters_at_zero, TOL
+
+ROUTE_TIE = 2e-2  # near-tie routing margin, relative to max |router logit| of the row
 
 pytestmark = pytest.mark.gpu
 
@@ -40,10 +48,13 @@ class MoeCase:
         self.orc = oracle.DenseOracle(shape, self.w_cpu)
 
     def oracle_moe(self, l, u):
-        return oracle.moe_layer(u.to(torch.bfloat16), self.m_cpu[l], self.mshape.top_k, self.bias)["out"]
+        r = oracle.moe_layer(u.to(torch.bfloat16), self.m_cpu[l], self.mshape.top_k, self.bias)
+        self.routes[l] = r
+        return r["out"]
 
     def step(self, K, V, tokens, slots, ctx):
         dev = "cuda:0"
+        self.routes = {}
         ref = self.orc.step(K, V, tokens, slots, ctx, moe=self.oracle_moe, capture=True)
         B = len(tokens)
         L, H, E, k = self.shape.n_layers, self.shape.hidden, self.mshape.n_experts, self.mshape.top_k
@@ -62,18 +73,46 @@ class MoeCase:
         assert code == 0, f"device status {code} family {st.family} index {st.index} event {st.event}"
         counters_at_zero(self.dec)
         cap = {n: t.cpu() for n, t in cap.items()}
+        diverged = set()  # rows whose routing took the other side of a near tie
         for l in range(L):  # (layer by layer first: a failure names the layer)
             # layer-local routing on the GPU's own bf16 router input
             r = oracle.moe_layer(cap["moe_in"][l], self.m_cpu[l], k, self.bias)
             assert torch.equal(cap["topk"][l], r["idx"]), f"layer {l}: top-k ids"
             assert torch.equal(cap["hist"][l], r["hist"]), f"layer {l}: expert histogram"
             assert torch.equal(cap["indptr"][l], r["indptr"]), f"layer {l}: exp_indptr"
+            # against the oracle's own routing: the same expert sets, or a near tie
             for b in range(B):
-                assert rel_err(cap["resid"][l, b], ref["residual"][l][b]) <= TOL, f"layer {l} row {b}"
+                if b not in diverged and not same_experts(cap["topk"][l][b], self.routes[l], b, k):
+                    diverged.add(b)
+            assert len(diverged) <= max(1, B // 8), f"layer {l}: {len(diverged)} of {B} rows routed differently"
+            for b in range(B):
+                if b not in diverged:
+                    assert rel_err(cap["resid"][l, b], ref["residual"][l][b]) <= TOL, f"layer {l} row {b}"
         for b in range(B):
-            assert rel_err(logits[b].cpu(), ref["logits"][b]) <= TOL, f"logits row {b}"
-            check_argmax(nxt[b].cpu(), ref["logits"][b])
+            if b not in diverged:
+                assert rel_err(logits[b].cpu(), ref["logits"][b]) <= TOL, f"logits row {b}"
+                check_argmax(nxt[b].cpu(), ref["logits"][b])
         return ref
+
+
+def same_experts(gpu_idx, route, b, k):
+    """Whether row b's GPU expert set equals the oracle's.  A differing set is
+    accepted as a near tie when every expert in the symmetric difference has
+    an oracle router logit within ROUTE_TIE * max |logit| of the boundary
+    between the k-th and (k+1)-th largest (the router input of the two sides
+    differs by the bf16 rounding of the normalised residual, which can move a
+    logit across that boundary); anything else fails."""
+    mine, theirs = set(gpu_idx.tolist()), set(route["idx"][b].tolist())
+    if mine == theirs:
+        return True
+    lg = route["logits"][b].double()
+    s = torch.sort(lg, descending=True).values
+    boundary = 0.5 * float(s[k - 1] + s[k]) if k < lg.numel() else float(s[-1])
+    margin = ROUTE_TIE * float(lg.abs().max())
+    far = [e for e in mine ^ theirs if abs(float(lg[e]) - boundary) > margin]
+    assert not far, f"row {b}: experts {sorted(mine)} vs oracle {sorted(theirs)}, {far} not near the top-{k} boundary"
+    record_margin(route_tie=True)
+    return False
 
 
 def _walk(case, steps):

@@ -5,7 +5,9 @@ materialise the residual and the normalised bf16 activations, every
 projection is a tcgen05 GEMM task (128 weight rows x the batch, fp32
 accumulators in tensor memory), and an attention task streams up to
 attn_split key chunks with an online softmax.  One plan and one kernel serve
-every B from 1 to max_batch (symbolic batch and contexts).  Checked through
+every B from 1 to max_batch (symbolic batch and contexts).  Up to 64 rows
+the activations are stored as bf16 value + bf16 remainder rows, multiplied
+in one MMA and added in the epilogue.  Checked through
 the C ABI on cuda:0: logits and the residual after every layer within max
 |gpu - oracle| <= 2e-2 * max |oracle|, greedy tokens (up to near ties), the
 task set exactly, every event counter at zero.
@@ -32,15 +34,17 @@ def _check(case, tokens, slots, ctx, K, V, hidden=True):
     return ref
 
 
-@pytest.mark.parametrize("sched", [mk.MK_SCHED_STATIC, mk.MK_SCHED_DYNAMIC])
-def test_tiny_wide_batch_symbolic_shapes(sched):
+@pytest.mark.parametrize("sched,split", [(mk.MK_SCHED_STATIC, 0), (mk.MK_SCHED_DYNAMIC, 0),
+                                         (mk.MK_SCHED_STATIC, 2)])
+def test_tiny_wide_batch_symbolic_shapes(sched, split):
     # one plan (max_batch 16): B = 16, 9, 1 and 12 with ragged contexts, the
-    # oracle's cache following the appends
+    # oracle's cache following the appends; activations as value + remainder
+    # rows (default) and as plain bf16 rows
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     fill = [64, 0, 70, 190, 5, 127, 128, 300, 1, 2, 255, 33, 64, 65, 129, 200]
-    case = DenseCase(wl.TINY, max_batch=16, max_ctx=320, n_slots=16, ctx_fill=fill, sched=sched)
-    assert case.dec.tiles()["wide"] == 1
+    case = DenseCase(wl.TINY, max_batch=16, max_ctx=320, n_slots=16, ctx_fill=fill, sched=sched, act_split=split)
+    assert case.dec.tiles()["wide"] == 1 and case.dec.tiles()["act_split"] == (split != 2)
     K, V = case.K_cpu.clone(), case.V_cpu.clone()
     tok = wl.token_ids(16, wl.TINY.vocab).tolist()
     steps = [(tok, list(range(16)), fill),

@@ -201,14 +201,19 @@ def test_shared_memory_split_per_max_batch():
         assert d.tiles()["ring_slots"] == want
         d.close()
     # above 8 rows the wide-batch path: no partial tiles; the staging buffer
-    # holds the MMA issuer's activation chunks (3 x rows x 128 B, rows = B
-    # rounded up to 16) or the QKV exchange (64 x rows fp32)
-    for mb, act in ((9, 8192), (64, 3 * 64 * 128)):
-        d = _host(wl.LLAMA_1B, max_batch=mb, max_ctx=1088, n_sm=148)
+    # holds the MMA issuer's activation chunks (3 stages x rows x 128 B, rows
+    # = max_batch rounded up to 16, twice that with the value + remainder
+    # split) or the QKV exchange (64 x rows fp32)
+    for mb, split, act in ((9, 0, 3 * 32 * 128), (64, 0, 3 * 128 * 128), (64, 2, 3 * 64 * 128)):
+        d = _host(wl.LLAMA_1B, max_batch=mb, max_ctx=1088, n_sm=148, act_split=split)
         t = d.tiles()
         assert t["tile_qkv"] == t["tile_o"] == t["tile_gu"] == t["tile_down"] == t["tile_lm"] == 128
+        assert t["act_split"] == (split != 2)
         assert t["ring_slots"] == (232448 - 9 * 1024 - act) // 16384
         d.close()
+    with pytest.raises(mk.MkError):  # value + remainder rows only up to 64 batch rows
+        _host(wl.LLAMA_1B, max_batch=128, max_ctx=1088, n_sm=148, act_split=1,
+              moe=(wl.MOE_64x8, None, None))
     with pytest.raises(mk.MkError):
         _host(wl.LLAMA_1B, max_batch=65, max_ctx=1088, n_sm=148)
 
