@@ -147,12 +147,7 @@ struct Smem {
   OpGeo geo[OP_COUNT];  // GEMV geometry per op, set in the prologue
   unsigned long long lm_seen[kComputeWarps][kMaxB];  // per compute warp: best argmax key it has published
   uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
-  // attention scratch: the group's queries, the chunk's scores, the new
-  // K and V rows (bf16, as in the cache) and the warps' exp-sums
-  alignas(16) float aq[4][64];
-  float asc[4][64];
-  uint4 anew[16];
-  float alsum[kComputeWarps][4];
+  float alsum[kComputeWarps][4], amax[kComputeWarps][4];  // attention: each warp's exp-sum and maximum per head
   volatile int released;  // regular tasks the controller has handed to compute
   volatile int dq_head, dq_tail, fq_head, fq_tail, notifier_stop;
   int bad;
@@ -577,25 +572,20 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       } break;
       case OP_ATTN: {
         // the task's key chunks (attn_split of them at most), one slot each:
-        // the chunk's cached (already rotated) keys and values, minus the row
-        // this step appends; K rows at the slot start, V rows half a slot in
+        // the chunk's 64 cache rows of K, then of V, as swizzled TMA boxes
+        // (rows past max_ctx read as zeros; the task masks rows past ctx)
         AttnTask a = decode_attn(idx, S.B, P.n_kv_heads, sm.nch, sm.pre);
         const int p = sm.ctx[a.b];
         const int c0 = a.c * P.attn_split, c1 = min(c0 + P.attn_split, ceil_div(p + 1, P.chunk));
+        const int plane = (layer * P.n_slots + sm.slot[a.b]) * P.n_kv_heads + a.g;
+        const unsigned char* gm = ws + P.off_tmap + (size_t)P.n_layers * kTmapPerLayer * kTmapBytes;
         for (int cc = c0; cc < c1; ++cc) {
-          const int n_old = max(0, min(P.chunk, p - cc * P.chunk));
           unsigned char* dst;
           uint64_t* bar;
           if (!next_slot(fam, idx, dst, bar)) return false;
-          const uint32_t bytes = (uint32_t)n_old * P.head_dim * 2;
-          mbar_arrive_expect_tx(bar, 2 * bytes);
-          if (n_old > 0) {
-            const size_t row0 = (((size_t)layer * P.n_slots + sm.slot[a.b]) * P.n_kv_heads + a.g) * P.max_ctx +
-                                (size_t)cc * P.chunk;
-            bulk_g2s(dst, (const unsigned char*)P.k_cache + row0 * P.head_dim * 2, bytes, bar);
-            bulk_g2s(dst + (size_t)P.chunk * P.head_dim * 2, (const unsigned char*)P.v_cache + row0 * P.head_dim * 2,
-                     bytes, bar);
-          }
+          mbar_arrive_expect_tx(bar, 2u * (uint32_t)P.chunk * 128u);
+          tma_load_3d(dst, gm + (size_t)TMG_KC * kTmapBytes, 0, cc * P.chunk, plane, bar);
+          tma_load_3d(dst + (size_t)P.chunk * 128, gm + (size_t)TMG_VC * kTmapBytes, 0, cc * P.chunk, plane, bar);
         }
       } break;
       default: break;
@@ -1548,18 +1538,47 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   bar_sync(BAR_COMP, kComputeThreads);  // the partial tiles are free for the next task
 }
 
+// ldmatrix: four 8x8 b16 matrices from shared memory; lane l gives the
+// address of row l % 8 of matrix l / 8 (16 bytes), register m receives the
+// matrix-m elements of the mma fragment layout (plain or transposed).
+__device__ __forceinline__ void ldsm_x4(const void* p, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(const void* p, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+// (x0, x1) as a bf16 pair (x0 in the low half): the values, and the remainders x - value
+__device__ __forceinline__ uint32_t bf16_pair(float x0, float x1) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(x0, x1);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(x0, x1);
+  hi = *reinterpret_cast<const uint32_t*>(&v);
+  lo = bf16_pair(x0 - __low2float(v), x1 - __high2float(v));
+}
+// 16-byte chunk c of row r of a 64-column bf16 tile under the 128-byte swizzle
+__device__ __forceinline__ int sw128_off(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+
 // One task of split-KV decode attention for the qpg query heads of a GQA
 // group: up to attn_split consecutive 64-key chunks of one sequence, one ring
-// slot each (flash-decoding partial: unnormalised output, running max, sum).
-// All 8 compute warps share a chunk: warp w scores keys [8w, 8w + 8) for
-// every head of the group (each K row is read from shared memory once; a lane
-// holds one 16-byte slice of a row and the matching 8 query values of each
-// head in registers), then accumulates those keys' V rows for every head
-// with an online rescale across the task's chunks (every warp derives the
-// same running maximum from the chunk's scores); the 8 warps' partial
-// outputs are summed through the staging buffer at the end.  The new key
-// (position ctx) is read from the cache in global memory: the ring copy of
-// its chunk may predate this step's append.
+// slot each (K rows, then V rows, as 128-byte-swizzled TMA boxes), one chunk
+// per compute warp (flash-decoding partials: unnormalised output, running
+// maximum, exp-sum).  A warp computes the chunk's scores S = Q K^T and
+// O += P V with bf16 warp MMAs (m16n8k16, fp32 accumulation): MMA row h
+// carries head h's query (or probabilities) as bf16 values and row h + 8 the
+// bf16 remainders, so that the products see about 16 significant bits and
+// the two rows' accumulators add up in the same lane; the softmax in between
+// is fp32 in registers (lane (g, q) holds head g's scores of keys 2q, 2q + 1
+// of each 8-key tile).  The warps' partials are combined through shared
+// memory at the end.  The new key (position ctx) is read from the cache in
+// global memory and written over its row of the slot, whose copy may predate
+// this step's append; the slot's rows past the last key are masked (scores)
+// and zeroed (values).
 __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                        unsigned char* ws, Control* ctl, const TaskDesc& d, uint32_t* trec) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
@@ -1567,143 +1586,149 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
   constexpr int D = 64;  // head_dim (the plan builder accepts 64 only)
   const AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
   const int p = sm.ctx[a.b];
-  const int n_chunks = ceil_div(p + 1, CH);
-  const int c0 = a.c * P.attn_split, c1 = min(c0 + P.attn_split, n_chunks);
-  const bool task_new = c1 == n_chunks;  // the task's last chunk holds the new key
-  // queries of the group (scaled by 1/sqrt(64)) and the new K/V rows
-  const float* q = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D +
-                   (size_t)a.g * qpg * D;
-  if (ct < qpg * D) sm.aq[ct >> 6][ct & 63] = __ldcg(q + ct) * 0.125f;
-  if (task_new && ct < 16) {
-    const size_t row = (((size_t)d.layer * P.n_slots + sm.slot[a.b]) * Hkv + a.g) * P.max_ctx + p;
-    const unsigned char* src = reinterpret_cast<const unsigned char*>(ct < 8 ? P.k_cache : P.v_cache) + row * D * 2;
-    sm.anew[ct] = __ldcg(reinterpret_cast<const uint4*>(src) + (ct & 7));
-  }
-  bar_sync(BAR_COMP, kComputeThreads);
-  if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
-  const unsigned char* knew = reinterpret_cast<const unsigned char*>(&sm.anew[0]);
-  const unsigned char* vnew = reinterpret_cast<const unsigned char*>(&sm.anew[8]);
-  const int kq = lane >> 3, ci = lane & 7;  // scores: lane = (key kq of 4, 16-byte column slice ci of 8)
-  const int hp = lane >> 3, j8 = lane & 7;  // probabilities: lane = (head hp, key j8 of this warp's 8)
-  float M[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running maximum per head (same in every warp)
-  float L[4] = {0.f, 0.f, 0.f, 0.f};                          // this warp's running exp-sum per head
-  float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
-  int last_slot = 0;
-  for (int cc = c0; cc < c1; ++cc) {
-    uint32_t par;
-    const int slot = task_slot(d, cc - c0, P.ring_slots, par);
-    last_slot = slot;
+  const int c0 = a.c * P.attn_split, c1 = min(c0 + P.attn_split, ceil_div(p + 1, CH));
+  const int g = lane >> 2, q4 = lane & 3;
+  const bool hv = g < qpg;  // this lane's MMA row is a head of the group
+  float m_run = -INFINITY, l_run = 0.f;
+  float o[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  const int cc = c0 + w;  // this warp's chunk (attn_split <= 8 chunks per task)
+  if (cc < c1) {
+    // query fragments (scaled by 1/sqrt(64)): dims 16t + 2q, +1 and +8, +9 of head g
+    uint32_t qa[4][4];
+    const float* qrow = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D +
+                        (size_t)(a.g * qpg + (hv ? g : 0)) * D;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float2 x01 = hv ? __ldcg(reinterpret_cast<const float2*>(qrow + 16 * t + 2 * q4)) : make_float2(0.f, 0.f);
+      const float2 x89 = hv ? __ldcg(reinterpret_cast<const float2*>(qrow + 16 * t + 2 * q4 + 8)) : make_float2(0.f, 0.f);
+      split_pair(x01.x * 0.125f, x01.y * 0.125f, qa[t][0], qa[t][1]);
+      split_pair(x89.x * 0.125f, x89.y * 0.125f, qa[t][2], qa[t][3]);
+    }
     const int n_old = max(0, min(CH, p - cc * CH));
     const bool has_new = (p - cc * CH) < CH;
     const int n_keys = n_old + (has_new ? 1 : 0);
+    uint4 knew = make_uint4(0, 0, 0, 0);
+    if (has_new && lane < 16) {
+      const size_t row = (((size_t)d.layer * P.n_slots + sm.slot[a.b]) * Hkv + a.g) * P.max_ctx + p;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(lane < 8 ? P.k_cache : P.v_cache) + row * D * 2;
+      knew = __ldcg(reinterpret_cast<const uint4*>(src) + (lane & 7));
+    }
+    if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
+    uint32_t par;
+    const int slot = task_slot(d, cc - c0, P.ring_slots, par);
     wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
-    if (trec && lane == 0 && cc == c0) trec[TR_DATA] = (uint32_t)global_ns();
-    const unsigned char* kbase = ring + (size_t)slot * P.slot_bytes;
-    const unsigned char* vbase = kbase + (size_t)CH * D * 2;
-    // the group's queries at this lane's 8 columns (from shared memory per
-    // chunk, so that they hold no registers across the chunk loop)
-    float qr[4][8];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&sm.aq[h][ci * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&sm.aq[h][ci * 8 + 4]);
-      qr[h][0] = a0.x; qr[h][1] = a0.y; qr[h][2] = a0.z; qr[h][3] = a0.w;
-      qr[h][4] = a1.x; qr[h][5] = a1.y; qr[h][6] = a1.z; qr[h][7] = a1.w;
+    if (trec && lane == 0) trec[TR_DATA] = (uint32_t)global_ns();
+    unsigned char* kb = ring + (size_t)slot * P.slot_bytes;
+    unsigned char* vb = kb + (size_t)CH * D * 2;
+    if (has_new) {
+      // the appended key and value over their row; value rows past it zeroed
+      if (lane < 16) *reinterpret_cast<uint4*>((lane < 8 ? kb : vb) + sw128_off(n_old, lane & 7)) = knew;
+      for (int i = lane; i < (CH - 1 - n_old) * 8; i += 32)
+        *reinterpret_cast<uint4*>(vb + sw128_off(n_old + 1 + (i >> 3), i & 7)) = make_uint4(0, 0, 0, 0);
+      __syncwarp();
     }
+    // scores: 8 key tiles x 4 dim steps
+    float sc[8][4];
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const int kk = 8 * w + 4 * pass + kq;
-      const unsigned char* row = (has_new && kk == n_old) ? knew : kbase + (size_t)kk * D * 2;
-      float kf[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + ci * 16), kf);
-      float sc[4];
+    for (int j = 0; j < 8; ++j) {
+      sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+      const int r = 8 * j + (lane & 7);
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        float acc = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc = fmaf(kf[j], qr[h][j], acc);
-        sc[h] = acc;
-      }
-#pragma unroll
-      for (int o = 1; o < 8; o <<= 1)
-#pragma unroll
-        for (int h = 0; h < 4; ++h) sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], o);
-      const float mine = ci == 0 ? sc[0] : ci == 1 ? sc[1] : ci == 2 ? sc[2] : sc[3];
-      if (ci < qpg) sm.asc[ci][kk] = kk < n_keys ? mine : -INFINITY;
-    }
-    bar_sync(BAR_COMP, kComputeThreads);
-    // the chunk's maximum per head joins the running maximum; earlier sums rescale
-    float scale[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      float m = -INFINITY;
-      if (h < qpg) m = fmaxf(sm.asc[h][lane], sm.asc[h][lane + 32]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const float mn = fmaxf(M[h], m);
-      scale[h] = h < qpg ? expf(M[h] - mn) : 0.f;  // 0 on the first chunk (M = -inf, mn finite)
-      M[h] = mn;
-    }
-    const float Mh = hp == 0 ? M[0] : hp == 1 ? M[1] : hp == 2 ? M[2] : M[3];
-    const float pl = (hp < qpg && 8 * w + j8 < n_keys) ? expf(sm.asc[hp][8 * w + j8] - Mh) : 0.f;
-    float ls = pl;
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      L[h] = L[h] * scale[h] + __shfl_sync(0xffffffffu, ls, 8 * h);
-      o0[h] *= scale[h];
-      o1[h] *= scale[h];
-    }
-    // P.V over this warp's keys: lane = output columns 2*lane, 2*lane + 1
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      const int kk = 8 * w + jj;
-      if (kk < n_keys) {
-        const unsigned char* row = (has_new && kk == n_old) ? vnew : vbase + (size_t)kk * D * 2;
-        const uint32_t v2 = *reinterpret_cast<const uint32_t*>(row + lane * 4);
-        const float va = __uint_as_float(v2 << 16), vb = __uint_as_float(v2 & 0xffff0000u);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float ph = __shfl_sync(0xffffffffu, pl, h * 8 + jj);
-          o0[h] = fmaf(ph, va, o0[h]);
-          o1[h] = fmaf(ph, vb, o1[h]);
-        }
+      for (int tt = 0; tt < 2; ++tt) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + sw128_off(r, 4 * tt + (lane >> 3)), b0, b1, b2, b3);
+        mma_16816(sc[j], qa[2 * tt][0], qa[2 * tt][1], qa[2 * tt][2], qa[2 * tt][3], b0, b1);
+        mma_16816(sc[j], qa[2 * tt + 1][0], qa[2 * tt + 1][1], qa[2 * tt + 1][2], qa[2 * tt + 1][3], b2, b3);
       }
     }
-    if (cc + 1 < c1) {  // (the last chunk's slot is released after the final barrier below)
-      bar_sync(BAR_COMP, kComputeThreads);  // every warp is done with the scores and the slot's K and V rows
-      if (ct == 0) mbar_arrive(&sm.empty[slot]);
+    // softmax of head g over the chunk, joined to the running state
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float v = (8 * j + 2 * q4 + e < n_keys) ? sc[j][e] + sc[j][2 + e] : -INFINITY;
+        sc[j][e] = v;
+        mx = fmaxf(mx, v);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);  // finite: the chunk has a key
+    const float scale = hv ? expf(m_run - m_new) : 0.f;
+    float ls = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float pv = hv ? expf(sc[j][e] - m_new) : 0.f;
+        sc[j][e] = pv;
+        ls += pv;
+      }
+    ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+    ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+    l_run = l_run * scale + ls;
+    m_run = m_new;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { o[j][0] *= scale; o[j][1] *= scale; o[j][2] *= scale; o[j][3] *= scale; }
+    // O += P V: 4 key steps (key tiles 2t, 2t + 1) x 8 dim tiles
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      uint32_t pa0, pa1, pa2, pa3;
+      split_pair(sc[2 * t][0], sc[2 * t][1], pa0, pa1);
+      split_pair(sc[2 * t + 1][0], sc[2 * t + 1][1], pa2, pa3);
+      const int r = 16 * t + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + sw128_off(r, 2 * jj + (lane >> 4)), b0, b1, b2, b3);
+        mma_16816(o[2 * jj], pa0, pa1, pa2, pa3, b0, b1);
+        mma_16816(o[2 * jj + 1], pa0, pa1, pa2, pa3, b2, b3);
+      }
     }
+    // (generic writes to the slot precede the producer's next TMA copy into it)
+    if (has_new) fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty[slot]);
   }
   if (trec && lane == 0) trec[TR_MATH] = (uint32_t)global_ns();
-  // the 8 warps' partial outputs, [w][h][64] in the staging buffer, and sums
+  // the warps' partials (value and remainder rows added), maxima and sums
   float* ob = sm.xs();
+  if (hv) {
 #pragma unroll
-  for (int h = 0; h < 4; ++h)
-    if (h < qpg) {
-      *reinterpret_cast<float2*>(ob + (w * 4 + h) * D + 2 * lane) = make_float2(o0[h], o1[h]);
-      if (lane == 0) sm.alsum[w][h] = L[h];
-    }
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float2*>(ob + (w * 4 + g) * D + 8 * j + 2 * q4) = make_float2(o[j][0] + o[j][2], o[j][1] + o[j][3]);
+    if (q4 == 0) { sm.alsum[w][g] = l_run; sm.amax[w][g] = m_run; }
+  }
   bar_sync(BAR_COMP, kComputeThreads);
-  if (ct == 0) mbar_arrive(&sm.empty[last_slot]);  // every warp has read the last chunk's K and V rows
-  if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
   if (ct < qpg * D) {
     const int h = ct >> 6, dd = ct & 63;  // h is uniform in a warp
-    float O = 0.f;
+    float M = -INFINITY;
 #pragma unroll
-    for (int ww = 0; ww < kComputeWarps; ++ww) O += ob[(ww * 4 + h) * D + dd];
+    for (int ww = 0; ww < kComputeWarps; ++ww) M = fmaxf(M, sm.amax[ww][h]);
+    float O = 0.f, Ls = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < kComputeWarps; ++ww) {
+      const float mw = sm.amax[ww][h];
+      if (mw != -INFINITY) {  // (warps without a chunk)
+        const float f = expf(mw - M);
+        O = fmaf(ob[(ww * 4 + h) * D + dd], f, O);
+        Ls = fmaf(sm.alsum[ww][h], f, Ls);
+      }
+    }
     float* part = reinterpret_cast<float*>(ws + P.off_apart) +
                   (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2)) + h * (D + 2);
     part[dd] = O;
     if (dd == 0) {
-      float Ls = 0.f;
-#pragma unroll
-      for (int ww = 0; ww < kComputeWarps; ++ww) Ls += sm.alsum[ww][h];
-      part[D] = h == 0 ? M[0] : h == 1 ? M[1] : h == 2 ? M[2] : M[3];
+      part[D] = M;
       part[D + 1] = Ls;
     }
   }
+  // every warp has read the partials before any of them writes the staging
+  // buffer again (the next task may start without a barrier of its own)
+  bar_sync(BAR_COMP, kComputeThreads);
+  if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
 }
 
 // wide batch: store v at column c of batch row b of an activation buffer with
@@ -2831,6 +2856,27 @@ static bool encode_weight_maps(const DevPlan& P, const unsigned char* ws, std::v
       { err = "norm gains must be 16-byte aligned"; return false; }
   if (reinterpret_cast<uintptr_t>(P.final_norm) & 15) { err = "final_norm must be 16-byte aligned"; return false; }
   const int H = P.hidden, D = P.head_dim, Hq = P.n_q_heads, Hkv = P.n_kv_heads, F = P.ffn;
+  {
+    // the K and V caches as [layer, slot, kv head][max_ctx][64]: one box per
+    // 64-key chunk of a (layer, slot, head), under the 128-byte swizzle (the
+    // attention tasks' ldmatrix reads are then conflict-free)
+    const void* caches[2] = {P.k_cache, P.v_cache};
+    for (int kv = 0; kv < 2; ++kv) {
+      if (reinterpret_cast<uintptr_t>(caches[kv]) & 15) { err = "the KV caches must be 16-byte aligned"; return false; }
+      CUtensorMap m;
+      const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)P.max_ctx,
+                                  (cuuint64_t)P.n_layers * P.n_slots * Hkv};
+      const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)P.max_ctx * D * 2};
+      const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)P.chunk, 1};
+      const cuuint32_t estr[3] = {1, 1, 1};
+      CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(caches[kv]), dims, strides, box,
+                       estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) { err = "tensor map of the KV cache rejected by the driver"; return false; }
+      const int index = P.n_layers * kTmapPerLayer + (kv ? TMG_VC : TMG_KC);
+      std::memcpy(image.data() + (P.off_tmap - P.off_families) + (size_t)index * kTmapBytes, &m, sizeof(m));
+    }
+  }
   if (P.wide) {
     // wide batch: every matrix in boxes of 64 columns x 128 rows (a tcgen05
     // A operand per box), the activations in boxes of 64 columns x all their rows

@@ -646,7 +646,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.slot_bytes = 16384;
   P.wide = wide ? 1 : 0;
   P.attn_split = o->attn_split ? o->attn_split : (wide ? 8 : 1);
-  if (P.attn_split < 1 || P.attn_split > 16) { err = "attn_split must be in [1, 16]"; return MK_ERR_INVALID_ARG; }
+  if (P.attn_split < 1 || P.attn_split > 8) { err = "attn_split must be in [1, 8]"; return MK_ERR_INVALID_ARG; }
   if (wide) {
     // tcgen05 GEMM tasks: kWideRows weight rows each (the MMA's M), every
     // weight matrix read in 64-column chunks, the batch as the MMA's N

@@ -207,7 +207,10 @@ constexpr int kMaxWideBatch = 64;    // batch rows of a wide step (tcgen05 GEMM 
 // normalised activations, the attention output and the SwiGLU output (bf16)
 constexpr int kWideRows = 128;
 constexpr int kBStages = 3;  // wide batch: activation-chunk stages of the MMA issuer (in the staging buffer)
-enum TmapGlobal : int { TMG_LM = 0, TMG_XN, TMG_ATTN, TMG_H, kTmapGlobal };
+// global tensor maps: the LM head, the wide-batch activation buffers, and the
+// K and V caches as [layer, slot, kv head][max_ctx][64] (one 64-key chunk per
+// box, 128-byte swizzle)
+enum TmapGlobal : int { TMG_LM = 0, TMG_XN, TMG_ATTN, TMG_H, TMG_KC, TMG_VC, kTmapGlobal };
 // A GEMV task's weights arrive in kGemvSlots ring slots, slot j holding columns
 // [j K / 8, (j + 1) K / 8) of all the task's rows (one 2-D TMA box per part),
 // through one tensor map per dense weight matrix: matrix m of layer l at

@@ -140,8 +140,9 @@ typedef struct mk_plan_opts {
   int fault;
   int fault_family;
   /* Key chunks (attn_chunk keys each) per attention task: 0 = default (1 for
-   * max_batch <= 8, 8 above), at most 16.  A task streams its chunks through
-   * the ring with an online softmax and leaves one partial for the merge. */
+   * max_batch <= 8, 8 above), at most 8.  Each compute warp of the task takes
+   * one chunk (tensor-core scores and P.V with an online softmax); the task
+   * leaves one partial for the merge. */
   int attn_split;
   /* MoE GroupGEMM tiles, chosen per expert from the run-time histogram
    * (0 = default: routing-aware; 1 = routing-aware; 2 = fixed): an expert
