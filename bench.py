@@ -397,6 +397,32 @@ def profile_moe(T):
         raise SystemExit(f"MoE layer device status {code}")
 
 
+def profile_wide(B):
+    """Four decode steps of the 1B-shaped model at batch B through one
+    max_batch 64 plan (the wide-batch path), contexts uniform in [128, 1024]
+    (a profiling case: 2.5 GB of weights plus at most 2.2 GB of cache)."""
+    import torch
+    import event_tensor_task_b200 as mk
+    import workloads as wl
+    dev = "cuda:0"
+    s = wl.LLAMA_1B
+    w = {k: v.to(dev) for k, v in wl.dense_weights(s, seed=0).items()}
+    ctx0 = [int(c) for c in wl.context_lengths(B, 128, 1024)]
+    max_ctx = max(ctx0) + 32
+    K, V = device_kv_cache(s, B, max_ctx, ctx0, dev)
+    dec = mk.DenseDecoder(s, w, K, V, max_batch=64, max_ctx=max_ctx, n_slots=B)
+    tok = torch.full((B,), 5, dtype=torch.int32, device=dev)
+    slots = torch.arange(B, dtype=torch.int32, device=dev)
+    ctx = torch.tensor(ctx0[:B], dtype=torch.int32, device=dev)
+    nxt = torch.empty(B, dtype=torch.int32, device=dev)
+    for _ in range(4):
+        dec.step(tok, slots, ctx, nxt)
+    torch.cuda.synchronize()
+    code, _ = dec.status()
+    if code != 0:
+        raise SystemExit(f"wide-batch step device status {code}")
+
+
 def moe_decoder_bench(dev, n_steps=64):
     """The MoE decoder: 16 layers with the 1B attention shape, each FFN the
     64-expert top-8 layer (F 1408), vocab 128256, tied embeddings; Zipf(1.2)
@@ -704,6 +730,8 @@ def main():
     ap.add_argument("--no-interp", action="store_true")
     ap.add_argument("--profile-moe", type=int, default=0, metavar="T",
                     help="only run 4 MoE-layer calls on T tokens (a short command for ncu) and exit")
+    ap.add_argument("--profile-wide", type=int, default=0, metavar="B",
+                    help="only run 4 wide-batch 1B decode steps at batch B (a short command for ncu) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -715,6 +743,9 @@ def main():
         return
     if args.profile_moe:
         profile_moe(args.profile_moe)
+        return
+    if args.profile_wide:
+        profile_wide(args.profile_wide)
         return
 
     import torch

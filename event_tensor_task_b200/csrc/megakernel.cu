@@ -59,18 +59,24 @@ constexpr int kDoneQ = 32;    // controller -> notifier
 constexpr int kFollowQ = 16;  // notifier -> controller
 constexpr int kMaxB = kMaxBatchRows;  // batch rows per step on this path
 constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
+constexpr int kMaxKc = 8;     // down-projection K segments (ffn / kseg <= 8192 / 1024)
 constexpr int kDynLookahead = 2;
 
 // Kernel instances: the plan kinds (MK_MODEL_*) and the wide-batch layouts
 // (max_batch > 8) of the dense and the MoE decoder, each with only the code
-// paths its plans take (the interpreter roles included).
+// paths its plans take (the interpreter roles included), each without and
+// with the per-task trace (kTraced: the recording code costs instruction
+// fetches even when it records nothing).
 constexpr int kKindDenseWide = 3;
 constexpr int kKindMoeDecWide = 4;  // the MoE decoder above 8 rows: wide attention half, MoE FFN
+constexpr int kTraced = 8;          // instance flag: MK_DEBUG_TRACE plans
 template <int K>
 struct Kind {
-  static constexpr bool wide = K == kKindDenseWide || K == kKindMoeDecWide;
-  static constexpr bool moe_layer = K == MK_MODEL_MOE_LAYER;
-  static constexpr bool moe_dec = K == MK_MODEL_MOE_DECODER || K == kKindMoeDecWide;
+  static constexpr int base = K & 7;
+  static constexpr bool trace = (K & kTraced) != 0;
+  static constexpr bool wide = base == kKindDenseWide || base == kKindMoeDecWide;
+  static constexpr bool moe_layer = base == MK_MODEL_MOE_LAYER;
+  static constexpr bool moe_dec = base == MK_MODEL_MOE_DECODER || base == kKindMoeDecWide;
   static constexpr bool moe = moe_layer || moe_dec;
 };
 
@@ -148,6 +154,9 @@ struct Smem {
   unsigned long long lm_seen[kComputeWarps][kMaxB];  // per compute warp: best argmax key it has published
   uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
   float alsum[kComputeWarps][4], amax[kComputeWarps][4];  // attention: each warp's exp-sum and maximum per head
+  int gemm_last;  // wide batch, split K: this CTA's task was the tile's last segment
+  // wide batch: this CTA's best argmax key per batch column, and what it published
+  unsigned long long lm_cta[kMaxBatch], lm_pub[kMaxBatch];
   volatile int released;  // regular tasks the controller has handed to compute
   volatile int dq_head, dq_tail, fq_head, fq_tail, notifier_stop;
   int bad;
@@ -417,7 +426,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
   // acquire the next ring slot: wait until the compute warps released it
   auto next_slot = [&](int fam, int idx, unsigned char*& dst, uint64_t*& bar) -> bool {
     if (!wait_mbar(&sm.empty[slot], phase ^ 1, ctl, tmo, fam, idx)) return false;
-    if (S.trace) sm.slot_t[slot] = (uint32_t)global_ns();
+    if (Kind<kKind>::trace && S.trace) sm.slot_t[slot] = (uint32_t)global_ns();
     dst = ring + (size_t)slot * P.slot_bytes;
     bar = &sm.full[slot];
     ring_seq++;
@@ -462,7 +471,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     d.rec = 0;
     int k = fifo_seq % kFifo;
     if (!wait_mbar(&sm.fifo_empty[k], ((fifo_seq / kFifo) & 1) ^ 1, ctl, tmo, fam, idx)) return false;
-    d.t_issue = S.trace ? (uint32_t)global_ns() : 0u;
+    d.t_issue = (Kind<kKind>::trace && S.trace) ? (uint32_t)global_ns() : 0u;
     sm.fifo[k] = d;
     mbar_arrive(&sm.fifo_full[k]);
     fifo_seq++;
@@ -473,13 +482,17 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       // per chunk and part (gate/up: the gate rows, then the up rows); the
       // activation (the B operand) is loaded by the MMA-issuing thread once
       // the task's event has fired (see gemm_issue_wide)
-      int row = idx * kWideRows, x0 = 0, nk = P.hidden / 64;
+      // (QKV, O and gate/up: K segment seg of tile idx / gseg)
+      const int gseg = op == OP_QKV ? P.gseg_qkv : op == OP_OPROJ ? P.gseg_o : op == OP_GATEUP ? P.gseg_gu : 1;
+      const int tile = idx / gseg, seg = idx - tile * gseg;
+      const int K = op == OP_OPROJ ? P.n_q_heads * P.head_dim : P.hidden;
+      int row = tile * kWideRows, x0 = seg * (K / gseg), nk = K / gseg / 64;
       const void* m0 = f.tm[0];
       if (op == OP_QKV) {
         const int nq = P.n_q_heads * P.head_dim / kWideRows, nkv = P.n_kv_heads * P.head_dim / kWideRows;
-        const int kind = idx < nq ? 0 : idx < nq + nkv ? 1 : 2;
+        const int kind = tile < nq ? 0 : tile < nq + nkv ? 1 : 2;
         m0 = f.tm[kind];
-        row = (idx - (kind == 0 ? 0 : kind == 1 ? nq : nq + nkv)) * kWideRows;
+        row = (tile - (kind == 0 ? 0 : kind == 1 ? nq : nq + nkv)) * kWideRows;
       } else if (op == OP_DOWN) {
         const int kc = idx / P.n_dtiles;
         row = (idx - kc * P.n_dtiles) * kWideRows;
@@ -689,12 +702,17 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
     case OP_QKV: n.ctr = ev_ctr(P, EV_QKV, t.layer, Kind<kKind>::wide ? 0 : decode_qkv(P, t.idx).group); break;
     case OP_ATTN: {
       AttnTask a = decode_attn(t.idx, S.B, Hkv, sm.nch, sm.pre);
-      n.ctr = ev_ctr(P, EV_CHUNK, t.layer, a.b, a.g);
-      n.ffam = fam_of(P, OP_MERGE, t.layer); n.fop = OP_MERGE; n.flayer = t.layer; n.fidx = a.b * Hkv + a.g;
+      if (sm.nch[a.b] == 1) {
+        // the pair's only task wrote the finished output: it counts for the merge
+        n.ctr = ev_ctr(P, EV_ATTN, t.layer);
+      } else {
+        n.ctr = ev_ctr(P, EV_CHUNK, t.layer, a.b, a.g);
+        n.ffam = fam_of(P, OP_MERGE, t.layer); n.fop = OP_MERGE; n.flayer = t.layer; n.fidx = a.b * Hkv + a.g;
+      }
     } break;
     case OP_MERGE: n.ctr = ev_ctr(P, EV_ATTN, t.layer); break;
     case OP_OPROJ: n.ctr = ev_ctr(P, EV_O, t.layer); break;
-    case OP_GATEUP: n.ctr = ev_ctr(P, EV_GU, t.layer, t.idx * P.tile_gu / P.kseg); break;
+    case OP_GATEUP: n.ctr = ev_ctr(P, EV_GU, t.layer, t.idx / P.gseg_gu * P.tile_gu / P.kseg); break;
     case OP_DOWN: n.ctr = ev_ctr(P, EV_IN, t.layer + 1); break;
     case OP_LM:
       n.ctr = ev_ctr(P, EV_LM, 0);
@@ -738,19 +756,23 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
         push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b] + g * sm.nch[b], sm.nch[b]);
     } break;
     case OP_MERGE: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
+    case OP_ATTN: {  // (a pair's only task counts for its merge: it fired EV_ATTN)
+      const AttnTask a = decode_attn(t.idx, S.B, Hkv, sm.nch, sm.pre);
+      if (sm.nch[a.b] == 1) push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles);
+    } break;
     case OP_OPROJ:
       if (Kind<kKind>::moe_dec) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, t.layer), 0, ceil_div(S.B, 8));
-      else if (Kind<kKind>::wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM2, t.layer), 0, ceil_div(S.B, 8));
+      else if (Kind<kKind>::wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM2, t.layer), 0, S.B);
       else push_range(P, S, ctl, ws, fam_of(P, OP_GATEUP, t.layer), 0, P.n_gutiles);
       break;
     case OP_GATEUP: {
-      int kc = t.idx * P.tile_gu / P.kseg;
+      int kc = t.idx / P.gseg_gu * P.tile_gu / P.kseg;
       push_range(P, S, ctl, ws, fam_of(P, OP_DOWN, t.layer), kc * P.n_dtiles, P.n_dtiles);
     } break;
     case OP_DOWN:
       if (Kind<kKind>::wide) {
-        if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, ceil_div(S.B, 8));
-        else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, ceil_div(S.B, 8));
+        if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, S.B);
+        else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, S.B);
       } else if (t.layer + 1 < P.n_layers) {
         push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
       } else {
@@ -770,8 +792,8 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
     case OP_COMBINE:  // MoE decoder: the layer's residual is complete
       if (Kind<kKind>::moe_dec) {
         if (Kind<kKind>::wide) {
-          if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, ceil_div(S.B, 8));
-          else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, ceil_div(S.B, 8));
+          if (t.layer + 1 < P.n_layers) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, t.layer + 1), 0, S.B);
+          else push_range(P, S, ctl, ws, fam_of(P, OP_NORMF, -1), 0, S.B);
         } else if (t.layer + 1 < P.n_layers) {
           push_range(P, S, ctl, ws, fam_of(P, OP_QKV, t.layer + 1), 0, P.n_qkv_tiles);
         } else {
@@ -793,7 +815,7 @@ template <int kKind>
 __device__ void notifier(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws, Control* ctl,
                          int* counters) {
   const int lane = threadIdx.x & 31;
-  const bool trace = S.trace != nullptr;
+  const bool trace = Kind<kKind>::trace && S.trace != nullptr;
   int tail = 0;
   unsigned long long n_batches = 0, fence_ns = 0;
   for (;;) {
@@ -899,7 +921,7 @@ __device__ void controller(const DevPlan& P, const StepParams& S, Smem& sm, unsi
   int released = 0;
   int dq_head = 0, fq_tail = 0;
   bool dead = false;
-  const bool trace = S.trace != nullptr;
+  const bool trace = Kind<kKind>::trace && S.trace != nullptr;
   int nrec = 0;
   uint32_t t_pop = 0, t_ready = 0;
   auto stamp = [&](int rec, int field, uint32_t v) {
@@ -1538,6 +1560,28 @@ __device__ __forceinline__ void gemv_task(const DevPlan& P, const StepParams& S,
   bar_sync(BAR_COMP, kComputeThreads);  // the partial tiles are free for the next task
 }
 
+// wide batch: store v at column c of batch row b of an activation buffer with
+// ld columns (its bf16 value, and with the split its bf16 remainder)
+__device__ __forceinline__ void store_act(const DevPlan& P, __nv_bfloat16* buf, size_t ld, int b, size_t c, float v) {
+  const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+  buf[(size_t)act_buf_row(P.act_split, b, 0) * ld + c] = hv;
+  if (P.act_split) buf[(size_t)act_buf_row(P.act_split, b, 1) * ld + c] = __float2bfloat16_rn(v - __bfloat162float(hv));
+}
+
+// wide batch: accumulator columns of batch rows 8 g8 .. 8 g8 + 7 from TMEM
+// address ta (value plus remainder products with the split)
+__device__ __forceinline__ void acc_rows8(uint32_t ta, int split, int g8, float (&v)[8]) {
+  if (split) {
+    float r[8];
+    tmem_ld8(ta + 16u * (uint32_t)g8, v);
+    tmem_ld8(ta + 16u * (uint32_t)g8 + 8u, r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] += r[i];
+  } else {
+    tmem_ld8(ta + 8u * (uint32_t)g8, v);
+  }
+}
+
 // ldmatrix: four 8x8 b16 matrices from shared memory; lane l gives the
 // address of row l % 8 of matrix l / 8 (16 bytes), register m receives the
 // matrix-m elements of the mma fragment layout (plain or transposed).
@@ -1566,9 +1610,11 @@ __device__ __forceinline__ int sw128_off(int r, int c) { return r * 128 + ((c ^ 
 
 // One task of split-KV decode attention for the qpg query heads of a GQA
 // group: up to attn_split consecutive 64-key chunks of one sequence, one ring
-// slot each (K rows, then V rows, as 128-byte-swizzled TMA boxes), one chunk
-// per compute warp (flash-decoding partials: unnormalised output, running
-// maximum, exp-sum).  A warp computes the chunk's scores S = Q K^T and
+// slot each (K rows, then V rows, as 128-byte-swizzled TMA boxes); compute
+// warp w takes chunks w, w + 8, ... of the task (flash-decoding partials:
+// unnormalised output, running maximum, exp-sum).  A (sequence, kv head)
+// whose chunks all fit one task writes its finished output here and skips
+// the merge.  A warp computes the chunk's scores S = Q K^T and
 // O += P V with bf16 warp MMAs (m16n8k16, fp32 accumulation): MMA row h
 // carries head h's query (or probabilities) as bf16 values and row h + 8 the
 // bf16 remainders, so that the products see about 16 significant bits and
@@ -1593,10 +1639,9 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
   float o[8][4];
 #pragma unroll
   for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  const int cc = c0 + w;  // this warp's chunk (attn_split <= 8 chunks per task)
-  if (cc < c1) {
-    // query fragments (scaled by 1/sqrt(64)): dims 16t + 2q, +1 and +8, +9 of head g
-    uint32_t qa[4][4];
+  // query fragments (scaled by 1/sqrt(64)): dims 16t + 2q, +1 and +8, +9 of head g
+  uint32_t qa[4][4];
+  if (c0 + w < c1) {
     const float* qrow = reinterpret_cast<const float*>(ws + P.off_q) + (size_t)a.b * P.n_q_heads * D +
                         (size_t)(a.g * qpg + (hv ? g : 0)) * D;
 #pragma unroll
@@ -1606,6 +1651,9 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
       split_pair(x01.x * 0.125f, x01.y * 0.125f, qa[t][0], qa[t][1]);
       split_pair(x89.x * 0.125f, x89.y * 0.125f, qa[t][2], qa[t][3]);
     }
+  }
+  // this warp's chunks c0 + w, c0 + w + 8, ... (online softmax across them)
+  for (int cc = c0 + w; cc < c1; cc += kComputeWarps) {
     const int n_old = max(0, min(CH, p - cc * CH));
     const bool has_new = (p - cc * CH) < CH;
     const int n_keys = n_old + (has_new ? 1 : 0);
@@ -1615,11 +1663,21 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
       const unsigned char* src = reinterpret_cast<const unsigned char*>(lane < 8 ? P.k_cache : P.v_cache) + row * D * 2;
       knew = __ldcg(reinterpret_cast<const uint4*>(src) + (lane & 7));
     }
-    if (trec && lane == 0) trec[TR_STAGED] = (uint32_t)global_ns();
+    if (trec && lane == 0 && cc == c0 + w) trec[TR_STAGED] = (uint32_t)global_ns();
     uint32_t par;
-    const int slot = task_slot(d, cc - c0, P.ring_slots, par);
+    const int R = P.ring_slots, i = cc - c0;
+    const int slot = task_slot(d, i, R, par);
+    if (i >= R) {
+      // The ring position also held chunk i - R of this task.  A parity wait
+      // on the full barrier cannot tell that use's phase from this one's, so
+      // first wait until chunk i - R has been released (its warp processes
+      // its chunks in increasing order, none waiting on a later chunk).
+      uint32_t par_prev;
+      task_slot(d, i - R, R, par_prev);
+      wait_mbar(&sm.empty[slot], par_prev, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    }
     wait_mbar(&sm.full[slot], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
-    if (trec && lane == 0) trec[TR_DATA] = (uint32_t)global_ns();
+    if (trec && lane == 0 && cc == c0 + w) trec[TR_DATA] = (uint32_t)global_ns();
     unsigned char* kb = ring + (size_t)slot * P.slot_bytes;
     unsigned char* vb = kb + (size_t)CH * D * 2;
     if (has_new) {
@@ -1717,40 +1775,25 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
         Ls = fmaf(sm.alsum[ww][h], f, Ls);
       }
     }
-    float* part = reinterpret_cast<float*>(ws + P.off_apart) +
-                  (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2)) + h * (D + 2);
-    part[dd] = O;
-    if (dd == 0) {
-      part[D] = M;
-      part[D + 1] = Ls;
+    if (sm.nch[a.b] == 1) {
+      // the pair's only task: the finished output (the merge of one partial)
+      const size_t oc = (size_t)(a.g * qpg + h) * D + dd;
+      reinterpret_cast<float*>(ws + P.off_attn)[(size_t)a.b * P.n_q_heads * D + oc] = O / Ls;
+      if (P.wide) store_act(P, reinterpret_cast<__nv_bfloat16*>(ws + P.off_attn_bf), (size_t)P.n_q_heads * D, a.b, oc, O / Ls);
+    } else {
+      float* part = reinterpret_cast<float*>(ws + P.off_apart) +
+                    (((size_t)a.b * Hkv + a.g) * P.max_chunks + a.c) * (size_t)(qpg * (D + 2)) + h * (D + 2);
+      part[dd] = O;
+      if (dd == 0) {
+        part[D] = M;
+        part[D + 1] = Ls;
+      }
     }
   }
   // every warp has read the partials before any of them writes the staging
   // buffer again (the next task may start without a barrier of its own)
   bar_sync(BAR_COMP, kComputeThreads);
   if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
-}
-
-// wide batch: store v at column c of batch row b of an activation buffer with
-// ld columns (its bf16 value, and with the split its bf16 remainder)
-__device__ __forceinline__ void store_act(const DevPlan& P, __nv_bfloat16* buf, size_t ld, int b, size_t c, float v) {
-  const __nv_bfloat16 hv = __float2bfloat16_rn(v);
-  buf[(size_t)act_buf_row(P.act_split, b, 0) * ld + c] = hv;
-  if (P.act_split) buf[(size_t)act_buf_row(P.act_split, b, 1) * ld + c] = __float2bfloat16_rn(v - __bfloat162float(hv));
-}
-
-// wide batch: accumulator columns of batch rows 8 g8 .. 8 g8 + 7 from TMEM
-// address ta (value plus remainder products with the split)
-__device__ __forceinline__ void acc_rows8(uint32_t ta, int split, int g8, float (&v)[8]) {
-  if (split) {
-    float r[8];
-    tmem_ld8(ta + 16u * (uint32_t)g8, v);
-    tmem_ld8(ta + 16u * (uint32_t)g8 + 8u, r);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] += r[i];
-  } else {
-    tmem_ld8(ta + 8u * (uint32_t)g8, v);
-  }
 }
 
 // Merge of the chunk partials of one (sequence, GQA group): the output of
@@ -1809,15 +1852,16 @@ __device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S
 // thread itself, after the event fired (the controller released the task),
 // into kBStages stages of the staging buffer.
 
-// NORM / NORM2 / NORMF: warp w takes batch row 8 idx + w: the residual (NORM
-// and NORMF add the previous layer's down-projection partials in a fixed
-// order; NORM stores the sum back as the residual), then RMSNorm times the
-// gain, stored as bf16 for the GEMM tasks.
-__device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S, unsigned char* ws,
+// NORM / NORM2 / NORMF (wide batch), batch row d.idx, all compute threads:
+// the row's residual (x plus the previous layer's down partials, summed in a
+// fixed order; kept in x by NORM) and its RMSNorm * gain as the GEMM tasks'
+// bf16 activation row (value, and remainder with the split).  Thread t takes
+// columns [8t, 8t + 8): every load of the row is issued before the first use.
+__device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws,
                                           const TaskDesc& d) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int b = d.idx * 8 + w, H = P.hidden, nblk = H >> 8;
-  if (b >= S.B) return;
+  const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
+  const int b = d.idx, H = P.hidden, c = 8 * ct;
+  const bool on = c < H;
   const LayerPtrs* layers = reinterpret_cast<const LayerPtrs*>(ws + P.off_layers);
   const int lx = d.op == OP_NORMF ? P.n_layers : d.layer;
   const bool parts = P.kind == MK_MODEL_DENSE && d.op != OP_NORM2 && lx > 0;  // (an MoE decoder's x is complete)
@@ -1825,55 +1869,63 @@ __device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S,
                                                                                    : P.final_norm;
   float* x = reinterpret_cast<float*>(ws + P.off_x) + (size_t)b * H;
   const float* dp = reinterpret_cast<const float*>(ws + P.off_dpart) + (size_t)b * H;
-  float v[kMaxBlk][8];
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f), e = a;
   float ss = 0.f;
+  if (on) {
+    a = __ldcg(reinterpret_cast<const float4*>(x + c));
+    e = __ldcg(reinterpret_cast<const float4*>(x + c) + 1);
+    if (parts) {
+      float4 pa[kMaxKc], pe[kMaxKc];
 #pragma unroll
-  for (int i = 0; i < kMaxBlk; ++i)
-    if (i < nblk) {
-      const int c = 256 * i + 8 * lane;
-      float4 a = __ldcg(reinterpret_cast<const float4*>(x + c)), e = __ldcg(reinterpret_cast<const float4*>(x + c) + 1);
-      if (parts)
-        for (int kc = 0; kc < P.n_kc; ++kc) {
+      for (int kc = 0; kc < kMaxKc; ++kc)
+        if (kc < P.n_kc) {
           const float4* d4 = reinterpret_cast<const float4*>(dp + (size_t)kc * P.max_batch * H + c);
-          const float4 p0 = __ldcg(d4), p1 = __ldcg(d4 + 1);
-          a.x += p0.x; a.y += p0.y; a.z += p0.z; a.w += p0.w;
-          e.x += p1.x; e.y += p1.y; e.z += p1.z; e.w += p1.w;
+          pa[kc] = __ldcg(d4);
+          pe[kc] = __ldcg(d4 + 1);
         }
-      v[i][0] = a.x; v[i][1] = a.y; v[i][2] = a.z; v[i][3] = a.w;
-      v[i][4] = e.x; v[i][5] = e.y; v[i][6] = e.z; v[i][7] = e.w;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) ss += v[i][j] * v[i][j];
-      if (d.op == OP_NORM && parts) {
+      for (int kc = 0; kc < kMaxKc; ++kc)
+        if (kc < P.n_kc) {
+          a.x += pa[kc].x; a.y += pa[kc].y; a.z += pa[kc].z; a.w += pa[kc].w;
+          e.x += pe[kc].x; e.y += pe[kc].y; e.z += pe[kc].z; e.w += pe[kc].w;
+        }
+      if (d.op == OP_NORM) {
         reinterpret_cast<float4*>(x + c)[0] = a;
         reinterpret_cast<float4*>(x + c)[1] = e;
       }
-      // debug capture: the residual after layer lx - 1 (what NORM and NORMF reduce)
-      if (S.cap_resid && lx > 0 && d.op != OP_NORM2) {
-        float4* c4 = reinterpret_cast<float4*>(S.cap_resid + ((size_t)(lx - 1) * S.B + b) * H + c);
-        c4[0] = a;
-        c4[1] = e;
-      }
     }
-  const float inv = 1.0f / sqrtf(warp_sum(ss) / (float)H + P.eps);
-  __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + P.off_xn);
-  __nv_bfloat16* xv = xn + (size_t)act_buf_row(P.act_split, b, 0) * H;
-  __nv_bfloat16* xr = xn + (size_t)act_buf_row(P.act_split, b, 1) * H;
-#pragma unroll
-  for (int i = 0; i < kMaxBlk; ++i)
-    if (i < nblk) {
-      const int c = 256 * i + 8 * lane;
-      float gf[8];
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(gp) + c / 8), gf);
-      __align__(16) __nv_bfloat16 o[8], rm[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float y = v[i][j] * inv * gf[j];
-        o[j] = __float2bfloat16_rn(y);
-        rm[j] = __float2bfloat16_rn(y - __bfloat162float(o[j]));
-      }
-      *reinterpret_cast<uint4*>(xv + c) = *reinterpret_cast<const uint4*>(o);
-      if (P.act_split) *reinterpret_cast<uint4*>(xr + c) = *reinterpret_cast<const uint4*>(rm);
+    // debug capture: the residual after layer lx - 1 (what NORM and NORMF reduce)
+    if (S.cap_resid && lx > 0 && d.op != OP_NORM2) {
+      float4* c4 = reinterpret_cast<float4*>(S.cap_resid + ((size_t)(lx - 1) * S.B + b) * H + c);
+      c4[0] = a;
+      c4[1] = e;
     }
+    ss = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + e.x * e.x + e.y * e.y + e.z * e.z + e.w * e.w;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) sm.red8[0][w] = ss;
+  bar_sync(BAR_COMP, kComputeThreads);
+  float tot = 0.f;
+#pragma unroll
+  for (int k = 0; k < kComputeWarps; ++k) tot += sm.red8[0][k];
+  const float inv = 1.0f / sqrtf(tot / (float)H + P.eps);
+  if (on) {
+    float gf[8];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(gp) + c / 8), gf);
+    const float v[8] = {a.x, a.y, a.z, a.w, e.x, e.y, e.z, e.w};
+    __align__(16) __nv_bfloat16 o[8], rm[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float y = v[j] * inv * gf[j];
+      o[j] = __float2bfloat16_rn(y);
+      rm[j] = __float2bfloat16_rn(y - __bfloat162float(o[j]));
+    }
+    __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + P.off_xn);
+    *reinterpret_cast<uint4*>(xn + (size_t)act_buf_row(P.act_split, b, 0) * H + c) = *reinterpret_cast<const uint4*>(o);
+    if (P.act_split)
+      *reinterpret_cast<uint4*>(xn + (size_t)act_buf_row(P.act_split, b, 1) * H + c) = *reinterpret_cast<const uint4*>(rm);
+  }
+  bar_sync(BAR_COMP, kComputeThreads);  // every warp has read the sums before the next task writes them
 }
 
 // MMA issue of a wide-batch GEMM task (one thread): per chunk c the task's
@@ -1883,7 +1935,7 @@ __device__ __forceinline__ void task_norm(const DevPlan& P, const StepParams& S,
 // is loaded once the MMAs of chunk c - 1 released its stage.
 __device__ __forceinline__ void gemm_issue_wide(const DevPlan& P, Smem& sm, unsigned char* ring, Control* ctl,
                                                 const TaskDesc& d, const void* bmap, int x0, int nk, int parts,
-                                                int N, uint32_t& bq) {
+                                                int N, uint32_t& bq, uint32_t* trec) {
   const int R = P.ring_slots;
   const uint32_t idesc = umma_idesc_bf16(kWideRows, N);
   const uint32_t tm = sm.tmem_base;
@@ -1910,9 +1962,11 @@ __device__ __forceinline__ void gemm_issue_wide(const DevPlan& P, Smem& sm, unsi
       sl[q] = task_slot(d, parts * c + q, R, par);
       wait_mbar(&sm.full[sl[q]], par, ctl, P.spin_timeout_ns, d.fam, d.idx);
     }
+    if (trec && c == 0) { trec[TR_DATA] = (uint32_t)global_ns(); trec[TR_ISSUE] = sm.slot_t[d.slot_ph & 0xffff]; }
     const uint32_t u = u0 + (uint32_t)c;
     const int st = (int)(u % kBStages);
     wait_mbar(&sm.bfull[st], (u / kBStages) & 1u, ctl, P.spin_timeout_ns, d.fam, d.idx);
+    if (trec && c == 0) trec[TR_LOADS] = (uint32_t)global_ns();
     tc_fence_after();
     const uint64_t b = umma_desc_sw128(stages + (size_t)st * bbytes);
     for (int q = 0; q < parts; ++q) {
@@ -1925,6 +1979,7 @@ __device__ __forceinline__ void gemm_issue_wide(const DevPlan& P, Smem& sm, unsi
   }
   bq = u0 + (uint32_t)nk;
   umma_commit(&sm.acc_bar);
+  if (trec) trec[TR_STAGED] = (uint32_t)global_ns();  // (the last MMA issued)
 }
 
 // A wide-batch GEMM task: QKV (+ RoPE, KV append), O projection (+ residual),
@@ -1933,14 +1988,18 @@ __device__ __forceinline__ void gemm_issue_wide(const DevPlan& P, Smem& sm, unsi
 // 32q + 31 of the tile; the two warps of a quadrant split the batch columns.
 __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ring,
                                                unsigned char* ws, Control* ctl, const TaskDesc& d, uint32_t& tc_n,
-                                               uint32_t& bq) {
+                                               uint32_t& bq, uint32_t* trec) {
   const int ct = threadIdx.x - kComputeBase, lane = ct & 31, w = ct >> 5;
   const int B = S.B, H = P.hidden, D = P.head_dim;
   const int N = P.act_split ? 16 * ceil_div(B, 8) : ceil_div(B, 16) * 16;  // MMA N (see act_buf_row)
   const int sp = P.act_split;
   const unsigned char* gmaps = ws + P.off_tmap + (size_t)P.n_layers * kTmapPerLayer * kTmapBytes;
   const void* xn_map = gmaps + (size_t)TMG_XN * kTmapBytes;
-  int x0 = 0, nk = H / 64, parts = 1;
+  // QKV, O and gate/up: K segment seg of tile idx / gseg (split K)
+  const int gseg = d.op == OP_QKV ? P.gseg_qkv : d.op == OP_OPROJ ? P.gseg_o : d.op == OP_GATEUP ? P.gseg_gu : 1;
+  const int tile = d.idx / gseg, seg = d.idx - tile * gseg;
+  const int K = d.op == OP_OPROJ ? P.n_q_heads * D : H;
+  int x0 = seg * (K / gseg), nk = K / gseg / 64, parts = 1;
   const void* bmap = xn_map;
   if (d.op == OP_OPROJ) bmap = gmaps + (size_t)TMG_ATTN * kTmapBytes;
   if (d.op == OP_GATEUP) parts = 2;
@@ -1950,33 +2009,80 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
     nk = P.kseg / 64;
   }
   if (w == 0) {
-    if (lane == 0) gemm_issue_wide(P, sm, ring, ctl, d, bmap, x0, nk, parts, N, bq);
+    if (lane == 0) gemm_issue_wide(P, sm, ring, ctl, d, bmap, x0, nk, parts, N, bq, trec);
     __syncwarp();
   }
   wait_local(&sm.acc_bar, tc_n & 1u, P.spin_timeout_ns);
   tc_n++;
   tc_fence_after();
+  if (trec && lane == 0) trec[TR_MATH] = (uint32_t)global_ns();
   const int q = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant = weight rows 32q .. 32q + 31
   const int r = 32 * q + lane;           // this lane's row of the tile
   const uint32_t ta = S_tmem_lane(sm.tmem_base, q);
   const int ng = ceil_div(ceil_div(B, 8), 2);  // groups of 8 batch rows per warpgroup
   const int gb0 = (w >> 2) * ng, gb1 = min(gb0 + ng, ceil_div(B, 8));  // this warp's groups
-  switch (d.op) {
+  // split K: every segment's task writes its partial tile (value + remainder
+  // products added) and counts in; the last one to count in sums the
+  // partials in segment order (the same order whichever task is last) and
+  // runs the tile's epilogue, the others stop here
+  float* gpart = reinterpret_cast<float*>(ws + P.off_gpart);
+  auto gp_at = [&](int sg, int part, int g8) -> float* {
+    return gpart + ((((size_t)tile * gseg + sg) * parts + part) * kWideRows + r) * P.act_rows + 8 * g8;
+  };
+  bool run_epi = true;
+  if (gseg > 1) {
+    for (int part = 0; part < parts; ++part)
+      for (int g8 = gb0; g8 < gb1; ++g8) {
+        float v[8];
+        acc_rows8(ta + 128u * (uint32_t)part, sp, g8, v);
+        float4* dst = reinterpret_cast<float4*>(gp_at(seg, part, g8));
+        __stcg(dst, make_float4(v[0], v[1], v[2], v[3]));
+        __stcg(dst + 1, make_float4(v[4], v[5], v[6], v[7]));
+      }
+    __threadfence();
+    tc_fence_before();
+    bar_sync(BAR_COMP, kComputeThreads);
+    if (ct == 0) {
+      int* ctr = reinterpret_cast<int*>(ws + P.off_gctr) + (d.op == OP_QKV ? 0 : d.op == OP_OPROJ ? 1 : 2) * kGctrPerOp + tile;
+      const int old = atomicAdd(ctr, 1);
+      __threadfence();
+      sm.gemm_last = old == gseg - 1;
+      if (old == gseg - 1) *ctr = 0;  // (no other task of this tile counts in again in this step)
+    }
+    bar_sync(BAR_COMP, kComputeThreads);
+    run_epi = sm.gemm_last != 0;
+  }
+  // the tile's values at this lane's row for batch rows 8 g8 .. 8 g8 + 7
+  // (part: gate 0 / up 1): from TMEM, or (split K) the segments' partials
+  // summed in segment order (their loads issued together)
+  auto rows8 = [&](int part, int g8, float (&v)[8]) {
+    if (gseg == 1) {
+      acc_rows8(ta + 128u * (uint32_t)part, sp, g8, v);
+      return;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    for (int sg = 0; sg < gseg; ++sg) {
+      const float4* src = reinterpret_cast<const float4*>(gp_at(sg, part, g8));
+      const float4 a = __ldcg(src), b = __ldcg(src + 1);
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w; v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+  };
+  if (run_epi) switch (d.op) {
     case OP_QKV: {
       // a tile is two heads (q, k or v rows); rotate-half pairs (j, j + 32)
       // of a head sit in quadrants (0, 1) and (2, 3): the odd quadrants hand
       // their values over through the staging buffer
       const int nq = P.n_q_heads * D / kWideRows, nkv = P.n_kv_heads * D / kWideRows;
-      const int kind = d.idx < nq ? 0 : d.idx < nq + nkv ? 1 : 2;
-      const int h0 = 2 * (d.idx - (kind == 0 ? 0 : kind == 1 ? nq : nq + nkv));
+      const int kind = tile < nq ? 0 : tile < nq + nkv ? 1 : 2;
+      const int h0 = 2 * (tile - (kind == 0 ? 0 : kind == 1 ? nq : nq + nkv));
       float* xch = sm.xs();  // [64][act_rows]
       if (q & 1)
         for (int g8 = gb0; g8 < gb1; ++g8) {
-          const int c8 = 8 * g8;
           float v[8];
-          acc_rows8(ta, sp, g8, v);
+          rows8(0, g8, v);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) xch[((q >> 1) * 32 + lane) * P.act_rows + c8 + i] = v[i];
+          for (int i = 0; i < 8; ++i) xch[((q >> 1) * 32 + lane) * P.act_rows + 8 * g8 + i] = v[i];
         }
       tc_fence_before();
       bar_sync(BAR_COMP, kComputeThreads);
@@ -1984,8 +2090,14 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
         const int hh = h0 + (q >> 1), j = lane;
         for (int g8 = gb0; g8 < gb1; ++g8) {
           const int c8 = 8 * g8;
+          float2 cs[8];  // (cos, sin) of (position, j): read-only, loaded ahead of the group's stores
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            cs[i] = (kind != 2 && c8 + i < B)
+                        ? __ldg(reinterpret_cast<const float2*>(ws + P.off_rope) + (size_t)sm.ctx[c8 + i] * 32 + j)
+                        : make_float2(1.f, 0.f);
           float v[8];
-          acc_rows8(ta, sp, g8, v);
+          rows8(0, g8, v);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int b = c8 + i;
@@ -1998,8 +2110,7 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
               vc[j] = __float2bfloat16_rn(v0);
               vc[j + 32] = __float2bfloat16_rn(v1);
             } else {
-              const float2 cs = __ldg(reinterpret_cast<const float2*>(ws + P.off_rope) + (size_t)pos * 32 + j);
-              const float x0r = v0 * cs.x - v1 * cs.y, x1r = v1 * cs.x + v0 * cs.y;
+              const float x0r = v0 * cs[i].x - v1 * cs[i].y, x1r = v1 * cs[i].x + v0 * cs[i].y;
               if (kind == 0) {
                 float* qb = reinterpret_cast<float*>(ws + P.off_q) + (size_t)b * P.n_q_heads * D + hh * D;
                 qb[j] = x0r;
@@ -2016,25 +2127,26 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
       }
     } break;
     case OP_OPROJ: {
+      // residual: x += o W_o^T, one fire-and-forget add per element (the
+      // tile's only writer, so the sum is x + o exactly as a load and store)
       float* x = reinterpret_cast<float*>(ws + P.off_x);
-      const int col = d.idx * kWideRows + r;
+      const int col = tile * kWideRows + r;
       for (int g8 = gb0; g8 < gb1; ++g8) {
-        const int c8 = 8 * g8;
         float v[8];
-        acc_rows8(ta, sp, g8, v);
+        rows8(0, g8, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          if (c8 + i < B) x[(size_t)(c8 + i) * H + col] += v[i];
+          if (8 * g8 + i < B) atomicAdd(x + (size_t)(8 * g8 + i) * H + col, v[i]);
       }
     } break;
     case OP_GATEUP: {
       __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_h_bf);
-      const int col = d.idx * kWideRows + r;
+      const int col = tile * kWideRows + r;
       for (int g8 = gb0; g8 < gb1; ++g8) {
         const int c8 = 8 * g8;
         float g[8], u[8];
-        acc_rows8(ta, sp, g8, g);
-        acc_rows8(ta + 128u, sp, g8, u);
+        rows8(0, g8, g);
+        rows8(1, g8, u);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           if (c8 + i < B) store_act(P, hb, P.ffn, c8 + i, col, g[i] / (1.0f + expf(-g[i])) * u[i]);
@@ -2046,7 +2158,7 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
       for (int g8 = gb0; g8 < gb1; ++g8) {
         const int c8 = 8 * g8;
         float v[8];
-        acc_rows8(ta, sp, g8, v);
+        rows8(0, g8, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           if (c8 + i < B) dp[(size_t)(c8 + i) * H + col] = v[i];
@@ -2054,15 +2166,15 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
     } break;
     case OP_LM: {
       // logits of vocabulary row `row`; per batch column the warp's best
-      // (logit, id) key, published with an atomic max when it beats the
-      // running maximum (order independent)
+      // (logit, id) key joins this CTA's running best in shared memory; after
+      // the task, a column's key is published with one global atomic max
+      // when it beats what this CTA published before (order independent)
       const int row = d.idx * kWideRows + r;
       const bool in = row < P.vocab;
-      unsigned long long* best = reinterpret_cast<unsigned long long*>(ws + P.off_lmbest);
       for (int g8 = gb0; g8 < gb1; ++g8) {
         const int c8 = 8 * g8;
         float v[8];
-        acc_rows8(ta, sp, g8, v);
+        rows8(0, g8, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int b = c8 + i;
@@ -2074,12 +2186,21 @@ __device__ __forceinline__ void task_gemm_wide(const DevPlan& P, const StepParam
             const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
             key = other > key ? other : key;
           }
-          if (lane == 0 && key > __ldcg(best + b)) atomicMax(best + b, key);
+          if (lane == 0) atomicMax(&sm.lm_cta[b], key);
         }
       }
+      tc_fence_before();
+      bar_sync(BAR_COMP, kComputeThreads);
+      unsigned long long* best = reinterpret_cast<unsigned long long*>(ws + P.off_lmbest);
+      for (int b = ct; b < B; b += kComputeThreads)
+        if (sm.lm_cta[b] > sm.lm_pub[b]) {
+          sm.lm_pub[b] = sm.lm_cta[b];
+          atomicMax(best + b, sm.lm_cta[b]);
+        }
     } break;
     default: break;
   }
+  if (trec && lane == 0) trec[TR_EPI] = (uint32_t)global_ns();
   tc_fence_before();
   bar_sync(BAR_COMP, kComputeThreads);  // the accumulator and the staging buffer are free for the next task
 }
@@ -2463,9 +2584,9 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
   int a_tag = -1;
   uint32_t tc_n = 0;  // tcgen05 tasks run (the phase of acc_bar)
   uint32_t bq = 0;    // wide batch: activation chunks the MMA issuer loaded (stage and phase)
-  constexpr bool kWide = kKind == kKindDenseWide || kKind == kKindMoeDecWide;
-  constexpr bool kMoe = kKind == MK_MODEL_MOE_LAYER || kKind == MK_MODEL_MOE_DECODER || kKind == kKindMoeDecWide;
-  constexpr bool tc = kKind != MK_MODEL_DENSE;
+  constexpr bool kWide = Kind<kKind>::wide;
+  constexpr bool kMoe = Kind<kKind>::moe;
+  constexpr bool tc = Kind<kKind>::base != MK_MODEL_DENSE;
   if constexpr (tc) {
     // tensor memory for the tcgen05 accumulators, held for the kernel's lifetime
     if (w == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -2481,7 +2602,7 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     if (!wait_local(&sm.go_bar[k & 1], (k >> 1) & 1, P.spin_timeout_ns)) break;
     const TaskDesc d = sm.cur[k & 1];
     if (d.op == OP_END) break;
-    uint32_t* trec = (d.rec > 0 && w == 0) ? trace_rec(S, d.rec) : nullptr;
+    uint32_t* trec = (Kind<kKind>::trace && d.rec > 0 && w == 0) ? trace_rec(S, d.rec) : nullptr;
     if (trec && lane == 0) trec[TR_CSTART] = (uint32_t)global_ns();
     GemvSpec g;
     bool moe_task = false;
@@ -2505,13 +2626,13 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
         task_combine(P, S, ws, d);
       }
     }
-    if (kKind == MK_MODEL_MOE_LAYER || moe_task) {
+    if (Kind<kKind>::moe_layer || moe_task) {
       a_tag = -1;  // MoE tasks use the staging buffer as scratch
     } else if (kWide && (d.op == OP_QKV || d.op == OP_OPROJ || d.op == OP_GATEUP || d.op == OP_DOWN ||
                          d.op == OP_LM)) {
-      if constexpr (kWide) task_gemm_wide(P, S, sm, ring, ws, ctl, d, tc_n, bq);
+      if constexpr (kWide) task_gemm_wide(P, S, sm, ring, ws, ctl, d, tc_n, bq, trec);
     } else if (kWide && (d.op == OP_NORM || d.op == OP_NORM2 || d.op == OP_NORMF)) {
-      if constexpr (kWide) task_norm(P, S, ws, d);
+      if constexpr (kWide) task_norm(P, S, sm, ws, d);
     } else if (!kWide && gemv_spec(P, d, g)) {
       // all B activation rows are staged together; an unchanged tag reuses them
       const GemvItem it = gemv_item(sm.geo[d.op], B, threadIdx.x - kComputeBase);
@@ -2613,6 +2734,9 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     sm.dq_head = sm.dq_tail = sm.fq_head = sm.fq_tail = sm.notifier_stop = 0;
   }
   if (tid < kComputeWarps * kMaxB) sm.lm_seen[tid / kMaxB][tid % kMaxB] = 0ull;
+  if (tid < kMaxBatch) sm.lm_cta[tid] = sm.lm_pub[tid] = 0ull;
+  if (P.wide && blockIdx.x == 0)  // split-K tile counters
+    for (int i = tid; i < 3 * kGctrPerOp; i += blockDim.x) reinterpret_cast<int*>(ws + P.off_gctr)[i] = 0;
   __syncthreads();
   if (!moe && !sm.bad && tid < B) {
     int c = S.ctx[tid], s = S.slots[tid], t = S.tokens[tid];
@@ -2680,7 +2804,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
     ctl->q_head = 0;
     ctl->q_tail = 0;
     if (moe) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, -1), 0, ceil_div(B, 8));
-    else if (P.wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, 0), 0, ceil_div(B, 8));  // EV_IN[0] armed at zero
+    else if (P.wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM, 0), 0, B);  // EV_IN[0] armed at zero
     else push_range(P, S, ctl, ws, fam_of(P, OP_QKV, 0), 0, P.n_qkv_tiles);  // EV_IN[0] is armed at zero
   }
   if (tid == 0) {
@@ -2727,13 +2851,19 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
 
 namespace mk {
 
-static const void* kernel_for(const DevPlan& P) {
+template <int kFlags>
+static const void* kernel_of(const DevPlan& P) {
   switch (P.kind) {
-    case MK_MODEL_MOE_LAYER: return (const void*)megakernel<MK_MODEL_MOE_LAYER>;
+    case MK_MODEL_MOE_LAYER: return (const void*)megakernel<MK_MODEL_MOE_LAYER | kFlags>;
     case MK_MODEL_MOE_DECODER:
-      return P.wide ? (const void*)megakernel<kKindMoeDecWide> : (const void*)megakernel<MK_MODEL_MOE_DECODER>;
-    default: return P.wide ? (const void*)megakernel<kKindDenseWide> : (const void*)megakernel<MK_MODEL_DENSE>;
+      return P.wide ? (const void*)megakernel<kKindMoeDecWide | kFlags>
+                    : (const void*)megakernel<MK_MODEL_MOE_DECODER | kFlags>;
+    default:
+      return P.wide ? (const void*)megakernel<kKindDenseWide | kFlags> : (const void*)megakernel<MK_MODEL_DENSE | kFlags>;
   }
+}
+static const void* kernel_for(const DevPlan& P) {
+  return (P.debug_flags & MK_DEBUG_TRACE) ? kernel_of<kTraced>(P) : kernel_of<0>(P);
 }
 
 mk_status dev_query(int* n_sm, int* smem_optin, int* device, std::string& err) {

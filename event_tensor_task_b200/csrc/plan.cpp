@@ -152,12 +152,12 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
   };
   const bool wide = P.wide != 0;
   auto nsplit = [&](int b) { return ceil_div(ceil_div(bd.ctx[b] + 1, P.chunk), P.attn_split); };
-  auto rows8 = [&](int i, int& b0, int& b1) { b0 = 8 * i; b1 = std::min(B, 8 * i + 8); };
   if (wide && op == OP_QKV) {
-    // a 128-row tile of [Wq; Wk; Wv]: two heads of q, k or v rows
-    const int nq = Hq * D / kWideRows, nk = Hkv * D / kWideRows;
-    const int kind = idx < nq ? 0 : idx < nq + nk ? 1 : 2;
-    const int h0 = 2 * (idx - (kind == 0 ? 0 : kind == 1 ? nq : nq + nk));
+    // a 128-row tile of [Wq; Wk; Wv]: two heads of q, k or v rows (every K
+    // segment's task is modelled as writing the tile's outputs)
+    const int nq = Hq * D / kWideRows, nk = Hkv * D / kWideRows, tile = idx / P.gseg_qkv;
+    const int kind = tile < nq ? 0 : tile < nq + nk ? 1 : 2;
+    const int h0 = 2 * (tile - (kind == 0 ? 0 : kind == 1 ? nq : nq + nk));
     t.wait_ev = counter(EV_N1, l);
     t.notify_ev = counter(EV_QKV, l, 0);
     for (int b = 0; b < B; ++b) {
@@ -178,9 +178,8 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
     case OP_NORM:
     case OP_NORM2:
     case OP_NORMF: {
-      // wide batch: rows 8 idx .. of the residual -> normalised bf16 rows
-      int b0, b1;
-      rows8(idx, b0, b1);
+      // wide batch: row idx of the residual -> its normalised bf16 row
+      const int b0 = idx, b1 = idx + 1;
       const int lx = op == OP_NORMF ? P.n_layers : l;
       if (mdec)  // (the MoE decoder's layers chain through the combine of the layer before)
         t.wait_ev = lx > 0 ? counter(EV_MCOMB, lx - 1) : counter(EV_IN, 0);
@@ -228,21 +227,32 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       for (int b = 0; b < B; ++b) { nsp[b] = nsplit(b); pre[b + 1] = pre[b] + nsp[b]; }
       AttnTask a = decode_attn(idx, B, Hkv, nsp.data(), pre.data());
       t.wait_ev = counter(EV_QKV, l, wide ? 0 : a.g);
-      t.notify_ev = counter(EV_CHUNK, l, a.b, a.g);
-      t.follow_fam = fam_index(OP_MERGE, l);
-      t.follow_idx = a.b * Hkv + a.g;
+      const bool single = nsp[a.b] == 1;  // the pair's only task: finished output, no merge
+      if (single) {
+        t.notify_ev = counter(EV_ATTN, l);
+      } else {
+        t.notify_ev = counter(EV_CHUNK, l, a.b, a.g);
+        t.follow_fam = fam_index(OP_MERGE, l);
+        t.follow_idx = a.b * Hkv + a.g;
+      }
       long long qb = a.b * QD + (long long)a.g * qpg * D;
       t.reads.push_back({BUF_Q, qb, qb + (long long)qpg * D});
       int p0 = a.c * P.attn_split * P.chunk, p1 = std::min(p0 + P.attn_split * P.chunk, bd.ctx[a.b] + 1);
       long long kb = kv_row(l, a.b, a.g, p0);
       t.reads.push_back({BUF_KC, kb, kb + (long long)(p1 - p0) * D});
       t.reads.push_back({BUF_VC, kb, kb + (long long)(p1 - p0) * D});
-      long long pb = ((long long)a.b * Hkv + a.g) * P.max_chunks + a.c;
-      t.writes.push_back({BUF_APART, pb, pb + 1});
+      if (single) {
+        long long ob = a.b * QD + (long long)a.g * qpg * D;
+        t.writes.push_back({BUF_ATTN, ob, ob + (long long)qpg * D});
+      } else {
+        long long pb = ((long long)a.b * Hkv + a.g) * P.max_chunks + a.c;
+        t.writes.push_back({BUF_APART, pb, pb + 1});
+      }
     } break;
     case OP_MERGE: {
       int b = idx / Hkv, g = idx % Hkv;
       int nch = nsplit(b);
+      if (nch == 1) { t.exists = false; break; }  // (the attention task wrote the output)
       long long pb = ((long long)b * Hkv + g) * P.max_chunks;
       t.reads.push_back({BUF_APART, pb, pb + nch});
       long long ob = b * QD + (long long)g * qpg * D;
@@ -252,24 +262,26 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
     case OP_OPROJ: {
       t.wait_ev = counter(EV_ATTN, l);
       t.notify_ev = counter(EV_O, l);
+      const int tile = idx / P.gseg_o;
       for (int b = 0; b < B; ++b) {
         t.reads.push_back({BUF_ATTN, b * QD, (b + 1) * QD});
-        long long xb = (long long)b * H + (long long)idx * P.tile_o;
+        long long xb = (long long)b * H + (long long)tile * P.tile_o;
         t.reads.push_back({BUF_X, xb, xb + P.tile_o});
         if (l > 0 && !mdec && !wide)
           for (int kc = 0; kc < P.n_kc; ++kc) {
-            long long pb = ((long long)kc * P.max_batch + b) * H + (long long)idx * P.tile_o;
+            long long pb = ((long long)kc * P.max_batch + b) * H + (long long)tile * P.tile_o;
             t.reads.push_back({BUF_DPART, pb, pb + P.tile_o});
           }
         t.writes.push_back({BUF_X, xb, xb + P.tile_o});
       }
     } break;
     case OP_GATEUP: {
+      const int tile = idx / P.gseg_gu;
       t.wait_ev = wide ? counter(EV_N2, l) : counter(EV_O, l);
-      t.notify_ev = counter(EV_GU, l, idx * P.tile_gu / P.kseg);
+      t.notify_ev = counter(EV_GU, l, tile * P.tile_gu / P.kseg);
       for (int b = 0; b < B; ++b) {
         t.reads.push_back({wide ? BUF_XN : BUF_X, (long long)b * H, (long long)(b + 1) * H});
-        long long hb = (long long)b * F + (long long)idx * P.tile_gu;
+        long long hb = (long long)b * F + (long long)tile * P.tile_gu;
         t.writes.push_back({BUF_H, hb, hb + P.tile_gu});
       }
     } break;
@@ -401,8 +413,8 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
     case EV_IN:
       if (mdec) break;  // (the MoE decoder's layers chain through EV_MCOMB)
       if (wide) {
-        if (c[0] < dp.n_layers) add(fam_index(OP_NORM, c[0]), 0, n8);
-        else add(fam_index(OP_NORMF, -1), 0, n8);
+        if (c[0] < dp.n_layers) add(fam_index(OP_NORM, c[0]), 0, bd.B);
+        else add(fam_index(OP_NORMF, -1), 0, bd.B);
       } else if (c[0] < dp.n_layers) {
         add(fam_index(OP_QKV, c[0]), 0, dp.n_qkv_tiles);
       } else {
@@ -418,8 +430,8 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
     case EV_MCOMB:
       if (!mdec) break;  // (the MoE layer's end is a follow-up)
       if (wide) {
-        if (c[0] + 1 < dp.n_layers) add(fam_index(OP_NORM, c[0] + 1), 0, n8);
-        else add(fam_index(OP_NORMF, -1), 0, n8);
+        if (c[0] + 1 < dp.n_layers) add(fam_index(OP_NORM, c[0] + 1), 0, bd.B);
+        else add(fam_index(OP_NORMF, -1), 0, bd.B);
       } else if (c[0] + 1 < dp.n_layers) {
         add(fam_index(OP_QKV, c[0] + 1), 0, dp.n_qkv_tiles);
       } else {
@@ -438,7 +450,7 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
     case EV_ATTN: add(fam_index(OP_OPROJ, c[0]), 0, dp.n_otiles); break;
     case EV_O:
       if (mdec) add(fam_index(OP_ROUTE, c[0]), 0, n8);
-      else if (wide) add(fam_index(OP_NORM2, c[0]), 0, n8);
+      else if (wide) add(fam_index(OP_NORM2, c[0]), 0, bd.B);
       else add(fam_index(OP_GATEUP, c[0]), 0, dp.n_gutiles);
       break;
     case EV_GU: add(fam_index(OP_DOWN, c[0]), c[1] * dp.n_dtiles, dp.n_dtiles); break;
@@ -628,8 +640,9 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.spin_timeout_ns = o->spin_timeout_ns > 0 ? o->spin_timeout_ns : 2000000000LL;
   P.fault_ctr = -1;
 
-  // K segment of the down projection (split-K), at most 2048 columns
-  int kseg = mdec ? 2048 : (o->kseg ? o->kseg : std::min(F, 2048));  // (no dense FFN in an MoE decoder)
+  // K segment of the down projection (split-K), at most 2048 columns (wide
+  // batch: 1024 by default, twice the down tasks for the phase)
+  int kseg = mdec ? 2048 : (o->kseg ? o->kseg : std::min(F, wide ? 1024 : 2048));  // (no dense FFN in an MoE decoder)
   while (kseg > 256 && F % kseg) kseg -= 256;
   P.kseg = kseg;
   // GEMV tiles on tensor cores: 16, 32 or 64 rows per task in whole 16-row
@@ -645,8 +658,10 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.chunk = o->attn_chunk ? o->attn_chunk : 64;
   P.slot_bytes = 16384;
   P.wide = wide ? 1 : 0;
-  P.attn_split = o->attn_split ? o->attn_split : (wide ? 8 : 1);
-  if (P.attn_split < 1 || P.attn_split > 8) { err = "attn_split must be in [1, 8]"; return MK_ERR_INVALID_ARG; }
+  // key chunks per attention task: small batches take a sequence's chunks
+  // (up to 2048 keys) in one task, which then also skips the merge
+  P.attn_split = o->attn_split ? o->attn_split : (wide ? 8 : 32);
+  if (P.attn_split < 1 || P.attn_split > 64) { err = "attn_split must be in [1, 64]"; return MK_ERR_INVALID_ARG; }
   if (wide) {
     // tcgen05 GEMM tasks: kWideRows weight rows each (the MMA's M), every
     // weight matrix read in 64-column chunks, the batch as the MMA's N
@@ -676,11 +691,25 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     { err = "tile_down must be 16, 32 or 64 and divide hidden"; return MK_ERR_UNSUPPORTED; }
   if (!wide && P.tile_lm != 32 && P.tile_lm != 64) { err = "tile_lm must be 32 or 64"; return MK_ERR_UNSUPPORTED; }
   if (P.chunk != 64) { err = "attn_chunk must be 64"; return MK_ERR_UNSUPPORTED; }
-  P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv;
-  P.n_otiles = H / P.tile_o;
-  P.n_gutiles = F / P.tile_gu;
+  // wide batch: K segments per GEMM tile (split K, see DevPlan::gseg_qkv):
+  // 4 segments of at least 2 chunks of 64 columns (2 for gate/up, which
+  // streams two weight parts), so that a phase has several tasks per SM
+  P.gseg_qkv = P.gseg_o = P.gseg_gu = 1;
+  if (wide) {
+    P.gseg_qkv = std::min(4, H / 128);
+    P.gseg_o = std::min(4, Hq * D / 128);
+    P.gseg_gu = std::min(2, H / 128);
+    if ((Hq + 2 * Hkv) * D / kWideRows > kGctrPerOp || H / kWideRows > kGctrPerOp ||
+        (!mdec && F / kWideRows > kGctrPerOp))
+      { err = "wide batch: at most 64 tiles of 128 rows per projection"; return MK_ERR_UNSUPPORTED; }
+  }
+  // task counts (wide batch: tiles x K segments; task i is segment i % gseg of tile i / gseg)
+  P.n_qkv_tiles = (Hq + 2 * Hkv) * D / P.tile_qkv * P.gseg_qkv;
+  P.n_otiles = H / P.tile_o * P.gseg_o;
+  P.n_gutiles = F / P.tile_gu * P.gseg_gu;
   P.n_dtiles = H / P.tile_down;
   P.n_kc = F / P.kseg;
+  if (wide && P.n_kc > 8) { err = "wide batch: at most 8 down-projection K segments (ffn / kseg)"; return MK_ERR_UNSUPPORTED; }
   P.n_lm_tiles = ceil_div(P.vocab, P.tile_lm);
   P.max_chunks = ceil_div(P.max_ctx, P.chunk);
 
@@ -745,6 +774,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     P.max_tiles = ceil_div(P.max_tokens * P.top_k, P.moe_tm) + std::min(P.n_experts, P.max_tokens * P.top_k);
     }
   const int e_tok8 = Emit(p.code).op(X_B).push(8).op(X_CEILDIV).ret();  // ceil(B / 8)
+  const int e_tok1 = Emit(p.code).op(X_B).ret();                         // B (wide batch: one norm task per row)
   static const int kMoeDecOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU, OP_EDOWN,
                                    OP_COMBINE};
   static const int kWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_NORM2, OP_GATEUP, OP_DOWN};
@@ -754,12 +784,12 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   const int* layer_ops = mdec ? (wide ? kMoeDecWideOps : kMoeDecOps) : wide ? kWideOps : kLayerOps;
   const int max_tasks_attn = Hkv * P.max_batch * ceil_div(P.max_chunks, P.attn_split);
   for (int l = 0; l < P.n_layers; ++l) {
-    if (wide) add_family(OP_NORM, l, e_tok8, ceil_div(P.max_batch, 8), 0);
+    if (wide) add_family(OP_NORM, l, e_tok1, P.max_batch, 0);
     add_family(OP_QKV, l, emit_const(p.code, P.n_qkv_tiles), P.n_qkv_tiles, 0);
     add_family(OP_ATTN, l, e_attn, max_tasks_attn, 0);
     add_family(OP_MERGE, l, e_merge, Hkv * P.max_batch, 1);
     add_family(OP_OPROJ, l, emit_const(p.code, P.n_otiles), P.n_otiles, 0);
-    if (dwide) add_family(OP_NORM2, l, e_tok8, ceil_div(P.max_batch, 8), 0);
+    if (dwide) add_family(OP_NORM2, l, e_tok1, P.max_batch, 0);
     if (mdec) {
       add_family(OP_ROUTE, l, e_tok8, ceil_div(P.max_tokens, 8), 0);
       add_family(OP_MINDPTR, l, emit_const(p.code, 1), 1, 1);
@@ -771,7 +801,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
       add_family(OP_DOWN, l, emit_const(p.code, P.n_dtiles * P.n_kc), P.n_dtiles * P.n_kc, 0);
     }
   }
-  if (wide) add_family(OP_NORMF, -1, e_tok8, ceil_div(P.max_batch, 8), 0);
+  if (wide) add_family(OP_NORMF, -1, e_tok1, P.max_batch, 0);
   add_family(OP_LM, -1, emit_const(p.code, P.n_lm_tiles), P.n_lm_tiles, 0);
   add_family(OP_LMFIN, -1, emit_const(p.code, 1), 1, 1);
   P.n_families = (int)p.fams.size();
@@ -800,12 +830,16 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
             Emit(p.code).push(0).coord(0).op(X_LT).push(P.n_dtiles * P.n_kc).op(X_MUL).ret());
   if (wide) add_event(EV_QKV, 2, L, 1, 1, emit_const(p.code, P.n_qkv_tiles));  // (a tile spans two kv heads)
   else add_event(EV_QKV, 2, L, Hkv, 1, emit_const(p.code, qkv_per_group));
+  // (b < B) * n_b * (n_b > 1), n_b = the pair's attention tasks: a pair with
+  // one task notifies EV_ATTN itself
   add_event(EV_CHUNK, 3, L, P.max_batch, Hkv,
             Emit(p.code).coord(1).op(X_B).op(X_LT).coord(1).op(X_CTX_AT).push(1).op(X_ADD)
-                .push(P.chunk).op(X_CEILDIV).push(P.attn_split).op(X_CEILDIV).op(X_MUL).ret());
+                .push(P.chunk).op(X_CEILDIV).push(P.attn_split).op(X_CEILDIV).op(X_MUL)
+                .push(1).coord(1).op(X_CTX_AT).push(1).op(X_ADD).push(P.chunk).op(X_CEILDIV)
+                .push(P.attn_split).op(X_CEILDIV).op(X_LT).op(X_MUL).ret());
   add_event(EV_ATTN, 1, L, 1, 1, Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret());
   add_event(EV_O, 1, L, 1, 1, emit_const(p.code, P.n_otiles));
-  add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu));
+  add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu * P.gseg_gu));
   add_event(EV_LM, 1, 1, 1, 1, emit_const(p.code, P.n_lm_tiles));
   if (mdec) {  // one element per layer (EV_MH: per layer and GroupGEMM tile)
     add_event(EV_ROUTE, 1, L, 1, 1, e_tok8);
@@ -817,9 +851,9 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     for (int id = EV_LM + 1; id <= EV_MCOMB; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // MoE: empty
   }
   if (wide) {
-    add_event(EV_N1, 1, L, 1, 1, e_tok8);
-    add_event(EV_N2, 1, dwide ? L : 0, 1, 1, e_tok8);
-    add_event(EV_NF, 1, 1, 1, 1, e_tok8);
+    add_event(EV_N1, 1, L, 1, 1, e_tok1);
+    add_event(EV_N2, 1, dwide ? L : 0, 1, 1, e_tok1);
+    add_event(EV_NF, 1, 1, 1, 1, e_tok1);
   } else {
     for (int id = EV_N1; id < EV_COUNT; ++id) add_event(id, 1, 0, 1, 1, emit_const(p.code, 0));  // wide only: empty
   }
@@ -928,6 +962,16 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   P.off_xn = take(2LL * ar * P.hidden);
   P.off_attn_bf = take(2LL * ar * P.hidden);
   P.off_h_bf = take(2LL * ar * P.ffn);
+  // wide batch, split K: the partial tiles of the largest phase (fp32
+  // [task][parts][128 rows][act_rows]) and the tiles' counters
+  long long gtasks = 0;
+  if (P.wide) {
+    if (P.gseg_qkv > 1) gtasks = std::max(gtasks, (long long)P.n_qkv_tiles);
+    if (P.gseg_o > 1) gtasks = std::max(gtasks, (long long)P.n_otiles);
+    if (P.gseg_gu > 1 && P.kind == MK_MODEL_DENSE) gtasks = std::max(gtasks, 2LL * P.n_gutiles);
+  }
+  P.off_gpart = take(gtasks * kWideRows * P.act_rows * 4);
+  P.off_gctr = take(P.wide ? 4LL * 3 * kGctrPerOp : 0);
   if (P.kind != MK_MODEL_DENSE) {
     // one MoE scratch block per MoE layer (layer 0's offsets; the others follow at moe_stride)
     const long long pairs = (long long)P.max_tokens * P.top_k;
@@ -1020,6 +1064,7 @@ mk_status validate_plan(const Plan& p, const Binding& bd_in, std::string& err) {
     }
     for (int i = 0; i < n; ++i) {
       p.task(f, i, bd, t);
+      if (!t.exists) continue;
       if (t.notify_ev >= 0) {
         notifiers[t.notify_ev]++;
         last_notifier_fam[t.notify_ev] = std::max(last_notifier_fam[t.notify_ev], f);
@@ -1319,7 +1364,11 @@ mk_status simulate_plan(const Plan& p, const Binding& bd_in, int n_orders, unsig
   std::mt19937 rng(seed);
   std::vector<int> want(p.dp.debug_slots, 0);
   for (int f = 0; f < p.dp.n_families; ++f)
-    for (int i = 0; i < p.actual_extent(f, bd); ++i) want[p.fams[f].debug_base + i] = 1;
+    for (int i = 0; i < p.actual_extent(f, bd); ++i) {
+      TaskRec t;
+      p.task(f, i, bd, t);
+      if (t.exists) want[p.fams[f].debug_base + i] = 1;
+    }
   std::vector<int> first_set;
   for (int k = 0; k < n_orders; ++k) {
     bool dynamic = moe || (k % 2) == 1;

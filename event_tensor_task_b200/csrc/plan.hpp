@@ -43,6 +43,8 @@ struct TaskRec {
   int notify_ev = -1;     // counter index decremented at completion (-1: none)
   int follow_fam = -1;    // follow-up family run by the notifier that reaches zero
   int follow_idx = -1;
+  bool exists = true;     // false: an index of the family this binding does not run (a merge of a
+                          // (sequence, kv head) whose chunks fit one attention task)
   std::vector<Region> reads, writes;
 };
 

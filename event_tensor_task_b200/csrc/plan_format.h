@@ -301,7 +301,15 @@ struct DevPlan {
   int32_t act_rows;   // batch rows of the activation buffers (max_batch rounded up to 16)
   int32_t act_split;  // 1: each activation row stored as its bf16 value and its bf16 remainder (see act_buf_row)
   int64_t off_xn, off_attn_bf, off_h_bf;  // bf16 [max_batch][H], [max_batch][H], [max_batch][F]
+  // wide batch, split K: QKV, O-projection and gate/up tiles run as gseg_*
+  // tasks over consecutive K segments; each writes its fp32 partial tile to
+  // off_gpart and counts in at the tile's counter (off_gctr, [3][64]); the
+  // last to count in sums the partials in segment order and runs the
+  // tile's epilogue (the counters are zeroed at launch and by that task)
+  int32_t gseg_qkv, gseg_o, gseg_gu, pad6;
+  int64_t off_gpart, off_gctr;
 };
+constexpr int kGctrPerOp = 64;  // split-K tile counters per GEMM op (tiles of 128 rows)
 
 MK_HD int seq_table_bytes(const DevPlan& P) { return seq_table_bytes_for(P.max_batch); }
 

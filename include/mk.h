@@ -371,10 +371,12 @@ mk_status mk_plan_family_info(const mk_plan* p, int family, mk_family_info* out)
  * exactly its number of notifies.  MK_ERR_INVALID_ARG for null arguments. */
 mk_status mk_plan_counter_region(const mk_plan* p, long long* byte_offset, int* n_counters);
 
-/* Tile sizes the plan chose, written to out[12] in this order: tile_qkv,
+/* Tile sizes the plan chose, written to out[15] in this order: tile_qkv,
  * tile_o, tile_gu, tile_down, kseg, tile_lm, attn_chunk, n_sm, ring_slots,
  * attn_split (key chunks per attention task), wide (1: the wide-batch path),
- * act_split (1: wide-batch activations as value + remainder rows). */
+ * act_split (1: wide-batch activations as value + remainder rows), and the
+ * K segments per tile of the QKV, O-projection and gate/up GEMM tasks (wide
+ * batch: a tile's segments run as separate tasks; 1 otherwise). */
 mk_status mk_plan_tiles(const mk_plan* p, int* out);
 
 /* Host validation for one binding of the symbols (B, ctx_lens host array):

@@ -14,7 +14,9 @@ Task families of one dense layer, in the order a layer runs them:
 * ``qkv``    — one per ``tile_qkv`` output rows of the stacked Q/K/V weights;
 * ``attn``   — one per (sequence b, kv head g, key chunk c),
   ``c < ceil((ctx_b + 1) / chunk)``;
-* ``merge``  — one per (b, g): combine that head group's chunk partials;
+* ``merge``  — one per (b, g) whose chunks span more than one attention task:
+  combine that head group's partials (a pair with one task writes its output
+  itself, without a merge);
 * ``oproj``  — one per ``tile_o`` rows of the output projection;
 * ``gateup`` — one per ``tile_gu`` rows of the gate (and the same rows of up);
 * ``down``   — one per (``tile_down`` rows, K segment of ``kseg`` columns).
@@ -30,8 +32,10 @@ K-segment-major: ``kc * (H / tile_down) + n``.
 
 With ``tiles["wide"]`` (the wide-batch layout, where the normalised
 activations are materialised) a layer also runs ``norm`` before ``qkv`` and
-``norm2`` before ``gateup``, and ``normf`` runs before ``lm``: one task per 8
-batch rows each.
+``norm2`` before ``gateup``, and ``normf`` runs before ``lm``: one task per
+batch row each.  Its ``qkv``, ``oproj`` and ``gateup`` tiles may run as
+``tiles["gseg"]`` = (q, o, g) tasks each, one per K segment (task i is
+segment i % s of tile i // s).
 """
 from __future__ import annotations
 
@@ -46,14 +50,15 @@ def dense_family_extents(shape, B: int, ctx, tiles: dict) -> dict:
     Hq, Hkv = shape.n_q_heads, shape.n_kv_heads
     nch = [_ceil(_ceil(int(ctx[b]) + 1, tiles["chunk"]), tiles.get("split", 1)) for b in range(B)]
     n_lm = _ceil(shape.vocab, tiles["tile_lm"])
-    norms = {"norm": _ceil(B, 8), "norm2": _ceil(B, 8), "normf": _ceil(B, 8)} if tiles.get("wide") else {}
+    norms = {"norm": B, "norm2": B, "normf": B} if tiles.get("wide") else {}
+    sq, so, sg = tiles.get("gseg", (1, 1, 1))  # K segments per tile, each its own task
     return {
         **norms,
-        "qkv": (Hq + 2 * Hkv) * D // tiles["tile_qkv"],
+        "qkv": (Hq + 2 * Hkv) * D // tiles["tile_qkv"] * sq,
         "attn": Hkv * sum(nch),
-        "merge": Hkv * B,
-        "oproj": H // tiles["tile_o"],
-        "gateup": shape.ffn // tiles["tile_gu"],
+        "merge": Hkv * sum(1 for n in nch if n > 1),
+        "oproj": H // tiles["tile_o"] * so,
+        "gateup": shape.ffn // tiles["tile_gu"] * sg,
         "down": (H // tiles["tile_down"]) * (shape.ffn // tiles["kseg"]),
         "lm": n_lm,
         "lmfin": 1,
@@ -72,7 +77,7 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
     wide = bool(tiles.get("wide"))
     out = set()
     for l in range(shape.n_layers):
-        for fam in ("qkv", "merge", "oproj", "gateup", "down") + (("norm", "norm2") if wide else ()):
+        for fam in ("qkv", "oproj", "gateup", "down") + (("norm", "norm2") if wide else ()):
             out.update((fam, l, i) for i in range(ext[fam]))
         base = 0
         for b in range(B):
@@ -80,6 +85,8 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
             for g in range(Hkv):
                 for c in range(nch):
                     out.add(("attn", l, Hkv * base + g * nch + c))
+                if nch > 1:
+                    out.add(("merge", l, b * Hkv + g))
             base += nch
     for fam in ("lm", "lmfin") + (("normf",) if wide else ()):
         out.update((fam, -1, i) for i in range(ext[fam]))

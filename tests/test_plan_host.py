@@ -97,7 +97,8 @@ def test_simulator_clean(sched, B, ctx):
     t = d.tiles()
     tiles = {k: t[k] for k in ("tile_qkv", "chunk", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm")}
     assert tiles == dict(tile_qkv=32, chunk=64, tile_o=32, tile_gu=32, tile_down=64, kseg=1024, tile_lm=64)
-    assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, tiles))
+    assert t["attn_split"] == 32  # a sequence's chunks up to 2048 keys in one attention task (no merge)
+    assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, dict(tiles, split=32)))
 
 
 def test_simulator_many_orders():
