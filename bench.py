@@ -285,6 +285,19 @@ def torch_baselines(s, w, K, V, max_ctx, tok0, dev, n_steps):
                     "eager and as one captured CUDA graph; device-timed with CUDA events"}
 
 
+def profile_torch():
+    """Five replays of the same-box per-op PyTorch CUDA graph of the 1B B=1
+    step (a short command for an ncu launch list of the baseline)."""
+    import torch
+    dev = "cuda:0"
+    s, w_cpu, w, K_cpu, V_cpu, K, V, max_ctx = setup_model(dev)
+    base = TorchPerOpDecoder(s, w, K, V, max_ctx, CTX0, WINDOW, 5, dev)
+    base.capture()
+    for _ in range(5):
+        base.graph.replay()
+    torch.cuda.synchronize()
+
+
 def device_kv_cache(s, n_slots, max_ctx, ctx, dev, seed=0):
     """A bf16 N(0, 1) cache drawn on the device (seeded), zero past each
     sequence's context: the symbolic-batch sweep's 64-sequence cache is too
@@ -407,10 +420,10 @@ def profile_wide(B):
     dev = "cuda:0"
     s = wl.LLAMA_1B
     w = {k: v.to(dev) for k, v in wl.dense_weights(s, seed=0).items()}
-    ctx0 = [int(c) for c in wl.context_lengths(B, 128, 1024)]
+    ctx0 = [int(c) for c in wl.context_lengths(64, 128, 1024)]
     max_ctx = max(ctx0) + 32
-    K, V = device_kv_cache(s, B, max_ctx, ctx0, dev)
-    dec = mk.DenseDecoder(s, w, K, V, max_batch=64, max_ctx=max_ctx, n_slots=B)
+    K, V = device_kv_cache(s, 64, max_ctx, ctx0, dev)
+    dec = mk.DenseDecoder(s, w, K, V, max_batch=64, max_ctx=max_ctx, n_slots=64)
     tok = torch.full((B,), 5, dtype=torch.int32, device=dev)
     slots = torch.arange(B, dtype=torch.int32, device=dev)
     ctx = torch.tensor(ctx0[:B], dtype=torch.int32, device=dev)
@@ -732,6 +745,8 @@ def main():
                     help="only run 4 MoE-layer calls on T tokens (a short command for ncu) and exit")
     ap.add_argument("--profile-wide", type=int, default=0, metavar="B",
                     help="only run 4 wide-batch 1B decode steps at batch B (a short command for ncu) and exit")
+    ap.add_argument("--profile-torch", action="store_true",
+                    help="only replay the per-op PyTorch CUDA graph of the B=1 step 5 times (for ncu) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -746,6 +761,9 @@ def main():
         return
     if args.profile_wide:
         profile_wide(args.profile_wide)
+        return
+    if args.profile_torch:
+        profile_torch()
         return
 
     import torch
@@ -873,6 +891,9 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
+    if baselines:  # the baselines' rate on the same algorithmic bytes as the headline step
+        for k in ("torch_eager", "torch_cuda_graph"):
+            baselines[k]["achieved_gbs"] = step_bytes / (baselines[k]["us_per_step"] * 1e-6) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "us_per_step": 1000.0 * ms_step, **step_pct,
