@@ -659,8 +659,10 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.slot_bytes = 16384;
   P.wide = wide ? 1 : 0;
   // key chunks per attention task: small batches take a sequence's chunks
-  // (up to 2048 keys) in one task, which then also skips the merge
-  P.attn_split = o->attn_split ? o->attn_split : (wide ? 8 : 32);
+  // (up to 2048 keys) in one task, which then also skips the merge; wide
+  // batches 16 (two per warp: a warp's second chunk loads while the first
+  // is computed; measured best of 4..16 at B = 16 and 64)
+  P.attn_split = o->attn_split ? o->attn_split : (wide ? 16 : 32);
   if (P.attn_split < 1 || P.attn_split > 64) { err = "attn_split must be in [1, 64]"; return MK_ERR_INVALID_ARG; }
   if (wide) {
     // tcgen05 GEMM tasks: kWideRows weight rows each (the MMA's M), every

@@ -139,10 +139,11 @@ typedef struct mk_plan_opts {
    * other values are refused with MK_ERR_INVALID_ARG. */
   int fault;
   int fault_family;
-  /* Key chunks (attn_chunk keys each) per attention task: 0 = default (1 for
-   * max_batch <= 8, 8 above), at most 8.  Each compute warp of the task takes
-   * one chunk (tensor-core scores and P.V with an online softmax); the task
-   * leaves one partial for the merge. */
+  /* Key chunks (attn_chunk keys each) per attention task: 0 = default (32 for
+   * max_batch <= 8, 16 above), at most 64.  Compute warp w of the task takes
+   * chunks w, w + 8, ... (warp-MMA scores and P.V with an online softmax); the
+   * task leaves one partial for the merge, or, when it holds all of its
+   * (sequence, kv head)'s chunks, the finished output and no merge runs. */
   int attn_split;
   /* MoE GroupGEMM tiles, chosen per expert from the run-time histogram
    * (0 = default: routing-aware; 1 = routing-aware; 2 = fixed): an expert

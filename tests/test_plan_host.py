@@ -159,6 +159,25 @@ def test_moe_plan_build_families_and_limits():
             mk.MoELayer(shp, None, max_tokens=64, n_sm=148, host_only=True)
 
 
+def test_plan_option_ranges():
+    # the option fields accept their documented values and refuse the rest
+    for v in (0, 1, 2):
+        mk.MoELayer(wl.MOE_64x8, None, max_tokens=8, n_sm=148, host_only=True, moe_tiles=v).close()
+    for bad in (dict(moe_tiles=3), dict(moe_tiles=-1)):
+        with pytest.raises(mk.MkError):
+            mk.MoELayer(wl.MOE_64x8, None, max_tokens=8, n_sm=148, host_only=True, **bad)
+    for split in (1, 8, 64):
+        d = _host(wl.LLAMA_1B, max_batch=4, max_ctx=4160, n_sm=148, attn_split=split)
+        assert d.tiles()["attn_split"] == split
+        d.close()
+    for bad in (dict(attn_split=65), dict(attn_split=-1), dict(act_split=3)):
+        with pytest.raises(mk.MkError):
+            _host(wl.LLAMA_1B, max_batch=16, max_ctx=1088, n_sm=148, **bad)
+    # wide-batch defaults: 16 chunks per attention task, split K 4 / 4 / 2
+    t = _host(wl.LLAMA_1B, max_batch=64, max_ctx=1088, n_sm=148).tiles()
+    assert (t["attn_split"], t["gseg_qkv"], t["gseg_o"], t["gseg_gu"], t["kseg"]) == (16, 4, 4, 2, 1024)
+
+
 def test_moe_plan_requires_dynamic_schedule_and_rejects_dense_calls():
     d = mk.mk_model_desc()
     d.kind = mk.MK_MODEL_MOE_LAYER
