@@ -155,6 +155,7 @@ struct Smem {
   uint32_t slot_t[kMaxSlots];  // trace: when the producer issued the slot's copies
   float alsum[kComputeWarps][4], amax[kComputeWarps][4];  // attention: each warp's exp-sum and maximum per head
   int gemm_last;  // wide batch, split K: this CTA's task was the tile's last segment
+  int attn_last;  // attention: this CTA's task was its (sequence, kv head)'s last to finish
   // wide batch: this CTA's best argmax key per batch column, and what it published
   unsigned long long lm_cta[kMaxBatch], lm_pub[kMaxBatch];
   volatile int released;  // regular tasks the controller has handed to compute
@@ -691,7 +692,6 @@ struct NotifyInfo {
 
 template <int kKind>
 __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const Smem& sm, const TaskDesc& t) {
-  const int Hkv = P.n_kv_heads;
   const bool dyn = P.sched == MK_SCHED_DYNAMIC;
   NotifyInfo n;
   n.ctr = -1; n.ffam = -1; n.fop = 0; n.flayer = -1; n.fidx = 0; n.need_old = 0;
@@ -700,17 +700,7 @@ __device__ NotifyInfo notify_info(const DevPlan& P, const StepParams& S, const S
     case OP_NORM2: n.ctr = ev_ctr(P, EV_N2, t.layer); break;
     case OP_NORMF: n.ctr = ev_ctr(P, EV_NF, 0); break;
     case OP_QKV: n.ctr = ev_ctr(P, EV_QKV, t.layer, Kind<kKind>::wide ? 0 : decode_qkv(P, t.idx).group); break;
-    case OP_ATTN: {
-      AttnTask a = decode_attn(t.idx, S.B, Hkv, sm.nch, sm.pre);
-      if (sm.nch[a.b] == 1) {
-        // the pair's only task wrote the finished output: it counts for the merge
-        n.ctr = ev_ctr(P, EV_ATTN, t.layer);
-      } else {
-        n.ctr = ev_ctr(P, EV_CHUNK, t.layer, a.b, a.g);
-        n.ffam = fam_of(P, OP_MERGE, t.layer); n.fop = OP_MERGE; n.flayer = t.layer; n.fidx = a.b * Hkv + a.g;
-      }
-    } break;
-    case OP_MERGE: n.ctr = ev_ctr(P, EV_ATTN, t.layer); break;
+    case OP_ATTN: n.ctr = ev_ctr(P, EV_ATTN, t.layer); break;  // (every task; a pair's last one merged the pair)
     case OP_OPROJ: n.ctr = ev_ctr(P, EV_O, t.layer); break;
     case OP_GATEUP: n.ctr = ev_ctr(P, EV_GU, t.layer, t.idx / P.gseg_gu * P.tile_gu / P.kseg); break;
     case OP_DOWN: n.ctr = ev_ctr(P, EV_IN, t.layer + 1); break;
@@ -755,11 +745,7 @@ __device__ void push_successors(const DevPlan& P, const StepParams& S, const Sme
       for (int b = 0; b < S.B; ++b)
         push_range(P, S, ctl, ws, fam_of(P, OP_ATTN, t.layer), Hkv * sm.pre[b] + g * sm.nch[b], sm.nch[b]);
     } break;
-    case OP_MERGE: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
-    case OP_ATTN: {  // (a pair's only task counts for its merge: it fired EV_ATTN)
-      const AttnTask a = decode_attn(t.idx, S.B, Hkv, sm.nch, sm.pre);
-      if (sm.nch[a.b] == 1) push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles);
-    } break;
+    case OP_ATTN: push_range(P, S, ctl, ws, fam_of(P, OP_OPROJ, t.layer), 0, P.n_otiles); break;
     case OP_OPROJ:
       if (Kind<kKind>::moe_dec) push_range(P, S, ctl, ws, fam_of(P, OP_ROUTE, t.layer), 0, ceil_div(S.B, 8));
       else if (Kind<kKind>::wide) push_range(P, S, ctl, ws, fam_of(P, OP_NORM2, t.layer), 0, S.B);
@@ -1608,6 +1594,52 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
 // 16-byte chunk c of row r of a 64-column bf16 tile under the 128-byte swizzle
 __device__ __forceinline__ int sw128_off(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
+// Merge of the attention partials of one (sequence, GQA group), run by the
+// pair's last attention task to finish: the output of
+// head h is sum_c e^(m_c - M) o_c / sum_c e^(m_c - M) l_c.  Warp pair
+// (2h, 2h + 1) takes head h, 32 output columns each; a batch of up to 16
+// chunks is loaded in one round trip (lane c: m and l of chunk c; every lane:
+// its column of all the batch's chunk outputs), with an online rescale across
+// batches.
+__device__ __forceinline__ void merge_pair(const DevPlan& P, const Smem& sm, unsigned char* ws, int b, int g) {
+  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
+  const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, D = P.head_dim;
+  const int h = w >> 1, dd = (w & 1) * 32 + lane;
+  if (h >= qpg) return;
+  const int nch = sm.nch[b];
+  const size_t cs = (size_t)qpg * (D + 2);
+  const float* part = reinterpret_cast<const float*>(ws + P.off_apart) + ((size_t)b * Hkv + g) * P.max_chunks * cs +
+                      h * (D + 2);
+  float M = -INFINITY, L = 0.f, O = 0.f;
+  for (int c0 = 0; c0 < nch; c0 += 16) {
+    const int n = min(16, nch - c0);
+    const int c = c0 + lane;
+    const bool in = lane < n;  // lane c - c0 of the batch
+    const float mc = in ? __ldcg(part + c * cs + D) : -INFINITY;
+    const float lc = in ? __ldcg(part + c * cs + D + 1) : 0.f;
+    float ov[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) ov[q] = q < n ? __ldcg(part + (c0 + q) * cs + dd) : 0.f;
+    float mb = mc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const float Mn = fmaxf(M, mb);
+    const float sc = expf(M - Mn);  // 0 on the first batch (M = -inf, Mn finite)
+    const float e = in ? expf(mc - Mn) : 0.f;
+    L = L * sc + warp_sum(lc * e);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < 16; ++q) acc[q & 3] = fmaf(ov[q], __shfl_sync(0xffffffffu, e, q), acc[q & 3]);
+    O = O * sc + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    M = Mn;
+  }
+  float* out = reinterpret_cast<float*>(ws + P.off_attn) + (size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D;
+  out[dd] = O / L;
+  if (P.wide)  // the O projection's B operand
+    store_act(P, reinterpret_cast<__nv_bfloat16*>(ws + P.off_attn_bf), (size_t)P.n_q_heads * D, b,
+              (size_t)(g * qpg + h) * D + dd, O / L);
+}
+
 // One task of split-KV decode attention for the qpg query heads of a GQA
 // group: up to attn_split consecutive 64-key chunks of one sequence, one ring
 // slot each (K rows, then V rows, as 128-byte-swizzled TMA boxes); compute
@@ -1790,58 +1822,29 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
       }
     }
   }
+  if (sm.nch[a.b] > 1) {
+    // the pair's tasks count in after writing their partials; the last one
+    // to count in merges them (the same arithmetic whichever task that is).
+    // The barrier orders every warp's partial stores before thread 0's fence,
+    // which releases them with the count (as at the grid barrier).
+    bar_sync(BAR_COMP, kComputeThreads);
+    if (ct == 0) {
+      int* cnt = reinterpret_cast<int*>(ws + P.off_actr) + a.b * Hkv + a.g;
+      __threadfence();
+      const int old = atomicAdd(cnt, 1);
+      __threadfence();
+      sm.attn_last = old == sm.nch[a.b] - 1;
+      if (old == sm.nch[a.b] - 1) *cnt = 0;  // (no other task of this pair counts in again this layer)
+    }
+    bar_sync(BAR_COMP, kComputeThreads);
+    if (sm.attn_last) merge_pair(P, sm, ws, a.b, a.g);
+  }
   // every warp has read the partials before any of them writes the staging
   // buffer again (the next task may start without a barrier of its own)
   bar_sync(BAR_COMP, kComputeThreads);
   if (trec && lane == 0) trec[TR_RED] = (uint32_t)global_ns();
 }
 
-// Merge of the chunk partials of one (sequence, GQA group): the output of
-// head h is sum_c e^(m_c - M) o_c / sum_c e^(m_c - M) l_c.  Warp pair
-// (2h, 2h + 1) takes head h, 32 output columns each; a batch of up to 16
-// chunks is loaded in one round trip (lane c: m and l of chunk c; every lane:
-// its column of all the batch's chunk outputs), with an online rescale across
-// batches.
-__device__ __forceinline__ void task_merge(const DevPlan& P, const StepParams& S, Smem& sm, unsigned char* ws,
-                                        const TaskDesc& d) {
-  const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
-  const int Hkv = P.n_kv_heads, qpg = P.n_q_heads / Hkv, D = P.head_dim;
-  const int h = w >> 1, dd = (w & 1) * 32 + lane;
-  if (h >= qpg) return;
-  const int b = d.idx / Hkv, g = d.idx % Hkv;
-  const int nch = sm.nch[b];
-  const size_t cs = (size_t)qpg * (D + 2);
-  const float* part = reinterpret_cast<const float*>(ws + P.off_apart) + ((size_t)b * Hkv + g) * P.max_chunks * cs +
-                      h * (D + 2);
-  float M = -INFINITY, L = 0.f, O = 0.f;
-  for (int c0 = 0; c0 < nch; c0 += 16) {
-    const int n = min(16, nch - c0);
-    const int c = c0 + lane;
-    const bool in = lane < n;  // lane c - c0 of the batch
-    const float mc = in ? __ldcg(part + c * cs + D) : -INFINITY;
-    const float lc = in ? __ldcg(part + c * cs + D + 1) : 0.f;
-    float ov[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) ov[q] = q < n ? __ldcg(part + (c0 + q) * cs + dd) : 0.f;
-    float mb = mc;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-    const float Mn = fmaxf(M, mb);
-    const float sc = expf(M - Mn);  // 0 on the first batch (M = -inf, Mn finite)
-    const float e = in ? expf(mc - Mn) : 0.f;
-    L = L * sc + warp_sum(lc * e);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int q = 0; q < 16; ++q) acc[q & 3] = fmaf(ov[q], __shfl_sync(0xffffffffu, e, q), acc[q & 3]);
-    O = O * sc + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-    M = Mn;
-  }
-  float* out = reinterpret_cast<float*>(ws + P.off_attn) + (size_t)b * P.n_q_heads * D + (size_t)(g * qpg + h) * D;
-  out[dd] = O / L;
-  if (P.wide)  // the O projection's B operand
-    store_act(P, reinterpret_cast<__nv_bfloat16*>(ws + P.off_attn_bf), (size_t)P.n_q_heads * D, b,
-              (size_t)(g * qpg + h) * D + dd, O / L);
-}
 
 // ---------------------------------------------------------------- wide batch
 // (max_batch > 8.)  The normalised activations are materialised in bf16 by
@@ -2652,8 +2655,6 @@ __device__ void compute(const DevPlan& P, const StepParams& S, Smem& sm, unsigne
     } else if (d.op == OP_ATTN) {
       task_attn(P, S, sm, ring, ws, ctl, d, trec);
       a_tag = -1;  // the staging buffer held the warps' partial outputs
-    } else if (d.op == OP_MERGE) {
-      task_merge(P, S, sm, ws, d);
     } else if (d.op == OP_LMFIN) {
       for (int b = threadIdx.x - kComputeBase; b < B; b += kComputeThreads) {
         unsigned long long k = __ldcg(reinterpret_cast<const unsigned long long*>(ws + P.off_lmbest) + b);
@@ -2735,6 +2736,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
   }
   if (tid < kComputeWarps * kMaxB) sm.lm_seen[tid / kMaxB][tid % kMaxB] = 0ull;
   if (tid < kMaxBatch) sm.lm_cta[tid] = sm.lm_pub[tid] = 0ull;
+  if (P.kind != MK_MODEL_MOE_LAYER && blockIdx.x == 0)  // attention pair counters
+    for (int i = tid; i < P.max_batch * P.n_kv_heads; i += blockDim.x) reinterpret_cast<int*>(ws + P.off_actr)[i] = 0;
   if (P.wide && blockIdx.x == 0)  // split-K tile counters
     for (int i = tid; i < 3 * kGctrPerOp; i += blockDim.x) reinterpret_cast<int*>(ws + P.off_gctr)[i] = 0;
   __syncthreads();

@@ -2,8 +2,7 @@
 //
 // The graph of one dense decode step, per layer l (events in brackets):
 //   QKV tiles        wait EV_IN[l]        notify EV_QKV[l][g]
-//   ATTN chunks      wait EV_QKV[l][g]    notify EV_CHUNK[l][b][g] -> MERGE(b,g)
-//   MERGE (follow-up)                     notify EV_ATTN[l]
+//   ATTN chunks      wait EV_QKV[l][g]    notify EV_ATTN[l] (the pair's last task merges)
 //   OPROJ tiles      wait EV_ATTN[l]      notify EV_O[l]
 //   GATEUP tiles     wait EV_O[l]         notify EV_GU[l][kc]
 //   DOWN tiles       wait EV_GU[l][kc]    notify EV_IN[l+1]
@@ -34,9 +33,9 @@ namespace mk {
 static const char* kOpNames[OP_COUNT] = {"end", "qkv", "attn", "merge", "oproj", "gateup", "down", "norm", "lm",
                                          "norm2", "lmfin", "route", "mindptr", "egu", "edown", "combine", "mfin",
                                          "normf"};
-static const int kLayerOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_GATEUP, OP_DOWN};
+static const int kLayerOps[] = {OP_QKV, OP_ATTN, OP_OPROJ, OP_GATEUP, OP_DOWN};
 static const int kLmOps[] = {OP_LM, OP_LMFIN};
-static constexpr int kFamPerLayer = 6;
+static constexpr int kFamPerLayer = 5;
 
 // ---------------------------------------------------------------- expressions
 namespace {
@@ -227,14 +226,12 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       for (int b = 0; b < B; ++b) { nsp[b] = nsplit(b); pre[b + 1] = pre[b] + nsp[b]; }
       AttnTask a = decode_attn(idx, B, Hkv, nsp.data(), pre.data());
       t.wait_ev = counter(EV_QKV, l, wide ? 0 : a.g);
-      const bool single = nsp[a.b] == 1;  // the pair's only task: finished output, no merge
-      if (single) {
-        t.notify_ev = counter(EV_ATTN, l);
-      } else {
-        t.notify_ev = counter(EV_CHUNK, l, a.b, a.g);
-        t.follow_fam = fam_index(OP_MERGE, l);
-        t.follow_idx = a.b * Hkv + a.g;
-      }
+      t.notify_ev = counter(EV_ATTN, l);
+      // A pair's last task to finish merges the pair's partials into the
+      // output (a counter inside the task, not an event of the plan): the
+      // model writes the output region from the pair's only task and the
+      // partial slots from the others.
+      const bool single = nsp[a.b] == 1;
       long long qb = a.b * QD + (long long)a.g * qpg * D;
       t.reads.push_back({BUF_Q, qb, qb + (long long)qpg * D});
       int p0 = a.c * P.attn_split * P.chunk, p1 = std::min(p0 + P.attn_split * P.chunk, bd.ctx[a.b] + 1);
@@ -248,16 +245,6 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
         long long pb = ((long long)a.b * Hkv + a.g) * P.max_chunks + a.c;
         t.writes.push_back({BUF_APART, pb, pb + 1});
       }
-    } break;
-    case OP_MERGE: {
-      int b = idx / Hkv, g = idx % Hkv;
-      int nch = nsplit(b);
-      if (nch == 1) { t.exists = false; break; }  // (the attention task wrote the output)
-      long long pb = ((long long)b * Hkv + g) * P.max_chunks;
-      t.reads.push_back({BUF_APART, pb, pb + nch});
-      long long ob = b * QD + (long long)g * qpg * D;
-      t.writes.push_back({BUF_ATTN, ob, ob + (long long)qpg * D});
-      t.notify_ev = counter(EV_ATTN, l);
     } break;
     case OP_OPROJ: {
       t.wait_ev = counter(EV_ATTN, l);
@@ -454,7 +441,7 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
       else add(fam_index(OP_GATEUP, c[0]), 0, dp.n_gutiles);
       break;
     case EV_GU: add(fam_index(OP_DOWN, c[0]), c[1] * dp.n_dtiles, dp.n_dtiles); break;
-    default: break;  // EV_CHUNK, EV_LM and EV_ROUTE trigger follow-ups
+    default: break;  // EV_LM and EV_ROUTE trigger follow-ups
   }
 }
 
@@ -660,9 +647,10 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.wide = wide ? 1 : 0;
   // key chunks per attention task: small batches take a sequence's chunks
   // (up to 2048 keys) in one task, which then also skips the merge; wide
-  // batches 16 (two per warp: a warp's second chunk loads while the first
-  // is computed; measured best of 4..16 at B = 16 and 64)
-  P.attn_split = o->attn_split ? o->attn_split : (wide ? 16 : 32);
+  // batches 24 (three per warp: a warp's next chunk loads while one is
+  // computed; of 8, 16, 24 and 32, 16 was fastest at B = 16, 32 at B = 32 and
+  // 24 at B = 64, 24 the best over the three)
+  P.attn_split = o->attn_split ? o->attn_split : (wide ? 24 : 32);
   if (P.attn_split < 1 || P.attn_split > 64) { err = "attn_split must be in [1, 64]"; return MK_ERR_INVALID_ARG; }
   if (wide) {
     // tcgen05 GEMM tasks: kWideRows weight rows each (the MMA's M), every
@@ -762,7 +750,6 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     p.code.push_back(X_RET);
     e_attn = e.start;
   }
-  int e_merge = Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret();
   // MoE decoder: the MoE FFN's geometry (as build_moe_plan) on at most max_batch tokens
   if (mdec) {
     P.kind = MK_MODEL_MOE_DECODER;
@@ -777,19 +764,17 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     }
   const int e_tok8 = Emit(p.code).op(X_B).push(8).op(X_CEILDIV).ret();  // ceil(B / 8)
   const int e_tok1 = Emit(p.code).op(X_B).ret();                         // B (wide batch: one norm task per row)
-  static const int kMoeDecOps[] = {OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU, OP_EDOWN,
-                                   OP_COMBINE};
-  static const int kWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_NORM2, OP_GATEUP, OP_DOWN};
-  static const int kMoeDecWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_MERGE, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU,
+  static const int kMoeDecOps[] = {OP_QKV, OP_ATTN, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU, OP_EDOWN, OP_COMBINE};
+  static const int kWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_OPROJ, OP_NORM2, OP_GATEUP, OP_DOWN};
+  static const int kMoeDecWideOps[] = {OP_NORM, OP_QKV, OP_ATTN, OP_OPROJ, OP_ROUTE, OP_MINDPTR, OP_EGU,
                                        OP_EDOWN, OP_COMBINE};
-  const int fam_per_layer = mdec ? (wide ? 10 : 9) : wide ? 8 : kFamPerLayer;
+  const int fam_per_layer = mdec ? (wide ? 9 : 8) : wide ? 7 : kFamPerLayer;
   const int* layer_ops = mdec ? (wide ? kMoeDecWideOps : kMoeDecOps) : wide ? kWideOps : kLayerOps;
   const int max_tasks_attn = Hkv * P.max_batch * ceil_div(P.max_chunks, P.attn_split);
   for (int l = 0; l < P.n_layers; ++l) {
     if (wide) add_family(OP_NORM, l, e_tok1, P.max_batch, 0);
     add_family(OP_QKV, l, emit_const(p.code, P.n_qkv_tiles), P.n_qkv_tiles, 0);
     add_family(OP_ATTN, l, e_attn, max_tasks_attn, 0);
-    add_family(OP_MERGE, l, e_merge, Hkv * P.max_batch, 1);
     add_family(OP_OPROJ, l, emit_const(p.code, P.n_otiles), P.n_otiles, 0);
     if (dwide) add_family(OP_NORM2, l, e_tok1, P.max_batch, 0);
     if (mdec) {
@@ -832,14 +817,11 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
             Emit(p.code).push(0).coord(0).op(X_LT).push(P.n_dtiles * P.n_kc).op(X_MUL).ret());
   if (wide) add_event(EV_QKV, 2, L, 1, 1, emit_const(p.code, P.n_qkv_tiles));  // (a tile spans two kv heads)
   else add_event(EV_QKV, 2, L, Hkv, 1, emit_const(p.code, qkv_per_group));
-  // (b < B) * n_b * (n_b > 1), n_b = the pair's attention tasks: a pair with
-  // one task notifies EV_ATTN itself
-  add_event(EV_CHUNK, 3, L, P.max_batch, Hkv,
-            Emit(p.code).coord(1).op(X_B).op(X_LT).coord(1).op(X_CTX_AT).push(1).op(X_ADD)
-                .push(P.chunk).op(X_CEILDIV).push(P.attn_split).op(X_CEILDIV).op(X_MUL)
-                .push(1).coord(1).op(X_CTX_AT).push(1).op(X_ADD).push(P.chunk).op(X_CEILDIV)
-                .push(P.attn_split).op(X_CEILDIV).op(X_LT).op(X_MUL).ret());
-  add_event(EV_ATTN, 1, L, 1, 1, Emit(p.code).op(X_B).push(Hkv).op(X_MUL).ret());
+  // (EV_CHUNK is unused: the attention tasks of a (sequence, kv head) merge
+  // their partials in the last of them to finish, see task_attn)
+  add_event(EV_CHUNK, 1, 1, 1, 1, emit_const(p.code, 0));
+  // every attention task of the layer: Hkv * sum_b n_b
+  add_event(EV_ATTN, 1, L, 1, 1, e_attn);
   add_event(EV_O, 1, L, 1, 1, emit_const(p.code, P.n_otiles));
   add_event(EV_GU, 2, L, P.n_kc, 1, emit_const(p.code, P.kseg / P.tile_gu * P.gseg_gu));
   add_event(EV_LM, 1, 1, 1, 1, emit_const(p.code, P.n_lm_tiles));
@@ -974,6 +956,7 @@ void lower_plan(Plan& p, std::vector<unsigned char>& image) {
   }
   P.off_gpart = take(gtasks * kWideRows * P.act_rows * 4);
   P.off_gctr = take(P.wide ? 4LL * 3 * kGctrPerOp : 0);
+  P.off_actr = take(P.kind == MK_MODEL_MOE_LAYER ? 0 : 4LL * P.max_batch * P.n_kv_heads);
   if (P.kind != MK_MODEL_DENSE) {
     // one MoE scratch block per MoE layer (layer 0's offsets; the others follow at moe_stride)
     const long long pairs = (long long)P.max_tokens * P.top_k;

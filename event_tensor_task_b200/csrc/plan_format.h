@@ -27,13 +27,13 @@ enum Op : int32_t {
   OP_END = 0,
   OP_QKV = 1,     // RMSNorm -> Q/K/V rows -> RoPE -> KV append
   OP_ATTN = 2,    // one key chunk of one (sequence, kv head) -> softmax partials
-  OP_MERGE = 3,   // follow-up: merge a head group's chunk partials
+  OP_MERGE = 3,   // (reserved: a pair's last attention task merges its partials)
   OP_OPROJ = 4,   // output projection rows + residual
   OP_GATEUP = 5,  // RMSNorm -> gate and up rows -> SwiGLU
   OP_DOWN = 6,    // down projection rows over one K segment -> partial
-  OP_NORM = 7,    // wide batch: 8 rows: residual (x + down partials) -> x, RMSNorm(x) * attn gain -> bf16
+  OP_NORM = 7,    // wide batch, one row: residual (x + down partials) -> x, RMSNorm(x) * attn gain -> bf16
   OP_LM = 8,      // final RMSNorm -> vocabulary rows -> logits + running argmax
-  OP_NORM2 = 9,   // wide batch: 8 rows: RMSNorm(x) * FFN gain -> bf16
+  OP_NORM2 = 9,   // wide batch, one row: RMSNorm(x) * FFN gain -> bf16
   OP_LMFIN = 10,  // follow-up: the running argmax -> next token
   // mixture-of-experts FFN layer (data-dependent task graph, dynamic schedule)
   OP_ROUTE = 11,    // 8 tokens: router logits -> top-k, weights, per-expert ranks
@@ -42,7 +42,7 @@ enum Op : int32_t {
   OP_EDOWN = 14,    // GroupGEMM tile: an expert's down rows x its routed rows
   OP_COMBINE = 15,  // 8 tokens: weighted sum of their top-k expert outputs
   OP_MFIN = 16,     // follow-up: end of the layer
-  OP_NORMF = 17,    // wide batch: 8 rows: final residual, RMSNorm * final gain -> bf16
+  OP_NORMF = 17,    // wide batch, one row: final residual, RMSNorm * final gain -> bf16
   OP_COUNT = 18
 };
 
@@ -129,8 +129,8 @@ MK_HD int expr_eval(const int32_t* code, int pc, const ExprEnv& env) {
 enum EvId : int32_t {
   EV_IN = 0,     // [L+1]        layer input ready (element l+1 notified by layer l's down tiles)
   EV_QKV = 1,    // [L][Hkv]     Q/K/V rows of one kv-head group written
-  EV_CHUNK = 2,  // [L][maxB][Hkv] key-chunk partials of one (b, g) written
-  EV_ATTN = 3,   // [L]          all head groups merged
+  EV_CHUNK = 2,  // (unused: armed at one element of count zero)
+  EV_ATTN = 3,   // [L]          every attention task done (each pair merged by its last task)
   EV_O = 4,      // [L]          output projection done
   EV_GU = 5,     // [L][n_kc]    SwiGLU outputs of one K segment written
   EV_LM = 6,     // [1]          all LM tiles done
@@ -308,6 +308,9 @@ struct DevPlan {
   // tile's epilogue (the counters are zeroed at launch and by that task)
   int32_t gseg_qkv, gseg_o, gseg_gu, pad6;
   int64_t off_gpart, off_gctr;
+  // attention: per (sequence, kv head) count of finished tasks; the last of a
+  // pair's tasks merges their partials (zeroed at launch and by that task)
+  int64_t off_actr;
 };
 constexpr int kGctrPerOp = 64;  // split-K tile counters per GEMM op (tiles of 128 rows)
 

@@ -140,10 +140,11 @@ typedef struct mk_plan_opts {
   int fault;
   int fault_family;
   /* Key chunks (attn_chunk keys each) per attention task: 0 = default (32 for
-   * max_batch <= 8, 16 above), at most 64.  Compute warp w of the task takes
-   * chunks w, w + 8, ... (warp-MMA scores and P.V with an online softmax); the
-   * task leaves one partial for the merge, or, when it holds all of its
-   * (sequence, kv head)'s chunks, the finished output and no merge runs. */
+   * max_batch <= 8, 24 above), at most 64.  Compute warp w of the task takes
+   * chunks w, w + 8, ... (warp-MMA scores and P.V with an online softmax).  A
+   * task that holds all of its (sequence, kv head)'s chunks writes the finished
+   * output; otherwise it leaves one partial, and the last of the pair's tasks
+   * to finish merges the pair's partials. */
   int attn_split;
   /* MoE GroupGEMM tiles, chosen per expert from the run-time histogram
    * (0 = default: routing-aware; 1 = routing-aware; 2 = fixed): an expert
@@ -222,7 +223,7 @@ typedef struct mk_family_info {
 
 #define MK_OP_QKV 1
 #define MK_OP_ATTN 2
-#define MK_OP_MERGE 3
+#define MK_OP_MERGE 3     /* reserved: not scheduled (a pair's last attention task merges the pair) */
 #define MK_OP_OPROJ 4
 #define MK_OP_GATEUP 5
 #define MK_OP_DOWN 6
@@ -234,9 +235,9 @@ typedef struct mk_family_info {
 #define MK_OP_EDOWN 14    /* GroupGEMM tile: down rows of one expert x its routed rows */
 #define MK_OP_COMBINE 15  /* weighted sum of each token's top_k expert outputs (8 tokens per task) */
 #define MK_OP_MFIN 16     /* follow-up: end of the layer */
-#define MK_OP_NORM 7      /* wide batch, 8 rows: residual materialised, RMSNorm * attention gain -> bf16 */
-#define MK_OP_NORM2 9     /* wide batch, 8 rows: RMSNorm * FFN gain -> bf16 */
-#define MK_OP_NORMF 17    /* wide batch, 8 rows: final residual, RMSNorm * final gain -> bf16 */
+#define MK_OP_NORM 7      /* wide batch, one row: residual materialised, RMSNorm * attention gain -> bf16 */
+#define MK_OP_NORM2 9     /* wide batch, one row: RMSNorm * FFN gain -> bf16 */
+#define MK_OP_NORMF 17    /* wide batch, one row: final residual, RMSNorm * final gain -> bf16 */
 
 typedef struct mk_sim_report {
   int orders_run;         /* random interleavings executed */

@@ -14,9 +14,8 @@ Task families of one dense layer, in the order a layer runs them:
 * ``qkv``    — one per ``tile_qkv`` output rows of the stacked Q/K/V weights;
 * ``attn``   — one per (sequence b, kv head g, key chunk c),
   ``c < ceil((ctx_b + 1) / chunk)``;
-* ``merge``  — one per (b, g) whose chunks span more than one attention task:
-  combine that head group's partials (a pair with one task writes its output
-  itself, without a merge);
+  (the last attention task of a (b, g) to finish merges that pair's partials
+  itself: no task of its own);
 * ``oproj``  — one per ``tile_o`` rows of the output projection;
 * ``gateup`` — one per ``tile_gu`` rows of the gate (and the same rows of up);
 * ``down``   — one per (``tile_down`` rows, K segment of ``kseg`` columns).
@@ -56,7 +55,6 @@ def dense_family_extents(shape, B: int, ctx, tiles: dict) -> dict:
         **norms,
         "qkv": (Hq + 2 * Hkv) * D // tiles["tile_qkv"] * sq,
         "attn": Hkv * sum(nch),
-        "merge": Hkv * sum(1 for n in nch if n > 1),
         "oproj": H // tiles["tile_o"] * so,
         "gateup": shape.ffn // tiles["tile_gu"] * sg,
         "down": (H // tiles["tile_down"]) * (shape.ffn // tiles["kseg"]),
@@ -85,8 +83,6 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
             for g in range(Hkv):
                 for c in range(nch):
                     out.add(("attn", l, Hkv * base + g * nch + c))
-                if nch > 1:
-                    out.add(("merge", l, b * Hkv + g))
             base += nch
     for fam in ("lm", "lmfin") + (("normf",) if wide else ()):
         out.update((fam, -1, i) for i in range(ext[fam]))

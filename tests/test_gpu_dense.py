@@ -77,7 +77,7 @@ def test_tiny_static_equals_dynamic_bitwise(tiny):
     # END per CTA, and every push was popped
     want = ot.expected_dense_tasks(wl.TINY, 3, ctx, dyn.tiles_for_oracle())
     st = dyn.dec.stats()
-    pushed = sum(1 for f, _, _ in want if f not in ("merge", "lmfin")) + st["n_sm"]
+    pushed = sum(1 for f, _, _ in want if f != "lmfin") + st["n_sm"]
     assert st["last_queue_tasks"] == pushed and st["last_queue_pops"] == pushed
     assert 0 < st["last_queue_ranges"] <= st["queue_ranges_cap"] and st["launches"] == 1
 

@@ -508,10 +508,9 @@ def test_task_set_wide_layout_by_hand():
     # 128-row tiles, kseg 1024, split 8; B = 9 at contexts 0..8 except one at
     # 600 (ceil(601 / 64) = 10 chunks -> 2 tasks), the others 1 task each.
     # Per layer: norm 9 (one per row), qkv (4 + 4) * 64 / 128 = 4 tiles x 2
-    # K segments = 8, attn 2 * (8 + 2) = 20, merge 2 (only the sequence at
-    # 600 has more than one task per kv head; a pair with one task writes its
-    # output itself), oproj 2 x 2 = 4, norm2 9, gateup 8 x 2 = 16, down 2;
-    # then normf 9, lm 8, lmfin 1.
+    # K segments = 8, attn 2 * (8 + 2) = 20 (a pair's last task merges its
+    # partials: no merge tasks), oproj 2 x 2 = 4, norm2 9, gateup 8 x 2 = 16,
+    # down 2; then normf 9, lm 8, lmfin 1.
     tiles = dict(tile_qkv=128, chunk=64, tile_o=128, tile_gu=128, tile_down=128, kseg=1024, tile_lm=128,
                  split=8, wide=True, gseg=(2, 2, 2))
     ctx = [0, 1, 2, 3, 4, 5, 6, 7, 600]
@@ -521,11 +520,10 @@ def test_task_set_wide_layout_by_hand():
         fams[(f, l)] = fams.get((f, l), 0) + 1
     for l in range(2):
         assert {k[0]: v for k, v in fams.items() if k[1] == l} == {
-            "norm": 9, "qkv": 8, "attn": 20, "merge": 2, "oproj": 4, "norm2": 9, "gateup": 16, "down": 2}
+            "norm": 9, "qkv": 8, "attn": 20, "oproj": 4, "norm2": 9, "gateup": 16, "down": 2}
     assert fams[("normf", -1)] == 9 and fams[("lm", -1)] == 8 and fams[("lmfin", -1)] == 1
     # the last sequence's two tasks per kv head: Hkv * 8 + g * 2 + c
     assert {i for f, l, i in tasks if f == "attn" and l == 0 and i >= 16} == {16, 17, 18, 19}
-    assert {i for f, l, i in tasks if f == "merge" and l == 0} == {8 * 2 + 0, 8 * 2 + 1}  # b = 8, g = 0, 1
 
 
 def test_moe_tiles_and_task_set_by_hand():

@@ -38,10 +38,9 @@ def test_plan_build_and_tiles():
     assert t["tile_qkv"] == 32 and t["tile_o"] == 32 and t["tile_gu"] == 32 and t["tile_down"] == 64
     assert t["kseg"] == 2048 and t["tile_lm"] == 64 and t["chunk"] == 64 and t["n_sm"] == 148
     fams = d.families()
-    assert len(fams) == 16 * 6 + 2
-    assert [f.name.decode() for f in fams[:6]] == ["qkv.0", "attn.0", "merge.0", "oproj.0", "gateup.0",
-                                                   "down.0"]
-    assert sum(f.followup for f in fams) == 16 + 1
+    assert len(fams) == 16 * 5 + 2
+    assert [f.name.decode() for f in fams[:5]] == ["qkv.0", "attn.0", "oproj.0", "gateup.0", "down.0"]
+    assert sum(f.followup for f in fams) == 1  # (LMFIN; a pair's last attention task merges the pair)
 
 
 def test_plan_rejects_oversized_tiles():
@@ -175,7 +174,7 @@ def test_plan_option_ranges():
             _host(wl.LLAMA_1B, max_batch=16, max_ctx=1088, n_sm=148, **bad)
     # wide-batch defaults: 16 chunks per attention task, split K 4 / 4 / 2
     t = _host(wl.LLAMA_1B, max_batch=64, max_ctx=1088, n_sm=148).tiles()
-    assert (t["attn_split"], t["gseg_qkv"], t["gseg_o"], t["gseg_gu"], t["kseg"]) == (16, 4, 4, 2, 1024)
+    assert (t["attn_split"], t["gseg_qkv"], t["gseg_o"], t["gseg_gu"], t["kseg"]) == (24, 4, 4, 2, 1024)
 
 
 def test_moe_plan_requires_dynamic_schedule_and_rejects_dense_calls():
