@@ -112,10 +112,10 @@ def mk_plan_family_info(plan: int, f: int) -> mk_family_info:
 
 
 def mk_plan_tiles(plan: int) -> dict:
-    out = (C.c_int * 15)()
+    out = (C.c_int * 16)()
     _check(lib().mk_plan_tiles(plan, out))
     keys = ("tile_qkv", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm", "chunk", "n_sm", "ring_slots",
-            "attn_split", "wide", "act_split", "gseg_qkv", "gseg_o", "gseg_gu")
+            "attn_split", "wide", "act_split", "gseg_qkv", "gseg_o", "gseg_gu", "attn_auto")
     return dict(zip(keys, list(out)))
 
 

@@ -238,8 +238,8 @@ mk_status mk_plan_tiles(const mk_plan* hp, int* o) {
   g_err.clear();
   if (!hp || !o) return fail(MK_ERR_INVALID_ARG, "null argument");
   const mk::DevPlan& P = hp->p.dp;
-  int v[15] = {P.tile_qkv, P.tile_o, P.tile_gu, P.tile_down, P.kseg, P.tile_lm, P.chunk, P.n_sm, P.ring_slots,
-               P.attn_split, P.wide, P.act_split, P.gseg_qkv, P.gseg_o, P.gseg_gu};
+  int v[16] = {P.tile_qkv, P.tile_o, P.tile_gu, P.tile_down, P.kseg, P.tile_lm, P.chunk, P.n_sm, P.ring_slots,
+               P.attn_split, P.wide, P.act_split, P.gseg_qkv, P.gseg_o, P.gseg_gu, P.attn_auto};
   std::memcpy(o, v, sizeof(v));
   return MK_OK;
 }

@@ -156,6 +156,7 @@ struct Smem {
   float alsum[kComputeWarps][4], amax[kComputeWarps][4];  // attention: each warp's exp-sum and maximum per head
   int gemm_last;  // wide batch, split K: this CTA's task was the tile's last segment
   int attn_last;  // attention: this CTA's task was its (sequence, kv head)'s last to finish
+  int asplit;     // key chunks per attention task in this step (step_attn_split)
   // wide batch: this CTA's best argmax key per batch column, and what it published
   unsigned long long lm_cta[kMaxBatch], lm_pub[kMaxBatch];
   volatile int released;  // regular tasks the controller has handed to compute
@@ -585,12 +586,12 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
         }
       } break;
       case OP_ATTN: {
-        // the task's key chunks (attn_split of them at most), one slot each:
+        // the task's key chunks (the step's split of them at most), one slot each:
         // the chunk's 64 cache rows of K, then of V, as swizzled TMA boxes
         // (rows past max_ctx read as zeros; the task masks rows past ctx)
         AttnTask a = decode_attn(idx, S.B, P.n_kv_heads, sm.nch, sm.pre);
         const int p = sm.ctx[a.b];
-        const int c0 = a.c * P.attn_split, c1 = min(c0 + P.attn_split, ceil_div(p + 1, P.chunk));
+        const int c0 = a.c * sm.asplit, c1 = min(c0 + sm.asplit, ceil_div(p + 1, P.chunk));
         const int plane = (layer * P.n_slots + sm.slot[a.b]) * P.n_kv_heads + a.g;
         const unsigned char* gm = ws + P.off_tmap + (size_t)P.n_layers * kTmapPerLayer * kTmapBytes;
         for (int cc = c0; cc < c1; ++cc) {
@@ -1641,7 +1642,7 @@ __device__ __forceinline__ void merge_pair(const DevPlan& P, const Smem& sm, uns
 }
 
 // One task of split-KV decode attention for the qpg query heads of a GQA
-// group: up to attn_split consecutive 64-key chunks of one sequence, one ring
+// group: up to the step's split (sm.asplit) of consecutive 64-key chunks of one sequence, one ring
 // slot each (K rows, then V rows, as 128-byte-swizzled TMA boxes); compute
 // warp w takes chunks w, w + 8, ... of the task (flash-decoding partials:
 // unnormalised output, running maximum, exp-sum).  A (sequence, kv head)
@@ -1664,7 +1665,7 @@ __device__ __forceinline__ void task_attn(const DevPlan& P, const StepParams& S,
   constexpr int D = 64;  // head_dim (the plan builder accepts 64 only)
   const AttnTask a = decode_attn(d.idx, S.B, Hkv, sm.nch, sm.pre);
   const int p = sm.ctx[a.b];
-  const int c0 = a.c * P.attn_split, c1 = min(c0 + P.attn_split, ceil_div(p + 1, CH));
+  const int c0 = a.c * sm.asplit, c1 = min(c0 + sm.asplit, ceil_div(p + 1, CH));
   const int g = lane >> 2, q4 = lane & 3;
   const bool hv = g < qpg;  // this lane's MMA row is a head of the group
   float m_run = -INFINITY, l_run = 0.f;
@@ -2683,7 +2684,7 @@ __device__ __forceinline__ void arm_events(const DevPlan& P, Smem& sm, const Fam
                                         int* counters, int B) {
   const int tid = threadIdx.x;
   for (int f = tid; f < P.n_families; f += blockDim.x) {
-    ExprEnv env{B, sm.ctx, {0, 0, 0}};
+    ExprEnv env{B, sm.ctx, {0, 0, 0}, sm.asplit};
     sm.fam_ext[f] = expr_eval(code, fams[f].extent_expr, env);
     sm.fam_op[f] = (signed char)fams[f].op;
     sm.fam_layer[f] = (signed char)fams[f].layer;
@@ -2699,7 +2700,7 @@ __device__ __forceinline__ void arm_events(const DevPlan& P, Smem& sm, const Fam
     }
     if (e == EV_COUNT) continue;
     int lin = i - P.ev[e].base;
-    ExprEnv env{B, sm.ctx, {0, 0, 0}};
+    ExprEnv env{B, sm.ctx, {0, 0, 0}, sm.asplit};
     for (int dd = P.ev[e].ndim - 1; dd >= 0; --dd) { env.coord[dd] = lin % P.ev[e].dims[dd]; lin /= P.ev[e].dims[dd]; }
     counters[i] = expr_eval(code, P.ev[e].count_expr, env) + (i == P.fault_ctr ? 1 : 0);
   }
@@ -2769,11 +2770,12 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
       set_geo(OP_DOWN, P.kseg, P.tile_down, 0);
       set_geo(OP_LM, P.hidden, P.tile_lm, 0);
     }
+    sm.asplit = moe ? P.attn_split : step_attn_split(P, B, sm.ctx);
     if (!moe) {
       int run = 0;
-      for (int b = 0; b < B; ++b) {  // attention tasks of sequence b: its key chunks, attn_split at a time
+      for (int b = 0; b < B; ++b) {  // attention tasks of sequence b: its key chunks, asplit at a time
         sm.pre[b] = run;
-        sm.nch[b] = ceil_div(ceil_div(sm.ctx[b] + 1, P.chunk), P.attn_split);
+        sm.nch[b] = ceil_div(ceil_div(sm.ctx[b] + 1, P.chunk), sm.asplit);
         run += sm.nch[b];
       }
       sm.pre[B] = run;

@@ -115,12 +115,12 @@ int Plan::counter(int ev, int c0, int c1, int c2) const {
 }
 
 int Plan::event_count(int ev, int c0, int c1, int c2, const Binding& bd) const {
-  ExprEnv env{bd.B, bd.ctx.data(), {c0, c1, c2}};
+  ExprEnv env{bd.B, bd.ctx.data(), {c0, c1, c2}, step_attn_split(dp, bd.B, bd.ctx.data())};
   return expr_eval(code.data(), dp.ev[ev].count_expr, env);
 }
 
 int Plan::family_extent(int f, const Binding& bd) const {
-  ExprEnv env{bd.B, bd.ctx.data(), {0, 0, 0}};
+  ExprEnv env{bd.B, bd.ctx.data(), {0, 0, 0}, step_attn_split(dp, bd.B, bd.ctx.data())};
   return expr_eval(code.data(), fams[f].extent_expr, env);
 }
 
@@ -150,7 +150,8 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
     nr = std::min(tm, rt->hist[e] - m * tm);
   };
   const bool wide = P.wide != 0;
-  auto nsplit = [&](int b) { return ceil_div(ceil_div(bd.ctx[b] + 1, P.chunk), P.attn_split); };
+  const int asplit = step_attn_split(P, bd.B, bd.ctx.data());  // key chunks per attention task this step
+  auto nsplit = [&](int b) { return ceil_div(ceil_div(bd.ctx[b] + 1, P.chunk), asplit); };
   if (wide && op == OP_QKV) {
     // a 128-row tile of [Wq; Wk; Wv]: two heads of q, k or v rows (every K
     // segment's task is modelled as writing the tile's outputs)
@@ -221,7 +222,7 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       }
     } break;
     case OP_ATTN: {
-      // task c of (b, g): key chunks c * attn_split .. of the sequence
+      // task c of (b, g): key chunks c * asplit .. of the sequence
       std::vector<int> nsp(B), pre(B + 1, 0);
       for (int b = 0; b < B; ++b) { nsp[b] = nsplit(b); pre[b + 1] = pre[b] + nsp[b]; }
       AttnTask a = decode_attn(idx, B, Hkv, nsp.data(), pre.data());
@@ -234,7 +235,7 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       const bool single = nsp[a.b] == 1;
       long long qb = a.b * QD + (long long)a.g * qpg * D;
       t.reads.push_back({BUF_Q, qb, qb + (long long)qpg * D});
-      int p0 = a.c * P.attn_split * P.chunk, p1 = std::min(p0 + P.attn_split * P.chunk, bd.ctx[a.b] + 1);
+      int p0 = a.c * asplit * P.chunk, p1 = std::min(p0 + asplit * P.chunk, bd.ctx[a.b] + 1);
       long long kb = kv_row(l, a.b, a.g, p0);
       t.reads.push_back({BUF_KC, kb, kb + (long long)(p1 - p0) * D});
       t.reads.push_back({BUF_VC, kb, kb + (long long)(p1 - p0) * D});
@@ -427,8 +428,9 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
       break;
     case EV_QKV: {
       int pre = 0;
+      const int asplit = step_attn_split(dp, bd.B, bd.ctx.data());
       for (int b = 0; b < bd.B; ++b) {
-        const int ns = ceil_div(ceil_div(bd.ctx[b] + 1, dp.chunk), dp.attn_split);
+        const int ns = ceil_div(ceil_div(bd.ctx[b] + 1, dp.chunk), asplit);
         if (wide) add(fam_index(OP_ATTN, c[0]), dp.n_kv_heads * pre, dp.n_kv_heads * ns);  // every kv head
         else add(fam_index(OP_ATTN, c[0]), dp.n_kv_heads * pre + c[1] * ns, ns);
         pre += ns;
@@ -645,12 +647,15 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   P.chunk = o->attn_chunk ? o->attn_chunk : 64;
   P.slot_bytes = 16384;
   P.wide = wide ? 1 : 0;
-  // key chunks per attention task: small batches take a sequence's chunks
-  // (up to 2048 keys) in one task, which then also skips the merge; wide
+  // key chunks per attention task: an option value is used as given; small
+  // batches (below) follow each step, at most 32 chunks (2048 keys); wide
   // batches 24 (three per warp: a warp's next chunk loads while one is
   // computed; of 8, 16, 24 and 32, 16 was fastest at B = 16, 32 at B = 32 and
   // 24 at B = 64, 24 the best over the three)
   P.attn_split = o->attn_split ? o->attn_split : (wide ? 24 : 32);
+  // up to 8 rows with no split given, the split follows each step's B and
+  // contexts (step_attn_split: 3 to 16 chunks on the 1B shape at B = 1..8)
+  P.attn_auto = (!o->attn_split && !wide) ? 1 : 0;
   if (P.attn_split < 1 || P.attn_split > 64) { err = "attn_split must be in [1, 64]"; return MK_ERR_INVALID_ARG; }
   if (wide) {
     // tcgen05 GEMM tasks: kWideRows weight rows each (the MMA's M), every
@@ -731,7 +736,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     p.fams.push_back(f);
     p.fam_names.push_back(std::string(kOpNames[op]) + (layer >= 0 ? "." + std::to_string(layer) : ""));
   };
-  // ATTN extent: Hkv * sum_b ceil((ctx_b + 1) / chunk)
+  // ATTN extent: Hkv * sum_b ceil(ceil((ctx_b + 1) / chunk) / asplit), asplit the step's split
   int e_attn;
   {
     Emit e(p.code);
@@ -743,7 +748,7 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
     p.code.push_back(X_VAR); p.code.push_back(X_CTX_AT);
     p.code.push_back(X_PUSH); p.code.push_back(1); p.code.push_back(X_ADD);
     p.code.push_back(X_PUSH); p.code.push_back(P.chunk); p.code.push_back(X_CEILDIV);
-    p.code.push_back(X_PUSH); p.code.push_back(P.attn_split); p.code.push_back(X_CEILDIV);
+    p.code.push_back(X_ASPLIT); p.code.push_back(X_CEILDIV);
     p.code.push_back(X_RET);
     p.code[len_at] = (int)(p.code.size() - body);
     p.code.push_back(X_MUL);
@@ -770,7 +775,8 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
                                        OP_EDOWN, OP_COMBINE};
   const int fam_per_layer = mdec ? (wide ? 9 : 8) : wide ? 7 : kFamPerLayer;
   const int* layer_ops = mdec ? (wide ? kMoeDecWideOps : kMoeDecOps) : wide ? kWideOps : kLayerOps;
-  const int max_tasks_attn = Hkv * P.max_batch * ceil_div(P.max_chunks, P.attn_split);
+  const int min_split = P.attn_auto ? std::min(kAttnSplitMin, P.attn_split) : P.attn_split;
+  const int max_tasks_attn = Hkv * P.max_batch * ceil_div(P.max_chunks, min_split);
   for (int l = 0; l < P.n_layers; ++l) {
     if (wide) add_family(OP_NORM, l, e_tok1, P.max_batch, 0);
     add_family(OP_QKV, l, emit_const(p.code, P.n_qkv_tiles), P.n_qkv_tiles, 0);

@@ -62,12 +62,14 @@ enum XOp : int32_t {
   X_MIN = 10, X_MAX = 11,
   X_LT = 12,      // pop b, a; push a < b
   X_SUM_B = 13,   // operand len; body of len words follows
+  X_ASPLIT = 14,  // the step's key chunks per attention task (step_attn_split)
 };
 
 struct ExprEnv {
   int B;
   const int* ctx;   // [B]
   int coord[3];
+  int asplit;       // key chunks per attention task in this step
 };
 
 MK_HD int expr_flat(const int32_t* code, int pc, const ExprEnv& env, int var) {
@@ -82,6 +84,7 @@ MK_HD int expr_flat(const int32_t* code, int pc, const ExprEnv& env, int var) {
       case X_COORD: st[sp++] = env.coord[code[pc++]]; break;
       case X_CTX_AT: { int i = st[sp - 1]; st[sp - 1] = (i >= 0 && i < env.B) ? env.ctx[i] : 0; } break;
       case X_VAR: st[sp++] = var; break;
+      case X_ASPLIT: st[sp++] = env.asplit; break;
       case X_ADD: sp--; st[sp - 1] = st[sp - 1] + st[sp]; break;
       case X_SUB: sp--; st[sp - 1] = st[sp - 1] - st[sp]; break;
       case X_MUL: sp--; st[sp - 1] = st[sp - 1] * st[sp]; break;
@@ -105,6 +108,7 @@ MK_HD int expr_eval(const int32_t* code, int pc, const ExprEnv& env) {
       case X_B: st[sp++] = env.B; break;
       case X_COORD: st[sp++] = env.coord[code[pc++]]; break;
       case X_CTX_AT: { int i = st[sp - 1]; st[sp - 1] = (i >= 0 && i < env.B) ? env.ctx[i] : 0; } break;
+      case X_ASPLIT: st[sp++] = env.asplit; break;
       case X_ADD: sp--; st[sp - 1] = st[sp - 1] + st[sp]; break;
       case X_SUB: sp--; st[sp - 1] = st[sp - 1] - st[sp]; break;
       case X_MUL: sp--; st[sp - 1] = st[sp - 1] * st[sp]; break;
@@ -297,7 +301,7 @@ struct DevPlan {
   int32_t pad5;
   // wide batch: tcgen05 GEMM tasks on materialised bf16 activations
   int32_t wide;       // 1: max_batch > kMaxBatchRows
-  int32_t attn_split; // key chunks per attention task
+  int32_t attn_split; // key chunks per attention task (adaptive plans: at most; see step_attn_split)
   int32_t act_rows;   // batch rows of the activation buffers (max_batch rounded up to 16)
   int32_t act_split;  // 1: each activation row stored as its bf16 value and its bf16 remainder (see act_buf_row)
   int64_t off_xn, off_attn_bf, off_h_bf;  // bf16 [max_batch][H], [max_batch][H], [max_batch][F]
@@ -306,7 +310,8 @@ struct DevPlan {
   // off_gpart and counts in at the tile's counter (off_gctr, [3][64]); the
   // last to count in sums the partials in segment order and runs the
   // tile's epilogue (the counters are zeroed at launch and by that task)
-  int32_t gseg_qkv, gseg_o, gseg_gu, pad6;
+  int32_t gseg_qkv, gseg_o, gseg_gu;
+  int32_t attn_auto;  // 1: the attention split follows each step's B and contexts (step_attn_split)
   int64_t off_gpart, off_gctr;
   // attention: per (sequence, kv head) count of finished tasks; the last of a
   // pair's tasks merges their partials (zeroed at launch and by that task)
@@ -371,5 +376,24 @@ MK_HD AttnTask decode_attn(int i, int B, int Hkv, const int* nch, const int* pre
 }
 
 MK_HD int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Key chunks per attention task in one step.  A plan with a fixed split
+// (attn_auto = 0) returns attn_split.  An adaptive plan cuts the step's
+// C = Hkv * sum_b ceil((ctx_b + 1) / chunk) chunk units into about two thirds
+// of n_sm tasks: s = ceil(C / ceil(2 n_sm / 3)), clamped to
+// [min(kAttnSplitMin, attn_split), attn_split].  (Measured on the 1B shape at
+// B = 1..8: fewer, longer tasks leave SMs idle; more tasks than that pay a
+// second wave and more merging; below 3 chunks a task's fixed costs dominate.)
+constexpr int kAttnSplitMin = 3;
+MK_HD int step_attn_split(const DevPlan& P, int B, const int* ctx) {
+  if (!P.attn_auto) return P.attn_split;
+  long long c = 0;
+  for (int b = 0; b < B; ++b) c += ceil_div(ctx[b] + 1, P.chunk);
+  c *= P.n_kv_heads;
+  const long long target = ceil_div(2 * P.n_sm, 3);
+  const long long s = (c + target - 1) / target;
+  const int lo = P.attn_split < kAttnSplitMin ? P.attn_split : kAttnSplitMin;
+  return s < lo ? lo : s > P.attn_split ? P.attn_split : (int)s;
+}
 
 }  // namespace mk

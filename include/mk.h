@@ -139,12 +139,16 @@ typedef struct mk_plan_opts {
    * other values are refused with MK_ERR_INVALID_ARG. */
   int fault;
   int fault_family;
-  /* Key chunks (attn_chunk keys each) per attention task: 0 = default (32 for
-   * max_batch <= 8, 24 above), at most 64.  Compute warp w of the task takes
-   * chunks w, w + 8, ... (warp-MMA scores and P.V with an online softmax).  A
-   * task that holds all of its (sequence, kv head)'s chunks writes the finished
-   * output; otherwise it leaves one partial, and the last of the pair's tasks
-   * to finish merges the pair's partials. */
+  /* Key chunks (attn_chunk keys each) per attention task, at most 64.  A
+   * value > 0 is used as given.  0 = default: 24 for max_batch > 8; for
+   * max_batch <= 8 the split follows each step: with C = n_kv_heads *
+   * sum_b ceil((ctx_b + 1) / attn_chunk) chunk units and T = ceil(2 n_sm / 3),
+   * split = ceil(C / T) clamped to [3, 32] (about two thirds of the SMs'
+   * worth of tasks).  Compute warp w of a task takes chunks w, w + 8, ...
+   * (warp-MMA scores and P.V with an online softmax).  A task that holds all
+   * of its (sequence, kv head)'s chunks writes the finished output; otherwise
+   * it leaves one partial, and the last of the pair's tasks to finish merges
+   * the pair's partials. */
   int attn_split;
   /* MoE GroupGEMM tiles, chosen per expert from the run-time histogram
    * (0 = default: routing-aware; 1 = routing-aware; 2 = fixed): an expert
@@ -373,12 +377,14 @@ mk_status mk_plan_family_info(const mk_plan* p, int family, mk_family_info* out)
  * exactly its number of notifies.  MK_ERR_INVALID_ARG for null arguments. */
 mk_status mk_plan_counter_region(const mk_plan* p, long long* byte_offset, int* n_counters);
 
-/* Tile sizes the plan chose, written to out[15] in this order: tile_qkv,
+/* Tile sizes the plan chose, written to out[16] in this order: tile_qkv,
  * tile_o, tile_gu, tile_down, kseg, tile_lm, attn_chunk, n_sm, ring_slots,
- * attn_split (key chunks per attention task), wide (1: the wide-batch path),
- * act_split (1: wide-batch activations as value + remainder rows), and the
- * K segments per tile of the QKV, O-projection and gate/up GEMM tasks (wide
- * batch: a tile's segments run as separate tasks; 1 otherwise). */
+ * attn_split (key chunks per attention task; with attn_auto, at most),
+ * wide (1: the wide-batch path), act_split (1: wide-batch activations as
+ * value + remainder rows), the K segments per tile of the QKV, O-projection
+ * and gate/up GEMM tasks (wide batch: a tile's segments run as separate
+ * tasks; 1 otherwise), and attn_auto (1: the split follows each step, see
+ * mk_plan_opts.attn_split). */
 mk_status mk_plan_tiles(const mk_plan* p, int* out);
 
 /* Host validation for one binding of the symbols (B, ctx_lens host array):

@@ -25,7 +25,11 @@ After the last layer: ``lm`` (``tile_lm`` vocabulary rows each) and
 
 An attention task may take ``split`` consecutive key chunks (``tiles["split"]``,
 default 1): sequence b then has ``nch_b = ceil(ceil((ctx_b + 1) / chunk) /
-split)`` attention tasks per kv head.  Linear index of an ``attn`` task:
+split)`` attention tasks per kv head.  With ``tiles["split_auto"]`` the split
+is chosen per step (``step_split``): the step's chunk units
+``C = Hkv * sum_b ceil((ctx_b + 1) / chunk)`` over about two thirds of
+``tiles["n_sm"]`` tasks, ``ceil(C / ceil(2 n_sm / 3))``, kept between
+``min(3, split)`` and ``split``.  Linear index of an ``attn`` task:
 ``Hkv * sum_{b'<b} nch_{b'} + g * nch_b + c``.  ``down`` tasks are numbered
 K-segment-major: ``kc * (H / tile_down) + n``.
 
@@ -43,11 +47,22 @@ def _ceil(a: int, b: int) -> int:
     return -(-a // b)
 
 
+def step_split(shape, B: int, ctx, tiles: dict) -> int:
+    """Key chunks per attention task in a step with these contexts."""
+    split = tiles.get("split", 1)
+    if not tiles.get("split_auto"):
+        return split
+    units = shape.n_kv_heads * sum(_ceil(int(ctx[b]) + 1, tiles["chunk"]) for b in range(B))
+    target = _ceil(2 * tiles["n_sm"], 3)
+    return max(min(3, split), min(split, _ceil(units, target)))
+
+
 def dense_family_extents(shape, B: int, ctx, tiles: dict) -> dict:
     """Number of tasks of each family in one layer (and after the last)."""
     H, D = shape.hidden, shape.head_dim
     Hq, Hkv = shape.n_q_heads, shape.n_kv_heads
-    nch = [_ceil(_ceil(int(ctx[b]) + 1, tiles["chunk"]), tiles.get("split", 1)) for b in range(B)]
+    split = step_split(shape, B, ctx, tiles)
+    nch = [_ceil(_ceil(int(ctx[b]) + 1, tiles["chunk"]), split) for b in range(B)]
     n_lm = _ceil(shape.vocab, tiles["tile_lm"])
     norms = {"norm": B, "norm2": B, "normf": B} if tiles.get("wide") else {}
     sq, so, sg = tiles.get("gseg", (1, 1, 1))  # K segments per tile, each its own task
@@ -73,13 +88,14 @@ def expected_dense_tasks(shape, B: int, ctx, tiles: dict) -> set:
     ext = dense_family_extents(shape, B, ctx, tiles)
     Hkv = shape.n_kv_heads
     wide = bool(tiles.get("wide"))
+    split = step_split(shape, B, ctx, tiles)
     out = set()
     for l in range(shape.n_layers):
         for fam in ("qkv", "oproj", "gateup", "down") + (("norm", "norm2") if wide else ()):
             out.update((fam, l, i) for i in range(ext[fam]))
         base = 0
         for b in range(B):
-            nch = _ceil(_ceil(int(ctx[b]) + 1, tiles["chunk"]), tiles.get("split", 1))
+            nch = _ceil(_ceil(int(ctx[b]) + 1, tiles["chunk"]), split)
             for g in range(Hkv):
                 for c in range(nch):
                     out.add(("attn", l, Hkv * base + g * nch + c))

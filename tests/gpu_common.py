@@ -50,7 +50,8 @@ class DenseCase:
         t = self.dec.tiles()
         return dict(tile_qkv=t["tile_qkv"], chunk=t["chunk"], tile_o=t["tile_o"], tile_gu=t["tile_gu"],
                     tile_down=t["tile_down"], kseg=t["kseg"], tile_lm=t["tile_lm"], split=t["attn_split"],
-                    wide=bool(t["wide"]), gseg=(t["gseg_qkv"], t["gseg_o"], t["gseg_gu"]))
+                    split_auto=bool(t["attn_auto"]), n_sm=t["n_sm"], wide=bool(t["wide"]),
+                    gseg=(t["gseg_qkv"], t["gseg_o"], t["gseg_gu"]))
 
     def gpu_step(self, tokens, slots, ctx, with_logits=True, counts=True, capture=False):
         """One step through mk_decode_step; with ``capture`` also the residual

@@ -494,6 +494,27 @@ def test_task_counts_golden():
     assert len(tasks) == rows["total"]
 
 
+def test_step_split_by_hand():
+    # the per-step attention split on the 1B shape (8 kv heads, 64-key
+    # chunks) with 148 SMs: T = ceil(2 * 148 / 3) = 99 tasks
+    tiles = dict(chunk=64, split=32, split_auto=True, n_sm=148)
+    s = wl.LLAMA_1B
+    # B=1 at 1024: 8 * ceil(1025 / 64) = 8 * 17 = 136 units, ceil(136 / 99) = 2, floor 3
+    assert ot.step_split(s, 1, [1024], tiles) == 3
+    # chunks 11, 39, 33, 4: 8 * 87 = 696 units, ceil(696 / 99) = 8 (7 * 99 = 693)
+    assert ot.step_split(s, 4, [696, 2450, 2106, 216], tiles) == 8
+    # chunks 11, 39, 33, 4, 21, 59, 7, 15: 8 * 189 = 1512, ceil(1512 / 99) = 16 (15 * 99 = 1485)
+    assert ot.step_split(s, 8, [696, 2450, 2106, 216, 1316, 3764, 443, 949], tiles) == 16
+    # 8 * 8 * 64 = 4096 units, ceil(4096 / 99) = 42, capped at 32
+    assert ot.step_split(s, 8, [4095] * 8, tiles) == 32
+    # a cap below the floor of 3 wins; without split_auto the split is fixed
+    assert ot.step_split(s, 1, [1024], dict(tiles, split=2)) == 2
+    assert ot.step_split(s, 8, [4095] * 8, dict(tiles, split_auto=False)) == 32
+    # the task set follows: B=1 at 1024 with split 3 has ceil(17 / 3) = 6 tasks per kv head
+    ext = ot.dense_family_extents(s, 1, [1024], dict(TILES_TINY, **tiles))
+    assert ext["attn"] == 8 * 6
+
+
 def test_task_set_brute_force_attn_numbering():
     ctx = [0, 63, 64, 200]
     tasks = ot.expected_dense_tasks(wl.TINY, 4, ctx, TILES_TINY)

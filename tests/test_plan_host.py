@@ -96,8 +96,29 @@ def test_simulator_clean(sched, B, ctx):
     t = d.tiles()
     tiles = {k: t[k] for k in ("tile_qkv", "chunk", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm")}
     assert tiles == dict(tile_qkv=32, chunk=64, tile_o=32, tile_gu=32, tile_down=64, kseg=1024, tile_lm=64)
-    assert t["attn_split"] == 32  # a sequence's chunks up to 2048 keys in one attention task (no merge)
-    assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, dict(tiles, split=32)))
+    assert t["attn_split"] == 32 and t["attn_auto"] == 1  # the split follows the step, at most 2048 keys
+    want = ot.expected_dense_tasks(wl.TINY, B, ctx, dict(tiles, split=32, split_auto=True, n_sm=t["n_sm"]))
+    assert rep.tasks_per_order == len(want)
+
+
+@pytest.mark.parametrize("B,ctx,split", [(1, [1024], 3), (2, [300, 250], 3), (3, [600, 900, 200], 10),
+                                         (4, [696, 2450, 2106, 216], 29), (8, [4095] * 8, 32)])
+def test_simulator_adaptive_attention_split(B, ctx, split):
+    # the lowered plan's tasks for a step (the per-step split evaluated in the
+    # plan's expressions and task model) against the oracle's task set, over
+    # splits from the floor of 3 to the cap of 32, with multi-task pairs: the
+    # 1B shape on 148 SMs at B=1 (T = 99), the tiny shape on 8 SMs (T = 6)
+    shape, n_sm = (wl.LLAMA_1B, 148) if B == 1 else (wl.TINY, 8)
+    d = _host(shape, max_batch=8, max_ctx=4160, n_sm=n_sm)
+    mk.mk_plan_validate(d.plan, B, ctx)
+    code, rep = mk.mk_plan_simulate(d.plan, B, ctx, n_orders=1, seed=3)
+    assert code == 0 and rep.races == 0 and rep.nonzero_counters == 0, rep.first_error
+    t = d.tiles()
+    tiles = {k: t[k] for k in ("tile_qkv", "chunk", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm", "n_sm")}
+    assert ot.step_split(shape, B, ctx, dict(tiles, split=t["attn_split"], split_auto=True)) == split
+    want = ot.expected_dense_tasks(shape, B, ctx, dict(tiles, split=t["attn_split"], split_auto=True))
+    assert rep.tasks_per_order == len(want)
+    d.close()
 
 
 def test_simulator_many_orders():
@@ -172,9 +193,14 @@ def test_plan_option_ranges():
     for bad in (dict(attn_split=65), dict(attn_split=-1), dict(act_split=3)):
         with pytest.raises(mk.MkError):
             _host(wl.LLAMA_1B, max_batch=16, max_ctx=1088, n_sm=148, **bad)
-    # wide-batch defaults: 16 chunks per attention task, split K 4 / 4 / 2
+    # a given split is fixed; no split up to 8 rows: adaptive, at most 32
+    assert _host(wl.LLAMA_1B, max_batch=4, max_ctx=4160, n_sm=148, attn_split=8).tiles()["attn_auto"] == 0
+    t = _host(wl.LLAMA_1B, max_batch=8, max_ctx=4160, n_sm=148).tiles()
+    assert (t["attn_split"], t["attn_auto"]) == (32, 1)
+    # wide-batch defaults: 24 chunks per attention task (fixed), split K 4 / 4 / 2
     t = _host(wl.LLAMA_1B, max_batch=64, max_ctx=1088, n_sm=148).tiles()
-    assert (t["attn_split"], t["gseg_qkv"], t["gseg_o"], t["gseg_gu"], t["kseg"]) == (24, 4, 4, 2, 1024)
+    assert (t["attn_split"], t["attn_auto"], t["gseg_qkv"], t["gseg_o"], t["gseg_gu"], t["kseg"]) == \
+        (24, 0, 4, 4, 2, 1024)
 
 
 def test_moe_plan_requires_dynamic_schedule_and_rejects_dense_calls():
