@@ -424,6 +424,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
   bool ok = true;
   ProdFam f;
   f.fam = -2;
+  const uint64_t wpol = l2_evict_first_policy();  // weight streams: first out of L2
 
   // acquire the next ring slot: wait until the compute warps released it
   auto next_slot = [&](int fam, int idx, unsigned char*& dst, uint64_t*& bar) -> bool {
@@ -448,11 +449,11 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
       mbar_arrive_expect_tx(bar, tm1 ? 2 * part_bytes : part_bytes);
       if (cw >= 64) {  // swizzled [rows][cw / 64][64] boxes
         const int xc = (x0 + j * cw) >> 6;
-        tma_load_3d(dst, tm0, 0, xc, y0, bar);
-        if (tm1) tma_load_3d(dst + part_bytes, tm1, 0, xc, y1, bar);
+        tma_load_3d_hint(dst, tm0, 0, xc, y0, bar, wpol);
+        if (tm1) tma_load_3d_hint(dst + part_bytes, tm1, 0, xc, y1, bar, wpol);
       } else {
-        tma_load_2d(dst, tm0, x0 + j * cw, y0, bar);
-        if (tm1) tma_load_2d(dst + part_bytes, tm1, x0 + j * cw, y1, bar);
+        tma_load_2d_hint(dst, tm0, x0 + j * cw, y0, bar, wpol);
+        if (tm1) tma_load_2d_hint(dst + part_bytes, tm1, x0 + j * cw, y1, bar, wpol);
       }
     }
     return true;
@@ -507,7 +508,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
           uint64_t* bar;
           if (!next_slot(fam, idx, dst, bar)) return false;
           mbar_arrive_expect_tx(bar, (uint32_t)kWideRows * 128u);
-          tma_load_2d(dst, part ? f.tm[1] : m0, x0 + c * 64, row, bar);
+          tma_load_2d_hint(dst, part ? f.tm[1] : m0, x0 + c * 64, row, bar, wpol);
         }
       emitted++;
       return true;
@@ -578,7 +579,7 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
           for (int part = 0; part < (gu ? 2 : 1); ++part) {
             if (!next_slot(fam, idx, dst, bar)) return false;
             mbar_arrive_expect_tx(bar, 128u * 128u);
-            tma_load_2d(dst, f.tm[part], c * 64, wrow, bar);
+            tma_load_2d_hint(dst, f.tm[part], c * 64, wrow, bar, wpol);
           }
           if (!next_slot(fam, idx, dst, bar)) return false;
           mbar_arrive_expect_tx(bar, bbytes);
