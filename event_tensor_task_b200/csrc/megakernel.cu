@@ -61,6 +61,7 @@ constexpr int kMaxB = kMaxBatchRows;  // batch rows per step on this path
 constexpr int kMaxBlk = 8;    // 256-column blocks of a row (K <= 2048)
 constexpr int kMaxKc = 8;     // down-projection K segments (ffn / kseg <= 8192 / 1024)
 constexpr int kDynLookahead = 2;
+constexpr long long kKvL2Bytes = 64ll << 20;  // half of the 126 MB L2 (see Smem::kv_ef)
 
 // Kernel instances: the plan kinds (MK_MODEL_*) and the wide-batch layouts
 // (max_batch > 8) of the dense and the MoE decoder, each with only the code
@@ -157,6 +158,7 @@ struct Smem {
   int gemm_last;  // wide batch, split K: this CTA's task was the tile's last segment
   int attn_last;  // attention: this CTA's task was its (sequence, kv head)'s last to finish
   int asplit;     // key chunks per attention task in this step (step_attn_split)
+  int kv_ef;      // this step's K/V reads exceed half of L2: load them evict-first too
   // wide batch: this CTA's best argmax key per batch column, and what it published
   unsigned long long lm_cta[kMaxBatch], lm_pub[kMaxBatch];
   volatile int released;  // regular tasks the controller has handed to compute
@@ -600,8 +602,14 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
           uint64_t* bar;
           if (!next_slot(fam, idx, dst, bar)) return false;
           mbar_arrive_expect_tx(bar, 2u * (uint32_t)P.chunk * 128u);
-          tma_load_3d(dst, gm + (size_t)TMG_KC * kTmapBytes, 0, cc * P.chunk, plane, bar);
-          tma_load_3d(dst + (size_t)P.chunk * 128, gm + (size_t)TMG_VC * kTmapBytes, 0, cc * P.chunk, plane, bar);
+          if (sm.kv_ef) {
+            tma_load_3d_hint(dst, gm + (size_t)TMG_KC * kTmapBytes, 0, cc * P.chunk, plane, bar, wpol);
+            tma_load_3d_hint(dst + (size_t)P.chunk * 128, gm + (size_t)TMG_VC * kTmapBytes, 0, cc * P.chunk, plane,
+                             bar, wpol);
+          } else {
+            tma_load_3d(dst, gm + (size_t)TMG_KC * kTmapBytes, 0, cc * P.chunk, plane, bar);
+            tma_load_3d(dst + (size_t)P.chunk * 128, gm + (size_t)TMG_VC * kTmapBytes, 0, cc * P.chunk, plane, bar);
+          }
         }
       } break;
       default: break;
@@ -2772,6 +2780,11 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const DevPlan P, const
       set_geo(OP_LM, P.hidden, P.tile_lm, 0);
     }
     sm.asplit = moe ? P.attn_split : step_attn_split(P, B, sm.ctx);
+    // K/V the step reads; below half of L2 it is kept at normal priority, so
+    // that it stays in L2 from one step to the next
+    long long kv = 0;
+    for (int b = 0; !moe && b < B; ++b) kv += sm.ctx[b] + 1;
+    sm.kv_ef = kv * P.n_layers * P.n_kv_heads * P.head_dim * 4 > kKvL2Bytes;
     if (!moe) {
       int run = 0;
       for (int b = 0; b < B; ++b) {  // attention tasks of sequence b: its key chunks, asplit at a time
