@@ -96,6 +96,14 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+// The default L2 priority as an explicit policy (for loads that take their
+// policy as an operand).
+__device__ __forceinline__ uint64_t l2_evict_normal_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // tma_load_2d with an L2 cache policy (l2_evict_first_policy) for the lines it reads.
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, int x, int y, uint64_t* bar,
                                                  uint64_t pol) {

@@ -427,6 +427,8 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
   ProdFam f;
   f.fam = -2;
   const uint64_t wpol = l2_evict_first_policy();  // weight streams: first out of L2
+  // K/V chunks: evict-first too when the step's K/V would not stay in L2 anyway
+  const uint64_t kvpol = sm.kv_ef ? wpol : l2_evict_normal_policy();
 
   // acquire the next ring slot: wait until the compute warps released it
   auto next_slot = [&](int fam, int idx, unsigned char*& dst, uint64_t*& bar) -> bool {
@@ -602,14 +604,9 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
           uint64_t* bar;
           if (!next_slot(fam, idx, dst, bar)) return false;
           mbar_arrive_expect_tx(bar, 2u * (uint32_t)P.chunk * 128u);
-          if (sm.kv_ef) {
-            tma_load_3d_hint(dst, gm + (size_t)TMG_KC * kTmapBytes, 0, cc * P.chunk, plane, bar, wpol);
-            tma_load_3d_hint(dst + (size_t)P.chunk * 128, gm + (size_t)TMG_VC * kTmapBytes, 0, cc * P.chunk, plane,
-                             bar, wpol);
-          } else {
-            tma_load_3d(dst, gm + (size_t)TMG_KC * kTmapBytes, 0, cc * P.chunk, plane, bar);
-            tma_load_3d(dst + (size_t)P.chunk * 128, gm + (size_t)TMG_VC * kTmapBytes, 0, cc * P.chunk, plane, bar);
-          }
+          tma_load_3d_hint(dst, gm + (size_t)TMG_KC * kTmapBytes, 0, cc * P.chunk, plane, bar, kvpol);
+          tma_load_3d_hint(dst + (size_t)P.chunk * 128, gm + (size_t)TMG_VC * kTmapBytes, 0, cc * P.chunk, plane, bar,
+                           kvpol);
         }
       } break;
       default: break;
