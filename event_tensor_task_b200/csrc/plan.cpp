@@ -153,16 +153,19 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
   const int asplit = step_attn_split(P, bd.B, bd.ctx.data());  // key chunks per attention task this step
   auto nsplit = [&](int b) { return ceil_div(ceil_div(bd.ctx[b] + 1, P.chunk), asplit); };
   if (wide && op == OP_QKV) {
-    // a 128-row tile of [Wq; Wk; Wv]: two heads of q, k or v rows (every K
-    // segment's task is modelled as writing the tile's outputs)
+    // a 128-row tile of [Wq; Wk; Wv]: two heads of q, k or v rows.  Of a
+    // tile's K-segment tasks, the last to finish runs the epilogue (a counter
+    // inside the tasks orders them, not an event): segment 0 stands for it
+    // here and writes the tile's outputs, the others only read their inputs
     const int nq = Hq * D / kWideRows, nk = Hkv * D / kWideRows, tile = idx / P.gseg_qkv;
+    const bool epi = idx % P.gseg_qkv == 0;
     const int kind = tile < nq ? 0 : tile < nq + nk ? 1 : 2;
     const int h0 = 2 * (tile - (kind == 0 ? 0 : kind == 1 ? nq : nq + nk));
     t.wait_ev = counter(EV_N1, l);
     t.notify_ev = counter(EV_QKV, l, 0);
     for (int b = 0; b < B; ++b) {
       t.reads.push_back({BUF_XN, (long long)b * H, (long long)(b + 1) * H});
-      for (int hh = h0; hh < h0 + 2; ++hh) {
+      for (int hh = h0; hh < h0 + 2 && epi; ++hh) {
         if (kind == 0) {
           const long long base = b * QD + (long long)hh * D;
           t.writes.push_back({BUF_Q, base, base + D});
@@ -251,8 +254,10 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
       t.wait_ev = counter(EV_ATTN, l);
       t.notify_ev = counter(EV_O, l);
       const int tile = idx / P.gseg_o;
+      const bool epi = idx % P.gseg_o == 0;  // (the epilogue's task of the tile, as for QKV)
       for (int b = 0; b < B; ++b) {
         t.reads.push_back({BUF_ATTN, b * QD, (b + 1) * QD});
+        if (!epi) continue;
         long long xb = (long long)b * H + (long long)tile * P.tile_o;
         t.reads.push_back({BUF_X, xb, xb + P.tile_o});
         if (l > 0 && !mdec && !wide)
@@ -265,10 +270,12 @@ void Plan::task(int f, int idx, const Binding& bd, TaskRec& t) const {
     } break;
     case OP_GATEUP: {
       const int tile = idx / P.gseg_gu;
+      const bool epi = idx % P.gseg_gu == 0;  // (the epilogue's task of the tile, as for QKV)
       t.wait_ev = wide ? counter(EV_N2, l) : counter(EV_O, l);
       t.notify_ev = counter(EV_GU, l, tile * P.tile_gu / P.kseg);
       for (int b = 0; b < B; ++b) {
         t.reads.push_back({wide ? BUF_XN : BUF_X, (long long)b * H, (long long)(b + 1) * H});
+        if (!epi) continue;
         long long hb = (long long)b * F + (long long)tile * P.tile_gu;
         t.writes.push_back({BUF_H, hb, hb + P.tile_gu});
       }
@@ -653,9 +660,10 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   // computed; of 8, 16, 24 and 32, 16 was fastest at B = 16, 32 at B = 32 and
   // 24 at B = 64, 24 the best over the three)
   P.attn_split = o->attn_split ? o->attn_split : (wide ? 24 : 32);
-  // up to 8 rows with no split given, the split follows each step's B and
-  // contexts (step_attn_split: 3 to 16 chunks on the 1B shape at B = 1..8)
-  P.attn_auto = (!o->attn_split && !wide) ? 1 : 0;
+  // with no split given, the split follows each step's B and contexts at
+  // steps of up to 8 rows, in narrow and wide plans alike (step_attn_split:
+  // 3 to 16 chunks on the 1B shape at B = 1..8)
+  P.attn_auto = !o->attn_split ? 1 : 0;
   if (P.attn_split < 1 || P.attn_split > 64) { err = "attn_split must be in [1, 64]"; return MK_ERR_INVALID_ARG; }
   if (wide) {
     // tcgen05 GEMM tasks: kWideRows weight rows each (the MMA's M), every

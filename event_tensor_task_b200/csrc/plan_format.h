@@ -311,7 +311,7 @@ struct DevPlan {
   // last to count in sums the partials in segment order and runs the
   // tile's epilogue (the counters are zeroed at launch and by that task)
   int32_t gseg_qkv, gseg_o, gseg_gu;
-  int32_t attn_auto;  // 1: the attention split follows each step's B and contexts (step_attn_split)
+  int32_t attn_auto;  // 1: the attention split follows each step's B and contexts (step_attn_split; wide plans: steps of at most kMaxBatchRows rows)
   int64_t off_gpart, off_gctr;
   // attention: per (sequence, kv head) count of finished tasks; the last of a
   // pair's tasks merges their partials (zeroed at launch and by that task)
@@ -378,15 +378,16 @@ MK_HD AttnTask decode_attn(int i, int B, int Hkv, const int* nch, const int* pre
 MK_HD int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Key chunks per attention task in one step.  A plan with a fixed split
-// (attn_auto = 0) returns attn_split.  An adaptive plan cuts the step's
-// C = Hkv * sum_b ceil((ctx_b + 1) / chunk) chunk units into about two thirds
-// of n_sm tasks: s = ceil(C / ceil(2 n_sm / 3)), clamped to
+// (attn_auto = 0) returns attn_split, and so does a wide-batch plan at a step
+// of more than kMaxBatchRows rows.  Otherwise the step's
+// C = Hkv * sum_b ceil((ctx_b + 1) / chunk) chunk units are cut into about two
+// thirds of n_sm tasks: s = ceil(C / ceil(2 n_sm / 3)), clamped to
 // [min(kAttnSplitMin, attn_split), attn_split].  (Measured on the 1B shape at
 // B = 1..8: fewer, longer tasks leave SMs idle; more tasks than that pay a
 // second wave and more merging; below 3 chunks a task's fixed costs dominate.)
 constexpr int kAttnSplitMin = 3;
 MK_HD int step_attn_split(const DevPlan& P, int B, const int* ctx) {
-  if (!P.attn_auto) return P.attn_split;
+  if (!P.attn_auto || (P.wide && B > kMaxBatchRows)) return P.attn_split;
   long long c = 0;
   for (int b = 0; b < B; ++b) c += ceil_div(ctx[b] + 1, P.chunk);
   c *= P.n_kv_heads;

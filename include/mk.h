@@ -140,11 +140,12 @@ typedef struct mk_plan_opts {
   int fault;
   int fault_family;
   /* Key chunks (attn_chunk keys each) per attention task, at most 64.  A
-   * value > 0 is used as given.  0 = default: 24 for max_batch > 8; for
-   * max_batch <= 8 the split follows each step: with C = n_kv_heads *
-   * sum_b ceil((ctx_b + 1) / attn_chunk) chunk units and T = ceil(2 n_sm / 3),
-   * split = ceil(C / T) clamped to [3, 32] (about two thirds of the SMs'
-   * worth of tasks).  Compute warp w of a task takes chunks w, w + 8, ...
+   * value > 0 is used as given.  0 = default: a step of up to 8 rows takes a
+   * split that follows the step: with C = n_kv_heads * sum_b
+   * ceil((ctx_b + 1) / attn_chunk) chunk units and T = ceil(2 n_sm / 3),
+   * split = ceil(C / T) clamped to [3, S] (about two thirds of the SMs'
+   * worth of tasks), S = 32 for max_batch <= 8 and 24 above; a step of more
+   * than 8 rows (a wide-batch plan) takes 24.  Compute warp w of a task takes chunks w, w + 8, ...
    * (warp-MMA scores and P.V with an online softmax).  A task that holds all
    * of its (sequence, kv head)'s chunks writes the finished output; otherwise
    * it leaves one partial, and the last of the pair's tasks to finish merges

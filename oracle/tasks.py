@@ -29,7 +29,8 @@ split)`` attention tasks per kv head.  With ``tiles["split_auto"]`` the split
 is chosen per step (``step_split``): the step's chunk units
 ``C = Hkv * sum_b ceil((ctx_b + 1) / chunk)`` over about two thirds of
 ``tiles["n_sm"]`` tasks, ``ceil(C / ceil(2 n_sm / 3))``, kept between
-``min(3, split)`` and ``split``.  Linear index of an ``attn`` task:
+``min(3, split)`` and ``split``; in the wide-batch layout only at steps of at
+most 8 rows (above that the split is ``split``).  Linear index of an ``attn`` task:
 ``Hkv * sum_{b'<b} nch_{b'} + g * nch_b + c``.  ``down`` tasks are numbered
 K-segment-major: ``kc * (H / tile_down) + n``.
 
@@ -50,7 +51,7 @@ def _ceil(a: int, b: int) -> int:
 def step_split(shape, B: int, ctx, tiles: dict) -> int:
     """Key chunks per attention task in a step with these contexts."""
     split = tiles.get("split", 1)
-    if not tiles.get("split_auto"):
+    if not tiles.get("split_auto") or (tiles.get("wide") and B > 8):
         return split
     units = shape.n_kv_heads * sum(_ceil(int(ctx[b]) + 1, tiles["chunk"]) for b in range(B))
     target = _ceil(2 * tiles["n_sm"], 3)

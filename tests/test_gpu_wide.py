@@ -37,9 +37,11 @@ def _check(case, tokens, slots, ctx, K, V, hidden=True):
 @pytest.mark.parametrize("sched,split", [(mk.MK_SCHED_STATIC, 0), (mk.MK_SCHED_DYNAMIC, 0),
                                          (mk.MK_SCHED_STATIC, 2)])
 def test_tiny_wide_batch_symbolic_shapes(sched, split):
-    # one plan (max_batch 16): B = 16, 9, 1 and 12 with ragged contexts, the
+    # one plan (max_batch 16): B = 16, 9, 1, 12 and 4 with ragged contexts, the
     # oracle's cache following the appends; activations as value + remainder
-    # rows (default) and as plain bf16 rows
+    # rows (default) and as plain bf16 rows.  The steps of at most 8 rows take
+    # the per-step attention split (B = 4 at these contexts: 3 chunks per task,
+    # so three of its (sequence, kv head) pairs have 2 tasks and a merge)
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     fill = [64, 0, 70, 190, 5, 127, 128, 300, 1, 2, 255, 33, 64, 65, 129, 200]
@@ -50,7 +52,8 @@ def test_tiny_wide_batch_symbolic_shapes(sched, split):
     steps = [(tok, list(range(16)), fill),
              (tok[:9], [15, 1, 3, 0, 5, 7, 2, 9, 11], [201, 1, 191, 65, 128, 301, 71, 3, 34]),
              (tok[:1], [6], [128]),
-             (tok[:12], list(range(12)), [65, 2, 72, 192, 6, 129, 129, 302, 3, 4, 256, 35])]
+             (tok[:12], list(range(12)), [65, 2, 72, 192, 6, 129, 129, 302, 3, 4, 256, 35]),
+             (tok[:4], [0, 7, 10, 15], [66, 303, 257, 202])]
     for tokens, slots, ctx in steps:
         _check(case, tokens, slots, ctx, K, V)
 

@@ -507,6 +507,11 @@ def test_step_split_by_hand():
     assert ot.step_split(s, 8, [696, 2450, 2106, 216, 1316, 3764, 443, 949], tiles) == 16
     # 8 * 8 * 64 = 4096 units, ceil(4096 / 99) = 42, capped at 32
     assert ot.step_split(s, 8, [4095] * 8, tiles) == 32
+    # the wide-batch layout: adaptive up to 8 rows (cap 24), fixed above
+    wide = dict(tiles, split=24, wide=True)
+    assert ot.step_split(s, 8, [4095] * 8, wide) == 24
+    assert ot.step_split(s, 4, [696, 2450, 2106, 216], wide) == 8
+    assert ot.step_split(s, 9, [0] * 9, wide) == 24
     # a cap below the floor of 3 wins; without split_auto the split is fixed
     assert ot.step_split(s, 1, [1024], dict(tiles, split=2)) == 2
     assert ot.step_split(s, 8, [4095] * 8, dict(tiles, split_auto=False)) == 32

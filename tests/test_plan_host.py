@@ -121,6 +121,23 @@ def test_simulator_adaptive_attention_split(B, ctx, split):
     d.close()
 
 
+@pytest.mark.parametrize("B,ctx,split", [(4, [600, 900, 200, 50], 10), (9, [600, 900, 200, 50, 0, 1, 2, 3, 4], 24)])
+def test_simulator_wide_plan_attention_split(B, ctx, split):
+    # a wide-batch plan (max_batch 16) takes the per-step split up to 8 rows
+    # and its fixed 24 above: the tiny shape on 8 SMs (T = 6)
+    d = _host(wl.TINY, max_batch=16, max_ctx=1024, n_sm=8)
+    t = d.tiles()
+    assert t["wide"] == 1 and t["attn_auto"] == 1 and t["attn_split"] == 24
+    mk.mk_plan_validate(d.plan, B, ctx)
+    code, rep = mk.mk_plan_simulate(d.plan, B, ctx, n_orders=1, seed=5)
+    assert code == 0 and rep.races == 0 and rep.nonzero_counters == 0, rep.first_error
+    tiles = {k: t[k] for k in ("tile_qkv", "chunk", "tile_o", "tile_gu", "tile_down", "kseg", "tile_lm", "n_sm")}
+    tiles.update(split=24, split_auto=True, wide=True, gseg=(t["gseg_qkv"], t["gseg_o"], t["gseg_gu"]))
+    assert ot.step_split(wl.TINY, B, ctx, tiles) == split
+    assert rep.tasks_per_order == len(ot.expected_dense_tasks(wl.TINY, B, ctx, tiles))
+    d.close()
+
+
 def test_simulator_many_orders():
     d = _host(wl.TINY, n_sm=5)
     code, rep = mk.mk_plan_simulate(d.plan, 2, [3, 128], n_orders=1000, seed=11)
@@ -197,10 +214,11 @@ def test_plan_option_ranges():
     assert _host(wl.LLAMA_1B, max_batch=4, max_ctx=4160, n_sm=148, attn_split=8).tiles()["attn_auto"] == 0
     t = _host(wl.LLAMA_1B, max_batch=8, max_ctx=4160, n_sm=148).tiles()
     assert (t["attn_split"], t["attn_auto"]) == (32, 1)
-    # wide-batch defaults: 24 chunks per attention task (fixed), split K 4 / 4 / 2
+    # wide-batch defaults: 24 chunks per attention task above 8 rows (adaptive
+    # up to 8), split K 4 / 4 / 2
     t = _host(wl.LLAMA_1B, max_batch=64, max_ctx=1088, n_sm=148).tiles()
     assert (t["attn_split"], t["attn_auto"], t["gseg_qkv"], t["gseg_o"], t["gseg_gu"], t["kseg"]) == \
-        (24, 0, 4, 4, 2, 1024)
+        (24, 1, 4, 4, 2, 1024)
 
 
 def test_moe_plan_requires_dynamic_schedule_and_rejects_dense_calls():
