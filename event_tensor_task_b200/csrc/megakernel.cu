@@ -2239,10 +2239,15 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
   const MoeW mw = moe_weights(P, reinterpret_cast<const LayerPtrs*>(ws + P.off_layers), d.layer);
   const bool dec = P.kind == MK_MODEL_MOE_DECODER;
   __nv_bfloat16* xhat = reinterpret_cast<__nv_bfloat16*>(mb + P.off_mxhat);
-  if (dec) {
-    // the layer's FFN input: RMSNorm(x) * ffn_norm of each token's residual row, in bf16
+  float* lg = sm.xs();  // [8][64] logits of this task's tokens
+  // this task's token rows, bf16 [8][H] after the logits: read by every warp
+  // for every expert (the staging buffer holds route_stage_bytes(H))
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<unsigned char*>(lg) + kRouteLogitBytes);
+  bar_sync(BAR_COMP, kComputeThreads);  // the staging buffer is free
+  {
     const int t = d.idx * 8 + w;
-    if (t < T) {
+    if (t < T && dec) {
+      // the layer's FFN input: RMSNorm(x) * ffn_norm of each token's residual row, in bf16
       const float* xr32 = reinterpret_cast<const float*>(ws + P.off_x) + (size_t)t * H;
       const uint4* gam = reinterpret_cast<const uint4*>(reinterpret_cast<const LayerPtrs*>(ws + P.off_layers)[d.layer].ffn_norm);
       float v[kMaxBlk][8];
@@ -2266,33 +2271,40 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
           __align__(16) __nv_bfloat16 o[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) o[j] = __float2bfloat16_rn(v[i][j] * inv * gf[j]);
-          *reinterpret_cast<uint4*>(xhat + (size_t)t * H + 256 * i + 8 * lane) = *reinterpret_cast<const uint4*>(o);
+          const uint4 ov = *reinterpret_cast<const uint4*>(o);
+          *reinterpret_cast<uint4*>(xhat + (size_t)t * H + 256 * i + 8 * lane) = ov;
+          *reinterpret_cast<uint4*>(xs + (size_t)w * H + 256 * i + 8 * lane) = ov;
           if (S.cap_moe_in)
-            *reinterpret_cast<uint4*>(S.cap_moe_in + ((size_t)d.layer * T + t) * H + 256 * i + 8 * lane) =
-                *reinterpret_cast<const uint4*>(o);
+            *reinterpret_cast<uint4*>(S.cap_moe_in + ((size_t)d.layer * T + t) * H + 256 * i + 8 * lane) = ov;
         }
+    } else if (t < T) {
+      const uint4* xr = reinterpret_cast<const uint4*>(S.moe_x) + (size_t)t * H / 8;
+#pragma unroll
+      for (int i = 0; i < kMaxBlk; ++i)
+        if (i < nblk) *reinterpret_cast<uint4*>(xs + (size_t)w * H + 256 * i + 8 * lane) = __ldcg(xr + 32 * i + lane);
     }
   }
-  float* lg = sm.xs();  // [8][64] logits of this task's tokens
-  bar_sync(BAR_COMP, kComputeThreads);  // the staging buffer is free (and the FFN inputs are written)
+  bar_sync(BAR_COMP, kComputeThreads);  // the token rows are staged (and the FFN inputs written)
+  // logits: warp w takes experts w, w + 8, ...; the token rows come from
+  // shared memory, so an expert costs one round trip (its router row) for all
+  // the task's tokens; each logit is summed in the fixed order (lane l:
+  // columns 256 i + 8 l + j in increasing i, j, then the xor butterfly)
   const uint4* wr = reinterpret_cast<const uint4*>(mw.router);
-  const uint4* xr = reinterpret_cast<const uint4*>(dec ? xhat : S.moe_x);
+  const int nt = min(8, T - d.idx * 8);
   for (int e = w; e < E; e += kComputeWarps) {
     uint4 wv[kMaxBlk];
 #pragma unroll
     for (int i = 0; i < kMaxBlk; ++i)
       if (i < nblk) wv[i] = __ldg(wr + ((size_t)e * H + 256 * i + 8 * lane) / 8);
     const float bias = mw.bias ? __ldg(mw.bias + e) : 0.f;
-    for (int tt = 0; tt < 8; ++tt) {
-      const int t = d.idx * 8 + tt;
-      if (t >= T) break;
+    for (int tt = 0; tt < nt; ++tt) {
       float acc = 0.f;
 #pragma unroll
       for (int i = 0; i < kMaxBlk; ++i)
         if (i < nblk) {
           float wf[8], xf[8];
           bf16x8_to_f32(wv[i], wf);
-          bf16x8_to_f32(__ldcg(xr + ((size_t)t * H + 256 * i + 8 * lane) / 8), xf);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(xs + (size_t)tt * H + 256 * i + 8 * lane), xf);
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc = fmaf(wf[j], xf[j], acc);  // the product is exact in fp32
         }
@@ -2348,7 +2360,7 @@ __device__ __forceinline__ void task_route(const DevPlan& P, const StepParams& S
   uint4* xg = reinterpret_cast<uint4*>(mb + P.off_mxg);
   const size_t dst_row = lane < K ? ((size_t)sel_e * P.moe_cap + rank) * (H / 8) : 0;  // lane j: pair j's row
   for (int i = 0; i < nblk; ++i) {
-    const uint4 v = __ldcg(xr + (size_t)t * (H / 8) + 32 * i + lane);
+    const uint4 v = *reinterpret_cast<const uint4*>(xs + (size_t)w * H + 256 * i + 8 * lane);  // (token t's staged row)
     for (int j = 0; j < K; ++j) xg[__shfl_sync(0xffffffffu, dst_row, j) + 32 * i + lane] = v;
   }
 }
@@ -2541,20 +2553,29 @@ __device__ __forceinline__ void task_combine(const DevPlan& P, const StepParams&
                                              const TaskDesc& d) {
   const int lane = threadIdx.x & 31, w = (threadIdx.x - kComputeBase) >> 5;
   const int H = P.hidden, K = P.top_k, nblk = H >> 8;
-  const int t = d.idx * 8 + w;
-  if (t >= S.B) return;
+  const int nt = min(8, S.B - d.idx * 8);  // this task's tokens
   const unsigned char* mb = moe_block(P, ws, d.layer);
   const int* mrow = reinterpret_cast<const int*>(mb + P.off_mrow);
   const float* mw = reinterpret_cast<const float*>(mb + P.off_mw);
   const float* my = reinterpret_cast<const float*>(mb + P.off_my);
   const bool dec = P.kind == MK_MODEL_MOE_DECODER;
-  float* xres = reinterpret_cast<float*>(ws + P.off_x) + (size_t)t * H;
-  int rows[8];
+  // items (token tt, 256-column block i) over the 8 warps, token fastest:
+  // with 8 tokens warp w takes token w's blocks (as one warp per token), with
+  // one token each warp takes one block (its loads in one round trip); each
+  // element sums its expert rows in the token's top-k order whichever warp
+  // takes it
+  int rows[8], cur = -1;
   float wts[8];
+  for (int it = w; it < nt * nblk; it += kComputeWarps) {
+    const int tt = it % nt, i = it / nt;
+    const int t = d.idx * 8 + tt;
+    float* xres = reinterpret_cast<float*>(ws + P.off_x) + (size_t)t * H;
+    if (tt != cur) {
+      cur = tt;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < K) { rows[j] = __ldcg(mrow + (size_t)t * K + j); wts[j] = __ldcg(mw + (size_t)t * K + j); }
-  for (int i = 0; i < nblk; ++i) {
+      for (int j = 0; j < 8; ++j)
+        if (j < K) { rows[j] = __ldcg(mrow + (size_t)t * K + j); wts[j] = __ldcg(mw + (size_t)t * K + j); }
+    }
     const int c = 256 * i + 8 * lane;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -457,12 +457,13 @@ void Plan::successors(int ci, const Binding& bd, std::vector<int>& out) const {
 // ---------------------------------------------------------------- build
 
 // Shared-memory split of a CTA (see kSmemFixed): the staging buffer sized for
-// `rows` batch rows, the partial tiles (for the dense GEMV tasks; none for
-// rows = 0), the rest to 16 KB ring slots.
-static void smem_layout(DevPlan& P, int rows, int smem_bytes) {
+// `rows` batch rows and at least min_act bytes, the partial tiles (for the
+// dense GEMV tasks; none for rows = 0), the rest to 16 KB ring slots.
+static void smem_layout(DevPlan& P, int rows, int smem_bytes, int min_act) {
   P.gbatch = kMaxBatchRows;
   // (B <= 4 stages 2B rows: each row's bf16 value and its bf16 remainder)
   P.act_bytes = std::max(8192, (std::min(2 * rows, kMaxBatchRows) * kActPitch * 2 + 127) / 128 * 128);
+  P.act_bytes = std::max(P.act_bytes, (min_act + 127) / 128 * 128);
   P.gred_bytes = rows > 0 ? 8 * P.gbatch * 64 * 4 : 0;
   P.smem_bytes = smem_bytes;
   P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - P.gred_bytes - seq_table_bytes(P)) /
@@ -515,7 +516,7 @@ static mk_status build_moe_plan(const mk_model_desc* m, const mk_plan_opts* o, i
   // sum over experts of ceil(hist_e / tm) <= T*k/tm + (experts with a row)
   P.max_tiles = ceil_div(TM * K, P.moe_tm) + std::min(E, TM * K);
   P.slot_bytes = 16384;
-  smem_layout(P, 0, smem_bytes);
+  smem_layout(P, 0, smem_bytes, route_stage_bytes(H));
   if (P.ring_slots < 5) { err = "not enough shared memory for a 5-slot ring"; return MK_ERR_UNSUPPORTED; }
 
   p.code.clear();
@@ -723,11 +724,12 @@ mk_status build_plan(const mk_model_desc* m, const mk_plan_opts* o, int n_sm, in
   if (wide) {
     P.gbatch = 0;
     P.act_bytes = std::max(std::max(8192, 64 * P.act_rows * 4), kBStages * act_buf_rows(P.act_split, P.act_rows) * 128);
+    if (mdec) P.act_bytes = std::max(P.act_bytes, (route_stage_bytes(H) + 127) / 128 * 128);  // (ROUTE tasks)
     P.gred_bytes = 0;
     P.smem_bytes = smem_bytes;
     P.ring_slots = std::min(16, (smem_bytes - kSmemFixed - P.act_bytes - seq_table_bytes(P)) / P.slot_bytes);
   } else {
-    smem_layout(P, P.max_batch, smem_bytes);
+    smem_layout(P, P.max_batch, smem_bytes, mdec ? route_stage_bytes(H) : 0);
   }
   if (P.ring_slots < 3) { err = "not enough shared memory for a 3-slot ring"; return MK_ERR_UNSUPPORTED; }
 

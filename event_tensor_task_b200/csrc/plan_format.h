@@ -251,6 +251,13 @@ MK_HD int act_buf_row(int split, int b, int part) { return split ? (b >> 3) * 16
 MK_HD int act_buf_rows(int split, int act_rows) { return split ? 2 * act_rows : act_rows; }
 
 MK_HD int moe_tile_rows(int h, int tm, int big) { return (big && h > tm) ? kMoeBigTileRows : tm; }
+
+// A ROUTE task's use of the staging buffer: the router logits of its 8
+// tokens ([8][64] fp32), then the tokens' bf16 input rows ([8][hidden]), read
+// by every warp for every expert.  Plans with ROUTE tasks size the staging
+// buffer to hold it.
+constexpr int kRouteLogitBytes = 8 * 64 * 4;
+MK_HD int route_stage_bytes(int hidden) { return kRouteLogitBytes + 8 * hidden * 2; }
 constexpr int kTmemCols = 256;  // TMEM columns a CTA of an MoE plan allocates
 
 // Fixed header of the plan; passed to the kernel by value.  Offsets are in
