@@ -463,7 +463,10 @@ __device__ void producer(const DevPlan& P, const StepParams& S, Smem& sm, unsign
     return true;
   };
 
-  auto emit = [&](int fam, int idx) -> bool {
+  // (always inlined: called from three places, the producer would otherwise
+  // become a call whose frame holds its state; ptxas reported stack frames of
+  // up to 2.3 KB for the MoE instances when it was not)
+  auto emit = [&](int fam, int idx) __attribute__((always_inline)) -> bool {
     int op = OP_END, layer = -1;
     if (fam >= 0) {
       op = sm.fam_op[fam];
